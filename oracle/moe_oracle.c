@@ -1,0 +1,402 @@
+/*
+ * moe_oracle.c -- plain, slow, obviously-correct CPU oracle for one routed
+ * MoE FFN layer on ggml-style block-quantized expert weights.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg may load this library.  It shares no code, header, table
+ * or constant with the CUDA library; neither includes the other.
+ *
+ * What it computes (all floating point in double unless stated):
+ *
+ *   Block formats -- FreeToken fork README, "Quant types" table (Standard
+ *   family: Q4_0, Q8_0).  32 weights per block, one fp16 scale d:
+ *     Q8_0 {fp16 d; int8 q[32]}           value q[i] * d
+ *     Q4_0 {fp16 d; uint8 qs[16]}         value (q[i] - 8) * d, byte j holds
+ *                                         element j (low nibble) and j+16
+ *                                         (high nibble)
+ *   Expert pool layout -- FreeToken fork README, "Known limits": experts back
+ *   to back, expert * nrows * (ncols / 32) blocks, no padding, one type.
+ *   Per expert: W_gate, W_up are [F rows][D/32 blocks], W_down [D][F/32].
+ *
+ *   Layer (the routed MoE FFN layer the pages serve; FreeToken wiki
+ *   explainer, opening section: a subset of experts is active per token):
+ *     L[t,e]  = sum_i x[t,i] W_r[i,e] + b[e]       (double, then rounded to fp32)
+ *     S_t     = the k experts of largest L[t,.], ordered by L descending,
+ *               ties to the lower expert index
+ *     p       = softmax over all E of L[t,.]      (double, max-subtracted)
+ *     g[t,j]  = p[S_tj] / sum_{i in S_t} p[i]      (renormalised top-k gates)
+ *     h       = silu(x_t . W_gate,e row) * (x_t . W_up,e row), silu(z) = z/(1+e^-z)
+ *     Y[t,j]  = W_down,e h                          (e = S_tj)
+ *     y_t     = sum_j g[t,j] Y[t,j]  (+ shared-expert FFN of x_t, weight 1)
+ *   Permutation: a stable counting sort of the flat (t, j) entries by expert.
+ *
+ *   Expert cache: a per-layer LRU over a fixed number of device slots
+ *   (FreeToken fork README, "About": global LRU expert caching; wiki
+ *   explainer: shared LRU expert caching follows token-level routing
+ *   locality; kongchang article, "From Static Allocation to Dynamic
+ *   Scheduling": VRAM as a cache with the full model in system RAM).
+ *   The replacement rules the pages leave open are fixed in orc_lru_request.
+ *
+ * Parity of every function here is pinned by the CPU tests against closed
+ * forms, brute force and hand-packed blocks.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_QK 32
+#define ORC_Q4_0 2
+#define ORC_Q8_0 8
+
+/* IEEE 754 binary16 -> double, decoded bit by bit (sign, 5-bit exponent with
+ * bias 15, 10-bit fraction; subnormals, infinities and NaN included). */
+double orc_half_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 10) & 0x1f;
+    int frac = h & 0x3ff;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -24);              /* 2^-14 * frac / 2^10 */
+    else if (expo == 31)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexp(1.0 + (double)frac / 1024.0, expo - 15);
+    return sign ? -v : v;
+}
+
+int orc_block_bytes(int qtype)
+{
+    if (qtype == ORC_Q8_0) return 2 + 32;
+    if (qtype == ORC_Q4_0) return 2 + 16;
+    return 0;
+}
+
+/* Dequantize one row of ncols weights (ncols % 32 == 0) into out[]. */
+int orc_dequant_row(const uint8_t *row, int qtype, int ncols, double *out)
+{
+    int bs = orc_block_bytes(qtype);
+    if (bs == 0 || ncols % ORC_QK) return -1;
+    for (int b = 0; b < ncols / ORC_QK; b++) {
+        const uint8_t *blk = row + (size_t)b * bs;
+        uint16_t dbits = (uint16_t)(blk[0] | (blk[1] << 8));   /* little endian */
+        double d = orc_half_to_double(dbits);
+        for (int i = 0; i < ORC_QK; i++) {
+            double v;
+            if (qtype == ORC_Q8_0) {
+                int q = (int)(int8_t)blk[2 + i];
+                v = (double)q * d;
+            } else {
+                int byte = blk[2 + (i % 16)];
+                int q = (i < 16) ? (byte & 0x0f) : (byte >> 4);
+                v = (double)(q - 8) * d;
+            }
+            out[b * ORC_QK + i] = v;
+        }
+    }
+    return 0;
+}
+
+/* Router logits in double, rounded once to fp32.  x [T,D], W_r [D,E]
+ * row-major, bias [E] or NULL. */
+void orc_router_logits(const float *x, const float *w_r, const float *bias,
+                       int T, int D, int E, float *logits)
+{
+    for (int t = 0; t < T; t++)
+        for (int e = 0; e < E; e++) {
+            double acc = 0.0;
+            for (int i = 0; i < D; i++)
+                acc += (double)x[(size_t)t * D + i] * (double)w_r[(size_t)i * E + e];
+            if (bias) acc += (double)bias[e];
+            logits[(size_t)t * E + e] = (float)acc;
+        }
+}
+
+/* Top-k selection, softmax and renormalisation per token.
+ * Selection: repeatedly take the not-yet-taken expert with the largest
+ * logit, the lower index on equal logits (a selection sort on the key
+ * (L descending, index ascending)).  Gates from the full softmax in double. */
+void orc_select(const float *logits, int T, int E, int k, int renorm,
+                int32_t *ids, double *gates)
+{
+    char *taken = (char *)malloc((size_t)E);
+    double *p = (double *)malloc(sizeof(double) * (size_t)E);
+    for (int t = 0; t < T; t++) {
+        const float *L = logits + (size_t)t * E;
+        memset(taken, 0, (size_t)E);
+        for (int j = 0; j < k; j++) {
+            int best = -1;
+            for (int e = 0; e < E; e++) {
+                if (taken[e]) continue;
+                if (best < 0 || L[e] > L[best]) best = e;   /* strict: keeps lower index */
+            }
+            taken[best] = 1;
+            ids[(size_t)t * k + j] = best;
+        }
+        double m = -INFINITY;
+        for (int e = 0; e < E; e++) if ((double)L[e] > m) m = (double)L[e];
+        double z = 0.0;
+        for (int e = 0; e < E; e++) { p[e] = exp((double)L[e] - m); z += p[e]; }
+        for (int e = 0; e < E; e++) p[e] /= z;
+        double s = 0.0;
+        for (int j = 0; j < k; j++) s += p[ids[(size_t)t * k + j]];
+        for (int j = 0; j < k; j++) {
+            double pj = p[ids[(size_t)t * k + j]];
+            gates[(size_t)t * k + j] = renorm ? pj / s : pj;
+        }
+    }
+    free(taken);
+    free(p);
+}
+
+/* Stable counting sort of the flat entries n = t*k + j by expert id:
+ * counts[e], offsets[e] = sum of earlier counts (offsets[E] = T*k),
+ * perm[pos] = n in order (expert, t, j), inv[n] = pos. */
+int orc_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
+                int32_t *offsets, int32_t *perm, int32_t *inv)
+{
+    int N = T * k;
+    for (int e = 0; e < E; e++) counts[e] = 0;
+    for (int n = 0; n < N; n++) {
+        if (ids[n] < 0 || ids[n] >= E) return -1;
+        counts[ids[n]]++;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; e++) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *cursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+    for (int e = 0; e <= E; e++) cursor[e] = offsets[e];
+    for (int n = 0; n < N; n++) {
+        int pos = cursor[ids[n]]++;
+        perm[pos] = n;
+        inv[n] = pos;
+    }
+    free(cursor);
+    return 0;
+}
+
+static double orc_silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* One expert's SwiGLU FFN of one activation row xt[D] -> Y[D].
+ * gate/up/down point at this expert's matrices in the pool. */
+static void orc_expert_ffn_row(const double *xt, const uint8_t *gate,
+                               const uint8_t *up, const uint8_t *down, int qtype,
+                               int D, int F, double *wrow, double *h, double *Y)
+{
+    size_t gate_row = (size_t)(D / ORC_QK) * orc_block_bytes(qtype);
+    size_t down_row = (size_t)(F / ORC_QK) * orc_block_bytes(qtype);
+    for (int r = 0; r < F; r++) {
+        double a = 0.0, u = 0.0;
+        orc_dequant_row(gate + r * gate_row, qtype, D, wrow);
+        for (int i = 0; i < D; i++) a += xt[i] * wrow[i];
+        orc_dequant_row(up + r * gate_row, qtype, D, wrow);
+        for (int i = 0; i < D; i++) u += xt[i] * wrow[i];
+        h[r] = orc_silu(a) * u;
+    }
+    for (int d = 0; d < D; d++) {
+        double acc = 0.0;
+        orc_dequant_row(down + d * down_row, qtype, F, wrow);
+        for (int f = 0; f < F; f++) acc += h[f] * wrow[f];
+        Y[d] = acc;
+    }
+}
+
+static size_t orc_expert_stride(int nrows, int ncols, int qtype)
+{
+    return (size_t)nrows * (size_t)(ncols / ORC_QK) * orc_block_bytes(qtype);
+}
+
+/* The routed layer for a list of tokens.
+ *  x [T,D] fp32 values; ids/gates [T,k] from orc_select (any k-subset works);
+ *  gate/up/down: pools of E experts in `qtype` (slot = expert id);
+ *  sh_*: optional shared expert (Q8_0, F = sh_F) added with weight 1;
+ *  tok_list[n_tok]: the tokens to evaluate (NULL = all T, n_tok = T);
+ *  y [n_tok, D] doubles.  dense != 0 evaluates all E experts per token and
+ *  weights each by its gate if selected and by 0 otherwise (the dense,
+ *  masked form of the same sum).  Returns 0, or -1 on bad arguments. */
+int orc_layer(const float *x, int T, int D, int F, int E, int k, int qtype,
+              const uint8_t *gate, const uint8_t *up, const uint8_t *down,
+              const int32_t *ids, const double *gates,
+              const uint8_t *sh_gate, const uint8_t *sh_up,
+              const uint8_t *sh_down, int sh_F, int sh_qtype,
+              const int32_t *tok_list, int n_tok, int dense, int nthreads,
+              double *y)
+{
+    if (orc_block_bytes(qtype) == 0 || D % ORC_QK || F % ORC_QK || k > E)
+        return -1;
+    if (sh_gate && (orc_block_bytes(sh_qtype) == 0 || sh_F % ORC_QK)) return -1;
+    if (!tok_list) n_tok = T;
+    size_t gstride = orc_expert_stride(F, D, qtype);
+    size_t dstride = orc_expert_stride(D, F, qtype);
+    int maxF = F > sh_F ? F : sh_F;
+    int maxW = D > maxF ? D : maxF;
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+#endif
+    for (int n = 0; n < n_tok; n++) {
+        int t = tok_list ? tok_list[n] : n;
+        if (t < 0 || t >= T) { bad |= 1; continue; }
+        double *xt = (double *)malloc(sizeof(double) * (size_t)D);
+        double *wrow = (double *)malloc(sizeof(double) * (size_t)maxW);
+        double *h = (double *)malloc(sizeof(double) * (size_t)maxF);
+        double *Y = (double *)malloc(sizeof(double) * (size_t)D);
+        double *yt = y + (size_t)n * D;
+        for (int i = 0; i < D; i++) { xt[i] = (double)x[(size_t)t * D + i]; yt[i] = 0.0; }
+        if (!dense) {
+            for (int j = 0; j < k; j++) {
+                int e = ids[(size_t)t * k + j];
+                if (e < 0 || e >= E) { bad |= 1; break; }
+                orc_expert_ffn_row(xt, gate + e * gstride, up + e * gstride,
+                                   down + e * dstride, qtype, D, F, wrow, h, Y);
+                double g = gates[(size_t)t * k + j];
+                for (int i = 0; i < D; i++) yt[i] += g * Y[i];
+            }
+        } else {
+            for (int e = 0; e < E; e++) {
+                double g = 0.0;
+                for (int j = 0; j < k; j++)
+                    if (ids[(size_t)t * k + j] == e) g = gates[(size_t)t * k + j];
+                orc_expert_ffn_row(xt, gate + e * gstride, up + e * gstride,
+                                   down + e * dstride, qtype, D, F, wrow, h, Y);
+                for (int i = 0; i < D; i++) yt[i] += g * Y[i];
+            }
+        }
+        if (sh_gate) {
+            orc_expert_ffn_row(xt, sh_gate, sh_up, sh_down, sh_qtype, D, sh_F,
+                               wrow, h, Y);
+            for (int i = 0; i < D; i++) yt[i] += Y[i];
+        }
+        free(xt); free(wrow); free(h); free(Y);
+    }
+    return bad ? -1 : 0;
+}
+
+/* Un-combined expert outputs: for each listed permuted position pos, with
+ * n = perm[pos], t = n / k, e = the expert of segment pos falls in,
+ * Y[i] = FFN_e(x_t) (no gate).  pos_list NULL = all T*k positions. */
+int orc_expert_rows(const float *x, int T, int D, int F, int E, int k,
+                    int qtype, const uint8_t *gate, const uint8_t *up,
+                    const uint8_t *down, const int32_t *perm,
+                    const int32_t *offsets, const int32_t *pos_list, int n_pos,
+                    int nthreads, double *Y)
+{
+    if (orc_block_bytes(qtype) == 0 || D % ORC_QK || F % ORC_QK) return -1;
+    if (!pos_list) n_pos = T * k;
+    size_t gstride = orc_expert_stride(F, D, qtype);
+    size_t dstride = orc_expert_stride(D, F, qtype);
+    int maxW = D > F ? D : F;
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+#endif
+    for (int n = 0; n < n_pos; n++) {
+        int pos = pos_list ? pos_list[n] : n;
+        if (pos < 0 || pos >= T * k) { bad |= 1; continue; }
+        int e = 0;
+        while (e < E && offsets[e + 1] <= pos) e++;
+        if (e >= E) { bad |= 1; continue; }
+        int t = perm[pos] / k;
+        double *xt = (double *)malloc(sizeof(double) * (size_t)D);
+        double *wrow = (double *)malloc(sizeof(double) * (size_t)maxW);
+        double *h = (double *)malloc(sizeof(double) * (size_t)F);
+        for (int i = 0; i < D; i++) xt[i] = (double)x[(size_t)t * D + i];
+        orc_expert_ffn_row(xt, gate + e * gstride, up + e * gstride,
+                           down + e * dstride, qtype, D, F, wrow, h,
+                           Y + (size_t)n * D);
+        free(xt); free(wrow); free(h);
+    }
+    return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Expert-cache LRU simulation (one layer).
+ *
+ * Rules (the pages name LRU replacement only; these fill in the rest):
+ *  - n_slots device slots, all empty at start;
+ *  - a request is a list of distinct expert ids for one step; it fails
+ *    (returns -2) if it holds more ids than slots, -1 on a bad id;
+ *  - every requested expert is stamped with the step number;
+ *  - ids are served in the order given; a resident id is a hit;
+ *  - a missing id takes the empty slot of lowest index if there is one,
+ *    otherwise evicts the resident expert with the oldest stamp that is not
+ *    requested in this step, the lower expert id on equal stamps.
+ * Outputs per requested id: slot[i], miss[i] (0/1), evicted[i] (expert id
+ * evicted to make room, or -1).  Returns the number of misses.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int E, n_slots;
+    int64_t step;
+    int32_t *slot_expert;   /* [n_slots], -1 = empty */
+    int32_t *expert_slot;   /* [E], -1 = not resident */
+    int64_t *stamp;         /* [E] */
+} orc_lru;
+
+void *orc_lru_new(int E, int n_slots)
+{
+    orc_lru *c = (orc_lru *)calloc(1, sizeof(orc_lru));
+    c->E = E; c->n_slots = n_slots; c->step = 0;
+    c->slot_expert = (int32_t *)malloc(sizeof(int32_t) * (size_t)n_slots);
+    c->expert_slot = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    c->stamp = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    for (int s = 0; s < n_slots; s++) c->slot_expert[s] = -1;
+    for (int e = 0; e < E; e++) c->expert_slot[e] = -1;
+    return c;
+}
+
+void orc_lru_free(void *p)
+{
+    orc_lru *c = (orc_lru *)p;
+    if (!c) return;
+    free(c->slot_expert); free(c->expert_slot); free(c->stamp); free(c);
+}
+
+int orc_lru_request(void *p, const int32_t *ids, int n, int32_t *slot,
+                    int32_t *miss, int32_t *evicted)
+{
+    orc_lru *c = (orc_lru *)p;
+    if (n > c->n_slots) return -2;
+    for (int i = 0; i < n; i++) {
+        if (ids[i] < 0 || ids[i] >= c->E) return -1;
+        for (int j = 0; j < i; j++) if (ids[j] == ids[i]) return -1;
+    }
+    c->step++;
+    char *wanted = (char *)calloc((size_t)c->E, 1);
+    for (int i = 0; i < n; i++) wanted[ids[i]] = 1;
+    int misses = 0;
+    for (int i = 0; i < n; i++) {
+        int e = ids[i];
+        evicted[i] = -1;
+        if (c->expert_slot[e] >= 0) {
+            slot[i] = c->expert_slot[e];
+            miss[i] = 0;
+        } else {
+            int s = -1;
+            for (int q = 0; q < c->n_slots; q++)
+                if (c->slot_expert[q] < 0) { s = q; break; }
+            if (s < 0) {
+                int victim = -1;
+                for (int v = 0; v < c->E; v++) {
+                    if (c->expert_slot[v] < 0 || wanted[v]) continue;
+                    if (victim < 0 || c->stamp[v] < c->stamp[victim]) victim = v;
+                }
+                s = c->expert_slot[victim];
+                c->expert_slot[victim] = -1;
+                evicted[i] = victim;
+            }
+            c->slot_expert[s] = e;
+            c->expert_slot[e] = s;
+            slot[i] = s;
+            miss[i] = 1;
+            misses++;
+        }
+        c->stamp[e] = c->step;
+    }
+    free(wanted);
+    return misses;
+}

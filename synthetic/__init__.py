@@ -1,0 +1,313 @@
+"""Seeded synthetic inputs for the routed, block-quantized MoE FFN layer.
+
+This module is shared by the CUDA path's tests/bench and by the oracle's tests.
+It only *produces inputs*: random activations, router weights and biases,
+routing traces, and ggml-style block encodings (Q8_0 / Q4_0) of random expert
+weights.  It holds none of the layer's arithmetic (no dequantization, routing,
+softmax, SwiGLU or combine); the decoders live separately in ``oracle/`` and in
+the CUDA library and share no code.
+
+Block formats (the quant types named in the FreeToken fork README, "Quant
+types" table: Standard family Q4_0 / Q8_0), 32 weights per block, blocks run
+along the reduction dimension of each weight row:
+
+* Q8_0: ``{fp16 d; int8 qs[32]}``  (34 bytes), value ``qs[i] * d``.
+* Q4_0: ``{fp16 d; uint8 qs[16]}`` (18 bytes), value ``(q_i - 8) * d`` where
+  byte ``j`` holds element ``j`` in its low nibble and element ``j + 16`` in its
+  high nibble (the GGUF order).
+
+Expert pools follow the FreeToken fork README, "Known limits": experts stored
+back to back as ``expert * nrows * (ncols / 32)`` blocks with no padding and
+one quant type for the whole pool.  Per expert, ``W_gate`` and ``W_up`` are
+``[F rows][D/32 blocks]`` and ``W_down`` is ``[D rows][F/32 blocks]``.
+
+Workload recipes (shapes, distributions, seeds) are in ``CONFIGS``.
+"""
+from __future__ import annotations
+
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field
+
+import numpy as np
+
+QK = 32
+Q4_0 = "q4_0"
+Q8_0 = "q8_0"
+# bytes per 32-weight block; a test checks these against include/moe.h
+BLOCK_BYTES = {Q4_0: 18, Q8_0: 34}
+# ggml type ids, also exported by the C header
+GGML_TYPE_ID = {Q4_0: 2, Q8_0: 8}
+
+
+# --------------------------------------------------------------------------
+# configurations
+# --------------------------------------------------------------------------
+@dataclass(frozen=True)
+class LayerConfig:
+    name: str
+    T: int
+    D: int
+    E: int
+    k: int
+    F: int
+    qtype: str
+    x_dtype: str            # "f32" or "bf16"
+    y_dtype: str            # "f32" or "bf16"
+    router_std: float = 0.02
+    expert_std: float = 0.02
+    zipf_s: float | None = None          # per-expert router bias (prefill config)
+    logits_from_trace: bool = False      # routing logits given directly
+    shared_F: int = 0                    # always-on shared expert, Q8_0
+    seed: int = 1000
+    renorm: bool = True
+    T_values: tuple = field(default_factory=tuple)   # documentation only
+
+
+CONFIGS = {
+    # Tiny routed layer: fp32 activations, Q8_0 experts, fp32 output.
+    "tiny": LayerConfig("tiny", T=4, D=256, E=8, k=2, F=512, qtype=Q8_0,
+                        x_dtype="f32", y_dtype="f32", router_std=0.05,
+                        seed=1000),
+    # Decode, 30B-A3B-shaped layer in Q4_0 at T in {1, 4, 16}.
+    "decode": LayerConfig("decode", T=16, D=2048, E=128, k=8, F=768,
+                          qtype=Q4_0, x_dtype="bf16", y_dtype="bf16",
+                          seed=1001, T_values=(1, 4, 16)),
+    # Prefill, same shapes in Q8_0, T=8192, Zipf(1.1) router bias.
+    "prefill": LayerConfig("prefill", T=8192, D=2048, E=128, k=8, F=768,
+                           qtype=Q8_0, x_dtype="bf16", y_dtype="bf16",
+                           zipf_s=1.1, seed=1002),
+    # Wide-expert layer: E=512, top-10, F=512, Q4_0 routed + Q8_0 shared
+    # expert, routing logits from a temporal-locality trace, T in {1, 2048}.
+    "wide": LayerConfig("wide", T=2048, D=2048, E=512, k=10, F=512,
+                        qtype=Q4_0, x_dtype="bf16", y_dtype="bf16",
+                        logits_from_trace=True, shared_F=512, seed=1003,
+                        T_values=(1, 2048)),
+    # Expert-cache streaming: 40 layers of the decode layer in Q8_0.
+    "cache": LayerConfig("cache", T=1, D=2048, E=128, k=8, F=768, qtype=Q8_0,
+                         x_dtype="bf16", y_dtype="bf16",
+                         logits_from_trace=True, seed=1004),
+}
+CACHE_LAYERS = 40
+CACHE_STEPS = 256
+CACHE_FRACTION = 0.4
+
+
+def with_T(cfg: LayerConfig, T: int) -> LayerConfig:
+    d = dict(cfg.__dict__)
+    d["T"] = T
+    return LayerConfig(**d)
+
+
+def expert_bytes(D: int, F: int, qtype: str) -> tuple[int, int, int]:
+    """Bytes of (gate, up, down) of one expert in the pool layout."""
+    bs = BLOCK_BYTES[qtype]
+    return F * (D // QK) * bs, F * (D // QK) * bs, D * (F // QK) * bs
+
+
+# --------------------------------------------------------------------------
+# scalar encodings
+# --------------------------------------------------------------------------
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (nearest, ties to even); returns uint16 bits."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    rounding = ((u >> 16) & 1) + np.uint32(0x7FFF)
+    return ((u + rounding) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _round_half_away(v: np.ndarray) -> np.ndarray:
+    return np.sign(v) * np.floor(np.abs(v) + np.float32(0.5))
+
+
+# --------------------------------------------------------------------------
+# block encoders (input generation only)
+# --------------------------------------------------------------------------
+def quantize_q8_0(w: np.ndarray) -> np.ndarray:
+    """Encode rows of float32 weights as Q8_0 blocks.
+
+    ``w``: [rows, cols] with cols % 32 == 0.  Returns uint8 [rows, cols/32*34].
+    Scale d = max|w| / 127 per block (fp32), q = round-half-away(w / d),
+    d stored as fp16.  An all-zero block gets d = 0, q = 0.
+    """
+    rows, cols = w.shape
+    assert cols % QK == 0
+    b = np.ascontiguousarray(w, dtype=np.float32).reshape(rows, cols // QK, QK)
+    amax = np.abs(b).max(axis=2)
+    d = (amax / np.float32(127.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = _round_half_away(b / d[..., None])
+    q = np.where(d[..., None] > 0, q, 0)
+    q = np.clip(q, -127, 127).astype(np.int8)
+    out = np.empty((rows, cols // QK, 34), dtype=np.uint8)
+    out[..., 0:2] = d.astype(np.float16).view(np.uint8).reshape(rows, cols // QK, 2)
+    out[..., 2:] = q.view(np.uint8)
+    return out.reshape(rows, -1)
+
+
+def quantize_q4_0(w: np.ndarray) -> np.ndarray:
+    """Encode rows of float32 weights as Q4_0 blocks.
+
+    Per block: m = the signed weight of largest magnitude (the positive one
+    when a positive and a negative weight tie in magnitude), d = -m / 8 so
+    that m lands exactly on code 0, q = clamp(round-half-away(w / d) + 8, 0,
+    15), d stored as fp16; value (q - 8) * d.  An all-zero block gets d = 0
+    and q = 8.  Returns uint8 [rows, cols/32*18].
+    """
+    rows, cols = w.shape
+    assert cols % QK == 0
+    b = np.ascontiguousarray(w, dtype=np.float32).reshape(rows, cols // QK, QK)
+    hi = b.max(axis=2)
+    lo = b.min(axis=2)
+    m = np.where(hi >= -lo, hi, lo)
+    d = (m / np.float32(-8.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = _round_half_away(b / d[..., None]) + 8
+    q = np.where(d[..., None] != 0, q, 8)
+    q = np.clip(q, 0, 15).astype(np.uint8)
+    out = np.empty((rows, cols // QK, 18), dtype=np.uint8)
+    out[..., 0:2] = d.astype(np.float16).view(np.uint8).reshape(rows, cols // QK, 2)
+    out[..., 2:] = q[..., :16] | (q[..., 16:] << 4)
+    return out.reshape(rows, -1)
+
+
+def quantize(w: np.ndarray, qtype: str) -> np.ndarray:
+    if qtype == Q8_0:
+        return quantize_q8_0(w)
+    if qtype == Q4_0:
+        return quantize_q4_0(w)
+    raise ValueError(f"unknown qtype {qtype}")
+
+
+# --------------------------------------------------------------------------
+# layer inputs
+# --------------------------------------------------------------------------
+def gen_expert_pool(seed: int, n_experts: int, D: int, F: int, qtype: str,
+                    std: float, threads: int | None = None):
+    """Draw n_experts SwiGLU experts ~N(0, std) and encode them.
+
+    Expert e draws from its own stream ``default_rng([seed, e])`` (gate, up,
+    down in that order), so the bytes do not depend on the thread count.
+    Returns (gate, up, down) uint8 arrays of shapes
+    [n, F, D/32*bs], [n, F, D/32*bs], [n, D, F/32*bs] (the pool layout).
+    """
+    bs = BLOCK_BYTES[qtype]
+    gate = np.empty((n_experts, F, D // QK * bs), np.uint8)
+    up = np.empty_like(gate)
+    down = np.empty((n_experts, D, F // QK * bs), np.uint8)
+    s32 = np.float32(std)
+
+    def one(e):
+        r = np.random.default_rng([seed, e])
+        gate[e] = quantize(r.standard_normal((F, D), np.float32) * s32, qtype)
+        up[e] = quantize(r.standard_normal((F, D), np.float32) * s32, qtype)
+        down[e] = quantize(r.standard_normal((D, F), np.float32) * s32, qtype)
+
+    if threads is None:
+        threads = min(32, os.cpu_count() or 1)
+    if threads <= 1 or n_experts == 1:
+        for e in range(n_experts):
+            one(e)
+    else:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(one, range(n_experts)))
+    return gate, up, down
+
+
+def zipf_bias(rng: np.random.Generator, E: int, s: float) -> np.ndarray:
+    """Per-expert router bias b_e = ln p_e with p_e proportional to rank_e^-s
+    over a random ranking of the experts (skews expert loads)."""
+    rank = rng.permutation(E) + 1
+    p = rank.astype(np.float64) ** (-s)
+    p /= p.sum()
+    return np.log(p).astype(np.float32)
+
+
+def locality_trace(rng: np.random.Generator, T: int, E: int, k: int,
+                   repeat: float = 0.8):
+    """Routing logits [T, E] whose top-k follows a temporal-locality trace.
+
+    Token 0 takes a uniform k-subset.  Token t keeps
+    n_rep = floor(repeat*k) + Bernoulli(frac(repeat*k)) experts drawn uniformly
+    from token t-1's set and draws the rest uniformly from the other experts.
+    The logits of each token are E draws of N(0,1), sorted, the k largest
+    given to the chosen set in random order and the rest to the others in
+    random order, so the top-k of the row is exactly the chosen set.
+    Returns (logits float32 [T, E], sets int32 [T, k]).
+    """
+    base = repeat * k
+    n_lo = int(math.floor(base))
+    frac = base - n_lo
+    logits = np.empty((T, E), np.float32)
+    sets = np.empty((T, k), np.int32)
+    prev = None
+    for t in range(T):
+        if prev is None:
+            cur = rng.choice(E, size=k, replace=False)
+        else:
+            n_rep = n_lo + int(rng.random() < frac)
+            n_rep = min(n_rep, k)
+            keep = rng.choice(prev, size=n_rep, replace=False)
+            others = np.setdiff1d(np.arange(E), prev, assume_unique=False)
+            new = rng.choice(others, size=k - n_rep, replace=False)
+            cur = np.concatenate([keep, new])
+        vals = np.sort(rng.standard_normal(E).astype(np.float32))[::-1]
+        row = np.empty(E, np.float32)
+        rest = np.setdiff1d(np.arange(E), cur)
+        row[rng.permutation(cur)] = vals[:k]
+        row[rng.permutation(rest)] = vals[k:]
+        logits[t] = row
+        sets[t] = cur
+        prev = cur
+    return logits, sets
+
+
+@dataclass
+class LayerInputs:
+    cfg: LayerConfig
+    x: np.ndarray                 # [T, D] float32 values (exact for bf16)
+    x_raw: np.ndarray             # bytes the GPU reads: float32 or uint16 bf16 bits
+    w_router: np.ndarray | None   # [D, E] float32
+    bias: np.ndarray | None       # [E] float32
+    logits: np.ndarray | None     # [T, E] float32 when routing comes from a trace
+    gate: np.ndarray              # pool bytes (see gen_expert_pool)
+    up: np.ndarray
+    down: np.ndarray
+    shared: tuple | None          # (gate, up, down) with one expert, Q8_0
+
+
+def gen_activations(rng: np.random.Generator, T: int, D: int, dtype: str):
+    x = rng.standard_normal((T, D), np.float32)
+    if dtype == "bf16":
+        raw = f32_to_bf16_bits(x)
+        return bf16_bits_to_f32(raw), raw
+    return x, x.copy()
+
+
+def make_layer(cfg: LayerConfig, T: int | None = None, seed: int | None = None,
+               experts: bool = True) -> LayerInputs:
+    """All inputs of one layer call, deterministic in (cfg, T, seed)."""
+    T = cfg.T if T is None else T
+    seed = cfg.seed if seed is None else seed
+    rng = np.random.default_rng([seed, 0x5EED, T])
+    if experts:
+        gate, up, down = gen_expert_pool(seed, cfg.E, cfg.D, cfg.F, cfg.qtype, cfg.expert_std)
+    else:
+        gate = up = down = None
+    shared = None
+    if cfg.shared_F:
+        shared = gen_expert_pool(seed + 7777, 1, cfg.D, cfg.shared_F, Q8_0, cfg.expert_std)
+    w_router = bias = logits = None
+    if cfg.logits_from_trace:
+        logits, _ = locality_trace(rng, T, cfg.E, cfg.k)
+    else:
+        w_router = (rng.standard_normal((cfg.D, cfg.E), np.float32)
+                    * np.float32(cfg.router_std))
+        if cfg.zipf_s is not None:
+            bias = zipf_bias(rng, cfg.E, cfg.zipf_s)
+    x, x_raw = gen_activations(rng, T, cfg.D, cfg.x_dtype)
+    return LayerInputs(cfg, x, x_raw, w_router, bias, logits, gate, up, down, shared)

@@ -1,0 +1,368 @@
+"""Pins of the CPU oracle against facts fixed outside it.
+
+Each test checks the oracle against something other than itself: the IEEE
+binary16 definition, hand-packed blocks with closed-form values, numpy's own
+routines on special cases, brute force on tiny inputs, invariants, or a
+hand-worked LRU trace.  A plausible slip in the oracle (a dropped term, a
+wrong sign or index, a transposed operand, a swapped nibble) fails one of them.
+"""
+import itertools
+import os
+
+import numpy as np
+import pytest
+
+import synthetic as S
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- fp16 scale
+@pytest.mark.parametrize("bits,val", [
+    (0x3C00, 1.0), (0xC000, -2.0), (0x3555, 0.333251953125), (0x7BFF, 65504.0),
+    (0x0001, 2.0 ** -24), (0x03FF, 1023 * 2.0 ** -24), (0x0400, 2.0 ** -14),
+    (0x8000, -0.0), (0x5A00, 192.0), (0xB400, -0.25),
+])
+def test_half_to_double_known_patterns(orc, bits, val):
+    assert orc.half_to_double(bits) == val
+
+
+def test_half_to_double_matches_numpy_all_finite(orc):
+    # every finite binary16 pattern against numpy's own float16 conversion
+    for bits in range(0, 0x10000, 7):
+        ref = float(np.array([bits], np.uint16).view(np.float16)[0])
+        got = orc.half_to_double(bits)
+        if np.isnan(ref):
+            assert np.isnan(got)
+        else:
+            assert got == ref, hex(bits)
+
+
+# ---------------------------------------------------------- hand-packed blocks
+def _golden_blocks():
+    out = []
+    with open(os.path.join(GOLDEN, "blocks.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            parts = line.split()
+            out.append((parts[0], parts[1], bytes.fromhex(parts[2]),
+                        np.array([float(v) for v in parts[3:]])))
+    return out
+
+
+@pytest.mark.parametrize("name,qtype,raw,vals", _golden_blocks(),
+                         ids=[b[0] for b in _golden_blocks()])
+def test_dequant_hand_packed_blocks(orc, name, qtype, raw, vals):
+    assert len(raw) == S.BLOCK_BYTES[qtype] == orc.block_bytes(qtype)
+    got = orc.dequant_row(np.frombuffer(raw, np.uint8), qtype, 32)
+    np.testing.assert_array_equal(got, vals)
+
+
+def test_dequant_row_of_several_blocks_keeps_block_order(orc):
+    blocks = _golden_blocks()
+    q4 = [b for b in blocks if b[1] == "q4_0"]
+    raw = b"".join(b[2] for b in q4)
+    got = orc.dequant_row(np.frombuffer(raw, np.uint8), "q4_0", 32 * len(q4))
+    np.testing.assert_array_equal(got, np.concatenate([b[3] for b in q4]))
+
+
+@pytest.mark.parametrize("qtype,slack,top", [("q8_0", 127, 127), ("q4_0", 8, 7)])
+def test_quantizer_roundtrip_error_bound(orc, qtype, slack, top):
+    # encoder (input generator) + decoder (oracle): |w - dequant(w)| <= |d|/2
+    # up to the fp16 rounding of d (relative 2^-11, times the largest code),
+    # except where the code clips at the top of the range: Q4_0 codes span
+    # [-8, 7] * d, so a weight of the opposite sign to the block's largest
+    # one can exceed 7.5|d| and lands on 7d (error |w| - 7|d| <= |d|).
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((16, 256)) * 0.02).astype(np.float32)
+    w[3, 32:64] = 0.0                      # an all-zero block
+    packed = S.quantize(w, qtype)
+    deq = orc.dequant_matrix(packed, qtype, 256)
+    bs = S.BLOCK_BYTES[qtype]
+    d16 = np.abs(packed.reshape(16, 8, bs)[:, :, :2].copy().view(np.float16)[..., 0]
+                 .astype(np.float64))
+    dd = np.repeat(d16, 32, axis=1)
+    bound = np.maximum(0.5 * dd, np.abs(w) - top * dd) + slack * 2.0 ** -11 * dd + 1e-12
+    assert np.all(np.abs(deq - w) <= bound)
+    assert np.all(np.abs(deq - w) <= dd * (1 + slack * 2.0 ** -11) + 1e-12)
+    assert np.all(deq[3, 32:64] == 0.0)
+
+
+def test_q4_0_largest_weight_lands_on_code_zero(orc):
+    rng = np.random.default_rng(6)
+    w = (rng.standard_normal((4, 64)) * 0.02).astype(np.float32)
+    packed = S.quantize_q4_0(w).reshape(4, 2, 18)
+    deq = orc.dequant_matrix(packed.reshape(4, -1), "q4_0", 64).reshape(4, 2, 32)
+    wb = w.reshape(4, 2, 32)
+    for r in range(4):
+        for b in range(2):
+            i = np.argmax(np.abs(wb[r, b]))
+            code = (packed[r, b, 2 + i % 16] >> (0 if i < 16 else 4)) & 0xF
+            assert code == 0
+            d16 = float(packed[r, b, :2].copy().view(np.float16)[0])
+            assert abs(deq[r, b, i] - wb[r, b, i]) <= 8 * abs(d16) * 2.0 ** -10
+
+
+# --------------------------------------------------------------- router logits
+def test_router_logits_against_numpy_matmul(orc):
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((5, 64)).astype(np.float32)
+    w = (rng.standard_normal((64, 12)) * 0.05).astype(np.float32)
+    b = rng.standard_normal(12).astype(np.float32)
+    ref = (x.astype(np.float64) @ w.astype(np.float64) + b).astype(np.float32)
+    np.testing.assert_array_equal(orc.router_logits(x, w, b), ref)
+
+
+def test_router_logits_identity_router_returns_x(orc):
+    x = np.arange(24, dtype=np.float32).reshape(3, 8) / 7
+    np.testing.assert_array_equal(orc.router_logits(x, np.eye(8, dtype=np.float32)), x)
+
+
+# ---------------------------------------------------------- top-k and gates
+def test_topk_brute_force_all_subsets(orc):
+    rng = np.random.default_rng(8)
+    for E, k in [(5, 2), (6, 3), (7, 1), (8, 4), (6, 6)]:
+        L = rng.standard_normal((20, E)).astype(np.float32)
+        ids, g = orc.select(L, k)
+        for t in range(20):
+            best = max(itertools.combinations(range(E), k),
+                       key=lambda s: sum(float(L[t, i]) for i in s))
+            assert set(ids[t]) == set(best)
+            assert list(L[t, ids[t]]) == sorted(L[t, ids[t]], reverse=True)
+
+
+def test_topk_ties_go_to_lower_index(orc):
+    L = np.array([[1, 3, 3, 2, 3], [0, 0, 0, 0, 0], [5, 4, 5, 4, 5]], np.float32)
+    ids, _ = orc.select(L, 3)
+    np.testing.assert_array_equal(ids, [[1, 2, 4], [0, 1, 2], [0, 2, 4]])
+
+
+def test_gates_are_softmax_of_selected_logits(orc):
+    rng = np.random.default_rng(9)
+    L = (rng.standard_normal((50, 32)) * 3).astype(np.float32)
+    ids, g = orc.select(L, 6)
+    sel = np.take_along_axis(L.astype(np.float64), ids, axis=1)
+    ref = np.exp(sel - sel.max(axis=1, keepdims=True))
+    ref /= ref.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(g, ref, rtol=1e-12, atol=0)
+    assert np.all(np.abs(g.sum(axis=1) - 1) <= 1e-12)
+    assert np.all(np.diff(g, axis=1) <= 0)    # descending logits -> descending gates
+
+
+def test_gates_without_renorm_are_full_softmax(orc):
+    rng = np.random.default_rng(10)
+    L = rng.standard_normal((10, 16)).astype(np.float32)
+    ids, g = orc.select(L, 4, renorm=False)
+    p = np.exp(L.astype(np.float64) - L.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(g, np.take_along_axis(p, ids, axis=1), rtol=1e-12)
+    ids_all, g_all = orc.select(L, 16)
+    np.testing.assert_allclose(g_all.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+
+
+def test_near_tie_detector(orc):
+    L = np.array([[3.0, 2.0, 1.0, 0.0],
+                  [3.0, 2.0, 2.0 - 5e-6, 0.0],     # k-th vs (k+1)-th gap
+                  [3.0, 3.0 - 2e-6, 1.0, 0.0]],    # gap inside the top-k
+                 np.float32)
+    np.testing.assert_array_equal(orc.near_tie_tokens(L, 2), [1, 2])
+
+
+# ---------------------------------------------------------------- permutation
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (4, 2, 8), (37, 8, 128), (300, 10, 512)])
+def test_permutation_invariants(orc, T, k, E):
+    rng = np.random.default_rng(T)
+    ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    counts, offsets, perm, inv = orc.permute(ids, E)
+    flat = ids.ravel()
+    np.testing.assert_array_equal(counts, np.bincount(flat, minlength=E))
+    assert offsets[0] == 0 and offsets[-1] == T * k
+    assert np.all(np.diff(offsets) == counts)
+    np.testing.assert_array_equal(perm[inv], np.arange(T * k))
+    np.testing.assert_array_equal(inv[perm], np.arange(T * k))
+    # library stable sort gives the same order (expert, then t, then j)
+    np.testing.assert_array_equal(perm, np.argsort(flat, kind="stable"))
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]]
+        assert np.all(flat[seg] == e) and np.all(np.diff(seg) > 0)
+
+
+# ------------------------------------------------------------------ the layer
+def _textbook_swiglu(x, Wg, Wu, Wd):
+    a = x @ Wg.T
+    u = x @ Wu.T
+    h = a / (1.0 + np.exp(-a)) * u
+    return h @ Wd.T
+
+
+def _pack_int_matrix(codes, qtype, dbits=0x3C00):
+    """Pack an integer matrix with scale 1.0 in every block (test-side
+    packing by the format definition; values = codes)."""
+    rows, cols = codes.shape
+    blocks = codes.reshape(rows, cols // 32, 32)
+    lo = blocks.astype(np.int64)
+    if qtype == "q8_0":
+        body = (lo & 0xFF).astype(np.uint8)
+    else:
+        c = (lo + 8).astype(np.uint8)
+        body = c[..., :16] | (c[..., 16:] << 4)
+    d = np.full((rows, cols // 32, 2), [dbits & 0xFF, dbits >> 8], np.uint8)
+    return np.concatenate([d, body], axis=2).reshape(rows, -1)
+
+
+@pytest.mark.parametrize("qtype", ["q8_0", "q4_0"])
+def test_single_expert_is_textbook_swiglu(orc, qtype):
+    # integer-valued weights (scale 1) so the dequantized matrices are known
+    # exactly; E=1, k=1 reduces the layer to a plain SwiGLU FFN.
+    rng = np.random.default_rng(11)
+    D, F = 64, 96
+    lo, hi = (-8, 8) if qtype == "q4_0" else (-20, 21)
+    Wg = rng.integers(lo, hi, (F, D))
+    Wu = rng.integers(lo, hi, (F, D))
+    Wd = rng.integers(lo, hi, (D, F))
+    x = (rng.integers(-3, 4, (3, D)) / 16).astype(np.float32)
+    gate = _pack_int_matrix(Wg, qtype)[None]
+    up = _pack_int_matrix(Wu, qtype)[None]
+    down = _pack_int_matrix(Wd, qtype)[None]
+    ids = np.zeros((3, 1), np.int32)
+    g = np.ones((3, 1))
+    y = orc.layer(x, ids, g, gate, up, down, qtype, F)
+    ref = _textbook_swiglu(x.astype(np.float64), Wg.astype(float), Wu.astype(float), Wd.astype(float))
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-9 * np.abs(ref).max())
+
+
+def test_routed_layer_is_gate_weighted_sum_of_single_experts(orc):
+    cfg = S.CONFIGS["tiny"]
+    L = S.make_layer(cfg)
+    _, ids, g = orc.route(L.x, L.w_router, None, cfg.k)
+    y = orc.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F)
+    for t in range(cfg.T):
+        acc = np.zeros(cfg.D)
+        for j in range(cfg.k):
+            e = ids[t, j]
+            ye = orc.layer(L.x[t:t + 1], np.zeros((1, 1), np.int32), np.ones((1, 1)),
+                           L.gate[e:e + 1], L.up[e:e + 1], L.down[e:e + 1], cfg.qtype, cfg.F)
+            acc += g[t, j] * ye[0]
+        np.testing.assert_allclose(y[t], acc, rtol=1e-12, atol=1e-15)
+
+
+def test_dense_masked_equals_routed(orc):
+    cfg = S.CONFIGS["tiny"]
+    L = S.make_layer(cfg)
+    _, ids, g = orc.route(L.x, L.w_router, None, cfg.k)
+    y = orc.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F)
+    yd = orc.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F, dense=True)
+    assert np.abs(y - yd).max() <= 1e-12 * np.abs(y).max()
+
+
+def test_dequantized_dense_evaluation_matches_layer(orc):
+    # dequantize each expert with the pinned block decoder and evaluate the
+    # textbook FFN with numpy; must equal the oracle's routed layer
+    cfg = S.CONFIGS["tiny"]
+    L = S.make_layer(cfg)
+    _, ids, g = orc.route(L.x, L.w_router, None, cfg.k)
+    y = orc.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F)
+    x64 = L.x.astype(np.float64)
+    ref = np.zeros_like(y)
+    for t in range(cfg.T):
+        for j in range(cfg.k):
+            e = ids[t, j]
+            Wg = orc.dequant_matrix(L.gate[e], cfg.qtype, cfg.D)
+            Wu = orc.dequant_matrix(L.up[e], cfg.qtype, cfg.D)
+            Wd = orc.dequant_matrix(L.down[e], cfg.qtype, cfg.F)
+            ref[t] += g[t, j] * _textbook_swiglu(x64[t:t + 1], Wg, Wu, Wd)[0]
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-12 * np.abs(ref).max())
+
+
+def test_shared_expert_adds_with_weight_one(orc):
+    rng = np.random.default_rng(12)
+    D, F, E, k, sF = 64, 64, 4, 2, 32
+    gate, up, down = S.gen_expert_pool(3, E, D, F, "q4_0", 0.05, threads=1)
+    shared = S.gen_expert_pool(4, 1, D, sF, "q8_0", 0.05, threads=1)
+    x = rng.standard_normal((3, D)).astype(np.float32)
+    ids = np.array([[0, 1], [2, 3], [1, 2]], np.int32)
+    g = np.array([[0.7, 0.3], [0.5, 0.5], [0.9, 0.1]])
+    y0 = orc.layer(x, ids, g, gate, up, down, "q4_0", F)
+    y1 = orc.layer(x, ids, g, gate, up, down, "q4_0", F, shared=shared)
+    ys = orc.layer(x, np.zeros((3, 1), np.int32), np.ones((3, 1)), *shared, "q8_0", sF)
+    np.testing.assert_allclose(y1, y0 + ys, rtol=1e-12, atol=1e-15)
+
+
+def test_token_subset_and_expert_rows(orc):
+    cfg = S.CONFIGS["tiny"]
+    L = S.make_layer(cfg)
+    _, ids, g = orc.route(L.x, L.w_router, None, cfg.k)
+    y = orc.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F)
+    ys = orc.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F, tokens=[3, 1])
+    np.testing.assert_array_equal(ys, y[[3, 1]])
+    counts, offsets, perm, inv = orc.permute(ids, cfg.E)
+    Y = orc.expert_rows(L.x, perm, offsets, cfg.k, L.gate, L.up, L.down, cfg.qtype, cfg.F)
+    comb = np.zeros_like(y)
+    for t in range(cfg.T):
+        for j in range(cfg.k):
+            comb[t] += g[t, j] * Y[inv[t * cfg.k + j]]
+    np.testing.assert_allclose(comb, y, rtol=1e-12, atol=1e-15)
+
+
+# ------------------------------------------------------------------ LRU cache
+def test_lru_hand_worked_trace(orc):
+    # E=6 experts, 3 slots; every requested expert is stamped with the step
+    # number (1, 2, ...).  Worked by hand from the replacement rules:
+    #  1: [0,1] both miss, empty slots 0,1             stamps 0@1 1@1
+    #  2: [1,2] 1 hits; 2 takes empty slot 2            1@2 2@2
+    #  3: [3]   no empty slot; oldest unrequested is 0  -> slot 0, evicts 0
+    #  4: [1,4] 1 hits; 4: oldest unrequested is 2@2 (3@3 is newer) -> slot 2
+    #  5: [5,0] 5: oldest of {3@3, 1@4, 4@4} is 3 -> slot 0;
+    #           0: 1@4 and 4@4 tie -> lower expert id 1 -> slot 1
+    c = orc.LRU(6, 3)
+    steps = [
+        ([0, 1], [0, 1], [True, True], [-1, -1]),
+        ([1, 2], [1, 2], [False, True], [-1, -1]),
+        ([3], [0], [True], [0]),
+        ([1, 4], [1, 2], [False, True], [-1, 2]),
+        ([5, 0], [0, 1], [True, True], [3, 1]),
+    ]
+    for req, slots, misses, ev in steps:
+        s, m, e = c.request(np.array(req, np.int32))
+        assert list(s) == slots and list(m) == misses and list(e) == ev, req
+
+
+def test_lru_wanted_expert_is_never_evicted(orc):
+    c = orc.LRU(5, 2)
+    c.request([1])          # 1@1 -> slot 0
+    c.request([0])          # 0@2 -> slot 1
+    # 1 is the least recently used but is requested again in this step, so
+    # the miss on 4 must evict 0 instead
+    s, m, e = c.request([4, 1])
+    assert list(m) == [True, False] and list(e) == [0, -1] and list(s) == [1, 0]
+
+
+def test_lru_capacity_and_bad_ids(orc):
+    c = orc.LRU(8, 3)
+    with pytest.raises(OverflowError):
+        c.request([0, 1, 2, 3])
+    with pytest.raises(ValueError):
+        c.request([0, 0])
+    with pytest.raises(ValueError):
+        c.request([9])
+
+
+def test_lru_invariants_random_trace(orc):
+    rng = np.random.default_rng(13)
+    E, n_slots, k = 32, 12, 8
+    c = orc.LRU(E, n_slots)
+    resident = {}
+    total_miss = 0
+    for step in range(200):
+        req = rng.choice(E, k, replace=False).astype(np.int32)
+        s, m, ev = c.request(req)
+        for e, slot, miss, vic in zip(req, s, m, ev):
+            assert miss == (e not in resident)
+            if vic >= 0:
+                assert vic not in req and resident.pop(vic) == slot
+            resident[e] = slot
+        assert len(resident) <= n_slots
+        assert len(set(resident.values())) == len(resident)
+        total_miss += int(m.sum())
+    assert 0 < total_miss < 200 * k
