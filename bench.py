@@ -1,0 +1,561 @@
+#!/usr/bin/env python
+"""Benchmark of the routed, block-quantized MoE FFN layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill|wide]
+
+One JSON line on rank 0.  Workloads (seeded synthetic inputs, see synthetic/):
+
+* decode (default): the 30B-A3B-shaped layer (D=2048, E=128, top-8,
+  F=768, Q4_0 experts, bf16 activations).  One step runs the layer at
+  T = 1, 4 and 16 tokens (21 tokens), each call on another replica of the
+  expert pool so that weights come from HBM, not L2 (6 replicas, 2 GB).
+* prefill: the same shapes in Q8_0 at T = 8192 with a Zipf(1.1) router
+  bias (skewed expert loads); 2 replicas of the pool.
+* wide: E=512, top-10, F=512 Q4_0 plus a Q8_0 shared expert, routing
+  logits from a temporal-locality trace, at T = 1 and T = 2048.
+
+Timing: W untimed steps, then K steps bracketed by a barrier and a device
+synchronize, timed with CUDA events on the launching stream; max over
+ranks.  Per-kernel times come from the library's own trace events recorded
+inside the timed steps (moe_trace).  SM clocks and throttle reasons are
+sampled through NVML while the timed steps run.  With N > 1 (torchrun)
+every rank runs an independent replica of the layer (the layer does not
+shard on one GPU's worth of work): weak scaling, no collective on the path.
+
+``--impl reference`` times the CPU oracle (oracle/) on the host cores on a
+bounded sample of the same workload: the only other place this file runs
+the oracle besides the cpu_baseline leg.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+HBM_SPEC_GBS = 8000.0
+TC_SPEC_TFLOPS = 2250.0
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """NVML sampling of SM clock and throttle reasons while a region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - no NVML
+            self.err = str(e)
+
+    def _poll(self):
+        nv = self.nv
+        while True:
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            if self._stop.wait(self.period):
+                break
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------- workloads
+def _dev_x(L, torch):
+    if L.cfg.x_dtype == "bf16":
+        return torch.from_numpy(L.x_raw.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(L.x_raw).cuda()
+
+
+class Workload:
+    """A list of layer calls making one step; replicas rotate per call."""
+
+    def __init__(self, name: str, torch, moe):
+        self.name = name
+        self.torch, self.moe = torch, moe
+        cfg = S.CONFIGS[name]
+        self.cfg = cfg
+        if name == "decode":
+            Ts, replicas = (1, 4, 16), 6
+        elif name == "prefill":
+            Ts, replicas = (8192,), 2
+        elif name == "wide":
+            Ts, replicas = (1, 2048), 2
+        else:
+            raise ValueError(name)
+        self.Ts = Ts
+        base = S.make_layer(cfg, T=max(Ts))
+        self.inputs = {max(Ts): base}
+        for T in Ts:
+            if T not in self.inputs:
+                self.inputs[T] = S.make_layer(cfg, T=T, experts=False)
+                self.inputs[T].gate, self.inputs[T].up, self.inputs[T].down = base.gate, base.up, base.down
+                self.inputs[T].shared = base.shared
+        dev = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        g, u, d = dev(base.gate), dev(base.up), dev(base.down)
+        self.expert_bytes = sum(S.expert_bytes(cfg.D, cfg.F, cfg.qtype))
+        self.pool_bytes = g.numel() + u.numel() + d.numel()
+        pools = [moe.ExpertPool(g, u, d, cfg.qtype)]
+        for _ in range(replicas - 1):
+            pools.append(moe.ExpertPool(g.clone(), u.clone(), d.clone(), cfg.qtype))
+        shared = None
+        if base.shared is not None:
+            sg, su, sd = (dev(a) for a in base.shared)
+            shared = moe.ExpertPool(sg, su, sd, "q8_0")
+            self.shared_bytes = sum(S.expert_bytes(cfg.D, cfg.shared_F, "q8_0"))
+        else:
+            self.shared_bytes = 0
+        xdt = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
+        ydt = torch.bfloat16 if cfg.y_dtype == "bf16" else torch.float32
+        self.layers = [moe.Layer(p, cfg.D, cfg.F, cfg.E, cfg.k, max(Ts), w_router=dev(base.w_router),
+                                 bias=dev(base.bias), shared=shared, shared_F=cfg.shared_F,
+                                 renorm=cfg.renorm, x_dtype=xdt, y_dtype=ydt) for p in pools]
+        self.x = {T: _dev_x(self.inputs[T], torch) for T in Ts}
+        self.logits = {T: dev(self.inputs[T].logits) for T in Ts}
+        self.y = {T: torch.empty((T, cfg.D), dtype=ydt, device="cuda") for T in Ts}
+        self.xdt, self.ydt = xdt, ydt
+        self.r = 0
+        self.tokens_per_step = sum(Ts)
+        self.calls_per_step = len(Ts)
+
+    def step(self, trace=None, x=None, y=None):
+        for T in self.Ts:
+            lay = self.layers[self.r]
+            self.r = (self.r + 1) % len(self.layers)
+            lay.forward(self.x[T] if x is None else x[T], logits=self.logits[T],
+                        out=self.y[T] if y is None else y[T], trace=trace)
+
+    # algorithmic work of one step, from the routing of each call
+    def distinct_experts(self):
+        out = {}
+        for T in self.Ts:
+            lay = self.layers[0]
+            lay.forward(self.x[T], logits=self.logits[T], out=self.y[T])
+            self.torch.cuda.synchronize()
+            out[T] = int(np.unique(lay.ids[:T].cpu().numpy()).size)
+        return out
+
+    def algorithmic(self):
+        cfg = self.cfg
+        distinct = self.distinct_experts()
+        gb, ub, db = S.expert_bytes(cfg.D, cfg.F, cfg.qtype)
+        act = 2 if cfg.x_dtype == "bf16" else 4
+        per_call = {}
+        for T in self.Ts:
+            n = distinct[T]
+            gateup = n * (gb + ub) + T * cfg.D * act + T * cfg.k * cfg.F * 4
+            down = n * db + T * cfg.k * cfg.F * 4 + T * cfg.k * cfg.D * 4
+            flops = 2.0 * T * cfg.k * 3 * cfg.D * cfg.F
+            if cfg.shared_F:
+                flops += 2.0 * T * 3 * cfg.D * cfg.shared_F
+            per_call[T] = {"distinct": n, "gateup_bytes": gateup, "down_bytes": down,
+                           "weight_bytes": n * (gb + ub + db) + self.shared_bytes,
+                           "flops": flops}
+        return per_call
+
+
+# ------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import torch
+    import quantized_routed_expert_top_b200 as moe
+    from quantized_routed_expert_top_b200 import build as B
+    if rank == 0 or not os.path.exists(moe.LIB_PATH):
+        B.build()
+    barrier(world)
+    moe.lib()
+    peaks = measured_peaks()
+    wl = Workload(args.workload, torch, moe)
+    algo = wl.algorithmic()
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, with the library's per-kernel trace events
+    trace = moe.KernelTrace(n_calls=args.steps * wl.calls_per_step)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            wl.step(trace=trace)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_step = t0.elapsed_time(t1) / args.steps
+    ms_step = max_over_ranks(ms_step, world)
+    durs = trace.durations()
+    launches = sum(len(c) for c in trace.calls)
+
+    # ---- end to end: pinned host x -> device, layer, device -> pinned host y
+    xh = {T: wl.x[T].cpu().pin_memory() for T in wl.Ts}
+    yh = {T: torch.empty(wl.y[T].shape, dtype=wl.ydt).pin_memory() for T in wl.Ts}
+    xd = {T: torch.empty_like(wl.x[T]) for T in wl.Ts}
+    h2d = sum(xh[T].numel() * xh[T].element_size() for T in wl.Ts)
+    d2h = sum(yh[T].numel() * yh[T].element_size() for T in wl.Ts)
+    if args.workload == "wide":
+        h2d += sum(wl.logits[T].numel() * 4 for T in wl.Ts)
+
+    def e2e_step():
+        for T in wl.Ts:
+            xd[T].copy_(xh[T], non_blocking=True)
+        wl.step(x=xd)
+        for T in wl.Ts:
+            yh[T].copy_(wl.y[T], non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    barrier(world)
+
+    tokens = wl.tokens_per_step * world
+    value = tokens / (ms_step / 1e3)
+    roof = roofline(wl, algo, durs, peaks, args)
+    out = {
+        "metric": "MoE-layer tokens/s",
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": dtype_of(wl.cfg),
+        "data": "synthetic (seeded; random-init Q4_0/Q8_0 experts, no checkpoint)",
+        "config": config_of(wl),
+        "roofline": roof,
+        "kernels_ms": {k: round(sum(v) / len(v), 5) for k, v in sorted(durs.items())},
+        "gpu_launches": launches,
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+        "peaks": peaks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, args)
+    if rank == 0 and args.workload == "decode" and not args.no_extra:
+        out["prefill"] = extra_prefill(args, torch, moe, peaks)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def dtype_of(cfg):
+    return f"{cfg.qtype} weights, bf16 activations, fp32 accumulate"
+
+
+def config_of(wl):
+    cfg = wl.cfg
+    c = {"workload": f"{wl.name}: MoE layer D={cfg.D} E={cfg.E} top-{cfg.k} F={cfg.F} "
+                     f"{cfg.qtype.upper()}" + (f" + shared F={cfg.shared_F} Q8_0" if cfg.shared_F else "")
+                     + f", T per call {list(wl.Ts)}",
+         "tokens_per_step": wl.tokens_per_step,
+         "l2": f"{len(wl.layers)} rotating replicas of the expert pool "
+               f"({wl.pool_bytes / 1e6:.0f} MB each): weights come from HBM"}
+    return c
+
+
+def roofline(wl, algo, durs, peaks, args):
+    """Roofline of the dominant kernel from the trace of the timed steps."""
+    tot = {k: sum(v) for k, v in durs.items()}
+    dom = max(tot, key=tot.get)
+    cfg = wl.cfg
+    n_calls = args.steps
+    if dom in ("gateup", "down"):
+        key = "gateup_bytes" if dom == "gateup" else "down_bytes"
+        bytes_step = sum(algo[T][key] for T in wl.Ts)
+        launches = len(durs[dom])
+        per_launch = bytes_step / wl.calls_per_step
+        avg_ms = tot[dom] / launches
+        # achieved over all launches: total algorithmic bytes / total time
+        achieved = bytes_step * n_calls / (tot[dom] / 1e3) / 1e9
+        bound, peak, unit = "hbm", peaks["hbm_gbs"], "GB/s"
+        if wl.name == "prefill":
+            flops_step = sum(algo[T]["flops"] for T in wl.Ts) * (2 / 3 if dom == "gateup" else 1 / 3)
+            achieved = flops_step * n_calls / (tot[dom] / 1e3) / 1e12
+            bound, peak, unit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
+            per_launch = flops_step
+    else:
+        achieved, bound, peak, unit, per_launch, avg_ms = None, "hbm", peaks["hbm_gbs"], "GB/s", None, tot[dom] / len(durs[dom])
+    r = {"kernel": dom, "bound": bound, "achieved": None if achieved is None else round(achieved, 2),
+         "peak": peak, "unit": unit,
+         "frac": None if achieved is None else round(achieved / peak, 4),
+         "frac_of_spec": None if achieved is None else round(
+             achieved / (HBM_SPEC_GBS if bound == "hbm" else TC_SPEC_TFLOPS), 4),
+         "algorithmic_per_launch": per_launch, "avg_launch_ms": round(avg_ms, 5),
+         "peak_source": f"{peaks['source']} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+         "traffic": ncu_traffic(dom, wl.name)}
+    return r
+
+
+def ncu_traffic(kernel, workload):
+    """dram read+write bytes per launch from the committed ncu summary, only
+    while the kernel sources still hash to what was profiled."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(p):
+        return None
+    import hashlib
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "quantized_routed_expert_top_b200", "csrc")
+    for f in sorted(os.listdir(src)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(src, f), "rb").read())
+    sha = h.hexdigest()[:16]
+    for line in open(p):
+        if line.startswith("traffic:"):
+            kv = dict(x.split("=", 1) for x in line.split()[1:])
+            if kv.get("kernel") == kernel and kv.get("workload") == workload and kv.get("src_sha") == sha:
+                return float(kv["bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------ prefill extra
+def extra_prefill(args, torch, moe, peaks):
+    wl = Workload("prefill", torch, moe)
+    algo = wl.algorithmic()
+    for _ in range(3):
+        wl.step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    trace = moe.KernelTrace(n_calls=steps)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        wl.step(trace=trace)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    durs = trace.durations()
+    flops = sum(algo[T]["flops"] for T in wl.Ts)
+    ffn_ms = sum(sum(durs.get(k, [])) for k in ("gateup", "down")) / steps
+    return {"workload": config_of(wl)["workload"], "tokens_per_s": round(8192 / (ms / 1e3), 1),
+            "ms_per_step": round(ms, 4),
+            "kernels_ms": {k: round(sum(v) / len(v), 4) for k, v in sorted(durs.items())},
+            "ffn_tflops": round(flops / (ffn_ms / 1e3) / 1e12, 2),
+            "ffn_tc_frac_of_measured": round(flops / (ffn_ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "ffn_tc_frac_of_spec": round(flops / (ffn_ms / 1e3) / 1e12 / TC_SPEC_TFLOPS, 4),
+            "flops_per_step": flops}
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_step_fn(wl_inputs, cfg, Ts, frac=1.0):
+    import oracle
+    oracle.build()
+
+    def step():
+        n = 0
+        for T in Ts:
+            L = wl_inputs[T]
+            if L.logits is not None:
+                ids, g = oracle.select(L.logits, cfg.k, cfg.renorm)
+            else:
+                _, ids, g = oracle.route(L.x, L.w_router, L.bias, cfg.k, cfg.renorm)
+            m = max(1, int(round(T * frac)))
+            toks = np.arange(m, dtype=np.int32)
+            oracle.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F, shared=L.shared,
+                         tokens=toks)
+            n += m
+        return n
+    return step
+
+
+def cpu_baseline(wl, args):
+    """The oracle as it stands, on the host cores, on a bounded sample."""
+    cores = os.cpu_count() or 1
+    frac = 1.0 if wl.name == "decode" else 32.0 / max(wl.Ts)
+    step = oracle_step_fn(wl.inputs, wl.cfg, wl.Ts, frac)
+    t = time.perf_counter()
+    n = step()
+    dt = time.perf_counter() - t
+    reps = 1
+    while time.perf_counter() - t < 10.0 and reps < 20:
+        n += step()
+        reps += 1
+    dt = time.perf_counter() - t
+    return {"value": round(n / dt, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} oracle step(s) of {wl.name} on {n // reps} tokens each "
+                      f"(route + layer, fp64, OpenMP over tokens), {dt:.1f} s wall"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle, timed on the host cores."""
+    if rank != 0:
+        return
+    name = args.workload
+    cfg = S.CONFIGS[name]
+    Ts = {"decode": (1, 4, 16), "prefill": (8192,), "wide": (1, 2048)}[name]
+    base = S.make_layer(cfg, T=max(Ts))
+    inputs = {max(Ts): base}
+    for T in Ts:
+        if T not in inputs:
+            inputs[T] = S.make_layer(cfg, T=T, experts=False)
+            inputs[T].gate, inputs[T].up, inputs[T].down = base.gate, base.up, base.down
+            inputs[T].shared = base.shared
+    # size the per-step sample so that warmup + steps end within ~3 minutes
+    step = oracle_step_fn(inputs, cfg, Ts, 1.0 if name == "decode" else 16.0 / max(Ts))
+    t = time.perf_counter()
+    n1 = step()
+    t1 = time.perf_counter() - t
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    frac = 1.0
+    if t1 > budget:
+        frac = max(budget / t1, 1.0 / n1)
+    total = sum(Ts) if name == "decode" else 16 * len(Ts)
+    step = oracle_step_fn(inputs, cfg, Ts, frac * (1.0 if name == "decode" else 16.0 / max(Ts)))
+    for _ in range(max(0, args.warmup - 1)):
+        step()
+    t = time.perf_counter()
+    n = 0
+    for _ in range(args.steps):
+        n += step()
+    dt = time.perf_counter() - t
+    value = n / dt
+    cores = os.cpu_count() or 1
+    out = {"metric": "MoE-layer tokens/s", "value": round(value, 4), "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+           "data": "synthetic (seeded)", "impl": "reference",
+           "config": {"workload": f"{name}: same layer as the default arm; each step a "
+                                  f"sample of {n // args.steps} of its {total} tokens"},
+           "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cores,
+                            "kind": "oracle",
+                            "sample": f"{n // args.steps} tokens per step, {args.steps} steps"},
+           "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["decode", "prefill", "wide"], default="decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+// abi.cu -- the extern "C" entry points of libmoe declared in include/moe.h:
+// argument checks (every dispatch has an erroring default), workspace
+// carving and kernel dispatch.  No call allocates device memory.
+#include "moe_internal.cuh"
+#include "moe_paths.cuh"
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+namespace moe {
+
+static thread_local std::string g_err;
+
+void set_error(const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+}
+
+moe_status cuda_status(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return MOE_OK;
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+}
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+static bool qtype_ok(int q) { return q == MOE_Q4_0 || q == MOE_Q8_0; }
+static bool act_dtype_ok(int d) { return d == MOE_F32 || d == MOE_BF16; }
+
+static moe_status check_shapes(const char *fn, int T, int D, int F, int E, int k) {
+    if (T < 0 || D <= 0 || F <= 0 || E <= 0 || k <= 0) {
+        set_error("%s: non-positive size (T=%d D=%d F=%d E=%d k=%d)", fn, T, D, F, E, k);
+        return MOE_ERR_SHAPE;
+    }
+    if (D % QK || F % QK) {
+        set_error("%s: D=%d and F=%d must be multiples of 32 (blocks run along the "
+                  "reduction dimension)", fn, D, F);
+        return MOE_ERR_SHAPE;
+    }
+    if (k > E || E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) {
+        set_error("%s: need 1 <= k <= E <= %d and k <= %d (k=%d E=%d)", fn, MOE_MAX_EXPERTS,
+                  MOE_MAX_TOPK, k, E);
+        return MOE_ERR_SHAPE;
+    }
+    return MOE_OK;
+}
+
+static moe_status check_pool(const char *fn, const moe_pool *p, int E) {
+    if (!p) { set_error("%s: pool is NULL", fn); return MOE_ERR_INVALID_ARG; }
+    if (!qtype_ok(p->qtype)) {
+        set_error("%s: unsupported quant type %d (Q4_0=2, Q8_0=8)", fn, (int)p->qtype);
+        return MOE_ERR_UNSUPPORTED_QTYPE;
+    }
+    if (!p->gate || !p->up || !p->down || p->n_slots <= 0) {
+        set_error("%s: pool has a NULL matrix or no slots", fn);
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (!p->slot_of_expert && p->n_slots < E) {
+        set_error("%s: pool without a slot map holds %d slots for %d experts", fn, (int)p->n_slots, E);
+        return MOE_ERR_SHAPE;
+    }
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_err.c_str(); }
+
+const char *moe_version(void) { return "libmoe 0.1 (sm_100a)"; }
+
+int moe_block_bytes(int32_t qtype) {
+    switch (qtype) {
+    case MOE_Q4_0: return MOE_Q4_0_BLOCK_BYTES;
+    case MOE_Q8_0: return MOE_Q8_0_BLOCK_BYTES;
+    default: return 0;
+    }
+}
+
+// ----------------------------------------------------------------- route
+size_t moe_route_workspace_size(int T, int D, int E, int k) {
+    return route_ws_bytes(T < 0 ? 0 : T, D, E, k);
+}
+
+moe_status moe_route(const void *x, int32_t x_dtype, const float *w_router, const float *bias,
+                     int T, int D, int E, int k, int renorm, int32_t *ids, float *gates,
+                     float *logits, void *workspace, size_t ws_bytes, moe_stream stream) {
+    g_err.clear();
+    if (w_router == nullptr) D = QK;   // logits given: D unused
+    moe_status st = check_shapes("moe_route", T, D, QK, E, k);
+    if (st != MOE_OK) return st;
+    if (!act_dtype_ok(x_dtype) || (w_router == nullptr && x_dtype != MOE_F32)) {
+        set_error("moe_route: x dtype %d not allowed (F32/BF16 activations, F32 logits)", x_dtype);
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (renorm != 0 && renorm != 1) { set_error("moe_route: renorm must be 0 or 1"); return MOE_ERR_INVALID_ARG; }
+    if (T == 0) return MOE_OK;
+    if (!x || !ids || !gates) { set_error("moe_route: NULL x, ids or gates"); return MOE_ERR_INVALID_ARG; }
+    if (!workspace || ws_bytes < route_ws_bytes(T, D, E, k)) {
+        set_error("moe_route: workspace needs %zu bytes, got %zu", route_ws_bytes(T, D, E, k), ws_bytes);
+        return MOE_ERR_WORKSPACE;
+    }
+    return launch_route(x, x_dtype, w_router, bias, T, D, E, k, renorm, ids, gates, logits,
+                        workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+// --------------------------------------------------------------- permute
+moe_status moe_permute(const int32_t *ids, int T, int k, int E, int32_t *counts, int32_t *offsets,
+                       int32_t *perm, int32_t *inv, moe_stream stream) {
+    g_err.clear();
+    moe_status st = check_shapes("moe_permute", T, QK, QK, E, k);
+    if (st != MOE_OK) return st;
+    if (!counts || !offsets) { set_error("moe_permute: NULL counts or offsets"); return MOE_ERR_INVALID_ARG; }
+    if (T > 0 && (!ids || !perm || !inv)) { set_error("moe_permute: NULL ids, perm or inv"); return MOE_ERR_INVALID_ARG; }
+    if ((long long)T * k > 0x7fffffffLL) { set_error("moe_permute: T*k overflows int32"); return MOE_ERR_SHAPE; }
+    return launch_permute(ids, T, k, E, counts, offsets, perm, inv, (cudaStream_t)stream);
+}
+
+// ------------------------------------------------------------ expert FFN
+size_t moe_expert_ffn_workspace_size(int T, int k, int D, int F) {
+    (void)D;
+    Carver c(nullptr, 0);
+    c.take<float>((size_t)(T < 0 ? 0 : T) * k * F);
+    return c.off;
+}
+
+moe_status moe_expert_ffn(const void *x, int32_t x_dtype, int T, int D, int F, int E, int k,
+                          const int32_t *perm, const int32_t *offsets, const moe_pool *pool,
+                          const uint8_t *expert_mask, float *out_rows, void *workspace,
+                          size_t ws_bytes, moe_stream stream) {
+    g_err.clear();
+    moe_status st = check_shapes("moe_expert_ffn", T, D, F, E, k);
+    if (st != MOE_OK) return st;
+    if ((st = check_pool("moe_expert_ffn", pool, E)) != MOE_OK) return st;
+    if (!act_dtype_ok(x_dtype)) { set_error("moe_expert_ffn: x dtype %d not F32/BF16", x_dtype); return MOE_ERR_INVALID_ARG; }
+    if (T == 0) return MOE_OK;
+    if (!x || !perm || !offsets || !out_rows) { set_error("moe_expert_ffn: NULL x, perm, offsets or out_rows"); return MOE_ERR_INVALID_ARG; }
+    size_t need = moe_expert_ffn_workspace_size(T, k, D, F);
+    if (!workspace || ws_bytes < need) {
+        set_error("moe_expert_ffn: workspace needs %zu bytes, got %zu", need, ws_bytes);
+        return MOE_ERR_WORKSPACE;
+    }
+    Carver c(workspace, ws_bytes);
+    float *H = c.take<float>((size_t)T * k * F);
+    return launch_ffn_generic(x, x_dtype, T, D, F, E, k, perm, offsets, *pool, expert_mask, H,
+                              out_rows, (cudaStream_t)stream);
+}
+
+// --------------------------------------------------------------- combine
+moe_status moe_combine(const float *rows, const int32_t *inv, const float *gates, int T, int k, int D,
+                       const float *shared_rows, void *y, int32_t y_dtype, moe_stream stream) {
+    g_err.clear();
+    if (T < 0 || k <= 0 || D <= 0 || k > MOE_MAX_TOPK) { set_error("moe_combine: bad sizes"); return MOE_ERR_SHAPE; }
+    if (y_dtype != MOE_F32 && y_dtype != MOE_BF16 && y_dtype != MOE_F16) {
+        set_error("moe_combine: unsupported output dtype %d", y_dtype);
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (T == 0) return MOE_OK;
+    if (!rows || !inv || !gates || !y) { set_error("moe_combine: NULL argument"); return MOE_ERR_INVALID_ARG; }
+    return launch_combine(rows, inv, gates, T, k, D, shared_rows, y, y_dtype, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------- fused forward
+size_t moe_layer_workspace_size(const moe_layer_args *a) {
+    if (!a) return 0;
+    return layer_ws_bytes(*a);
+}
+
+moe_status moe_layer_forward(const moe_layer_args *a, void *workspace, size_t ws_bytes,
+                             moe_stream stream) {
+    g_err.clear();
+    if (!a) { set_error("moe_layer_forward: args is NULL"); return MOE_ERR_INVALID_ARG; }
+    const int D_eff = a->D;
+    moe_status st = check_shapes("moe_layer_forward", a->T, D_eff, a->F, a->E, a->k);
+    if (st != MOE_OK) return st;
+    if ((st = check_pool("moe_layer_forward", a->pool, a->E)) != MOE_OK) return st;
+    if (a->shared) {
+        if ((st = check_pool("moe_layer_forward (shared)", a->shared, 1)) != MOE_OK) return st;
+        if (a->shared_F <= 0 || a->shared_F % QK) {
+            set_error("moe_layer_forward: shared_F=%d must be a positive multiple of 32", a->shared_F);
+            return MOE_ERR_SHAPE;
+        }
+    }
+    if (!act_dtype_ok(a->x_dtype)) { set_error("moe_layer_forward: x dtype %d not F32/BF16", a->x_dtype); return MOE_ERR_INVALID_ARG; }
+    if (a->y_dtype != MOE_F32 && a->y_dtype != MOE_BF16) {
+        set_error("moe_layer_forward: y dtype %d not F32/BF16", a->y_dtype);
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (a->renorm != 0 && a->renorm != 1) { set_error("moe_layer_forward: renorm must be 0 or 1"); return MOE_ERR_INVALID_ARG; }
+    if (a->T == 0) return MOE_OK;
+    if (!a->x || !a->y || (!a->w_router && !a->logits_in)) {
+        set_error("moe_layer_forward: NULL x, y, or both w_router and logits_in");
+        return MOE_ERR_INVALID_ARG;
+    }
+    size_t need = layer_ws_bytes(*a);
+    if (!workspace || ws_bytes < need) {
+        set_error("moe_layer_forward: workspace needs %zu bytes, got %zu", need, ws_bytes);
+        return MOE_ERR_WORKSPACE;
+    }
+    return layer_forward(*a, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+}  // extern "C"

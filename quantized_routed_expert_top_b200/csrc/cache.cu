@@ -1,0 +1,296 @@
+// cache.cu -- per-layer HBM expert cache fed from a pinned host pool.
+//
+// The full expert set stays in pinned host memory; each layer owns n_slots
+// device slots used as an LRU cache (FreeToken fork README, "About": global
+// LRU expert caching; wiki explainer: LRU caching follows token-level
+// routing locality; kongchang article: VRAM as a cache, system RAM as the
+// source of truth).  Replacement rules:
+//  - each request is one step; every requested expert is stamped with it;
+//  - ids are served in the order given; resident ids are hits;
+//  - a miss takes the empty slot of lowest index, else evicts the resident
+//    expert with the oldest stamp among those NOT requested in this step
+//    (lower expert id on equal stamps).
+// Missed experts are copied host->device with cudaMemcpyAsync on the copy
+// stream, which first waits for an event recorded on the compute stream (a
+// victim slot may still be read by earlier kernels).  The copy-done event of
+// the layer lets the compute stream wait (moe_cache_sync) only when the
+// missing experts are needed, so the FFN of resident experts overlaps the
+// copies.  The layer's device slot map is refreshed from a pinned staging
+// buffer (two per layer, alternating; each reuse waits, with a time limit,
+// for the copy that last read it).
+#include "moe_internal.cuh"
+
+#include <chrono>
+#include <new>
+#include <thread>
+#include <vector>
+
+struct moe_cache {
+    moe_cache_desc d;
+    struct Layer {
+        std::vector<int32_t> slot_expert;   // [n_slots] -1 empty
+        std::vector<int32_t> expert_slot;   // [E] -1 not resident
+        std::vector<int64_t> stamp;         // [E]
+        int64_t step = 0;
+        bool pending = false;
+        cudaEvent_t copied = nullptr;
+        cudaEvent_t map_done[2] = {nullptr, nullptr};
+        int map_buf = 0;
+    };
+    std::vector<Layer> layers;
+    int32_t *pinned_maps = nullptr;       // [n_layers][2][E]
+    cudaEvent_t compute_ready = nullptr;
+    int64_t hits = 0, misses = 0, bytes = 0;
+    int fail_copy_at = -1;                // test hook: fail the n-th copy
+    int copies_issued = 0;
+};
+
+namespace moe {
+static moe_status wait_event_bounded(cudaEvent_t ev, double seconds) {
+    auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        cudaError_t e = cudaEventQuery(ev);
+        if (e == cudaSuccess) return MOE_OK;
+        if (e != cudaErrorNotReady) return cuda_status(e, "cudaEventQuery");
+        double dt = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+        if (dt > seconds) {
+            set_error("expert cache: wait for a slot-map copy exceeded %.1f s", seconds);
+            return MOE_ERR_TIMEOUT;
+        }
+        std::this_thread::yield();
+    }
+}
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out) {
+    if (!desc || !out) { set_error("moe_cache_init: NULL argument"); return MOE_ERR_INVALID_ARG; }
+    *out = nullptr;
+    const moe_cache_desc &d = *desc;
+    if (d.n_layers <= 0 || d.E <= 0 || d.E > MOE_MAX_EXPERTS || d.n_slots <= 0 || d.n_slots > d.E) {
+        set_error("moe_cache_init: need n_layers > 0, 0 < n_slots <= E <= %d", MOE_MAX_EXPERTS);
+        return MOE_ERR_SHAPE;
+    }
+    if (d.qtype != MOE_Q4_0 && d.qtype != MOE_Q8_0) {
+        set_error("moe_cache_init: unsupported quant type %d", (int)d.qtype);
+        return MOE_ERR_UNSUPPORTED_QTYPE;
+    }
+    if (!d.host_gate || !d.host_up || !d.host_down || !d.dev_gate || !d.dev_up || !d.dev_down ||
+        !d.dev_slot_map || !d.copy_stream || !d.bytes_gate || !d.bytes_up || !d.bytes_down) {
+        set_error("moe_cache_init: NULL pool pointer, copy stream or zero expert size");
+        return MOE_ERR_INVALID_ARG;
+    }
+    for (int l = 0; l < d.n_layers; l++)
+        if (!d.host_gate[l] || !d.host_up[l] || !d.host_down[l]) {
+            set_error("moe_cache_init: NULL host pool of layer %d", l);
+            return MOE_ERR_INVALID_ARG;
+        }
+    moe_cache *c = new (std::nothrow) moe_cache();
+    if (!c) { set_error("moe_cache_init: out of host memory"); return MOE_ERR_INVALID_ARG; }
+    c->d = d;
+    c->layers.resize(d.n_layers);
+    moe_status st = MOE_OK;
+    cudaError_t e = cudaHostAlloc((void **)&c->pinned_maps, sizeof(int32_t) * d.n_layers * 2 * d.E,
+                                  cudaHostAllocDefault);
+    if (e != cudaSuccess) st = cuda_status(e, "moe_cache_init: pinned slot maps");
+    if (st == MOE_OK) st = cuda_status(cudaEventCreateWithFlags(&c->compute_ready, cudaEventDisableTiming), "cudaEventCreate");
+    for (int l = 0; l < d.n_layers && st == MOE_OK; l++) {
+        auto &L = c->layers[l];
+        L.slot_expert.assign(d.n_slots, -1);
+        L.expert_slot.assign(d.E, -1);
+        L.stamp.assign(d.E, 0);
+        st = cuda_status(cudaEventCreateWithFlags(&L.copied, cudaEventDisableTiming), "cudaEventCreate");
+        for (int b = 0; b < 2 && st == MOE_OK; b++)
+            st = cuda_status(cudaEventCreateWithFlags(&L.map_done[b], cudaEventDisableTiming), "cudaEventCreate");
+        for (int i = 0; i < 2 * d.E; i++) c->pinned_maps[(size_t)l * 2 * d.E + i] = -1;
+    }
+    // all slot maps start empty (-1)
+    if (st == MOE_OK)
+        st = cuda_status(cudaMemcpy(d.dev_slot_map, c->pinned_maps, sizeof(int32_t) * d.E,
+                                    cudaMemcpyHostToDevice), "moe_cache_init: slot map");
+    for (int l = 1; l < d.n_layers && st == MOE_OK; l++)
+        st = cuda_status(cudaMemcpy(d.dev_slot_map + (size_t)l * d.E, c->pinned_maps,
+                                    sizeof(int32_t) * d.E, cudaMemcpyHostToDevice),
+                         "moe_cache_init: slot map");
+    if (st != MOE_OK) { moe_cache_destroy(c); return st; }
+    *out = c;
+    return MOE_OK;
+}
+
+void moe_cache_destroy(moe_cache *c) {
+    if (!c) return;
+    for (auto &L : c->layers) {
+        if (L.copied) cudaEventDestroy(L.copied);
+        for (auto &ev : L.map_done) if (ev) cudaEventDestroy(ev);
+    }
+    if (c->compute_ready) cudaEventDestroy(c->compute_ready);
+    if (c->pinned_maps) cudaFreeHost(c->pinned_maps);
+    delete c;
+}
+
+// Test hook (not in the public header): make the n-th expert copy (0-based,
+// counted over the cache's lifetime) fail as if cudaMemcpyAsync had failed.
+void moe_cache_debug_fail_copy(moe_cache *c, int nth) {
+    if (c) { c->fail_copy_at = nth; c->copies_issued = 0; }
+}
+
+moe_status moe_cache_request(moe_cache *c, int layer, const int32_t *ids, int n, int32_t *slots,
+                             int32_t *miss, int32_t *evicted, int *n_miss, moe_stream compute) {
+    if (!c || (!ids && n > 0)) { set_error("moe_cache_request: NULL argument"); return MOE_ERR_INVALID_ARG; }
+    const moe_cache_desc &d = c->d;
+    if (layer < 0 || layer >= d.n_layers) { set_error("moe_cache_request: layer %d out of range", layer); return MOE_ERR_INVALID_ARG; }
+    if (n < 0) { set_error("moe_cache_request: n < 0"); return MOE_ERR_INVALID_ARG; }
+    if (n > d.n_slots) {
+        set_error("moe_cache_request: %d experts requested but the layer has %d slots", n, d.n_slots);
+        return MOE_ERR_CAPACITY;
+    }
+    auto &L = c->layers[layer];
+    std::vector<char> wanted(d.E, 0);
+    for (int i = 0; i < n; i++) {
+        if (ids[i] < 0 || ids[i] >= d.E) { set_error("moe_cache_request: expert id %d out of range", ids[i]); return MOE_ERR_INVALID_ARG; }
+        if (wanted[ids[i]]) { set_error("moe_cache_request: expert id %d repeated", ids[i]); return MOE_ERR_INVALID_ARG; }
+        wanted[ids[i]] = 1;
+    }
+    cudaStream_t cs = (cudaStream_t)compute;
+    cudaStream_t xs = (cudaStream_t)d.copy_stream;
+    // staging buffer for this request's slot map: wait until its last copy ran
+    const int buf = L.map_buf;
+    moe_status st = wait_event_bounded(L.map_done[buf], 10.0);
+    if (st != MOE_OK) return st;
+
+    // LRU decisions (committed below; on a copy failure the touched slots are
+    // invalidated so the resident set stays truthful)
+    const int64_t step = L.step + 1;
+    std::vector<int> miss_idx;
+    std::vector<int32_t> out_slot(n), out_ev(n, -1);
+    std::vector<int32_t> se = L.slot_expert, es = L.expert_slot;
+    std::vector<int64_t> stamp = L.stamp;
+    for (int i = 0; i < n; i++) {
+        const int e = ids[i];
+        if (es[e] >= 0) {
+            out_slot[i] = es[e];
+        } else {
+            int s = -1;
+            for (int q = 0; q < d.n_slots; q++) if (se[q] < 0) { s = q; break; }
+            if (s < 0) {
+                int victim = -1;
+                for (int v = 0; v < d.E; v++) {
+                    if (es[v] < 0 || wanted[v]) continue;
+                    if (victim < 0 || stamp[v] < stamp[victim]) victim = v;
+                }
+                s = es[victim];
+                es[victim] = -1;
+                out_ev[i] = victim;
+            }
+            se[s] = e;
+            es[e] = s;
+            out_slot[i] = s;
+            miss_idx.push_back(i);
+        }
+        stamp[e] = step;
+    }
+
+    // copies of the misses on the copy stream, after the compute stream
+    moe_status cst = MOE_OK;
+    if (!miss_idx.empty()) {
+        cst = cuda_status(cudaEventRecord(c->compute_ready, cs), "cudaEventRecord");
+        if (cst == MOE_OK) cst = cuda_status(cudaStreamWaitEvent(xs, c->compute_ready, 0), "cudaStreamWaitEvent");
+        for (size_t m = 0; m < miss_idx.size() && cst == MOE_OK; m++) {
+            const int i = miss_idx[m];
+            const int e = ids[i];
+            const size_t slot = (size_t)layer * d.n_slots + out_slot[i];
+            struct { void *dst; const void *src; size_t n; } cp[3] = {
+                {(char *)d.dev_gate + slot * d.bytes_gate, (const char *)d.host_gate[layer] + (size_t)e * d.bytes_gate, d.bytes_gate},
+                {(char *)d.dev_up + slot * d.bytes_up, (const char *)d.host_up[layer] + (size_t)e * d.bytes_up, d.bytes_up},
+                {(char *)d.dev_down + slot * d.bytes_down, (const char *)d.host_down[layer] + (size_t)e * d.bytes_down, d.bytes_down},
+            };
+            for (auto &q : cp) {
+                if (c->fail_copy_at >= 0 && c->copies_issued == c->fail_copy_at) {
+                    c->copies_issued++;
+                    set_error("moe_cache_request: injected copy failure");
+                    cst = MOE_ERR_CUDA;
+                    break;
+                }
+                c->copies_issued++;
+                cst = cuda_status(cudaMemcpyAsync(q.dst, q.src, q.n, cudaMemcpyHostToDevice, xs),
+                                  "moe_cache_request: cudaMemcpyAsync");
+                if (cst != MOE_OK) break;
+            }
+        }
+        if (cst == MOE_OK) cst = cuda_status(cudaEventRecord(L.copied, xs), "cudaEventRecord");
+    }
+    if (cst != MOE_OK) {
+        // invalidate every slot this request wrote into: the resident set is
+        // the old one minus the victims, and no missed expert is resident
+        for (int i : miss_idx) {
+            const int s = out_slot[i];
+            se[s] = -1;
+            es[ids[i]] = -1;
+        }
+        // keep the old recency of experts that were not served
+        stamp = L.stamp;
+    }
+    L.slot_expert.swap(se);
+    L.expert_slot.swap(es);
+    L.stamp.swap(stamp);
+    L.step = step;
+    L.pending = L.pending || (!miss_idx.empty() && cst == MOE_OK);
+
+    // device slot map of the layer
+    int32_t *hm = c->pinned_maps + ((size_t)layer * 2 + buf) * d.E;
+    for (int e = 0; e < d.E; e++) hm[e] = L.expert_slot[e];
+    moe_status mst = cuda_status(cudaMemcpyAsync(d.dev_slot_map + (size_t)layer * d.E, hm,
+                                                 sizeof(int32_t) * d.E, cudaMemcpyHostToDevice, cs),
+                                 "moe_cache_request: slot map copy");
+    if (mst == MOE_OK) mst = cuda_status(cudaEventRecord(L.map_done[buf], cs), "cudaEventRecord");
+    L.map_buf ^= 1;
+    if (cst != MOE_OK) return cst;
+    if (mst != MOE_OK) return mst;
+
+    const int nm = (int)miss_idx.size();
+    c->hits += n - nm;
+    c->misses += nm;
+    c->bytes += (int64_t)nm * (int64_t)(d.bytes_gate + d.bytes_up + d.bytes_down);
+    if (n_miss) *n_miss = nm;
+    for (int i = 0; i < n; i++) {
+        if (slots) slots[i] = out_slot[i];
+        if (evicted) evicted[i] = out_ev[i];
+        if (miss) miss[i] = 0;
+    }
+    if (miss) for (int i : miss_idx) miss[i] = 1;
+    return MOE_OK;
+}
+
+moe_status moe_cache_sync(moe_cache *c, int layer, moe_stream compute) {
+    if (!c || layer < 0 || layer >= c->d.n_layers) { set_error("moe_cache_sync: bad cache or layer"); return MOE_ERR_INVALID_ARG; }
+    auto &L = c->layers[layer];
+    if (!L.pending) return MOE_OK;
+    L.pending = false;
+    return cuda_status(cudaStreamWaitEvent((cudaStream_t)compute, L.copied, 0), "cudaStreamWaitEvent");
+}
+
+moe_status moe_cache_layer_pool(moe_cache *c, int layer, moe_pool *out) {
+    if (!c || !out || layer < 0 || layer >= c->d.n_layers) { set_error("moe_cache_layer_pool: bad argument"); return MOE_ERR_INVALID_ARG; }
+    const moe_cache_desc &d = c->d;
+    const size_t base = (size_t)layer * d.n_slots;
+    out->qtype = d.qtype;
+    out->n_slots = d.n_slots;
+    out->gate = (const char *)d.dev_gate + base * d.bytes_gate;
+    out->up = (const char *)d.dev_up + base * d.bytes_up;
+    out->down = (const char *)d.dev_down + base * d.bytes_down;
+    out->slot_of_expert = d.dev_slot_map + (size_t)layer * d.E;
+    return MOE_OK;
+}
+
+moe_status moe_cache_stats(moe_cache *c, int64_t *hits, int64_t *misses, int64_t *bytes_copied) {
+    if (!c) { set_error("moe_cache_stats: NULL cache"); return MOE_ERR_INVALID_ARG; }
+    if (hits) *hits = c->hits;
+    if (misses) *misses = c->misses;
+    if (bytes_copied) *bytes_copied = c->bytes;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,281 @@
+// route.cu -- router logits, softmax, top-k and renormalised gates.
+//
+// L = x . W_r (+ b) in fp32; the top-k experts per token are taken in
+// descending logit order with ties to the lower expert id; the gates are the
+// softmax probabilities of the selected experts renormalised over the
+// selection (equivalently a softmax over the selected logits).
+//
+// Two logit paths:
+//  * small T (decode): split-K GEMV.  W_r is only D*E*4 bytes (1 MiB at
+//    D=2048, E=128) but at T=1 one CTA cannot stream it fast, so the D rows
+//    are split over many CTAs; each writes fp32 partial sums to the
+//    workspace, and the CTA that finishes last (atomic ticket) adds the
+//    partials in split order (deterministic), adds the bias and runs the
+//    warp-per-token selection.  One launch.
+//  * large T (prefill): a register-tiled SIMT GEMM writes the logits, then a
+//    warp-per-token selection kernel.
+// Logits stay fp32 end to end (no TF32): the tie rule compares logits at a
+// 1e-5 resolution.
+#include "moe_internal.cuh"
+
+#include <algorithm>
+#include <cfloat>
+#include <climits>
+
+namespace moe {
+
+constexpr int kSplitMaxT = 16;      // tokens handled by the split-K path
+constexpr int kSplitRows = 32;      // D rows per split CTA
+
+// --------------------------------------------------------------- selection
+// One warp selects the top-k of a logit row L[0..E) (any memory space) and
+// writes ids/gates for that token.  E <= 1024 (32 values per lane), k <= 32.
+__device__ void warp_select(const float *L, int E, int k, int renorm,
+                            int32_t *ids_out, float *gates_out) {
+    const int lane = threadIdx.x & 31;
+    const int per_lane = (E + 31) >> 5;
+    unsigned taken = 0u;
+    float my_v = -INFINITY;
+    int my_i = INT_MAX;
+    for (int j = 0; j < k; j++) {
+        float bv = -INFINITY;
+        int bi = INT_MAX;
+        for (int i = 0; i < per_lane; i++) {
+            int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u)) {
+                float v = L[e];
+                if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (lane == j) { my_v = bv; my_i = bi; }
+    }
+    // gates: lane j < k holds selection j; the first selection is the max
+    const float m = __shfl_sync(0xffffffffu, my_v, 0);
+    float ex = (lane < k) ? expf(my_v - m) : 0.0f;
+    float denom;
+    if (renorm) {
+        denom = warp_sum(ex);
+    } else {
+        float z = 0.0f;
+        for (int i = 0; i < per_lane; i++) {
+            int e = lane + 32 * i;
+            if (e < E) z += expf(L[e] - m);
+        }
+        denom = warp_sum(z);
+    }
+    if (lane < k) {
+        ids_out[lane] = my_i;
+        gates_out[lane] = ex / denom;
+    }
+}
+
+// ------------------------------------------------- small T: split-K + select
+template <typename XT>
+__global__ void __launch_bounds__(1024)
+route_splitk_kernel(const XT *__restrict__ x, const float *__restrict__ W,
+                    const float *__restrict__ bias, int T, int D, int E, int k,
+                    int renorm, int nsplit, float *__restrict__ partial,
+                    unsigned *__restrict__ ticket, int32_t *__restrict__ ids,
+                    float *__restrict__ gates, float *__restrict__ logits_out) {
+    extern __shared__ float smem[];
+    float *xs = smem;                         // [T][kSplitRows]
+    __shared__ int s_last;
+    const int s = blockIdx.x;
+    const int i0 = s * kSplitRows;
+    const int rows = min(kSplitRows, D - i0);
+    for (int idx = threadIdx.x; idx < T * kSplitRows; idx += blockDim.x) {
+        int t = idx / kSplitRows, r = idx % kSplitRows;
+        xs[idx] = (r < rows) ? load_act(x, (size_t)t * D + i0 + r) : 0.0f;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float acc[kSplitMaxT];
+#pragma unroll
+        for (int t = 0; t < kSplitMaxT; t++) acc[t] = 0.0f;
+        for (int r = 0; r < rows; r++) {
+            float w = __ldg(W + (size_t)(i0 + r) * E + e);
+#pragma unroll
+            for (int t = 0; t < kSplitMaxT; t++)
+                if (t < T) acc[t] = fmaf(xs[t * kSplitRows + r], w, acc[t]);
+        }
+#pragma unroll
+        for (int t = 0; t < kSplitMaxT; t++)
+            if (t < T) partial[((size_t)s * T + t) * E + e] = acc[t];
+    }
+    // last CTA to finish reduces the partials and selects
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(ticket, 1u) == (unsigned)(nsplit - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    float *Ls = smem;                          // reuse: [T][E]
+    for (int idx = threadIdx.x; idx < T * E; idx += blockDim.x) {
+        int t = idx / E, e = idx % E;
+        float v = 0.0f;
+        for (int q = 0; q < nsplit; q++) v += __ldcg(partial + ((size_t)q * T + t) * E + e);
+        if (bias) v += __ldg(bias + e);
+        Ls[idx] = v;
+        if (logits_out) logits_out[idx] = v;
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int t = warp; t < T; t += nwarps)
+        warp_select(Ls + (size_t)t * E, E, k, renorm, ids + (size_t)t * k, gates + (size_t)t * k);
+    if (threadIdx.x == 0) *ticket = 0u;        // ready for the next call
+}
+
+// ------------------------------------------------------ large T: tiled GEMM
+constexpr int kTM = 64, kTN = 64, kTK = 16;  // 256 threads, 4x4 outputs each
+
+template <typename XT>
+__global__ void __launch_bounds__(256)
+route_logits_tiled_kernel(const XT *__restrict__ x, const float *__restrict__ W,
+                          const float *__restrict__ bias, int T, int D, int E,
+                          float *__restrict__ logits) {
+    __shared__ float As[kTK][kTM + 4];
+    __shared__ float Bs[kTK][kTN + 4];
+    const int t0 = blockIdx.x * kTM, e0 = blockIdx.y * kTN;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < D; k0 += kTK) {
+        for (int idx = threadIdx.x; idx < kTM * kTK; idx += 256) {
+            int m = idx / kTK, kk = idx % kTK;
+            int t = t0 + m;
+            As[kk][m] = (t < T) ? load_act(x, (size_t)t * D + k0 + kk) : 0.0f;
+        }
+        for (int idx = threadIdx.x; idx < kTK * kTN; idx += 256) {
+            int kk = idx / kTN, n = idx % kTN;
+            int e = e0 + n;
+            Bs[kk][n] = (e < E) ? __ldg(W + (size_t)(k0 + kk) * E + e) : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < kTK; kk++) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; j++) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+#pragma unroll
+                for (int j = 0; j < 4; j++) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        int t = t0 + ty * 4 + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            int e = e0 + tx * 4 + j;
+            if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (bias ? __ldg(bias + e) : 0.0f);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256)
+route_select_kernel(const float *__restrict__ logits, const float *__restrict__ bias_if_raw,
+                    int T, int E, int k, int renorm, int32_t *__restrict__ ids,
+                    float *__restrict__ gates, float *__restrict__ logits_copy) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (warp >= T) return;
+    const float *L = logits + (size_t)warp * E;
+    if (bias_if_raw || logits_copy) {
+        // routing from given logits with a bias or a requested copy: stage
+        // the biased row in the copy buffer and select from there
+        const int lane = threadIdx.x & 31;
+        float *C = logits_copy + (size_t)warp * E;
+        for (int e = lane; e < E; e += 32) C[e] = L[e] + (bias_if_raw ? __ldg(bias_if_raw + e) : 0.0f);
+        __syncwarp();
+        L = C;
+    }
+    warp_select(L, E, k, renorm, ids + (size_t)warp * k, gates + (size_t)warp * k);
+}
+
+// ------------------------------------------------------------------- host
+static size_t splitk_partial_bytes(int T, int D, int E) {
+    int nsplit = (D + kSplitRows - 1) / kSplitRows;
+    return (size_t)nsplit * T * E * sizeof(float);
+}
+
+size_t route_ws_bytes(int T, int D, int E, int k) {
+    (void)k;
+    Carver c(nullptr, 0);
+    c.take<unsigned>(64);
+    if (T <= kSplitMaxT) c.take<char>(splitk_partial_bytes(T, D, E));
+    else c.take<float>((size_t)T * E);   // logits scratch when none requested
+    return c.off;
+}
+
+moe_status launch_route(const void *x, int x_dtype, const float *w_router,
+                        const float *bias, int T, int D, int E, int k, int renorm,
+                        int32_t *ids, float *gates, float *logits, void *ws,
+                        size_t ws_bytes, cudaStream_t s, Tracer *tr) {
+    Carver c(ws, ws_bytes);
+    unsigned *ticket = c.take<unsigned>(64);
+    if (w_router == nullptr) {
+        // x holds the logits [T, E] fp32
+        float *copy = logits;
+        if (bias && !copy) {
+            copy = c.take<float>((size_t)T * E);
+            if (!c.fits()) { set_error("moe_route: workspace too small"); return MOE_ERR_WORKSPACE; }
+        }
+        int blocks = (T * 32 + 255) / 256;
+        mark(tr, MOE_KERNEL_ROUTE_SELECT);
+        route_select_kernel<<<blocks, 256, 0, s>>>((const float *)x, bias, T, E, k, renorm,
+                                                   ids, gates, copy);
+        return cuda_status(cudaGetLastError(), "route_select_kernel");
+    }
+    if (T <= kSplitMaxT) {
+        float *partial = (float *)c.take<char>(splitk_partial_bytes(T, D, E));
+        if (!c.fits()) { set_error("moe_route: workspace too small"); return MOE_ERR_WORKSPACE; }
+        int nsplit = (D + kSplitRows - 1) / kSplitRows;
+        int threads = (int)round_up(E, 32);
+        if (threads < 128) threads = 128;
+        size_t sm = (size_t)std::max(T * kSplitRows, T * E) * sizeof(float);
+        mark(tr, MOE_KERNEL_ROUTE);
+        if (x_dtype == MOE_BF16) {
+            auto kern = route_splitk_kernel<__nv_bfloat16>;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            kern<<<nsplit, threads, sm, s>>>((const __nv_bfloat16 *)x, w_router, bias, T, D, E, k,
+                                             renorm, nsplit, partial, ticket, ids, gates, logits);
+        } else {
+            auto kern = route_splitk_kernel<float>;
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            kern<<<nsplit, threads, sm, s>>>((const float *)x, w_router, bias, T, D, E, k, renorm,
+                                             nsplit, partial, ticket, ids, gates, logits);
+        }
+        return cuda_status(cudaGetLastError(), "route_splitk_kernel");
+    }
+    float *L = logits;
+    if (!L) {
+        L = c.take<float>((size_t)T * E);
+        if (!c.fits()) { set_error("moe_route: workspace too small"); return MOE_ERR_WORKSPACE; }
+    }
+    dim3 grid((T + kTM - 1) / kTM, (E + kTN - 1) / kTN);
+    mark(tr, MOE_KERNEL_ROUTE_LOGITS);
+    if (x_dtype == MOE_BF16)
+        route_logits_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            (const __nv_bfloat16 *)x, w_router, bias, T, D, E, L);
+    else
+        route_logits_tiled_kernel<float><<<grid, 256, 0, s>>>((const float *)x, w_router, bias,
+                                                              T, D, E, L);
+    moe_status st = cuda_status(cudaGetLastError(), "route_logits_tiled_kernel");
+    if (st != MOE_OK) return st;
+    int blocks = (T * 32 + 255) / 256;
+    mark(tr, MOE_KERNEL_ROUTE_SELECT);
+    route_select_kernel<<<blocks, 256, 0, s>>>(L, nullptr, T, E, k, renorm, ids, gates, nullptr);
+    return cuda_status(cudaGetLastError(), "route_select_kernel");
+}
+
+}  // namespace moe

@@ -18,3 +18,14 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def moe():
+    """The CUDA library's Python binding, built in-tree first (nvcc only;
+    no GPU needed to build or load)."""
+    from quantized_routed_expert_top_b200 import build
+    build.build()
+    import quantized_routed_expert_top_b200 as m
+    m.lib()
+    return m

@@ -1,0 +1,151 @@
+"""The C-ABI boundary on the host: the library loads, exports every symbol
+that include/moe.h declares, its tables match the header, and bad arguments
+come back as status codes before any kernel is enqueued (no GPU needed)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import synthetic as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def _header_defines():
+    out = {}
+    for m in re.finditer(r"#define\s+(MOE_\w+)\s+(\d+)", open(HEADER).read()):
+        out[m.group(1)] = int(m.group(2))
+    return out
+
+
+def test_every_declared_symbol_is_exported(moe):
+    names = _declared_functions()
+    assert len(names) >= 17
+    L = C.CDLL(moe.LIB_PATH)
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_block_tables_agree_with_header(moe, orc):
+    h = _header_defines()
+    assert h["MOE_QK"] == S.QK == 32
+    assert h["MOE_Q4_0_BLOCK_BYTES"] == S.BLOCK_BYTES["q4_0"] == moe.BLOCK_BYTES[moe.Q4_0]
+    assert h["MOE_Q8_0_BLOCK_BYTES"] == S.BLOCK_BYTES["q8_0"] == moe.BLOCK_BYTES[moe.Q8_0]
+    assert moe.lib().moe_block_bytes(moe.Q4_0) == 18 == orc.block_bytes("q4_0")
+    assert moe.lib().moe_block_bytes(moe.Q8_0) == 34 == orc.block_bytes("q8_0")
+    assert moe.lib().moe_block_bytes(3) == 0        # unknown type -> 0, never garbage
+    assert S.GGML_TYPE_ID == {"q4_0": moe.Q4_0, "q8_0": moe.Q8_0}
+
+
+def _err(L):
+    return L.moe_last_error().decode()
+
+
+P = C.c_void_p
+FAKE = C.c_void_p(0x1000)      # never dereferenced: every call below fails its checks first
+
+
+def test_route_argument_errors(moe):
+    L = moe.lib()
+    ws, n = FAKE, 1 << 20
+    # k > E
+    assert L.moe_route(FAKE, moe.BF16, FAKE, None, 4, 256, 8, 9, 1, FAKE, FAKE, None, ws, n, None) == 3
+    assert "k" in _err(L)
+    # D not a multiple of 32
+    assert L.moe_route(FAKE, moe.BF16, FAKE, None, 4, 100, 8, 2, 1, FAKE, FAKE, None, ws, n, None) == 3
+    # bad dtype, bad renorm flag
+    assert L.moe_route(FAKE, 7, FAKE, None, 4, 256, 8, 2, 1, FAKE, FAKE, None, ws, n, None) == 1
+    assert L.moe_route(FAKE, moe.BF16, FAKE, None, 4, 256, 8, 2, 2, FAKE, FAKE, None, ws, n, None) == 1
+    # given logits must be F32
+    assert L.moe_route(FAKE, moe.BF16, None, None, 4, 0, 8, 2, 1, FAKE, FAKE, None, ws, n, None) == 1
+    # NULL outputs
+    assert L.moe_route(FAKE, moe.BF16, FAKE, None, 4, 256, 8, 2, 1, None, FAKE, None, ws, n, None) == 1
+    # workspace too small
+    assert L.moe_route(FAKE, moe.BF16, FAKE, None, 4, 256, 8, 2, 1, FAKE, FAKE, None, ws, 1, None) == 7
+    # too many experts
+    assert L.moe_route(FAKE, moe.BF16, FAKE, None, 4, 256, 2048, 2, 1, FAKE, FAKE, None, ws, n, None) == 3
+    # T == 0 is a successful no-op
+    assert L.moe_route(None, moe.BF16, FAKE, None, 0, 256, 8, 2, 1, None, None, None, None, 0, None) == 0
+
+
+def test_expert_ffn_rejects_unknown_and_missing_pools(moe):
+    L = moe.lib()
+    bad = moe.Pool(3, 8, 0x1000, 0x1000, 0x1000, None)       # qtype 3 is not supported
+    assert L.moe_expert_ffn(FAKE, moe.BF16, 4, 256, 512, 8, 2, FAKE, FAKE, C.byref(bad), None,
+                            FAKE, FAKE, 1 << 30, None) == 2
+    assert "quant type" in _err(L)
+    nul = moe.Pool(moe.Q8_0, 8, 0x1000, 0, 0x1000, None)
+    assert L.moe_expert_ffn(FAKE, moe.BF16, 4, 256, 512, 8, 2, FAKE, FAKE, C.byref(nul), None,
+                            FAKE, FAKE, 1 << 30, None) == 1
+    ok = moe.Pool(moe.Q8_0, 8, 0x1000, 0x1000, 0x1000, None)
+    # F not a multiple of 32
+    assert L.moe_expert_ffn(FAKE, moe.BF16, 4, 256, 500, 8, 2, FAKE, FAKE, C.byref(ok), None,
+                            FAKE, FAKE, 1 << 30, None) == 3
+    # workspace too small
+    assert L.moe_expert_ffn(FAKE, moe.BF16, 4, 256, 512, 8, 2, FAKE, FAKE, C.byref(ok), None,
+                            FAKE, FAKE, 16, None) == 7
+    assert L.moe_expert_ffn_workspace_size(4, 2, 256, 512) >= 4 * 2 * 512 * 4
+
+
+def test_combine_and_permute_errors(moe):
+    L = moe.lib()
+    assert L.moe_combine(FAKE, FAKE, FAKE, 4, 2, 256, None, FAKE, 9, None) == 1
+    assert L.moe_combine(None, FAKE, FAKE, 4, 2, 256, None, FAKE, moe.F32, None) == 1
+    assert L.moe_permute(FAKE, 4, 3, 2, FAKE, FAKE, FAKE, FAKE, None) == 3     # k > E
+    assert L.moe_permute(FAKE, 4, 2, 8, None, FAKE, FAKE, FAKE, None) == 1
+
+
+def test_layer_forward_errors(moe):
+    L = moe.lib()
+    pool = moe.Pool(moe.Q4_0, 8, 0x1000, 0x1000, 0x1000, None)
+    a = moe.LayerArgs()
+    a.T, a.D, a.E, a.k, a.F, a.renorm = 4, 256, 8, 2, 512, 1
+    a.x_dtype, a.y_dtype = moe.BF16, moe.BF16
+    a.x, a.y, a.w_router = 0x1000, 0x1000, 0x1000
+    a.pool = C.pointer(pool)
+    need = L.moe_layer_workspace_size(C.byref(a))
+    assert need > 0
+    assert L.moe_layer_forward(C.byref(a), FAKE, need - 1, None) == 7
+    a.y_dtype = moe.F16
+    assert L.moe_layer_forward(C.byref(a), FAKE, need, None) == 1
+    a.y_dtype = moe.BF16
+    sh = moe.Pool(moe.Q8_0, 1, 0x1000, 0x1000, 0x1000, None)
+    a.shared = C.pointer(sh)
+    a.shared_F = 100
+    assert L.moe_layer_forward(C.byref(a), FAKE, 1 << 40, None) == 3
+    a.shared_F = 512
+    badpool = moe.Pool(5, 8, 0x1000, 0x1000, 0x1000, None)
+    a.pool = C.pointer(badpool)
+    assert L.moe_layer_forward(C.byref(a), FAKE, 1 << 40, None) == 2
+    assert L.moe_layer_forward(None, FAKE, 0, None) == 1
+
+
+def test_cache_init_argument_errors(moe):
+    L = moe.lib()
+    h = C.c_void_p()
+    assert L.moe_cache_init(None, C.byref(h)) == 1
+    d = moe.CacheDesc()
+    d.n_layers, d.E, d.n_slots, d.qtype = 2, 8, 9, moe.Q8_0      # more slots than experts
+    assert L.moe_cache_init(C.byref(d), C.byref(h)) == 3
+    d.n_slots, d.qtype = 4, 3
+    assert L.moe_cache_init(C.byref(d), C.byref(h)) == 2
+    d.qtype = moe.Q8_0
+    assert L.moe_cache_init(C.byref(d), C.byref(h)) == 1          # NULL pools
+    assert not h.value
+
+
+def test_error_message_is_per_call(moe):
+    L = moe.lib()
+    L.moe_permute(FAKE, 4, 3, 2, FAKE, FAKE, FAKE, FAKE, None)
+    assert _err(L)
+    assert L.moe_route(None, moe.BF16, FAKE, None, 0, 256, 8, 2, 1, None, None, None, None, 0, None) == 0
+    assert _err(L) == ""

@@ -1,0 +1,253 @@
+"""CUDA path vs the CPU oracle, element by element, on seeded inputs.
+
+Routing indices and the permutation must be bit-exact (a selection decided
+by a logit gap under 1e-5 is logged instead); gates within 1e-6; layer
+outputs within max|gpu-oracle|/max|oracle| <= 2e-3.  Full-size configs are
+compared on sampled tokens/rows the oracle computes one by one, in the same
+launch configuration the bench times (moe_layer_forward).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+from helpers import (GATE_TOL, REL_TOL, check_ids, dev, dev_pool, dev_shared, dev_x,
+                     gates_at, oracle_route, rel_err)
+
+pytestmark = pytest.mark.gpu
+
+_cache = {}
+
+
+def layer_inputs(name, T=None, seed=None):
+    key = (name, T, seed)
+    if key not in _cache:
+        _cache[key] = S.make_layer(S.CONFIGS[name], T=T, seed=seed)
+    return _cache[key]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda(moe):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    yield
+    _cache.clear()
+
+
+def _route_gpu(moe, L):
+    if L.logits is not None:
+        return moe.route(dev(L.logits), None, dev(L.bias), L.cfg.k, L.cfg.renorm, want_logits=True)
+    return moe.route(dev_x(L), dev(L.w_router), dev(L.bias), L.cfg.k, L.cfg.renorm,
+                     want_logits=True)
+
+
+ROUTE_CASES = [("tiny", None), ("decode", 1), ("decode", 4), ("decode", 16), ("decode", 17),
+               ("decode", 37), ("prefill", 8192), ("wide", 1), ("wide", 2048)]
+
+
+@pytest.mark.parametrize("name,T", ROUTE_CASES)
+def test_route_parity(moe, name, T):
+    L = layer_inputs(name, T)
+    ids, gates, logits = _route_gpu(moe, L)
+    torch.cuda.synchronize()
+    ref_logits, ref_ids, ref_g = oracle_route(L)
+    ids, gates, logits = ids.cpu().numpy(), gates.cpu().numpy(), logits.cpu().numpy()
+    scale = 1.0 + np.abs(ref_logits)
+    assert np.all(np.abs(logits - ref_logits) <= 2e-5 * scale)
+    check_ids(ids, ref_ids, ref_logits, L.cfg.k, log=print)
+    # gates of the GPU's selection, from the oracle's logits (valid on ties too)
+    g_ref = gates_at(ref_logits, ids, L.cfg.renorm)
+    assert np.abs(gates - g_ref).max() <= GATE_TOL
+    assert np.all(np.abs(gates.sum(axis=1) - 1) <= 1e-5)
+
+
+def test_route_ties_and_extremes(moe):
+    # exact ties in the logits go to the lower expert id; E=1024, k=32
+    rng = np.random.default_rng(3)
+    E, k, T = 1024, 32, 5
+    Lg = rng.standard_normal((T, E)).astype(np.float32)
+    Lg[0, :] = 0.0                         # all equal -> ids 0..k-1
+    Lg[1, 100:140] = 5.0                   # a block of equal maxima
+    ids, gates = moe.route(dev(Lg), None, None, k)
+    torch.cuda.synchronize()
+    ref_ids, ref_g = oracle.select(Lg, k)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
+    assert np.abs(gates.cpu().numpy() - ref_g).max() <= GATE_TOL
+    # k = E
+    ids2, g2 = moe.route(dev(Lg[:, :8].copy()), None, None, 8)
+    r2, rg2 = oracle.select(Lg[:, :8], 8)
+    np.testing.assert_array_equal(ids2.cpu().numpy(), r2)
+    assert np.abs(g2.cpu().numpy() - rg2).max() <= GATE_TOL
+
+
+def test_route_without_renorm(moe):
+    L = layer_inputs("tiny")
+    ids, gates = moe.route(dev_x(L), dev(L.w_router), None, L.cfg.k, renorm=False)
+    logits, ref_ids, _ = oracle.route(L.x, L.w_router, None, L.cfg.k)
+    ref_ids2, ref_g = oracle.select(logits, L.cfg.k, renorm=False)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids2)
+    assert np.abs(gates.cpu().numpy() - ref_g).max() <= GATE_TOL
+
+
+@pytest.mark.parametrize("T,k,E", [(1, 8, 128), (16, 8, 128), (37, 2, 8), (8192, 8, 128),
+                                   (2048, 10, 512), (3, 32, 1024), (1000, 1, 1)])
+def test_permute_parity(moe, T, k, E):
+    rng = np.random.default_rng(T * 31 + k)
+    if E == 128 and T == 8192:       # skewed, like the prefill routing
+        p = (np.arange(1, E + 1) ** -1.1)
+        p /= p.sum()
+        ids = np.stack([rng.choice(E, k, replace=False, p=p) for _ in range(T)])
+    else:
+        ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)])
+    ids = ids.astype(np.int32)
+    counts, offsets, perm, inv = moe.permute(dev(ids), E)
+    torch.cuda.synchronize()
+    rc, ro, rp, ri = oracle.permute(ids, E)
+    np.testing.assert_array_equal(counts.cpu().numpy(), rc)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), ro)
+    np.testing.assert_array_equal(perm.cpu().numpy(), rp)
+    np.testing.assert_array_equal(inv.cpu().numpy(), ri)
+
+
+def _sample(n, m, seed):
+    if n <= m:
+        return np.arange(n, dtype=np.int32)
+    rng = np.random.default_rng(seed)
+    s = np.sort(rng.choice(n, m, replace=False)).astype(np.int32)
+    s[0], s[-1] = 0, n - 1                 # both ends of the range
+    return np.unique(s)
+
+
+@pytest.mark.parametrize("name,T,n_rows", [("tiny", None, 999), ("decode", 16, 999),
+                                           ("decode", 5, 999), ("prefill", 8192, 40),
+                                           ("wide", 2048, 40)])
+def test_expert_ffn_and_combine_parity(moe, name, T, n_rows):
+    L = layer_inputs(name, T)
+    cfg = L.cfg
+    ids_d, gates_d = _route_gpu(moe, L)[:2]
+    counts, offsets, perm, inv = moe.permute(ids_d, cfg.E)
+    pool = dev_pool(moe, L)
+    rows = moe.expert_ffn(dev_x(L), perm, offsets, pool, cfg.k, cfg.F)
+    y = moe.combine(rows, inv, gates_d, y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    Tn = L.x.shape[0]
+    pos = _sample(Tn * cfg.k, n_rows, 11)
+    ref = oracle.expert_rows(L.x, perm.cpu().numpy(), offsets.cpu().numpy(), cfg.k, L.gate,
+                             L.up, L.down, cfg.qtype, cfg.F, positions=pos)
+    got = rows.cpu().numpy()[pos]
+    assert rel_err(got, ref) <= REL_TOL
+    # combine of the GPU rows, recomputed in double from the same rows
+    toks = _sample(Tn, 64, 12)
+    rows_h, inv_h, g_h = rows.cpu().numpy().astype(np.float64), inv.cpu().numpy(), gates_d.cpu().numpy()
+    yref = np.stack([sum(g_h[t, j] * rows_h[inv_h[t * cfg.k + j]] for j in range(cfg.k)) for t in toks])
+    assert np.abs(y.cpu().numpy()[toks] - yref).max() <= 1e-5 * np.abs(yref).max()
+
+
+def _layer(moe, L, T_max=None):
+    cfg = L.cfg
+    T = L.x.shape[0]
+    shared = dev_shared(moe, L)
+    xdt = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
+    ydt = torch.bfloat16 if cfg.y_dtype == "bf16" else torch.float32
+    return moe.Layer(dev_pool(moe, L), cfg.D, cfg.F, cfg.E, cfg.k, T_max or T,
+                     w_router=dev(L.w_router), bias=dev(L.bias), shared=shared,
+                     shared_F=cfg.shared_F, renorm=cfg.renorm, x_dtype=xdt, y_dtype=ydt)
+
+
+def _check_layer(moe, L, y_gpu, ids_gpu, n_tok, log=print):
+    cfg = L.cfg
+    T = L.x.shape[0]
+    ref_logits, ref_ids, ref_g = oracle_route(L)
+    ids_gpu = ids_gpu.cpu().numpy()[:T]
+    tied = check_ids(ids_gpu, ref_ids, ref_logits, cfg.k, log=log)
+    toks = _sample(T, n_tok, 13)
+    # tokens whose selection differs (near ties) are checked against the
+    # oracle run on the GPU's selection
+    use_ids = ref_ids.copy()
+    use_g = ref_g.copy()
+    if tied:
+        use_ids[tied] = ids_gpu[tied]
+        use_g[tied] = gates_at(ref_logits[tied], ids_gpu[tied], cfg.renorm)
+    ref = oracle.layer(L.x, use_ids, use_g, L.gate, L.up, L.down, cfg.qtype, cfg.F,
+                       shared=L.shared, tokens=toks)
+    got = y_gpu.float().cpu().numpy()[toks]
+    err = rel_err(got, ref)
+    assert err <= REL_TOL, err
+    return err
+
+
+LAYER_CASES = [("tiny", None, 99), ("decode", 1, 99), ("decode", 4, 99), ("decode", 16, 99),
+               ("decode", 37, 99), ("prefill", 8192, 48), ("wide", 1, 99), ("wide", 2048, 40)]
+
+
+@pytest.mark.parametrize("name,T,n_tok", LAYER_CASES)
+def test_layer_forward_parity(moe, name, T, n_tok):
+    L = layer_inputs(name, T)
+    lay = _layer(moe, L)
+    if L.logits is not None:
+        y = lay.forward(dev_x(L), logits=dev(L.logits))
+    else:
+        y = lay.forward(dev_x(L))
+    torch.cuda.synchronize()
+    _check_layer(moe, L, y, lay.ids, n_tok)
+
+
+def test_layer_forward_repeated_calls_are_identical(moe):
+    # the workspace carries state between calls (the router's ticket); a
+    # second call must reproduce the first bit for bit
+    L = layer_inputs("decode", 4)
+    lay = _layer(moe, L)
+    x = dev_x(L)
+    y1 = lay.forward(x).clone()
+    y2 = lay.forward(x).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_layer_zero_tokens_is_noop(moe):
+    L = layer_inputs("tiny")
+    lay = _layer(moe, L, T_max=4)
+    y = lay.forward(dev_x(L)[:0])
+    torch.cuda.synchronize()
+    assert y.shape == (0, L.cfg.D)
+
+
+@pytest.mark.parametrize("qtype", ["q4_0", "q8_0"])
+def test_layer_odd_shapes(moe, qtype):
+    # D, F multiples of 32 but not of 256; E = k; ragged T
+    cfg = S.LayerConfig("odd", T=7, D=96, E=3, k=3, F=160, qtype=qtype, x_dtype="bf16",
+                        y_dtype="f32", router_std=0.1, seed=77)
+    L = S.make_layer(cfg)
+    lay = _layer(moe, L)
+    y = lay.forward(dev_x(L))
+    torch.cuda.synchronize()
+    _check_layer(moe, L, y, lay.ids, 99)
+
+
+def test_single_expert_layer(moe):
+    cfg = S.LayerConfig("one", T=9, D=256, E=1, k=1, F=256, qtype="q8_0", x_dtype="f32",
+                        y_dtype="f32", seed=78)
+    L = S.make_layer(cfg)
+    lay = _layer(moe, L)
+    y = lay.forward(dev_x(L))
+    torch.cuda.synchronize()
+    _check_layer(moe, L, y, lay.ids, 99)
+    assert np.all(lay.gates.cpu().numpy() == 1.0)
+
+
+def test_masked_two_phase_rows_are_bit_identical(moe):
+    L = layer_inputs("decode", 16)
+    cfg = L.cfg
+    ids_d, gates_d = _route_gpu(moe, L)[:2]
+    counts, offsets, perm, inv = moe.permute(ids_d, cfg.E)
+    pool = dev_pool(moe, L)
+    x = dev_x(L)
+    full = moe.expert_ffn(x, perm, offsets, pool, cfg.k, cfg.F)
+    rng = np.random.default_rng(4)
+    m = torch.from_numpy(rng.integers(0, 2, cfg.E).astype(np.uint8)).cuda()
+    two = torch.full_like(full, float("nan"))
+    moe.expert_ffn(x, perm, offsets, pool, cfg.k, cfg.F, mask=m, out=two)
+    moe.expert_ffn(x, perm, offsets, pool, cfg.k, cfg.F, mask=1 - m, out=two)
+    torch.cuda.synchronize()
+    assert torch.equal(full, two)
