@@ -254,7 +254,7 @@ class Layer:
         a.shared_F = self.shared_F if self.shared is not None else 0
         a.renorm = int(self.renorm)
         a.x_dtype = _DT[self.x_dtype]
-        a.y_dtype = _DT[self.y_dtype]
+        a.y_dtype = _DT[self.y_dtype if y is None else y.dtype]
         a.x = None if x is None else x.data_ptr()
         a.w_router = None if self.w_router is None else self.w_router.data_ptr()
         a.bias = None if self.bias is None else self.bias.data_ptr()
@@ -299,6 +299,9 @@ class KernelTrace:
 
     def __init__(self, n_calls: int, per_call: int = 16):
         self.pool = [torch.cuda.Event(enable_timing=True) for _ in range(n_calls * per_call)]
+        for e in self.pool:          # torch creates events lazily: force the handles
+            e.record()
+        torch.cuda.synchronize()
         self.per_call = per_call
         self.calls = []
         self._next = 0

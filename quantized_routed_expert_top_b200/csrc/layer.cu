@@ -81,7 +81,13 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
     }
     st = launch_combine(w.rows, w.inv, gates, a.T, a.k, a.D, a.shared ? w.sh_rows : nullptr, a.y,
                         a.y_dtype, s, tr);
-    if (tr) tr->end();
+    if (tr) {
+        tr->end();
+        if (st == MOE_OK && tr->err != cudaSuccess) {
+            cudaGetLastError();   // the failed record is reported here, not left sticky
+            return cuda_status(tr->err, "moe_layer_forward: trace event record");
+        }
+    }
     return st;
 }
 

@@ -46,10 +46,12 @@ struct Tracer {
     moe_trace *t = nullptr;
     cudaStream_t s = nullptr;
     bool open = false;
+    cudaError_t err = cudaSuccess;
     // before launching a kernel of `kind`
     void mark(int kind) {
         if (!t || t->count >= t->capacity || t->count >= MOE_TRACE_MAX) return;
-        cudaEventRecord((cudaEvent_t)t->events[t->count], s);
+        cudaError_t e = cudaEventRecord((cudaEvent_t)t->events[t->count], s);
+        if (e != cudaSuccess && err == cudaSuccess) err = e;
         t->kinds[t->count] = kind;
         t->count++;
         open = true;
@@ -57,7 +59,8 @@ struct Tracer {
     // after the last kernel
     void end() {
         if (!t || !open || t->count >= t->capacity) return;
-        cudaEventRecord((cudaEvent_t)t->events[t->count], s);
+        cudaError_t e = cudaEventRecord((cudaEvent_t)t->events[t->count], s);
+        if (e != cudaSuccess && err == cudaSuccess) err = e;
         t->kinds[t->count] = 0;
         t->count++;
         open = false;

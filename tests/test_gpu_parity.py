@@ -56,9 +56,14 @@ def test_route_parity(moe, name, T):
     scale = 1.0 + np.abs(ref_logits)
     assert np.all(np.abs(logits - ref_logits) <= 2e-5 * scale)
     check_ids(ids, ref_ids, ref_logits, L.cfg.k, log=print)
-    # gates of the GPU's selection, from the oracle's logits (valid on ties too)
+    # (a) the gate arithmetic: softmax/renormalisation of the GPU's own fp32
+    # logits at the GPU's selection, to 1e-6
+    assert np.abs(gates - gates_at(logits, ids, L.cfg.renorm)).max() <= GATE_TOL
+    # (b) end to end against the oracle's logits: 1e-6 plus the propagated
+    # fp32 logit error (|dg_j| <= g_j * 2 max_i |dL_i| <= 2 max_i |dL_i|)
+    dL = np.abs(logits.astype(np.float64) - ref_logits).max(axis=1, keepdims=True)
     g_ref = gates_at(ref_logits, ids, L.cfg.renorm)
-    assert np.abs(gates - g_ref).max() <= GATE_TOL
+    assert np.all(np.abs(gates - g_ref) <= GATE_TOL + 2 * dL)
     assert np.all(np.abs(gates.sum(axis=1) - 1) <= 1e-5)
 
 
@@ -156,6 +161,7 @@ def _layer(moe, L, T_max=None):
 
 
 def _check_layer(moe, L, y_gpu, ids_gpu, n_tok, log=print):
+    """Parity of an fp32 layer output with the oracle on sampled tokens."""
     cfg = L.cfg
     T = L.x.shape[0]
     ref_logits, ref_ids, ref_g = oracle_route(L)
@@ -183,14 +189,19 @@ LAYER_CASES = [("tiny", None, 99), ("decode", 1, 99), ("decode", 4, 99), ("decod
 
 @pytest.mark.parametrize("name,T,n_tok", LAYER_CASES)
 def test_layer_forward_parity(moe, name, T, n_tok):
+    # the 2e-3 bar applies to the fp32-accumulated result (fp32 output); the
+    # configured output type (bf16 for most configs) must then be exactly the
+    # round-to-nearest-even of that fp32 result
     L = layer_inputs(name, T)
     lay = _layer(moe, L)
-    if L.logits is not None:
-        y = lay.forward(dev_x(L), logits=dev(L.logits))
-    else:
-        y = lay.forward(dev_x(L))
+    Tn = L.x.shape[0]
+    logits = None if L.logits is None else dev(L.logits)
+    y32 = torch.empty((Tn, L.cfg.D), dtype=torch.float32, device="cuda")
+    lay.forward(dev_x(L), logits=logits, out=y32)
+    y = lay.forward(dev_x(L), logits=logits)
     torch.cuda.synchronize()
-    _check_layer(moe, L, y, lay.ids, n_tok)
+    print(f"rel err {_check_layer(moe, L, y32, lay.ids, n_tok):.3e}")
+    assert torch.equal(y, y32.to(y.dtype))
 
 
 def test_layer_forward_repeated_calls_are_identical(moe):
