@@ -116,6 +116,27 @@ moe_status moe_route(const void *x, int32_t x_dtype, const float *w_router,
                      int32_t *ids, float *gates, float *logits,
                      void *workspace, size_t ws_bytes, moe_stream stream);
 
+/* moe_route_noalloc: the same routing as moe_route for small batches, for
+ * callers that cannot allocate device memory when they route (code running
+ * inside an allocator's own callbacks, serving loops that freeze their
+ * memory footprint after start-up, embedders whose runtime owns every
+ * device allocation and lends no scratch buffer).  It takes no workspace:
+ * its scratch is a fixed array inside the library, 2 MiB per GPU that loads
+ * the library, held until the process exits.  The pages have no counterpart
+ * to this entry point; it exists for such callers only.
+ *   Arguments as moe_route, except: w_router must not be NULL, and
+ *   T <= 16 and ceil(D/32) * T * E <= 524288 (else MOE_ERR_SHAPE, with the
+ *   limit in the message).
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before capturing any stream.  Every call on a device shares the array
+ *   and leaves its contents behind (the completion counter is cleared at the
+ *   start of each call); calls that overlap on the GPU race, so serialise
+ *   them (one stream, or events between streams). */
+moe_status moe_route_noalloc(const void *x, int32_t x_dtype, const float *w_router,
+                             const float *bias, int T, int D, int E, int k, int renorm,
+                             int32_t *ids, float *gates, float *logits, moe_stream stream);
+
 /* --------------------------------------------------------- permutation
  * moe_permute: stable grouping of the T*k (token, slot) entries by expert.
  *   ids     device int32 [T, k], each in [0, E).

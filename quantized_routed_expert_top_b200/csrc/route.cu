@@ -21,6 +21,7 @@
 #include <algorithm>
 #include <cfloat>
 #include <climits>
+#include <mutex>
 
 namespace moe {
 
@@ -279,3 +280,111 @@ moe_status launch_route(const void *x, int x_dtype, const float *w_router,
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Allocation-free routing entry point.
+//
+// Some callers cannot allocate device memory at the point where they route:
+// code running inside a custom allocator's own callbacks, serving loops that
+// forbid allocation after start-up so their memory footprint stays fixed,
+// and embedders whose runtime owns every device allocation and offers no
+// scratch buffer.  For them moe_route_noalloc runs the small-T router (the
+// split-K logits + top-k kernel above) with its scratch in a fixed
+// file-scope device array instead of a caller workspace.
+//
+// kNoAllocFloats bounds the scratch: ceil(D/32) * T * E fp32 partial sums
+// (T <= 16) must fit in it; one more word is the completion ticket.  The
+// array lives in every GPU that loads this library until the process exits.
+// Every call on a device shares it, so calls that overlap on the GPU (other
+// streams, other host threads) race and must be serialised by the caller.
+// The ticket is cleared with a memset before each launch; the partial sums
+// are fully written before they are read and need no clearing.
+// ---------------------------------------------------------------------------
+namespace moe {
+
+constexpr size_t kNoAllocFloats = size_t(1) << 19;     // 2 MiB of partial sums
+
+static __device__ __align__(256) float g_route_scratch[kNoAllocFloats + 64];
+
+// Device address of g_route_scratch, looked up once per device (host code
+// cannot use the array's name as a device pointer).
+static void *noalloc_scratch_address(int dev, moe_status *st) {
+    static std::mutex mu;
+    static void *addr[128] = {nullptr};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 128) {
+        set_error("moe_route_noalloc: device ordinal %d out of range", dev);
+        *st = MOE_ERR_INVALID_ARG;
+        return nullptr;
+    }
+    if (!addr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess) {
+            *st = cuda_status(e, "moe_route_noalloc: cudaGetSymbolAddress");
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    *st = MOE_OK;
+    return addr[dev];
+}
+
+}  // namespace moe
+
+extern "C" moe_status moe_route_noalloc(const void *x, int32_t x_dtype, const float *w_router,
+                                        const float *bias, int T, int D, int E, int k, int renorm,
+                                        int32_t *ids, float *gates, float *logits,
+                                        moe_stream stream) {
+    using namespace moe;
+    if (T < 0 || D <= 0 || E <= 0 || k <= 0 || D % QK || k > E || E > MOE_MAX_EXPERTS ||
+        k > MOE_MAX_TOPK) {
+        set_error("moe_route_noalloc: bad shape (T=%d D=%d E=%d k=%d)", T, D, E, k);
+        return MOE_ERR_SHAPE;
+    }
+    if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) {
+        set_error("moe_route_noalloc: x dtype %d not F32/BF16", x_dtype);
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (renorm != 0 && renorm != 1) {
+        set_error("moe_route_noalloc: renorm must be 0 or 1");
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (T == 0) return MOE_OK;
+    if (!x || !w_router || !ids || !gates) {
+        set_error("moe_route_noalloc: NULL x, w_router, ids or gates");
+        return MOE_ERR_INVALID_ARG;
+    }
+    const int nsplit = (D + kSplitRows - 1) / kSplitRows;
+    if (T > kSplitMaxT || (size_t)nsplit * T * E > kNoAllocFloats) {
+        set_error("moe_route_noalloc: T=%d D=%d E=%d needs T <= %d and ceil(D/32)*T*E <= %zu "
+                  "scratch floats", T, D, E, kSplitMaxT, kNoAllocFloats);
+        return MOE_ERR_SHAPE;
+    }
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return cuda_status(ce, "moe_route_noalloc: cudaGetDevice");
+    moe_status st;
+    float *scratch = (float *)noalloc_scratch_address(dev, &st);
+    if (!scratch) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned *ticket = (unsigned *)(scratch + kNoAllocFloats);
+    float *partial = scratch;
+    ce = cudaMemsetAsync(ticket, 0, sizeof(unsigned), s);
+    if (ce != cudaSuccess) return cuda_status(ce, "moe_route_noalloc: ticket clear");
+    int threads = (int)round_up(E, 32);
+    if (threads < 128) threads = 128;
+    size_t sm = (size_t)std::max(T * kSplitRows, T * E) * sizeof(float);
+    if (x_dtype == MOE_BF16) {
+        auto kern = route_splitk_kernel<__nv_bfloat16>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        kern<<<nsplit, threads, sm, s>>>((const __nv_bfloat16 *)x, w_router, bias, T, D, E, k,
+                                         renorm, nsplit, partial, ticket, ids, gates, logits);
+    } else {
+        auto kern = route_splitk_kernel<float>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        kern<<<nsplit, threads, sm, s>>>((const float *)x, w_router, bias, T, D, E, k, renorm,
+                                         nsplit, partial, ticket, ids, gates, logits);
+    }
+    return cuda_status(cudaGetLastError(), "moe_route_noalloc: route_splitk_kernel");
+}
