@@ -211,12 +211,24 @@ class Workload:
         self.r = 0
         self.tokens_per_step = sum(Ts)
         self.calls_per_step = len(Ts)
+        self.kernels_per_call = self._count_kernels()
 
-    def step(self, trace=None, x=None, y=None):
+    def _count_kernels(self):
+        """Kernels one layer call launches (from a traced eager call)."""
+        tr = self.moe.KernelTrace(n_calls=1)
+        T = self.Ts[0]
+        self.layers[0].forward(self.x[T], logits=self.logits[T], out=self.y[T], trace=tr)
+        self.torch.cuda.synchronize()
+        kinds = [k for k, _, _ in tr.calls[0]]
+        # the decode FFN segment covers two kernels (gate/up, down + combine)
+        return len(kinds) + kinds.count("ffn_decode")
+
+    def step(self, trace=None, x=None, y=None, logits=None):
         for T in self.Ts:
             lay = self.layers[self.r]
             self.r = (self.r + 1) % len(self.layers)
-            lay.forward(self.x[T] if x is None else x[T], logits=self.logits[T],
+            lay.forward(self.x[T] if x is None else x[T],
+                        logits=self.logits[T] if logits is None else logits[T],
                         out=self.y[T] if y is None else y[T], trace=trace)
 
     # algorithmic work of one step, from the routing of each call
@@ -234,21 +246,41 @@ class Workload:
         distinct = self.distinct_experts()
         gb, ub, db = S.expert_bytes(cfg.D, cfg.F, cfg.qtype)
         act = 2 if cfg.x_dtype == "bf16" else 4
+        yb = 2 if cfg.y_dtype == "bf16" else 4
         per_call = {}
         for T in self.Ts:
             n = distinct[T]
-            gateup = n * (gb + ub) + T * cfg.D * act + T * cfg.k * cfg.F * 4
-            down = n * db + T * cfg.k * cfg.F * 4 + T * cfg.k * cfg.D * 4
             flops = 2.0 * T * cfg.k * 3 * cfg.D * cfg.F
             if cfg.shared_F:
                 flops += 2.0 * T * 3 * cfg.D * cfg.shared_F
-            per_call[T] = {"distinct": n, "gateup_bytes": gateup, "down_bytes": down,
-                           "weight_bytes": n * (gb + ub + db) + self.shared_bytes,
-                           "flops": flops}
+            x_b = T * cfg.D * act
+            # algorithmic HBM bytes of each traced segment (weights once,
+            # activations in and out once)
+            seg = {
+                "ffn_decode": n * (gb + ub + db) + self.shared_bytes + x_b + T * cfg.D * yb,
+                "gateup": n * (gb + ub) + x_b + T * cfg.k * cfg.F * 4,
+                "down": n * db + T * cfg.k * cfg.F * 4 + T * cfg.k * cfg.D * 4,
+                "route": (cfg.D * cfg.E * 4 if base_router(self) else T * cfg.E * 4) + x_b,
+            }
+            per_call[T] = {"distinct": n, "seg_bytes": seg, "flops": flops,
+                           "weight_bytes": n * (gb + ub + db) + self.shared_bytes}
         return per_call
 
 
+def base_router(wl):
+    return wl.inputs[wl.Ts[0]].w_router is not None
+
+
 # ------------------------------------------------------------- our arm
+def capture_graph(torch, fn, n):
+    """Capture n calls of fn (library launches only) into one CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(n):
+            fn()
+    return g
+
+
 def run_ours(args, world, rank, local):
     import torch
     import quantized_routed_expert_top_b200 as moe
@@ -262,26 +294,39 @@ def run_ours(args, world, rank, local):
     algo = wl.algorithmic()
     stream = torch.cuda.current_stream()
 
-    for _ in range(args.warmup):
-        wl.step()
+    # eager calls first (first-use set-up), then the steps as CUDA graphs: the
+    # decode layer is a handful of short kernels and would otherwise wait on
+    # the host's launch path (--no-graph launches every step eagerly)
+    wl.step()
+    torch.cuda.synchronize()
+    trace = moe.KernelTrace(n_calls=args.steps * wl.calls_per_step)
+    if args.no_graph:
+        class _Eager:
+            def __init__(self, fn, n): self.fn, self.n = fn, n
+            def replay(self):
+                for _ in range(self.n): self.fn()
+        g_warm = _Eager(wl.step, args.warmup)
+        g_timed = _Eager(lambda: wl.step(trace=trace), args.steps)
+    else:
+        g_warm = capture_graph(torch, wl.step, args.warmup)
+        g_timed = capture_graph(torch, lambda: wl.step(trace=trace), args.steps)
+    g_warm.replay()
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, with the library's per-kernel trace events
-    trace = moe.KernelTrace(n_calls=args.steps * wl.calls_per_step)
+    # ---- timed region: K steps (one graph replay), trace events inside
     barrier(world)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, period_s=0.0005) as clk:
         t0.record(stream)
-        for _ in range(args.steps):
-            wl.step(trace=trace)
+        g_timed.replay()
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     ms_step = t0.elapsed_time(t1) / args.steps
     ms_step = max_over_ranks(ms_step, world)
     durs = trace.durations()
-    launches = sum(len(c) for c in trace.calls)
+    launches = wl.kernels_per_call * wl.calls_per_step * args.steps
 
     # ---- end to end: pinned host x -> device, layer, device -> pinned host y
     xh = {T: wl.x[T].cpu().pin_memory() for T in wl.Ts}
@@ -289,24 +334,31 @@ def run_ours(args, world, rank, local):
     xd = {T: torch.empty_like(wl.x[T]) for T in wl.Ts}
     h2d = sum(xh[T].numel() * xh[T].element_size() for T in wl.Ts)
     d2h = sum(yh[T].numel() * yh[T].element_size() for T in wl.Ts)
-    if args.workload == "wide":
-        h2d += sum(wl.logits[T].numel() * 4 for T in wl.Ts)
+    lh = {T: None if wl.logits[T] is None else wl.logits[T].cpu().pin_memory() for T in wl.Ts}
+    ld = {T: None if wl.logits[T] is None else torch.empty_like(wl.logits[T]) for T in wl.Ts}
+    h2d += sum(lh[T].numel() * 4 for T in wl.Ts if lh[T] is not None)
 
     def e2e_step():
         for T in wl.Ts:
             xd[T].copy_(xh[T], non_blocking=True)
-        wl.step(x=xd)
+            if lh[T] is not None:
+                ld[T].copy_(lh[T], non_blocking=True)
+        wl.step(x=xd, logits=ld if wl.logits[wl.Ts[0]] is not None else None)
         for T in wl.Ts:
             yh[T].copy_(wl.y[T], non_blocking=True)
 
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
+    if args.no_graph:
+        for _ in range(args.warmup):
+            e2e_step()
+        g_e2e = _Eager(e2e_step, args.steps)
+    else:
+        g_e2e = capture_graph(torch, e2e_step, args.steps)
+        capture_graph(torch, e2e_step, args.warmup).replay()
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    g_e2e.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
@@ -336,6 +388,7 @@ def run_ours(args, world, rank, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
         "peaks": peaks,
+        "launch": "eager" if args.no_graph else "cuda-graph replay",
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, args)
@@ -361,36 +414,30 @@ def config_of(wl):
 
 
 def roofline(wl, algo, durs, peaks, args):
-    """Roofline of the dominant kernel from the trace of the timed steps."""
+    """Roofline of the dominant traced segment over the timed steps."""
     tot = {k: sum(v) for k, v in durs.items()}
     dom = max(tot, key=tot.get)
-    cfg = wl.cfg
-    n_calls = args.steps
-    if dom in ("gateup", "down"):
-        key = "gateup_bytes" if dom == "gateup" else "down_bytes"
-        bytes_step = sum(algo[T][key] for T in wl.Ts)
-        launches = len(durs[dom])
-        per_launch = bytes_step / wl.calls_per_step
-        avg_ms = tot[dom] / launches
-        # achieved over all launches: total algorithmic bytes / total time
-        achieved = bytes_step * n_calls / (tot[dom] / 1e3) / 1e9
-        bound, peak, unit = "hbm", peaks["hbm_gbs"], "GB/s"
-        if wl.name == "prefill":
-            flops_step = sum(algo[T]["flops"] for T in wl.Ts) * (2 / 3 if dom == "gateup" else 1 / 3)
-            achieved = flops_step * n_calls / (tot[dom] / 1e3) / 1e12
-            bound, peak, unit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
-            per_launch = flops_step
+    launches = len(durs[dom])
+    avg_ms = tot[dom] / launches
+    if wl.name == "prefill" and dom in ("gateup", "down", "ffn_tc"):
+        frac_flops = {"gateup": 2 / 3, "down": 1 / 3}.get(dom, 1.0)
+        work_step = sum(algo[T]["flops"] for T in wl.Ts) * frac_flops
+        achieved = work_step * args.steps / (tot[dom] / 1e3) / 1e12
+        bound, peak, unit, spec = "tensor", peaks["bf16_tflops"], "TFLOP/s", TC_SPEC_TFLOPS
+        psrc = "bf16_tflops (fp16 operands run at the bf16 rate)"
     else:
-        achieved, bound, peak, unit, per_launch, avg_ms = None, "hbm", peaks["hbm_gbs"], "GB/s", None, tot[dom] / len(durs[dom])
-    r = {"kernel": dom, "bound": bound, "achieved": None if achieved is None else round(achieved, 2),
-         "peak": peak, "unit": unit,
-         "frac": None if achieved is None else round(achieved / peak, 4),
-         "frac_of_spec": None if achieved is None else round(
-             achieved / (HBM_SPEC_GBS if bound == "hbm" else TC_SPEC_TFLOPS), 4),
-         "algorithmic_per_launch": per_launch, "avg_launch_ms": round(avg_ms, 5),
-         "peak_source": f"{peaks['source']} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
-         "traffic": ncu_traffic(dom, wl.name)}
-    return r
+        work_step = sum(algo[T]["seg_bytes"].get(dom, 0) for T in wl.Ts)
+        achieved = work_step * args.steps / (tot[dom] / 1e3) / 1e9
+        bound, peak, unit, spec = "hbm", peaks["hbm_gbs"], "GB/s", HBM_SPEC_GBS
+        psrc = "hbm_gbs"
+    return {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+            "unit": unit, "frac": round(achieved / peak, 4), "frac_of_spec": round(achieved / spec, 4),
+            "algorithmic_per_launch": round(work_step / wl.calls_per_step, 1),
+            "avg_launch_ms": round(avg_ms, 5),
+            "per_T": {str(T): {"work": algo[T]["seg_bytes"].get(dom) if bound == "hbm" else algo[T]["flops"],
+                               "distinct_experts": algo[T]["distinct"]} for T in wl.Ts},
+            "peak_source": f"{peaks['source']} {psrc}",
+            "traffic": ncu_traffic(dom, wl.name)}
 
 
 def ncu_traffic(kernel, workload):
@@ -540,6 +587,8 @@ def main():
     ap.add_argument("--workload", choices=["decode", "prefill", "wide"], default="decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the steps eagerly instead of replaying CUDA graphs")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

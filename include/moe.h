@@ -224,7 +224,10 @@ typedef enum {
     MOE_KERNEL_SHARED_GATEUP = 8,
     MOE_KERNEL_SHARED_DOWN = 9,
     MOE_KERNEL_CONVERT = 10,       /* activation cast for the tensor-core path */
-    MOE_KERNEL_ZERO = 11           /* accumulator clear */
+    MOE_KERNEL_ZERO = 11,          /* accumulator clear */
+    MOE_KERNEL_FFN_DECODE = 12     /* decode gate/up + down (+combine) pair; the
+                                      two kernels overlap through programmatic
+                                      dependent launch, so they are timed as one */
 } moe_kernel_kind;
 
 #define MOE_TRACE_MAX 24

@@ -41,7 +41,7 @@ class Pool(C.Structure):
 TRACE_MAX = 24
 KERNEL_KINDS = {1: "route", 2: "route_logits", 3: "route_select", 4: "permute", 5: "gateup",
                 6: "down", 7: "combine", 8: "shared_gateup", 9: "shared_down", 10: "convert",
-                11: "zero"}
+                11: "zero", 12: "ffn_decode"}
 
 
 class Trace(C.Structure):

@@ -120,8 +120,13 @@ moe_status moe_route(const void *x, int32_t x_dtype, const float *w_router, cons
         set_error("moe_route: workspace needs %zu bytes, got %zu", route_ws_bytes(T, D, E, k), ws_bytes);
         return MOE_ERR_WORKSPACE;
     }
-    return launch_route(x, x_dtype, w_router, bias, T, D, E, k, renorm, ids, gates, logits,
-                        workspace, ws_bytes, (cudaStream_t)stream);
+    bool permuted = false;
+    // the route workspace starts with 64 words of counters; word 32 is the
+    // status word of the bounded waits
+    int *err = (int *)workspace + 32;
+    return launch_route_permute(x, x_dtype, w_router, bias, T, D, E, k, renorm, ids, gates,
+                                logits, nullptr, nullptr, nullptr, nullptr, err, workspace,
+                                ws_bytes, (cudaStream_t)stream, nullptr, &permuted);
 }
 
 // --------------------------------------------------------------- permute
@@ -138,9 +143,11 @@ moe_status moe_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
 
 // ------------------------------------------------------------ expert FFN
 size_t moe_expert_ffn_workspace_size(int T, int k, int D, int F) {
-    (void)D;
     Carver c(nullptr, 0);
-    c.take<float>((size_t)(T < 0 ? 0 : T) * k * F);
+    T = T < 0 ? 0 : T;
+    c.take<int>(16);
+    if (decode_path_ok(T, D, F, 0)) c.take<__half>(decode_hs_halves(T, k, F, 0));
+    else c.take<float>((size_t)T * k * F);
     return c.off;
 }
 
@@ -161,6 +168,13 @@ moe_status moe_expert_ffn(const void *x, int32_t x_dtype, int T, int D, int F, i
         return MOE_ERR_WORKSPACE;
     }
     Carver c(workspace, ws_bytes);
+    int *status = c.take<int>(16);
+    if (decode_path_ok(T, D, F, 0)) {
+        __half *Hs = c.take<__half>(decode_hs_halves(T, k, F, 0));
+        return launch_ffn_decode(x, x_dtype, T, D, F, E, k, perm, offsets, nullptr, *pool,
+                                 expert_mask, nullptr, 0, Hs, nullptr, MOE_F32, out_rows, status,
+                                 (cudaStream_t)stream, nullptr);
+    }
     float *H = c.take<float>((size_t)T * k * F);
     return launch_ffn_generic(x, x_dtype, T, D, F, E, k, perm, offsets, *pool, expert_mask, H,
                               out_rows, (cudaStream_t)stream);

@@ -1,0 +1,961 @@
+// ffn_decode.cu -- the decode (small T) expert FFN: a dequant-fused grouped
+// GEMV streamed from HBM by the TMA engine.
+//
+// Decode reads every active expert's packed blocks once and does a handful
+// of FLOPs per weight, so the roofline is HBM bandwidth.  Two persistent
+// kernels, one CTA per SM, each with one producer warp and sixteen consumer
+// warps around a ring of shared-memory stages:
+//
+//  * dec_gateup: work unit = (expert, 16-row tile of F).  The producer
+//    copies the 16 gate rows and 16 up rows of a K-slice (<= 32 blocks) with
+//    cp.async.bulk (one copy per row slice, rows padded so that the
+//    consumers' 32-bit loads hit 32 distinct banks).  Consumer warp w takes
+//    matrix w / 8 and K-group w % 8.  Codes are turned into exact fp16 values
+//    c + q (c = 1024 for Q4_0 codes, 1152 for Q8_0 codes) with bit operations
+//    only, and mma.sync m16n8k16 runs with the expert's tokens as the N
+//    dimension (the activations are broadcast inside the tensor core).  The
+//    constant is removed through the MMA's accumulator input: it starts at
+//    -c * sum_k x_k (per block and token, precomputed once), so the block's
+//    result is sum (q - off) x exactly up to fp32 rounding, and the block
+//    scale d multiplies that fp32 result; no weight is rounded.  A fixed-
+//    order cross-warp sum, SwiGLU and the token's gate weight give Hs = g * h
+//    in fp16, stored in the fragment order the next kernel reads.
+//  * dec_down: work unit = 16 rows of D; the unit walks all active experts in
+//    ascending id (then the shared expert); warp w takes experts of parity
+//    w / 8 and K-group w % 8.  Codes become exact (q - off) fp16 values, the
+//    block scale multiplies the fp32 MMA result, and each warp adds its part
+//    into per-token shared-memory sums reduced over warps in a fixed order at
+//    the end of the unit: the combine is folded in, y is deterministic and
+//    no [T*k, D] buffer exists.  With rows_out set it writes every permuted
+//    row's Y instead (no gate, no combine): the two-phase expert-cache path.
+//
+// dec_down is launched with programmatic dependent launch: it copies its
+// down-projection weights while dec_gateup is still running and waits
+// (griddepcontrol.wait) only before copying Hs.
+//
+// Fragment order of an activation block (32 values, one 64-byte row piece):
+// for c = 0..3 eight halves [v(4c), v(4c+2), v(4c+1), v(4c+3), v(16+4c),
+// v(18+4c), v(17+4c), v(19+4c)], matching the codes one 32-bit word of a
+// Q4_0 block gives thread c (byte j = v_j | v_{j+16} << 4), and the two
+// words (bytes 4c.., 16+4c..) of a Q8_0 block.
+#include "moe_internal.cuh"
+#include "sm100.cuh"
+
+#include <cuda.h>
+#include <algorithm>
+#include <cstring>
+
+namespace moe {
+
+constexpr int kTile = 16;                       // rows per MMA tile
+constexpr int kMaxStages = 8;
+constexpr size_t kDecSmemMax = 225 * 1024;      // dynamic; leaves room for static smem
+constexpr int kDW = 16;                         // consumer warps
+constexpr int kDThreads = (kDW + 1) * 32;       // + producer warp
+constexpr int kMaxTk = 16 * MOE_MAX_TOPK;       // T*k entries the token tables hold
+
+struct DecArgs {
+    int T, D, F, E, k, sF;
+    int q8, sq8;                   // routed / shared experts are Q8_0 (else Q4_0)
+    const int32_t *perm, *offsets;
+    const float *gates;            // [T, k] or NULL (rows mode: no gate)
+    const uint8_t *mask;           // [E] or NULL
+    const uint8_t *gate, *up, *down;
+    const int32_t *slot_map;
+    const uint8_t *sh_gate, *sh_up, *sh_down;
+    const void *x;
+    int x_bf16;
+    __half *Hs;                    // [T*k + T][hrow] fragment order
+    int hrow;                      // halves per Hs row
+    void *y;                       // [T, D] (combine mode)
+    int y_dtype;
+    float *rows_out;               // [T*k, D] (rows mode) or NULL
+    int *err;
+};
+
+// slice geometry: blocks per K-slice (<= 32, a multiple of 8)
+__host__ __device__ inline int slice_blocks(int ncols) {
+    int nb = ncols / QK;
+    return nb <= 32 ? nb : 32;
+}
+// Staged weight row: the slice plus padding chosen so that the row stride in
+// 32-bit words is an odd multiple of 4: threads (g = 0..7, c = 0..3) loading
+// word c of row g then touch 32 distinct banks.
+__host__ __device__ inline int staged_row_bytes(int sb, int bs) {
+    const int w = sb * bs / 4;                  // sb * bs is a multiple of 16
+    return sb * bs + ((w % 8 == 0) ? 16 : 32);
+}
+// Shared-memory pitch of a weight row staged by a 2-D TMA copy: the row
+// bytes rounded up to 16 and then to an ODD multiple of 16, so the pitch in
+// 32-bit words is 4 x odd: threads (g = 0..7, c = 0..3) loading word c of
+// row g hit 32 distinct banks.  The extra bytes are out-of-bounds elements
+// of the box, which the copy engine fills with zeros.
+__host__ __device__ inline int tma_row_bytes(int rb) {
+    int r = (rb + 15) / 16 * 16;
+    if (((r / 16) & 1) == 0) r += 16;
+    return r;
+}
+// Blocks per K-slice for a block size: the largest multiple of 8 dividing
+// the row's nb blocks whose staged row still fits one box (<= 256 elements
+// of 8 bytes = 2048 bytes).
+__host__ __device__ inline int slice_blocks_q(int nb, int bs) {
+    for (int sb = nb; sb >= 8; sb -= 8)
+        if (nb % sb == 0 && tma_row_bytes(sb * bs) <= 2048) return sb;
+    return 8;
+}
+
+// The weight pools as 2-D tensors of 8-byte elements (one row of blocks per
+// tensor row), boxes of 16 rows: one TMA request per 16-row tile and slice.
+struct DecMaps {
+    CUtensorMap gate, up, down;        // routed pool
+    CUtensorMap sgate, sup, sdown;     // shared expert
+};
+
+// Staged activation row (fp16 fragment order): stride = 64 mod 128 bytes so
+// that rows n, n+1 read by one quarter-warp's 16-byte loads do not collide.
+__host__ __device__ inline int staged_act_bytes(int ncols) { return ncols * 2 + 64; }
+
+// ---------------------------------------------------------- shared loads
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float ldsf(uint32_t a) { return __uint_as_float(lds32(a)); }
+
+// 32-bit word at a shared address whose alignment mod 4 is MIS (0 or 2),
+// known at compile time.
+template <int MIS>
+__device__ __forceinline__ uint32_t lds_word(uint32_t a) {
+    if constexpr (MIS == 0) {
+        return lds32(a);
+    } else {
+        const uint32_t lo = lds32(a - 2), hi = lds32(a + 2);
+        return __funnelshift_r(lo, hi, 16);
+    }
+}
+
+__device__ __forceinline__ float h2f(uint32_t bits) {
+    return __half2float(__ushort_as_half((unsigned short)bits));
+}
+
+// ------------------------------------------------------------ active list
+struct Active {
+    int n_routed;   // active routed experts
+    int n_virt;     // + 1 when a shared expert exists
+};
+
+__device__ Active build_active_list(const DecArgs &a, int *act) {
+    __shared__ int s_n;
+    if (threadIdx.x < 32) {
+        int base = 0;
+        for (int e0 = 0; e0 < a.E; e0 += 32) {
+            int e = e0 + threadIdx.x;
+            bool on = false;
+            if (e < a.E) {
+                int c = __ldg(a.offsets + e + 1) - __ldg(a.offsets + e);
+                on = c > 0 && (!a.mask || __ldg(a.mask + e));
+            }
+            unsigned b = __ballot_sync(0xffffffffu, on);
+            if (on) act[base + __popc(b & ((1u << threadIdx.x) - 1u))] = e;
+            base += __popc(b);
+        }
+        if (threadIdx.x == 0) s_n = base;
+    }
+    __syncthreads();
+    Active r;
+    r.n_routed = s_n;
+    r.n_virt = s_n + (a.sF > 0 ? 1 : 0);
+    return r;
+}
+
+// Virtual expert v: routed act[v] for v < n_routed, else the shared expert.
+struct Virt {
+    int seg0, cnt, Fv;
+    size_t slot;
+    bool shared;
+    bool q8;
+};
+
+__device__ __forceinline__ Virt virt(const DecArgs &a, const int *act, int n_routed, int v) {
+    Virt r;
+    if (v < n_routed) {
+        int e = act[v];
+        r.seg0 = __ldg(a.offsets + e);
+        r.cnt = __ldg(a.offsets + e + 1) - r.seg0;
+        r.Fv = a.F;
+        r.slot = (size_t)slot_of(a.slot_map, e);
+        r.shared = false;
+        r.q8 = a.q8 != 0;
+    } else {
+        r.seg0 = a.T * a.k;
+        r.cnt = a.T;
+        r.Fv = a.sF;
+        r.slot = 0;
+        r.shared = true;
+        r.q8 = a.sq8 != 0;
+    }
+    return r;
+}
+
+// Token tables in shared memory: tok[pos] = token of permuted entry pos
+// (T*k entries) followed by tok[T*k + t] = t for the shared expert; gw[pos]
+// = gate weight of entry pos.
+__device__ void load_token_tables(const DecArgs &a, int *tok, float *gw) {
+    const int Tk = a.T * a.k;
+    for (int p = threadIdx.x; p < Tk + a.T; p += blockDim.x) {
+        if (p < Tk) {
+            const int n = __ldg(a.perm + p);
+            tok[p] = n / a.k;
+            if (gw) gw[p] = a.gates ? __ldg(a.gates + n) : 1.0f;
+        } else {
+            tok[p] = p - Tk;
+            if (gw) gw[p] = 1.0f;
+        }
+    }
+}
+
+// index (in halves) of row element i (0..31 within its block) in fragment order
+__host__ __device__ __forceinline__ int frag_slot(int i) {
+    const int c = (i & 15) >> 2, j = i & 3, hi = i >> 4;
+    const int jj = (j == 0) ? 0 : (j == 2) ? 1 : (j == 1) ? 2 : 3;
+    return c * 8 + hi * 4 + jj;
+}
+
+// ---------------------------------------------------- code extraction
+// Exact fp16 pairs of (const + code) for the 8 weights of one row that
+// thread c owns in a block: r[0] = (v4c, v4c+2), r[1] = (v4c+1, v4c+3),
+// r[2] = (v16+4c, v18+4c), r[3] = (v17+4c, v19+4c), where
+// v = 1024 + q (Q4_0, 0 <= q < 16) or v = 1152 + q (Q8_0, int8 q).
+// qa: shared address of the block's first code byte + 4c.
+template <bool Q8, int MIS>
+__device__ __forceinline__ void magic_codes(uint32_t qa, uint32_t *r) {
+    if constexpr (!Q8) {
+        const uint32_t w = lds_word<MIS>(qa);
+        const uint32_t M = 0x000F000Fu, MAG = 0x64006400u;
+        r[0] = lop3_and_or(w, M, MAG);
+        r[2] = lop3_and_or(w >> 4, M, MAG);
+        r[1] = lop3_and_or(w >> 8, M, MAG);
+        r[3] = lop3_and_or(w >> 12, M, MAG);
+    } else {
+        const uint32_t w0 = lds_word<MIS>(qa) ^ 0x80808080u;
+        const uint32_t w1 = lds_word<MIS>(qa + 16) ^ 0x80808080u;
+        const uint32_t HI = 0x64646464u;
+        r[0] = prmt(w0, HI, 0x4240);
+        r[1] = prmt(w0, HI, 0x4341);
+        r[2] = prmt(w1, HI, 0x4240);
+        r[3] = prmt(w1, HI, 0x4341);
+    }
+}
+
+// offset of the magic constant in half2 form: 1032 (Q4_0) or 1152 (Q8_0)
+template <bool Q8> __device__ __forceinline__ uint32_t magic_off2() {
+    return Q8 ? 0x64806480u : 0x64086408u;
+}
+template <bool Q8> __host__ __device__ constexpr float magic_off() { return Q8 ? 1152.f : 1032.f; }
+template <bool Q8> __host__ __device__ constexpr int qbytes() { return Q8 ? kQ8Bytes : kQ4Bytes; }
+
+// ---------------------------------------------------------------- gate/up
+// One K-slice of one 16-row tile for one warp: WB blocks starting at the
+// warp's first block.  row: shared address of row g at that block; xa: the B
+// row of column g (and g+8) at that block; sa: the -off*sum(x) entries of
+// columns 2c, 2c+1 (and +8) at that block.  MIS0 = alignment mod 4 of the
+// first block's start (the code bytes start 2 bytes later; BS is 2 mod 4).
+template <bool Q8, int NTILE, int WB, int MIS0>
+__device__ __forceinline__ void gateup_slice(uint32_t row, uint32_t r8, const uint32_t *xa,
+                                             const uint32_t (*sa)[2], int c, float (*acc)[4]) {
+    constexpr int BS = qbytes<Q8>();
+#pragma unroll
+    for (int bl = 0; bl < WB; bl++) {
+        const uint32_t blk = row + bl * BS;
+        uint32_t lo[4], hi[4];
+        if (((MIS0 + 2 * bl + 2) & 3) == 0) {
+            magic_codes<Q8, 0>(blk + 2 + 4 * c, lo);
+            magic_codes<Q8, 0>(blk + r8 + 2 + 4 * c, hi);
+        } else {
+            magic_codes<Q8, 2>(blk + 2 + 4 * c, lo);
+            magic_codes<Q8, 2>(blk + r8 + 2 + 4 * c, hi);
+        }
+        const float dlo = h2f(lds16(blk)), dhi = h2f(lds16(blk + r8));
+        const uint32_t a0[4] = {lo[0], hi[0], lo[1], hi[1]};
+        const uint32_t a1[4] = {lo[2], hi[2], lo[3], hi[3]};
+#pragma unroll
+        for (int nt = 0; nt < NTILE; nt++) {
+            const uint4 b = lds128(xa[nt] + bl * 64);
+            const float s0 = ldsf(sa[nt][0] + bl * 4), s1 = ldsf(sa[nt][1] + bl * 4);
+            float p[4] = {s0, s1, s0, s1};
+            mma_16816(p, a0, b.x, b.y, p);
+            mma_16816(p, a1, b.z, b.w, p);
+            acc[nt][0] = fmaf(dlo, p[0], acc[nt][0]);
+            acc[nt][1] = fmaf(dlo, p[1], acc[nt][1]);
+            acc[nt][2] = fmaf(dhi, p[2], acc[nt][2]);
+            acc[nt][3] = fmaf(dhi, p[3], acc[nt][3]);
+        }
+    }
+}
+
+// K1 geometry of one quant type at a given D
+struct GuGeo {
+    int sb, nsl, pitch;                 // blocks per slice, slices, staged row pitch
+};
+__host__ __device__ inline GuGeo gu_geo(int D, bool q8) {
+    const int bs = q8 ? kQ8Bytes : kQ4Bytes, nb = D / QK;
+    GuGeo g;
+    g.sb = slice_blocks_q(nb, bs);
+    g.nsl = nb / g.sb;
+    g.pitch = tma_row_bytes(g.sb * bs);
+    return g;
+}
+
+template <int NT, int WB4, int WB8>
+__global__ void __launch_bounds__(kDThreads, 1)
+dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int T = a.T, D = a.D;
+    const int nbD = D / QK;
+    const GuGeo geo4 = gu_geo(D, false), geo8 = gu_geo(D, true);
+    const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
+    const int pitch_max = max(any4 ? geo4.pitch : 0, any8 ? geo8.pitch : 0);
+    const int stage_bytes = (int)round_up((size_t)2 * kTile * pitch_max, 128);
+    const int xrow = staged_act_bytes(D);
+    const int mat = warp >> 3, kg = warp & 7;
+
+    // carve (from a 1024-aligned base; tensor copies need 128-byte aligned
+    // destinations): xs [T+1 rows, the last zero] | Sx tables [2][T+1][nbD]
+    // | stages | red [2][kDW][NT][32][4] | barriers | act | tok | gw
+    uint8_t *base = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
+    const size_t xs_bytes = round_up((size_t)(T + 1) * xrow, 16);
+    uint8_t *xs = base;
+    float *sxt = (float *)(base + xs_bytes);
+    uint8_t *stages = base + round_up(xs_bytes + (size_t)2 * (T + 1) * nbD * 4, 1024);
+    float *red = (float *)(stages + (size_t)S * stage_bytes);
+    uint64_t *full = (uint64_t *)(red + 2 * kDW * NT * 32 * 4);
+    uint64_t *empty = full + kMaxStages;
+    int *act = (int *)(empty + kMaxStages);
+    int *tok = act + a.E + 1;
+    float *gw = (float *)(tok + kMaxTk + 16);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kDW);
+        }
+        fence_mbar_init();
+    }
+    // routing results come from the previous kernel
+    pdl_wait();
+    pdl_launch_dependents();
+    const Active A = build_active_list(a, act);   // includes __syncthreads
+    const int tiles_r = a.F / kTile, tiles_s = a.sF / kTile;
+    const int U = A.n_routed * tiles_r + (a.sF > 0 ? tiles_s : 0);
+
+    if (warp == kDW) {
+        // ---------------------------------------------------- producer
+        // per (unit, slice): one 16-row box of gate and one of up
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+                int v, tile;
+                if (u < A.n_routed * tiles_r) { v = u / tiles_r; tile = u % tiles_r; }
+                else { v = A.n_routed; tile = u - A.n_routed * tiles_r; }
+                const Virt vi = virt(a, act, A.n_routed, v);
+                const int bs = vi.q8 ? kQ8Bytes : kQ4Bytes;
+                const GuGeo gg = vi.q8 ? geo8 : geo4;
+                const CUtensorMap *mg = vi.shared ? &maps.sgate : &maps.gate;
+                const CUtensorMap *mu = vi.shared ? &maps.sup : &maps.up;
+                const int y = (vi.shared ? 0 : (int)vi.slot * a.F) + tile * kTile;
+                for (int sl = 0; sl < gg.nsl; sl++) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                    uint8_t *dst = stages + (size_t)stage * stage_bytes;
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * kTile * gg.pitch));
+                    const int x = sl * gg.sb * bs / 8;
+                    tma_load_2d(dst, mg, x, y, &full[stage]);
+                    tma_load_2d(dst + kTile * gg.pitch, mu, x, y, &full[stage]);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+            // drain: every issued stage must have landed before the CTA exits
+            for (int s2 = 0; s2 < S; s2++) {
+                mbar_wait(&empty[stage], phase ^ 1, a.err, kErrTimeoutDrain);
+                if (++stage == S) { stage = 0; phase ^= 1; }
+            }
+        }
+        return;
+    }
+
+    // ------------------------------------------------------- consumers
+    load_token_tables(a, tok, gw);
+    // stage the activations once, fp16 in fragment order; row T is zero
+    for (int idx = tid; idx < (T + 1) * (nbD * 4); idx += kDW * 32) {
+        const int t = idx / (nbD * 4), rem = idx % (nbD * 4), b = rem >> 2, cc = rem & 3;
+        uint4 pk = make_uint4(0u, 0u, 0u, 0u);
+        if (t < T) {
+            const size_t base = (size_t)t * D + b * QK;
+            const int src[8] = {4 * cc, 4 * cc + 2, 4 * cc + 1, 4 * cc + 3,
+                                16 + 4 * cc, 18 + 4 * cc, 17 + 4 * cc, 19 + 4 * cc};
+            uint32_t h[8];
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                const float v = a.x_bf16 ? load_act((const __nv_bfloat16 *)a.x, base + src[q])
+                                         : load_act((const float *)a.x, base + src[q]);
+                h[q] = (uint32_t)__half_as_ushort(__float2half_rn(v));
+            }
+            pk.x = h[0] | (h[1] << 16);
+            pk.y = h[2] | (h[3] << 16);
+            pk.z = h[4] | (h[5] << 16);
+            pk.w = h[6] | (h[7] << 16);
+        }
+        *reinterpret_cast<uint4 *>(xs + (size_t)t * xrow + b * 64 + cc * 16) = pk;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
+    // -off * (sum of the 32 fp16 activations of each block), for both codes
+    for (int idx = tid; idx < (T + 1) * nbD; idx += kDW * 32) {
+        const int t = idx / nbD, b = idx % nbD;
+        const __half *hp = reinterpret_cast<const __half *>(xs + (size_t)t * xrow + b * 64);
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i++) s += __half2float(hp[i]);
+        sxt[idx] = -magic_off<false>() * s;
+        sxt[(size_t)(T + 1) * nbD + idx] = -magic_off<true>() * s;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
+
+    const uint32_t xs_a = smem_u32(xs), sx_a = smem_u32(sxt), st_a = smem_u32(stages);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    int ub = 0;                                          // unit counter (red buffer parity)
+    for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ub ^= 1) {
+        int v, tile;
+        if (u < A.n_routed * tiles_r) { v = u / tiles_r; tile = u % tiles_r; }
+        else { v = A.n_routed; tile = u - A.n_routed * tiles_r; }
+        const Virt vi = virt(a, act, A.n_routed, v);
+        const int ntile = vi.cnt > 8 ? 2 : 1;
+        const GuGeo gg = vi.q8 ? geo8 : geo4;
+        const int kb0 = kg * (vi.q8 ? WB8 : WB4);       // warp's first block in a slice
+        // B rows (column g, g+8) and C columns (2c, 2c+1, +8) of this unit
+        uint32_t xa[NT], sa[NT][2];
+        const uint32_t sxq = sx_a + (vi.q8 ? (uint32_t)((T + 1) * nbD * 4) : 0u);
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+            const int n = g + 8 * nt;
+            const int tb = n < vi.cnt ? tok[vi.seg0 + n] : T;
+            xa[nt] = xs_a + tb * xrow + kb0 * 64 + c * 16;
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+                const int m = 8 * nt + 2 * c + j;
+                const int tc = m < vi.cnt ? tok[vi.seg0 + m] : T;
+                sa[nt][j] = sxq + (uint32_t)((tc * nbD + kb0) * 4);
+            }
+        }
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
+        const int bsz = vi.q8 ? kQ8Bytes : kQ4Bytes;
+        const int mis0 = (kb0 * bsz) & 3;               // 0 or 2
+        const uint32_t r8 = 8u * gg.pitch;
+
+        for (int sl = 0; sl < gg.nsl; sl++) {
+            if (!mbar_wait(&full[stage], phase, a.err, kErrTimeoutFull)) { ok = false; break; }
+            const uint32_t row = st_a + stage * stage_bytes + (mat * kTile + g) * gg.pitch + kb0 * bsz;
+            uint32_t xs_s[NT], sa_s[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; nt++) {
+                xs_s[nt] = xa[nt] + sl * gg.sb * 64;
+                sa_s[nt][0] = sa[nt][0] + sl * gg.sb * 4;
+                sa_s[nt][1] = sa[nt][1] + sl * gg.sb * 4;
+            }
+#define MOE_GU(Q8, NTL, MIS) gateup_slice<Q8, NTL, (Q8 ? WB8 : WB4), MIS>(row, r8, xs_s, sa_s, c, acc)
+            if (!vi.q8) {
+                if (ntile == 1) { if (mis0 == 0) MOE_GU(false, 1, 0); else MOE_GU(false, 1, 2); }
+                else if (NT > 1) { if (mis0 == 0) MOE_GU(false, NT, 0); else MOE_GU(false, NT, 2); }
+            } else {
+                if (ntile == 1) { if (mis0 == 0) MOE_GU(true, 1, 0); else MOE_GU(true, 1, 2); }
+                else if (NT > 1) { if (mis0 == 0) MOE_GU(true, NT, 0); else MOE_GU(true, NT, 2); }
+            }
+#undef MOE_GU
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        // cross-warp reduction (double-buffered partials, one barrier per
+        // unit) in a fixed order, SwiGLU, gate weight, fp16 store
+        float *redb = red + (size_t)ub * kDW * NT * 128;
+        float *rw = redb + (size_t)warp * NT * 128;
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) rw[nt * 128 + lane * 4 + q] = acc[nt][q];
+        asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
+        for (int o = tid; o < kTile * 8 * ntile; o += kDW * 32) {
+            const int rr = o % kTile, n = o / kTile;        // row within tile, column
+            if (n < vi.cnt) {
+                const int nt = n >> 3, nn = n & 7;
+                const int L = (rr & 7) * 4 + (nn >> 1);
+                const int q = ((rr >> 3) << 1) | (nn & 1);
+                float sg = 0.f, su = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; w++) {
+                    sg += redb[((size_t)w * NT + nt) * 128 + L * 4 + q];
+                    su += redb[((size_t)(8 + w) * NT + nt) * 128 + L * 4 + q];
+                }
+                const int pos = vi.seg0 + n;
+                const float h = silu(sg) * su * gw[pos];
+                const int r = tile * kTile + rr;
+                a.Hs[(size_t)pos * a.hrow + (r >> 5) * 32 + frag_slot(r & 31)] = __float2half_rn(h);
+            }
+        }
+    }
+}
+
+// --------------------------------------------------------------------- down
+// One expert's 16-row tile for one warp: WB blocks from the warp's first
+// block; codes become exact (q - off) fp16 values and the block scale
+// multiplies the fp32 MMA result.  ha: B row of column g (and g+8).
+template <bool Q8, int NTILE, int WB, int MIS0>
+__device__ __forceinline__ void down_expert(uint32_t row, uint32_t r8, const uint32_t *ha, int c,
+                                            float (*acc)[4]) {
+    constexpr int BS = qbytes<Q8>();
+    const uint32_t off2 = magic_off2<Q8>();
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int bl = 0; bl < WB; bl++) {
+        const uint32_t blk = row + bl * BS;
+        uint32_t lo[4], hi[4];
+        if (((MIS0 + 2 * bl + 2) & 3) == 0) {
+            magic_codes<Q8, 0>(blk + 2 + 4 * c, lo);
+            magic_codes<Q8, 0>(blk + r8 + 2 + 4 * c, hi);
+        } else {
+            magic_codes<Q8, 2>(blk + 2 + 4 * c, lo);
+            magic_codes<Q8, 2>(blk + r8 + 2 + 4 * c, hi);
+        }
+        const float dlo = h2f(lds16(blk)), dhi = h2f(lds16(blk + r8));
+        const uint32_t a0[4] = {hsub2_u(lo[0], off2), hsub2_u(hi[0], off2), hsub2_u(lo[1], off2),
+                                hsub2_u(hi[1], off2)};
+        const uint32_t a1[4] = {hsub2_u(lo[2], off2), hsub2_u(hi[2], off2), hsub2_u(lo[3], off2),
+                                hsub2_u(hi[3], off2)};
+#pragma unroll
+        for (int nt = 0; nt < NTILE; nt++) {
+            const uint4 b = lds128(ha[nt] + bl * 64);
+            float p[4];
+            mma_16816(p, a0, b.x, b.y, zero);
+            mma_16816(p, a1, b.z, b.w, p);
+            acc[nt][0] = fmaf(dlo, p[0], acc[nt][0]);
+            acc[nt][1] = fmaf(dlo, p[1], acc[nt][1]);
+            acc[nt][2] = fmaf(dhi, p[2], acc[nt][2]);
+            acc[nt][3] = fmaf(dhi, p[3], acc[nt][3]);
+        }
+    }
+}
+
+// Requires F, shared F <= 1024 (one K-slice per expert).
+template <int NT, int WB, bool ROWS>
+__global__ void __launch_bounds__(kDThreads, 1)
+dec_down_kernel(DecArgs a, int S, int hrows, const __grid_constant__ DecMaps maps) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int T = a.T, D = a.D;
+    const int Fmax = a.F > a.sF ? a.F : a.sF;
+    const int hstride = staged_act_bytes(Fmax);
+    const int pr = tma_row_bytes((a.F / QK) * (a.q8 ? kQ8Bytes : kQ4Bytes));
+    const int ps = a.sF > 0 ? tma_row_bytes((a.sF / QK) * (a.sq8 ? kQ8Bytes : kQ4Bytes)) : 0;
+    const int wbytes = kTile * (pr > ps ? pr : ps);
+    const int stage_bytes = (int)round_up((size_t)wbytes + (size_t)hrows * hstride, 128);
+    const int ncols = ROWS ? 16 : T;                   // accumulator columns per warp
+    const int par = warp >> 3, kg = warp & 7;
+
+    // carve (from a 1024-aligned base; tensor copies need 128-byte aligned
+    // destinations): stages | zero row | yacc [kDW][ncols][16] | barriers |
+    // act | tok
+    uint8_t *stages = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
+    uint8_t *zrow = stages + (size_t)S * stage_bytes;
+    float *yacc = (float *)(zrow + round_up((size_t)hstride, 16));
+    uint64_t *full = (uint64_t *)(yacc + kDW * ncols * kTile);
+    uint64_t *empty = full + kMaxStages;
+    int *act = (int *)(empty + kMaxStages);
+    int *tok = act + a.E + 1;
+
+    if (tid == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 8);             // the 8 warps of one parity group
+        }
+        fence_mbar_init();
+    }
+    for (int i = tid; i < kDW * ncols * kTile; i += blockDim.x) yacc[i] = 0.f;
+    for (int i = tid; i < hstride / 4; i += blockDim.x) reinterpret_cast<uint32_t *>(zrow)[i] = 0u;
+    // routing (perm/offsets) is complete: the gate/up kernel waited for it
+    // before letting this grid launch
+    load_token_tables(a, tok, nullptr);
+    const Active A = build_active_list(a, act);
+    const int U = D / kTile;
+    const int NV = A.n_virt;
+
+    if (warp == kDW) {
+        if (lane == 0) {
+            bool ok = true, waited = false;
+            int pending[kMaxStages], pend_v[kMaxStages];
+            int npend = 0;
+            auto issue_h = [&](int st, int v) {
+                const Virt vi = virt(a, act, A.n_routed, v);
+                uint8_t *dst = stages + (size_t)st * stage_bytes + wbytes;
+                for (int n = 0; n < vi.cnt; n++)
+                    bulk_g2s(dst + n * hstride, a.Hs + (size_t)(vi.seg0 + n) * a.hrow,
+                             (uint32_t)(vi.Fv * 2), &full[st]);
+            };
+            long long i = 0;                    // issue index
+            for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+                for (int v = 0; v < NV && ok; v++, i++) {
+                    const int stage = (int)(i % S);
+                    const uint32_t ph = (uint32_t)((i / S) & 1);
+                    const Virt vi = virt(a, act, A.n_routed, v);
+                    const int pitch = vi.shared ? ps : pr;
+                    if (!mbar_wait(&empty[stage], ph ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                    uint8_t *dst = stages + (size_t)stage * stage_bytes;
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(kTile * pitch + vi.cnt * vi.Fv * 2));
+                    tma_load_2d(dst, vi.shared ? &maps.sdown : &maps.down, 0,
+                                (vi.shared ? 0 : (int)vi.slot * a.D) + u * kTile, &full[stage]);
+                    if (waited) {
+                        issue_h(stage, v);
+                    } else {
+                        pending[npend] = stage; pend_v[npend] = v; npend++;
+                        if (npend == S) {
+                            // every stage holds prefetched weights: now wait for Hs
+                            pdl_wait();
+                            waited = true;
+                            for (int q = 0; q < npend; q++) issue_h(pending[q], pend_v[q]);
+                            npend = 0;
+                        }
+                    }
+                }
+            }
+            if (!waited) {
+                pdl_wait();
+                for (int q = 0; q < npend; q++) issue_h(pending[q], pend_v[q]);
+            }
+            // drain
+            for (int q = 0; q < S; q++, i++) {
+                const int stage = (int)(i % S);
+                mbar_wait(&empty[stage], (uint32_t)(((i / S) & 1) ^ 1), a.err, kErrTimeoutDrain);
+            }
+        }
+        return;
+    }
+
+    // ------------------------------------------------------- consumers
+    bool ok = true;
+    float *yw = yacc + (size_t)warp * ncols * kTile;
+    const uint32_t st_a = smem_u32(stages), z_a = smem_u32(zrow);
+    long long ibase = 0;
+    for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ibase += NV) {
+        for (int v = par; v < NV && ok; v += 2) {
+            const long long i = ibase + v;
+            const int stage = (int)(i % S);
+            const uint32_t ph = (uint32_t)((i / S) & 1);
+            const Virt vi = virt(a, act, A.n_routed, v);
+            const int bsz = vi.q8 ? kQ8Bytes : kQ4Bytes;
+            const int rstride = vi.shared ? ps : pr;
+            const int wb = (vi.Fv / QK) / 8;           // blocks per K-group (<= WB)
+            const int kbw = kg * wb;
+            const int ntile = vi.cnt > 8 ? 2 : 1;
+            float acc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+                for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
+            if (!mbar_wait(&full[stage], ph, a.err, kErrTimeoutFull)) { ok = false; break; }
+            const uint32_t sbase = st_a + stage * stage_bytes;
+            const uint32_t row = sbase + g * rstride + kbw * bsz;
+            uint32_t ha[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; nt++) {
+                const int n = g + 8 * nt;
+                ha[nt] = (n < vi.cnt ? sbase + wbytes + n * hstride : z_a) + kbw * 64 + c * 16;
+            }
+            const int mis0 = (kbw * bsz) & 3;
+            const uint32_t r8 = 8u * rstride;
+#define MOE_DN(Q8, NTL, W, MIS) down_expert<Q8, NTL, W, MIS>(row, r8, ha, c, acc)
+#define MOE_DN_W(Q8, NTL, MIS)                                              \
+    do {                                                                    \
+        if (wb == 3) MOE_DN(Q8, NTL, 3, MIS);                               \
+        else if (wb == 2) MOE_DN(Q8, NTL, 2, MIS);                          \
+        else if (wb == 1) MOE_DN(Q8, NTL, 1, MIS);                          \
+        else MOE_DN(Q8, NTL, 4, MIS);                                       \
+    } while (0)
+            if (!vi.q8) {
+                if (ntile == 1) { if (mis0 == 0) MOE_DN_W(false, 1, 0); else MOE_DN_W(false, 1, 2); }
+                else if (NT > 1) { if (mis0 == 0) MOE_DN_W(false, NT, 0); else MOE_DN_W(false, NT, 2); }
+            } else {
+                if (ntile == 1) { if (mis0 == 0) MOE_DN_W(true, 1, 0); else MOE_DN_W(true, 1, 2); }
+                else if (NT > 1) { if (mis0 == 0) MOE_DN_W(true, NT, 0); else MOE_DN_W(true, NT, 2); }
+            }
+#undef MOE_DN_W
+#undef MOE_DN
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            // C fragment: rows g / g+8 of the d-tile, columns 2c, 2c+1 (+8 nt)
+#pragma unroll
+            for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const int n = nt * 8 + 2 * c + (q & 1);
+                    const int r = g + ((q >> 1) << 3);
+                    if (n < vi.cnt) {
+                        const int col = ROWS ? n : tok[vi.seg0 + n];
+                        yw[col * kTile + r] += acc[nt][q];
+                    }
+                }
+            if (ROWS) {
+                // flush this expert's rows: fixed-order sum over the group's warps
+                const int bid = 2 + par;
+                asm volatile("bar.sync %0, %1;" ::"r"(bid), "n"(8 * 32));
+                const int gt = tid - par * 256;
+                for (int o = gt; o < vi.cnt * kTile; o += 256) {
+                    const int n = o / kTile, r = o % kTile;
+                    float s = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 8; w++) s += yacc[((size_t)(par * 8 + w) * ncols + n) * kTile + r];
+                    a.rows_out[(size_t)(vi.seg0 + n) * D + u * kTile + r] = s;
+                }
+                asm volatile("bar.sync %0, %1;" ::"r"(bid), "n"(8 * 32));
+                for (int o = gt; o < 8 * ncols * kTile; o += 256) yacc[(size_t)par * 8 * ncols * kTile + o] = 0.f;
+                asm volatile("bar.sync %0, %1;" ::"r"(bid), "n"(8 * 32));
+            }
+        }
+        if (!ok) break;
+        if (!ROWS) {
+            asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
+            for (int o = tid; o < T * kTile; o += kDW * 32) {
+                const int t = o / kTile, r = o % kTile;
+                float s = 0.f;
+#pragma unroll
+                for (int w = 0; w < kDW; w++) s += yacc[((size_t)w * ncols + t) * kTile + r];
+                const size_t yi = (size_t)t * D + u * kTile + r;
+                if (a.y_dtype == MOE_BF16) ((__nv_bfloat16 *)a.y)[yi] = __float2bfloat16_rn(s);
+                else ((float *)a.y)[yi] = s;
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
+            for (int o = tid; o < kDW * ncols * kTile; o += kDW * 32) yacc[o] = 0.f;
+            asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
+        }
+    }
+}
+
+// ------------------------------------------------------------------- host
+// D: a multiple of 256 with a compiled slice geometry; F, shared F:
+// multiples of 256 up to 1024 (one box per expert tile in the down kernel).
+static bool gu_shape_ok(int D) { return D == 256 || D == 512 || D == 768 || D == 1024 || D == 2048; }
+
+bool decode_path_ok(int T, int D, int F, int sF) {
+    return T >= 1 && T <= 16 && gu_shape_ok(D) && F % 256 == 0 && F <= 1024 &&
+           (sF == 0 || (sF % 256 == 0 && sF <= 1024));
+}
+
+size_t decode_hs_halves(int T, int k, int F, int sF) {
+    return (size_t)(T * k + T) * (size_t)std::max(F, sF);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// rows x row_bytes (8-byte elements) at base; boxes of box_rows rows and
+// box_bytes (>= the slice, the excess zero-filled out of bounds)
+static moe_status encode_rows(CUtensorMap *m, const void *base, size_t row_bytes, size_t nrows,
+                              int box_bytes, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) { set_error("decode path: cuTensorMapEncodeTiled unavailable"); return MOE_ERR_CUDA; }
+    const cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / 8), (cuuint64_t)nrows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(box_bytes / 8), (cuuint32_t)box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("decode path: tensor map encoding failed (%d) for %zu x %zu bytes", (int)r, nrows,
+                  row_bytes);
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+static moe_status encode_maps(const DecArgs &a, int n_slots, DecMaps *m) {
+    memset(m, 0, sizeof(*m));
+    const int nbD = a.D / QK;
+    const int br = a.q8 ? kQ8Bytes : kQ4Bytes;
+    const GuGeo gr = gu_geo(a.D, a.q8);
+    moe_status st;
+    if ((st = encode_rows(&m->gate, a.gate, (size_t)nbD * br, (size_t)n_slots * a.F, gr.pitch, kTile)))
+        return st;
+    if ((st = encode_rows(&m->up, a.up, (size_t)nbD * br, (size_t)n_slots * a.F, gr.pitch, kTile)))
+        return st;
+    const size_t rbd = (size_t)(a.F / QK) * br;
+    if ((st = encode_rows(&m->down, a.down, rbd, (size_t)n_slots * a.D, tma_row_bytes((int)rbd), kTile)))
+        return st;
+    if (a.sF > 0) {
+        const int bsh = a.sq8 ? kQ8Bytes : kQ4Bytes;
+        const GuGeo gs = gu_geo(a.D, a.sq8);
+        if ((st = encode_rows(&m->sgate, a.sh_gate, (size_t)nbD * bsh, a.sF, gs.pitch, kTile))) return st;
+        if ((st = encode_rows(&m->sup, a.sh_up, (size_t)nbD * bsh, a.sF, gs.pitch, kTile))) return st;
+        const size_t rbs = (size_t)(a.sF / QK) * bsh;
+        if ((st = encode_rows(&m->sdown, a.sh_down, rbs, a.D, tma_row_bytes((int)rbs), kTile))) return st;
+    }
+    return MOE_OK;
+}
+
+template <typename... Args>
+static cudaError_t launch_pdl(void (*kern)(Args...), int grid, size_t smem, cudaStream_t s,
+                             Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kDThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+static size_t tables_bytes(int E) {
+    return (size_t)(E + 1) * sizeof(int) + (size_t)(kMaxTk + 16) * (sizeof(int) + sizeof(float));
+}
+
+template <int NT>
+static cudaError_t launch_gateup(const DecArgs &a, const DecMaps &m, int grid, size_t smem,
+                                 cudaStream_t s, int S) {
+    switch (a.D) {
+    case 256: return launch_pdl(dec_gateup_kernel<NT, 1, 1>, grid, smem, s, a, S, m);
+    case 512: return launch_pdl(dec_gateup_kernel<NT, 2, 2>, grid, smem, s, a, S, m);
+    case 768: return launch_pdl(dec_gateup_kernel<NT, 3, 3>, grid, smem, s, a, S, m);
+    case 1024: return launch_pdl(dec_gateup_kernel<NT, 4, 4>, grid, smem, s, a, S, m);
+    default: return launch_pdl(dec_gateup_kernel<NT, 8, 4>, grid, smem, s, a, S, m);
+    }
+}
+
+template <int NT>
+static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Tracer *tr) {
+    const int sms = num_sms();
+    DecMaps maps;
+    moe_status st = encode_maps(a, n_slots, &maps);
+    if (st != MOE_OK) return st;
+    const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
+    // ---- gate/up
+    {
+        const int nbD = a.D / QK;
+        const int pitch = std::max(any4 ? gu_geo(a.D, false).pitch : 0, any8 ? gu_geo(a.D, true).pitch : 0);
+        const int stage_bytes = (int)round_up((size_t)2 * kTile * pitch, 128);
+        // mirrors the kernel's carve; + 1024 for aligning the base
+        const size_t fixed = round_up(round_up((size_t)(a.T + 1) * staged_act_bytes(a.D), 16) +
+                                      (size_t)2 * (a.T + 1) * nbD * 4, 1024) +
+                             (size_t)2 * kDW * NT * 32 * 4 * sizeof(float) +
+                             2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
+        if (fixed >= kDecSmemMax) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
+        int S = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - fixed) / stage_bytes);
+        if (S < 2) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
+        const size_t smem = fixed + (size_t)S * stage_bytes;
+        const int U_max = a.E * (a.F / kTile) + a.sF / kTile;
+        const int grid = std::max(1, std::min(sms, U_max));
+        mark(tr, MOE_KERNEL_FFN_DECODE);
+        cudaError_t e = launch_gateup<NT>(a, maps, grid, smem, s, S);
+        if (e != cudaSuccess) return cuda_status(e, "dec_gateup_kernel");
+    }
+    // ---- down (+ combine)
+    {
+        const int Fmax = std::max(a.F, a.sF);
+        const int hrows = std::min(a.T, 16);
+        const int pr = tma_row_bytes((a.F / QK) * (a.q8 ? kQ8Bytes : kQ4Bytes));
+        const int ps = a.sF > 0 ? tma_row_bytes((a.sF / QK) * (a.sq8 ? kQ8Bytes : kQ4Bytes)) : 0;
+        const size_t wbytes = (size_t)kTile * std::max(pr, ps);
+        const int stage_bytes = (int)round_up(wbytes + (size_t)hrows * staged_act_bytes(Fmax), 128);
+        const int ncols = a.rows_out ? 16 : a.T;
+        const size_t fixed = round_up((size_t)staged_act_bytes(Fmax), 16) +
+                             (size_t)kDW * ncols * kTile * sizeof(float) +
+                             2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
+        if (fixed >= kDecSmemMax) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
+        int S = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - fixed) / stage_bytes);
+        if (S < 2) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
+        const size_t smem = fixed + (size_t)S * stage_bytes;
+        const int grid = std::max(1, std::min(sms, a.D / kTile));
+        // no trace mark here: an event between the two kernels would cancel
+        // their programmatic overlap
+        cudaError_t e = a.rows_out
+            ? launch_pdl(dec_down_kernel<NT, 4, true>, grid, smem, s, a, S, hrows, maps)
+            : launch_pdl(dec_down_kernel<NT, 4, false>, grid, smem, s, a, S, hrows, maps);
+        if (e != cudaSuccess) return cuda_status(e, "dec_down_kernel");
+    }
+    return MOE_OK;
+}
+
+moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, int E, int k,
+                             const int32_t *perm, const int32_t *offsets, const float *gates,
+                             const moe_pool &pool, const uint8_t *mask, const moe_pool *shared,
+                             int sF, __half *Hs, void *y, int y_dtype, float *rows_out, int *err,
+                             cudaStream_t s, Tracer *tr) {
+    DecArgs a{};
+    a.T = T; a.D = D; a.F = F; a.E = E; a.k = k; a.sF = shared ? sF : 0;
+    a.perm = perm; a.offsets = offsets; a.gates = gates; a.mask = mask;
+    a.gate = (const uint8_t *)pool.gate; a.up = (const uint8_t *)pool.up;
+    a.down = (const uint8_t *)pool.down; a.slot_map = pool.slot_of_expert;
+    if (pool.qtype != MOE_Q4_0 && pool.qtype != MOE_Q8_0) {
+        set_error("decode path: unsupported quant type %d", (int)pool.qtype);
+        return MOE_ERR_UNSUPPORTED_QTYPE;
+    }
+    if (T * k > kMaxTk) {
+        set_error("decode path: T*k=%d exceeds %d", T * k, kMaxTk);
+        return MOE_ERR_SHAPE;
+    }
+    a.q8 = pool.qtype == MOE_Q8_0;
+    if (shared) {
+        a.sh_gate = (const uint8_t *)shared->gate; a.sh_up = (const uint8_t *)shared->up;
+        a.sh_down = (const uint8_t *)shared->down;
+        if (shared->qtype != MOE_Q4_0 && shared->qtype != MOE_Q8_0) {
+            set_error("decode path: unsupported shared-expert quant type %d", (int)shared->qtype);
+            return MOE_ERR_UNSUPPORTED_QTYPE;
+        }
+        a.sq8 = shared->qtype == MOE_Q8_0;
+    }
+    a.x = x; a.x_bf16 = (x_dtype == MOE_BF16);
+    a.Hs = Hs; a.hrow = std::max(F, a.sF);
+    a.y = y; a.y_dtype = y_dtype; a.rows_out = rows_out; a.err = err;
+    return T > 8 ? run_decode<2>(a, pool.n_slots, s, tr) : run_decode<1>(a, pool.n_slots, s, tr);
+}
+
+}  // namespace moe

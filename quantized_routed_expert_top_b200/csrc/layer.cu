@@ -7,6 +7,7 @@
 namespace moe {
 
 struct LayerWs {
+    int *status;         // device status words (first bytes of the workspace)
     void *route_ws;
     size_t route_bytes;
     int32_t *ids;
@@ -16,11 +17,13 @@ struct LayerWs {
     float *rows;         // [T*k, D] fp32
     float *shH;          // [T, shared_F]
     float *sh_rows;      // [T, D]
+    __half *Hs;          // decode path: g*h in fp16 fragment order
 };
 
 static LayerWs carve(const moe_layer_args &a, Carver &c) {
     LayerWs w{};
     const size_t Tk = (size_t)a.T * a.k;
+    w.status = c.take<int>(16);
     w.route_bytes = route_ws_bytes(a.T, a.w_router ? a.D : QK, a.E, a.k);
     w.route_ws = c.take<char>(w.route_bytes);
     w.ids = c.take<int32_t>(Tk);
@@ -29,6 +32,10 @@ static LayerWs carve(const moe_layer_args &a, Carver &c) {
     w.offsets = c.take<int32_t>(a.E + 1);
     w.perm = c.take<int32_t>(Tk);
     w.inv = c.take<int32_t>(Tk);
+    if (decode_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0)) {
+        w.Hs = c.take<__half>(decode_hs_halves(a.T, a.k, a.F, a.shared ? a.shared_F : 0));
+        return w;
+    }
     w.H = c.take<float>(Tk * a.F);
     w.rows = c.take<float>(Tk * a.D);
     if (a.shared) {
@@ -62,15 +69,32 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
     int32_t *ids = a.ids_out ? a.ids_out : w.ids;
     float *gates = a.gates_out ? a.gates_out : w.gates;
     moe_status st;
+    bool permuted = false;
     if (a.w_router)
-        st = launch_route(a.x, a.x_dtype, a.w_router, a.bias, a.T, a.D, a.E, a.k, a.renorm, ids,
-                          gates, a.logits_out, w.route_ws, w.route_bytes, s, tr);
+        st = launch_route_permute(a.x, a.x_dtype, a.w_router, a.bias, a.T, a.D, a.E, a.k, a.renorm,
+                                  ids, gates, a.logits_out, w.counts, w.offsets, w.perm, w.inv,
+                                  w.status, w.route_ws, w.route_bytes, s, tr, &permuted);
     else
-        st = launch_route(a.logits_in, MOE_F32, nullptr, a.bias, a.T, QK, a.E, a.k, a.renorm, ids,
-                          gates, a.logits_out, w.route_ws, w.route_bytes, s, tr);
+        st = launch_route_permute(a.logits_in, MOE_F32, nullptr, a.bias, a.T, QK, a.E, a.k,
+                                  a.renorm, ids, gates, a.logits_out, w.counts, w.offsets, w.perm,
+                                  w.inv, w.status, w.route_ws, w.route_bytes, s, tr, &permuted);
     if (st != MOE_OK) return st;
-    if ((st = launch_permute(ids, a.T, a.k, a.E, w.counts, w.offsets, w.perm, w.inv, s, tr)) != MOE_OK)
+    if (!permuted &&
+        (st = launch_permute(ids, a.T, a.k, a.E, w.counts, w.offsets, w.perm, w.inv, s, tr)) != MOE_OK)
         return st;
+    if (w.Hs) {
+        st = launch_ffn_decode(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.offsets, gates,
+                               *a.pool, nullptr, a.shared, a.shared ? a.shared_F : 0, w.Hs, a.y,
+                               a.y_dtype, nullptr, w.status, s, tr);
+        if (tr) {
+            tr->end();
+            if (st == MOE_OK && tr->err != cudaSuccess) {
+                cudaGetLastError();
+                return cuda_status(tr->err, "moe_layer_forward: trace event record");
+            }
+        }
+        return st;
+    }
     if ((st = launch_ffn_generic(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.offsets,
                                  *a.pool, nullptr, w.H, w.rows, s, tr)) != MOE_OK)
         return st;

@@ -39,7 +39,7 @@ struct Carver {
     bool fits() const { return off <= cap; }
 };
 
-inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+__host__ __device__ inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
 // Records the caller's events around each kernel of a call (moe_trace).
 struct Tracer {
@@ -47,10 +47,19 @@ struct Tracer {
     cudaStream_t s = nullptr;
     bool open = false;
     cudaError_t err = cudaSuccess;
+    // inside stream capture a plain record only orders the graph; the
+    // external flag makes it a record node that timestamps at replay
+    cudaError_t record(cudaEvent_t ev) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        cudaStreamIsCapturing(s, &cs);
+        if (cs == cudaStreamCaptureStatusActive)
+            return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+        return cudaEventRecord(ev, s);
+    }
     // before launching a kernel of `kind`
     void mark(int kind) {
         if (!t || t->count >= t->capacity || t->count >= MOE_TRACE_MAX) return;
-        cudaError_t e = cudaEventRecord((cudaEvent_t)t->events[t->count], s);
+        cudaError_t e = record((cudaEvent_t)t->events[t->count]);
         if (e != cudaSuccess && err == cudaSuccess) err = e;
         t->kinds[t->count] = kind;
         t->count++;
@@ -59,7 +68,7 @@ struct Tracer {
     // after the last kernel
     void end() {
         if (!t || !open || t->count >= t->capacity) return;
-        cudaError_t e = cudaEventRecord((cudaEvent_t)t->events[t->count], s);
+        cudaError_t e = record((cudaEvent_t)t->events[t->count]);
         if (e != cudaSuccess && err == cudaSuccess) err = e;
         t->kinds[t->count] = 0;
         t->count++;
@@ -134,6 +143,14 @@ moe_status launch_route(const void *x, int x_dtype, const float *w_router,
                         int32_t *ids, float *gates, float *logits, void *ws,
                         size_t ws_bytes, cudaStream_t s, Tracer *tr = nullptr);
 size_t route_ws_bytes(int T, int D, int E, int k);
+// routing plus, where a fused kernel exists (small T), the permutation in
+// the same launch; *permuted tells the caller whether it still has to permute
+moe_status launch_route_permute(const void *x, int x_dtype, const float *w_router,
+                                const float *bias, int T, int D, int E, int k, int renorm,
+                                int32_t *ids, float *gates, float *logits, int32_t *counts,
+                                int32_t *offsets, int32_t *perm, int32_t *inv, int *err,
+                                void *ws, size_t ws_bytes, cudaStream_t s, Tracer *tr,
+                                bool *permuted);
 // permute.cu
 moe_status launch_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
                           int32_t *offsets, int32_t *perm, int32_t *inv,
@@ -144,6 +161,14 @@ moe_status launch_ffn_generic(const void *x, int x_dtype, int T, int D, int F, i
                               const moe_pool &pool, const uint8_t *mask, float *H,
                               float *out_rows, cudaStream_t s, Tracer *tr = nullptr,
                               bool shared = false);
+// ffn_decode.cu -- TMA-streamed grouped GEMV for small T (see file header)
+bool decode_path_ok(int T, int D, int F, int sF);
+size_t decode_hs_halves(int T, int k, int F, int sF);
+moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, int E, int k,
+                             const int32_t *perm, const int32_t *offsets, const float *gates,
+                             const moe_pool &pool, const uint8_t *mask, const moe_pool *shared,
+                             int sF, __half *Hs, void *y, int y_dtype, float *rows_out, int *err,
+                             cudaStream_t s, Tracer *tr);
 // combine.cu
 moe_status launch_combine(const float *rows, const int32_t *inv, const float *gates,
                           int T, int k, int D, const float *shared_rows, void *y,

@@ -17,7 +17,10 @@
 // Logits stay fp32 end to end (no TF32): the tie rule compares logits at a
 // 1e-5 resolution.
 #include "moe_internal.cuh"
+#include "permute.cuh"
+#include "sm100.cuh"
 
+#include <cooperative_groups.h>
 #include <algorithm>
 #include <cfloat>
 #include <climits>
@@ -203,6 +206,204 @@ route_select_kernel(const float *__restrict__ logits, const float *__restrict__ 
     warp_select(L, E, k, renorm, ids + (size_t)warp * k, gates + (size_t)warp * k);
 }
 
+// ------------------------------------ small T: one cluster, DSMEM reduction
+// The D rows of W_r are split over the CS CTAs of one thread-block cluster.
+// Each CTA pulls its contiguous slab of W_r with bulk async copies (double
+// buffered), computes partial logits for all T tokens and E experts, and
+// keeps them in its shared memory.  After a cluster barrier, CTA r
+// finalises tokens t = r, r + CS, ...: it adds the CS partials of the token
+// in rank order through distributed shared memory (deterministic), adds the
+// bias and selects.  Optionally CTA 0 then gathers every token's ids through
+// DSMEM and runs the stable permutation, so the whole routing + grouping is
+// one launch.
+constexpr int kClusterCTAs = 16;
+constexpr int kRouteThreads = 256;
+constexpr int kRouteChunkBytes = 32 * 1024;
+
+namespace cg = cooperative_groups;
+
+template <typename XT, int EPT, int TT>
+__global__ void __launch_bounds__(kRouteThreads)
+route_cluster_kernel(const XT *__restrict__ x, const float *__restrict__ W,
+                     const float *__restrict__ bias, int T, int D, int E, int k, int renorm,
+                     int32_t *__restrict__ ids, float *__restrict__ gates,
+                     float *__restrict__ logits_out, int32_t *__restrict__ counts,
+                     int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+                     int32_t *__restrict__ inv, int *__restrict__ err) {
+    // TT: tokens rounded up to 1, 2, 4, 8 or 16 (padding tokens are zero)
+    extern __shared__ __align__(128) uint8_t smem_rc[];
+    uint8_t *smem = smem_rc;
+    __shared__ __align__(8) uint64_t bar[2];
+    __shared__ int32_t scratch[32 + 8 * 32 + 1];
+    constexpr int CS = kClusterCTAs;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int tid = threadIdx.x;
+    const int rpc = (D + CS - 1) / CS;
+    const int r0 = min(D, rank * rpc), r1 = min(D, r0 + rpc);
+    const int rows = r1 - r0;
+    const int ch = max(1, kRouteChunkBytes / (E * 4));      // rows per chunk
+    const int nch = (rows + ch - 1) / ch;
+    // threads: EPT experts each; when E is small, RS groups of threads split
+    // the rows of every chunk (summed in a fixed order afterwards)
+    const int epad = (E + 31) & ~31;
+    const int RS = (EPT == 1 && epad < kRouteThreads) ? kRouteThreads / epad : 1;
+    const int rs = tid / epad, el = tid % epad;
+
+    float *wbuf = (float *)smem;                              // 2 chunks; later the partials
+    float *xs = (float *)(smem + 2 * kRouteChunkBytes);       // [rows][TT]
+    float *Lrow = xs + (size_t)rpc * TT;                      // [E]
+    int32_t *ids_s = (int32_t *)(Lrow + E);                   // [T * k] (own tokens)
+    int32_t *ids_all = ids_s + T * k;                         // [T * k] (rank 0)
+    int32_t *hist = ids_all + T * k;                          // [8 * E]   (rank 0)
+    float *rsum = (float *)hist;                              // [RS][TT][E] before the finalise
+
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int c) {
+        const int rr = r0 + c * ch, n = min(ch, r1 - rr);
+        const uint32_t bytes = (uint32_t)(n * E * 4);
+        mbar_arrive_expect_tx(&bar[c & 1], bytes);
+        bulk_g2s(wbuf + (size_t)(c & 1) * (kRouteChunkBytes / 4), W + (size_t)rr * E, bytes, &bar[c & 1]);
+    };
+    if (tid == 0) {
+        if (nch > 0) issue(0);
+        if (nch > 1) issue(1);
+    }
+    for (int i = tid; i < rows * TT; i += kRouteThreads) {
+        const int r = i / TT, t = i % TT;
+        xs[i] = (t < T) ? load_act(x, (size_t)t * D + r0 + r) : 0.f;
+    }
+    __syncthreads();
+
+    float acc[EPT][TT];
+#pragma unroll
+    for (int q = 0; q < EPT; q++)
+#pragma unroll
+        for (int t = 0; t < TT; t++) acc[q][t] = 0.f;
+    for (int c = 0; c < nch; c++) {
+        mbar_wait(&bar[c & 1], (c >> 1) & 1, err, kErrTimeoutFull);
+        const float *wb = wbuf + (size_t)(c & 1) * (kRouteChunkBytes / 4);
+        const int n = min(ch, r1 - (r0 + c * ch));
+        for (int r = (RS > 1 ? rs : 0); r < n; r += RS) {
+            const float *xr = xs + (size_t)(c * ch + r) * TT;
+            float xv[TT];
+            if constexpr (TT % 4 == 0) {
+#pragma unroll
+                for (int t = 0; t < TT; t += 4) {
+                    const float4 q4 = *reinterpret_cast<const float4 *>(xr + t);
+                    xv[t] = q4.x; xv[t + 1] = q4.y; xv[t + 2] = q4.z; xv[t + 3] = q4.w;
+                }
+            } else {
+#pragma unroll
+                for (int t = 0; t < TT; t++) xv[t] = xr[t];
+            }
+#pragma unroll
+            for (int q = 0; q < EPT; q++) {
+                const int e = (RS > 1 ? el : tid) + q * kRouteThreads;
+                if (e < E) {
+                    const float w = wb[r * E + e];
+#pragma unroll
+                    for (int t = 0; t < TT; t++) acc[q][t] = fmaf(xv[t], w, acc[q][t]);
+                }
+            }
+        }
+        __syncthreads();                   // everyone is done with this buffer
+        if (tid == 0 && c + 2 < nch) issue(c + 2);
+    }
+    // partial logits of this CTA's rows: [T][E], in the (now free) W buffers
+    float *part = wbuf;
+    if (RS > 1) {
+        if (el < E)
+#pragma unroll
+            for (int t = 0; t < TT; t++) rsum[((size_t)rs * TT + t) * E + el] = acc[0][t];
+        __syncthreads();
+        for (int i = tid; i < T * E; i += kRouteThreads) {
+            const int t = i / E, e = i % E;
+            float v = 0.f;
+            for (int q = 0; q < RS; q++) v += rsum[((size_t)q * TT + t) * E + e];
+            part[i] = v;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < EPT; q++) {
+            const int e = tid + q * kRouteThreads;
+            if (e < E)
+#pragma unroll
+                for (int t = 0; t < TT; t++)
+                    if (t < T) part[t * E + e] = acc[q][t];
+        }
+    }
+    cluster.sync();
+
+    // finalise this CTA's tokens: partials summed in rank order (DSMEM)
+    for (int t = rank; t < T; t += CS) {
+        for (int e = tid; e < E; e += kRouteThreads) {
+            float pv[CS];
+#pragma unroll
+            for (int q = 0; q < CS; q++) pv[q] = cluster.map_shared_rank(part, q)[t * E + e];
+            float v = 0.f;
+#pragma unroll
+            for (int q = 0; q < CS; q++) v += pv[q];
+            if (bias) v += __ldg(bias + e);
+            Lrow[e] = v;
+            if (logits_out) logits_out[(size_t)t * E + e] = v;
+        }
+        __syncthreads();
+        if (tid < 32) warp_select(Lrow, E, k, renorm, ids + (size_t)t * k, gates + (size_t)t * k);
+        if (tid < 32 && perm) {
+            // keep a copy of this token's ids for the permutation gather
+            __syncwarp();
+            if (tid < k) ids_s[t * k + tid] = __ldcg(ids + (size_t)t * k + tid);
+        }
+        __syncthreads();
+    }
+    cluster.sync();                        // ids visible cluster-wide; partials no longer read
+    if (perm && rank == 0) {
+        for (int i = tid; i < T * k; i += kRouteThreads) {
+            const int t = i / k;
+            ids_all[i] = cluster.map_shared_rank(ids_s, t % CS)[i];
+        }
+        __syncthreads();
+        block_permute<kRouteThreads / 32>(ids_all, T * k, E, hist, scratch, counts, offsets, perm, inv);
+    }
+    cluster.sync();                        // no CTA exits while rank 0 may read its ids
+}
+
+// ------------------------------------------ given logits: select + permute
+// One CTA (small T): warps select tokens, then the stable permutation.
+__global__ void __launch_bounds__(kRouteThreads)
+select_permute_kernel(const float *__restrict__ logits, const float *__restrict__ bias, int T,
+                      int E, int k, int renorm, int32_t *__restrict__ ids,
+                      float *__restrict__ gates, float *__restrict__ logits_copy,
+                      int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
+                      int32_t *__restrict__ perm, int32_t *__restrict__ inv) {
+    extern __shared__ __align__(128) uint8_t smem_sp[];
+    __shared__ int32_t scratch[32 + 8 * 32 + 1];
+    float *Ls = (float *)smem_sp;                                // [T][E]
+    int32_t *ids_s = (int32_t *)(Ls + (size_t)T * E);         // [T * k]
+    int32_t *hist = ids_s + T * k;                            // [8][E]
+    for (int i = threadIdx.x; i < T * E; i += kRouteThreads) {
+        float v = logits[i];
+        if (bias) v += __ldg(bias + i % E);
+        Ls[i] = v;
+        if (logits_copy) logits_copy[i] = v;
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int t = warp; t < T; t += kRouteThreads / 32) {
+        warp_select(Ls + (size_t)t * E, E, k, renorm, ids + (size_t)t * k, gates + (size_t)t * k);
+        __syncwarp();
+        if (lane < k) ids_s[t * k + lane] = __ldcg(ids + (size_t)t * k + lane);
+    }
+    __syncthreads();
+    if (perm) block_permute<kRouteThreads / 32>(ids_s, T * k, E, hist, scratch, counts, offsets, perm, inv);
+}
+
 // ------------------------------------------------------------------- host
 static size_t splitk_partial_bytes(int T, int D, int E) {
     int nsplit = (D + kSplitRows - 1) / kSplitRows;
@@ -216,6 +417,103 @@ size_t route_ws_bytes(int T, int D, int E, int k) {
     if (T <= kSplitMaxT) c.take<char>(splitk_partial_bytes(T, D, E));
     else c.take<float>((size_t)T * E);   // logits scratch when none requested
     return c.off;
+}
+
+static int t_bucket(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16; }
+
+static size_t cluster_smem_bytes(int T, int D, int E, int k) {
+    const int rpc = (D + kClusterCTAs - 1) / kClusterCTAs;
+    const int TT = t_bucket(T);
+    const int epad = (E + 31) & ~31;
+    const int RS = (epad < kRouteThreads) ? kRouteThreads / epad : 1;
+    const size_t tail = std::max((size_t)8 * E * 4, (size_t)RS * TT * E * 4);
+    return 2 * (size_t)kRouteChunkBytes + (size_t)rpc * TT * 4 + (size_t)E * 4 +
+           2 * (size_t)T * k * 4 + tail + 256;
+}
+
+static bool cluster_route_ok(int T, int D, int E, int k, const void *w_router) {
+    return w_router && T >= 1 && T <= kSplitMaxT && E % 4 == 0 && E * 4 <= kRouteChunkBytes &&
+           T * E * 4 <= 2 * kRouteChunkBytes && cluster_smem_bytes(T, D, E, k) <= 200 * 1024;
+}
+
+static bool select_permute_ok(int T, int E, int k) {
+    return (size_t)T * E * 4 + (size_t)T * k * 4 + 8 * (size_t)E * 4 <= 200 * 1024 && T <= 64;
+}
+
+template <typename XT, int EPT, int TT>
+static cudaError_t launch_cluster(const void *x, const float *W, const float *bias, int T, int D,
+                                  int E, int k, int renorm, int32_t *ids, float *gates,
+                                  float *logits, int32_t *counts, int32_t *offsets, int32_t *perm,
+                                  int32_t *inv, int *err, cudaStream_t s) {
+    auto kern = route_cluster_kernel<XT, EPT, TT>;
+    const size_t sm = cluster_smem_bytes(T, D, E, k);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kClusterCTAs);
+    cfg.blockDim = dim3(kRouteThreads);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterCTAs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, (const XT *)x, W, bias, T, D, E, k, renorm, ids, gates,
+                              logits, counts, offsets, perm, inv, err);
+}
+
+moe_status launch_route_permute(const void *x, int x_dtype, const float *w_router,
+                                const float *bias, int T, int D, int E, int k, int renorm,
+                                int32_t *ids, float *gates, float *logits, int32_t *counts,
+                                int32_t *offsets, int32_t *perm, int32_t *inv, int *err,
+                                void *ws, size_t ws_bytes, cudaStream_t s, Tracer *tr,
+                                bool *permuted) {
+    *permuted = false;
+    if (cluster_route_ok(T, D, E, k, w_router)) {
+        mark(tr, MOE_KERNEL_ROUTE);
+        const int ept = (E + kRouteThreads - 1) / kRouteThreads;
+        cudaError_t e;
+        const bool bf = x_dtype == MOE_BF16;
+        const int tt = t_bucket(T);
+#define MOE_CL(EP, TB)                                                                            \
+    e = bf ? launch_cluster<__nv_bfloat16, EP, TB>(x, w_router, bias, T, D, E, k, renorm, ids,    \
+                                                   gates, logits, counts, offsets, perm, inv,     \
+                                                   err, s)                                        \
+           : launch_cluster<float, EP, TB>(x, w_router, bias, T, D, E, k, renorm, ids, gates,     \
+                                           logits, counts, offsets, perm, inv, err, s)
+#define MOE_CL_T(EP)                                                                              \
+    do {                                                                                          \
+        if (tt == 1) MOE_CL(EP, 1); else if (tt == 2) MOE_CL(EP, 2);                              \
+        else if (tt == 4) MOE_CL(EP, 4); else if (tt == 8) MOE_CL(EP, 8); else MOE_CL(EP, 16);   \
+    } while (0)
+        if (ept == 1) MOE_CL_T(1);
+        else if (ept == 2) MOE_CL_T(2);
+        else MOE_CL_T(4);
+#undef MOE_CL_T
+#undef MOE_CL
+        if (e != cudaSuccess) return cuda_status(e, "route_cluster_kernel");
+        *permuted = perm != nullptr;
+        return MOE_OK;
+    }
+    if (!w_router && perm && select_permute_ok(T, E, k)) {
+        const size_t sm = (size_t)T * E * 4 + (size_t)T * k * 4 + 8 * (size_t)E * 4;
+        cudaError_t e = cudaFuncSetAttribute(select_permute_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return cuda_status(e, "select_permute_kernel smem attribute");
+        mark(tr, MOE_KERNEL_ROUTE_SELECT);
+        select_permute_kernel<<<1, kRouteThreads, sm, s>>>((const float *)x, bias, T, E, k, renorm,
+                                                           ids, gates, logits, counts, offsets,
+                                                           perm, inv);
+        *permuted = true;
+        return cuda_status(cudaGetLastError(), "select_permute_kernel");
+    }
+    return launch_route(x, x_dtype, w_router, bias, T, D, E, k, renorm, ids, gates, logits, ws,
+                        ws_bytes, s, tr);
 }
 
 moe_status launch_route(const void *x, int x_dtype, const float *w_router,

@@ -202,6 +202,7 @@ def test_layer_forward_parity(moe, name, T, n_tok):
     torch.cuda.synchronize()
     print(f"rel err {_check_layer(moe, L, y32, lay.ids, n_tok):.3e}")
     assert torch.equal(y, y32.to(y.dtype))
+    assert int(lay.ws[:4].view(torch.int32)[0]) == 0      # no bounded wait ran out
 
 
 def test_layer_forward_repeated_calls_are_identical(moe):
@@ -262,3 +263,24 @@ def test_masked_two_phase_rows_are_bit_identical(moe):
     moe.expert_ffn(x, perm, offsets, pool, cfg.k, cfg.F, mask=1 - m, out=two)
     torch.cuda.synchronize()
     assert torch.equal(full, two)
+
+
+@pytest.mark.parametrize("name,T", [("decode", 1), ("decode", 16), ("wide", 1)])
+def test_graph_replay_matches_eager(moe, name, T):
+    # the bench replays captured CUDA graphs: the replayed layer must give the
+    # eager call's output bit for bit (same kernels, same order)
+    L = layer_inputs(name, T)
+    lay = _layer(moe, L)
+    x = dev_x(L)
+    lg = None if L.logits is None else dev(L.logits)
+    y_eager = lay.forward(x, logits=lg).clone()
+    out = torch.empty_like(y_eager)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        lay.forward(x, logits=lg, out=out)
+    out.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, y_eager)
