@@ -171,7 +171,7 @@ moe_status moe_expert_ffn(const void *x, int32_t x_dtype, int T, int D, int F, i
     int *status = c.take<int>(16);
     if (decode_path_ok(T, D, F, 0)) {
         __half *Hs = c.take<__half>(decode_hs_halves(T, k, F, 0));
-        return launch_ffn_decode(x, x_dtype, T, D, F, E, k, perm, offsets, nullptr, *pool,
+        return launch_ffn_decode(x, x_dtype, T, D, F, E, k, perm, nullptr, offsets, nullptr, *pool,
                                  expert_mask, nullptr, 0, Hs, nullptr, MOE_F32, out_rows, status,
                                  (cudaStream_t)stream, nullptr);
     }

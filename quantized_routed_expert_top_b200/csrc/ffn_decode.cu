@@ -20,19 +20,23 @@
 //    scale d multiplies that fp32 result; no weight is rounded.  A fixed-
 //    order cross-warp sum, SwiGLU and the token's gate weight give Hs = g * h
 //    in fp16, stored in the fragment order the next kernel reads.
-//  * dec_down: work unit = 16 rows of D; the unit walks all active experts in
-//    ascending id (then the shared expert); warp w takes experts of parity
-//    w / 8 and K-group w % 8.  Codes become exact (q - off) fp16 values, the
-//    block scale multiplies the fp32 MMA result, and each warp adds its part
-//    into per-token shared-memory sums reduced over warps in a fixed order at
-//    the end of the unit: the combine is folded in, y is deterministic and
-//    no [T*k, D] buffer exists.  With rows_out set it writes every permuted
-//    row's Y instead (no gate, no combine): the two-phase expert-cache path.
+//  * dec_down: work unit = (expert, 64 rows of D): one 2-D box of the
+//    expert's down projection over the full F (~28 KB at F=768 Q4_0) and
+//    the expert's Hs rows (contiguous in permuted order, one bulk copy).
+//    Consumer warps form 4 groups of 4; a group owns every 4th unit of the
+//    CTA and a warp one 16-row M-tile of it over the whole reduction, so no
+//    partial sums cross warps.  Codes become exact (q - off) fp16 values and
+//    the block scale multiplies the fp32 MMA result.  Each warp stores its
+//    fp32 Y rows (permuted order) to global memory.
+//  * dec_combine (fused layer only): y[t] = sum over j of the Y row of
+//    (t, j), then the shared expert's row, in that fixed order; the gate
+//    weight is already inside Hs.  Without y (the two-phase expert-cache
+//    path) the Y rows are the result: un-gated, masked experts skipped.
 //
 // dec_down is launched with programmatic dependent launch: it copies its
 // down-projection weights while dec_gateup is still running and waits
 // (griddepcontrol.wait) only before copying Hs.
-//
+
 // Fragment order of an activation block (32 values, one 64-byte row piece):
 // for c = 0..3 eight halves [v(4c), v(4c+2), v(4c+1), v(4c+3), v(16+4c),
 // v(18+4c), v(17+4c), v(19+4c)], matching the codes one 32-bit word of a
@@ -69,7 +73,8 @@ struct DecArgs {
     int hrow;                      // halves per Hs row
     void *y;                       // [T, D] (combine mode)
     int y_dtype;
-    float *rows_out;               // [T*k, D] (rows mode) or NULL
+    float *rows_out;               // [T*k (+T), D] Y rows, permuted order (+ shared rows)
+    const int32_t *inv;            // [T*k] for the combine (fused layer)
     int *err;
 };
 
@@ -98,8 +103,8 @@ __host__ __device__ inline int tma_row_bytes(int rb) {
 // Blocks per K-slice for a block size: the largest multiple of 8 dividing
 // the row's nb blocks whose staged row still fits one box (<= 256 elements
 // of 8 bytes = 2048 bytes).
-__host__ __device__ inline int slice_blocks_q(int nb, int bs) {
-    for (int sb = nb; sb >= 8; sb -= 8)
+__host__ __device__ inline int slice_blocks_q(int nb, int bs, int max_sb) {
+    for (int sb = nb < max_sb ? nb : max_sb; sb >= 8; sb -= 8)
         if (nb % sb == 0 && tma_row_bytes(sb * bs) <= 2048) return sb;
     return 8;
 }
@@ -156,19 +161,31 @@ struct Active {
     int n_virt;     // + 1 when a shared expert exists
 };
 
+// act: shared int[4 * (E + 1)]: expert id, segment start, token count and
+// slot of every active expert (ascending id), read once from global memory
+// so that per-unit lookups stay in shared memory.
 __device__ Active build_active_list(const DecArgs &a, int *act) {
     __shared__ int s_n;
+    int *aseg = act + (a.E + 1), *acnt = aseg + (a.E + 1), *aslot = acnt + (a.E + 1);
     if (threadIdx.x < 32) {
         int base = 0;
         for (int e0 = 0; e0 < a.E; e0 += 32) {
             int e = e0 + threadIdx.x;
             bool on = false;
+            int s0 = 0, c = 0;
             if (e < a.E) {
-                int c = __ldg(a.offsets + e + 1) - __ldg(a.offsets + e);
+                s0 = __ldg(a.offsets + e);
+                c = __ldg(a.offsets + e + 1) - s0;
                 on = c > 0 && (!a.mask || __ldg(a.mask + e));
             }
             unsigned b = __ballot_sync(0xffffffffu, on);
-            if (on) act[base + __popc(b & ((1u << threadIdx.x) - 1u))] = e;
+            if (on) {
+                const int i = base + __popc(b & ((1u << threadIdx.x) - 1u));
+                act[i] = e;
+                aseg[i] = s0;
+                acnt[i] = c;
+                aslot[i] = slot_of(a.slot_map, e);
+            }
             base += __popc(b);
         }
         if (threadIdx.x == 0) s_n = base;
@@ -191,11 +208,11 @@ struct Virt {
 __device__ __forceinline__ Virt virt(const DecArgs &a, const int *act, int n_routed, int v) {
     Virt r;
     if (v < n_routed) {
-        int e = act[v];
-        r.seg0 = __ldg(a.offsets + e);
-        r.cnt = __ldg(a.offsets + e + 1) - r.seg0;
+        const int *aseg = act + (a.E + 1), *acnt = aseg + (a.E + 1), *aslot = acnt + (a.E + 1);
+        r.seg0 = aseg[v];
+        r.cnt = acnt[v];
         r.Fv = a.F;
-        r.slot = (size_t)slot_of(a.slot_map, e);
+        r.slot = (size_t)aslot[v];
         r.shared = false;
         r.q8 = a.q8 != 0;
     } else {
@@ -309,10 +326,12 @@ __device__ __forceinline__ void gateup_slice(uint32_t row, uint32_t r8, const ui
 struct GuGeo {
     int sb, nsl, pitch;                 // blocks per slice, slices, staged row pitch
 };
-__host__ __device__ inline GuGeo gu_geo(int D, bool q8) {
+// max_sb: 64 for T <= 8; 32 for larger T, whose activation tables leave
+// room for fewer stages (smaller slices keep the ring deeper)
+__host__ __device__ inline GuGeo gu_geo(int D, bool q8, int max_sb) {
     const int bs = q8 ? kQ8Bytes : kQ4Bytes, nb = D / QK;
     GuGeo g;
-    g.sb = slice_blocks_q(nb, bs);
+    g.sb = slice_blocks_q(nb, bs, max_sb);
     g.nsl = nb / g.sb;
     g.pitch = tma_row_bytes(g.sb * bs);
     return g;
@@ -326,7 +345,8 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     const int g = lane >> 2, c = lane & 3;
     const int T = a.T, D = a.D;
     const int nbD = D / QK;
-    const GuGeo geo4 = gu_geo(D, false), geo8 = gu_geo(D, true);
+    constexpr int kMaxSb = NT == 1 ? 64 : 32;
+    const GuGeo geo4 = gu_geo(D, false, kMaxSb), geo8 = gu_geo(D, true, kMaxSb);
     const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
     const int pitch_max = max(any4 ? geo4.pitch : 0, any8 ? geo8.pitch : 0);
     const int stage_bytes = (int)round_up((size_t)2 * kTile * pitch_max, 128);
@@ -344,8 +364,10 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     float *red = (float *)(stages + (size_t)S * stage_bytes);
     uint64_t *full = (uint64_t *)(red + 2 * kDW * NT * 32 * 4);
     uint64_t *empty = full + kMaxStages;
-    int *act = (int *)(empty + kMaxStages);
-    int *tok = act + a.E + 1;
+    uint64_t *rfull = empty + kMaxStages;          // [2] partials of a unit written
+    uint64_t *rempty = rfull + 2;                  // [2] a unit's epilogue done
+    int *act = (int *)(rempty + 2);
+    int *tok = act + 4 * (a.E + 1);
     float *gw = (float *)(tok + kMaxTk + 16);
 
     if (tid == 0) {
@@ -353,7 +375,47 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kDW);
         }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&rfull[b], kDW * 32);
+            mbar_init(&rempty[b], kDW * 32);
+        }
         fence_mbar_init();
+    }
+    // The activations do not depend on the routing kernel this grid may
+    // overlap with: stage them (fp16, fragment order; row T is zero) and the
+    // per-block -off * sum(x) tables before waiting for it.
+    if (warp < kDW) {
+        for (int idx = tid; idx < (T + 1) * (nbD * 4); idx += kDW * 32) {
+            const int t = idx / (nbD * 4), rem = idx % (nbD * 4), b = rem >> 2, cc = rem & 3;
+            uint4 pk = make_uint4(0u, 0u, 0u, 0u);
+            if (t < T) {
+                const size_t xb = (size_t)t * D + b * QK;
+                const int src[8] = {4 * cc, 4 * cc + 2, 4 * cc + 1, 4 * cc + 3,
+                                    16 + 4 * cc, 18 + 4 * cc, 17 + 4 * cc, 19 + 4 * cc};
+                uint32_t h[8];
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    const float v = a.x_bf16 ? load_act((const __nv_bfloat16 *)a.x, xb + src[q])
+                                             : load_act((const float *)a.x, xb + src[q]);
+                    h[q] = (uint32_t)__half_as_ushort(__float2half_rn(v));
+                }
+                pk.x = h[0] | (h[1] << 16);
+                pk.y = h[2] | (h[3] << 16);
+                pk.z = h[4] | (h[5] << 16);
+                pk.w = h[6] | (h[7] << 16);
+            }
+            *reinterpret_cast<uint4 *>(xs + (size_t)t * xrow + b * 64 + cc * 16) = pk;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
+        for (int idx = tid; idx < (T + 1) * nbD; idx += kDW * 32) {
+            const int t = idx / nbD, b = idx % nbD;
+            const __half *hp = reinterpret_cast<const __half *>(xs + (size_t)t * xrow + b * 64);
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; i++) sum += __half2float(hp[i]);
+            sxt[idx] = -magic_off<false>() * sum;
+            sxt[(size_t)(T + 1) * nbD + idx] = -magic_off<true>() * sum;
+        }
     }
     // routing results come from the previous kernel
     pdl_wait();
@@ -400,47 +462,42 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
 
     // ------------------------------------------------------- consumers
     load_token_tables(a, tok, gw);
-    // stage the activations once, fp16 in fragment order; row T is zero
-    for (int idx = tid; idx < (T + 1) * (nbD * 4); idx += kDW * 32) {
-        const int t = idx / (nbD * 4), rem = idx % (nbD * 4), b = rem >> 2, cc = rem & 3;
-        uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-        if (t < T) {
-            const size_t base = (size_t)t * D + b * QK;
-            const int src[8] = {4 * cc, 4 * cc + 2, 4 * cc + 1, 4 * cc + 3,
-                                16 + 4 * cc, 18 + 4 * cc, 17 + 4 * cc, 19 + 4 * cc};
-            uint32_t h[8];
-#pragma unroll
-            for (int q = 0; q < 8; q++) {
-                const float v = a.x_bf16 ? load_act((const __nv_bfloat16 *)a.x, base + src[q])
-                                         : load_act((const float *)a.x, base + src[q]);
-                h[q] = (uint32_t)__half_as_ushort(__float2half_rn(v));
-            }
-            pk.x = h[0] | (h[1] << 16);
-            pk.y = h[2] | (h[3] << 16);
-            pk.z = h[4] | (h[5] << 16);
-            pk.w = h[6] | (h[7] << 16);
-        }
-        *reinterpret_cast<uint4 *>(xs + (size_t)t * xrow + b * 64 + cc * 16) = pk;
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
-    // -off * (sum of the 32 fp16 activations of each block), for both codes
-    for (int idx = tid; idx < (T + 1) * nbD; idx += kDW * 32) {
-        const int t = idx / nbD, b = idx % nbD;
-        const __half *hp = reinterpret_cast<const __half *>(xs + (size_t)t * xrow + b * 64);
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; i++) s += __half2float(hp[i]);
-        sxt[idx] = -magic_off<false>() * s;
-        sxt[(size_t)(T + 1) * nbD + idx] = -magic_off<true>() * s;
-    }
     asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
 
     const uint32_t xs_a = smem_u32(xs), sx_a = smem_u32(sxt), st_a = smem_u32(stages);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    int ub = 0;                                          // unit counter (red buffer parity)
-    for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ub ^= 1) {
+    // The cross-warp reduction of unit j is deferred until after unit j+1's
+    // partials are written (two partial buffers, mbarriers instead of a
+    // CTA-wide barrier), so warps that finish a unit early do not idle.
+    auto epilogue = [&](int j, const Virt &pv, int ptile) {
+        const int b = j & 1;
+        if (!mbar_wait(&rfull[b], (uint32_t)((j >> 1) & 1), a.err, kErrTimeoutFull)) { ok = false; return; }
+        const float *redb = red + (size_t)b * kDW * NT * 128;
+        const int o = tid;                               // one output per thread
+        const int rr = o % kTile, n = o / kTile;         // row within tile, column
+        if (n < pv.cnt && n < 8 * NT) {
+            const int nt = n >> 3, nn = n & 7;
+            const int L = (rr & 7) * 4 + (nn >> 1);
+            const int q = ((rr >> 3) << 1) | (nn & 1);
+            float sg = 0.f, su = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; w++) {
+                sg += redb[((size_t)w * NT + nt) * 128 + L * 4 + q];
+                su += redb[((size_t)(8 + w) * NT + nt) * 128 + L * 4 + q];
+            }
+            const int pos = pv.seg0 + n;
+            const float h = silu(sg) * su * gw[pos];
+            const int r = ptile * kTile + rr;
+            a.Hs[(size_t)pos * a.hrow + (r >> 5) * 32 + frag_slot(r & 31)] = __float2half_rn(h);
+        }
+        mbar_arrive(&rempty[b]);
+    };
+    int j = 0;
+    Virt pv{};
+    int ptile = 0;
+    for (int u = blockIdx.x; u < U && ok; u += gridDim.x, j++) {
         int v, tile;
         if (u < A.n_routed * tiles_r) { v = u / tiles_r; tile = u % tiles_r; }
         else { v = A.n_routed; tile = u - A.n_routed * tiles_r; }
@@ -457,10 +514,10 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
             const int tb = n < vi.cnt ? tok[vi.seg0 + n] : T;
             xa[nt] = xs_a + tb * xrow + kb0 * 64 + c * 16;
 #pragma unroll
-            for (int j = 0; j < 2; j++) {
-                const int m = 8 * nt + 2 * c + j;
+            for (int jj = 0; jj < 2; jj++) {
+                const int m = 8 * nt + 2 * c + jj;
                 const int tc = m < vi.cnt ? tok[vi.seg0 + m] : T;
-                sa[nt][j] = sxq + (uint32_t)((tc * nbD + kb0) * 4);
+                sa[nt][jj] = sxq + (uint32_t)((tc * nbD + kb0) * 4);
             }
         }
         float acc[NT][4];
@@ -496,51 +553,49 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
             if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        // cross-warp reduction (double-buffered partials, one barrier per
-        // unit) in a fixed order, SwiGLU, gate weight, fp16 store
-        float *redb = red + (size_t)ub * kDW * NT * 128;
-        float *rw = redb + (size_t)warp * NT * 128;
+        // partials of unit j into buffer j % 2, once unit j-2's epilogue is done
+        const int b = j & 1;
+        if (j >= 2 && !mbar_wait(&rempty[b], (uint32_t)(((j - 2) >> 1) & 1), a.err, kErrTimeoutEmpty)) {
+            ok = false;
+            break;
+        }
+        float *rw = red + ((size_t)b * kDW + warp) * NT * 128;
 #pragma unroll
         for (int nt = 0; nt < NT; nt++)
 #pragma unroll
             for (int q = 0; q < 4; q++) rw[nt * 128 + lane * 4 + q] = acc[nt][q];
-        asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
-        for (int o = tid; o < kTile * 8 * ntile; o += kDW * 32) {
-            const int rr = o % kTile, n = o / kTile;        // row within tile, column
-            if (n < vi.cnt) {
-                const int nt = n >> 3, nn = n & 7;
-                const int L = (rr & 7) * 4 + (nn >> 1);
-                const int q = ((rr >> 3) << 1) | (nn & 1);
-                float sg = 0.f, su = 0.f;
-#pragma unroll
-                for (int w = 0; w < 8; w++) {
-                    sg += redb[((size_t)w * NT + nt) * 128 + L * 4 + q];
-                    su += redb[((size_t)(8 + w) * NT + nt) * 128 + L * 4 + q];
-                }
-                const int pos = vi.seg0 + n;
-                const float h = silu(sg) * su * gw[pos];
-                const int r = tile * kTile + rr;
-                a.Hs[(size_t)pos * a.hrow + (r >> 5) * 32 + frag_slot(r & 31)] = __float2half_rn(h);
-            }
-        }
+        mbar_arrive(&rfull[b]);
+        if (j >= 1) epilogue(j - 1, pv, ptile);
+        pv = vi;
+        ptile = tile;
     }
+    if (ok && j >= 1) epilogue(j - 1, pv, ptile);
 }
 
 // --------------------------------------------------------------------- down
-// One expert's 16-row tile for one warp: WB blocks from the warp's first
-// block; codes become exact (q - off) fp16 values and the block scale
-// multiplies the fp32 MMA result.  ha: B row of column g (and g+8).
-template <bool Q8, int NTILE, int WB, int MIS0>
-__device__ __forceinline__ void down_expert(uint32_t row, uint32_t r8, const uint32_t *ha, int c,
-                                            float (*acc)[4]) {
+// Work unit = (expert, 64 rows of D): one 2-D box of the expert's down
+// projection (64 rows x F/32 blocks, one TMA request of ~28 KB at F=768
+// Q4_0) plus the expert's Hs rows, which are contiguous in permuted order
+// (one bulk copy).  The 16 consumer warps form 4 groups of 4; group q takes
+// every 4th unit of the CTA and warp m of a group one 16-row M-tile of it
+// over the FULL reduction length, so no partial sums cross warps.  Each
+// warp writes its Y rows (fp32, permuted order) to global memory; the
+// combine is a separate, deterministic kernel.
+constexpr int kDnRows = 64;
+
+// 8 consecutive blocks of one 16-row tile for one warp; the block group
+// starts 4-byte aligned (8 blocks of 18 or 34 bytes).
+template <bool Q8, int NTILE>
+__device__ __forceinline__ void down_blocks8(uint32_t row, uint32_t r8, const uint32_t *ha, int c,
+                                             float (*acc)[4]) {
     constexpr int BS = qbytes<Q8>();
     const uint32_t off2 = magic_off2<Q8>();
     const float zero[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int bl = 0; bl < WB; bl++) {
+    for (int bl = 0; bl < 8; bl++) {
         const uint32_t blk = row + bl * BS;
         uint32_t lo[4], hi[4];
-        if (((MIS0 + 2 * bl + 2) & 3) == 0) {
+        if (((2 * bl + 2) & 3) == 0) {
             magic_codes<Q8, 0>(blk + 2 + 4 * c, lo);
             magic_codes<Q8, 0>(blk + r8 + 2 + 4 * c, hi);
         } else {
@@ -566,197 +621,180 @@ __device__ __forceinline__ void down_expert(uint32_t row, uint32_t r8, const uin
     }
 }
 
-// Requires F, shared F <= 1024 (one K-slice per expert).
-template <int NT, int WB, bool ROWS>
+// Local unit i of a CTA goes to consumer group i % G; the stage ring is
+// split per group (G * Sg stages, group q owns stages q, q + G, ...), so a
+// group only ever waits on stages it consumes itself and can never be two
+// phases ahead of one of them.
+struct DnSlot {
+    int stage;
+    uint32_t phase;
+};
+__device__ __forceinline__ DnSlot dn_slot(int i, int G, int Sg) {
+    const int m = i / G;
+    return {i % G + G * (m % Sg), (uint32_t)((m / Sg) & 1)};
+}
+
+template <int NT>
 __global__ void __launch_bounds__(kDThreads, 1)
-dec_down_kernel(DecArgs a, int S, int hrows, const __grid_constant__ DecMaps maps) {
+dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ DecMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
-    const int T = a.T, D = a.D;
-    const int Fmax = a.F > a.sF ? a.F : a.sF;
-    const int hstride = staged_act_bytes(Fmax);
+    const int D = a.D;
+    const int S = G * Sg;
+    const int hbytes = a.hrow * 2;                      // staged Hs row = its global stride
     const int pr = tma_row_bytes((a.F / QK) * (a.q8 ? kQ8Bytes : kQ4Bytes));
     const int ps = a.sF > 0 ? tma_row_bytes((a.sF / QK) * (a.sq8 ? kQ8Bytes : kQ4Bytes)) : 0;
-    const int wbytes = kTile * (pr > ps ? pr : ps);
-    const int stage_bytes = (int)round_up((size_t)wbytes + (size_t)hrows * hstride, 128);
-    const int ncols = ROWS ? 16 : T;                   // accumulator columns per warp
-    const int par = warp >> 3, kg = warp & 7;
+    const int wbytes = kDnRows * (pr > ps ? pr : ps);
+    const int stage_bytes = (int)round_up((size_t)wbytes + (size_t)hrows * hbytes, 128);
+    const int grp = warp >> 2, mt = warp & 3;
 
-    // carve (from a 1024-aligned base; tensor copies need 128-byte aligned
-    // destinations): stages | zero row | yacc [kDW][ncols][16] | barriers |
-    // act | tok
+    // carve (1024-aligned base: tensor copies need 128-byte destinations)
     uint8_t *stages = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
-    uint8_t *zrow = stages + (size_t)S * stage_bytes;
-    float *yacc = (float *)(zrow + round_up((size_t)hstride, 16));
-    uint64_t *full = (uint64_t *)(yacc + kDW * ncols * kTile);
+    uint64_t *full = (uint64_t *)(stages + (size_t)S * stage_bytes);
     uint64_t *empty = full + kMaxStages;
     int *act = (int *)(empty + kMaxStages);
-    int *tok = act + a.E + 1;
 
     if (tid == 0) {
         for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 8);             // the 8 warps of one parity group
+            mbar_init(&empty[s], 4);             // the 4 warps of the owning group
         }
         fence_mbar_init();
     }
-    for (int i = tid; i < kDW * ncols * kTile; i += blockDim.x) yacc[i] = 0.f;
-    for (int i = tid; i < hstride / 4; i += blockDim.x) reinterpret_cast<uint32_t *>(zrow)[i] = 0u;
     // routing (perm/offsets) is complete: the gate/up kernel waited for it
     // before letting this grid launch
-    load_token_tables(a, tok, nullptr);
     const Active A = build_active_list(a, act);
-    const int U = D / kTile;
-    const int NV = A.n_virt;
+    const int tiles = D / kDnRows;
+    const int U = A.n_virt * tiles;
 
     if (warp == kDW) {
         if (lane == 0) {
             bool ok = true, waited = false;
-            int pending[kMaxStages], pend_v[kMaxStages];
+            int pend_s[kMaxStages], pend_v[kMaxStages];
             int npend = 0;
             auto issue_h = [&](int st, int v) {
                 const Virt vi = virt(a, act, A.n_routed, v);
-                uint8_t *dst = stages + (size_t)st * stage_bytes + wbytes;
-                for (int n = 0; n < vi.cnt; n++)
-                    bulk_g2s(dst + n * hstride, a.Hs + (size_t)(vi.seg0 + n) * a.hrow,
-                             (uint32_t)(vi.Fv * 2), &full[st]);
+                bulk_g2s(stages + (size_t)st * stage_bytes + wbytes, a.Hs + (size_t)vi.seg0 * a.hrow,
+                         (uint32_t)(vi.cnt * hbytes), &full[st]);
             };
-            long long i = 0;                    // issue index
-            for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-                for (int v = 0; v < NV && ok; v++, i++) {
-                    const int stage = (int)(i % S);
-                    const uint32_t ph = (uint32_t)((i / S) & 1);
-                    const Virt vi = virt(a, act, A.n_routed, v);
-                    const int pitch = vi.shared ? ps : pr;
-                    if (!mbar_wait(&empty[stage], ph ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
-                    uint8_t *dst = stages + (size_t)stage * stage_bytes;
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(kTile * pitch + vi.cnt * vi.Fv * 2));
-                    tma_load_2d(dst, vi.shared ? &maps.sdown : &maps.down, 0,
-                                (vi.shared ? 0 : (int)vi.slot * a.D) + u * kTile, &full[stage]);
-                    if (waited) {
-                        issue_h(stage, v);
-                    } else {
-                        pending[npend] = stage; pend_v[npend] = v; npend++;
-                        if (npend == S) {
-                            // every stage holds prefetched weights: now wait for Hs
-                            pdl_wait();
-                            waited = true;
-                            for (int q = 0; q < npend; q++) issue_h(pending[q], pend_v[q]);
-                            npend = 0;
-                        }
+            int i = 0;                          // local unit index
+            for (int u = blockIdx.x; u < U && ok; u += gridDim.x, i++) {
+                const int v = u / tiles, dt = u % tiles;
+                const DnSlot sl = dn_slot(i, G, Sg);
+                const Virt vi = virt(a, act, A.n_routed, v);
+                const int pitch = vi.shared ? ps : pr;
+                if (!mbar_wait(&empty[sl.stage], sl.phase ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                uint8_t *dst = stages + (size_t)sl.stage * stage_bytes;
+                mbar_arrive_expect_tx(&full[sl.stage], (uint32_t)(kDnRows * pitch + vi.cnt * hbytes));
+                tma_load_2d(dst, vi.shared ? &maps.sdown : &maps.down, 0,
+                            (vi.shared ? 0 : (int)vi.slot * D) + dt * kDnRows, &full[sl.stage]);
+                if (waited) {
+                    issue_h(sl.stage, v);
+                } else {
+                    pend_s[npend] = sl.stage; pend_v[npend] = v; npend++;
+                    if (npend == S) {
+                        // every stage holds prefetched weights: now wait for Hs
+                        pdl_wait();
+                        waited = true;
+                        for (int q = 0; q < npend; q++) issue_h(pend_s[q], pend_v[q]);
+                        npend = 0;
                     }
                 }
             }
             if (!waited) {
                 pdl_wait();
-                for (int q = 0; q < npend; q++) issue_h(pending[q], pend_v[q]);
+                for (int q = 0; q < npend; q++) issue_h(pend_s[q], pend_v[q]);
             }
-            // drain
-            for (int q = 0; q < S; q++, i++) {
-                const int stage = (int)(i % S);
-                mbar_wait(&empty[stage], (uint32_t)(((i / S) & 1) ^ 1), a.err, kErrTimeoutDrain);
+            // drain: wait for the consumers of the last S units (one per stage)
+            for (int q = i - S; q < i; q++) {
+                if (q < 0) continue;
+                const DnSlot sl = dn_slot(q, G, Sg);
+                mbar_wait(&empty[sl.stage], sl.phase, a.err, kErrTimeoutDrain);
             }
         }
         return;
     }
+    if (grp >= G) return;
 
     // ------------------------------------------------------- consumers
-    bool ok = true;
-    float *yw = yacc + (size_t)warp * ncols * kTile;
-    const uint32_t st_a = smem_u32(stages), z_a = smem_u32(zrow);
-    long long ibase = 0;
-    for (int u = blockIdx.x; u < U && ok; u += gridDim.x, ibase += NV) {
-        for (int v = par; v < NV && ok; v += 2) {
-            const long long i = ibase + v;
-            const int stage = (int)(i % S);
-            const uint32_t ph = (uint32_t)((i / S) & 1);
-            const Virt vi = virt(a, act, A.n_routed, v);
-            const int bsz = vi.q8 ? kQ8Bytes : kQ4Bytes;
-            const int rstride = vi.shared ? ps : pr;
-            const int wb = (vi.Fv / QK) / 8;           // blocks per K-group (<= WB)
-            const int kbw = kg * wb;
-            const int ntile = vi.cnt > 8 ? 2 : 1;
-            float acc[NT][4];
+    const uint32_t st_a = smem_u32(stages);
+    int i = grp;
+    for (int u = blockIdx.x + grp * gridDim.x; u < U; u += G * gridDim.x, i += G) {
+        const int v = u / tiles, dt = u % tiles;
+        const DnSlot sl = dn_slot(i, G, Sg);
+        const Virt vi = virt(a, act, A.n_routed, v);
+        const int bsz = vi.q8 ? kQ8Bytes : kQ4Bytes;
+        const int pitch = vi.shared ? ps : pr;
+        const int nb = vi.Fv / QK;
+        const int ntile = vi.cnt > 8 ? 2 : 1;
+        float acc[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; nt++)
+        for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-                for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
-            if (!mbar_wait(&full[stage], ph, a.err, kErrTimeoutFull)) { ok = false; break; }
-            const uint32_t sbase = st_a + stage * stage_bytes;
-            const uint32_t row = sbase + g * rstride + kbw * bsz;
-            uint32_t ha[NT];
+            for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
+        if (!mbar_wait(&full[sl.stage], sl.phase, a.err, kErrTimeoutFull)) break;
+        const uint32_t sbase = st_a + sl.stage * stage_bytes;
+        uint32_t row = sbase + (mt * kTile + g) * pitch;
+        const uint32_t r8 = 8u * pitch;
+        uint32_t ha[NT];
 #pragma unroll
-            for (int nt = 0; nt < NT; nt++) {
-                const int n = g + 8 * nt;
-                ha[nt] = (n < vi.cnt ? sbase + wbytes + n * hstride : z_a) + kbw * 64 + c * 16;
-            }
-            const int mis0 = (kbw * bsz) & 3;
-            const uint32_t r8 = 8u * rstride;
-#define MOE_DN(Q8, NTL, W, MIS) down_expert<Q8, NTL, W, MIS>(row, r8, ha, c, acc)
-#define MOE_DN_W(Q8, NTL, MIS)                                              \
-    do {                                                                    \
-        if (wb == 3) MOE_DN(Q8, NTL, 3, MIS);                               \
-        else if (wb == 2) MOE_DN(Q8, NTL, 2, MIS);                          \
-        else if (wb == 1) MOE_DN(Q8, NTL, 1, MIS);                          \
-        else MOE_DN(Q8, NTL, 4, MIS);                                       \
-    } while (0)
-            if (!vi.q8) {
-                if (ntile == 1) { if (mis0 == 0) MOE_DN_W(false, 1, 0); else MOE_DN_W(false, 1, 2); }
-                else if (NT > 1) { if (mis0 == 0) MOE_DN_W(false, NT, 0); else MOE_DN_W(false, NT, 2); }
-            } else {
-                if (ntile == 1) { if (mis0 == 0) MOE_DN_W(true, 1, 0); else MOE_DN_W(true, 1, 2); }
-                else if (NT > 1) { if (mis0 == 0) MOE_DN_W(true, NT, 0); else MOE_DN_W(true, NT, 2); }
-            }
-#undef MOE_DN_W
+        for (int nt = 0; nt < NT; nt++) {
+            const int n = g + 8 * nt;
+            // columns past the expert's token count read whatever the stage
+            // holds there; an MMA column depends only on its own B column,
+            // and those columns are never stored
+            ha[nt] = sbase + wbytes + (n < hrows ? n : 0) * hbytes + c * 16;
+        }
+        for (int kb = 0; kb < nb; kb += 8) {
+#define MOE_DN(Q8, NTL) down_blocks8<Q8, NTL>(row, r8, ha, c, acc)
+            if (!vi.q8) { if (ntile == 1) MOE_DN(false, 1); else if (NT > 1) MOE_DN(false, NT); }
+            else { if (ntile == 1) MOE_DN(true, 1); else if (NT > 1) MOE_DN(true, NT); }
 #undef MOE_DN
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-            // C fragment: rows g / g+8 of the d-tile, columns 2c, 2c+1 (+8 nt)
+            row += 8 * bsz;
 #pragma unroll
-            for (int nt = 0; nt < NT; nt++)
-#pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    const int n = nt * 8 + 2 * c + (q & 1);
-                    const int r = g + ((q >> 1) << 3);
-                    if (n < vi.cnt) {
-                        const int col = ROWS ? n : tok[vi.seg0 + n];
-                        yw[col * kTile + r] += acc[nt][q];
-                    }
-                }
-            if (ROWS) {
-                // flush this expert's rows: fixed-order sum over the group's warps
-                const int bid = 2 + par;
-                asm volatile("bar.sync %0, %1;" ::"r"(bid), "n"(8 * 32));
-                const int gt = tid - par * 256;
-                for (int o = gt; o < vi.cnt * kTile; o += 256) {
-                    const int n = o / kTile, r = o % kTile;
-                    float s = 0.f;
-#pragma unroll
-                    for (int w = 0; w < 8; w++) s += yacc[((size_t)(par * 8 + w) * ncols + n) * kTile + r];
-                    a.rows_out[(size_t)(vi.seg0 + n) * D + u * kTile + r] = s;
-                }
-                asm volatile("bar.sync %0, %1;" ::"r"(bid), "n"(8 * 32));
-                for (int o = gt; o < 8 * ncols * kTile; o += 256) yacc[(size_t)par * 8 * ncols * kTile + o] = 0.f;
-                asm volatile("bar.sync %0, %1;" ::"r"(bid), "n"(8 * 32));
-            }
+            for (int nt = 0; nt < NT; nt++) ha[nt] += 8 * 64;
         }
-        if (!ok) break;
-        if (!ROWS) {
-            asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
-            for (int o = tid; o < T * kTile; o += kDW * 32) {
-                const int t = o / kTile, r = o % kTile;
-                float s = 0.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[sl.stage]);
+        // C fragment: rows g / g+8 of the M-tile, columns 2c, 2c+1 (+8 nt)
+        float *out = a.rows_out + (size_t)vi.seg0 * D + dt * kDnRows + mt * kTile;
 #pragma unroll
-                for (int w = 0; w < kDW; w++) s += yacc[((size_t)w * ncols + t) * kTile + r];
-                const size_t yi = (size_t)t * D + u * kTile + r;
-                if (a.y_dtype == MOE_BF16) ((__nv_bfloat16 *)a.y)[yi] = __float2bfloat16_rn(s);
-                else ((float *)a.y)[yi] = s;
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const int n = nt * 8 + 2 * c + (q & 1);
+                const int r = g + ((q >> 1) << 3);
+                if (n < vi.cnt) out[(size_t)n * D + r] = acc[nt][q];
             }
-            asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
-            for (int o = tid; o < kDW * ncols * kTile; o += kDW * 32) yacc[o] = 0.f;
-            asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
-        }
+    }
+}
+
+// y[t, :] = sum_j rows[inv[t*k + j], :] (+ rows[T*k + t, :] for the shared
+// expert), in j order; rows already carry the gate weight.
+__global__ void __launch_bounds__(256)
+dec_combine_kernel(const float *__restrict__ rows, const int32_t *__restrict__ inv, int T, int k,
+                   int D, int shared, void *__restrict__ y, int y_dtype) {
+    pdl_wait();
+    const int t = blockIdx.x;
+    const int d0 = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+    if (d0 >= D) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; j++) {
+        const float4 r = __ldg(reinterpret_cast<const float4 *>(rows + (size_t)__ldg(inv + (size_t)t * k + j) * D + d0));
+        acc.x += r.x; acc.y += r.y; acc.z += r.z; acc.w += r.w;
+    }
+    if (shared) {
+        const float4 r = __ldg(reinterpret_cast<const float4 *>(rows + (size_t)(T * k + t) * D + d0));
+        acc.x += r.x; acc.y += r.y; acc.z += r.z; acc.w += r.w;
+    }
+    const size_t yi = (size_t)t * D + d0;
+    if (y_dtype == MOE_BF16) {
+        __nv_bfloat162 *yp = reinterpret_cast<__nv_bfloat162 *>((__nv_bfloat16 *)y + yi);
+        yp[0] = __floats2bfloat162_rn(acc.x, acc.y);
+        yp[1] = __floats2bfloat162_rn(acc.z, acc.w);
+    } else {
+        *reinterpret_cast<float4 *>((float *)y + yi) = acc;
     }
 }
 
@@ -770,9 +808,12 @@ bool decode_path_ok(int T, int D, int F, int sF) {
            (sF == 0 || (sF % 256 == 0 && sF <= 1024));
 }
 
+// Hs rows are padded by 32 halves (64 bytes): row stride = 64 mod 128 bytes,
+// so the down kernel's 16-byte fragment loads of rows n, n+1 do not collide
 size_t decode_hs_halves(int T, int k, int F, int sF) {
-    return (size_t)(T * k + T) * (size_t)std::max(F, sF);
+    return (size_t)(T * k + T) * (size_t)(std::max(F, sF) + 32);
 }
+size_t decode_rows_floats(int T, int k, int D) { return (size_t)(T * k + T) * D; }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -812,26 +853,26 @@ static moe_status encode_rows(CUtensorMap *m, const void *base, size_t row_bytes
     return MOE_OK;
 }
 
-static moe_status encode_maps(const DecArgs &a, int n_slots, DecMaps *m) {
+static moe_status encode_maps(const DecArgs &a, int n_slots, int max_sb, DecMaps *m) {
     memset(m, 0, sizeof(*m));
     const int nbD = a.D / QK;
     const int br = a.q8 ? kQ8Bytes : kQ4Bytes;
-    const GuGeo gr = gu_geo(a.D, a.q8);
+    const GuGeo gr = gu_geo(a.D, a.q8, max_sb);
     moe_status st;
     if ((st = encode_rows(&m->gate, a.gate, (size_t)nbD * br, (size_t)n_slots * a.F, gr.pitch, kTile)))
         return st;
     if ((st = encode_rows(&m->up, a.up, (size_t)nbD * br, (size_t)n_slots * a.F, gr.pitch, kTile)))
         return st;
     const size_t rbd = (size_t)(a.F / QK) * br;
-    if ((st = encode_rows(&m->down, a.down, rbd, (size_t)n_slots * a.D, tma_row_bytes((int)rbd), kTile)))
+    if ((st = encode_rows(&m->down, a.down, rbd, (size_t)n_slots * a.D, tma_row_bytes((int)rbd), kDnRows)))
         return st;
     if (a.sF > 0) {
         const int bsh = a.sq8 ? kQ8Bytes : kQ4Bytes;
-        const GuGeo gs = gu_geo(a.D, a.sq8);
+        const GuGeo gs = gu_geo(a.D, a.sq8, max_sb);
         if ((st = encode_rows(&m->sgate, a.sh_gate, (size_t)nbD * bsh, a.sF, gs.pitch, kTile))) return st;
         if ((st = encode_rows(&m->sup, a.sh_up, (size_t)nbD * bsh, a.sF, gs.pitch, kTile))) return st;
         const size_t rbs = (size_t)(a.sF / QK) * bsh;
-        if ((st = encode_rows(&m->sdown, a.sh_down, rbs, a.D, tma_row_bytes((int)rbs), kTile))) return st;
+        if ((st = encode_rows(&m->sdown, a.sh_down, rbs, a.D, tma_row_bytes((int)rbs), kDnRows))) return st;
     }
     return MOE_OK;
 }
@@ -855,7 +896,7 @@ static cudaError_t launch_pdl(void (*kern)(Args...), int grid, size_t smem, cuda
 }
 
 static size_t tables_bytes(int E) {
-    return (size_t)(E + 1) * sizeof(int) + (size_t)(kMaxTk + 16) * (sizeof(int) + sizeof(float));
+    return 4 * (size_t)(E + 1) * sizeof(int) + (size_t)(kMaxTk + 16) * (sizeof(int) + sizeof(float));
 }
 
 template <int NT>
@@ -866,7 +907,7 @@ static cudaError_t launch_gateup(const DecArgs &a, const DecMaps &m, int grid, s
     case 512: return launch_pdl(dec_gateup_kernel<NT, 2, 2>, grid, smem, s, a, S, m);
     case 768: return launch_pdl(dec_gateup_kernel<NT, 3, 3>, grid, smem, s, a, S, m);
     case 1024: return launch_pdl(dec_gateup_kernel<NT, 4, 4>, grid, smem, s, a, S, m);
-    default: return launch_pdl(dec_gateup_kernel<NT, 8, 4>, grid, smem, s, a, S, m);
+    default: return launch_pdl(dec_gateup_kernel<NT, (NT == 1 ? 8 : 4), 4>, grid, smem, s, a, S, m);
     }
 }
 
@@ -874,19 +915,21 @@ template <int NT>
 static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Tracer *tr) {
     const int sms = num_sms();
     DecMaps maps;
-    moe_status st = encode_maps(a, n_slots, &maps);
+    const int max_sb = NT == 1 ? 64 : 32;
+    moe_status st = encode_maps(a, n_slots, max_sb, &maps);
     if (st != MOE_OK) return st;
     const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
     // ---- gate/up
     {
         const int nbD = a.D / QK;
-        const int pitch = std::max(any4 ? gu_geo(a.D, false).pitch : 0, any8 ? gu_geo(a.D, true).pitch : 0);
+        const int pitch = std::max(any4 ? gu_geo(a.D, false, max_sb).pitch : 0,
+                                   any8 ? gu_geo(a.D, true, max_sb).pitch : 0);
         const int stage_bytes = (int)round_up((size_t)2 * kTile * pitch, 128);
         // mirrors the kernel's carve; + 1024 for aligning the base
         const size_t fixed = round_up(round_up((size_t)(a.T + 1) * staged_act_bytes(a.D), 16) +
                                       (size_t)2 * (a.T + 1) * nbD * 4, 1024) +
                              (size_t)2 * kDW * NT * 32 * 4 * sizeof(float) +
-                             2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
+                             (2 * kMaxStages + 4) * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
         if (fixed >= kDecSmemMax) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
         int S = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - fixed) / stage_bytes);
         if (S < 2) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
@@ -897,38 +940,54 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         cudaError_t e = launch_gateup<NT>(a, maps, grid, smem, s, S);
         if (e != cudaSuccess) return cuda_status(e, "dec_gateup_kernel");
     }
-    // ---- down (+ combine)
+    // ---- down: Y rows
     {
-        const int Fmax = std::max(a.F, a.sF);
         const int hrows = std::min(a.T, 16);
         const int pr = tma_row_bytes((a.F / QK) * (a.q8 ? kQ8Bytes : kQ4Bytes));
         const int ps = a.sF > 0 ? tma_row_bytes((a.sF / QK) * (a.sq8 ? kQ8Bytes : kQ4Bytes)) : 0;
-        const size_t wbytes = (size_t)kTile * std::max(pr, ps);
-        const int stage_bytes = (int)round_up(wbytes + (size_t)hrows * staged_act_bytes(Fmax), 128);
-        const int ncols = a.rows_out ? 16 : a.T;
-        const size_t fixed = round_up((size_t)staged_act_bytes(Fmax), 16) +
-                             (size_t)kDW * ncols * kTile * sizeof(float) +
-                             2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
-        if (fixed >= kDecSmemMax) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
-        int S = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - fixed) / stage_bytes);
-        if (S < 2) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
-        const size_t smem = fixed + (size_t)S * stage_bytes;
-        const int grid = std::max(1, std::min(sms, a.D / kTile));
+        const size_t wbytes = (size_t)kDnRows * std::max(pr, ps);
+        const size_t stage_bytes = round_up(wbytes + (size_t)hrows * a.hrow * 2, 128);
+        const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
+        if (fixed + stage_bytes > kDecSmemMax) {
+            set_error("decode path: a %zu-byte stage does not fit shared memory", stage_bytes);
+            return MOE_ERR_SHAPE;
+        }
+        // as many consumer groups (4 warps each) as stages fit, up to 4;
+        // then up to 2 stages per group
+        const int fit = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - fixed) / stage_bytes);
+        const int G = fit >= 4 ? 4 : fit >= 2 ? 2 : 1;
+        const int Sg = std::min(2, fit / G);
+        const size_t smem = fixed + (size_t)G * Sg * stage_bytes;
+        const int U_max = (a.E + 1) * (a.D / kDnRows);
+        const int grid = std::max(1, std::min(sms, U_max));
         // no trace mark here: an event between the two kernels would cancel
         // their programmatic overlap
-        cudaError_t e = a.rows_out
-            ? launch_pdl(dec_down_kernel<NT, 4, true>, grid, smem, s, a, S, hrows, maps)
-            : launch_pdl(dec_down_kernel<NT, 4, false>, grid, smem, s, a, S, hrows, maps);
+        cudaError_t e = launch_pdl(dec_down_kernel<NT>, grid, smem, s, a, G, Sg, hrows, maps);
         if (e != cudaSuccess) return cuda_status(e, "dec_down_kernel");
+    }
+    // ---- combine (fused layer only): y = sum of the gated rows (+ shared)
+    if (a.y) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(a.T, (a.D / 4 + 255) / 256);
+        cfg.blockDim = dim3(256);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, dec_combine_kernel, (const float *)a.rows_out,
+                                           a.inv, a.T, a.k, a.D, a.sF > 0 ? 1 : 0, a.y, a.y_dtype);
+        if (e != cudaSuccess) return cuda_status(e, "dec_combine_kernel");
     }
     return MOE_OK;
 }
 
 moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, int E, int k,
-                             const int32_t *perm, const int32_t *offsets, const float *gates,
-                             const moe_pool &pool, const uint8_t *mask, const moe_pool *shared,
-                             int sF, __half *Hs, void *y, int y_dtype, float *rows_out, int *err,
-                             cudaStream_t s, Tracer *tr) {
+                             const int32_t *perm, const int32_t *inv, const int32_t *offsets,
+                             const float *gates, const moe_pool &pool, const uint8_t *mask,
+                             const moe_pool *shared, int sF, __half *Hs, void *y, int y_dtype,
+                             float *rows_out, int *err, cudaStream_t s, Tracer *tr) {
     DecArgs a{};
     a.T = T; a.D = D; a.F = F; a.E = E; a.k = k; a.sF = shared ? sF : 0;
     a.perm = perm; a.offsets = offsets; a.gates = gates; a.mask = mask;
@@ -953,8 +1012,13 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
         a.sq8 = shared->qtype == MOE_Q8_0;
     }
     a.x = x; a.x_bf16 = (x_dtype == MOE_BF16);
-    a.Hs = Hs; a.hrow = std::max(F, a.sF);
+    a.Hs = Hs; a.hrow = std::max(F, a.sF) + 32;
     a.y = y; a.y_dtype = y_dtype; a.rows_out = rows_out; a.err = err;
+    a.inv = inv;
+    if (y && !rows_out) {
+        set_error("decode path: the fused combine needs a rows buffer");
+        return MOE_ERR_INVALID_ARG;
+    }
     return T > 8 ? run_decode<2>(a, pool.n_slots, s, tr) : run_decode<1>(a, pool.n_slots, s, tr);
 }
 

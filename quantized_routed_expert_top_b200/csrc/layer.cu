@@ -34,6 +34,7 @@ static LayerWs carve(const moe_layer_args &a, Carver &c) {
     w.inv = c.take<int32_t>(Tk);
     if (decode_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0)) {
         w.Hs = c.take<__half>(decode_hs_halves(a.T, a.k, a.F, a.shared ? a.shared_F : 0));
+        w.rows = c.take<float>(decode_rows_floats(a.T, a.k, a.D));
         return w;
     }
     w.H = c.take<float>(Tk * a.F);
@@ -83,9 +84,9 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
         (st = launch_permute(ids, a.T, a.k, a.E, w.counts, w.offsets, w.perm, w.inv, s, tr)) != MOE_OK)
         return st;
     if (w.Hs) {
-        st = launch_ffn_decode(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.offsets, gates,
-                               *a.pool, nullptr, a.shared, a.shared ? a.shared_F : 0, w.Hs, a.y,
-                               a.y_dtype, nullptr, w.status, s, tr);
+        st = launch_ffn_decode(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.inv, w.offsets,
+                               gates, *a.pool, nullptr, a.shared, a.shared ? a.shared_F : 0, w.Hs,
+                               a.y, a.y_dtype, w.rows, w.status, s, tr);
         if (tr) {
             tr->end();
             if (st == MOE_OK && tr->err != cudaSuccess) {

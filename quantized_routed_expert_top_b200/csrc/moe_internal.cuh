@@ -164,11 +164,15 @@ moe_status launch_ffn_generic(const void *x, int x_dtype, int T, int D, int F, i
 // ffn_decode.cu -- TMA-streamed grouped GEMV for small T (see file header)
 bool decode_path_ok(int T, int D, int F, int sF);
 size_t decode_hs_halves(int T, int k, int F, int sF);
+size_t decode_rows_floats(int T, int k, int D);
+// y != NULL: fused layer (gates folded into the rows, rows_out is scratch
+// for [T*k + T, D] rows, combined into y); y == NULL: rows mode (rows_out =
+// un-gated Y rows [T*k, D] in permuted order, mask honoured)
 moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, int E, int k,
-                             const int32_t *perm, const int32_t *offsets, const float *gates,
-                             const moe_pool &pool, const uint8_t *mask, const moe_pool *shared,
-                             int sF, __half *Hs, void *y, int y_dtype, float *rows_out, int *err,
-                             cudaStream_t s, Tracer *tr);
+                             const int32_t *perm, const int32_t *inv, const int32_t *offsets,
+                             const float *gates, const moe_pool &pool, const uint8_t *mask,
+                             const moe_pool *shared, int sF, __half *Hs, void *y, int y_dtype,
+                             float *rows_out, int *err, cudaStream_t s, Tracer *tr);
 // combine.cu
 moe_status launch_combine(const float *rows, const int32_t *inv, const float *gates,
                           int T, int k, int D, const float *shared_rows, void *y,

@@ -249,6 +249,9 @@ route_cluster_kernel(const XT *__restrict__ x, const float *__restrict__ W,
     const int epad = (E + 31) & ~31;
     const int RS = (EPT == 1 && epad < kRouteThreads) ? kRouteThreads / epad : 1;
     const int rs = tid / epad, el = tid % epad;
+    // the expert-FFN grid that follows may launch now: it stages its
+    // activations and then waits (griddepcontrol.wait) for this grid
+    pdl_launch_dependents();
 
     float *wbuf = (float *)smem;                              // 2 chunks; later the partials
     float *xs = (float *)(smem + 2 * kRouteChunkBytes);       // [rows][TT]

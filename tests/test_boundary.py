@@ -93,7 +93,10 @@ def test_expert_ffn_rejects_unknown_and_missing_pools(moe):
     # workspace too small
     assert L.moe_expert_ffn(FAKE, moe.BF16, 4, 256, 512, 8, 2, FAKE, FAKE, C.byref(ok), None,
                             FAKE, FAKE, 16, None) == 7
-    assert L.moe_expert_ffn_workspace_size(4, 2, 256, 512) >= 4 * 2 * 512 * 4
+    # scratch for the hidden activations: fp16 rows on the small-batch path,
+    # fp32 rows on the general one (D=96 has no small-batch kernel)
+    assert L.moe_expert_ffn_workspace_size(4, 2, 256, 512) >= 4 * 2 * 512 * 2
+    assert L.moe_expert_ffn_workspace_size(4, 2, 96, 512) >= 4 * 2 * 512 * 4
 
 
 def test_combine_and_permute_errors(moe):
