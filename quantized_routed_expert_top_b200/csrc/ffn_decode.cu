@@ -56,6 +56,10 @@ constexpr int kMaxStages = 8;
 constexpr size_t kDecSmemMax = 225 * 1024;      // dynamic; leaves room for static smem
 constexpr int kDW = 16;                         // consumer warps
 constexpr int kDThreads = (kDW + 1) * 32;       // + producer warp
+constexpr int kEW = 2;                          // gate/up epilogue warps
+constexpr int kGThreads = kDThreads + kEW * 32; // gate/up block
+// gate/up partial-sum buffers between the MMA warps and the epilogue warps
+template <int NT> constexpr int gu_red_bufs() { return NT == 1 ? 4 : 3; }
 constexpr int kMaxTk = 16 * MOE_MAX_TOPK;       // T*k entries the token tables hold
 
 struct DecArgs {
@@ -161,30 +165,39 @@ struct Active {
     int n_virt;     // + 1 when a shared expert exists
 };
 
-// act: shared int[4 * (E + 1)]: expert id, segment start, token count and
-// slot of every active expert (ascending id), read once from global memory
-// so that per-unit lookups stay in shared memory.
+// act: shared int[6 * (E + 1)]: expert id, segment start, token count and
+// slot of every active expert (ascending id), then the raw offsets and
+// slots.  All threads load the raw tables in one round of global loads;
+// one warp then compacts them, so per-unit lookups stay in shared memory.
 __device__ Active build_active_list(const DecArgs &a, int *act) {
     __shared__ int s_n;
-    int *aseg = act + (a.E + 1), *acnt = aseg + (a.E + 1), *aslot = acnt + (a.E + 1);
+    const int E1 = a.E + 1;
+    int *aseg = act + E1, *acnt = aseg + E1, *aslot = acnt + E1;
+    int *roff = aslot + E1, *ron = roff + E1;
+    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) {
+        roff[e] = __ldg(a.offsets + e);
+        if (e < a.E) ron[e] = (!a.mask || __ldg(a.mask + e)) ? slot_of(a.slot_map, e) : -1;
+    }
+    __syncthreads();
     if (threadIdx.x < 32) {
         int base = 0;
         for (int e0 = 0; e0 < a.E; e0 += 32) {
-            int e = e0 + threadIdx.x;
+            const int e = e0 + threadIdx.x;
             bool on = false;
-            int s0 = 0, c = 0;
+            int s0 = 0, c = 0, sl = 0;
             if (e < a.E) {
-                s0 = __ldg(a.offsets + e);
-                c = __ldg(a.offsets + e + 1) - s0;
-                on = c > 0 && (!a.mask || __ldg(a.mask + e));
+                s0 = roff[e];
+                c = roff[e + 1] - s0;
+                sl = ron[e];
+                on = c > 0 && (!a.mask || sl >= 0);
             }
-            unsigned b = __ballot_sync(0xffffffffu, on);
+            const unsigned b = __ballot_sync(0xffffffffu, on);
             if (on) {
                 const int i = base + __popc(b & ((1u << threadIdx.x) - 1u));
                 act[i] = e;
                 aseg[i] = s0;
                 acnt[i] = c;
-                aslot[i] = slot_of(a.slot_map, e);
+                aslot[i] = sl;
             }
             base += __popc(b);
         }
@@ -338,7 +351,7 @@ __host__ __device__ inline GuGeo gu_geo(int D, bool q8, int max_sb) {
 }
 
 template <int NT, int WB4, int WB8>
-__global__ void __launch_bounds__(kDThreads, 1)
+__global__ void __launch_bounds__(kGThreads, 1)
 dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -355,29 +368,32 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
 
     // carve (from a 1024-aligned base; tensor copies need 128-byte aligned
     // destinations): xs [T+1 rows, the last zero] | Sx tables [2][T+1][nbD]
-    // | stages | red [2][kDW][NT][32][4] | barriers | act | tok | gw
+    // | stages | red [NB][kDW][NT][32][4] | barriers | act | tok | gw | units
     uint8_t *base = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
     const size_t xs_bytes = round_up((size_t)(T + 1) * xrow, 16);
     uint8_t *xs = base;
     float *sxt = (float *)(base + xs_bytes);
     uint8_t *stages = base + round_up(xs_bytes + (size_t)2 * (T + 1) * nbD * 4, 1024);
+    constexpr int NB = gu_red_bufs<NT>();
     float *red = (float *)(stages + (size_t)S * stage_bytes);
-    uint64_t *full = (uint64_t *)(red + 2 * kDW * NT * 32 * 4);
+    uint64_t *full = (uint64_t *)(red + NB * kDW * NT * 32 * 4);
     uint64_t *empty = full + kMaxStages;
-    uint64_t *rfull = empty + kMaxStages;          // [2] partials of a unit written
-    uint64_t *rempty = rfull + 2;                  // [2] a unit's epilogue done
-    int *act = (int *)(rempty + 2);
-    int *tok = act + 4 * (a.E + 1);
+    uint64_t *rfull = empty + kMaxStages;          // [4] partials of a unit written
+    uint64_t *rempty = rfull + 4;                  // [4] a unit's epilogue done
+    int *act = (int *)(rempty + 4);
+    int *tok = act + 6 * (a.E + 1);
     float *gw = (float *)(tok + kMaxTk + 16);
+    int4 *utab = reinterpret_cast<int4 *>(                 // this CTA's units
+        (reinterpret_cast<uintptr_t>(gw + kMaxTk + 16) + 15) & ~(uintptr_t)15);
 
     if (tid == 0) {
         for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kDW);
         }
-        for (int b = 0; b < 2; b++) {
-            mbar_init(&rfull[b], kDW * 32);
-            mbar_init(&rempty[b], kDW * 32);
+        for (int b = 0; b < NB; b++) {
+            mbar_init(&rfull[b], kDW);            // one elected lane per MMA warp
+            mbar_init(&rempty[b], kEW);           // one per epilogue warp
         }
         fence_mbar_init();
     }
@@ -423,18 +439,30 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     const Active A = build_active_list(a, act);   // includes __syncthreads
     const int tiles_r = a.F / kTile, tiles_s = a.sF / kTile;
     const int U = A.n_routed * tiles_r + (a.sF > 0 ? tiles_s : 0);
+    // unit table: local unit i = global unit blockIdx.x + i * gridDim.x as
+    // (virtual expert, tile, segment start, token count)
+    const int n_local = U > (int)blockIdx.x ? (U - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    for (int i = tid; i < n_local; i += blockDim.x) {
+        const int u = blockIdx.x + i * gridDim.x;
+        int v, tile;
+        if (u < A.n_routed * tiles_r) { v = u / tiles_r; tile = u % tiles_r; }
+        else { v = A.n_routed; tile = u - A.n_routed * tiles_r; }
+        const Virt vi = virt(a, act, A.n_routed, v);
+        utab[i] = make_int4(v, tile, vi.seg0, vi.cnt);
+    }
+    load_token_tables(a, tok, gw);
+    __syncthreads();
 
     if (warp == kDW) {
         // ---------------------------------------------------- producer
         // per (unit, slice): one 16-row box of gate and one of up
         if (lane == 0) {
+            const uint64_t pol = l2_evict_first_policy();    // weights: read once
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-                int v, tile;
-                if (u < A.n_routed * tiles_r) { v = u / tiles_r; tile = u % tiles_r; }
-                else { v = A.n_routed; tile = u - A.n_routed * tiles_r; }
+            for (int i = 0; i < n_local && ok; i++) {
+                const int v = utab[i].x, tile = utab[i].y;
                 const Virt vi = virt(a, act, A.n_routed, v);
                 const int bs = vi.q8 ? kQ8Bytes : kQ4Bytes;
                 const GuGeo gg = vi.q8 ? geo8 : geo4;
@@ -446,8 +474,8 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
                     uint8_t *dst = stages + (size_t)stage * stage_bytes;
                     mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * kTile * gg.pitch));
                     const int x = sl * gg.sb * bs / 8;
-                    tma_load_2d(dst, mg, x, y, &full[stage]);
-                    tma_load_2d(dst + kTile * gg.pitch, mu, x, y, &full[stage]);
+                    tma_load_2d_hint(dst, mg, x, y, &full[stage], pol);
+                    tma_load_2d_hint(dst + kTile * gg.pitch, mu, x, y, &full[stage], pol);
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
             }
@@ -460,63 +488,63 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
         return;
     }
 
-    // ------------------------------------------------------- consumers
-    load_token_tables(a, tok, gw);
-    asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
+    if (warp > kDW) {
+        // ----------------------------------------------------- epilogue
+        // unit j: the 8 K-group partials of gate and of up summed in
+        // K-group order, SwiGLU, the token's gate weight, Hs in fp16
+        const int et = tid - kDThreads;
+        for (int j = 0; j < n_local; j++) {
+            const int b = j % NB;
+            if (!mbar_wait_warp(&rfull[b], (uint32_t)((j / NB) & 1), a.err, kErrTimeoutFull)) return;
+            const int4 ud = utab[j];
+            const int tile = ud.y, seg0 = ud.z, cnt = ud.w;
+            const float *redb = red + (size_t)b * kDW * NT * 128;
+            for (int o = et; o < kTile * cnt; o += kEW * 32) {
+                const int rr = o % kTile, n = o / kTile;
+                const int nt = n >> 3, nn = n & 7;
+                const int L = (rr & 7) * 4 + (nn >> 1);
+                const int q = ((rr >> 3) << 1) | (nn & 1);
+                float sg = 0.f, su = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; w++) {
+                    sg += redb[((size_t)w * NT + nt) * 128 + L * 4 + q];
+                    su += redb[((size_t)(8 + w) * NT + nt) * 128 + L * 4 + q];
+                }
+                const int pos = seg0 + n;
+                const float h = silu(sg) * su * gw[pos];
+                const int r = tile * kTile + rr;
+                a.Hs[(size_t)pos * a.hrow + (r >> 5) * 32 + frag_slot(r & 31)] = __float2half_rn(h);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[b]);
+        }
+        return;
+    }
 
+    // ------------------------------------------------------ MMA warps
     const uint32_t xs_a = smem_u32(xs), sx_a = smem_u32(sxt), st_a = smem_u32(stages);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    // The cross-warp reduction of unit j is deferred until after unit j+1's
-    // partials are written (two partial buffers, mbarriers instead of a
-    // CTA-wide barrier), so warps that finish a unit early do not idle.
-    auto epilogue = [&](int j, const Virt &pv, int ptile) {
-        const int b = j & 1;
-        if (!mbar_wait(&rfull[b], (uint32_t)((j >> 1) & 1), a.err, kErrTimeoutFull)) { ok = false; return; }
-        const float *redb = red + (size_t)b * kDW * NT * 128;
-        const int o = tid;                               // one output per thread
-        const int rr = o % kTile, n = o / kTile;         // row within tile, column
-        if (n < pv.cnt && n < 8 * NT) {
-            const int nt = n >> 3, nn = n & 7;
-            const int L = (rr & 7) * 4 + (nn >> 1);
-            const int q = ((rr >> 3) << 1) | (nn & 1);
-            float sg = 0.f, su = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; w++) {
-                sg += redb[((size_t)w * NT + nt) * 128 + L * 4 + q];
-                su += redb[((size_t)(8 + w) * NT + nt) * 128 + L * 4 + q];
-            }
-            const int pos = pv.seg0 + n;
-            const float h = silu(sg) * su * gw[pos];
-            const int r = ptile * kTile + rr;
-            a.Hs[(size_t)pos * a.hrow + (r >> 5) * 32 + frag_slot(r & 31)] = __float2half_rn(h);
-        }
-        mbar_arrive(&rempty[b]);
-    };
-    int j = 0;
-    Virt pv{};
-    int ptile = 0;
-    for (int u = blockIdx.x; u < U && ok; u += gridDim.x, j++) {
-        int v, tile;
-        if (u < A.n_routed * tiles_r) { v = u / tiles_r; tile = u % tiles_r; }
-        else { v = A.n_routed; tile = u - A.n_routed * tiles_r; }
-        const Virt vi = virt(a, act, A.n_routed, v);
-        const int ntile = vi.cnt > 8 ? 2 : 1;
-        const GuGeo gg = vi.q8 ? geo8 : geo4;
-        const int kb0 = kg * (vi.q8 ? WB8 : WB4);       // warp's first block in a slice
+    for (int j = 0; j < n_local && ok; j++) {
+        const int4 ud = utab[j];
+        const int tile = ud.y, seg0 = ud.z, cnt = ud.w;
+        const bool q8 = ud.x < A.n_routed ? a.q8 != 0 : a.sq8 != 0;
+        const int ntile = cnt > 8 ? 2 : 1;
+        const GuGeo gg = q8 ? geo8 : geo4;
+        const int kb0 = kg * (q8 ? WB8 : WB4);          // warp's first block in a slice
         // B rows (column g, g+8) and C columns (2c, 2c+1, +8) of this unit
         uint32_t xa[NT], sa[NT][2];
-        const uint32_t sxq = sx_a + (vi.q8 ? (uint32_t)((T + 1) * nbD * 4) : 0u);
+        const uint32_t sxq = sx_a + (q8 ? (uint32_t)((T + 1) * nbD * 4) : 0u);
 #pragma unroll
         for (int nt = 0; nt < NT; nt++) {
             const int n = g + 8 * nt;
-            const int tb = n < vi.cnt ? tok[vi.seg0 + n] : T;
+            const int tb = n < cnt ? tok[seg0 + n] : T;
             xa[nt] = xs_a + tb * xrow + kb0 * 64 + c * 16;
 #pragma unroll
             for (int jj = 0; jj < 2; jj++) {
                 const int m = 8 * nt + 2 * c + jj;
-                const int tc = m < vi.cnt ? tok[vi.seg0 + m] : T;
+                const int tc = m < cnt ? tok[seg0 + m] : T;
                 sa[nt][jj] = sxq + (uint32_t)((tc * nbD + kb0) * 4);
             }
         }
@@ -525,12 +553,12 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
         for (int nt = 0; nt < NT; nt++)
 #pragma unroll
             for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
-        const int bsz = vi.q8 ? kQ8Bytes : kQ4Bytes;
+        const int bsz = q8 ? kQ8Bytes : kQ4Bytes;
         const int mis0 = (kb0 * bsz) & 3;               // 0 or 2
         const uint32_t r8 = 8u * gg.pitch;
 
         for (int sl = 0; sl < gg.nsl; sl++) {
-            if (!mbar_wait(&full[stage], phase, a.err, kErrTimeoutFull)) { ok = false; break; }
+            if (!mbar_wait_warp(&full[stage], phase, a.err, kErrTimeoutFull)) { ok = false; break; }
             const uint32_t row = st_a + stage * stage_bytes + (mat * kTile + g) * gg.pitch + kb0 * bsz;
             uint32_t xs_s[NT], sa_s[NT][2];
 #pragma unroll
@@ -540,7 +568,7 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
                 sa_s[nt][1] = sa[nt][1] + sl * gg.sb * 4;
             }
 #define MOE_GU(Q8, NTL, MIS) gateup_slice<Q8, NTL, (Q8 ? WB8 : WB4), MIS>(row, r8, xs_s, sa_s, c, acc)
-            if (!vi.q8) {
+            if (!q8) {
                 if (ntile == 1) { if (mis0 == 0) MOE_GU(false, 1, 0); else MOE_GU(false, 1, 2); }
                 else if (NT > 1) { if (mis0 == 0) MOE_GU(false, NT, 0); else MOE_GU(false, NT, 2); }
             } else {
@@ -553,9 +581,10 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
             if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        // partials of unit j into buffer j % 2, once unit j-2's epilogue is done
-        const int b = j & 1;
-        if (j >= 2 && !mbar_wait(&rempty[b], (uint32_t)(((j - 2) >> 1) & 1), a.err, kErrTimeoutEmpty)) {
+        // partials of unit j into buffer j % NB, once the epilogue of unit
+        // j - NB has read that buffer
+        const int b = j % NB;
+        if (j >= NB && !mbar_wait_warp(&rempty[b], (uint32_t)((j / NB - 1) & 1), a.err, kErrTimeoutEmpty)) {
             ok = false;
             break;
         }
@@ -564,12 +593,9 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
         for (int nt = 0; nt < NT; nt++)
 #pragma unroll
             for (int q = 0; q < 4; q++) rw[nt * 128 + lane * 4 + q] = acc[nt][q];
-        mbar_arrive(&rfull[b]);
-        if (j >= 1) epilogue(j - 1, pv, ptile);
-        pv = vi;
-        ptile = tile;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfull[b]);
     }
-    if (ok && j >= 1) epilogue(j - 1, pv, ptile);
 }
 
 // --------------------------------------------------------------------- down
@@ -670,6 +696,7 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
 
     if (warp == kDW) {
         if (lane == 0) {
+            const uint64_t pol = l2_evict_first_policy();    // weights: read once
             bool ok = true, waited = false;
             int pend_s[kMaxStages], pend_v[kMaxStages];
             int npend = 0;
@@ -687,8 +714,8 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
                 if (!mbar_wait(&empty[sl.stage], sl.phase ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
                 uint8_t *dst = stages + (size_t)sl.stage * stage_bytes;
                 mbar_arrive_expect_tx(&full[sl.stage], (uint32_t)(kDnRows * pitch + vi.cnt * hbytes));
-                tma_load_2d(dst, vi.shared ? &maps.sdown : &maps.down, 0,
-                            (vi.shared ? 0 : (int)vi.slot * D) + dt * kDnRows, &full[sl.stage]);
+                tma_load_2d_hint(dst, vi.shared ? &maps.sdown : &maps.down, 0,
+                                 (vi.shared ? 0 : (int)vi.slot * D) + dt * kDnRows, &full[sl.stage], pol);
                 if (waited) {
                     issue_h(sl.stage, v);
                 } else {
@@ -733,7 +760,7 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
         for (int nt = 0; nt < NT; nt++)
 #pragma unroll
             for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
-        if (!mbar_wait(&full[sl.stage], sl.phase, a.err, kErrTimeoutFull)) break;
+        if (!mbar_wait_warp(&full[sl.stage], sl.phase, a.err, kErrTimeoutFull)) break;
         const uint32_t sbase = st_a + sl.stage * stage_bytes;
         uint32_t row = sbase + (mt * kTile + g) * pitch;
         const uint32_t r8 = 8u * pitch;
@@ -878,11 +905,11 @@ static moe_status encode_maps(const DecArgs &a, int n_slots, int max_sb, DecMaps
 }
 
 template <typename... Args>
-static cudaError_t launch_pdl(void (*kern)(Args...), int grid, size_t smem, cudaStream_t s,
-                             Args... args) {
+static cudaError_t launch_pdl(void (*kern)(Args...), int grid, int block, size_t smem,
+                             cudaStream_t s, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kDThreads);
+    cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -895,19 +922,26 @@ static cudaError_t launch_pdl(void (*kern)(Args...), int grid, size_t smem, cuda
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// the gate/up kernel's per-CTA unit table (16 bytes a unit)
+static size_t unit_table_bytes(const DecArgs &a, int sms) {
+    const int U_max = a.E * (a.F / kTile) + a.sF / kTile;
+    const int grid = std::max(1, std::min(sms, U_max));
+    return (size_t)((U_max + grid - 1) / grid) * 16 + 16;
+}
+
 static size_t tables_bytes(int E) {
-    return 4 * (size_t)(E + 1) * sizeof(int) + (size_t)(kMaxTk + 16) * (sizeof(int) + sizeof(float));
+    return 6 * (size_t)(E + 1) * sizeof(int) + (size_t)(kMaxTk + 16) * (sizeof(int) + sizeof(float));
 }
 
 template <int NT>
 static cudaError_t launch_gateup(const DecArgs &a, const DecMaps &m, int grid, size_t smem,
                                  cudaStream_t s, int S) {
     switch (a.D) {
-    case 256: return launch_pdl(dec_gateup_kernel<NT, 1, 1>, grid, smem, s, a, S, m);
-    case 512: return launch_pdl(dec_gateup_kernel<NT, 2, 2>, grid, smem, s, a, S, m);
-    case 768: return launch_pdl(dec_gateup_kernel<NT, 3, 3>, grid, smem, s, a, S, m);
-    case 1024: return launch_pdl(dec_gateup_kernel<NT, 4, 4>, grid, smem, s, a, S, m);
-    default: return launch_pdl(dec_gateup_kernel<NT, (NT == 1 ? 8 : 4), 4>, grid, smem, s, a, S, m);
+    case 256: return launch_pdl(dec_gateup_kernel<NT, 1, 1>, grid, kGThreads, smem, s, a, S, m);
+    case 512: return launch_pdl(dec_gateup_kernel<NT, 2, 2>, grid, kGThreads, smem, s, a, S, m);
+    case 768: return launch_pdl(dec_gateup_kernel<NT, 3, 3>, grid, kGThreads, smem, s, a, S, m);
+    case 1024: return launch_pdl(dec_gateup_kernel<NT, 4, 4>, grid, kGThreads, smem, s, a, S, m);
+    default: return launch_pdl(dec_gateup_kernel<NT, (NT == 1 ? 8 : 4), 4>, grid, kGThreads, smem, s, a, S, m);
     }
 }
 
@@ -928,8 +962,9 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         // mirrors the kernel's carve; + 1024 for aligning the base
         const size_t fixed = round_up(round_up((size_t)(a.T + 1) * staged_act_bytes(a.D), 16) +
                                       (size_t)2 * (a.T + 1) * nbD * 4, 1024) +
-                             (size_t)2 * kDW * NT * 32 * 4 * sizeof(float) +
-                             (2 * kMaxStages + 4) * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
+                             (size_t)gu_red_bufs<NT>() * kDW * NT * 32 * 4 * sizeof(float) +
+                             (2 * kMaxStages + 8) * sizeof(uint64_t) + tables_bytes(a.E) +
+                             unit_table_bytes(a, sms) + 1024;
         if (fixed >= kDecSmemMax) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
         int S = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - fixed) / stage_bytes);
         if (S < 2) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
@@ -962,7 +997,7 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         const int grid = std::max(1, std::min(sms, U_max));
         // no trace mark here: an event between the two kernels would cancel
         // their programmatic overlap
-        cudaError_t e = launch_pdl(dec_down_kernel<NT>, grid, smem, s, a, G, Sg, hrows, maps);
+        cudaError_t e = launch_pdl(dec_down_kernel<NT>, grid, kDThreads, smem, s, a, G, Sg, hrows, maps);
         if (e != cudaSuccess) return cuda_status(e, "dec_down_kernel");
     }
     // ---- combine (fused layer only): y = sum of the gated rows (+ shared)

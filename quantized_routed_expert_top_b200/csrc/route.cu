@@ -32,33 +32,51 @@ constexpr int kSplitMaxT = 16;      // tokens handled by the split-K path
 constexpr int kSplitRows = 32;      // D rows per split CTA
 
 // --------------------------------------------------------------- selection
+// Orderable key of a logit: a larger value gives a larger unsigned key; -0
+// and +0 share one key, so equal logits tie and the lower id wins.
+__device__ __forceinline__ unsigned order_key(float v) {
+    const unsigned b = __float_as_uint(v == 0.0f ? 0.0f : v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // One warp selects the top-k of a logit row L[0..E) (any memory space) and
-// writes ids/gates for that token.  E <= 1024 (32 values per lane), k <= 32.
+// writes ids/gates for that token (and the ids to ids_copy when given).
+// E <= 1024 (32 values per lane), k <= 32.  Each lane keeps its best
+// remaining candidate; a round is two warp reductions (largest key, then
+// the lowest id holding it) and only the winning lane rescans its values.
 __device__ void warp_select(const float *L, int E, int k, int renorm,
-                            int32_t *ids_out, float *gates_out) {
+                            int32_t *ids_out, float *gates_out, int32_t *ids_copy = nullptr) {
     const int lane = threadIdx.x & 31;
     const int per_lane = (E + 31) >> 5;
     unsigned taken = 0u;
-    float my_v = -INFINITY;
-    int my_i = INT_MAX;
-    for (int j = 0; j < k; j++) {
-        float bv = -INFINITY;
-        int bi = INT_MAX;
+    float bv = -INFINITY;
+    int bi = INT_MAX;
+    auto local_best = [&]() {
+        bv = -INFINITY;
+        bi = INT_MAX;
         for (int i = 0; i < per_lane; i++) {
-            int e = lane + 32 * i;
+            const int e = lane + 32 * i;
             if (e < E && !((taken >> i) & 1u)) {
-                float v = L[e];
+                const float v = L[e];
                 if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    };
+    local_best();
+    float my_v = -INFINITY;
+    int my_i = INT_MAX;
+    for (int j = 0; j < k; j++) {
+        const unsigned key = (bi == INT_MAX) ? 0u : order_key(bv);
+        const unsigned kmax = __reduce_max_sync(0xffffffffu, key);
+        const unsigned cand = (bi != INT_MAX && key == kmax) ? (unsigned)bi : 0xffffffffu;
+        const unsigned win = __reduce_min_sync(0xffffffffu, cand);
+        const int wi = (win == 0xffffffffu) ? INT_MAX : (int)win;
+        const float wv = __shfl_sync(0xffffffffu, bv, wi == INT_MAX ? 0 : (wi & 31));
+        if (lane == j) { my_v = (wi == INT_MAX) ? -INFINITY : wv; my_i = wi; }
+        if (wi != INT_MAX && (wi & 31) == lane) {
+            taken |= 1u << (wi >> 5);
+            local_best();
         }
-        if (bi != INT_MAX && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == j) { my_v = bv; my_i = bi; }
     }
     // gates: lane j < k holds selection j; the first selection is the max
     const float m = __shfl_sync(0xffffffffu, my_v, 0);
@@ -77,6 +95,7 @@ __device__ void warp_select(const float *L, int E, int k, int renorm,
     if (lane < k) {
         ids_out[lane] = my_i;
         gates_out[lane] = ex / denom;
+        if (ids_copy) ids_copy[lane] = my_i;
     }
 }
 
@@ -207,93 +226,102 @@ route_select_kernel(const float *__restrict__ logits, const float *__restrict__ 
 }
 
 // ------------------------------------ small T: one cluster, DSMEM reduction
-// The D rows of W_r are split over the CS CTAs of one thread-block cluster.
-// Each CTA pulls its contiguous slab of W_r with bulk async copies (double
-// buffered), computes partial logits for all T tokens and E experts, and
-// keeps them in its shared memory.  After a cluster barrier, CTA r
-// finalises tokens t = r, r + CS, ...: it adds the CS partials of the token
-// in rank order through distributed shared memory (deterministic), adds the
-// bias and selects.  Optionally CTA 0 then gathers every token's ids through
-// DSMEM and runs the stable permutation, so the whole routing + grouping is
-// one launch.
+// Latency-bound: at T <= 16 the router reads W_r (D*E*4 bytes, 1 MiB at
+// D=2048, E=128) once and does T FMAs per weight, so what matters is how
+// many dependent memory round trips the critical path holds.  One cluster
+// of CS CTAs:
+//  1. CTA r takes rows [r*rpc, (r+1)*rpc) of W_r.  Thread (row group rg,
+//     expert quad q) issues all its 16-byte row loads at once, then does
+//     the FMAs for every token; the row groups are summed in a fixed order
+//     in shared memory: CTA partial P_r[t][e].
+//  2. cluster barrier; CTA r finalises tokens t = r, r + CS, ...: the CS
+//     partials of the token are added in rank order through distributed
+//     shared memory (deterministic), plus the bias (prefetched at start),
+//     and one warp selects.  The selected ids are also stored straight into
+//     CTA 0's shared memory.
+//  3. cluster barrier; CTA 0 runs the stable permutation over all ids.
 constexpr int kClusterCTAs = 16;
 constexpr int kRouteThreads = 256;
-constexpr int kRouteChunkBytes = 32 * 1024;
+constexpr int kRouteBatch = 16;      // 16-byte W_r loads in flight per thread
 
 namespace cg = cooperative_groups;
 
-template <typename XT, int EPT, int TT>
+struct RouteGeo {
+    int rpc, Q, RG;                    // rows per CTA, expert quads, row groups
+};
+// the row-group sums; later (CTA 0) the permutation histograms [8][E]
+__host__ __device__ inline size_t route_red_floats(const RouteGeo &g, int TT, int E) {
+    const size_t a = (size_t)g.RG * TT * E, b = (size_t)8 * E;
+    return a > b ? a : b;
+}
+__host__ __device__ inline RouteGeo route_geo(int D, int E) {
+    RouteGeo g;
+    g.rpc = (D + kClusterCTAs - 1) / kClusterCTAs;
+    g.Q = E / 4;
+    g.RG = kRouteThreads / g.Q;
+    return g;
+}
+
+template <typename XT, int TT>
 __global__ void __launch_bounds__(kRouteThreads)
 route_cluster_kernel(const XT *__restrict__ x, const float *__restrict__ W,
                      const float *__restrict__ bias, int T, int D, int E, int k, int renorm,
                      int32_t *__restrict__ ids, float *__restrict__ gates,
                      float *__restrict__ logits_out, int32_t *__restrict__ counts,
                      int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
-                     int32_t *__restrict__ inv, int *__restrict__ err) {
+                     int32_t *__restrict__ inv) {
     // TT: tokens rounded up to 1, 2, 4, 8 or 16 (padding tokens are zero)
     extern __shared__ __align__(128) uint8_t smem_rc[];
-    uint8_t *smem = smem_rc;
-    __shared__ __align__(8) uint64_t bar[2];
     __shared__ int32_t scratch[32 + 8 * 32 + 1];
     constexpr int CS = kClusterCTAs;
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int tid = threadIdx.x;
-    const int rpc = (D + CS - 1) / CS;
-    const int r0 = min(D, rank * rpc), r1 = min(D, r0 + rpc);
+    const RouteGeo geo = route_geo(D, E);
+    const int r0 = min(D, rank * geo.rpc), r1 = min(D, r0 + geo.rpc);
     const int rows = r1 - r0;
-    const int ch = max(1, kRouteChunkBytes / (E * 4));      // rows per chunk
-    const int nch = (rows + ch - 1) / ch;
-    // threads: EPT experts each; when E is small, RS groups of threads split
-    // the rows of every chunk (summed in a fixed order afterwards)
-    const int epad = (E + 31) & ~31;
-    const int RS = (EPT == 1 && epad < kRouteThreads) ? kRouteThreads / epad : 1;
-    const int rs = tid / epad, el = tid % epad;
+    const int q = tid % geo.Q, rg = tid / geo.Q;
     // the expert-FFN grid that follows may launch now: it stages its
     // activations and then waits (griddepcontrol.wait) for this grid
     pdl_launch_dependents();
 
-    float *wbuf = (float *)smem;                              // 2 chunks; later the partials
-    float *xs = (float *)(smem + 2 * kRouteChunkBytes);       // [rows][TT]
-    float *Lrow = xs + (size_t)rpc * TT;                      // [E]
-    int32_t *ids_s = (int32_t *)(Lrow + E);                   // [T * k] (own tokens)
-    int32_t *ids_all = ids_s + T * k;                         // [T * k] (rank 0)
-    int32_t *hist = ids_all + T * k;                          // [8 * E]   (rank 0)
-    float *rsum = (float *)hist;                              // [RS][TT][E] before the finalise
+    float *xs = (float *)smem_rc;                             // [rpc][TT]
+    float *red = xs + round_up((size_t)geo.rpc * TT, 4);      // [RG][TT][E]; red[0] = P_r
+    float *bias_s = red + route_red_floats(geo, TT, E);       // [E]
+    float *Lrow = bias_s + E;                                 // [E]
+    int32_t *ids_all = (int32_t *)(Lrow + E);                 // [T * k] (rank 0)
+    int32_t *hist = (int32_t *)red;                           // [8 * E] (rank 0, after step 2)
 
-    if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    auto issue = [&](int c) {
-        const int rr = r0 + c * ch, n = min(ch, r1 - rr);
-        const uint32_t bytes = (uint32_t)(n * E * 4);
-        mbar_arrive_expect_tx(&bar[c & 1], bytes);
-        bulk_g2s(wbuf + (size_t)(c & 1) * (kRouteChunkBytes / 4), W + (size_t)rr * E, bytes, &bar[c & 1]);
-    };
-    if (tid == 0) {
-        if (nch > 0) issue(0);
-        if (nch > 1) issue(1);
-    }
+    // activations of this CTA's rows and the bias: first loads in flight
     for (int i = tid; i < rows * TT; i += kRouteThreads) {
         const int r = i / TT, t = i % TT;
         xs[i] = (t < T) ? load_act(x, (size_t)t * D + r0 + r) : 0.f;
     }
-    __syncthreads();
+    for (int e = tid; e < E; e += kRouteThreads) bias_s[e] = bias ? __ldg(bias + e) : 0.f;
 
-    float acc[EPT][TT];
+    float acc[4][TT];
 #pragma unroll
-    for (int q = 0; q < EPT; q++)
+    for (int j = 0; j < 4; j++)
 #pragma unroll
-        for (int t = 0; t < TT; t++) acc[q][t] = 0.f;
-    for (int c = 0; c < nch; c++) {
-        mbar_wait(&bar[c & 1], (c >> 1) & 1, err, kErrTimeoutFull);
-        const float *wb = wbuf + (size_t)(c & 1) * (kRouteChunkBytes / 4);
-        const int n = min(ch, r1 - (r0 + c * ch));
-        for (int r = (RS > 1 ? rs : 0); r < n; r += RS) {
-            const float *xr = xs + (size_t)(c * ch + r) * TT;
+        for (int t = 0; t < TT; t++) acc[j][t] = 0.f;
+    const bool active = rg < geo.RG;
+    const int my_rows = active ? (rows - rg + geo.RG - 1) / geo.RG : 0;
+    const float4 *Wq = reinterpret_cast<const float4 *>(W + (size_t)(r0 + rg) * E) + q;
+    const size_t wstep = (size_t)geo.RG * E / 4;              // float4s between my rows
+    bool synced = false;
+    for (int b0 = 0; b0 < my_rows || !synced; b0 += kRouteBatch) {
+        float4 w[kRouteBatch];
+#pragma unroll
+        for (int i = 0; i < kRouteBatch; i++)
+            if (b0 + i < my_rows) w[i] = __ldg(Wq + (size_t)(b0 + i) * wstep);
+        if (!synced) {                     // xs complete (its loads were issued first)
+            __syncthreads();
+            synced = true;
+        }
+#pragma unroll
+        for (int i = 0; i < kRouteBatch; i++) {
+            if (b0 + i >= my_rows) break;
+            const float *xr = xs + (size_t)(rg + (b0 + i) * geo.RG) * TT;
             float xv[TT];
             if constexpr (TT % 4 == 0) {
 #pragma unroll
@@ -306,75 +334,52 @@ route_cluster_kernel(const XT *__restrict__ x, const float *__restrict__ W,
                 for (int t = 0; t < TT; t++) xv[t] = xr[t];
             }
 #pragma unroll
-            for (int q = 0; q < EPT; q++) {
-                const int e = (RS > 1 ? el : tid) + q * kRouteThreads;
-                if (e < E) {
-                    const float w = wb[r * E + e];
-#pragma unroll
-                    for (int t = 0; t < TT; t++) acc[q][t] = fmaf(xv[t], w, acc[q][t]);
-                }
+            for (int t = 0; t < TT; t++) {
+                acc[0][t] = fmaf(xv[t], w[i].x, acc[0][t]);
+                acc[1][t] = fmaf(xv[t], w[i].y, acc[1][t]);
+                acc[2][t] = fmaf(xv[t], w[i].z, acc[2][t]);
+                acc[3][t] = fmaf(xv[t], w[i].w, acc[3][t]);
             }
         }
-        __syncthreads();                   // everyone is done with this buffer
-        if (tid == 0 && c + 2 < nch) issue(c + 2);
     }
-    // partial logits of this CTA's rows: [T][E], in the (now free) W buffers
-    float *part = wbuf;
-    if (RS > 1) {
-        if (el < E)
+    // row groups -> P_r[t][e] (= red[0]), summed in row-group order
+    if (active)
 #pragma unroll
-            for (int t = 0; t < TT; t++) rsum[((size_t)rs * TT + t) * E + el] = acc[0][t];
-        __syncthreads();
+        for (int t = 0; t < TT; t++)
+            *reinterpret_cast<float4 *>(red + ((size_t)rg * TT + t) * E + 4 * q) =
+                make_float4(acc[0][t], acc[1][t], acc[2][t], acc[3][t]);
+    __syncthreads();
+    if (geo.RG > 1)
         for (int i = tid; i < T * E; i += kRouteThreads) {
-            const int t = i / E, e = i % E;
-            float v = 0.f;
-            for (int q = 0; q < RS; q++) v += rsum[((size_t)q * TT + t) * E + e];
-            part[i] = v;
+            float v = red[i];
+            for (int g = 1; g < geo.RG; g++) v += red[(size_t)g * TT * E + i];
+            red[i] = v;
         }
-    } else {
-#pragma unroll
-        for (int q = 0; q < EPT; q++) {
-            const int e = tid + q * kRouteThreads;
-            if (e < E)
-#pragma unroll
-                for (int t = 0; t < TT; t++)
-                    if (t < T) part[t * E + e] = acc[q][t];
-        }
-    }
     cluster.sync();
 
     // finalise this CTA's tokens: partials summed in rank order (DSMEM)
+    int32_t *ids0 = cluster.map_shared_rank(ids_all, 0);
     for (int t = rank; t < T; t += CS) {
         for (int e = tid; e < E; e += kRouteThreads) {
             float pv[CS];
 #pragma unroll
-            for (int q = 0; q < CS; q++) pv[q] = cluster.map_shared_rank(part, q)[t * E + e];
+            for (int r = 0; r < CS; r++) pv[r] = cluster.map_shared_rank(red, r)[t * E + e];
             float v = 0.f;
 #pragma unroll
-            for (int q = 0; q < CS; q++) v += pv[q];
-            if (bias) v += __ldg(bias + e);
+            for (int r = 0; r < CS; r++) v += pv[r];
+            v += bias_s[e];
             Lrow[e] = v;
             if (logits_out) logits_out[(size_t)t * E + e] = v;
         }
         __syncthreads();
-        if (tid < 32) warp_select(Lrow, E, k, renorm, ids + (size_t)t * k, gates + (size_t)t * k);
-        if (tid < 32 && perm) {
-            // keep a copy of this token's ids for the permutation gather
-            __syncwarp();
-            if (tid < k) ids_s[t * k + tid] = __ldcg(ids + (size_t)t * k + tid);
-        }
+        if (tid < 32)
+            warp_select(Lrow, E, k, renorm, ids + (size_t)t * k, gates + (size_t)t * k,
+                        perm ? ids0 + t * k : nullptr);
         __syncthreads();
     }
-    cluster.sync();                        // ids visible cluster-wide; partials no longer read
-    if (perm && rank == 0) {
-        for (int i = tid; i < T * k; i += kRouteThreads) {
-            const int t = i / k;
-            ids_all[i] = cluster.map_shared_rank(ids_s, t % CS)[i];
-        }
-        __syncthreads();
+    cluster.sync();                        // ids in CTA 0; partials no longer read
+    if (perm && rank == 0)
         block_permute<kRouteThreads / 32>(ids_all, T * k, E, hist, scratch, counts, offsets, perm, inv);
-    }
-    cluster.sync();                        // no CTA exits while rank 0 may read its ids
 }
 
 // ------------------------------------------ given logits: select + permute
@@ -425,30 +430,27 @@ size_t route_ws_bytes(int T, int D, int E, int k) {
 static int t_bucket(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 8 ? 8 : 16; }
 
 static size_t cluster_smem_bytes(int T, int D, int E, int k) {
-    const int rpc = (D + kClusterCTAs - 1) / kClusterCTAs;
+    const RouteGeo g = route_geo(D, E);
     const int TT = t_bucket(T);
-    const int epad = (E + 31) & ~31;
-    const int RS = (epad < kRouteThreads) ? kRouteThreads / epad : 1;
-    const size_t tail = std::max((size_t)8 * E * 4, (size_t)RS * TT * E * 4);
-    return 2 * (size_t)kRouteChunkBytes + (size_t)rpc * TT * 4 + (size_t)E * 4 +
-           2 * (size_t)T * k * 4 + tail + 256;
+    return (round_up((size_t)g.rpc * TT, 4) + route_red_floats(g, TT, E) + 2 * (size_t)E) * 4 +
+           (size_t)T * k * 4 + 256;
 }
 
 static bool cluster_route_ok(int T, int D, int E, int k, const void *w_router) {
-    return w_router && T >= 1 && T <= kSplitMaxT && E % 4 == 0 && E * 4 <= kRouteChunkBytes &&
-           T * E * 4 <= 2 * kRouteChunkBytes && cluster_smem_bytes(T, D, E, k) <= 200 * 1024;
+    return w_router && T >= 1 && T <= kSplitMaxT && E % 4 == 0 && E / 4 <= kRouteThreads &&
+           cluster_smem_bytes(T, D, E, k) <= 200 * 1024;
 }
 
 static bool select_permute_ok(int T, int E, int k) {
     return (size_t)T * E * 4 + (size_t)T * k * 4 + 8 * (size_t)E * 4 <= 200 * 1024 && T <= 64;
 }
 
-template <typename XT, int EPT, int TT>
+template <typename XT, int TT>
 static cudaError_t launch_cluster(const void *x, const float *W, const float *bias, int T, int D,
                                   int E, int k, int renorm, int32_t *ids, float *gates,
                                   float *logits, int32_t *counts, int32_t *offsets, int32_t *perm,
-                                  int32_t *inv, int *err, cudaStream_t s) {
-    auto kern = route_cluster_kernel<XT, EPT, TT>;
+                                  int32_t *inv, cudaStream_t s) {
+    auto kern = route_cluster_kernel<XT, TT>;
     const size_t sm = cluster_smem_bytes(T, D, E, k);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
@@ -467,7 +469,7 @@ static cudaError_t launch_cluster(const void *x, const float *W, const float *bi
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, (const XT *)x, W, bias, T, D, E, k, renorm, ids, gates,
-                              logits, counts, offsets, perm, inv, err);
+                              logits, counts, offsets, perm, inv);
 }
 
 moe_status launch_route_permute(const void *x, int x_dtype, const float *w_router,
@@ -479,25 +481,16 @@ moe_status launch_route_permute(const void *x, int x_dtype, const float *w_route
     *permuted = false;
     if (cluster_route_ok(T, D, E, k, w_router)) {
         mark(tr, MOE_KERNEL_ROUTE);
-        const int ept = (E + kRouteThreads - 1) / kRouteThreads;
         cudaError_t e;
         const bool bf = x_dtype == MOE_BF16;
         const int tt = t_bucket(T);
-#define MOE_CL(EP, TB)                                                                            \
-    e = bf ? launch_cluster<__nv_bfloat16, EP, TB>(x, w_router, bias, T, D, E, k, renorm, ids,    \
-                                                   gates, logits, counts, offsets, perm, inv,     \
-                                                   err, s)                                        \
-           : launch_cluster<float, EP, TB>(x, w_router, bias, T, D, E, k, renorm, ids, gates,     \
-                                           logits, counts, offsets, perm, inv, err, s)
-#define MOE_CL_T(EP)                                                                              \
-    do {                                                                                          \
-        if (tt == 1) MOE_CL(EP, 1); else if (tt == 2) MOE_CL(EP, 2);                              \
-        else if (tt == 4) MOE_CL(EP, 4); else if (tt == 8) MOE_CL(EP, 8); else MOE_CL(EP, 16);   \
-    } while (0)
-        if (ept == 1) MOE_CL_T(1);
-        else if (ept == 2) MOE_CL_T(2);
-        else MOE_CL_T(4);
-#undef MOE_CL_T
+#define MOE_CL(TB)                                                                                \
+    e = bf ? launch_cluster<__nv_bfloat16, TB>(x, w_router, bias, T, D, E, k, renorm, ids, gates, \
+                                               logits, counts, offsets, perm, inv, s)             \
+           : launch_cluster<float, TB>(x, w_router, bias, T, D, E, k, renorm, ids, gates, logits, \
+                                       counts, offsets, perm, inv, s)
+        if (tt == 1) MOE_CL(1); else if (tt == 2) MOE_CL(2); else if (tt == 4) MOE_CL(4);
+        else if (tt == 8) MOE_CL(8); else MOE_CL(16);
 #undef MOE_CL
         if (e != cudaSuccess) return cuda_status(e, "route_cluster_kernel");
         *permuted = perm != nullptr;

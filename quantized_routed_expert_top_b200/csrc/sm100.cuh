@@ -66,6 +66,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     return true;
 }
 
+// mbar_wait by every lane of a warp with one outcome for the whole warp (a
+// lane that timed out makes all lanes report the timeout), so warp-wide
+// synchronisation after it never waits for a lane that left.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, int *err, int code) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, err, code));
+}
+
 // Bulk async copy global -> shared (TMA engine), completion counted in bytes
 // on `bar`.  dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -84,6 +91,27 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, 
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// L2 eviction priority for data read once per call (expert weights): lines
+// loaded under this policy are the first candidates for replacement, so a
+// weight stream far larger than L2 does not push out what the following
+// kernels reuse (their code, the router weights, activations, routing
+// tables).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// tma_load_2d with an L2 cache-policy hint
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const void *tmap, int x, int y,
+                                                 uint64_t *bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
 
