@@ -99,6 +99,59 @@ __device__ void warp_select(const float *L, int E, int k, int renorm,
     }
 }
 
+// All threads of a block select the top-k of one token's logits L[0..E)
+// (shared memory): each element's rank is the number of elements that beat
+// it (larger logit, or equal logit and lower id); ranks below k are the
+// selection, in order.  One pass of compares instead of k dependent warp
+// reductions.  NaN logits are never selected.  key: shared uint32[E];
+// sel_v / sel_i: shared [32].  Writes ids/gates (and ids_copy) for the
+// token; ends with the block synchronised.
+__device__ void block_select(const float *L, unsigned *key, float *sel_v, int *sel_i, int E, int k,
+                             int renorm, int32_t *ids_out, float *gates_out, int32_t *ids_copy) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const float v = L[e];
+        key[e] = (v != v) ? 0u : order_key(v);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const unsigned kv = key[e];
+        if (kv == 0u) continue;                       // NaN
+        int r = 0;
+#pragma unroll 4
+        for (int e2 = 0; e2 < E; e2++) {
+            const unsigned kw = key[e2];
+            r += (kw > kv) | ((kw == kv) & (e2 < e));
+        }
+        if (r < k) {
+            sel_i[r] = e;
+            sel_v[r] = L[e];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const float my_v = (lane < k) ? sel_v[lane] : -INFINITY;
+        const int my_i = (lane < k) ? sel_i[lane] : INT_MAX;
+        // gates exactly as warp_select computes them
+        const float m = __shfl_sync(0xffffffffu, my_v, 0);
+        float ex = (lane < k) ? expf(my_v - m) : 0.0f;
+        float denom;
+        if (renorm) {
+            denom = warp_sum(ex);
+        } else {
+            float z = 0.0f;
+            for (int e = lane; e < E; e += 32) z += expf(L[e] - m);
+            denom = warp_sum(z);
+        }
+        if (lane < k) {
+            ids_out[lane] = my_i;
+            gates_out[lane] = ex / denom;
+            if (ids_copy) ids_copy[lane] = my_i;
+        }
+    }
+    __syncthreads();
+}
+
 // ------------------------------------------------- small T: split-K + select
 template <typename XT>
 __global__ void __launch_bounds__(1024)
@@ -237,8 +290,8 @@ route_select_kernel(const float *__restrict__ logits, const float *__restrict__ 
 //  2. cluster barrier; CTA r finalises tokens t = r, r + CS, ...: the CS
 //     partials of the token are added in rank order through distributed
 //     shared memory (deterministic), plus the bias (prefetched at start),
-//     and one warp selects.  The selected ids are also stored straight into
-//     CTA 0's shared memory.
+//     and the whole CTA selects by ranks.  The selected ids are also stored
+//     straight into CTA 0's shared memory.
 //  3. cluster barrier; CTA 0 runs the stable permutation over all ids.
 constexpr int kClusterCTAs = 16;
 constexpr int kRouteThreads = 256;
@@ -289,7 +342,10 @@ route_cluster_kernel(const XT *__restrict__ x, const float *__restrict__ W,
     float *red = xs + round_up((size_t)geo.rpc * TT, 4);      // [RG][TT][E]; red[0] = P_r
     float *bias_s = red + route_red_floats(geo, TT, E);       // [E]
     float *Lrow = bias_s + E;                                 // [E]
-    int32_t *ids_all = (int32_t *)(Lrow + E);                 // [T * k] (rank 0)
+    unsigned *key = (unsigned *)(Lrow + E);                   // [E]
+    float *sel_v = (float *)(key + E);                        // [32]
+    int32_t *sel_i = (int32_t *)(sel_v + 32);                 // [32]
+    int32_t *ids_all = sel_i + 32;                            // [T * k] (rank 0)
     int32_t *hist = (int32_t *)red;                           // [8 * E] (rank 0, after step 2)
 
     // activations of this CTA's rows and the bias: first loads in flight
@@ -372,10 +428,8 @@ route_cluster_kernel(const XT *__restrict__ x, const float *__restrict__ W,
             if (logits_out) logits_out[(size_t)t * E + e] = v;
         }
         __syncthreads();
-        if (tid < 32)
-            warp_select(Lrow, E, k, renorm, ids + (size_t)t * k, gates + (size_t)t * k,
-                        perm ? ids0 + t * k : nullptr);
-        __syncthreads();
+        block_select(Lrow, key, sel_v, sel_i, E, k, renorm, ids + (size_t)t * k, gates + (size_t)t * k,
+                     perm ? ids0 + t * k : nullptr);
     }
     cluster.sync();                        // ids in CTA 0; partials no longer read
     if (perm && rank == 0)
@@ -432,7 +486,7 @@ static int t_bucket(int T) { return T <= 1 ? 1 : T <= 2 ? 2 : T <= 4 ? 4 : T <= 
 static size_t cluster_smem_bytes(int T, int D, int E, int k) {
     const RouteGeo g = route_geo(D, E);
     const int TT = t_bucket(T);
-    return (round_up((size_t)g.rpc * TT, 4) + route_red_floats(g, TT, E) + 2 * (size_t)E) * 4 +
+    return (round_up((size_t)g.rpc * TT, 4) + route_red_floats(g, TT, E) + 3 * (size_t)E + 64) * 4 +
            (size_t)T * k * 4 + 256;
 }
 
