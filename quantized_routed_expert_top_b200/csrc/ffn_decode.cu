@@ -59,7 +59,10 @@ constexpr int kDThreads = (kDW + 1) * 32;       // + producer warp
 constexpr int kEW = 2;                          // gate/up epilogue warps
 constexpr int kGThreads = kDThreads + kEW * 32; // gate/up block
 // gate/up partial-sum buffers between the MMA warps and the epilogue warps
-template <int NT> constexpr int gu_red_bufs() { return NT == 1 ? 4 : 3; }
+constexpr int kGuRedBufs = 2;
+// gate/up units cover at most 8 tokens of an expert (one MMA N tile); an
+// expert with more tokens gets one unit per 8-token column group
+constexpr int kGuCols = 8;
 constexpr int kMaxTk = 16 * MOE_MAX_TOPK;       // T*k entries the token tables hold
 
 struct DecArgs {
@@ -339,8 +342,7 @@ __device__ __forceinline__ void gateup_slice(uint32_t row, uint32_t r8, const ui
 struct GuGeo {
     int sb, nsl, pitch;                 // blocks per slice, slices, staged row pitch
 };
-// max_sb: 64 for T <= 8; 32 for larger T, whose activation tables leave
-// room for fewer stages (smaller slices keep the ring deeper)
+// max_sb: the largest slice (in blocks) a stage may hold
 __host__ __device__ inline GuGeo gu_geo(int D, bool q8, int max_sb) {
     const int bs = q8 ? kQ8Bytes : kQ4Bytes, nb = D / QK;
     GuGeo g;
@@ -350,15 +352,16 @@ __host__ __device__ inline GuGeo gu_geo(int D, bool q8, int max_sb) {
     return g;
 }
 
-template <int NT, int WB4, int WB8>
+template <int MAXSB, int WB4, int WB8>
 __global__ void __launch_bounds__(kGThreads, 1)
 dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
+    constexpr int NT = 1;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
     const int T = a.T, D = a.D;
     const int nbD = D / QK;
-    constexpr int kMaxSb = NT == 1 ? 64 : 32;
+    constexpr int kMaxSb = MAXSB;
     const GuGeo geo4 = gu_geo(D, false, kMaxSb), geo8 = gu_geo(D, true, kMaxSb);
     const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
     const int pitch_max = max(any4 ? geo4.pitch : 0, any8 ? geo8.pitch : 0);
@@ -374,7 +377,7 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     uint8_t *xs = base;
     float *sxt = (float *)(base + xs_bytes);
     uint8_t *stages = base + round_up(xs_bytes + (size_t)2 * (T + 1) * nbD * 4, 1024);
-    constexpr int NB = gu_red_bufs<NT>();
+    constexpr int NB = kGuRedBufs;
     float *red = (float *)(stages + (size_t)S * stage_bytes);
     uint64_t *full = (uint64_t *)(red + NB * kDW * NT * 32 * 4);
     uint64_t *empty = full + kMaxStages;
@@ -436,21 +439,50 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     // routing results come from the previous kernel
     pdl_wait();
     pdl_launch_dependents();
+    load_token_tables(a, tok, gw);                // in flight with the next loads
     const Active A = build_active_list(a, act);   // includes __syncthreads
     const int tiles_r = a.F / kTile, tiles_s = a.sF / kTile;
-    const int U = A.n_routed * tiles_r + (a.sF > 0 ? tiles_s : 0);
+    // units: (virtual expert, 8-token column group, 16-row tile), expert-
+    // major; ucum[v] = first unit of virtual expert v (in the raw-table
+    // space of the active list, free now)
+    int *ucum = act + 4 * (a.E + 1);
+    if (warp == 0) {
+        int base = 0;
+        for (int v0 = 0; v0 < A.n_virt; v0 += 32) {
+            const int v = v0 + lane;
+            int nu = 0;
+            if (v < A.n_virt) {
+                const Virt vi = virt(a, act, A.n_routed, v);
+                nu = (vi.cnt + kGuCols - 1) / kGuCols * (vi.shared ? tiles_s : tiles_r);
+            }
+            int incl = nu;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (v < A.n_virt) ucum[v] = base + incl - nu;
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) ucum[A.n_virt] = base;
+    }
+    __syncthreads();
+    const int U = ucum[A.n_virt];
     // unit table: local unit i = global unit blockIdx.x + i * gridDim.x as
-    // (virtual expert, tile, segment start, token count)
+    // (virtual expert, tile, first permuted row, token count <= 8)
     const int n_local = U > (int)blockIdx.x ? (U - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     for (int i = tid; i < n_local; i += blockDim.x) {
         const int u = blockIdx.x + i * gridDim.x;
-        int v, tile;
-        if (u < A.n_routed * tiles_r) { v = u / tiles_r; tile = u % tiles_r; }
-        else { v = A.n_routed; tile = u - A.n_routed * tiles_r; }
-        const Virt vi = virt(a, act, A.n_routed, v);
-        utab[i] = make_int4(v, tile, vi.seg0, vi.cnt);
+        int lo = 0, hi = A.n_virt - 1;               // last v with ucum[v] <= u
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (ucum[mid] <= u) lo = mid; else hi = mid - 1;
+        }
+        const Virt vi = virt(a, act, A.n_routed, lo);
+        const int tv = vi.shared ? tiles_s : tiles_r;
+        const int rem = u - ucum[lo], grp = rem / tv, tile = rem % tv;
+        utab[i] = make_int4(lo, tile, vi.seg0 + grp * kGuCols, min(kGuCols, vi.cnt - grp * kGuCols));
     }
-    load_token_tables(a, tok, gw);
     __syncthreads();
 
     if (warp == kDW) {
@@ -530,7 +562,6 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
         const int4 ud = utab[j];
         const int tile = ud.y, seg0 = ud.z, cnt = ud.w;
         const bool q8 = ud.x < A.n_routed ? a.q8 != 0 : a.sq8 != 0;
-        const int ntile = cnt > 8 ? 2 : 1;
         const GuGeo gg = q8 ? geo8 : geo4;
         const int kb0 = kg * (q8 ? WB8 : WB4);          // warp's first block in a slice
         // B rows (column g, g+8) and C columns (2c, 2c+1, +8) of this unit
@@ -568,13 +599,8 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
                 sa_s[nt][1] = sa[nt][1] + sl * gg.sb * 4;
             }
 #define MOE_GU(Q8, NTL, MIS) gateup_slice<Q8, NTL, (Q8 ? WB8 : WB4), MIS>(row, r8, xs_s, sa_s, c, acc)
-            if (!q8) {
-                if (ntile == 1) { if (mis0 == 0) MOE_GU(false, 1, 0); else MOE_GU(false, 1, 2); }
-                else if (NT > 1) { if (mis0 == 0) MOE_GU(false, NT, 0); else MOE_GU(false, NT, 2); }
-            } else {
-                if (ntile == 1) { if (mis0 == 0) MOE_GU(true, 1, 0); else MOE_GU(true, 1, 2); }
-                else if (NT > 1) { if (mis0 == 0) MOE_GU(true, NT, 0); else MOE_GU(true, NT, 2); }
-            }
+            if (!q8) { if (mis0 == 0) MOE_GU(false, 1, 0); else MOE_GU(false, 1, 2); }
+            else { if (mis0 == 0) MOE_GU(true, 1, 0); else MOE_GU(true, 1, 2); }
 #undef MOE_GU
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
@@ -923,8 +949,14 @@ static cudaError_t launch_pdl(void (*kern)(Args...), int grid, int block, size_t
 }
 
 // the gate/up kernel's per-CTA unit table (16 bytes a unit)
+// units at most: sum over experts of ceil(tokens / 8) <= E + T*k/8 groups
+static int gu_units_max(const DecArgs &a) {
+    const int groups = a.E + (a.T * a.k) / kGuCols;
+    return groups * (a.F / kTile) + (a.T + kGuCols - 1) / kGuCols * (a.sF / kTile);
+}
+
 static size_t unit_table_bytes(const DecArgs &a, int sms) {
-    const int U_max = a.E * (a.F / kTile) + a.sF / kTile;
+    const int U_max = gu_units_max(a);
     const int grid = std::max(1, std::min(sms, U_max));
     return (size_t)((U_max + grid - 1) / grid) * 16 + 16;
 }
@@ -933,15 +965,21 @@ static size_t tables_bytes(int E) {
     return 6 * (size_t)(E + 1) * sizeof(int) + (size_t)(kMaxTk + 16) * (sizeof(int) + sizeof(float));
 }
 
-template <int NT>
+// one slice per 16-row tile: each stage is a whole unit (two 18.7 KB boxes
+// at D=2048, Q4_0)
+static int gu_max_sb(int T) { (void)T; return 64; }
+
 static cudaError_t launch_gateup(const DecArgs &a, const DecMaps &m, int grid, size_t smem,
                                  cudaStream_t s, int S) {
+    const bool wide = gu_max_sb(a.T) == 64;
     switch (a.D) {
-    case 256: return launch_pdl(dec_gateup_kernel<NT, 1, 1>, grid, kGThreads, smem, s, a, S, m);
-    case 512: return launch_pdl(dec_gateup_kernel<NT, 2, 2>, grid, kGThreads, smem, s, a, S, m);
-    case 768: return launch_pdl(dec_gateup_kernel<NT, 3, 3>, grid, kGThreads, smem, s, a, S, m);
-    case 1024: return launch_pdl(dec_gateup_kernel<NT, 4, 4>, grid, kGThreads, smem, s, a, S, m);
-    default: return launch_pdl(dec_gateup_kernel<NT, (NT == 1 ? 8 : 4), 4>, grid, kGThreads, smem, s, a, S, m);
+    case 256: return launch_pdl(dec_gateup_kernel<32, 1, 1>, grid, kGThreads, smem, s, a, S, m);
+    case 512: return launch_pdl(dec_gateup_kernel<32, 2, 2>, grid, kGThreads, smem, s, a, S, m);
+    case 768: return launch_pdl(dec_gateup_kernel<32, 3, 3>, grid, kGThreads, smem, s, a, S, m);
+    case 1024: return launch_pdl(dec_gateup_kernel<32, 4, 4>, grid, kGThreads, smem, s, a, S, m);
+    default:
+        return wide ? launch_pdl(dec_gateup_kernel<64, 8, 4>, grid, kGThreads, smem, s, a, S, m)
+                    : launch_pdl(dec_gateup_kernel<32, 4, 4>, grid, kGThreads, smem, s, a, S, m);
     }
 }
 
@@ -949,7 +987,7 @@ template <int NT>
 static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Tracer *tr) {
     const int sms = num_sms();
     DecMaps maps;
-    const int max_sb = NT == 1 ? 64 : 32;
+    const int max_sb = a.D <= 1024 ? 32 : gu_max_sb(a.T);
     moe_status st = encode_maps(a, n_slots, max_sb, &maps);
     if (st != MOE_OK) return st;
     const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
@@ -962,17 +1000,17 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         // mirrors the kernel's carve; + 1024 for aligning the base
         const size_t fixed = round_up(round_up((size_t)(a.T + 1) * staged_act_bytes(a.D), 16) +
                                       (size_t)2 * (a.T + 1) * nbD * 4, 1024) +
-                             (size_t)gu_red_bufs<NT>() * kDW * NT * 32 * 4 * sizeof(float) +
+                             (size_t)kGuRedBufs * kDW * 32 * 4 * sizeof(float) +
                              (2 * kMaxStages + 8) * sizeof(uint64_t) + tables_bytes(a.E) +
                              unit_table_bytes(a, sms) + 1024;
         if (fixed >= kDecSmemMax) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
         int S = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - fixed) / stage_bytes);
         if (S < 2) { set_error("decode path: shared memory too small"); return MOE_ERR_SHAPE; }
         const size_t smem = fixed + (size_t)S * stage_bytes;
-        const int U_max = a.E * (a.F / kTile) + a.sF / kTile;
+        const int U_max = gu_units_max(a);
         const int grid = std::max(1, std::min(sms, U_max));
         mark(tr, MOE_KERNEL_FFN_DECODE);
-        cudaError_t e = launch_gateup<NT>(a, maps, grid, smem, s, S);
+        cudaError_t e = launch_gateup(a, maps, grid, smem, s, S);
         if (e != cudaSuccess) return cuda_status(e, "dec_gateup_kernel");
     }
     // ---- down: Y rows

@@ -248,6 +248,21 @@ def test_single_expert_layer(moe):
     assert np.all(lay.gates.cpu().numpy() == 1.0)
 
 
+def test_layer_crowded_experts_with_shared(moe):
+    # T=16 over 4 experts with a skewed router bias: experts with more than
+    # 8 tokens (several MMA column groups) plus a shared expert over all 16
+    cfg = S.LayerConfig("crowd", T=16, D=512, E=4, k=2, F=256, qtype="q4_0", x_dtype="bf16",
+                        y_dtype="f32", router_std=0.05, zipf_s=1.5, shared_F=256, seed=79)
+    L = S.make_layer(cfg)
+    lay = _layer(moe, L)
+    y = lay.forward(dev_x(L))
+    torch.cuda.synchronize()
+    counts = np.bincount(lay.ids.cpu().numpy()[:16].ravel(), minlength=4)
+    assert counts.max() > 8, counts
+    _check_layer(moe, L, y, lay.ids, 16)
+    assert int(lay.ws[:4].view(torch.int32)[0]) == 0
+
+
 def test_masked_two_phase_rows_are_bit_identical(moe):
     L = layer_inputs("decode", 16)
     cfg = L.cfg
