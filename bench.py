@@ -164,7 +164,7 @@ def _dev_x(L, torch):
 class Workload:
     """A list of layer calls making one step; replicas rotate per call."""
 
-    def __init__(self, name: str, torch, moe):
+    def __init__(self, name: str, torch, moe, n_replicas=0):
         self.name = name
         self.torch, self.moe = torch, moe
         cfg = S.CONFIGS[name]
@@ -177,6 +177,8 @@ class Workload:
             Ts, replicas = (1, 2048), 2
         else:
             raise ValueError(name)
+        if n_replicas:     # fewer replicas: a small case for profilers (weights may hit L2)
+            replicas = int(n_replicas)
         self.Ts = Ts
         base = S.make_layer(cfg, T=max(Ts))
         self.inputs = {max(Ts): base}
@@ -290,7 +292,7 @@ def run_ours(args, world, rank, local):
     barrier(world)
     moe.lib()
     peaks = measured_peaks()
-    wl = Workload(args.workload, torch, moe)
+    wl = Workload(args.workload, torch, moe, args.replicas)
     algo = wl.algorithmic()
     stream = torch.cuda.current_stream()
 
@@ -440,19 +442,26 @@ def roofline(wl, algo, durs, peaks, args):
             "traffic": ncu_traffic(dom, wl.name)}
 
 
-def ncu_traffic(kernel, workload):
-    """dram read+write bytes per launch from the committed ncu summary, only
-    while the kernel sources still hash to what was profiled."""
-    p = os.path.join(ROOT, "profiles", "traffic.md")
-    if not os.path.exists(p):
-        return None
+# the source files whose code runs in each traced segment's kernels
+SEGMENT_SOURCES = {"ffn_decode": ("ffn_decode.cu", "sm100.cuh")}
+
+
+def segment_sha(kernel):
     import hashlib
     h = hashlib.sha256()
     src = os.path.join(ROOT, "quantized_routed_expert_top_b200", "csrc")
-    for f in sorted(os.listdir(src)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(src, f), "rb").read())
-    sha = h.hexdigest()[:16]
+    for f in SEGMENT_SOURCES.get(kernel, ()):
+        h.update(open(os.path.join(src, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """dram read+write bytes per launch from the committed ncu summary, only
+    while the segment's kernel sources still hash to what was profiled."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(p) or kernel not in SEGMENT_SOURCES:
+        return None
+    sha = segment_sha(kernel)
     for line in open(p):
         if line.startswith("traffic:"):
             kv = dict(x.split("=", 1) for x in line.split()[1:])
@@ -587,6 +596,8 @@ def main():
     ap.add_argument("--workload", choices=["decode", "prefill", "wide"], default="decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="pool replicas (default: the workload's; fewer only for profiling)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the steps eagerly instead of replaying CUDA graphs")
     args = ap.parse_args()
