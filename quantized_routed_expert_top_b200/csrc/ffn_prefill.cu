@@ -1,0 +1,550 @@
+// ffn_prefill.cu -- the prefill expert FFN (large T) on the 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// Prefill is a grouped GEMM: every expert multiplies its segment of tokens
+// (rows of the permuted order) by its weights.  Two launches:
+//
+//  * gate/up: H[p, f] = silu(x_t . Wg[f]) * (x_t . Wu[f]) for the rows p of
+//    expert e (token t = perm[p] / k), tile = 128 rows x 128 columns of F,
+//    both matrices (two MMAs of N=128 into 256 TMEM columns), K = D.
+//  * down:    Y[p, d] = H[p] . Wd[d], tile = 128 rows x 256 columns of D,
+//    K = F.  Y rows are fp32 in permuted order; the gate-weighted combine is
+//    the separate deterministic combine kernel.
+//
+// The weights stay in their ggml blocks in HBM.  They cannot feed the tensor
+// cores directly (a per-32 fp16 scale), so B-producer warps dequantise each
+// K-slice (64 weights of 256 rows) into fp16, d*q rounded once, written in the
+// 128-byte-swizzled K-major layout the MMA descriptors name.  A-producer
+// warps copy the activation rows (gathered through the permutation from an
+// fp16 copy of x, or the contiguous rows of H) the same way.  One thread
+// issues tcgen05.mma (M=128, K=16 steps) and commits each stage back to its
+// producers; two TMEM accumulators (2 x 256 columns) let the epilogue warps
+// drain one tile while the next accumulates.
+//
+// Numerics: weights d*q rounded to fp16 (relative error <= 2^-11 per weight),
+// activations fp16 (x is bf16 or fp32 on input: exact in fp16 over the
+// normal range), fp32 accumulation; H is stored fp16.
+#include "moe_internal.cuh"
+#include "sm100.cuh"
+
+#include <algorithm>
+
+namespace moe {
+
+constexpr int kPM = 128;                 // tile rows = MMA M
+constexpr int kPK = 64;                  // K per stage: one 128-byte row of fp16
+constexpr int kPNg = 128;                // gate/up: F columns per tile (per matrix)
+constexpr int kPNd = 256;                // down: D columns per tile
+constexpr int kPS = 4;                   // stages
+constexpr int kPStageA = kPM * kPK * 2;  // 16 KB
+constexpr int kPStageB = 256 * kPK * 2;  // 32 KB (256 weight rows)
+constexpr int kPStage = kPStageA + kPStageB;
+constexpr int kPAW = 4, kPBW = 4, kPEW = 4;
+constexpr int kPMmaWarp = kPAW + kPBW;                       // warp 8
+constexpr int kPThreads = (kPAW + kPBW + 1 + kPEW) * 32;     // 416
+constexpr int kPTmemCols = 512;                              // 2 accumulators x 256
+constexpr size_t kPSmem = (size_t)kPS * kPStage + 1024 + 2048 + 4 * (MOE_MAX_EXPERTS + 2) * 4;
+
+enum : int { kPGateUp = 0, kPDown = 1 };
+
+struct PfArgs {
+    int T, D, F, E, k;
+    int q8;                       // routed pool is Q8_0 (else Q4_0)
+    int shared, sq8;              // shared expert present (F columns, Q8_0 / Q4_0)
+    const int32_t *perm, *offsets;
+    const uint8_t *gate, *up, *down;
+    const int32_t *slot_map;
+    const uint8_t *sh_gate, *sh_up, *sh_down;
+    const __half *x16;            // [T, D]
+    __half *H;                    // [T*k + T, F]
+    float *Y;                     // [T*k + T, D]
+    int *err;
+};
+
+// ----------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16, fp32 accumulate
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// arrive (once) on an mbarrier when every tcgen05.mma issued so far by this
+// thread has completed
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+// 32 lanes x 32 columns of fp32 from TMEM: thread i gets lane (base + i)
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (start address and offsets in 16-byte units; version 1;
+// layout type 2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)1 << 16;                       // leading byte offset (unused with swizzle)
+    d |= (uint64_t)(1024 >> 4) << 32;             // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                       // descriptor version
+    d |= (uint64_t)2 << 61;                       // 128-byte swizzle
+    return d;
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, A and B fp16, both
+// K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t f16_idesc(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kPM >> 4) << 24);
+}
+
+// byte offset of 16-byte chunk j (0..7) of row r in a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t sw128_off(int r, int j) {
+    return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
+}
+
+// ------------------------------------------------------------- dequantise
+// 64 consecutive weights (two blocks starting at an even block index) of one
+// row into 8 chunks of 8 fp16, natural order.  The pair starts 4-byte aligned.
+__device__ __forceinline__ void dq_pair_q8(const uint8_t *src, uint4 *out) {
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(src);
+    uint32_t v[17];
+#pragma unroll
+    for (int i = 0; i < 17; i++) v[i] = __ldg(w + i);
+    const uint32_t d0 = v[0] & 0xFFFFu, d1 = v[8] >> 16;
+    const uint32_t dd0 = d0 | (d0 << 16), dd1 = d1 | (d1 << 16);
+    const uint32_t OFF = 0x64806480u, HI = 0x64646464u;
+    uint32_t h[32];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        // block 0 codes start at byte 2 of the pair; block 1 codes at byte 36
+        const uint32_t c0 = __funnelshift_r(v[i], v[i + 1], 16) ^ 0x80808080u;
+        const uint32_t c1 = v[9 + i] ^ 0x80808080u;
+        h[2 * i] = hmul2_u(hsub2_u(prmt(c0, HI, 0x5140), OFF), dd0);
+        h[2 * i + 1] = hmul2_u(hsub2_u(prmt(c0, HI, 0x7362), OFF), dd0);
+        h[16 + 2 * i] = hmul2_u(hsub2_u(prmt(c1, HI, 0x5140), OFF), dd1);
+        h[16 + 2 * i + 1] = hmul2_u(hsub2_u(prmt(c1, HI, 0x7362), OFF), dd1);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; c++) out[c] = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+}
+
+// Q4_0 pair: 36 bytes; byte j of a block = element j | element j+16 << 4.
+__device__ __forceinline__ void dq_pair_q4(const uint8_t *src, uint4 *out) {
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(src);
+    uint32_t v[9];
+#pragma unroll
+    for (int i = 0; i < 9; i++) v[i] = __ldg(w + i);
+    const uint32_t d0 = v[0] & 0xFFFFu, d1 = v[4] >> 16;
+    const uint32_t dd0 = d0 | (d0 << 16), dd1 = d1 | (d1 << 16);
+    const uint32_t OFF = 0x64086408u, M = 0x000F000Fu, MAG = 0x64006400u;
+    uint32_t lo[16], hi[16];    // per block: elements 0..15 (lo), 16..31 (hi) as half2
+#pragma unroll
+    for (int b = 0; b < 2; b++) {
+        const uint32_t dd = b ? dd1 : dd0;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const uint32_t c = b ? v[5 + i] : __funnelshift_r(v[i], v[i + 1], 16);
+            const uint32_t t0 = prmt(c, 0u, 0x4140), t1 = prmt(c, 0u, 0x4342);   // bytes 0,1 / 2,3
+            lo[8 * b + 2 * i] = hmul2_u(hsub2_u(lop3_and_or(t0, M, MAG), OFF), dd);
+            lo[8 * b + 2 * i + 1] = hmul2_u(hsub2_u(lop3_and_or(t1, M, MAG), OFF), dd);
+            hi[8 * b + 2 * i] = hmul2_u(hsub2_u(lop3_and_or(t0 >> 4, M, MAG), OFF), dd);
+            hi[8 * b + 2 * i + 1] = hmul2_u(hsub2_u(lop3_and_or(t1 >> 4, M, MAG), OFF), dd);
+        }
+    }
+    // chunks: block b -> elements 32b + [0..7], [8..15] (low nibbles), [16..23], [24..31]
+#pragma unroll
+    for (int b = 0; b < 2; b++) {
+        out[4 * b + 0] = make_uint4(lo[8 * b + 0], lo[8 * b + 1], lo[8 * b + 2], lo[8 * b + 3]);
+        out[4 * b + 1] = make_uint4(lo[8 * b + 4], lo[8 * b + 5], lo[8 * b + 6], lo[8 * b + 7]);
+        out[4 * b + 2] = make_uint4(hi[8 * b + 0], hi[8 * b + 1], hi[8 * b + 2], hi[8 * b + 3]);
+        out[4 * b + 3] = make_uint4(hi[8 * b + 4], hi[8 * b + 5], hi[8 * b + 6], hi[8 * b + 7]);
+    }
+}
+
+// ------------------------------------------------------------------ tiles
+// Virtual experts 0..E-1 (segments of the permutation) and, with a shared
+// expert, E (rows T*k .. T*k+T-1, token = row - T*k).  Tiles are listed
+// expert-major, then by column tile, then by row tile, so the row tiles that
+// share a weight tile run on neighbouring CTAs at about the same time.
+struct PfTile {
+    int v, seg0, rows, m, n;      // rows = the expert's row count
+};
+
+__device__ __forceinline__ PfTile pf_tile(const int *tcum, const int *segs, int nv, int nt, int tau) {
+    int lo = 0, hi = nv - 1;      // last v with tcum[v] <= tau
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tcum[mid] <= tau) lo = mid; else hi = mid - 1;
+    }
+    PfTile t;
+    t.v = lo;
+    t.seg0 = segs[lo];
+    t.rows = segs[lo + 1] - segs[lo];
+    const int r = tau - tcum[lo];
+    const int mt = (t.rows + kPM - 1) / kPM;
+    t.n = r / mt;
+    t.m = r % mt;
+    return t;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_pf[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t *stages = smem_pf + ((1024u - (smem_u32(smem_pf) & 1023u)) & 1023u);
+    uint64_t *full = (uint64_t *)(stages + (size_t)kPS * kPStage);
+    uint64_t *empty = full + kPS;
+    uint64_t *accf = empty + kPS;                  // [2] accumulator ready
+    uint64_t *acce = accf + 2;                     // [2] accumulator drained
+    uint32_t *tmem_slot = (uint32_t *)(acce + 2);
+    int *segs = (int *)(tmem_slot + 4);            // [nv + 1] segment starts
+    int *tcum = segs + (MOE_MAX_EXPERTS + 2);      // [nv + 1] first tile of each expert
+
+    const int Tk = a.T * a.k;
+    const int nv = a.E + (a.shared ? 1 : 0);
+    const int N = MODE == kPGateUp ? a.F : a.D;    // output columns
+    const int K = MODE == kPGateUp ? a.D : a.F;    // reduction length
+    const int BN = MODE == kPGateUp ? kPNg : kPNd;
+    const int nt = N / BN, nk = K / kPK;
+
+    if (tid == 0) {
+        for (int s = 0; s < kPS; s++) {
+            mbar_init(&full[s], (kPAW + kPBW) * 32);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], kPEW * 32);
+        }
+        fence_mbar_init();
+    }
+    if (warp == kPMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(kPTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // the permutation and segments come from the routing kernels
+    pdl_wait();
+    for (int v = tid; v <= nv; v += blockDim.x)
+        segs[v] = v <= a.E ? __ldg(a.offsets + v) : Tk + a.T;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (warp == 0) {
+        int base = 0;
+        for (int v0 = 0; v0 < nv; v0 += 32) {
+            const int v = v0 + lane;
+            int ntiles = 0;
+            if (v < nv) ntiles = (segs[v + 1] - segs[v] + kPM - 1) / kPM * nt;
+            int incl = ntiles;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (v < nv) tcum[v] = base + incl - ntiles;
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) tcum[nv] = base;
+    }
+    __syncthreads();
+    const int n_tiles = tcum[nv];
+
+    if (warp < kPAW) {
+        // ------------------------------------------ A producers (1 row each)
+        const int r = tid;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
+            const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
+            const int row = t.m * kPM + r;
+            const bool valid = row < t.rows;
+            const __half *src = nullptr;
+            if (valid) {
+                const int p = t.seg0 + row;
+                if (MODE == kPGateUp) {
+                    const int tok = p < Tk ? __ldg(a.perm + p) / a.k : p - Tk;
+                    src = a.x16 + (size_t)tok * a.D;
+                } else {
+                    src = a.H + (size_t)p * a.F;
+                }
+            }
+            for (int ks = 0; ks < nk; ks++, it++) {
+                const int s = it % kPS;
+                const uint32_t ph = (it / kPS) & 1;
+                uint4 c[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++)
+                    c[j] = valid ? __ldg(reinterpret_cast<const uint4 *>(src + ks * kPK) + j)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+                if (!mbar_wait(&empty[s], ph ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                uint8_t *dst = stages + (size_t)s * kPStage;
+#pragma unroll
+                for (int j = 0; j < 8; j++) *reinterpret_cast<uint4 *>(dst + sw128_off(r, j)) = c[j];
+                fence_proxy_async_smem();
+                mbar_arrive(&full[s]);
+            }
+        }
+    } else if (warp < kPAW + kPBW) {
+        // --------------------------------- B producers (2 weight rows each)
+        const int bt = tid - kPAW * 32;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
+            const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
+            const bool sh = t.v == a.E;
+            const bool q8 = sh ? a.sq8 != 0 : a.q8 != 0;
+            const int bs = q8 ? kQ8Bytes : kQ4Bytes;
+            const size_t rb = (size_t)(K / QK) * bs;                 // bytes per weight row
+            const size_t slot = sh ? 0 : (size_t)(a.slot_map ? __ldg(a.slot_map + t.v) : t.v);
+            const uint8_t *rowp[2];
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int br = bt + 128 * h;                         // row of the B tile
+                if (MODE == kPGateUp) {
+                    // rows 0..127: gate rows n*128.., rows 128..255: up rows
+                    const uint8_t *base = br < 128 ? (sh ? a.sh_gate : a.gate) : (sh ? a.sh_up : a.up);
+                    rowp[h] = base + (slot * a.F + (size_t)t.n * kPNg + (br & 127)) * rb;
+                } else {
+                    const uint8_t *base = sh ? a.sh_down : a.down;
+                    rowp[h] = base + (slot * a.D + (size_t)t.n * kPNd + br) * rb;
+                }
+            }
+            for (int ks = 0; ks < nk; ks++, it++) {
+                const int s = it % kPS;
+                const uint32_t ph = (it / kPS) & 1;
+                uint4 c[2][8];
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    const uint8_t *p = rowp[h] + (size_t)ks * 2 * bs;
+                    if (q8) dq_pair_q8(p, c[h]); else dq_pair_q4(p, c[h]);
+                }
+                if (!mbar_wait(&empty[s], ph ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                uint8_t *dst = stages + (size_t)s * kPStage + kPStageA;
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    const int br = bt + 128 * h;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) *reinterpret_cast<uint4 *>(dst + sw128_off(br, j)) = c[h][j];
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&full[s]);
+            }
+        }
+    } else if (warp == kPMmaWarp) {
+        // ----------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t st0 = smem_u32(stages);
+            uint32_t it = 0;
+            int lt = 0;
+            bool ok = true;
+            for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x, lt++) {
+                const int ab = lt & 1;
+                if (!mbar_wait(&acce[ab], (uint32_t)(((lt >> 1) & 1) ^ 1), a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t dacc = tmem + (uint32_t)(ab * 256);
+                for (int ks = 0; ks < nk; ks++, it++) {
+                    const int s = it % kPS;
+                    const uint32_t ph = (it / kPS) & 1;
+                    if (!mbar_wait(&full[s], ph, a.err, kErrTimeoutFull)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = st0 + (uint32_t)s * kPStage, sb = sa + kPStageA;
+#pragma unroll
+                    for (int kk = 0; kk < kPK / 16; kk++) {
+                        const uint64_t ad = sw128_desc(sa + kk * 32);
+                        const uint32_t acc = (ks | kk) != 0;
+                        if (MODE == kPGateUp) {
+                            tc_mma(dacc, ad, sw128_desc(sb + kk * 32), f16_idesc(kPNg), acc);
+                            tc_mma(dacc + kPNg, ad, sw128_desc(sb + kPNg * 128 + kk * 32), f16_idesc(kPNg), acc);
+                        } else {
+                            tc_mma(dacc, ad, sw128_desc(sb + kk * 32), f16_idesc(kPNd), acc);
+                        }
+                    }
+                    tc_commit(&empty[s]);        // the stage is free once these MMAs are done
+                }
+                if (!ok) break;
+                tc_commit(&accf[ab]);            // the tile's accumulator is complete
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------- epilogue
+        const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int r = q * 32 + lane;             // tile row
+        int lt = 0;
+        bool ok = true;
+        for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x, lt++) {
+            const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
+            const int ab = lt & 1;
+            if (!mbar_wait_warp(&accf[ab], (uint32_t)((lt >> 1) & 1), a.err, kErrTimeoutFull)) { ok = false; break; }
+            tc_fence_after();
+            const int row = t.m * kPM + r;
+            const bool valid = row < t.rows;
+            const size_t p = (size_t)t.seg0 + row;
+            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * 256);
+            if (MODE == kPGateUp) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < kPNg; c0 += 32) {
+                    uint32_t g[32], u[32];
+                    tc_ld32(tq + c0, g);
+                    tc_ld32(tq + kPNg + c0, u);
+                    tc_wait_ld();
+                    uint32_t hv[16];
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        const float h0 = silu(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+                        const float h1 = silu(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+                        const __half2 hh = __floats2half2_rn(h0, h1);
+                        hv[i] = *reinterpret_cast<const uint32_t *>(&hh);
+                    }
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(a.H + p * a.F + (size_t)t.n * kPNg + c0);
+#pragma unroll
+                        for (int i = 0; i < 4; i++)
+                            dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c0 = 0; c0 < kPNd; c0 += 32) {
+                    uint32_t y[32];
+                    tc_ld32(tq + c0, y);
+                    tc_wait_ld();
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(a.Y + p * a.D + (size_t)t.n * kPNd + c0);
+#pragma unroll
+                        for (int i = 0; i < 8; i++)
+                            dst[i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acce[ab]);
+        }
+    }
+    // everyone is done with the accumulators: release tensor memory
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kPMmaWarp) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     ::"r"(tmem), "r"(kPTmemCols) : "memory");
+    }
+}
+
+// x (bf16 or fp32) -> fp16, 8 elements per thread
+template <typename XT>
+__global__ void __launch_bounds__(256) pf_convert_kernel(const XT *__restrict__ x, __half *__restrict__ y,
+                                                         size_t n8) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    uint32_t h[4];
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+        const __half2 hh = __floats2half2_rn(load_act(x, 8 * i + 2 * q), load_act(x, 8 * i + 2 * q + 1));
+        h[q] = *reinterpret_cast<const uint32_t *>(&hh);
+    }
+    reinterpret_cast<uint4 *>(y)[i] = make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// ------------------------------------------------------------------- host
+bool prefill_path_ok(int T, int D, int F, int sF, int E) {
+    return T > 16 && D % kPNd == 0 && F % kPNg == 0 && F % kPK == 0 && D % kPK == 0 &&
+           (sF == 0 || sF == F) && E <= MOE_MAX_EXPERTS;
+}
+
+size_t prefill_x16_halves(int T, int D) { return (size_t)T * D; }
+size_t prefill_h_halves(int T, int k, int F, int sF) { return (size_t)(T * k + (sF ? T : 0)) * F; }
+size_t prefill_y_floats(int T, int k, int D, int sF) { return (size_t)(T * k + (sF ? T : 0)) * D; }
+
+template <int MODE>
+static cudaError_t launch_pf(const PfArgs &a, int grid, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kPThreads);
+    cfg.dynamicSmemBytes = kPSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaFuncSetAttribute(pf_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kPSmem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, pf_gemm_kernel<MODE>, a);
+}
+
+moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, int E, int k,
+                              const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
+                              const moe_pool *shared, int sF, __half *x16, __half *H, float *Y,
+                              int *err, cudaStream_t s, Tracer *tr) {
+    if (pool.qtype != MOE_Q4_0 && pool.qtype != MOE_Q8_0) {
+        set_error("prefill path: unsupported quant type %d", (int)pool.qtype);
+        return MOE_ERR_UNSUPPORTED_QTYPE;
+    }
+    if (shared && shared->qtype != MOE_Q4_0 && shared->qtype != MOE_Q8_0) {
+        set_error("prefill path: unsupported shared-expert quant type %d", (int)shared->qtype);
+        return MOE_ERR_UNSUPPORTED_QTYPE;
+    }
+    if (!prefill_path_ok(T, D, F, shared ? sF : 0, E)) {
+        set_error("prefill path: shape T=%d D=%d F=%d not supported", T, D, F);
+        return MOE_ERR_SHAPE;
+    }
+    PfArgs a{};
+    a.T = T; a.D = D; a.F = F; a.E = E; a.k = k;
+    a.q8 = pool.qtype == MOE_Q8_0;
+    a.shared = shared ? 1 : 0;
+    a.sq8 = shared ? shared->qtype == MOE_Q8_0 : 0;
+    a.perm = perm; a.offsets = offsets;
+    a.gate = (const uint8_t *)pool.gate; a.up = (const uint8_t *)pool.up;
+    a.down = (const uint8_t *)pool.down; a.slot_map = pool.slot_of_expert;
+    if (shared) {
+        a.sh_gate = (const uint8_t *)shared->gate; a.sh_up = (const uint8_t *)shared->up;
+        a.sh_down = (const uint8_t *)shared->down;
+    }
+    a.x16 = x16; a.H = H; a.Y = Y; a.err = err;
+
+    // activations to fp16 once (the MMA takes both operands in one type)
+    const size_t n8 = (size_t)T * D / 8;
+    mark(tr, MOE_KERNEL_CONVERT);
+    if (x_dtype == MOE_BF16)
+        pf_convert_kernel<__nv_bfloat16><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(
+            (const __nv_bfloat16 *)x, x16, n8);
+    else
+        pf_convert_kernel<float><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const float *)x, x16, n8);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e, "pf_convert_kernel");
+    const int grid = num_sms();
+    mark(tr, MOE_KERNEL_GATEUP);
+    if ((e = launch_pf<kPGateUp>(a, grid, s)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<gate/up>");
+    mark(tr, MOE_KERNEL_DOWN);
+    if ((e = launch_pf<kPDown>(a, grid, s)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<down>");
+    return MOE_OK;
+}
+
+}  // namespace moe

@@ -18,6 +18,7 @@ struct LayerWs {
     float *shH;          // [T, shared_F]
     float *sh_rows;      // [T, D]
     __half *Hs;          // decode path: g*h in fp16 fragment order
+    __half *x16, *H16;   // prefill path: fp16 activations and hidden rows
 };
 
 static LayerWs carve(const moe_layer_args &a, Carver &c) {
@@ -35,6 +36,13 @@ static LayerWs carve(const moe_layer_args &a, Carver &c) {
     if (decode_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0)) {
         w.Hs = c.take<__half>(decode_hs_halves(a.T, a.k, a.F, a.shared ? a.shared_F : 0));
         w.rows = c.take<float>(decode_rows_floats(a.T, a.k, a.D));
+        return w;
+    }
+    if (prefill_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0, a.E)) {
+        const int sF = a.shared ? a.shared_F : 0;
+        w.x16 = c.take<__half>(prefill_x16_halves(a.T, a.D));
+        w.H16 = c.take<__half>(prefill_h_halves(a.T, a.k, a.F, sF));
+        w.rows = c.take<float>(prefill_y_floats(a.T, a.k, a.D, sF));
         return w;
     }
     w.H = c.take<float>(Tk * a.F);
@@ -87,6 +95,24 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
         st = launch_ffn_decode(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.inv, w.offsets,
                                gates, *a.pool, nullptr, a.shared, a.shared ? a.shared_F : 0, w.Hs,
                                a.y, a.y_dtype, w.rows, w.status, s, tr);
+        if (tr) {
+            tr->end();
+            if (st == MOE_OK && tr->err != cudaSuccess) {
+                cudaGetLastError();
+                return cuda_status(tr->err, "moe_layer_forward: trace event record");
+            }
+        }
+        return st;
+    }
+    if (w.H16) {
+        const int sF = a.shared ? a.shared_F : 0;
+        if ((st = launch_ffn_prefill(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.offsets,
+                                     *a.pool, a.shared, sF, w.x16, w.H16, w.rows, w.status, s,
+                                     tr)) != MOE_OK)
+            return st;
+        st = launch_combine(w.rows, w.inv, gates, a.T, a.k, a.D,
+                            a.shared ? w.rows + (size_t)a.T * a.k * a.D : nullptr, a.y, a.y_dtype,
+                            s, tr);
         if (tr) {
             tr->end();
             if (st == MOE_OK && tr->err != cudaSuccess) {

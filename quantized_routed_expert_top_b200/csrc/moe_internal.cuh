@@ -165,6 +165,16 @@ moe_status launch_ffn_generic(const void *x, int x_dtype, int T, int D, int F, i
 bool decode_path_ok(int T, int D, int F, int sF);
 size_t decode_hs_halves(int T, int k, int F, int sF);
 size_t decode_rows_floats(int T, int k, int D);
+// ffn_prefill.cu -- large T on the tensor cores: x -> fp16, gate/up grouped
+// GEMM (H fp16), down grouped GEMM (Y fp32 rows, then the combine kernel)
+bool prefill_path_ok(int T, int D, int F, int sF, int E);
+size_t prefill_x16_halves(int T, int D);
+size_t prefill_h_halves(int T, int k, int F, int sF);
+size_t prefill_y_floats(int T, int k, int D, int sF);
+moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, int E, int k,
+                              const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
+                              const moe_pool *shared, int sF, __half *x16, __half *H, float *Y,
+                              int *err, cudaStream_t s, Tracer *tr);
 // y != NULL: fused layer (gates folded into the rows, rows_out is scratch
 // for [T*k + T, D] rows, combined into y); y == NULL: rows mode (rows_out =
 // un-gated Y rows [T*k, D] in permuted order, mask honoured)
