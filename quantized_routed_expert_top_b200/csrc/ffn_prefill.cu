@@ -27,7 +27,9 @@
 #include "moe_internal.cuh"
 #include "sm100.cuh"
 
+#include <cuda.h>
 #include <algorithm>
+#include <cstring>
 
 namespace moe {
 
@@ -35,7 +37,8 @@ constexpr int kPM = 128;                 // tile rows = MMA M
 constexpr int kPK = 64;                  // K per stage: one 128-byte row of fp16
 constexpr int kPNg = 128;                // gate/up: F columns per tile (per matrix)
 constexpr int kPNd = 256;                // down: D columns per tile
-constexpr int kPS = 4;                   // stages
+constexpr int kPS = 3;                   // fp16 operand stages
+constexpr int kPR = 3;                   // raw weight windows in flight
 constexpr int kPStageA = kPM * kPK * 2;  // 16 KB
 constexpr int kPStageB = 256 * kPK * 2;  // 32 KB (256 weight rows)
 constexpr int kPStage = kPStageA + kPStageB;
@@ -43,9 +46,22 @@ constexpr int kPAW = 4, kPBW = 4, kPEW = 4;
 constexpr int kPMmaWarp = kPAW + kPBW;                       // warp 8
 constexpr int kPThreads = (kPAW + kPBW + 1 + kPEW) * 32;     // 416
 constexpr int kPTmemCols = 512;                              // 2 accumulators x 256
-constexpr size_t kPSmem = (size_t)kPS * kPStage + 1024 + 2048 + 4 * (MOE_MAX_EXPERTS + 2) * 4;
+constexpr int kPRawRow = 80;             // raw window of one weight row (Q8_0: 5 x 16 B)
+constexpr int kPRaw = 256 * kPRawRow;    // one raw window buffer (20 KB)
+// stages | raw ring | barriers + TMEM slot (256 B) | segs, tcum [2][E+2]
+__host__ __device__ inline size_t pf_smem_bytes(int E) {
+    return (size_t)kPS * kPStage + (size_t)kPR * kPRaw + 256 + 2 * (size_t)(E + 2) * 4 + 1024;
+}
 
 enum : int { kPGateUp = 0, kPDown = 1 };
+
+// Tensor maps over the weight pools (8-byte elements, one row of blocks per
+// tensor row), boxes of one raw window (the 16-byte-aligned 80 or 48 bytes
+// holding a block pair) x 128 rows (gate, up) or 256 rows (down).
+struct PfMaps {
+    CUtensorMap w0, w1;           // gate/up: gate, up; down: down, -
+    CUtensorMap s0, s1;           // the shared expert's
+};
 
 struct PfArgs {
     int T, D, F, E, k;
@@ -125,14 +141,23 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int j) {
     return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
 }
 
+// named barrier 2 over the B-producer warps, returning the AND of `ok`
+__device__ __forceinline__ bool bar_and_b(bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+        " bar.red.and.pred q, 2, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r) : "r"((uint32_t)ok), "n"(kPBW * 32) : "memory");
+    return r != 0;
+}
+
 // ------------------------------------------------------------- dequantise
 // 64 consecutive weights (two blocks starting at an even block index) of one
-// row into 8 chunks of 8 fp16, natural order.  The pair starts 4-byte aligned.
-__device__ __forceinline__ void dq_pair_q8(const uint8_t *src, uint4 *out) {
-    const uint32_t *w = reinterpret_cast<const uint32_t *>(src);
-    uint32_t v[17];
-#pragma unroll
-    for (int i = 0; i < 17; i++) v[i] = __ldg(w + i);
+// row into 8 chunks of 8 fp16, natural order.  w: the row's raw window as
+// 32-bit words; the pair starts at word O.
+template <int O>
+__device__ __forceinline__ void dq_pair_q8(const uint32_t *w, uint4 *out) {
+    const uint32_t *v = w + O;
     const uint32_t d0 = v[0] & 0xFFFFu, d1 = v[8] >> 16;
     const uint32_t dd0 = d0 | (d0 << 16), dd1 = d1 | (d1 << 16);
     const uint32_t OFF = 0x64806480u, HI = 0x64646464u;
@@ -152,11 +177,9 @@ __device__ __forceinline__ void dq_pair_q8(const uint8_t *src, uint4 *out) {
 }
 
 // Q4_0 pair: 36 bytes; byte j of a block = element j | element j+16 << 4.
-__device__ __forceinline__ void dq_pair_q4(const uint8_t *src, uint4 *out) {
-    const uint32_t *w = reinterpret_cast<const uint32_t *>(src);
-    uint32_t v[9];
-#pragma unroll
-    for (int i = 0; i < 9; i++) v[i] = __ldg(w + i);
+template <int O>
+__device__ __forceinline__ void dq_pair_q4(const uint32_t *w, uint4 *out) {
+    const uint32_t *v = w + O;
     const uint32_t d0 = v[0] & 0xFFFFu, d1 = v[4] >> 16;
     const uint32_t dd0 = d0 | (d0 << 16), dd1 = d1 | (d1 << 16);
     const uint32_t OFF = 0x64086408u, M = 0x000F000Fu, MAG = 0x64006400u;
@@ -211,17 +234,19 @@ __device__ __forceinline__ PfTile pf_tile(const int *tcum, const int *segs, int 
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a) {
+__global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const __grid_constant__ PfMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_pf[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t *stages = smem_pf + ((1024u - (smem_u32(smem_pf) & 1023u)) & 1023u);
-    uint64_t *full = (uint64_t *)(stages + (size_t)kPS * kPStage);
+    uint8_t *raw = stages + (size_t)kPS * kPStage;  // ring of raw weight windows
+    uint64_t *full = (uint64_t *)(raw + (size_t)kPR * kPRaw);
     uint64_t *empty = full + kPS;
     uint64_t *accf = empty + kPS;                  // [2] accumulator ready
     uint64_t *acce = accf + 2;                     // [2] accumulator drained
-    uint32_t *tmem_slot = (uint32_t *)(acce + 2);
+    uint64_t *rfull = acce + 2;                    // [kPR] raw window landed
+    uint32_t *tmem_slot = (uint32_t *)(rfull + kPR);
     int *segs = (int *)(tmem_slot + 4);            // [nv + 1] segment starts
-    int *tcum = segs + (MOE_MAX_EXPERTS + 2);      // [nv + 1] first tile of each expert
+    int *tcum = segs + (a.E + 2);                  // [nv + 1] first tile of each expert
 
     const int Tk = a.T * a.k;
     const int nv = a.E + (a.shared ? 1 : 0);
@@ -239,6 +264,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a) {
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], kPEW * 32);
         }
+        for (int r = 0; r < kPR; r++) mbar_init(&rfull[r], 1);
         fence_mbar_init();
     }
     if (warp == kPMmaWarp) {
@@ -275,86 +301,169 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a) {
     const int n_tiles = tcum[nv];
 
     if (warp < kPAW) {
-        // ------------------------------------------ A producers (1 row each)
-        const int r = tid;
-        uint32_t it = 0;
+        // ------------------------------------------ A producers
+        // thread t copies 16-byte chunk t % 8 of rows t / 8 + 16 i (i < 8)
+        // with asynchronous copies straight into the swizzled stage, kPS - 1
+        // stages ahead of the one it publishes (rows past the expert's end
+        // are zero-filled).
+        const int j = tid & 7, r0 = tid >> 3;
+        constexpr int AH = kPS - 1;
+        int n_loc = 0;                                   // this CTA's tiles
+        for (int tau = blockIdx.x; tau < n_tiles; tau += gridDim.x) n_loc++;
+        const int n_st = n_loc * nk;                     // stages in all
+        // issue cursor
+        int gi = 0, ti = -1, ksi = nk;
+        const __half *src[8];
         bool ok = true;
-        for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
-            const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
-            const int row = t.m * kPM + r;
-            const bool valid = row < t.rows;
-            const __half *src = nullptr;
-            if (valid) {
-                const int p = t.seg0 + row;
-                if (MODE == kPGateUp) {
-                    const int tok = p < Tk ? __ldg(a.perm + p) / a.k : p - Tk;
-                    src = a.x16 + (size_t)tok * a.D;
-                } else {
-                    src = a.H + (size_t)p * a.F;
+        auto issue = [&]() {
+            if (gi >= n_st) { asm volatile("cp.async.commit_group;" ::: "memory"); gi++; return; }
+            if (ksi == nk) {                             // next tile: its rows
+                ti++;
+                ksi = 0;
+                const PfTile t = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int row = t.m * kPM + r0 + 16 * i;
+                    src[i] = nullptr;
+                    if (row < t.rows) {
+                        const int p = t.seg0 + row;
+                        if (MODE == kPGateUp) {
+                            const int tok = p < Tk ? __ldg(a.perm + p) / a.k : p - Tk;
+                            src[i] = a.x16 + (size_t)tok * a.D;
+                        } else {
+                            src[i] = a.H + (size_t)p * a.F;
+                        }
+                    }
                 }
             }
-            for (int ks = 0; ks < nk; ks++, it++) {
-                const int s = it % kPS;
-                const uint32_t ph = (it / kPS) & 1;
-                uint4 c[8];
+            const int s = gi % kPS;
+            if (!mbar_wait(&empty[s], ((gi / kPS) & 1) ^ 1, a.err, kErrTimeoutEmpty)) ok = false;
+            const uint32_t dst = smem_u32(stages + (size_t)s * kPStage);
 #pragma unroll
-                for (int j = 0; j < 8; j++)
-                    c[j] = valid ? __ldg(reinterpret_cast<const uint4 *>(src + ks * kPK) + j)
-                                 : make_uint4(0u, 0u, 0u, 0u);
-                if (!mbar_wait(&empty[s], ph ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
-                uint8_t *dst = stages + (size_t)s * kPStage;
-#pragma unroll
-                for (int j = 0; j < 8; j++) *reinterpret_cast<uint4 *>(dst + sw128_off(r, j)) = c[j];
-                fence_proxy_async_smem();
-                mbar_arrive(&full[s]);
+            for (int i = 0; i < 8; i++) {
+                const __half *g = src[i] ? src[i] + ksi * kPK + 8 * j : a.x16;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                             ::"r"(dst + sw128_off(r0 + 16 * i, j)), "l"(g), "r"(src[i] ? 16 : 0) : "memory");
             }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            gi++;
+            ksi++;
+        };
+        for (int q = 0; q < AH; q++) issue();
+        for (int g = 0; g < n_st && ok; g++) {
+            issue();                                     // stage g + AH
+            asm volatile("cp.async.wait_group %0;" ::"n"(AH) : "memory");   // stage g landed
+            fence_proxy_async_smem();
+            mbar_arrive(&full[g % kPS]);
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kPAW + kPBW) {
-        // --------------------------------- B producers (2 weight rows each)
+        // ------------------------------------------------- B producers
+        // Raw windows (the 16-byte-aligned bytes holding a K-slice's block
+        // pair, for all 256 weight rows of the tile) arrive by tensor copies
+        // kPR - 1 stages ahead; thread t dequantises rows t and t + 128 of
+        // the current window into the swizzled fp16 stage.
         const int bt = tid - kPAW * 32;
-        uint32_t it = 0;
-        bool ok = true;
-        for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
-            const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
-            const bool sh = t.v == a.E;
+        int n_loc = 0;
+        for (int tau = blockIdx.x; tau < n_tiles; tau += gridDim.x) n_loc++;
+        const int n_st = n_loc * nk;
+        // raw-window issue cursor (thread bt == 0 only)
+        int gi = 0, ti = -1, ksi = nk;
+        PfTile tI{};
+        auto issue = [&]() {
+            if (gi >= n_st) return;
+            if (ksi == nk) {
+                ti++;
+                ksi = 0;
+                tI = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
+            }
+            const bool sh = tI.v == a.E;
             const bool q8 = sh ? a.sq8 != 0 : a.q8 != 0;
             const int bs = q8 ? kQ8Bytes : kQ4Bytes;
-            const size_t rb = (size_t)(K / QK) * bs;                 // bytes per weight row
-            const size_t slot = sh ? 0 : (size_t)(a.slot_map ? __ldg(a.slot_map + t.v) : t.v);
-            const uint8_t *rowp[2];
-#pragma unroll
-            for (int h = 0; h < 2; h++) {
-                const int br = bt + 128 * h;                         // row of the B tile
-                if (MODE == kPGateUp) {
-                    // rows 0..127: gate rows n*128.., rows 128..255: up rows
-                    const uint8_t *base = br < 128 ? (sh ? a.sh_gate : a.gate) : (sh ? a.sh_up : a.up);
-                    rowp[h] = base + (slot * a.F + (size_t)t.n * kPNg + (br & 127)) * rb;
-                } else {
-                    const uint8_t *base = sh ? a.sh_down : a.down;
-                    rowp[h] = base + (slot * a.D + (size_t)t.n * kPNd + br) * rb;
-                }
+            const int wb = q8 ? 80 : 48;                         // window bytes
+            const int x = (int)(((size_t)ksi * 2 * bs & ~(size_t)15) / 8);
+            const int slot = sh ? 0 : (a.slot_map ? __ldg(a.slot_map + tI.v) : tI.v);
+            const int r = gi % kPR;
+            uint8_t *dst = raw + (size_t)r * kPRaw;
+            mbar_arrive_expect_tx(&rfull[r], (uint32_t)(256 * wb));
+            if (MODE == kPGateUp) {
+                const int y = slot * a.F + tI.n * kPNg;
+                tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, y, &rfull[r]);
+                tma_load_2d(dst + 128 * wb, sh ? &maps.s1 : &maps.w1, x, y, &rfull[r]);
+            } else {
+                tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, slot * a.D + tI.n * kPNd, &rfull[r]);
             }
-            for (int ks = 0; ks < nk; ks++, it++) {
-                const int s = it % kPS;
-                const uint32_t ph = (it / kPS) & 1;
+            gi++;
+            ksi++;
+        };
+        if (bt == 0)
+            for (int q = 0; q < kPR - 1; q++) issue();
+        bool ok = true;
+        int g = 0;
+        for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
+            const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
+            const bool q8 = (t.v == a.E) ? a.sq8 != 0 : a.q8 != 0;
+            const int wb = q8 ? 80 : 48;
+            for (int ks = 0; ks < nk; ks++, g++) {
+                // every producer is done with the window of stage g - 1: its
+                // buffer takes the window of stage g + kPR - 1; a wait that
+                // ran out anywhere ends every producer's loop here
+                ok = bar_and_b(ok);
+                if (!ok) break;
+                if (bt == 0) issue();
+                const int r = g % kPR;
+                if (!mbar_wait(&rfull[r], (uint32_t)((g / kPR) & 1), a.err, kErrTimeoutFull)) { ok = false; continue; }
                 uint4 c[2][8];
+                const int o = ks & 3;                            // word offset of the pair
 #pragma unroll
                 for (int h = 0; h < 2; h++) {
-                    const uint8_t *p = rowp[h] + (size_t)ks * 2 * bs;
-                    if (q8) dq_pair_q8(p, c[h]); else dq_pair_q4(p, c[h]);
+                    const uint8_t *rp = raw + (size_t)r * kPRaw + (bt + 128 * h) * wb;
+                    if (q8) {
+                        uint32_t w[20];
+#pragma unroll
+                        for (int q = 0; q < 5; q++) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(rp + 16 * q);
+                            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                        }
+                        switch (o) {
+                        case 0: dq_pair_q8<0>(w, c[h]); break;
+                        case 1: dq_pair_q8<1>(w, c[h]); break;
+                        case 2: dq_pair_q8<2>(w, c[h]); break;
+                        default: dq_pair_q8<3>(w, c[h]); break;
+                        }
+                    } else {
+                        uint32_t w[12];
+#pragma unroll
+                        for (int q = 0; q < 3; q++) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(rp + 16 * q);
+                            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                        }
+                        switch (o) {
+                        case 0: dq_pair_q4<0>(w, c[h]); break;
+                        case 1: dq_pair_q4<1>(w, c[h]); break;
+                        case 2: dq_pair_q4<2>(w, c[h]); break;
+                        default: dq_pair_q4<3>(w, c[h]); break;
+                        }
+                    }
                 }
-                if (!mbar_wait(&empty[s], ph ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                const int s = g % kPS;
+                if (!mbar_wait(&empty[s], ((g / kPS) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; continue; }
                 uint8_t *dst = stages + (size_t)s * kPStage + kPStageA;
 #pragma unroll
                 for (int h = 0; h < 2; h++) {
                     const int br = bt + 128 * h;
 #pragma unroll
-                    for (int j = 0; j < 8; j++) *reinterpret_cast<uint4 *>(dst + sw128_off(br, j)) = c[h][j];
+                    for (int jj = 0; jj < 8; jj++) *reinterpret_cast<uint4 *>(dst + sw128_off(br, jj)) = c[h][jj];
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&full[s]);
             }
+            ok = bar_and_b(ok);                                  // a failure in a tile's last stage
         }
+        // windows still in flight must land before the CTA exits
+        if (bt == 0)
+            for (; g < gi; g++)
+                mbar_wait(&rfull[g % kPR], (uint32_t)((g / kPR) & 1), a.err, kErrTimeoutDrain);
     } else if (warp == kPMmaWarp) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
@@ -472,8 +581,10 @@ __global__ void __launch_bounds__(256) pf_convert_kernel(const XT *__restrict__ 
 }
 
 // ------------------------------------------------------------------- host
+// K (D for gate/up, F for down) a multiple of 256: the last block pair of a
+// row then sits at the end of its 16-byte window, so no window reads past a row
 bool prefill_path_ok(int T, int D, int F, int sF, int E) {
-    return T > 16 && D % kPNd == 0 && F % kPNg == 0 && F % kPK == 0 && D % kPK == 0 &&
+    return T > 16 && D % kPNd == 0 && F % kPNg == 0 && D % 256 == 0 && F % 256 == 0 &&
            (sF == 0 || sF == F) && E <= MOE_MAX_EXPERTS;
 }
 
@@ -481,12 +592,44 @@ size_t prefill_x16_halves(int T, int D) { return (size_t)T * D; }
 size_t prefill_h_halves(int T, int k, int F, int sF) { return (size_t)(T * k + (sF ? T : 0)) * F; }
 size_t prefill_y_floats(int T, int k, int D, int sF) { return (size_t)(T * k + (sF ? T : 0)) * D; }
 
+typedef CUresult (*PfEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                               const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                               const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// rows x row_bytes (8-byte elements) at base, boxes of box_bytes x box_rows
+static moe_status pf_encode(CUtensorMap *m, const void *base, size_t row_bytes, size_t nrows,
+                            int box_bytes, int box_rows) {
+    static PfEncodeFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PfEncodeFn)p;
+    }
+    if (!fn) { set_error("prefill path: cuTensorMapEncodeTiled unavailable"); return MOE_ERR_CUDA; }
+    const cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / 8), (cuuint64_t)nrows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(box_bytes / 8), (cuuint32_t)box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("prefill path: tensor map encoding failed (%d)", (int)r);
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
 template <int MODE>
-static cudaError_t launch_pf(const PfArgs &a, int grid, cudaStream_t s) {
+static cudaError_t launch_pf(const PfArgs &a, const PfMaps &m, int grid, cudaStream_t s) {
+    const size_t smem = pf_smem_bytes(a.E);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kPThreads);
-    cfg.dynamicSmemBytes = kPSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -494,9 +637,9 @@ static cudaError_t launch_pf(const PfArgs &a, int grid, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaFuncSetAttribute(pf_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kPSmem);
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, pf_gemm_kernel<MODE>, a);
+    return cudaLaunchKernelEx(&cfg, pf_gemm_kernel<MODE>, a, m);
 }
 
 moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, int E, int k,
@@ -539,11 +682,31 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
         pf_convert_kernel<float><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const float *)x, x16, n8);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "pf_convert_kernel");
+    // weight tensor maps: raw windows of 80 (Q8_0) or 48 (Q4_0) bytes
+    const int br = pool.qtype == MOE_Q8_0 ? kQ8Bytes : kQ4Bytes;
+    const int wr = pool.qtype == MOE_Q8_0 ? 80 : 48;
+    PfMaps mg, md;
+    memset(&mg, 0, sizeof(mg));
+    memset(&md, 0, sizeof(md));
+    moe_status st;
+    const size_t rows_f = (size_t)pool.n_slots * F, rows_d = (size_t)pool.n_slots * D;
+    if ((st = pf_encode(&mg.w0, pool.gate, (size_t)(D / QK) * br, rows_f, wr, kPNg)) ||
+        (st = pf_encode(&mg.w1, pool.up, (size_t)(D / QK) * br, rows_f, wr, kPNg)) ||
+        (st = pf_encode(&md.w0, pool.down, (size_t)(F / QK) * br, rows_d, wr, kPNd)))
+        return st;
+    if (shared) {
+        const int bsh = shared->qtype == MOE_Q8_0 ? kQ8Bytes : kQ4Bytes;
+        const int wsh = shared->qtype == MOE_Q8_0 ? 80 : 48;
+        if ((st = pf_encode(&mg.s0, shared->gate, (size_t)(D / QK) * bsh, F, wsh, kPNg)) ||
+            (st = pf_encode(&mg.s1, shared->up, (size_t)(D / QK) * bsh, F, wsh, kPNg)) ||
+            (st = pf_encode(&md.s0, shared->down, (size_t)(F / QK) * bsh, D, wsh, kPNd)))
+            return st;
+    }
     const int grid = num_sms();
     mark(tr, MOE_KERNEL_GATEUP);
-    if ((e = launch_pf<kPGateUp>(a, grid, s)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<gate/up>");
+    if ((e = launch_pf<kPGateUp>(a, mg, grid, s)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<gate/up>");
     mark(tr, MOE_KERNEL_DOWN);
-    if ((e = launch_pf<kPDown>(a, grid, s)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<down>");
+    if ((e = launch_pf<kPDown>(a, md, grid, s)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<down>");
     return MOE_OK;
 }
 
