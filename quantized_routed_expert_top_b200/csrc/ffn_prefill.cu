@@ -42,9 +42,10 @@ constexpr int kPR = 3;                   // raw weight windows in flight
 constexpr int kPStageA = kPM * kPK * 2;  // 16 KB
 constexpr int kPStageB = 256 * kPK * 2;  // 32 KB (256 weight rows)
 constexpr int kPStage = kPStageA + kPStageB;
-constexpr int kPAW = 4, kPBW = 4, kPEW = 4;
-constexpr int kPMmaWarp = kPAW + kPBW;                       // warp 8
-constexpr int kPThreads = (kPAW + kPBW + 1 + kPEW) * 32;     // 416
+constexpr int kPAW = 2, kPBW = 8, kPEW = 4;                  // A copiers, B dequantisers, epilogue
+constexpr int kPMmaWarp = kPAW + kPBW;                       // warp 10
+constexpr int kPThreads = (kPAW + kPBW + 1 + kPEW) * 32;     // 480
+constexpr int kPARows = kPM / (kPAW * 32 / 8);               // rows per A thread (16)
 constexpr int kPTmemCols = 512;                              // 2 accumulators x 256
 constexpr int kPRawRow = 80;             // raw window of one weight row (Q8_0: 5 x 16 B)
 constexpr int kPRaw = 256 * kPRawRow;    // one raw window buffer (20 KB)
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
 
     if (warp < kPAW) {
         // ------------------------------------------ A producers
-        // thread t copies 16-byte chunk t % 8 of rows t / 8 + 16 i (i < 8)
+        // thread t copies 16-byte chunk t % 8 of rows t / 8 + 8 i (i < 16)
         // with asynchronous copies straight into the swizzled stage, kPS - 1
         // stages ahead of the one it publishes (rows past the expert's end
         // are zero-filled).
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
         const int n_st = n_loc * nk;                     // stages in all
         // issue cursor
         int gi = 0, ti = -1, ksi = nk;
-        const __half *src[8];
+        const __half *src[kPARows];
         bool ok = true;
         auto issue = [&]() {
             if (gi >= n_st) { asm volatile("cp.async.commit_group;" ::: "memory"); gi++; return; }
@@ -322,8 +323,8 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                 ksi = 0;
                 const PfTile t = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const int row = t.m * kPM + r0 + 16 * i;
+                for (int i = 0; i < kPARows; i++) {
+                    const int row = t.m * kPM + r0 + 8 * i;
                     src[i] = nullptr;
                     if (row < t.rows) {
                         const int p = t.seg0 + row;
@@ -340,29 +341,32 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
             if (!mbar_wait(&empty[s], ((gi / kPS) & 1) ^ 1, a.err, kErrTimeoutEmpty)) ok = false;
             const uint32_t dst = smem_u32(stages + (size_t)s * kPStage);
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
+            for (int i = 0; i < kPARows; i++) {
                 const __half *g = src[i] ? src[i] + ksi * kPK + 8 * j : a.x16;
                 asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                             ::"r"(dst + sw128_off(r0 + 16 * i, j)), "l"(g), "r"(src[i] ? 16 : 0) : "memory");
+                             ::"r"(dst + sw128_off(r0 + 8 * i, j)), "l"(g), "r"(src[i] ? 16 : 0) : "memory");
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
             gi++;
             ksi++;
         };
+        // stage g is published before stage g + AH is issued: issuing waits
+        // for the MMAs of stage g - 1 to free their slot, and publishing
+        // first keeps that wait off the MMAs' critical path
         for (int q = 0; q < AH; q++) issue();
         for (int g = 0; g < n_st && ok; g++) {
-            issue();                                     // stage g + AH
-            asm volatile("cp.async.wait_group %0;" ::"n"(AH) : "memory");   // stage g landed
+            asm volatile("cp.async.wait_group %0;" ::"n"(AH - 1) : "memory");   // stage g landed
             fence_proxy_async_smem();
             mbar_arrive(&full[g % kPS]);
+            issue();                                     // stage g + AH
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kPAW + kPBW) {
         // ------------------------------------------------- B producers
         // Raw windows (the 16-byte-aligned bytes holding a K-slice's block
         // pair, for all 256 weight rows of the tile) arrive by tensor copies
-        // kPR - 1 stages ahead; thread t dequantises rows t and t + 128 of
-        // the current window into the swizzled fp16 stage.
+        // kPR - 1 stages ahead; thread t dequantises weight row t of the
+        // current window into the swizzled fp16 stage.
         const int bt = tid - kPAW * 32;
         int n_loc = 0;
         for (int tau = blockIdx.x; tau < n_tiles; tau += gridDim.x) n_loc++;
@@ -413,11 +417,11 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                 if (bt == 0) issue();
                 const int r = g % kPR;
                 if (!mbar_wait(&rfull[r], (uint32_t)((g / kPR) & 1), a.err, kErrTimeoutFull)) { ok = false; continue; }
-                uint4 c[2][8];
+                uint4 c[1][8];
                 const int o = ks & 3;                            // word offset of the pair
 #pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    const uint8_t *rp = raw + (size_t)r * kPRaw + (bt + 128 * h) * wb;
+                for (int h = 0; h < 1; h++) {
+                    const uint8_t *rp = raw + (size_t)r * kPRaw + bt * wb;
                     if (q8) {
                         uint32_t w[20];
 #pragma unroll
@@ -450,11 +454,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                 if (!mbar_wait(&empty[s], ((g / kPS) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; continue; }
                 uint8_t *dst = stages + (size_t)s * kPStage + kPStageA;
 #pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    const int br = bt + 128 * h;
-#pragma unroll
-                    for (int jj = 0; jj < 8; jj++) *reinterpret_cast<uint4 *>(dst + sw128_off(br, jj)) = c[h][jj];
-                }
+                for (int jj = 0; jj < 8; jj++) *reinterpret_cast<uint4 *>(dst + sw128_off(bt, jj)) = c[0][jj];
                 fence_proxy_async_smem();
                 mbar_arrive(&full[s]);
             }

@@ -259,6 +259,93 @@ route_logits_tiled_kernel(const XT *__restrict__ x, const float *__restrict__ W,
     }
 }
 
+// Large-T router logits, register-tiled SIMT GEMM: a CTA computes 64 tokens
+// x 128 experts, a thread 4 tokens x 8 experts (two runs of 4, so its
+// 16-byte shared loads of W_r are conflict-free), with the next 32-row
+// K-tile loaded into registers while the current one is used.  Every
+// logit is one thread's fmaf chain over k in ascending order plus the bias,
+// the same arithmetic as route_logits_tiled_kernel.  E % 4 == 0.
+constexpr int kSM = 64, kSN = 128, kSK = 32;
+
+template <typename XT>
+__global__ void __launch_bounds__(256)
+route_logits_sgemm_kernel(const XT *__restrict__ x, const float *__restrict__ W,
+                          const float *__restrict__ bias, int T, int D, int E,
+                          float *__restrict__ logits) {
+    extern __shared__ __align__(16) float smem_lg[];
+    float *As = smem_lg;                                   // [2][kSK][kSM + 1]
+    float *Bs = As + 2 * kSK * (kSM + 1);                  // [2][kSK][kSN + 4]
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int t0 = blockIdx.x * kSM, e0 = blockIdx.y * kSN;
+    // global -> register staging: A = 8 consecutive k of one token, B = 4
+    // float4 of W_r rows
+    const int am = tid >> 2, ak = (tid & 3) * 8;
+    const int bc = (tid & 31) * 4, br = tid >> 5;
+    float ra[8];
+    float4 rb[4];
+    auto load = [&](int k0) {
+        const int t = t0 + am;
+#pragma unroll
+        for (int i = 0; i < 8; i++) ra[i] = (t < T) ? load_act(x, (size_t)t * D + k0 + ak + i) : 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int e = e0 + bc;
+            rb[i] = (e < E) ? __ldg(reinterpret_cast<const float4 *>(W + (size_t)(k0 + br + 8 * i) * E + e))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto store = [&](int buf) {
+        float *a = As + buf * kSK * (kSM + 1);
+        float *b = Bs + buf * kSK * (kSN + 4);
+#pragma unroll
+        for (int i = 0; i < 8; i++) a[(ak + i) * (kSM + 1) + am] = ra[i];
+#pragma unroll
+        for (int i = 0; i < 4; i++) *reinterpret_cast<float4 *>(b + (br + 8 * i) * (kSN + 4) + bc) = rb[i];
+    };
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int j = 0; j < 8; j++) acc[i][j] = 0.f;
+    load(0);
+    store(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = 0; k0 < D; k0 += kSK) {
+        if (k0 + kSK < D) load(k0 + kSK);
+        const float *a = As + buf * kSK * (kSM + 1);
+        const float *b = Bs + buf * kSK * (kSN + 4);
+#pragma unroll
+        for (int kk = 0; kk < kSK; kk++) {
+            float av[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) av[i] = a[kk * (kSM + 1) + ty * 4 + i];
+            const float4 b0 = *reinterpret_cast<const float4 *>(b + kk * (kSN + 4) + tx * 4);
+            const float4 b1 = *reinterpret_cast<const float4 *>(b + kk * (kSN + 4) + 64 + tx * 4);
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+#pragma unroll
+                for (int j = 0; j < 8; j++) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        if (k0 + kSK < D) {
+            store(buf ^ 1);
+            __syncthreads();
+            buf ^= 1;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const int t = t0 + ty * 4 + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int e = e0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+            if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (bias ? __ldg(bias + e) : 0.0f);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256)
 route_select_kernel(const float *__restrict__ logits, const float *__restrict__ bias_if_raw,
                     int T, int E, int k, int renorm, int32_t *__restrict__ ids,
@@ -611,14 +698,34 @@ moe_status launch_route(const void *x, int x_dtype, const float *w_router,
         L = c.take<float>((size_t)T * E);
         if (!c.fits()) { set_error("moe_route: workspace too small"); return MOE_ERR_WORKSPACE; }
     }
-    dim3 grid((T + kTM - 1) / kTM, (E + kTN - 1) / kTN);
     mark(tr, MOE_KERNEL_ROUTE_LOGITS);
-    if (x_dtype == MOE_BF16)
-        route_logits_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16 *)x, w_router, bias, T, D, E, L);
-    else
-        route_logits_tiled_kernel<float><<<grid, 256, 0, s>>>((const float *)x, w_router, bias,
-                                                              T, D, E, L);
+    if (E % 4 == 0) {
+        const dim3 grid((T + kSM - 1) / kSM, (E + kSN - 1) / kSN);
+        const size_t sm = (size_t)(2 * kSK * (kSM + 1) + 2 * kSK * (kSN + 4)) * sizeof(float);
+        cudaError_t e;
+        if (x_dtype == MOE_BF16) {
+            e = cudaFuncSetAttribute(route_logits_sgemm_kernel<__nv_bfloat16>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            if (e == cudaSuccess)
+                route_logits_sgemm_kernel<__nv_bfloat16><<<grid, 256, sm, s>>>(
+                    (const __nv_bfloat16 *)x, w_router, bias, T, D, E, L);
+        } else {
+            e = cudaFuncSetAttribute(route_logits_sgemm_kernel<float>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            if (e == cudaSuccess)
+                route_logits_sgemm_kernel<float><<<grid, 256, sm, s>>>((const float *)x, w_router,
+                                                                       bias, T, D, E, L);
+        }
+        if (e != cudaSuccess) return cuda_status(e, "route_logits_sgemm_kernel attribute");
+    } else {
+        dim3 grid((T + kTM - 1) / kTM, (E + kTN - 1) / kTN);
+        if (x_dtype == MOE_BF16)
+            route_logits_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+                (const __nv_bfloat16 *)x, w_router, bias, T, D, E, L);
+        else
+            route_logits_tiled_kernel<float><<<grid, 256, 0, s>>>((const float *)x, w_router, bias,
+                                                                  T, D, E, L);
+    }
     moe_status st = cuda_status(cudaGetLastError(), "route_logits_tiled_kernel");
     if (st != MOE_OK) return st;
     int blocks = (T * 32 + 255) / 256;
