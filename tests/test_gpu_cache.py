@@ -1,0 +1,127 @@
+"""Expert cache on the GPU: the hit/miss/victim sequence against the oracle's
+LRU simulation, layer outputs with the cache against the fully resident
+pool (bit for bit: same kernels, same reduction order, only the slot
+addresses differ), and an injected copy failure.
+
+A small stack of layers (Q8_0, D=256, F=256, E=16, k=4, 6 slots per layer)
+routed from per-layer locality traces, T=1 per step, as the cache workload
+does at full size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+N_LAYERS, E, K, D, F, SLOTS, STEPS = 3, 16, 4, 256, 256, 6, 30
+
+
+@pytest.fixture(scope="module")
+def stack(moe):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    pools = [S.gen_expert_pool(900 + l, E, D, F, "q8_0", 0.02) for l in range(N_LAYERS)]
+    traces = [S.locality_trace(np.random.default_rng([910, l]), STEPS, E, K)[0]
+              for l in range(N_LAYERS)]
+    x = S.make_layer(S.LayerConfig("cachex", T=STEPS, D=D, E=E, k=K, F=F, qtype="q8_0",
+                                   x_dtype="bf16", y_dtype="f32", seed=920), experts=False)
+    return pools, traces, x
+
+
+def _cache(moe, pools, stream):
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    hg = [pin(p[0]) for p in pools]
+    hu = [pin(p[1]) for p in pools]
+    hd = [pin(p[2]) for p in pools]
+    return moe.ExpertCache(hg, hu, hd, "q8_0", SLOTS, stream)
+
+
+def _ids(logits_row):
+    ids, _ = oracle.select(logits_row[None, :].astype(np.float64), K, True)
+    return ids[0]
+
+
+def test_cache_sequence_matches_lru_simulation(moe, stack):
+    pools, traces, _ = stack
+    cache = _cache(moe, pools, torch.cuda.Stream())
+    sims = [oracle.LRU(E, SLOTS) for _ in range(N_LAYERS)]
+    n_miss = 0
+    for t in range(STEPS):
+        for l in range(N_LAYERS):
+            ids = _ids(traces[l][t])
+            got = cache.request(l, ids)
+            want = sims[l].request(ids)
+            for g, w in zip(got, want):
+                assert np.array_equal(np.asarray(g), np.asarray(w)), (t, l, got, want)
+            n_miss += int(want[1].sum())
+    torch.cuda.synchronize()
+    hits, misses, nbytes = cache.stats()
+    assert misses == n_miss and hits + misses == STEPS * N_LAYERS * K
+    assert nbytes == n_miss * sum(p[0][0].nbytes + p[1][0].nbytes + p[2][0].nbytes
+                                  for p in pools[:1])
+    cache.close()
+
+
+def test_cached_layers_are_bit_identical_to_resident(moe, stack):
+    pools, traces, x = stack
+    stream = torch.cuda.current_stream()
+    cache = _cache(moe, pools, torch.cuda.Stream())
+    xd = torch.from_numpy(x.x_raw.view(np.int16)).cuda().view(torch.bfloat16)
+    resident = [moe.Layer(moe.ExpertPool.from_numpy(*p, "q8_0"), D, F, E, K, 1,
+                          y_dtype=torch.float32) for p in pools]
+    cached = [moe.Layer(cache.pools[l], D, F, E, K, 1, y_dtype=torch.float32)
+              for l in range(N_LAYERS)]
+    for t in range(STEPS):
+        for l in range(N_LAYERS):
+            lg = torch.from_numpy(traces[l][t:t + 1]).cuda()
+            cache.request(l, _ids(traces[l][t]), stream=stream)
+            cache.sync(l, stream=stream)
+            y_c = cached[l].forward(xd[t:t + 1], logits=lg).clone()
+            y_r = resident[l].forward(xd[t:t + 1], logits=lg).clone()
+            torch.cuda.synchronize()
+            assert torch.equal(y_c, y_r), (t, l)
+            assert torch.equal(cached[l].ids[:1], resident[l].ids[:1])
+    cache.close()
+
+
+def test_injected_copy_failure_is_reported_and_recovered(moe, stack):
+    # a failed miss copy raises; the experts of the failed request are not
+    # left mapped to half-written slots, and a retry serves the layer exactly
+    pools, traces, x = stack
+    stream = torch.cuda.current_stream()
+    cache = _cache(moe, pools, torch.cuda.Stream())
+    xd = torch.from_numpy(x.x_raw.view(np.int16)).cuda().view(torch.bfloat16)
+    first = _ids(traces[0][0])
+    cache.request(0, first, stream=stream)
+    cache.sync(0, stream=stream)
+    torch.cuda.synchronize()
+    ids, t_ids = None, None
+    for t in range(1, STEPS):
+        cand = _ids(traces[0][t])
+        if not set(cand.tolist()) <= set(first.tolist()):
+            ids, t_ids = cand, t
+            break
+    assert ids is not None
+    missing = [e for e in ids.tolist() if e not in set(first.tolist())]
+    cache.inject_copy_failure(0)
+    with pytest.raises(moe.MoeError):
+        cache.request(0, ids, stream=stream)
+    torch.cuda.synchronize()
+    smap = cache.slot_map[0].cpu().numpy()
+    assert all(smap[e] == -1 for e in missing)
+    # retry (no failure armed now) and compare the layer with the resident one
+    cache.inject_copy_failure(-1)
+    cache.request(0, ids, stream=stream)
+    cache.sync(0, stream=stream)
+    lg = torch.from_numpy(traces[0][t_ids:t_ids + 1]).cuda()
+    lay_c = moe.Layer(cache.pools[0], D, F, E, K, 1, y_dtype=torch.float32)
+    lay_r = moe.Layer(moe.ExpertPool.from_numpy(*pools[0], "q8_0"), D, F, E, K, 1,
+                      y_dtype=torch.float32)
+    y_c = lay_c.forward(xd[t_ids:t_ids + 1], logits=lg).clone()
+    y_r = lay_r.forward(xd[t_ids:t_ids + 1], logits=lg).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y_c, y_r)
+    cache.close()
