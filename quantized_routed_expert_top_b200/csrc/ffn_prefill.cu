@@ -6,7 +6,8 @@
 //
 //  * gate/up: H[p, f] = silu(x_t . Wg[f]) * (x_t . Wu[f]) for the rows p of
 //    expert e (token t = perm[p] / k), tile = 128 rows x 128 columns of F,
-//    both matrices (two MMAs of N=128 into 256 TMEM columns), K = D.
+//    both matrices (one MMA of N=256: the B stage holds the 128 gate rows,
+//    then the 128 up rows), K = D.
 //  * down:    Y[p, d] = H[p] . Wd[d], tile = 128 rows x 256 columns of D,
 //    K = F.  Y rows are fp32 in permuted order; the gate-weighted combine is
 //    the separate deterministic combine kernel.
@@ -304,61 +305,44 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
     if (warp < kPAW) {
         // ------------------------------------------ A producers
         // thread t copies 16-byte chunk t % 8 of rows t / 8 + 8 i (i < 16)
-        // with asynchronous copies straight into the swizzled stage, kPS - 1
-        // stages ahead of the one it publishes (rows past the expert's end
-        // are zero-filled).
+        // with asynchronous copies straight into the swizzled stage (rows
+        // past the expert's end are zero-filled); each thread's arrival on
+        // the stage's full barrier is itself asynchronous, made when its
+        // copies have landed, so a producer runs up to kPS stages ahead and
+        // waits only for the MMAs that free the slot it refills.
         const int j = tid & 7, r0 = tid >> 3;
-        constexpr int AH = kPS - 1;
-        int n_loc = 0;                                   // this CTA's tiles
-        for (int tau = blockIdx.x; tau < n_tiles; tau += gridDim.x) n_loc++;
-        const int n_st = n_loc * nk;                     // stages in all
-        // issue cursor
-        int gi = 0, ti = -1, ksi = nk;
-        const __half *src[kPARows];
+        int g = 0;
         bool ok = true;
-        auto issue = [&]() {
-            if (gi >= n_st) { asm volatile("cp.async.commit_group;" ::: "memory"); gi++; return; }
-            if (ksi == nk) {                             // next tile: its rows
-                ti++;
-                ksi = 0;
-                const PfTile t = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
+        for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
+            const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
+            const __half *src[kPARows];
 #pragma unroll
-                for (int i = 0; i < kPARows; i++) {
-                    const int row = t.m * kPM + r0 + 8 * i;
-                    src[i] = nullptr;
-                    if (row < t.rows) {
-                        const int p = t.seg0 + row;
-                        if (MODE == kPGateUp) {
-                            const int tok = p < Tk ? __ldg(a.perm + p) / a.k : p - Tk;
-                            src[i] = a.x16 + (size_t)tok * a.D;
-                        } else {
-                            src[i] = a.H + (size_t)p * a.F;
-                        }
+            for (int i = 0; i < kPARows; i++) {
+                const int row = t.m * kPM + r0 + 8 * i;
+                src[i] = nullptr;
+                if (row < t.rows) {
+                    const int p = t.seg0 + row;
+                    if (MODE == kPGateUp) {
+                        const int tok = p < Tk ? __ldg(a.perm + p) / a.k : p - Tk;
+                        src[i] = a.x16 + (size_t)tok * a.D;
+                    } else {
+                        src[i] = a.H + (size_t)p * a.F;
                     }
                 }
             }
-            const int s = gi % kPS;
-            if (!mbar_wait(&empty[s], ((gi / kPS) & 1) ^ 1, a.err, kErrTimeoutEmpty)) ok = false;
-            const uint32_t dst = smem_u32(stages + (size_t)s * kPStage);
+            for (int ks = 0; ks < nk; ks++, g++) {
+                const int s = g % kPS;
+                if (!mbar_wait(&empty[s], ((g / kPS) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                const uint32_t dst = smem_u32(stages + (size_t)s * kPStage);
 #pragma unroll
-            for (int i = 0; i < kPARows; i++) {
-                const __half *g = src[i] ? src[i] + ksi * kPK + 8 * j : a.x16;
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                             ::"r"(dst + sw128_off(r0 + 8 * i, j)), "l"(g), "r"(src[i] ? 16 : 0) : "memory");
+                for (int i = 0; i < kPARows; i++) {
+                    const __half *gp = src[i] ? src[i] + ks * kPK + 8 * j : a.x16;
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                                 ::"r"(dst + sw128_off(r0 + 8 * i, j)), "l"(gp), "r"(src[i] ? 16 : 0) : "memory");
+                }
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[s]))
+                             : "memory");
             }
-            asm volatile("cp.async.commit_group;" ::: "memory");
-            gi++;
-            ksi++;
-        };
-        // stage g is published before stage g + AH is issued: issuing waits
-        // for the MMAs of stage g - 1 to free their slot, and publishing
-        // first keeps that wait off the MMAs' critical path
-        for (int q = 0; q < AH; q++) issue();
-        for (int g = 0; g < n_st && ok; g++) {
-            asm volatile("cp.async.wait_group %0;" ::"n"(AH - 1) : "memory");   // stage g landed
-            fence_proxy_async_smem();
-            mbar_arrive(&full[g % kPS]);
-            issue();                                     // stage g + AH
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kPAW + kPBW) {
@@ -480,6 +464,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                     const int s = it % kPS;
                     const uint32_t ph = (it / kPS) & 1;
                     if (!mbar_wait(&full[s], ph, a.err, kErrTimeoutFull)) { ok = false; break; }
+                    fence_proxy_async_smem();    // rows written by the copiers' asynchronous copies
                     tc_fence_after();
                     const uint32_t sa = st0 + (uint32_t)s * kPStage, sb = sa + kPStageA;
 #pragma unroll
@@ -487,8 +472,8 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                         const uint64_t ad = sw128_desc(sa + kk * 32);
                         const uint32_t acc = (ks | kk) != 0;
                         if (MODE == kPGateUp) {
-                            tc_mma(dacc, ad, sw128_desc(sb + kk * 32), f16_idesc(kPNg), acc);
-                            tc_mma(dacc + kPNg, ad, sw128_desc(sb + kPNg * 128 + kk * 32), f16_idesc(kPNg), acc);
+                            // gate rows 0..127 and up rows 128..255 of the B stage: one N=256
+                            tc_mma(dacc, ad, sw128_desc(sb + kk * 32), f16_idesc(2 * kPNg), acc);
                         } else {
                             tc_mma(dacc, ad, sw128_desc(sb + kk * 32), f16_idesc(kPNd), acc);
                         }
