@@ -443,7 +443,9 @@ def roofline(wl, algo, durs, peaks, args):
 
 
 # the source files whose code runs in each traced segment's kernels
-SEGMENT_SOURCES = {"ffn_decode": ("ffn_decode.cu", "sm100.cuh")}
+SEGMENT_SOURCES = {"ffn_decode": ("ffn_decode.cu", "sm100.cuh"),
+                   "gateup": ("ffn_prefill.cu", "sm100.cuh", "moe_internal.cuh"),
+                   "down": ("ffn_prefill.cu", "sm100.cuh", "moe_internal.cuh")}
 
 
 def segment_sha(kernel):

@@ -510,8 +510,8 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                     uint32_t hv[16];
 #pragma unroll
                     for (int i = 0; i < 16; i++) {
-                        const float h0 = silu(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-                        const float h1 = silu(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+                        const float h0 = silu_fast(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+                        const float h1 = silu_fast(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
                         const __half2 hh = __floats2half2_rn(h0, h1);
                         hv[i] = *reinterpret_cast<const uint32_t *>(&hh);
                     }

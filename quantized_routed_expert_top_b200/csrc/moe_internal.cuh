@@ -100,6 +100,10 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+// the same with the hardware exponential and an approximate division (a few
+// fp32 ulp): for results rounded to fp16 right after, where those ulps vanish;
+// no slow path for huge or non-finite arguments
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // Decode one block (32 weights) from global memory into w[32] (fp32).
 // The block start is 2-byte aligned (18- or 34-byte stride), so 16-bit loads.
