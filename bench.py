@@ -2,7 +2,7 @@
 """Benchmark of the routed, block-quantized MoE FFN layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|wide]
+                    [--workload decode|prefill|wide|cache]
 
 One JSON line on rank 0.  Workloads (seeded synthetic inputs, see synthetic/):
 
@@ -14,6 +14,11 @@ One JSON line on rank 0.  Workloads (seeded synthetic inputs, see synthetic/):
   bias (skewed expert loads); 2 replicas of the pool.
 * wide: E=512, top-10, F=512 Q4_0 plus a Q8_0 shared expert, routing
   logits from a temporal-locality trace, at T = 1 and T = 2048.
+* cache: one token per step through a 40-layer stack of the decode layer in
+  Q8_0 whose experts live in pinned host memory, 51 HBM slots (40%) per
+  layer, misses copied on a side stream; also reports the hit rate, the
+  copy bytes and the exposed copy time against the same stack fully
+  resident.
 
 Timing: W untimed steps, then K steps bracketed by a barrier and a device
 synchronize, timed with CUDA events on the launching stream; max over
@@ -472,6 +477,228 @@ def ncu_traffic(kernel, workload):
     return None
 
 
+# ------------------------------------------------------------- cache arm
+def h2d_probe(torch, nbytes=1 << 30):
+    """Pinned host -> device copy bandwidth in GB/s: one 1 GiB copy after a warm-up."""
+    h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        d.copy_(h, non_blocking=True)
+        e0.record(s)
+        d.copy_(h, non_blocking=True)
+        e1.record(s)
+    s.synchronize()
+    gbs = nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9
+    del h, d
+    return gbs
+
+
+class CacheStack:
+    """A stack of the Q8_0 decode layer whose experts live in pinned host
+    memory; each layer keeps a fraction of its experts in HBM slots (LRU) and
+    copies misses on a side stream.  One step = one token through the stack,
+    routed by per-layer temporal-locality traces; the residual stream is
+    x <- bf16(x + y) after each layer."""
+
+    def __init__(self, torch, moe, n_layers, n_tokens):
+        cfg = S.CONFIGS["cache"]
+        self.torch, self.moe, self.cfg = torch, moe, cfg
+        E, k, D, F = cfg.E, cfg.k, cfg.D, cfg.F
+        self.n_layers, self.n_tokens = n_layers, n_tokens
+        self.n_slots = int(math.floor(S.CACHE_FRACTION * E))
+        # one layer's experts, the same bytes for every layer (the copy and
+        # kernel costs do not depend on the values; drawing 40 pools would
+        # take minutes of host time)
+        self.pool_np = S.gen_expert_pool(cfg.seed, E, D, F, cfg.qtype, cfg.expert_std)
+        pin = lambda a: torch.empty(a.shape, dtype=torch.uint8, pin_memory=True).copy_(torch.from_numpy(a))
+        self.host = [[pin(a) for _ in range(n_layers)] for a in self.pool_np]
+        self.sets, lg = [], []
+        for l in range(n_layers):
+            logits, sets = S.locality_trace(np.random.default_rng([cfg.seed, l]), n_tokens, E, k)
+            lg.append(logits)
+            self.sets.append(sets)
+        self.logits_host = np.ascontiguousarray(np.stack(lg, axis=1))   # [tokens, layers, E]
+        self.logits = torch.from_numpy(self.logits_host).cuda()
+        _, raw = S.gen_activations(np.random.default_rng([cfg.seed, 0x70]), 1, D, "bf16")
+        self.x0 = torch.from_numpy(raw.view(np.int16)).cuda().view(torch.bfloat16)
+        self.x = self.x0.clone()
+        self.y = torch.empty_like(self.x)
+        self.copy_stream = torch.cuda.Stream()
+        self.cache = moe.ExpertCache(*self.host, cfg.qtype, self.n_slots, self.copy_stream)
+        self.layers = [moe.Layer(self.cache.pools[l], D, F, E, k, 1) for l in range(n_layers)]
+        self.resident = None
+
+    def make_resident(self):
+        """The same stack with every expert resident in HBM (one pool per layer)."""
+        torch, moe, cfg = self.torch, self.moe, self.cfg
+        pools = []
+        for l in range(self.n_layers):
+            g, u, d = (torch.from_numpy(a).cuda() for a in self.pool_np)
+            pools.append(moe.ExpertPool(g, u, d, cfg.qtype))
+        self.resident = [moe.Layer(p, cfg.D, cfg.F, cfg.E, cfg.k, 1) for p in pools]
+
+    def token(self, t, resident=False, logits=None, trace=None):
+        stream = self.torch.cuda.current_stream()
+        lg = self.logits[t] if logits is None else logits
+        for l in range(self.n_layers):
+            if resident:
+                lay = self.resident[l]
+            else:
+                self.cache.request(l, self.sets[l][t], stream=stream)
+                self.cache.sync(l, stream=stream)
+                lay = self.layers[l]
+            lay.forward(self.x, logits=lg[l:l + 1], out=self.y, trace=trace)
+            if not resident:
+                self.cache.release(l, stream=stream)
+            self.x.add_(self.y)
+
+    def kernels_per_layer_call(self):
+        tr = self.moe.KernelTrace(n_calls=1)
+        self.resident[0].forward(self.x0, logits=self.logits[0, 0:1], out=self.y, trace=tr)
+        self.torch.cuda.synchronize()
+        kinds = [k for k, _, _ in tr.calls[0]]
+        return len(kinds) + 2 * kinds.count("ffn_decode")
+
+
+def oracle_cache_sample(pool_np, logits_host, n_layers, n_sample):
+    """The oracle on one token through the first n_sample layers of the stack."""
+    import oracle
+    oracle.build()
+    cfg = S.CONFIGS["cache"]
+    g, u, d = pool_np
+    x0, _ = S.gen_activations(np.random.default_rng([cfg.seed, 0x70]), 1, cfg.D, "bf16")
+    x = x0.astype(np.float32)
+    t = time.perf_counter()
+    for l in range(n_sample):
+        ids, gw = oracle.select(logits_host[0, l][None, :].astype(np.float64), cfg.k, cfg.renorm)
+        y = oracle.layer(x, ids, gw, g, u, d, cfg.qtype, cfg.F)
+        x = S.bf16_bits_to_f32(S.f32_to_bf16_bits((x + np.asarray(y, np.float32)).astype(np.float32)))
+    dt = time.perf_counter() - t
+    return n_sample / (dt * n_layers), dt
+
+
+def cache_layers(args):
+    cfg = S.CONFIGS["cache"]
+    gb, ub, db = S.expert_bytes(cfg.D, cfg.F, cfg.qtype)
+    layer_bytes = cfg.E * (gb + ub + db)
+    want = args.cache_layers or S.CACHE_LAYERS
+    ram = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES")
+    fit = int(0.5 * ram // layer_bytes)
+    if fit >= want:
+        return want, None
+    return max(1, fit), (f"{want} layers need {want * layer_bytes / 1e9:.1f} GB of pinned host "
+                         f"memory; this host has {ram / 1e9:.0f} GB, so {max(1, fit)} layers")
+
+
+def run_cache(args, world, rank, local):
+    import torch
+    import quantized_routed_expert_top_b200 as moe
+    from quantized_routed_expert_top_b200 import build as B
+    if rank == 0 or not os.path.exists(moe.LIB_PATH):
+        B.build()
+    barrier(world)
+    moe.lib()
+    peaks = measured_peaks()
+    n_layers, reduced = cache_layers(args)
+    n_tok = args.warmup + args.steps
+    st = CacheStack(torch, moe, n_layers, n_tok)
+    st.make_resident()
+    kpl = st.kernels_per_layer_call()
+    pcie = h2d_probe(torch)
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(resident):
+        st.x.copy_(st.x0)
+        for t in range(args.warmup):
+            st.token(t, resident)
+        torch.cuda.synchronize()
+        h0, m0, b0 = st.cache.stats()
+        barrier(world)
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        for t in range(args.warmup, n_tok):
+            st.token(t, resident)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        h1, m1, b1 = st.cache.stats()
+        return e0.elapsed_time(e1), (h1 - h0, m1 - m0, b1 - b0)
+
+    with ClockSampler(local, period_s=0.002) as clk:
+        ms_cache, (hits, misses, nbytes) = timed(False)
+    ms_res, _ = timed(True)
+    ms_cache = max_over_ranks(ms_cache, world)
+
+    # end to end: each token's x and its per-layer trace logits come from
+    # pinned host memory, its output goes back to pinned host memory; the
+    # cache continues from where the timed run left it
+    xh = st.x0.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    lh = torch.from_numpy(st.logits_host).pin_memory()
+    lbuf = torch.empty_like(st.logits[0])
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for t in range(args.warmup, n_tok):
+        st.x.copy_(xh, non_blocking=True)
+        lbuf.copy_(lh[t], non_blocking=True)
+        st.token(t, logits=lbuf)
+        yh.copy_(st.x, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world)
+
+    steps = args.steps
+    tok_s = steps * world / (ms_cache / 1e3)
+    achieved = nbytes / (ms_cache / 1e3) / 1e9
+    cfg = st.cfg
+    out = {
+        "metric": "MoE-layer tokens/s",
+        "value": round(tok_s, 3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_cache / steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype_of(cfg),
+        "data": "synthetic (seeded; random-init Q8_0 experts, per-layer locality traces)",
+        "config": {"workload": f"cache: one token per step through a {n_layers}-layer stack of the "
+                               f"MoE layer D={cfg.D} E={cfg.E} top-{cfg.k} F={cfg.F} Q8_0, experts "
+                               f"in pinned host memory, {st.n_slots} HBM slots per layer (LRU)",
+                   "layers": n_layers, "slots_per_layer": st.n_slots,
+                   "l2": "each step streams its misses from host memory; the resident comparison "
+                         "keeps one pool per layer in HBM",
+                   **({"reduced": reduced} if reduced else {})},
+        "roofline": {"kernel": "expert miss copies (host to device)", "bound": "pcie",
+                     "achieved": round(achieved, 2), "peak": round(pcie, 2), "unit": "GB/s",
+                     "frac": round(achieved / pcie, 4),
+                     "peak_source": "pinned 1 GiB host-to-device copy measured in this run",
+                     "traffic": None},
+        "cache": {"hit_rate": round(hits / max(1, hits + misses), 4),
+                  "misses_per_token": round(misses / steps, 3),
+                  "bytes_copied_per_token": int(nbytes // steps),
+                  "exposed_copy_ms_per_token": round((ms_cache - ms_res) / steps, 4),
+                  "resident_tokens_per_s": round(steps / (ms_res / 1e3), 3)},
+        "gpu_launches": kpl * n_layers * steps,
+        "e2e": {"value": round(steps * world / (ms_e2e / 1e3), 3), "unit": "tokens/s",
+                "h2d_bytes_per_step": xh.numel() * xh.element_size() + lh[0].numel() * 4,
+                "d2h_bytes_per_step": yh.numel() * yh.element_size()},
+        "clocks": clk.summary(),
+        "peaks": peaks,
+        "launch": "eager (the host LRU runs at every layer call)",
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ns = min(n_layers, 4)
+        v, dt = oracle_cache_sample(st.pool_np, st.logits_host, n_layers, ns)
+        out["cpu_baseline"] = {"value": round(v, 5), "unit": "tokens/s", "cores": os.cpu_count() or 1,
+                               "kind": "oracle",
+                               "sample": f"one token through {ns} of the {n_layers} layers (fp64), "
+                                         f"{dt:.1f} s, scaled to the whole stack"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 # ------------------------------------------------------------ prefill extra
 def extra_prefill(args, torch, moe, peaks):
     wl = Workload("prefill", torch, moe)
@@ -540,12 +767,51 @@ def cpu_baseline(wl, args):
                       f"(route + layer, fp64, OpenMP over tokens), {dt:.1f} s wall"}
 
 
+def run_reference_cache(args, world):
+    """Reference arm of the cache workload: the oracle on one token through a
+    sample of the stack's layers per step, scaled to the whole stack (the
+    oracle has no cache: it computes the same layers from the host pool)."""
+    cfg = S.CONFIGS["cache"]
+    n_layers, reduced = cache_layers(args)
+    pool = S.gen_expert_pool(cfg.seed, cfg.E, cfg.D, cfg.F, cfg.qtype, cfg.expert_std)
+    lg = np.ascontiguousarray(np.stack(
+        [S.locality_trace(np.random.default_rng([cfg.seed, l]), 1, cfg.E, cfg.k)[0] for l in range(n_layers)],
+        axis=1))
+    ns = 1
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_cache_sample(pool, lg, n_layers, ns)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_cache_sample(pool, lg, n_layers, ns)
+    dt = time.perf_counter() - t
+    value = args.steps * ns / (dt * n_layers)
+    cores = os.cpu_count() or 1
+    out = {"metric": "MoE-layer tokens/s", "value": round(value, 5), "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+           "data": "synthetic (seeded)", "impl": "reference",
+           "config": {"workload": f"cache: same {n_layers}-layer stack as the default arm; each step "
+                                  f"one token through {ns} layer, scaled to the stack",
+                      **({"reduced": reduced} if reduced else {})},
+           "cpu_baseline": {"value": round(value, 5), "unit": "tokens/s", "cores": cores,
+                            "kind": "oracle",
+                            "sample": f"one token through {ns} of {n_layers} layers per step, "
+                                      f"{args.steps} steps"},
+           "e2e": {"value": round(value, 5), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
 def run_reference(args, world, rank):
     """Reference arm: the CPU oracle, timed on the host cores."""
     if rank != 0:
         return
     name = args.workload
     cfg = S.CONFIGS[name]
+    if name == "cache":
+        run_reference_cache(args, world)
+        return
     Ts = {"decode": (1, 4, 16), "prefill": (8192,), "wide": (1, 2048)}[name]
     base = S.make_layer(cfg, T=max(Ts))
     inputs = {max(Ts): base}
@@ -595,7 +861,9 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "prefill", "wide"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "prefill", "wide", "cache"], default="decode")
+    ap.add_argument("--cache-layers", type=int, default=0,
+                    help="layers of the cache stack (default: 40, fewer if host memory is short)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--replicas", type=int, default=0,
@@ -612,7 +880,10 @@ def main():
         return
     world, rank, local = dist_setup()
     try:
-        run_ours(args, world, rank, local)
+        if args.workload == "cache":
+            run_cache(args, world, rank, local)
+        else:
+            run_ours(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -314,6 +314,15 @@ moe_status moe_cache_request(moe_cache *cache, int layer, const int32_t *ids,
                              int32_t *evicted, int *n_miss, moe_stream compute);
 /* Make `compute` wait for the copies of the layer's last request. */
 moe_status moe_cache_sync(moe_cache *cache, int layer, moe_stream compute);
+/* Optional: every kernel that reads the layer's slots for its last request
+ * has been enqueued on `compute` (call it after the layer's FFN).  Records an
+ * event there; the layer's next request then starts its miss copies as soon
+ * as that work is done, instead of after everything enqueued on `compute`
+ * up to the request, so copies for later layers overlap the FFN of earlier
+ * ones.  Consumed by that next request (without a new call, the request
+ * falls back to waiting for all of `compute`).  MOE_ERR_INVALID_ARG on a bad
+ * cache or layer. */
+moe_status moe_cache_release(moe_cache *cache, int layer, moe_stream compute);
 /* The device pool view of one layer (slot-mapped). */
 moe_status moe_cache_layer_pool(moe_cache *cache, int layer, moe_pool *out);
 moe_status moe_cache_stats(moe_cache *cache, int64_t *hits, int64_t *misses,

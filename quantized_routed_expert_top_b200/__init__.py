@@ -101,6 +101,7 @@ def lib():
         L.moe_cache_destroy.restype = None
         L.moe_cache_request.argtypes = [_v, _i, _v, _i, _v, _v, _v, C.POINTER(_i), _v]
         L.moe_cache_sync.argtypes = [_v, _i, _v]
+        L.moe_cache_release.argtypes = [_v, _i, _v]
         L.moe_cache_layer_pool.argtypes = [_v, _i, C.POINTER(Pool)]
         L.moe_cache_stats.argtypes = [_v, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
                                       C.POINTER(C.c_int64)]
@@ -401,6 +402,10 @@ class ExpertCache:
 
     def sync(self, layer: int, stream=None):
         _check(lib().moe_cache_sync(self._h, layer, _stream(stream)))
+
+    def release(self, layer: int, stream=None):
+        """Every kernel reading the layer's slots for its last request is enqueued."""
+        _check(lib().moe_cache_release(self._h, layer, _stream(stream)))
 
     def stats(self):
         h, m, b = C.c_int64(), C.c_int64(), C.c_int64()

@@ -12,7 +12,11 @@
 //    (lower expert id on equal stamps).
 // Missed experts are copied host->device with cudaMemcpyAsync on the copy
 // stream, which first waits for an event recorded on the compute stream (a
-// victim slot may still be read by earlier kernels).  The copy-done event of
+// victim slot may still be read by earlier kernels): the layer's release
+// event when the caller recorded one after the layer's last FFN
+// (moe_cache_release; the slots of a layer are read by that layer's kernels
+// only, so copies for later layers then overlap the FFN of earlier ones),
+// else an event over everything enqueued on the compute stream so far.  The copy-done event of
 // the layer lets the compute stream wait (moe_cache_sync) only when the
 // missing experts are needed, so the FFN of resident experts overlaps the
 // copies.  The layer's device slot map is refreshed from a pinned staging
@@ -33,7 +37,9 @@ struct moe_cache {
         std::vector<int64_t> stamp;         // [E]
         int64_t step = 0;
         bool pending = false;
+        bool released = false;              // release_ev marks the last use of the slots
         cudaEvent_t copied = nullptr;
+        cudaEvent_t release_ev = nullptr;
         cudaEvent_t map_done[2] = {nullptr, nullptr};
         int map_buf = 0;
     };
@@ -103,6 +109,8 @@ moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out) {
         L.expert_slot.assign(d.E, -1);
         L.stamp.assign(d.E, 0);
         st = cuda_status(cudaEventCreateWithFlags(&L.copied, cudaEventDisableTiming), "cudaEventCreate");
+        if (st == MOE_OK)
+            st = cuda_status(cudaEventCreateWithFlags(&L.release_ev, cudaEventDisableTiming), "cudaEventCreate");
         for (int b = 0; b < 2 && st == MOE_OK; b++)
             st = cuda_status(cudaEventCreateWithFlags(&L.map_done[b], cudaEventDisableTiming), "cudaEventCreate");
         for (int i = 0; i < 2 * d.E; i++) c->pinned_maps[(size_t)l * 2 * d.E + i] = -1;
@@ -124,6 +132,7 @@ void moe_cache_destroy(moe_cache *c) {
     if (!c) return;
     for (auto &L : c->layers) {
         if (L.copied) cudaEventDestroy(L.copied);
+        if (L.release_ev) cudaEventDestroy(L.release_ev);
         for (auto &ev : L.map_done) if (ev) cudaEventDestroy(ev);
     }
     if (c->compute_ready) cudaEventDestroy(c->compute_ready);
@@ -196,8 +205,12 @@ moe_status moe_cache_request(moe_cache *c, int layer, const int32_t *ids, int n,
     // copies of the misses on the copy stream, after the compute stream
     moe_status cst = MOE_OK;
     if (!miss_idx.empty()) {
-        cst = cuda_status(cudaEventRecord(c->compute_ready, cs), "cudaEventRecord");
-        if (cst == MOE_OK) cst = cuda_status(cudaStreamWaitEvent(xs, c->compute_ready, 0), "cudaStreamWaitEvent");
+        if (L.released) {
+            cst = cuda_status(cudaStreamWaitEvent(xs, L.release_ev, 0), "cudaStreamWaitEvent");
+        } else {
+            cst = cuda_status(cudaEventRecord(c->compute_ready, cs), "cudaEventRecord");
+            if (cst == MOE_OK) cst = cuda_status(cudaStreamWaitEvent(xs, c->compute_ready, 0), "cudaStreamWaitEvent");
+        }
         for (size_t m = 0; m < miss_idx.size() && cst == MOE_OK; m++) {
             const int i = miss_idx[m];
             const int e = ids[i];
@@ -238,6 +251,7 @@ moe_status moe_cache_request(moe_cache *c, int layer, const int32_t *ids, int n,
     L.stamp.swap(stamp);
     L.step = step;
     L.pending = L.pending || (!miss_idx.empty() && cst == MOE_OK);
+    L.released = false;                   // the release point covered the previous request only
 
     // device slot map of the layer
     int32_t *hm = c->pinned_maps + ((size_t)layer * 2 + buf) * d.E;
@@ -270,6 +284,14 @@ moe_status moe_cache_sync(moe_cache *c, int layer, moe_stream compute) {
     if (!L.pending) return MOE_OK;
     L.pending = false;
     return cuda_status(cudaStreamWaitEvent((cudaStream_t)compute, L.copied, 0), "cudaStreamWaitEvent");
+}
+
+moe_status moe_cache_release(moe_cache *c, int layer, moe_stream compute) {
+    if (!c || layer < 0 || layer >= c->d.n_layers) { set_error("moe_cache_release: bad cache or layer"); return MOE_ERR_INVALID_ARG; }
+    auto &L = c->layers[layer];
+    moe_status st = cuda_status(cudaEventRecord(L.release_ev, (cudaStream_t)compute), "cudaEventRecord");
+    L.released = st == MOE_OK;
+    return st;
 }
 
 moe_status moe_cache_layer_pool(moe_cache *c, int layer, moe_pool *out) {

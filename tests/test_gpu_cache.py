@@ -125,3 +125,33 @@ def test_injected_copy_failure_is_reported_and_recovered(moe, stack):
     torch.cuda.synchronize()
     assert torch.equal(y_c, y_r)
     cache.close()
+
+
+def test_released_copies_overlap_and_stay_exact(moe, stack):
+    # with a release point after every layer's FFN, a layer's miss copies wait
+    # only for that layer's previous FFN: the host enqueues all steps of all
+    # layers before synchronising once, and every output must still equal the
+    # fully resident layers' bit for bit
+    pools, traces, x = stack
+    stream = torch.cuda.current_stream()
+    cache = _cache(moe, pools, torch.cuda.Stream())
+    xd = torch.from_numpy(x.x_raw.view(np.int16)).cuda().view(torch.bfloat16)
+    resident = [moe.Layer(moe.ExpertPool.from_numpy(*p, "q8_0"), D, F, E, K, 1,
+                          y_dtype=torch.float32) for p in pools]
+    cached = [moe.Layer(cache.pools[l], D, F, E, K, 1, y_dtype=torch.float32)
+              for l in range(N_LAYERS)]
+    lg = [torch.from_numpy(traces[l]).cuda() for l in range(N_LAYERS)]
+    y_c = torch.empty((STEPS, N_LAYERS, D), dtype=torch.float32, device="cuda")
+    y_r = torch.empty_like(y_c)
+    for t in range(STEPS):
+        for l in range(N_LAYERS):
+            cache.request(l, _ids(traces[l][t]), stream=stream)
+            cache.sync(l, stream=stream)
+            cached[l].forward(xd[t:t + 1], logits=lg[l][t:t + 1], out=y_c[t, l:l + 1])
+            cache.release(l, stream=stream)
+            resident[l].forward(xd[t:t + 1], logits=lg[l][t:t + 1], out=y_r[t, l:l + 1])
+    torch.cuda.synchronize()
+    assert torch.equal(y_c, y_r)
+    hits, misses, _ = cache.stats()
+    assert misses > 0 and hits > 0
+    cache.close()
