@@ -227,9 +227,8 @@ class Workload:
         self.layers[0].forward(self.x[T], logits=self.logits[T], out=self.y[T], trace=tr)
         self.torch.cuda.synchronize()
         kinds = [k for k, _, _ in tr.calls[0]]
-        # the decode FFN segment covers two kernels (gate/up, down with the
-        # combine in its tail)
-        return len(kinds) + kinds.count("ffn_decode")
+        # the decode FFN segment covers three kernels (gate/up, down, combine)
+        return len(kinds) + 2 * kinds.count("ffn_decode")
 
     def step(self, trace=None, x=None, y=None, logits=None):
         for T in self.Ts:
@@ -582,7 +581,7 @@ class CacheStack:
         self.resident[0].forward(self.x0, logits=self.logits[0, 0:1], out=self.y, trace=tr)
         self.torch.cuda.synchronize()
         kinds = [k for k, _, _ in tr.calls[0]]
-        return len(kinds) + kinds.count("ffn_decode")
+        return len(kinds) + 2 * kinds.count("ffn_decode")
 
 
 def oracle_cache_sample(pool_np, logits_host, n_layers, n_sample):

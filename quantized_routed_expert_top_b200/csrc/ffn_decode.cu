@@ -28,15 +28,10 @@
 //    partial sums cross warps.  Codes become exact (q - off) fp16 values and
 //    the block scale multiplies the fp32 MMA result.  Each warp stores its
 //    fp32 Y rows (permuted order) to global memory.
-//  * combine (fused layer only): y[t] = sum over j of the Y row of (t, j),
-//    then the shared expert's row, in that fixed order; the gate weight is
-//    already inside Hs.  It runs in dec_down's tail: each unit counts, per
-//    token and 64-column chunk, the rows it has stored (after a memory
-//    fence); the unit that stores the chunk's last row sums it, so the sum
-//    order is fixed whichever unit finishes last.  With no counters,
-//    dec_combine runs as a kernel of its own.  Without y (the two-phase
-//    expert-cache path) the Y rows are the result: un-gated, masked experts
-//    skipped.
+//  * dec_combine (fused layer only): y[t] = sum over j of the Y row of
+//    (t, j), then the shared expert's row, in that fixed order; the gate
+//    weight is already inside Hs.  Without y (the two-phase expert-cache
+//    path) the Y rows are the result: un-gated, masked experts skipped.
 //
 // dec_down is launched with programmatic dependent launch: it copies its
 // down-projection weights while dec_gateup is still running and waits
@@ -87,7 +82,6 @@ struct DecArgs {
     int y_dtype;
     float *rows_out;               // [T*k (+T), D] Y rows, permuted order (+ shared rows)
     const int32_t *inv;            // [T*k] for the combine (fused layer)
-    int *ctr;                      // [T][D / 64] combine counters (fused layer) or NULL
     int *err;
 };
 
@@ -444,10 +438,6 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     }
     // routing results come from the previous kernel
     pdl_wait();
-    // the down grid's combine counters start at zero; it touches them only
-    // after waiting for this grid to complete
-    if (a.ctr && blockIdx.x == 0)
-        for (int i = tid; i < a.T * (a.D / 64); i += blockDim.x) a.ctr[i] = 0;
     pdl_launch_dependents();
     load_token_tables(a, tok, gw);                // in flight with the next loads
     const Active A = build_active_list(a, act);   // includes __syncthreads
@@ -696,30 +686,6 @@ __device__ __forceinline__ DnSlot dn_slot(int i, int G, int Sg) {
     return {i % G + G * (m % Sg), (uint32_t)((m / Sg) & 1)};
 }
 
-// y[t, c0 .. c0 + 63] = sum_j rows[inv[t*k + j]] (+ the shared row), in j
-// order; lane l takes columns c0 + 2l, c0 + 2l + 1.  Rows come from other
-// CTAs of this grid: loaded from L2.
-__device__ __forceinline__ void combine_chunk(const DecArgs &a, int t, int c0, int lane) {
-    const int c = c0 + 2 * lane;
-    float2 acc = make_float2(0.f, 0.f);
-    for (int j = 0; j < a.k; j++) {
-        const int r = __ldg(a.inv + (size_t)t * a.k + j);
-        const float2 v = __ldcg(reinterpret_cast<const float2 *>(a.rows_out + (size_t)r * a.D + c));
-        acc.x += v.x;
-        acc.y += v.y;
-    }
-    if (a.sF > 0) {
-        const float2 v = __ldcg(reinterpret_cast<const float2 *>(a.rows_out + (size_t)(a.T * a.k + t) * a.D + c));
-        acc.x += v.x;
-        acc.y += v.y;
-    }
-    const size_t yi = (size_t)t * a.D + c;
-    if (a.y_dtype == MOE_BF16)
-        *reinterpret_cast<__nv_bfloat162 *>((__nv_bfloat16 *)a.y + yi) = __floats2bfloat162_rn(acc.x, acc.y);
-    else
-        *reinterpret_cast<float2 *>((float *)a.y + yi) = acc;
-}
-
 template <int NT>
 __global__ void __launch_bounds__(kDThreads, 1)
 dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ DecMaps maps) {
@@ -820,12 +786,7 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
         for (int nt = 0; nt < NT; nt++)
 #pragma unroll
             for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
-        // with the fused combine a group's warps meet at a barrier after each
-        // unit, so a warp whose wait ran out still goes there (and the group
-        // leaves together); without it the warp just stops
-        const bool got = mbar_wait_warp(&full[sl.stage], sl.phase, a.err, kErrTimeoutFull);
-        if (!got && !a.ctr) break;
-        if (got) {
+        if (!mbar_wait_warp(&full[sl.stage], sl.phase, a.err, kErrTimeoutFull)) break;
         const uint32_t sbase = st_a + sl.stage * stage_bytes;
         uint32_t row = sbase + (mt * kTile + g) * pitch;
         const uint32_t r8 = 8u * pitch;
@@ -859,34 +820,6 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
                 const int r = g + ((q >> 1) << 3);
                 if (n < vi.cnt) out[(size_t)n * D + r] = acc[nt][q];
             }
-        }
-        if (a.ctr) {
-            // every row of this unit's 64 columns is stored and visible
-            __threadfence();
-            uint32_t all;
-            asm volatile(
-                "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
-                " bar.red.and.pred q, %2, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
-                : "=r"(all) : "r"((uint32_t)got), "r"(1 + grp) : "memory");
-            if (!all) break;
-            if (mt == 0) {
-                const int n = lane;                      // token row of the unit (cnt <= 16)
-                int t = 0;
-                bool last = false;
-                if (n < vi.cnt) {
-                    t = vi.shared ? n : __ldg(a.perm + vi.seg0 + n) / a.k;
-                    const int need = a.k + (a.sF > 0 ? 1 : 0);
-                    last = atomicAdd(a.ctr + t * tiles + dt, 1) == need - 1;
-                }
-                unsigned m = __ballot_sync(0xffffffffu, last);
-                if (m) __threadfence();
-                while (m) {
-                    const int src = __ffs(m) - 1;
-                    m &= m - 1;
-                    combine_chunk(a, __shfl_sync(0xffffffffu, t, src), dt * kDnRows, lane);
-                }
-            }
-        }
     }
 }
 
@@ -934,7 +867,6 @@ size_t decode_hs_halves(int T, int k, int F, int sF) {
     return (size_t)(T * k + T) * (size_t)(std::max(F, sF) + 32);
 }
 size_t decode_rows_floats(int T, int k, int D) { return (size_t)(T * k + T) * D; }
-size_t decode_ctr_ints(int T, int D) { return (size_t)T * (D / kDnRows); }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -1106,8 +1038,8 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         cudaError_t e = launch_pdl(dec_down_kernel<NT>, grid, kDThreads, smem, s, a, G, Sg, hrows, maps);
         if (e != cudaSuccess) return cuda_status(e, "dec_down_kernel");
     }
-    // ---- combine (fused layer without counters): y = sum of the gated rows (+ shared)
-    if (a.y && !a.ctr) {
+    // ---- combine (fused layer only): y = sum of the gated rows (+ shared)
+    if (a.y) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(a.T, (a.D / 4 + 255) / 256);
         cfg.blockDim = dim3(256);
@@ -1128,7 +1060,7 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
                              const int32_t *perm, const int32_t *inv, const int32_t *offsets,
                              const float *gates, const moe_pool &pool, const uint8_t *mask,
                              const moe_pool *shared, int sF, __half *Hs, void *y, int y_dtype,
-                             float *rows_out, int *err, cudaStream_t s, Tracer *tr, int *ctr) {
+                             float *rows_out, int *err, cudaStream_t s, Tracer *tr) {
     DecArgs a{};
     a.T = T; a.D = D; a.F = F; a.E = E; a.k = k; a.sF = shared ? sF : 0;
     a.perm = perm; a.offsets = offsets; a.gates = gates; a.mask = mask;
@@ -1156,7 +1088,6 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
     a.Hs = Hs; a.hrow = std::max(F, a.sF) + 32;
     a.y = y; a.y_dtype = y_dtype; a.rows_out = rows_out; a.err = err;
     a.inv = inv;
-    a.ctr = y ? ctr : nullptr;
     if (y && !rows_out) {
         set_error("decode path: the fused combine needs a rows buffer");
         return MOE_ERR_INVALID_ARG;

@@ -18,7 +18,6 @@ struct LayerWs {
     float *shH;          // [T, shared_F]
     float *sh_rows;      // [T, D]
     __half *Hs;          // decode path: g*h in fp16 fragment order
-    int32_t *ctr;        // decode path: fused-combine counters [T][D/64]
     __half *x16, *H16;   // prefill path: fp16 activations and hidden rows
 };
 
@@ -37,7 +36,6 @@ static LayerWs carve(const moe_layer_args &a, Carver &c) {
     if (decode_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0)) {
         w.Hs = c.take<__half>(decode_hs_halves(a.T, a.k, a.F, a.shared ? a.shared_F : 0));
         w.rows = c.take<float>(decode_rows_floats(a.T, a.k, a.D));
-        w.ctr = c.take<int32_t>(decode_ctr_ints(a.T, a.D));
         return w;
     }
     if (prefill_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0, a.E)) {
@@ -96,7 +94,7 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
     if (w.Hs) {
         st = launch_ffn_decode(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.inv, w.offsets,
                                gates, *a.pool, nullptr, a.shared, a.shared ? a.shared_F : 0, w.Hs,
-                               a.y, a.y_dtype, w.rows, w.status, s, tr, w.ctr);
+                               a.y, a.y_dtype, w.rows, w.status, s, tr);
         if (tr) {
             tr->end();
             if (st == MOE_OK && tr->err != cudaSuccess) {

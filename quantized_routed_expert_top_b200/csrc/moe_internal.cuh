@@ -169,8 +169,6 @@ moe_status launch_ffn_generic(const void *x, int x_dtype, int T, int D, int F, i
 bool decode_path_ok(int T, int D, int F, int sF);
 size_t decode_hs_halves(int T, int k, int F, int sF);
 size_t decode_rows_floats(int T, int k, int D);
-// per (token, 64-column chunk of D) counters of the down kernel's fused combine
-size_t decode_ctr_ints(int T, int D);
 // ffn_prefill.cu -- large T on the tensor cores: x -> fp16, gate/up grouped
 // GEMM (H fp16), down grouped GEMM (Y fp32 rows, then the combine kernel)
 bool prefill_path_ok(int T, int D, int F, int sF, int E);
@@ -188,7 +186,7 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
                              const int32_t *perm, const int32_t *inv, const int32_t *offsets,
                              const float *gates, const moe_pool &pool, const uint8_t *mask,
                              const moe_pool *shared, int sF, __half *Hs, void *y, int y_dtype,
-                             float *rows_out, int *err, cudaStream_t s, Tracer *tr, int *ctr = nullptr);
+                             float *rows_out, int *err, cudaStream_t s, Tracer *tr);
 // combine.cu
 moe_status launch_combine(const float *rows, const int32_t *inv, const float *gates,
                           int T, int k, int D, const float *shared_rows, void *y,
