@@ -5,9 +5,9 @@
 // (rows of the permuted order) by its weights.  Two launches:
 //
 //  * gate/up: H[p, f] = silu(x_t . Wg[f]) * (x_t . Wu[f]) for the rows p of
-//    expert e (token t = perm[p] / k), tile = 128 rows x 128 columns of F,
-//    both matrices (one MMA of N=256: the B stage holds the 128 gate rows,
-//    then the 128 up rows), K = D.
+//    expert e (token t = perm[p] / k), tile = 128 rows x 128 columns of F of
+//    both matrices (one MMA of N=256: the weight stage holds the 128 gate
+//    rows, then the 128 up rows), K = D.
 //  * down:    Y[p, d] = H[p] . Wd[d], tile = 128 rows x 256 columns of D,
 //    K = F.  Y rows are fp32 in permuted order; the gate-weighted combine is
 //    the separate deterministic combine kernel.
@@ -15,12 +15,17 @@
 // The weights stay in their ggml blocks in HBM.  They cannot feed the tensor
 // cores directly (a per-32 fp16 scale), so B-producer warps dequantise each
 // K-slice (64 weights of 256 rows) into fp16, d*q rounded once, written in the
-// 128-byte-swizzled K-major layout the MMA descriptors name.  A-producer
-// warps copy the activation rows (gathered through the permutation from an
-// fp16 copy of x, or the contiguous rows of H) the same way.  One thread
-// issues tcgen05.mma (M=128, K=16 steps) and commits each stage back to its
-// producers; two TMEM accumulators (2 x 256 columns) let the epilogue warps
-// drain one tile while the next accumulates.
+// 128-byte-swizzled K-major layout the MMA descriptors name.  Their input is
+// a ring of raw windows (four blocks of every weight row, two K-slices, per
+// tensor copy); each B warp works through its 32 rows on its own and
+// releases a window when done, the last release letting the window be
+// refilled.  A-producer warps copy the activation rows (gathered through the
+// permutation from an fp16 copy of x, or the contiguous rows of H) into their
+// own ring with asynchronous copies whose arrivals are themselves
+// asynchronous.  One thread issues tcgen05.mma (M=128, K=16 steps) once both
+// rings hold the stage and commits each stage back to both; two TMEM
+// accumulators (2 x 256 columns) let the epilogue warps drain one tile while
+// the next accumulates.
 //
 // Numerics: weights d*q rounded to fp16 (relative error <= 2^-11 per weight),
 // activations fp16 (x is bf16 or fp32 on input: exact in fp16 over the
@@ -38,28 +43,33 @@ constexpr int kPM = 128;                 // tile rows = MMA M
 constexpr int kPK = 64;                  // K per stage: one 128-byte row of fp16
 constexpr int kPNg = 128;                // gate/up: F columns per tile (per matrix)
 constexpr int kPNd = 256;                // down: D columns per tile
-constexpr int kPS = 3;                   // fp16 operand stages
-constexpr int kPR = 3;                   // raw weight windows in flight
+constexpr int kPSA = 3;                  // activation stages (16 KB)
+constexpr int kPSB = 2;                  // dequantised weight stages (32 KB)
+constexpr int kPR = 3;                   // raw weight windows in flight (36 KB, two K stages each)
 constexpr int kPStageA = kPM * kPK * 2;  // 16 KB
 constexpr int kPStageB = 256 * kPK * 2;  // 32 KB (256 weight rows)
-constexpr int kPStage = kPStageA + kPStageB;
+
 constexpr int kPAW = 2, kPBW = 8, kPEW = 4;                  // A copiers, B dequantisers, epilogue
 constexpr int kPMmaWarp = kPAW + kPBW;                       // warp 10
 constexpr int kPThreads = (kPAW + kPBW + 1 + kPEW) * 32;     // 480
 constexpr int kPARows = kPM / (kPAW * 32 / 8);               // rows per A thread (16)
 constexpr int kPTmemCols = 512;                              // 2 accumulators x 256
-constexpr int kPRawRow = 80;             // raw window of one weight row (Q8_0: 5 x 16 B)
-constexpr int kPRaw = 256 * kPRawRow;    // one raw window buffer (20 KB)
-// stages | raw ring | barriers + TMEM slot (256 B) | segs, tcum [2][E+2]
+// A raw window holds four blocks (K = 128, two MMA stages) of each of the
+// 256 weight rows: the 16-byte-aligned 144 bytes (Q8_0) or 80 bytes (Q4_0)
+// around them; four blocks start 0 or 8 bytes past a 16-byte boundary.
+constexpr int kPRawRow = 144;
+constexpr int kPRaw = 256 * kPRawRow;    // one raw window buffer (36 KB)
+// A ring | B ring | raw ring | barriers + TMEM slot (256 B) | segs, tcum [2][E+2]
 __host__ __device__ inline size_t pf_smem_bytes(int E) {
-    return (size_t)kPS * kPStage + (size_t)kPR * kPRaw + 256 + 2 * (size_t)(E + 2) * 4 + 1024;
+    return (size_t)kPSA * kPStageA + (size_t)kPSB * kPStageB + (size_t)kPR * kPRaw + 256 +
+           2 * (size_t)(E + 2) * 4 + 1024;
 }
 
 enum : int { kPGateUp = 0, kPDown = 1 };
 
 // Tensor maps over the weight pools (8-byte elements, one row of blocks per
-// tensor row), boxes of one raw window (the 16-byte-aligned 80 or 48 bytes
-// holding a block pair) x 128 rows (gate, up) or 256 rows (down).
+// tensor row), boxes of one raw window (the 16-byte-aligned 144 or 80 bytes
+// holding four blocks) x 128 rows (gate, up) or 256 rows (down).
 struct PfMaps {
     CUtensorMap w0, w1;           // gate/up: gate, up; down: down, -
     CUtensorMap s0, s1;           // the shared expert's
@@ -141,16 +151,6 @@ __host__ __device__ constexpr uint32_t f16_idesc(int n) {
 // byte offset of 16-byte chunk j (0..7) of row r in a 128-byte-swizzled tile
 __device__ __forceinline__ uint32_t sw128_off(int r, int j) {
     return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
-}
-
-// named barrier 2 over the B-producer warps, returning the AND of `ok`
-__device__ __forceinline__ bool bar_and_b(bool ok) {
-    uint32_t r;
-    asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
-        " bar.red.and.pred q, 2, %2, p;\n selp.u32 %0, 1, 0, q;\n}"
-        : "=r"(r) : "r"((uint32_t)ok), "n"(kPBW * 32) : "memory");
-    return r != 0;
 }
 
 // ------------------------------------------------------------- dequantise
@@ -239,16 +239,20 @@ template <int MODE>
 __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const __grid_constant__ PfMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_pf[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint8_t *stages = smem_pf + ((1024u - (smem_u32(smem_pf) & 1023u)) & 1023u);
-    uint8_t *raw = stages + (size_t)kPS * kPStage;  // ring of raw weight windows
-    uint64_t *full = (uint64_t *)(raw + (size_t)kPR * kPRaw);
-    uint64_t *empty = full + kPS;
-    uint64_t *accf = empty + kPS;                  // [2] accumulator ready
-    uint64_t *acce = accf + 2;                     // [2] accumulator drained
-    uint64_t *rfull = acce + 2;                    // [kPR] raw window landed
-    uint32_t *tmem_slot = (uint32_t *)(rfull + kPR);
-    int *segs = (int *)(tmem_slot + 4);            // [nv + 1] segment starts
-    int *tcum = segs + (a.E + 2);                  // [nv + 1] first tile of each expert
+    uint8_t *ringA = smem_pf + ((1024u - (smem_u32(smem_pf) & 1023u)) & 1023u);
+    uint8_t *ringB = ringA + (size_t)kPSA * kPStageA;
+    uint8_t *raw = ringB + (size_t)kPSB * kPStageB;           // raw weight windows
+    uint64_t *fullA = (uint64_t *)(raw + (size_t)kPR * kPRaw);
+    uint64_t *emptyA = fullA + kPSA;
+    uint64_t *fullB = emptyA + kPSA;
+    uint64_t *emptyB = fullB + kPSB;
+    uint64_t *rfull = emptyB + kPSB;                          // raw window landed
+    uint64_t *rempty = rfull + kPR;                           // raw window read by every B warp
+    uint64_t *accf = rempty + kPR;                            // [2] accumulator ready
+    uint64_t *acce = accf + 2;                                // [2] accumulator drained
+    uint32_t *tmem_slot = (uint32_t *)(acce + 2);
+    int *segs = (int *)(tmem_slot + 4);                       // [nv + 1] segment starts
+    int *tcum = segs + (a.E + 2);                             // [nv + 1] first tile of each expert
 
     const int Tk = a.T * a.k;
     const int nv = a.E + (a.shared ? 1 : 0);
@@ -258,15 +262,22 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
     const int nt = N / BN, nk = K / kPK;
 
     if (tid == 0) {
-        for (int s = 0; s < kPS; s++) {
-            mbar_init(&full[s], (kPAW + kPBW) * 32);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kPSA; s++) {
+            mbar_init(&fullA[s], kPAW * 32);
+            mbar_init(&emptyA[s], 1);
+        }
+        for (int s = 0; s < kPSB; s++) {
+            mbar_init(&fullB[s], kPBW * 32);
+            mbar_init(&emptyB[s], 1);
+        }
+        for (int r = 0; r < kPR; r++) {
+            mbar_init(&rfull[r], 1);
+            mbar_init(&rempty[r], kPBW);
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], kPEW * 32);
         }
-        for (int r = 0; r < kPR; r++) mbar_init(&rfull[r], 1);
         fence_mbar_init();
     }
     if (warp == kPMmaWarp) {
@@ -301,15 +312,12 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
     }
     __syncthreads();
     const int n_tiles = tcum[nv];
+    int n_loc = 0;                                   // this CTA's tiles
+    for (int tau = blockIdx.x; tau < n_tiles; tau += gridDim.x) n_loc++;
+    const int n_st = n_loc * nk;                     // K stages in all
 
     if (warp < kPAW) {
         // ------------------------------------------ A producers
-        // thread t copies 16-byte chunk t % 8 of rows t / 8 + 8 i (i < 16)
-        // with asynchronous copies straight into the swizzled stage (rows
-        // past the expert's end are zero-filled); each thread's arrival on
-        // the stage's full barrier is itself asynchronous, made when its
-        // copies have landed, so a producer runs up to kPS stages ahead and
-        // waits only for the MMAs that free the slot it refills.
         const int j = tid & 7, r0 = tid >> 3;
         int g = 0;
         bool ok = true;
@@ -331,45 +339,49 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                 }
             }
             for (int ks = 0; ks < nk; ks++, g++) {
-                const int s = g % kPS;
-                if (!mbar_wait(&empty[s], ((g / kPS) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
-                const uint32_t dst = smem_u32(stages + (size_t)s * kPStage);
+                const int s = g % kPSA;
+                if (!mbar_wait(&emptyA[s], ((g / kPSA) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                const uint32_t dst = smem_u32(ringA + (size_t)s * kPStageA);
 #pragma unroll
                 for (int i = 0; i < kPARows; i++) {
                     const __half *gp = src[i] ? src[i] + ks * kPK + 8 * j : a.x16;
                     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                                  ::"r"(dst + sw128_off(r0 + 8 * i, j)), "l"(gp), "r"(src[i] ? 16 : 0) : "memory");
                 }
-                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[s]))
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&fullA[s]))
                              : "memory");
             }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kPAW + kPBW) {
         // ------------------------------------------------- B producers
-        // Raw windows (the 16-byte-aligned bytes holding a K-slice's block
-        // pair, for all 256 weight rows of the tile) arrive by tensor copies
-        // kPR - 1 stages ahead; thread t dequantises weight row t of the
-        // current window into the swizzled fp16 stage.
-        const int bt = tid - kPAW * 32;
-        int n_loc = 0;
-        for (int tau = blockIdx.x; tau < n_tiles; tau += gridDim.x) n_loc++;
-        const int n_st = n_loc * nk;
-        // raw-window issue cursor (thread bt == 0 only)
-        int gi = 0, ti = -1, ksi = nk;
+        // Raw windows (the 16-byte-aligned bytes holding four blocks = two
+        // K stages, for all 256 weight rows of the tile) arrive by tensor
+        // copies kPR - 1 windows ahead.  Each warp dequantises its 32 rows of the
+        // window into the swizzled fp16 stage on its own; lane 0 of the
+        // first warp refills a raw buffer once all warps have read it.
+        const int bw = warp - kPAW, bt = tid - kPAW * 32;
+        const bool issuer = bw == 0 && lane == 0;
+        const int nw = nk / 2;                           // windows per tile
+        const int n_win = n_loc * nw;
+        int gi = 0, ti = -1, wi = nw;                    // window issue cursor
         PfTile tI{};
-        auto issue = [&]() {
-            if (gi >= n_st) return;
-            if (ksi == nk) {
+        auto issue = [&]() -> bool {
+            if (gi >= n_win) return true;
+            if (gi >= kPR) {                             // the buffer's previous window is read
+                const int q = gi - kPR;
+                if (!mbar_wait(&rempty[q % kPR], (uint32_t)((q / kPR) & 1), a.err, kErrTimeoutEmpty)) return false;
+            }
+            if (wi == nw) {
                 ti++;
-                ksi = 0;
+                wi = 0;
                 tI = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
             }
             const bool sh = tI.v == a.E;
             const bool q8 = sh ? a.sq8 != 0 : a.q8 != 0;
             const int bs = q8 ? kQ8Bytes : kQ4Bytes;
-            const int wb = q8 ? 80 : 48;                         // window bytes
-            const int x = (int)(((size_t)ksi * 2 * bs & ~(size_t)15) / 8);
+            const int wb = q8 ? 144 : 80;                        // window bytes
+            const int x = (int)(((size_t)wi * 4 * bs & ~(size_t)15) / 8);
             const int slot = sh ? 0 : (a.slot_map ? __ldg(a.slot_map + tI.v) : tI.v);
             const int r = gi % kPR;
             uint8_t *dst = raw + (size_t)r * kPRaw;
@@ -382,76 +394,85 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                 tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, slot * a.D + tI.n * kPNd, &rfull[r]);
             }
             gi++;
-            ksi++;
+            wi++;
+            return true;
         };
-        if (bt == 0)
-            for (int q = 0; q < kPR - 1; q++) issue();
         bool ok = true;
-        int g = 0;
+        if (issuer)
+            for (int q = 0; q < kPR - 1 && ok; q++) ok = issue();
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        int g = 0, gw = 0;                               // stage, window counters
         for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
             const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
             const bool q8 = (t.v == a.E) ? a.sq8 != 0 : a.q8 != 0;
-            const int wb = q8 ? 80 : 48;
-            for (int ks = 0; ks < nk; ks++, g++) {
-                // every producer is done with the window of stage g - 1: its
-                // buffer takes the window of stage g + kPR - 1; a wait that
-                // ran out anywhere ends every producer's loop here
-                ok = bar_and_b(ok);
-                if (!ok) break;
-                if (bt == 0) issue();
-                const int r = g % kPR;
-                if (!mbar_wait(&rfull[r], (uint32_t)((g / kPR) & 1), a.err, kErrTimeoutFull)) { ok = false; continue; }
-                uint4 c[1][8];
-                const int o = ks & 3;                            // word offset of the pair
+            const int wb = q8 ? 144 : 80;
+            for (int ks = 0; ks < nk && ok; ks++, g++) {
+                const int half = ks & 1;                         // which block pair of the window
+                if (half == 0) {
+                    bool iok = true;
+                    if (issuer) iok = issue();                   // window gw + kPR - 1
+                    ok = __shfl_sync(0xffffffffu, iok ? 1 : 0, 0) != 0;
+                    if (!ok) break;
+                }
+                const int r = gw % kPR;
+                if (half == 0 &&
+                    !mbar_wait_warp(&rfull[r], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutFull)) { ok = false; break; }
+                uint4 c[8];
+                // the pair starts 8 * (group % 2) + (2 * bs) * half bytes into the window
+                const int odd = (ks >> 1) & 1;
+                const uint8_t *rp = raw + (size_t)r * kPRaw + bt * wb;
+                if (q8) {
+                    // words 16 * half .. +19 hold the pair at word 2*odd + half
+                    uint32_t w[20];
 #pragma unroll
-                for (int h = 0; h < 1; h++) {
-                    const uint8_t *rp = raw + (size_t)r * kPRaw + bt * wb;
-                    if (q8) {
-                        uint32_t w[20];
+                    for (int q = 0; q < 5; q++) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(rp + 64 * half + 16 * q);
+                        w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                    }
+                    switch (2 * odd + half) {
+                    case 0: dq_pair_q8<0>(w, c); break;
+                    case 1: dq_pair_q8<1>(w, c); break;
+                    case 2: dq_pair_q8<2>(w, c); break;
+                    default: dq_pair_q8<3>(w, c); break;
+                    }
+                } else {
+                    // words 8 * half .. +11 hold the pair at word 2*odd + half
+                    uint32_t w[12];
 #pragma unroll
-                        for (int q = 0; q < 5; q++) {
-                            const uint4 v = *reinterpret_cast<const uint4 *>(rp + 16 * q);
-                            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-                        }
-                        switch (o) {
-                        case 0: dq_pair_q8<0>(w, c[h]); break;
-                        case 1: dq_pair_q8<1>(w, c[h]); break;
-                        case 2: dq_pair_q8<2>(w, c[h]); break;
-                        default: dq_pair_q8<3>(w, c[h]); break;
-                        }
-                    } else {
-                        uint32_t w[12];
-#pragma unroll
-                        for (int q = 0; q < 3; q++) {
-                            const uint4 v = *reinterpret_cast<const uint4 *>(rp + 16 * q);
-                            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-                        }
-                        switch (o) {
-                        case 0: dq_pair_q4<0>(w, c[h]); break;
-                        case 1: dq_pair_q4<1>(w, c[h]); break;
-                        case 2: dq_pair_q4<2>(w, c[h]); break;
-                        default: dq_pair_q4<3>(w, c[h]); break;
-                        }
+                    for (int q = 0; q < 3; q++) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(rp + 32 * half + 16 * q);
+                        w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                    }
+                    switch (2 * odd + half) {
+                    case 0: dq_pair_q4<0>(w, c); break;
+                    case 1: dq_pair_q4<1>(w, c); break;
+                    case 2: dq_pair_q4<2>(w, c); break;
+                    default: dq_pair_q4<3>(w, c); break;
                     }
                 }
-                const int s = g % kPS;
-                if (!mbar_wait(&empty[s], ((g / kPS) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; continue; }
-                uint8_t *dst = stages + (size_t)s * kPStage + kPStageA;
+                if (half == 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&rempty[r]);      // this warp is done with the window
+                    gw++;
+                }
+                const int s = g % kPSB;
+                if (!mbar_wait_warp(&emptyB[s], ((g / kPSB) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                uint8_t *dst = ringB + (size_t)s * kPStageB;
 #pragma unroll
-                for (int jj = 0; jj < 8; jj++) *reinterpret_cast<uint4 *>(dst + sw128_off(bt, jj)) = c[0][jj];
+                for (int jj = 0; jj < 8; jj++) *reinterpret_cast<uint4 *>(dst + sw128_off(bt, jj)) = c[jj];
                 fence_proxy_async_smem();
-                mbar_arrive(&full[s]);
+                mbar_arrive(&fullB[s]);
             }
-            ok = bar_and_b(ok);                                  // a failure in a tile's last stage
         }
         // windows still in flight must land before the CTA exits
-        if (bt == 0)
-            for (; g < gi; g++)
-                mbar_wait(&rfull[g % kPR], (uint32_t)((g / kPR) & 1), a.err, kErrTimeoutDrain);
+        if (issuer)
+            for (; gw < gi; gw++)
+                mbar_wait(&rfull[gw % kPR], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutDrain);
     } else if (warp == kPMmaWarp) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t st0 = smem_u32(stages);
+            const uint32_t sA0 = smem_u32(ringA), sB0 = smem_u32(ringB);
+            const uint32_t idesc = f16_idesc(256);       // gate|up rows, or 256 down rows
             uint32_t it = 0;
             int lt = 0;
             bool ok = true;
@@ -461,24 +482,17 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                 tc_fence_after();
                 const uint32_t dacc = tmem + (uint32_t)(ab * 256);
                 for (int ks = 0; ks < nk; ks++, it++) {
-                    const int s = it % kPS;
-                    const uint32_t ph = (it / kPS) & 1;
-                    if (!mbar_wait(&full[s], ph, a.err, kErrTimeoutFull)) { ok = false; break; }
-                    fence_proxy_async_smem();    // rows written by the copiers' asynchronous copies
+                    const int sa = it % kPSA, sb = it % kPSB;
+                    if (!mbar_wait(&fullA[sa], (it / kPSA) & 1, a.err, kErrTimeoutFull) ||
+                        !mbar_wait(&fullB[sb], (it / kPSB) & 1, a.err, kErrTimeoutFull)) { ok = false; break; }
+                    fence_proxy_async_smem();
                     tc_fence_after();
-                    const uint32_t sa = st0 + (uint32_t)s * kPStage, sb = sa + kPStageA;
+                    const uint32_t aa = sA0 + (uint32_t)sa * kPStageA, bb = sB0 + (uint32_t)sb * kPStageB;
 #pragma unroll
-                    for (int kk = 0; kk < kPK / 16; kk++) {
-                        const uint64_t ad = sw128_desc(sa + kk * 32);
-                        const uint32_t acc = (ks | kk) != 0;
-                        if (MODE == kPGateUp) {
-                            // gate rows 0..127 and up rows 128..255 of the B stage: one N=256
-                            tc_mma(dacc, ad, sw128_desc(sb + kk * 32), f16_idesc(2 * kPNg), acc);
-                        } else {
-                            tc_mma(dacc, ad, sw128_desc(sb + kk * 32), f16_idesc(kPNd), acc);
-                        }
-                    }
-                    tc_commit(&empty[s]);        // the stage is free once these MMAs are done
+                    for (int kk = 0; kk < kPK / 16; kk++)
+                        tc_mma(dacc, sw128_desc(aa + kk * 32), sw128_desc(bb + kk * 32), idesc, (ks | kk) != 0);
+                    tc_commit(&emptyA[sa]);      // the stages are free once these MMAs are done
+                    tc_commit(&emptyB[sb]);
                 }
                 if (!ok) break;
                 tc_commit(&accf[ab]);            // the tile's accumulator is complete
@@ -503,15 +517,15 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
             if (MODE == kPGateUp) {
 #pragma unroll 1
                 for (int c0 = 0; c0 < kPNg; c0 += 32) {
-                    uint32_t g[32], u[32];
-                    tc_ld32(tq + c0, g);
-                    tc_ld32(tq + kPNg + c0, u);
+                    uint32_t gv[32], uv[32];
+                    tc_ld32(tq + c0, gv);
+                    tc_ld32(tq + kPNg + c0, uv);
                     tc_wait_ld();
                     uint32_t hv[16];
 #pragma unroll
                     for (int i = 0; i < 16; i++) {
-                        const float h0 = silu_fast(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-                        const float h1 = silu_fast(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+                        const float h0 = silu_fast(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
+                        const float h1 = silu_fast(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
                         const __half2 hh = __floats2half2_rn(h0, h1);
                         hv[i] = *reinterpret_cast<const uint32_t *>(&hh);
                     }
@@ -570,7 +584,7 @@ __global__ void __launch_bounds__(256) pf_convert_kernel(const XT *__restrict__ 
 // row then sits at the end of its 16-byte window, so no window reads past a row
 bool prefill_path_ok(int T, int D, int F, int sF, int E) {
     return T > 16 && D % kPNd == 0 && F % kPNg == 0 && D % 256 == 0 && F % 256 == 0 &&
-           (sF == 0 || sF == F) && E <= MOE_MAX_EXPERTS;
+           (sF == 0 || sF == F) && E <= MOE_MAX_EXPERTS && pf_smem_bytes(E) <= 227 * 1024;
 }
 
 size_t prefill_x16_halves(int T, int D) { return (size_t)T * D; }
@@ -669,7 +683,7 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
     if (e != cudaSuccess) return cuda_status(e, "pf_convert_kernel");
     // weight tensor maps: raw windows of 80 (Q8_0) or 48 (Q4_0) bytes
     const int br = pool.qtype == MOE_Q8_0 ? kQ8Bytes : kQ4Bytes;
-    const int wr = pool.qtype == MOE_Q8_0 ? 80 : 48;
+    const int wr = pool.qtype == MOE_Q8_0 ? 144 : 80;
     PfMaps mg, md;
     memset(&mg, 0, sizeof(mg));
     memset(&md, 0, sizeof(md));
@@ -681,7 +695,7 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
         return st;
     if (shared) {
         const int bsh = shared->qtype == MOE_Q8_0 ? kQ8Bytes : kQ4Bytes;
-        const int wsh = shared->qtype == MOE_Q8_0 ? 80 : 48;
+        const int wsh = shared->qtype == MOE_Q8_0 ? 144 : 80;
         if ((st = pf_encode(&mg.s0, shared->gate, (size_t)(D / QK) * bsh, F, wsh, kPNg)) ||
             (st = pf_encode(&mg.s1, shared->up, (size_t)(D / QK) * bsh, F, wsh, kPNg)) ||
             (st = pf_encode(&md.s0, shared->down, (size_t)(F / QK) * bsh, D, wsh, kPNd)))
