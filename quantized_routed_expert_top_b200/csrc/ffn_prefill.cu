@@ -580,8 +580,10 @@ __global__ void __launch_bounds__(256) pf_convert_kernel(const XT *__restrict__ 
 }
 
 // ------------------------------------------------------------------- host
-// K (D for gate/up, F for down) a multiple of 256: the last block pair of a
-// row then sits at the end of its 16-byte window, so no window reads past a row
+// K (D for gate/up, F for down) a multiple of 256: a row is then a multiple of
+// 272 (Q8_0) or 144 (Q4_0) bytes, its last four blocks start 8 bytes past a
+// 16-byte boundary and their window ends exactly at the row's end, so no
+// window reads past a row
 bool prefill_path_ok(int T, int D, int F, int sF, int E) {
     return T > 16 && D % kPNd == 0 && F % kPNg == 0 && D % 256 == 0 && F % 256 == 0 &&
            (sF == 0 || sF == F) && E <= MOE_MAX_EXPERTS && pf_smem_bytes(E) <= 227 * 1024;
@@ -681,7 +683,7 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
         pf_convert_kernel<float><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const float *)x, x16, n8);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "pf_convert_kernel");
-    // weight tensor maps: raw windows of 80 (Q8_0) or 48 (Q4_0) bytes
+    // weight tensor maps: raw windows of 144 (Q8_0) or 80 (Q4_0) bytes
     const int br = pool.qtype == MOE_Q8_0 ? kQ8Bytes : kQ4Bytes;
     const int wr = pool.qtype == MOE_Q8_0 ? 144 : 80;
     PfMaps mg, md;
