@@ -39,6 +39,20 @@
  *  - Shapes: D % 32 == 0, F % 32 == 0 (blocks run along the reduction
  *    dimension), 1 <= k <= E <= MOE_MAX_EXPERTS, k <= MOE_MAX_TOPK, T >= 0.
  *    T == 0 is a no-op that succeeds.
+ *  - Errors found on the GPU (a bounded wait inside a kernel that ran out,
+ *    an expert whose slot is outside [0, n_slots)) cannot be returned by the
+ *    enqueuing call.  The kernels record the first such error in a status
+ *    word: the first int32 of the workspace.  moe_workspace_status() reads
+ *    it (and can clear it); a new workspace is zero-filled, so it starts at
+ *    MOE_DEV_OK.  A kernel that records an error skips the work it concerns
+ *    and returns; the outputs that work would have written are unspecified,
+ *    every other output is exact.
+ *  - Numerics: activations (x) and the hidden rows h are rounded to fp16
+ *    inside the FFN kernels (bf16 has 8 significant bits, fp16 11, so a bf16
+ *    x in fp16's normal range [2^-14, 65504] converts exactly).  Inputs
+ *    with |x| > 65504 overflow to inf and values under 2^-14 lose bits;
+ *    keep activations inside that range (post-normalisation hidden states
+ *    are).  Routing stays fp32 throughout.
  *  - Pointers named "device" must be device memory (or managed); "host"
  *    means host memory (pinned where stated).
  */
@@ -69,6 +83,16 @@ typedef enum {
     MOE_ERR_WORKSPACE = 7           /* workspace missing or too small */
 } moe_status;
 
+/* Codes of the device status word (see moe_workspace_status). */
+typedef enum {
+    MOE_DEV_OK = 0,
+    MOE_DEV_TIMEOUT_FULL = 1,      /* a consumer waited too long for data */
+    MOE_DEV_TIMEOUT_EMPTY = 2,     /* a producer waited too long for a free buffer */
+    MOE_DEV_TIMEOUT_DRAIN = 3,     /* copies still in flight at exit waited too long */
+    MOE_DEV_BAD_SLOT = 4,          /* an expert with tokens maps outside [0, n_slots) */
+    MOE_DEV_TIMEOUT_MMA = 5        /* tensor-core work did not complete in time */
+} moe_device_status;
+
 /* ggml type ids */
 typedef enum { MOE_Q4_0 = 2, MOE_Q8_0 = 8 } moe_qtype;
 
@@ -79,7 +103,10 @@ typedef struct CUstream_st *moe_stream;
 
 /* A device expert pool (see the layout above).  slot_of_expert maps expert
  * id -> slot (device int32[E]); NULL means slot = expert id.  Every expert
- * that a call reaches must map to a slot in [0, n_slots). */
+ * that a call reaches (tokens routed to it, and not masked out) must map to
+ * a slot in [0, n_slots): the kernels check each one before forming any
+ * address, skip an expert that does not, and record MOE_DEV_BAD_SLOT in the
+ * workspace's status word (an expert cache marks non-resident experts -1). */
 typedef struct {
     int32_t qtype;                  /* moe_qtype */
     int32_t n_slots;
@@ -94,6 +121,17 @@ const char *moe_last_error(void);
 const char *moe_version(void);
 /* Bytes of one 32-weight block of a quant type; 0 for an unknown type. */
 int moe_block_bytes(int32_t qtype);
+
+/* moe_workspace_status: the device status word of a workspace (its first
+ * int32, written by the kernels of the calls that used it; see the
+ * conventions above).  Waits for the work enqueued on `stream` so far, then
+ * stores the word in *code (a moe_device_status) and, if clear != 0, resets
+ * it to MOE_DEV_OK (the reset is enqueued on `stream` and waited for).
+ * Returns MOE_OK when the word is MOE_DEV_OK, MOE_ERR_TIMEOUT for the
+ * timeout codes, MOE_ERR_INVALID_ARG for MOE_DEV_BAD_SLOT (with a message),
+ * MOE_ERR_CUDA if the copy fails.  Blocks the calling thread; not for use
+ * inside stream capture. */
+moe_status moe_workspace_status(void *workspace, int32_t *code, int clear, moe_stream stream);
 
 /* ------------------------------------------------------------- routing
  * moe_route: router logits, softmax, top-k and renormalised gates.
@@ -128,11 +166,18 @@ moe_status moe_route(const void *x, int32_t x_dtype, const float *w_router,
  *   T <= 16 and ceil(D/32) * T * E <= 524288 (else MOE_ERR_SHAPE, with the
  *   limit in the message).
  *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before capturing any stream.  Every call on a device shares the array
- *   and leaves its contents behind (the completion counter is cleared at the
- *   start of each call); calls that overlap on the GPU race, so serialise
- *   them (one stream, or events between streams). */
+ *   (cudaGetSymbolAddress) with that device current.  Under CUDA's lazy
+ *   module loading (the default) that first call may also load the
+ *   library's device code, and loading allocates device memory: make one
+ *   call per device at start-up, before the point where allocation is
+ *   forbidden and before capturing any stream.  Later calls allocate
+ *   nothing.  The address stays valid for the life of the device's primary
+ *   context: after cudaDeviceReset on that device this entry point must not
+ *   be called again until the process has reloaded the library.  Every call
+ *   on a device shares the array and leaves its contents behind (the
+ *   completion counter is cleared at the start of each call); calls that
+ *   overlap on the GPU race, so serialise them (one stream, or events
+ *   between streams). */
 moe_status moe_route_noalloc(const void *x, int32_t x_dtype, const float *w_router,
                              const float *bias, int T, int D, int E, int k, int renorm,
                              int32_t *ids, float *gates, float *logits, moe_stream stream);
@@ -158,6 +203,12 @@ moe_status moe_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
  * the segment of offsets that holds pos):
  *   out_rows[pos, :] = W_down,e ( silu(W_gate,e x_t) * (W_up,e x_t) )
  * (no gate weight; moe_combine applies it).
+ * Kernels, by shape (the same as moe_layer_forward's):
+ *   1 <= T <= 16, D in {256, 512, 768, 1024, 2048}, F % 256 == 0, F <= 1024:
+ *     the dequant-fused grouped GEMV (mma.sync, TMA-streamed weights);
+ *   T > 16, D % 256 == 0, F % 256 == 0, E <= 720: the grouped GEMM on the
+ *     tcgen05 tensor cores (weights dequantised to fp16 in shared memory);
+ *   any other shape: a portable CUDA-core kernel (correct, not tuned).
  *   x           device [T, D], x_dtype F32 or BF16.
  *   perm,offsets from moe_permute.
  *   pool        expert weights (see moe_pool); pool->qtype fixes the format.
@@ -203,7 +254,32 @@ moe_status moe_combine(const float *rows, const int32_t *inv, const float *gates
  *   y, y_dtype           device [T, D] output (F32 or BF16)
  *   ids_out, gates_out   device [T, k] or NULL: routing decisions
  *   logits_out           device fp32 [T, E] or NULL
- *   trace                NULL, or per-kernel timing of this call (moe_trace) */
+ *   trace                NULL, or per-kernel timing of this call (moe_trace)
+ *   phases               0 = the whole layer; else an OR of MOE_PHASE_* bits
+ *                        (below): the parts this call runs
+ *   expert_mask          device uint8 [E] or NULL: the FFN part of this call
+ *                        runs only experts with a nonzero entry (NULL: all)
+ *   counts_out, offsets_out, perm_out, inv_out
+ *                        device int32 [E], [E+1], [T*k], [T*k] or NULL: the
+ *                        permutation as moe_permute defines it; when given,
+ *                        the call keeps its permutation there instead of in
+ *                        the workspace.
+ * Phases let an expert cache overlap its miss copies with the FFN of the
+ * experts already resident (kongchang article, "From Static Allocation to
+ * Dynamic Scheduling"; FreeToken wiki explainer on hiding transfer time):
+ *   call 1  ROUTE | FFN | SHARED, expert_mask = resident experts
+ *           (or ROUTE alone, when the ids must reach the host first)
+ *   wait    moe_cache_sync(...)  (the misses' copies)
+ *   call 2  FFN | COMBINE, expert_mask = the experts just copied
+ * The calls of one layer step must get the same arguments (except phases
+ * and expert_mask) and the same workspace, on one stream.  Each expert row
+ * is computed by the same kernel in the same order whatever the split, so
+ * the result is bit-identical to a single call. */
+#define MOE_PHASE_ROUTE 1u    /* logits, top-k, gates, permutation */
+#define MOE_PHASE_FFN 2u      /* routed experts' FFN (those expert_mask admits) */
+#define MOE_PHASE_SHARED 4u   /* the shared expert's FFN */
+#define MOE_PHASE_COMBINE 8u  /* gate-weighted combine into y */
+#define MOE_PHASE_ALL 15u
 
 /* Per-kernel timing of one moe_layer_forward call.  The caller creates
  * `capacity` CUDA events (cudaEvent_t, timing enabled) and passes them in
@@ -243,7 +319,7 @@ typedef struct {
     int32_t renorm;
     int32_t x_dtype;
     int32_t y_dtype;
-    int32_t reserved;
+    int32_t phases;
     const void *x;
     const float *w_router;
     const float *bias;
@@ -255,6 +331,11 @@ typedef struct {
     float *gates_out;
     float *logits_out;
     moe_trace *trace;
+    const uint8_t *expert_mask;
+    int32_t *counts_out;
+    int32_t *offsets_out;
+    int32_t *perm_out;
+    int32_t *inv_out;
 } moe_layer_args;
 
 size_t moe_layer_workspace_size(const moe_layer_args *args);
@@ -325,8 +406,14 @@ moe_status moe_cache_sync(moe_cache *cache, int layer, moe_stream compute);
 moe_status moe_cache_release(moe_cache *cache, int layer, moe_stream compute);
 /* The device pool view of one layer (slot-mapped). */
 moe_status moe_cache_layer_pool(moe_cache *cache, int layer, moe_pool *out);
+/* Counters since moe_cache_init: hits, misses, bytes copied, and
+ * exposed_ns, the time the compute stream spent waiting in moe_cache_sync
+ * for miss copies (measured on the GPU between two events recorded around
+ * the wait; copies that finished before the compute stream reached the
+ * sync point add nothing).  Waits for the compute stream to pass the sync
+ * points it has not yet passed.  Any output pointer may be NULL. */
 moe_status moe_cache_stats(moe_cache *cache, int64_t *hits, int64_t *misses,
-                           int64_t *bytes_copied);
+                           int64_t *bytes_copied, int64_t *exposed_ns);
 
 #ifdef __cplusplus
 }

@@ -25,6 +25,11 @@ _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_QTYPE",
           3: "MOE_ERR_SHAPE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_CAPACITY",
           6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_WORKSPACE"}
+# device status word codes (moe_device_status)
+DEV_OK, DEV_TIMEOUT_FULL, DEV_TIMEOUT_EMPTY, DEV_TIMEOUT_DRAIN, DEV_BAD_SLOT, DEV_TIMEOUT_MMA = range(6)
+# moe_layer_forward phases
+PHASE_ROUTE, PHASE_FFN, PHASE_SHARED, PHASE_COMBINE = 1, 2, 4, 8
+PHASE_ALL = 15
 
 
 class MoeError(RuntimeError):
@@ -52,12 +57,14 @@ class Trace(C.Structure):
 class LayerArgs(C.Structure):
     _fields_ = [("T", C.c_int32), ("D", C.c_int32), ("E", C.c_int32), ("k", C.c_int32),
                 ("F", C.c_int32), ("shared_F", C.c_int32), ("renorm", C.c_int32),
-                ("x_dtype", C.c_int32), ("y_dtype", C.c_int32), ("reserved", C.c_int32),
+                ("x_dtype", C.c_int32), ("y_dtype", C.c_int32), ("phases", C.c_int32),
                 ("x", C.c_void_p), ("w_router", C.c_void_p), ("bias", C.c_void_p),
                 ("logits_in", C.c_void_p), ("pool", C.POINTER(Pool)),
                 ("shared", C.POINTER(Pool)), ("y", C.c_void_p), ("ids_out", C.c_void_p),
                 ("gates_out", C.c_void_p), ("logits_out", C.c_void_p),
-                ("trace", C.POINTER(Trace))]
+                ("trace", C.POINTER(Trace)), ("expert_mask", C.c_void_p),
+                ("counts_out", C.c_void_p), ("offsets_out", C.c_void_p),
+                ("perm_out", C.c_void_p), ("inv_out", C.c_void_p)]
 
 
 class CacheDesc(C.Structure):
@@ -84,6 +91,7 @@ def lib():
         L.moe_last_error.restype = C.c_char_p
         L.moe_version.restype = C.c_char_p
         L.moe_block_bytes.argtypes = [C.c_int32]
+        L.moe_workspace_status.argtypes = [_v, C.POINTER(C.c_int32), _i, _v]
         L.moe_route_workspace_size.restype = _sz
         L.moe_route_workspace_size.argtypes = [_i, _i, _i, _i]
         L.moe_route.argtypes = [_v, C.c_int32, _v, _v, _i, _i, _i, _i, _i, _v, _v, _v, _v, _sz, _v]
@@ -104,7 +112,9 @@ def lib():
         L.moe_cache_release.argtypes = [_v, _i, _v]
         L.moe_cache_layer_pool.argtypes = [_v, _i, C.POINTER(Pool)]
         L.moe_cache_stats.argtypes = [_v, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
-                                      C.POINTER(C.c_int64)]
+                                      C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
+        L.moe_route_noalloc.argtypes = [_v, C.c_int32, _v, _v, _i, _i, _i, _i, _i, _v, _v, _v,
+                                        _v]
         L.moe_cache_debug_fail_copy.argtypes = [_v, _i]
         L.moe_cache_debug_fail_copy.restype = None
         _lib = L
@@ -140,6 +150,14 @@ def _qt(q):
 
 def _zeros_ws(nbytes, device):
     return torch.zeros(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def workspace_status(ws, clear: bool = True, stream=None):
+    """moe_workspace_status: (status, code) of a workspace's device status
+    word; waits for the stream.  status is MOE_OK when code == DEV_OK."""
+    code = C.c_int32(0)
+    st = lib().moe_workspace_status(_p(ws), C.byref(code), int(clear), _stream(stream))
+    return st, code.value
 
 
 # ----------------------------------------------------------------- pools
@@ -199,18 +217,25 @@ def permute(ids, E: int, stream=None):
 
 
 def expert_ffn(x, perm, offsets, pool: ExpertPool, k: int, F: int, mask=None, out=None,
-               stream=None):
-    """moe_expert_ffn -> out_rows [T*k, D] fp32 in permuted order."""
-    _dev(x, perm, offsets, mask, out)
+               stream=None, ws=None):
+    """moe_expert_ffn -> out_rows [T*k, D] fp32 in permuted order.  ``ws``:
+    an optional caller workspace (zero-filled uint8 tensor of at least
+    expert_ffn_workspace_size bytes), e.g. to read its status word after."""
+    _dev(x, perm, offsets, mask, out, ws)
     T, D = x.shape
     E = offsets.numel() - 1
     if out is None:
         out = torch.empty((T * k, D), dtype=torch.float32, device=x.device)
-    ws = _zeros_ws(lib().moe_expert_ffn_workspace_size(T, k, D, F), x.device)
+    if ws is None:
+        ws = _zeros_ws(expert_ffn_workspace_size(T, k, D, F), x.device)
     _check(lib().moe_expert_ffn(_p(x), _DT[x.dtype], T, D, F, E, k, _p(perm), _p(offsets),
                                 C.byref(pool.c), _p(mask), _p(out), _p(ws), ws.numel(),
                                 _stream(stream)))
     return out
+
+
+def expert_ffn_workspace_size(T: int, k: int, D: int, F: int) -> int:
+    return int(lib().moe_expert_ffn_workspace_size(T, k, D, F))
 
 
 def combine(rows, inv, gates, shared_rows=None, y_dtype=torch.bfloat16, out=None, stream=None):
@@ -249,7 +274,8 @@ class Layer:
         self.gates = torch.empty((T_max, k), dtype=torch.float32, device=self.device)
         self.ws = _zeros_ws(self.workspace_size(T_max), self.device)
 
-    def _args(self, T, x, logits, y, logits_out=None, trace=None):
+    def _args(self, T, x, logits, y, logits_out=None, trace=None, phases=0, mask=None,
+              routing_out=None):
         a = LayerArgs()
         a.T, a.D, a.E, a.k, a.F = T, self.D, self.E, self.k, self.F
         a.shared_F = self.shared_F if self.shared is not None else 0
@@ -267,6 +293,10 @@ class Layer:
         a.gates_out = self.gates.data_ptr()
         a.logits_out = None if logits_out is None else logits_out.data_ptr()
         a.trace = C.pointer(trace) if trace is not None else None
+        a.phases = int(phases)
+        a.expert_mask = None if mask is None else mask.data_ptr()
+        if routing_out is not None:
+            a.counts_out, a.offsets_out, a.perm_out, a.inv_out = (t.data_ptr() for t in routing_out)
         return a
 
     def workspace_size(self, T):
@@ -274,9 +304,21 @@ class Layer:
         a.x = 1  # non-null placeholders: the size depends on shapes only
         return lib().moe_layer_workspace_size(C.byref(a))
 
-    def forward(self, x, logits=None, out=None, logits_out=None, stream=None, trace=None):
-        """Run the layer; ``trace`` is an optional KernelTrace."""
-        _dev(x, logits, out, logits_out)
+    def routing_buffers(self, T=None):
+        """Device int32 (counts [E], offsets [E+1], perm [T*k], inv [T*k]) for
+        ``forward(routing_out=...)``."""
+        T = self.T_max if T is None else T
+        n = max(T * self.k, 1)
+        mk = lambda m: torch.empty(m, dtype=torch.int32, device=self.device)
+        return (mk(self.E), mk(self.E + 1), mk(n)[: T * self.k], mk(n)[: T * self.k])
+
+    def forward(self, x, logits=None, out=None, logits_out=None, stream=None, trace=None,
+                phases=0, mask=None, routing_out=None):
+        """Run the layer (or the parts ``phases`` names, PHASE_* bits; 0 =
+        all); ``mask``: device uint8 [E] restricting the FFN part;
+        ``routing_out``: a routing_buffers() tuple that receives the
+        permutation; ``trace`` is an optional KernelTrace."""
+        _dev(x, logits, out, logits_out, mask)
         T = (x if x is not None else logits).shape[0]
         if T > self.T_max:
             raise ValueError(f"T={T} exceeds T_max={self.T_max}")
@@ -284,7 +326,8 @@ class Layer:
             raise ValueError(f"x dtype {x.dtype} != {self.x_dtype}")
         if out is None:
             out = torch.empty((T, self.D), dtype=self.y_dtype, device=self.device)
-        a = self._args(T, x, logits, out, logits_out, trace.c if trace is not None else None)
+        a = self._args(T, x, logits, out, logits_out, trace.c if trace is not None else None,
+                       phases, mask, routing_out)
         _check(lib().moe_layer_forward(C.byref(a), _p(self.ws), self.ws.numel(), _stream(stream)))
         if trace is not None:
             trace.record()
@@ -408,9 +451,17 @@ class ExpertCache:
         _check(lib().moe_cache_release(self._h, layer, _stream(stream)))
 
     def stats(self):
+        """(hits, misses, bytes copied)."""
         h, m, b = C.c_int64(), C.c_int64(), C.c_int64()
-        _check(lib().moe_cache_stats(self._h, C.byref(h), C.byref(m), C.byref(b)))
+        _check(lib().moe_cache_stats(self._h, C.byref(h), C.byref(m), C.byref(b), None))
         return h.value, m.value, b.value
+
+    def exposed_ns(self):
+        """Time the compute stream has waited in sync() for copies (ns);
+        waits for the compute stream to pass its pending sync points."""
+        e = C.c_int64()
+        _check(lib().moe_cache_stats(self._h, None, None, None, C.byref(e)))
+        return e.value
 
     def inject_copy_failure(self, nth: int):
         lib().moe_cache_debug_fail_copy(self._h, nth)

@@ -3,6 +3,7 @@
 // carving and kernel dispatch.  No call allocates device memory.
 #include "moe_internal.cuh"
 #include "moe_paths.cuh"
+#include "sm100.cuh"
 
 #include <cstdarg>
 #include <cstdio>
@@ -97,6 +98,37 @@ int moe_block_bytes(int32_t qtype) {
     }
 }
 
+// ------------------------------------------------------ device status word
+moe_status moe_workspace_status(void *workspace, int32_t *code, int clear, moe_stream stream) {
+    g_err.clear();
+    if (!workspace || !code) { set_error("moe_workspace_status: NULL workspace or code"); return MOE_ERR_INVALID_ARG; }
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t v = 0;
+    moe_status st = cuda_status(cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s),
+                                "moe_workspace_status: read");
+    if (st == MOE_OK) st = cuda_status(cudaStreamSynchronize(s), "moe_workspace_status: wait");
+    if (st != MOE_OK) return st;
+    *code = v;
+    if (clear && v != kErrNone) {
+        st = cuda_status(cudaMemsetAsync(workspace, 0, sizeof(int32_t), s), "moe_workspace_status: clear");
+        if (st == MOE_OK) st = cuda_status(cudaStreamSynchronize(s), "moe_workspace_status: wait");
+        if (st != MOE_OK) return st;
+    }
+    switch (v) {
+    case kErrNone: return MOE_OK;
+    case kErrBadSlot:
+        set_error("device status: an expert with tokens maps to a slot outside [0, n_slots); "
+                  "its rows were skipped");
+        return MOE_ERR_INVALID_ARG;
+    case kErrTimeoutFull: case kErrTimeoutEmpty: case kErrTimeoutDrain: case kErrTimeoutMma:
+        set_error("device status: a bounded wait inside a kernel ran out (code %d)", (int)v);
+        return MOE_ERR_TIMEOUT;
+    default:
+        set_error("device status: unknown code %d", (int)v);
+        return MOE_ERR_INVALID_ARG;
+    }
+}
+
 // ----------------------------------------------------------------- route
 size_t moe_route_workspace_size(int T, int D, int E, int k) {
     return route_ws_bytes(T < 0 ? 0 : T, D, E, k);
@@ -121,9 +153,9 @@ moe_status moe_route(const void *x, int32_t x_dtype, const float *w_router, cons
         return MOE_ERR_WORKSPACE;
     }
     bool permuted = false;
-    // the route workspace starts with 64 words of counters; word 32 is the
-    // status word of the bounded waits
-    int *err = (int *)workspace + 32;
+    // the route workspace starts with 64 words: word 0 is the status word,
+    // word 1 the split-K completion ticket
+    int *err = (int *)workspace;
     return launch_route_permute(x, x_dtype, w_router, bias, T, D, E, k, renorm, ids, gates,
                                 logits, nullptr, nullptr, nullptr, nullptr, err, workspace,
                                 ws_bytes, (cudaStream_t)stream, nullptr, &permuted);
@@ -142,13 +174,27 @@ moe_status moe_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
 }
 
 // ------------------------------------------------------------ expert FFN
+// Workspace pieces of moe_expert_ffn: the status word, then the decode
+// path's fp16 hidden rows, or the tensor-core path's fp16 activations and
+// hidden rows, or the portable path's fp32 hidden rows.  E is not an
+// argument of the size query, so for T > 16 it covers both of the latter.
 size_t moe_expert_ffn_workspace_size(int T, int k, int D, int F) {
-    Carver c(nullptr, 0);
     T = T < 0 ? 0 : T;
+    Carver c(nullptr, 0);
     c.take<int>(16);
-    if (decode_path_ok(T, D, F, 0)) c.take<__half>(decode_hs_halves(T, k, F, 0));
-    else c.take<float>((size_t)T * k * F);
-    return c.off;
+    if (decode_path_ok(T, D, F, 0)) {
+        c.take<__half>(decode_hs_halves(T, k, F, 0));
+        return c.off;
+    }
+    Carver g = c;
+    g.take<float>((size_t)T * k * F);
+    if (T > 16 && D % 256 == 0 && F % 256 == 0) {
+        Carver p = c;
+        p.take<__half>(prefill_x16_halves(T, D));
+        p.take<__half>(prefill_h_halves(T, k, F, 0));
+        return p.off > g.off ? p.off : g.off;
+    }
+    return g.off;
 }
 
 moe_status moe_expert_ffn(const void *x, int32_t x_dtype, int T, int D, int F, int E, int k,
@@ -172,12 +218,19 @@ moe_status moe_expert_ffn(const void *x, int32_t x_dtype, int T, int D, int F, i
     if (decode_path_ok(T, D, F, 0)) {
         __half *Hs = c.take<__half>(decode_hs_halves(T, k, F, 0));
         return launch_ffn_decode(x, x_dtype, T, D, F, E, k, perm, nullptr, offsets, nullptr, *pool,
-                                 expert_mask, nullptr, 0, Hs, nullptr, MOE_F32, out_rows, status,
-                                 (cudaStream_t)stream, nullptr);
+                                 expert_mask, true, nullptr, 0, false, Hs, nullptr, MOE_F32,
+                                 out_rows, status, (cudaStream_t)stream, nullptr);
+    }
+    if (prefill_path_ok(T, D, F, 0, E)) {
+        __half *x16 = c.take<__half>(prefill_x16_halves(T, D));
+        __half *H16 = c.take<__half>(prefill_h_halves(T, k, F, 0));
+        return launch_ffn_prefill(x, x_dtype, T, D, F, E, k, perm, offsets, *pool, expert_mask,
+                                  true, nullptr, 0, x16, H16, out_rows, status,
+                                  (cudaStream_t)stream, nullptr);
     }
     float *H = c.take<float>((size_t)T * k * F);
     return launch_ffn_generic(x, x_dtype, T, D, F, E, k, perm, offsets, *pool, expert_mask, H,
-                              out_rows, (cudaStream_t)stream);
+                              out_rows, status, (cudaStream_t)stream);
 }
 
 // --------------------------------------------------------------- combine
@@ -221,9 +274,16 @@ moe_status moe_layer_forward(const moe_layer_args *a, void *workspace, size_t ws
         return MOE_ERR_INVALID_ARG;
     }
     if (a->renorm != 0 && a->renorm != 1) { set_error("moe_layer_forward: renorm must be 0 or 1"); return MOE_ERR_INVALID_ARG; }
+    if ((unsigned)a->phases & ~MOE_PHASE_ALL) {
+        set_error("moe_layer_forward: phases %d has bits outside MOE_PHASE_ALL", (int)a->phases);
+        return MOE_ERR_INVALID_ARG;
+    }
     if (a->T == 0) return MOE_OK;
-    if (!a->x || !a->y || (!a->w_router && !a->logits_in)) {
-        set_error("moe_layer_forward: NULL x, y, or both w_router and logits_in");
+    const unsigned ph = a->phases ? (unsigned)a->phases : MOE_PHASE_ALL;
+    const bool need_x = (ph & (MOE_PHASE_FFN | MOE_PHASE_SHARED)) || ((ph & MOE_PHASE_ROUTE) && a->w_router);
+    if ((need_x && !a->x) || ((ph & MOE_PHASE_COMBINE) && !a->y) ||
+        ((ph & MOE_PHASE_ROUTE) && !a->w_router && !a->logits_in)) {
+        set_error("moe_layer_forward: NULL x, y, or both w_router and logits_in, for phases %u", ph);
         return MOE_ERR_INVALID_ARG;
     }
     size_t need = layer_ws_bytes(*a);

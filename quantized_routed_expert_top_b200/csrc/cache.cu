@@ -22,6 +22,11 @@
 // copies.  The layer's device slot map is refreshed from a pinned staging
 // buffer (two per layer, alternating; each reuse waits, with a time limit,
 // for the copy that last read it).
+// Exposed copy time: moe_cache_sync brackets the compute stream's wait with
+// two timing events; the time between them is how long the compute stream
+// stood still for copies (zero when the copies had already landed).  The
+// pairs are read back lazily (at the next sync once complete, or in
+// moe_cache_stats).
 #include "moe_internal.cuh"
 
 #include <chrono>
@@ -49,9 +54,28 @@ struct moe_cache {
     int64_t hits = 0, misses = 0, bytes = 0;
     int fail_copy_at = -1;                // test hook: fail the n-th copy
     int copies_issued = 0;
+    // exposed copy time: (before, after) event pairs around each wait
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> wait_pairs;
+    std::vector<cudaEvent_t> free_events;
+    int64_t exposed_ns = 0;
 };
 
 namespace moe {
+static cudaEvent_t take_event(moe_cache *c) {
+    if (!c->free_events.empty()) {
+        cudaEvent_t e = c->free_events.back();
+        c->free_events.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Add the completed wait pairs to exposed_ns (all of them if `all`, waiting
+// for each; else only those already complete).
+static moe_status harvest_waits(moe_cache *c, bool all);
+
 static moe_status wait_event_bounded(cudaEvent_t ev, double seconds) {
     auto t0 = std::chrono::steady_clock::now();
     for (;;) {
@@ -66,6 +90,28 @@ static moe_status wait_event_bounded(cudaEvent_t ev, double seconds) {
         std::this_thread::yield();
     }
 }
+static moe_status harvest_waits(moe_cache *c, bool all) {
+    size_t keep = 0;
+    moe_status st = MOE_OK;
+    for (size_t i = 0; i < c->wait_pairs.size(); i++) {
+        auto pr = c->wait_pairs[i];
+        if (st == MOE_OK && all) st = wait_event_bounded(pr.second, 60.0);
+        const bool done = st == MOE_OK && cudaEventQuery(pr.second) == cudaSuccess;
+        if (!done) {
+            c->wait_pairs[keep++] = pr;
+            continue;
+        }
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, pr.first, pr.second) == cudaSuccess)
+            c->exposed_ns += (int64_t)((double)ms * 1e6);
+        c->free_events.push_back(pr.first);
+        c->free_events.push_back(pr.second);
+    }
+    c->wait_pairs.resize(keep);
+    cudaGetLastError();     // a not-ready query is not an error of any later call
+    return st;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -136,6 +182,11 @@ void moe_cache_destroy(moe_cache *c) {
         for (auto &ev : L.map_done) if (ev) cudaEventDestroy(ev);
     }
     if (c->compute_ready) cudaEventDestroy(c->compute_ready);
+    for (auto &pr : c->wait_pairs) {
+        cudaEventDestroy(pr.first);
+        cudaEventDestroy(pr.second);
+    }
+    for (auto ev : c->free_events) cudaEventDestroy(ev);
     if (c->pinned_maps) cudaFreeHost(c->pinned_maps);
     delete c;
 }
@@ -283,7 +334,22 @@ moe_status moe_cache_sync(moe_cache *c, int layer, moe_stream compute) {
     auto &L = c->layers[layer];
     if (!L.pending) return MOE_OK;
     L.pending = false;
-    return cuda_status(cudaStreamWaitEvent((cudaStream_t)compute, L.copied, 0), "cudaStreamWaitEvent");
+    cudaStream_t cs = (cudaStream_t)compute;
+    harvest_waits(c, false);
+    cudaEvent_t e0 = take_event(c), e1 = take_event(c);
+    if (e0 && e1 && cudaEventRecord(e0, cs) == cudaSuccess) {
+        moe_status st = cuda_status(cudaStreamWaitEvent(cs, L.copied, 0), "cudaStreamWaitEvent");
+        if (st != MOE_OK) return st;
+        st = cuda_status(cudaEventRecord(e1, cs), "cudaEventRecord");
+        if (st != MOE_OK) return st;
+        c->wait_pairs.emplace_back(e0, e1);
+        return MOE_OK;
+    }
+    // no timing events: wait without measuring
+    if (e0) c->free_events.push_back(e0);
+    if (e1) c->free_events.push_back(e1);
+    cudaGetLastError();
+    return cuda_status(cudaStreamWaitEvent(cs, L.copied, 0), "cudaStreamWaitEvent");
 }
 
 moe_status moe_cache_release(moe_cache *c, int layer, moe_stream compute) {
@@ -307,11 +373,17 @@ moe_status moe_cache_layer_pool(moe_cache *c, int layer, moe_pool *out) {
     return MOE_OK;
 }
 
-moe_status moe_cache_stats(moe_cache *c, int64_t *hits, int64_t *misses, int64_t *bytes_copied) {
+moe_status moe_cache_stats(moe_cache *c, int64_t *hits, int64_t *misses, int64_t *bytes_copied,
+                           int64_t *exposed_ns) {
     if (!c) { set_error("moe_cache_stats: NULL cache"); return MOE_ERR_INVALID_ARG; }
     if (hits) *hits = c->hits;
     if (misses) *misses = c->misses;
     if (bytes_copied) *bytes_copied = c->bytes;
+    if (exposed_ns) {
+        moe_status st = harvest_waits(c, true);
+        if (st != MOE_OK) return st;
+        *exposed_ns = c->exposed_ns;
+    }
     return MOE_OK;
 }
 

@@ -47,6 +47,7 @@
 
 #include <cuda.h>
 #include <algorithm>
+#include <climits>
 #include <cstring>
 
 namespace moe {
@@ -66,8 +67,11 @@ constexpr int kGuCols = 8;
 constexpr int kMaxTk = 16 * MOE_MAX_TOPK;       // T*k entries the token tables hold
 
 struct DecArgs {
-    int T, D, F, E, k, sF;
+    int T, D, F, E, k, sF;         // sF: shared expert's F when this call runs it, else 0
     int q8, sq8;                   // routed / shared experts are Q8_0 (else Q4_0)
+    int routed;                    // this call runs the routed experts (those mask admits)
+    int n_slots;                   // slots of the routed pool
+    int comb_shared;               // the combine adds the shared rows (layer has one)
     const int32_t *perm, *offsets;
     const float *gates;            // [T, k] or NULL (rows mode: no gate)
     const uint8_t *mask;           // [E] or NULL
@@ -172,6 +176,12 @@ struct Active {
 // slot of every active expert (ascending id), then the raw offsets and
 // slots.  All threads load the raw tables in one round of global loads;
 // one warp then compacts them, so per-unit lookups stay in shared memory.
+// An expert is active when it has tokens, this call runs routed experts and
+// the mask (if any) admits it.  An active expert whose slot lies outside
+// [0, n_slots) is left out and recorded as kErrBadSlot: no address is ever
+// formed from such a slot.
+constexpr int kMaskedOut = INT_MIN;
+
 __device__ Active build_active_list(const DecArgs &a, int *act) {
     __shared__ int s_n;
     const int E1 = a.E + 1;
@@ -179,7 +189,8 @@ __device__ Active build_active_list(const DecArgs &a, int *act) {
     int *roff = aslot + E1, *ron = roff + E1;
     for (int e = threadIdx.x; e <= a.E; e += blockDim.x) {
         roff[e] = __ldg(a.offsets + e);
-        if (e < a.E) ron[e] = (!a.mask || __ldg(a.mask + e)) ? slot_of(a.slot_map, e) : -1;
+        if (e < a.E)
+            ron[e] = (a.routed && (!a.mask || __ldg(a.mask + e))) ? slot_of(a.slot_map, e) : kMaskedOut;
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -192,7 +203,10 @@ __device__ Active build_active_list(const DecArgs &a, int *act) {
                 s0 = roff[e];
                 c = roff[e + 1] - s0;
                 sl = ron[e];
-                on = c > 0 && (!a.mask || sl >= 0);
+                const bool want = c > 0 && sl != kMaskedOut;
+                const bool bad = want && (sl < 0 || sl >= a.n_slots);
+                if (bad && a.err) atomicCAS(a.err, 0, kErrBadSlot);
+                on = want && !bad;
             }
             const unsigned b = __ballot_sync(0xffffffffu, on);
             if (on) {
@@ -240,6 +254,16 @@ __device__ __forceinline__ Virt virt(const DecArgs &a, const int *act, int n_rou
         r.q8 = a.sq8 != 0;
     }
     return r;
+}
+
+// Producer's exit: wait (bounded) until the last fill of every stage it used
+// has landed, so no copy still writes shared memory when the CTA ends.  The
+// full barrier of a stage completes the phase of a fill when its bytes
+// arrive, whatever the consumers did.
+__device__ __forceinline__ void drain_fills(uint64_t *full, int S, uint32_t used, uint32_t last_ph,
+                                            int *err) {
+    for (int s = 0; s < S; s++)
+        if ((used >> s) & 1u) mbar_wait(&full[s], (last_ph >> s) & 1u, err, kErrTimeoutDrain);
 }
 
 // Token tables in shared memory: tok[pos] = token of permuted entry pos
@@ -492,6 +516,7 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
             const uint64_t pol = l2_evict_first_policy();    // weights: read once
             int stage = 0;
             uint32_t phase = 0;
+            uint32_t used = 0u, last_ph = 0u;                 // per stage: issued, parity of its last fill
             bool ok = true;
             for (int i = 0; i < n_local && ok; i++) {
                 const int v = utab[i].x, tile = utab[i].y;
@@ -508,14 +533,14 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
                     const int x = sl * gg.sb * bs / 8;
                     tma_load_2d_hint(dst, mg, x, y, &full[stage], pol);
                     tma_load_2d_hint(dst + kTile * gg.pitch, mu, x, y, &full[stage], pol);
+                    used |= 1u << stage;
+                    last_ph = (last_ph & ~(1u << stage)) | (phase << stage);
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
             }
-            // drain: every issued stage must have landed before the CTA exits
-            for (int s2 = 0; s2 < S; s2++) {
-                mbar_wait(&empty[stage], phase ^ 1, a.err, kErrTimeoutDrain);
-                if (++stage == S) { stage = 0; phase ^= 1; }
-            }
+            // drain: every copy this thread issued must have landed before the
+            // CTA exits (also when a consumer gave up waiting)
+            drain_fills(full, S, used, last_ph, a.err);
         }
         return;
     }
@@ -724,6 +749,7 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
         if (lane == 0) {
             const uint64_t pol = l2_evict_first_policy();    // weights: read once
             bool ok = true, waited = false;
+            uint32_t used = 0u, last_ph = 0u;
             int pend_s[kMaxStages], pend_v[kMaxStages];
             int npend = 0;
             auto issue_h = [&](int st, int v) {
@@ -742,6 +768,8 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
                 mbar_arrive_expect_tx(&full[sl.stage], (uint32_t)(kDnRows * pitch + vi.cnt * hbytes));
                 tma_load_2d_hint(dst, vi.shared ? &maps.sdown : &maps.down, 0,
                                  (vi.shared ? 0 : (int)vi.slot * D) + dt * kDnRows, &full[sl.stage], pol);
+                used |= 1u << sl.stage;
+                last_ph = (last_ph & ~(1u << sl.stage)) | (sl.phase << sl.stage);
                 if (waited) {
                     issue_h(sl.stage, v);
                 } else {
@@ -759,12 +787,8 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
                 pdl_wait();
                 for (int q = 0; q < npend; q++) issue_h(pend_s[q], pend_v[q]);
             }
-            // drain: wait for the consumers of the last S units (one per stage)
-            for (int q = i - S; q < i; q++) {
-                if (q < 0) continue;
-                const DnSlot sl = dn_slot(q, G, Sg);
-                mbar_wait(&empty[sl.stage], sl.phase, a.err, kErrTimeoutDrain);
-            }
+            // drain: every copy issued (weights and Hs) must have landed
+            drain_fills(full, S, used, last_ph, a.err);
         }
         return;
     }
@@ -991,6 +1015,8 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
     moe_status st = encode_maps(a, n_slots, max_sb, &maps);
     if (st != MOE_OK) return st;
     const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
+    // gate/up and down run when this call has routed experts or the shared one
+    if (a.routed || a.sF > 0) {
     // ---- gate/up
     {
         const int nbD = a.D / QK;
@@ -1038,6 +1064,7 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         cudaError_t e = launch_pdl(dec_down_kernel<NT>, grid, kDThreads, smem, s, a, G, Sg, hrows, maps);
         if (e != cudaSuccess) return cuda_status(e, "dec_down_kernel");
     }
+    }
     // ---- combine (fused layer only): y = sum of the gated rows (+ shared)
     if (a.y) {
         cudaLaunchConfig_t cfg = {};
@@ -1050,7 +1077,7 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         cudaError_t e = cudaLaunchKernelEx(&cfg, dec_combine_kernel, (const float *)a.rows_out,
-                                           a.inv, a.T, a.k, a.D, a.sF > 0 ? 1 : 0, a.y, a.y_dtype);
+                                           a.inv, a.T, a.k, a.D, a.comb_shared, a.y, a.y_dtype);
         if (e != cudaSuccess) return cuda_status(e, "dec_combine_kernel");
     }
     return MOE_OK;
@@ -1059,10 +1086,14 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
 moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, int E, int k,
                              const int32_t *perm, const int32_t *inv, const int32_t *offsets,
                              const float *gates, const moe_pool &pool, const uint8_t *mask,
-                             const moe_pool *shared, int sF, __half *Hs, void *y, int y_dtype,
-                             float *rows_out, int *err, cudaStream_t s, Tracer *tr) {
+                             bool routed, const moe_pool *shared, int sF, bool comb_shared,
+                             __half *Hs, void *y, int y_dtype, float *rows_out, int *err,
+                             cudaStream_t s, Tracer *tr) {
     DecArgs a{};
     a.T = T; a.D = D; a.F = F; a.E = E; a.k = k; a.sF = shared ? sF : 0;
+    a.routed = routed ? 1 : 0;
+    a.n_slots = pool.n_slots;
+    a.comb_shared = comb_shared ? 1 : 0;
     a.perm = perm; a.offsets = offsets; a.gates = gates; a.mask = mask;
     a.gate = (const uint8_t *)pool.gate; a.up = (const uint8_t *)pool.up;
     a.down = (const uint8_t *)pool.down; a.slot_map = pool.slot_of_expert;

@@ -10,10 +10,13 @@
 //
 // Experts without tokens are skipped: every CTA compacts the list of active
 // experts (count > 0 and, when a mask is given, mask != 0) in shared memory
-// and walks (active expert, row tile) work items with a grid stride.
+// and walks (active expert, row tile) work items with a grid stride.  An
+// active expert whose slot lies outside [0, n_slots) is left out and
+// recorded as kErrBadSlot in the status word; no address is formed from it.
 // perm == NULL means the identity grouping of T rows for a single expert
 // (used for the always-on shared expert).
 #include "moe_internal.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 
@@ -21,8 +24,8 @@ constexpr int kGenWarps = 8;
 constexpr int kTokGroup = 4;
 
 // Build the active-expert list in shared memory; returns how many.
-__device__ int build_active(const int32_t *offsets, const uint8_t *mask, int E,
-                            int *act) {
+__device__ int build_active(const int32_t *offsets, const uint8_t *mask, const int32_t *slot_map,
+                            int n_slots, int E, int *err, int *act) {
     __shared__ int n_act;
     if (threadIdx.x == 0) n_act = 0;
     __syncthreads();
@@ -36,6 +39,13 @@ __device__ int build_active(const int32_t *offsets, const uint8_t *mask, int E,
             if (e < E) {
                 int c = (offsets ? __ldg(offsets + e + 1) - __ldg(offsets + e) : 1);
                 on = c > 0 && (!mask || __ldg(mask + e));
+                if (on) {
+                    const int sl = slot_of(slot_map, e);
+                    if (sl < 0 || sl >= n_slots) {
+                        if (err) atomicCAS(err, 0, kErrBadSlot);
+                        on = false;
+                    }
+                }
             }
             unsigned b = __ballot_sync(0xffffffffu, on);
             if (on) act[base + __popc(b & ((1u << threadIdx.x) - 1u))] = e;
@@ -52,10 +62,10 @@ __global__ void __launch_bounds__(kGenWarps * 32)
 ffn_gateup_generic_kernel(const XT *__restrict__ x, int T, int D, int F, int E, int k,
                           const int32_t *__restrict__ perm, const int32_t *__restrict__ offsets,
                           const uint8_t *__restrict__ gate, const uint8_t *__restrict__ up,
-                          const int32_t *__restrict__ slot_map, const uint8_t *__restrict__ mask,
-                          float *__restrict__ H) {
+                          const int32_t *__restrict__ slot_map, int n_slots,
+                          const uint8_t *__restrict__ mask, float *__restrict__ H, int *err) {
     extern __shared__ int act[];
-    const int n_act = build_active(offsets, mask, E, act);
+    const int n_act = build_active(offsets, mask, slot_map, n_slots, E, err, act);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nb = D / QK;
     const size_t row_bytes = (size_t)nb * block_bytes<QT>();
@@ -108,9 +118,10 @@ __global__ void __launch_bounds__(kGenWarps * 32)
 ffn_down_generic_kernel(const float *__restrict__ H, int T, int D, int F, int E, int k,
                         const int32_t *__restrict__ offsets,
                         const uint8_t *__restrict__ down, const int32_t *__restrict__ slot_map,
-                        const uint8_t *__restrict__ mask, float *__restrict__ out) {
+                        int n_slots, const uint8_t *__restrict__ mask, float *__restrict__ out,
+                        int *err) {
     extern __shared__ int act[];
-    const int n_act = build_active(offsets, mask, E, act);
+    const int n_act = build_active(offsets, mask, slot_map, n_slots, E, err, act);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nb = F / QK;
     const size_t row_bytes = (size_t)nb * block_bytes<QT>();
@@ -148,38 +159,39 @@ ffn_down_generic_kernel(const float *__restrict__ H, int T, int D, int F, int E,
 template <int QT>
 static moe_status run_generic(const void *x, int x_dtype, int T, int D, int F, int E, int k,
                               const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
-                              const uint8_t *mask, float *H, float *out, cudaStream_t s,
-                              Tracer *tr, bool shared) {
+                              const uint8_t *mask, float *H, float *out, int *err,
+                              cudaStream_t s, Tracer *tr, bool shared) {
     const int grid = num_sms() * 4;
     const size_t sm = (size_t)E * sizeof(int);
     mark(tr, shared ? MOE_KERNEL_SHARED_GATEUP : MOE_KERNEL_GATEUP);
     if (x_dtype == MOE_BF16)
         ffn_gateup_generic_kernel<QT, __nv_bfloat16><<<grid, kGenWarps * 32, sm, s>>>(
             (const __nv_bfloat16 *)x, T, D, F, E, k, perm, offsets, (const uint8_t *)pool.gate,
-            (const uint8_t *)pool.up, pool.slot_of_expert, mask, H);
+            (const uint8_t *)pool.up, pool.slot_of_expert, pool.n_slots, mask, H, err);
     else
         ffn_gateup_generic_kernel<QT, float><<<grid, kGenWarps * 32, sm, s>>>(
             (const float *)x, T, D, F, E, k, perm, offsets, (const uint8_t *)pool.gate,
-            (const uint8_t *)pool.up, pool.slot_of_expert, mask, H);
+            (const uint8_t *)pool.up, pool.slot_of_expert, pool.n_slots, mask, H, err);
     moe_status st = cuda_status(cudaGetLastError(), "ffn_gateup_generic_kernel");
     if (st != MOE_OK) return st;
     mark(tr, shared ? MOE_KERNEL_SHARED_DOWN : MOE_KERNEL_DOWN);
     ffn_down_generic_kernel<QT><<<grid, kGenWarps * 32, sm, s>>>(
-        H, T, D, F, E, k, offsets, (const uint8_t *)pool.down, pool.slot_of_expert, mask, out);
+        H, T, D, F, E, k, offsets, (const uint8_t *)pool.down, pool.slot_of_expert, pool.n_slots,
+        mask, out, err);
     return cuda_status(cudaGetLastError(), "ffn_down_generic_kernel");
 }
 
 moe_status launch_ffn_generic(const void *x, int x_dtype, int T, int D, int F, int E, int k,
                               const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
-                              const uint8_t *mask, float *H, float *out_rows, cudaStream_t s,
-                              Tracer *tr, bool shared) {
+                              const uint8_t *mask, float *H, float *out_rows, int *err,
+                              cudaStream_t s, Tracer *tr, bool shared) {
     switch (pool.qtype) {
     case MOE_Q4_0:
         return run_generic<MOE_Q4_0>(x, x_dtype, T, D, F, E, k, perm, offsets, pool, mask, H,
-                                     out_rows, s, tr, shared);
+                                     out_rows, err, s, tr, shared);
     case MOE_Q8_0:
         return run_generic<MOE_Q8_0>(x, x_dtype, T, D, F, E, k, perm, offsets, pool, mask, H,
-                                     out_rows, s, tr, shared);
+                                     out_rows, err, s, tr, shared);
     default:
         set_error("expert FFN: unsupported quant type %d", (int)pool.qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;

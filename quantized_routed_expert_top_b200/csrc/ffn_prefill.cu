@@ -28,8 +28,15 @@
 // the next accumulates.
 //
 // Numerics: weights d*q rounded to fp16 (relative error <= 2^-11 per weight),
-// activations fp16 (x is bf16 or fp32 on input: exact in fp16 over the
-// normal range), fp32 accumulation; H is stored fp16.
+// activations fp16 (a bf16 x in fp16's normal range converts exactly; an fp32
+// x is rounded to fp16's 11 significant bits), fp32 accumulation; H is
+// stored fp16.
+//
+// Experts: the tile list covers the experts that have tokens, that this
+// call runs (the routed ones the mask admits, and the shared one when
+// present) and whose slot lies in [0, n_slots); an expert with tokens whose
+// slot does not is left out and recorded as kErrBadSlot, so no address is
+// ever formed from it.
 #include "moe_internal.cuh"
 #include "sm100.cuh"
 
@@ -59,6 +66,7 @@ constexpr int kPTmemCols = 512;                              // 2 accumulators x
 // around them; four blocks start 0 or 8 bytes past a 16-byte boundary.
 constexpr int kPRawRow = 144;
 constexpr int kPRaw = 256 * kPRawRow;    // one raw window buffer (36 KB)
+constexpr int kPfMaxExperts = 720;       // segs + tcum of E + 2 entries each fit with the rings
 // A ring | B ring | raw ring | barriers + TMEM slot (256 B) | segs, tcum [2][E+2]
 __host__ __device__ inline size_t pf_smem_bytes(int E) {
     return (size_t)kPSA * kPStageA + (size_t)kPSB * kPStageB + (size_t)kPR * kPRaw + 256 +
@@ -78,7 +86,10 @@ struct PfMaps {
 struct PfArgs {
     int T, D, F, E, k;
     int q8;                       // routed pool is Q8_0 (else Q4_0)
-    int shared, sq8;              // shared expert present (F columns, Q8_0 / Q4_0)
+    int shared, sq8;              // this call runs the shared expert (F columns, Q8_0 / Q4_0)
+    int routed;                   // this call runs the routed experts the mask admits
+    int n_slots;                  // slots of the routed pool
+    const uint8_t *mask;          // [E] or NULL
     const int32_t *perm, *offsets;
     const uint8_t *gate, *up, *down;
     const int32_t *slot_map;
@@ -250,7 +261,8 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
     uint64_t *rempty = rfull + kPR;                           // raw window read by every B warp
     uint64_t *accf = rempty + kPR;                            // [2] accumulator ready
     uint64_t *acce = accf + 2;                                // [2] accumulator drained
-    uint32_t *tmem_slot = (uint32_t *)(acce + 2);
+    uint64_t *mma_done = acce + 2;                            // every MMA of the CTA completed
+    uint32_t *tmem_slot = (uint32_t *)(mma_done + 1);
     int *segs = (int *)(tmem_slot + 4);                       // [nv + 1] segment starts
     int *tcum = segs + (a.E + 2);                             // [nv + 1] first tile of each expert
 
@@ -278,6 +290,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], kPEW * 32);
         }
+        mbar_init(mma_done, 1);
         fence_mbar_init();
     }
     if (warp == kPMmaWarp) {
@@ -298,7 +311,21 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
         for (int v0 = 0; v0 < nv; v0 += 32) {
             const int v = v0 + lane;
             int ntiles = 0;
-            if (v < nv) ntiles = (segs[v + 1] - segs[v] + kPM - 1) / kPM * nt;
+            if (v < nv) {
+                int cnt = segs[v + 1] - segs[v];
+                if (v < a.E && cnt > 0) {
+                    if (!a.routed || (a.mask && !__ldg(a.mask + v))) {
+                        cnt = 0;
+                    } else {
+                        const int sl = a.slot_map ? __ldg(a.slot_map + v) : v;
+                        if (sl < 0 || sl >= a.n_slots) {
+                            atomicCAS(a.err, 0, kErrBadSlot);
+                            cnt = 0;
+                        }
+                    }
+                }
+                ntiles = (cnt + kPM - 1) / kPM * nt;
+            }
             int incl = ntiles;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -497,6 +524,10 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                 if (!ok) break;
                 tc_commit(&accf[ab]);            // the tile's accumulator is complete
             }
+            // tensor memory is freed at exit: wait until every MMA issued
+            // here has completed (also after a wait that gave up)
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0, a.err, kErrTimeoutMma);
         }
         __syncwarp();
     } else {
@@ -586,7 +617,7 @@ __global__ void __launch_bounds__(256) pf_convert_kernel(const XT *__restrict__ 
 // window reads past a row
 bool prefill_path_ok(int T, int D, int F, int sF, int E) {
     return T > 16 && D % kPNd == 0 && F % kPNg == 0 && D % 256 == 0 && F % 256 == 0 &&
-           (sF == 0 || sF == F) && E <= MOE_MAX_EXPERTS && pf_smem_bytes(E) <= 227 * 1024;
+           (sF == 0 || sF == F) && E <= kPfMaxExperts && pf_smem_bytes(E) <= 227 * 1024;
 }
 
 size_t prefill_x16_halves(int T, int D) { return (size_t)T * D; }
@@ -645,8 +676,9 @@ static cudaError_t launch_pf(const PfArgs &a, const PfMaps &m, int grid, cudaStr
 
 moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, int E, int k,
                               const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
-                              const moe_pool *shared, int sF, __half *x16, __half *H, float *Y,
-                              int *err, cudaStream_t s, Tracer *tr) {
+                              const uint8_t *mask, bool routed, const moe_pool *shared, int sF,
+                              __half *x16, __half *H, float *Y, int *err, cudaStream_t s,
+                              Tracer *tr) {
     if (pool.qtype != MOE_Q4_0 && pool.qtype != MOE_Q8_0) {
         set_error("prefill path: unsupported quant type %d", (int)pool.qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
@@ -664,6 +696,9 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
     a.q8 = pool.qtype == MOE_Q8_0;
     a.shared = shared ? 1 : 0;
     a.sq8 = shared ? shared->qtype == MOE_Q8_0 : 0;
+    a.routed = routed ? 1 : 0;
+    a.n_slots = pool.n_slots;
+    a.mask = mask;
     a.perm = perm; a.offsets = offsets;
     a.gate = (const uint8_t *)pool.gate; a.up = (const uint8_t *)pool.up;
     a.down = (const uint8_t *)pool.down; a.slot_map = pool.slot_of_expert;

@@ -1,13 +1,15 @@
 // layer.cu -- the whole layer in one call: route -> permute -> expert FFNs
-// (+ shared expert) -> gate-weighted combine.  The workspace holds every
-// intermediate; its layout is fixed by carve() so that the size query and
-// the call agree.
+// (+ shared expert) -> gate-weighted combine, or any subset of those parts
+// (phases) for callers that split a layer step around an expert cache's
+// copies.  The workspace holds every intermediate; its layout is fixed by
+// carve() so that the size query and the call agree, and so that the calls
+// of one split step find each other's results in it.
 #include "moe_paths.cuh"
 
 namespace moe {
 
 struct LayerWs {
-    int *status;         // device status words (first bytes of the workspace)
+    int *status;         // device status word (first bytes of the workspace)
     void *route_ws;
     size_t route_bytes;
     int32_t *ids;
@@ -60,6 +62,17 @@ size_t layer_ws_bytes(const moe_layer_args &a) {
     return c.off;
 }
 
+static moe_status end_trace(Tracer *tr, moe_status st) {
+    if (tr) {
+        tr->end();
+        if (st == MOE_OK && tr->err != cudaSuccess) {
+            cudaGetLastError();   // the failed record is reported here, not left sticky
+            return cuda_status(tr->err, "moe_layer_forward: trace event record");
+        }
+    }
+    return st;
+}
+
 moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cudaStream_t s) {
     Carver c(ws, ws_bytes);
     LayerWs w = carve(a, c);
@@ -75,71 +88,69 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
         trace.s = s;
         tr = &trace;
     }
+    const unsigned ph = a.phases ? (unsigned)a.phases : MOE_PHASE_ALL;
+    const bool do_route = ph & MOE_PHASE_ROUTE, do_ffn = ph & MOE_PHASE_FFN;
+    const bool do_shared = (ph & MOE_PHASE_SHARED) && a.shared;
+    const bool do_comb = ph & MOE_PHASE_COMBINE;
     int32_t *ids = a.ids_out ? a.ids_out : w.ids;
     float *gates = a.gates_out ? a.gates_out : w.gates;
+    int32_t *counts = a.counts_out ? a.counts_out : w.counts;
+    int32_t *offsets = a.offsets_out ? a.offsets_out : w.offsets;
+    int32_t *perm = a.perm_out ? a.perm_out : w.perm;
+    int32_t *inv = a.inv_out ? a.inv_out : w.inv;
     moe_status st;
-    bool permuted = false;
-    if (a.w_router)
-        st = launch_route_permute(a.x, a.x_dtype, a.w_router, a.bias, a.T, a.D, a.E, a.k, a.renorm,
-                                  ids, gates, a.logits_out, w.counts, w.offsets, w.perm, w.inv,
-                                  w.status, w.route_ws, w.route_bytes, s, tr, &permuted);
-    else
-        st = launch_route_permute(a.logits_in, MOE_F32, nullptr, a.bias, a.T, QK, a.E, a.k,
-                                  a.renorm, ids, gates, a.logits_out, w.counts, w.offsets, w.perm,
-                                  w.inv, w.status, w.route_ws, w.route_bytes, s, tr, &permuted);
-    if (st != MOE_OK) return st;
-    if (!permuted &&
-        (st = launch_permute(ids, a.T, a.k, a.E, w.counts, w.offsets, w.perm, w.inv, s, tr)) != MOE_OK)
-        return st;
+    if (do_route) {
+        bool permuted = false;
+        if (a.w_router)
+            st = launch_route_permute(a.x, a.x_dtype, a.w_router, a.bias, a.T, a.D, a.E, a.k,
+                                      a.renorm, ids, gates, a.logits_out, counts, offsets, perm,
+                                      inv, w.status, w.route_ws, w.route_bytes, s, tr, &permuted);
+        else
+            st = launch_route_permute(a.logits_in, MOE_F32, nullptr, a.bias, a.T, QK, a.E, a.k,
+                                      a.renorm, ids, gates, a.logits_out, counts, offsets, perm,
+                                      inv, w.status, w.route_ws, w.route_bytes, s, tr, &permuted);
+        if (st != MOE_OK) return st;
+        if (!permuted &&
+            (st = launch_permute(ids, a.T, a.k, a.E, counts, offsets, perm, inv, s, tr)) != MOE_OK)
+            return st;
+    }
+    const int sF = a.shared ? a.shared_F : 0;
     if (w.Hs) {
-        st = launch_ffn_decode(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.inv, w.offsets,
-                               gates, *a.pool, nullptr, a.shared, a.shared ? a.shared_F : 0, w.Hs,
-                               a.y, a.y_dtype, w.rows, w.status, s, tr);
-        if (tr) {
-            tr->end();
-            if (st == MOE_OK && tr->err != cudaSuccess) {
-                cudaGetLastError();
-                return cuda_status(tr->err, "moe_layer_forward: trace event record");
-            }
-        }
-        return st;
+        if (!do_ffn && !do_shared && !do_comb) return end_trace(tr, MOE_OK);
+        st = launch_ffn_decode(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, perm, inv, offsets, gates,
+                               *a.pool, a.expert_mask, do_ffn, do_shared ? a.shared : nullptr, sF,
+                               a.shared != nullptr, w.Hs, do_comb ? a.y : nullptr, a.y_dtype,
+                               w.rows, w.status, s, tr);
+        return end_trace(tr, st);
     }
     if (w.H16) {
-        const int sF = a.shared ? a.shared_F : 0;
-        if ((st = launch_ffn_prefill(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.offsets,
-                                     *a.pool, a.shared, sF, w.x16, w.H16, w.rows, w.status, s,
-                                     tr)) != MOE_OK)
+        if ((do_ffn || do_shared) &&
+            (st = launch_ffn_prefill(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, perm, offsets,
+                                     *a.pool, a.expert_mask, do_ffn,
+                                     do_shared ? a.shared : nullptr, sF, w.x16, w.H16, w.rows,
+                                     w.status, s, tr)) != MOE_OK)
             return st;
-        st = launch_combine(w.rows, w.inv, gates, a.T, a.k, a.D,
-                            a.shared ? w.rows + (size_t)a.T * a.k * a.D : nullptr, a.y, a.y_dtype,
-                            s, tr);
-        if (tr) {
-            tr->end();
-            if (st == MOE_OK && tr->err != cudaSuccess) {
-                cudaGetLastError();
-                return cuda_status(tr->err, "moe_layer_forward: trace event record");
-            }
-        }
+        st = MOE_OK;
+        if (do_comb)
+            st = launch_combine(w.rows, inv, gates, a.T, a.k, a.D,
+                                a.shared ? w.rows + (size_t)a.T * a.k * a.D : nullptr, a.y,
+                                a.y_dtype, s, tr);
+        return end_trace(tr, st);
+    }
+    if (do_ffn &&
+        (st = launch_ffn_generic(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, perm, offsets, *a.pool,
+                                 a.expert_mask, w.H, w.rows, w.status, s, tr)) != MOE_OK)
         return st;
-    }
-    if ((st = launch_ffn_generic(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, w.perm, w.offsets,
-                                 *a.pool, nullptr, w.H, w.rows, s, tr)) != MOE_OK)
+    if (do_shared &&
+        (st = launch_ffn_generic(a.x, a.x_dtype, a.T, a.D, a.shared_F, 1, 1, nullptr, nullptr,
+                                 *a.shared, nullptr, w.shH, w.sh_rows, w.status, s, tr, true)) !=
+            MOE_OK)
         return st;
-    if (a.shared) {
-        if ((st = launch_ffn_generic(a.x, a.x_dtype, a.T, a.D, a.shared_F, 1, 1, nullptr, nullptr,
-                                     *a.shared, nullptr, w.shH, w.sh_rows, s, tr, true)) != MOE_OK)
-            return st;
-    }
-    st = launch_combine(w.rows, w.inv, gates, a.T, a.k, a.D, a.shared ? w.sh_rows : nullptr, a.y,
-                        a.y_dtype, s, tr);
-    if (tr) {
-        tr->end();
-        if (st == MOE_OK && tr->err != cudaSuccess) {
-            cudaGetLastError();   // the failed record is reported here, not left sticky
-            return cuda_status(tr->err, "moe_layer_forward: trace event record");
-        }
-    }
-    return st;
+    st = MOE_OK;
+    if (do_comb)
+        st = launch_combine(w.rows, inv, gates, a.T, a.k, a.D, a.shared ? w.sh_rows : nullptr,
+                            a.y, a.y_dtype, s, tr);
+    return end_trace(tr, st);
 }
 
 }  // namespace moe

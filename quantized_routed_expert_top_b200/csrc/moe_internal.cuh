@@ -163,7 +163,7 @@ moe_status launch_permute(const int32_t *ids, int T, int k, int E, int32_t *coun
 moe_status launch_ffn_generic(const void *x, int x_dtype, int T, int D, int F, int E,
                               int k, const int32_t *perm, const int32_t *offsets,
                               const moe_pool &pool, const uint8_t *mask, float *H,
-                              float *out_rows, cudaStream_t s, Tracer *tr = nullptr,
+                              float *out_rows, int *err, cudaStream_t s, Tracer *tr = nullptr,
                               bool shared = false);
 // ffn_decode.cu -- TMA-streamed grouped GEMV for small T (see file header)
 bool decode_path_ok(int T, int D, int F, int sF);
@@ -175,18 +175,24 @@ bool prefill_path_ok(int T, int D, int F, int sF, int E);
 size_t prefill_x16_halves(int T, int D);
 size_t prefill_h_halves(int T, int k, int F, int sF);
 size_t prefill_y_floats(int T, int k, int D, int sF);
+// routed: run the routed experts the mask (if any) admits; shared != NULL:
+// run the shared expert too (rows T*k .. T*k+T-1 of H and Y)
 moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, int E, int k,
                               const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
-                              const moe_pool *shared, int sF, __half *x16, __half *H, float *Y,
-                              int *err, cudaStream_t s, Tracer *tr);
-// y != NULL: fused layer (gates folded into the rows, rows_out is scratch
-// for [T*k + T, D] rows, combined into y); y == NULL: rows mode (rows_out =
-// un-gated Y rows [T*k, D] in permuted order, mask honoured)
+                              const uint8_t *mask, bool routed, const moe_pool *shared, int sF,
+                              __half *x16, __half *H, float *Y, int *err, cudaStream_t s,
+                              Tracer *tr);
+// gates != NULL: fused layer (gates folded into the rows; rows_out holds
+// [T*k + T, D] gated rows); gates == NULL: rows mode (un-gated Y rows [T*k, D]
+// in permuted order).  routed: run the routed experts the mask admits;
+// shared != NULL: run the shared expert (rows T*k..); y != NULL: combine the
+// rows into y afterwards (adding the shared rows when comb_shared).
 moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, int E, int k,
                              const int32_t *perm, const int32_t *inv, const int32_t *offsets,
                              const float *gates, const moe_pool &pool, const uint8_t *mask,
-                             const moe_pool *shared, int sF, __half *Hs, void *y, int y_dtype,
-                             float *rows_out, int *err, cudaStream_t s, Tracer *tr);
+                             bool routed, const moe_pool *shared, int sF, bool comb_shared,
+                             __half *Hs, void *y, int y_dtype, float *rows_out, int *err,
+                             cudaStream_t s, Tracer *tr);
 // combine.cu
 moe_status launch_combine(const float *rows, const int32_t *inv, const float *gates,
                           int T, int k, int D, const float *shared_rows, void *y,

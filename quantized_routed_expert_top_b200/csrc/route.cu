@@ -554,6 +554,32 @@ select_permute_kernel(const float *__restrict__ logits, const float *__restrict_
 }
 
 // ------------------------------------------------------------------- host
+// The split-K router launch shared by moe_route (T <= 16 without the cluster
+// kernel) and moe_route_noalloc.
+static moe_status launch_splitk(const void *x, int x_dtype, const float *w_router,
+                                const float *bias, int T, int D, int E, int k, int renorm,
+                                int nsplit, float *partial, unsigned *ticket, int32_t *ids,
+                                float *gates, float *logits, cudaStream_t s, const char *what) {
+    int threads = (int)round_up(E, 32);
+    if (threads < 128) threads = 128;
+    const size_t sm = (size_t)std::max(T * kSplitRows, T * E) * sizeof(float);
+    cudaError_t e;
+    if (x_dtype == MOE_BF16) {
+        auto kern = route_splitk_kernel<__nv_bfloat16>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return cuda_status(e, what);
+        kern<<<nsplit, threads, sm, s>>>((const __nv_bfloat16 *)x, w_router, bias, T, D, E, k,
+                                         renorm, nsplit, partial, ticket, ids, gates, logits);
+    } else {
+        auto kern = route_splitk_kernel<float>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return cuda_status(e, what);
+        kern<<<nsplit, threads, sm, s>>>((const float *)x, w_router, bias, T, D, E, k, renorm,
+                                         nsplit, partial, ticket, ids, gates, logits);
+    }
+    return cuda_status(cudaGetLastError(), what);
+}
+
 static size_t splitk_partial_bytes(int T, int D, int E) {
     int nsplit = (D + kSplitRows - 1) / kSplitRows;
     return (size_t)nsplit * T * E * sizeof(float);
@@ -658,7 +684,8 @@ moe_status launch_route(const void *x, int x_dtype, const float *w_router,
                         int32_t *ids, float *gates, float *logits, void *ws,
                         size_t ws_bytes, cudaStream_t s, Tracer *tr) {
     Carver c(ws, ws_bytes);
-    unsigned *ticket = c.take<unsigned>(64);
+    // 64-word header: word 0 is the status word, word 1 the completion ticket
+    unsigned *ticket = c.take<unsigned>(64) + 1;
     if (w_router == nullptr) {
         // x holds the logits [T, E] fp32
         float *copy = logits;
@@ -675,23 +702,10 @@ moe_status launch_route(const void *x, int x_dtype, const float *w_router,
     if (T <= kSplitMaxT) {
         float *partial = (float *)c.take<char>(splitk_partial_bytes(T, D, E));
         if (!c.fits()) { set_error("moe_route: workspace too small"); return MOE_ERR_WORKSPACE; }
-        int nsplit = (D + kSplitRows - 1) / kSplitRows;
-        int threads = (int)round_up(E, 32);
-        if (threads < 128) threads = 128;
-        size_t sm = (size_t)std::max(T * kSplitRows, T * E) * sizeof(float);
+        const int nsplit = (D + kSplitRows - 1) / kSplitRows;
         mark(tr, MOE_KERNEL_ROUTE);
-        if (x_dtype == MOE_BF16) {
-            auto kern = route_splitk_kernel<__nv_bfloat16>;
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-            kern<<<nsplit, threads, sm, s>>>((const __nv_bfloat16 *)x, w_router, bias, T, D, E, k,
-                                             renorm, nsplit, partial, ticket, ids, gates, logits);
-        } else {
-            auto kern = route_splitk_kernel<float>;
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-            kern<<<nsplit, threads, sm, s>>>((const float *)x, w_router, bias, T, D, E, k, renorm,
-                                             nsplit, partial, ticket, ids, gates, logits);
-        }
-        return cuda_status(cudaGetLastError(), "route_splitk_kernel");
+        return launch_splitk(x, x_dtype, w_router, bias, T, D, E, k, renorm, nsplit, partial,
+                             ticket, ids, gates, logits, s, "route_splitk_kernel");
     }
     float *L = logits;
     if (!L) {
@@ -827,19 +841,6 @@ extern "C" moe_status moe_route_noalloc(const void *x, int32_t x_dtype, const fl
     float *partial = scratch;
     ce = cudaMemsetAsync(ticket, 0, sizeof(unsigned), s);
     if (ce != cudaSuccess) return cuda_status(ce, "moe_route_noalloc: ticket clear");
-    int threads = (int)round_up(E, 32);
-    if (threads < 128) threads = 128;
-    size_t sm = (size_t)std::max(T * kSplitRows, T * E) * sizeof(float);
-    if (x_dtype == MOE_BF16) {
-        auto kern = route_splitk_kernel<__nv_bfloat16>;
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        kern<<<nsplit, threads, sm, s>>>((const __nv_bfloat16 *)x, w_router, bias, T, D, E, k,
-                                         renorm, nsplit, partial, ticket, ids, gates, logits);
-    } else {
-        auto kern = route_splitk_kernel<float>;
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        kern<<<nsplit, threads, sm, s>>>((const float *)x, w_router, bias, T, D, E, k, renorm,
-                                         nsplit, partial, ticket, ids, gates, logits);
-    }
-    return cuda_status(cudaGetLastError(), "moe_route_noalloc: route_splitk_kernel");
+    return launch_splitk(x, x_dtype, w_router, bias, T, D, E, k, renorm, nsplit, partial, ticket,
+                         ids, gates, logits, s, "moe_route_noalloc: route_splitk_kernel");
 }

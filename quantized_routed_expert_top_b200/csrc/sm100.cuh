@@ -9,11 +9,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
-// status word values written into a kernel's error flag
-enum : int { kErrNone = 0, kErrTimeoutFull = 1, kErrTimeoutEmpty = 2, kErrTimeoutDrain = 3,
-             kErrBadSlot = 4, kErrTimeoutMma = 5 };
+// status word values written into a kernel's error flag (moe_device_status)
+enum : int { kErrNone = MOE_DEV_OK, kErrTimeoutFull = MOE_DEV_TIMEOUT_FULL,
+             kErrTimeoutEmpty = MOE_DEV_TIMEOUT_EMPTY, kErrTimeoutDrain = MOE_DEV_TIMEOUT_DRAIN,
+             kErrBadSlot = MOE_DEV_BAD_SLOT, kErrTimeoutMma = MOE_DEV_TIMEOUT_MMA };
 
 // ~4 s at 2 GHz: far above any legitimate wait in these kernels
 constexpr long long kWaitBudgetCycles = 8000000000LL;

@@ -152,3 +152,43 @@ def test_error_message_is_per_call(moe):
     assert _err(L)
     assert L.moe_route(None, moe.BF16, FAKE, None, 0, 256, 8, 2, 1, None, None, None, None, 0, None) == 0
     assert _err(L) == ""
+
+
+def test_workspace_status_and_phase_errors(moe):
+    L = moe.lib()
+    code = C.c_int32(-1)
+    assert L.moe_workspace_status(None, C.byref(code), 1, None) == 1
+    assert L.moe_workspace_status(FAKE, None, 1, None) == 1
+    pool = moe.Pool(moe.Q4_0, 8, 0x1000, 0x1000, 0x1000, None)
+    a = moe.LayerArgs()
+    a.T, a.D, a.E, a.k, a.F, a.renorm = 4, 256, 8, 2, 512, 1
+    a.x_dtype, a.y_dtype = moe.BF16, moe.BF16
+    a.x, a.y, a.w_router = 0x1000, 0x1000, 0x1000
+    a.pool = C.pointer(pool)
+    a.phases = 16                       # no such phase bit
+    assert L.moe_layer_forward(C.byref(a), FAKE, 1 << 40, None) == 1
+    assert "phases" in _err(L)
+    a.phases = moe.PHASE_COMBINE        # combining needs y
+    a.y = None
+    assert L.moe_layer_forward(C.byref(a), FAKE, 1 << 40, None) == 1
+    a.phases, a.y = moe.PHASE_ROUTE, None   # routing alone writes no y
+    a.w_router = None                       # ... but needs a router or logits
+    assert L.moe_layer_forward(C.byref(a), FAKE, 1 << 40, None) == 1
+
+
+def test_cache_stats_rejects_null_cache(moe):
+    L = moe.lib()
+    assert L.moe_cache_stats(None, None, None, None, None) == 1
+
+
+def test_device_status_codes_agree_with_header(moe):
+    src = open(HEADER).read()
+    names = ["MOE_DEV_OK", "MOE_DEV_TIMEOUT_FULL", "MOE_DEV_TIMEOUT_EMPTY", "MOE_DEV_TIMEOUT_DRAIN",
+             "MOE_DEV_BAD_SLOT", "MOE_DEV_TIMEOUT_MMA"]
+    vals = [int(re.search(n + r"\s*=\s*(\d+)", src).group(1)) for n in names]
+    assert vals == [moe.DEV_OK, moe.DEV_TIMEOUT_FULL, moe.DEV_TIMEOUT_EMPTY, moe.DEV_TIMEOUT_DRAIN,
+                    moe.DEV_BAD_SLOT, moe.DEV_TIMEOUT_MMA]
+    ph = {n: int(v, 0) for n, v in re.findall(r"#define\s+(MOE_PHASE_\w+)\s+(\w+?)u", src)}
+    assert ph == {"MOE_PHASE_ROUTE": moe.PHASE_ROUTE, "MOE_PHASE_FFN": moe.PHASE_FFN,
+                  "MOE_PHASE_SHARED": moe.PHASE_SHARED, "MOE_PHASE_COMBINE": moe.PHASE_COMBINE,
+                  "MOE_PHASE_ALL": moe.PHASE_ALL}

@@ -13,6 +13,7 @@ import torch
 
 import oracle
 import synthetic as S
+from helpers import check_ids
 
 pytestmark = pytest.mark.gpu
 
@@ -154,4 +155,107 @@ def test_released_copies_overlap_and_stay_exact(moe, stack):
     assert torch.equal(y_c, y_r)
     hits, misses, _ = cache.stats()
     assert misses > 0 and hits > 0
+    cache.close()
+
+
+def _masks(E, ids, miss):
+    """Device uint8 masks of the requested experts that were resident (hits)
+    and of those whose copies were just enqueued (misses)."""
+    hit = np.zeros(E, np.uint8)
+    mis = np.zeros(E, np.uint8)
+    ids = np.asarray(ids)
+    hit[ids[~miss]] = 1
+    mis[ids[miss]] = 1
+    return torch.from_numpy(hit).cuda(), torch.from_numpy(mis).cuda()
+
+
+def _two_phase(moe, cache, lay, l, ids, x, lg, out, stream):
+    """One cached layer step with the miss copies overlapping the FFN of the
+    resident experts: route + resident FFN, wait for the copies, the copied
+    experts' FFN + combine."""
+    _, miss, _ = cache.request(l, ids, stream=stream)
+    m_hit, m_miss = _masks(lay.E, ids, miss)
+    lay.forward(x, logits=lg, out=out, mask=m_hit,
+                phases=moe.PHASE_ROUTE | moe.PHASE_FFN | moe.PHASE_SHARED)
+    cache.sync(l, stream=stream)
+    lay.forward(x, logits=lg, out=out, mask=m_miss, phases=moe.PHASE_FFN | moe.PHASE_COMBINE)
+    return int(miss.sum())
+
+
+def test_two_phase_cached_layers_are_bit_identical_to_resident(moe, stack):
+    pools, traces, x = stack
+    stream = torch.cuda.current_stream()
+    cache = _cache(moe, pools, torch.cuda.Stream())
+    xd = torch.from_numpy(x.x_raw.view(np.int16)).cuda().view(torch.bfloat16)
+    resident = [moe.Layer(moe.ExpertPool.from_numpy(*p, "q8_0"), D, F, E, K, 1,
+                          y_dtype=torch.float32) for p in pools]
+    cached = [moe.Layer(cache.pools[l], D, F, E, K, 1, y_dtype=torch.float32)
+              for l in range(N_LAYERS)]
+    n_miss = 0
+    for t in range(STEPS):
+        for l in range(N_LAYERS):
+            lg = torch.from_numpy(traces[l][t:t + 1]).cuda()
+            y_c = torch.full((1, D), float("nan"), device="cuda")
+            n_miss += _two_phase(moe, cache, cached[l], l, _ids(traces[l][t]), xd[t:t + 1], lg,
+                                 y_c, stream)
+            cache.release(l, stream=stream)
+            y_r = resident[l].forward(xd[t:t + 1], logits=lg).clone()
+            torch.cuda.synchronize()
+            assert torch.equal(y_c, y_r), (t, l)
+            assert moe.workspace_status(cached[l].ws) == (0, moe.DEV_OK)
+    assert n_miss > 0
+    assert cache.exposed_ns() >= 0
+    cache.close()
+
+
+def test_exposed_copy_time_is_measured(moe, stack):
+    # a copy the compute stream must wait for (the first, cold request of a
+    # layer, synced at once) shows up as exposed time; requests that hit
+    # add nothing
+    pools, traces, _ = stack
+    stream = torch.cuda.current_stream()
+    cache = _cache(moe, pools, torch.cuda.Stream())
+    assert cache.exposed_ns() == 0
+    ids = _ids(traces[0][0])
+    cache.request(0, ids, stream=stream)
+    cache.sync(0, stream=stream)
+    torch.cuda.synchronize()
+    e1 = cache.exposed_ns()
+    assert e1 > 0
+    cache.request(0, ids, stream=stream)      # all hits: nothing to wait for
+    cache.sync(0, stream=stream)
+    torch.cuda.synchronize()
+    assert cache.exposed_ns() == e1
+    cache.close()
+
+
+def test_cache_at_the_full_layer_shape_matches_the_oracle(moe):
+    # the expert-cache layer at its real shape (Q8_0, D=2048, F=768, E=128,
+    # top-8, 51 slots = 40%) for a few cold-start steps: each step's output
+    # against the oracle, two-phase (resident experts, then the copied ones)
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    cfg = S.CONFIGS["cache"]
+    n_slots = int(np.floor(S.CACHE_FRACTION * cfg.E))
+    pool = S.gen_expert_pool(cfg.seed, cfg.E, cfg.D, cfg.F, cfg.qtype, cfg.expert_std)
+    steps = 6
+    logits, sets = S.locality_trace(np.random.default_rng([cfg.seed, 0]), steps, cfg.E, cfg.k)
+    xin = S.make_layer(S.with_T(cfg, steps), experts=False)
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    cache = moe.ExpertCache([pin(pool[0])], [pin(pool[1])], [pin(pool[2])], cfg.qtype, n_slots,
+                            torch.cuda.Stream())
+    lay = moe.Layer(cache.pools[0], cfg.D, cfg.F, cfg.E, cfg.k, 1, y_dtype=torch.float32)
+    stream = torch.cuda.current_stream()
+    xd = torch.from_numpy(xin.x_raw.view(np.int16)).cuda().view(torch.bfloat16)
+    lgd = torch.from_numpy(logits).cuda()
+    for t in range(steps):
+        ids, g = oracle.select(logits[t:t + 1].astype(np.float64), cfg.k, cfg.renorm)
+        y = torch.full((1, cfg.D), float("nan"), device="cuda")
+        _two_phase(moe, cache, lay, 0, ids[0], xd[t:t + 1], lgd[t:t + 1], y, stream)
+        torch.cuda.synchronize()
+        check_ids(lay.ids.cpu().numpy()[:1], ids, logits[t:t + 1], cfg.k, log=print)
+        ref = oracle.layer(xin.x[t:t + 1], ids, g, *pool, cfg.qtype, cfg.F)
+        err = np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max()
+        assert err <= 2e-3, (t, err)
+    assert moe.workspace_status(lay.ws) == (0, moe.DEV_OK)
     cache.close()
