@@ -16,9 +16,15 @@ One JSON line on rank 0.  Workloads (seeded synthetic inputs, see synthetic/):
   logits from a temporal-locality trace, at T = 1 and T = 2048.
 * cache: one token per step through a 40-layer stack of the decode layer in
   Q8_0 whose experts live in pinned host memory, 51 HBM slots (40%) per
-  layer, misses copied on a side stream; also reports the hit rate, the
-  copy bytes and the exposed copy time against the same stack fully
-  resident.
+  layer, misses copied on a side stream while the resident experts' FFN
+  runs; reports tokens/s with routing read back from the GPU per layer
+  (dependent) and with the ids known ahead (two_phase, lookahead), the hit
+  rate, the copy bytes and the exposed copy time, against the same stack
+  fully resident.
+
+The default run (decode) prints the decode line with every other
+configuration under "configs" (tiny, prefill, wide_t1, wide_t2048, cache),
+each with its own roofline, end-to-end number and oracle baseline.
 
 Timing: W untimed steps, then K steps bracketed by a barrier and a device
 synchronize, timed with CUDA events on the launching stream; max over
@@ -167,29 +173,39 @@ def _dev_x(L, torch):
     return torch.from_numpy(L.x_raw).cuda()
 
 
+# tokens per call and pool replicas (enough that the pool copies together
+# exceed L2, so every call reads its experts from HBM)
+WORKLOADS = {
+    "decode": ((1, 4, 16), 6),
+    "tiny": ((4,), 1),
+    "prefill": ((8192,), 2),
+    "wide": ((1, 2048), 2),
+    "wide_t1": ((1,), 2),
+    "wide_t2048": ((2048,), 2),
+}
+
+
 class Workload:
     """A list of layer calls making one step; replicas rotate per call."""
 
-    def __init__(self, name: str, torch, moe, n_replicas=0):
+    def __init__(self, name: str, torch, moe, n_replicas=0, base=None):
         self.name = name
         self.torch, self.moe = torch, moe
-        cfg = S.CONFIGS[name]
+        cfg_name = name.split("_")[0]
+        cfg = S.CONFIGS[cfg_name]
         self.cfg = cfg
-        if name == "decode":
-            Ts, replicas = (1, 4, 16), 6
-        elif name == "prefill":
-            Ts, replicas = (8192,), 2
-        elif name == "wide":
-            Ts, replicas = (1, 2048), 2
-        else:
-            raise ValueError(name)
+        Ts, replicas = WORKLOADS[name]
         if n_replicas:     # fewer replicas: a small case for profilers (weights may hit L2)
             replicas = int(n_replicas)
         self.Ts = Ts
-        base = S.make_layer(cfg, T=max(Ts))
-        self.inputs = {max(Ts): base}
+        if base is None:
+            base = S.make_layer(cfg, T=max(Ts))
+        self.base = base
+        self.inputs = {}
         for T in Ts:
-            if T not in self.inputs:
+            if T == base.x.shape[0]:
+                self.inputs[T] = base
+            else:
                 self.inputs[T] = S.make_layer(cfg, T=T, experts=False)
                 self.inputs[T].gate, self.inputs[T].up, self.inputs[T].down = base.gate, base.up, base.down
                 self.inputs[T].shared = base.shared
@@ -239,7 +255,6 @@ class Workload:
                         logits=self.logits[T] if logits is None else logits[T],
                         out=self.y[T] if y is None else y[T], trace=trace)
 
-    # algorithmic work of one step, from the routing of each call
     def distinct_experts(self):
         out = {}
         for T in self.Ts:
@@ -250,33 +265,33 @@ class Workload:
         return out
 
     def algorithmic(self):
+        """Algorithmic work of each call: HBM bytes of each traced segment
+        (weights of the distinct experts once, activations in and out once)
+        and tensor FLOPs."""
         cfg = self.cfg
         distinct = self.distinct_experts()
         gb, ub, db = S.expert_bytes(cfg.D, cfg.F, cfg.qtype)
+        sg, su, sd = (S.expert_bytes(cfg.D, cfg.shared_F, "q8_0") if cfg.shared_F else (0, 0, 0))
         act = 2 if cfg.x_dtype == "bf16" else 4
         yb = 2 if cfg.y_dtype == "bf16" else 4
         per_call = {}
         for T in self.Ts:
             n = distinct[T]
-            flops = 2.0 * T * cfg.k * 3 * cfg.D * cfg.F
-            if cfg.shared_F:
-                flops += 2.0 * T * 3 * cfg.D * cfg.shared_F
+            rows = T * cfg.k + (T if cfg.shared_F else 0)
+            fl_gu = 2.0 * T * cfg.k * 2 * cfg.D * cfg.F + (2.0 * T * 2 * cfg.D * cfg.shared_F)
+            fl_dn = 2.0 * T * cfg.k * cfg.D * cfg.F + (2.0 * T * cfg.D * cfg.shared_F)
             x_b = T * cfg.D * act
-            # algorithmic HBM bytes of each traced segment (weights once,
-            # activations in and out once)
+            h_b = rows * cfg.F * 2                       # fp16 hidden rows
             seg = {
                 "ffn_decode": n * (gb + ub + db) + self.shared_bytes + x_b + T * cfg.D * yb,
-                "gateup": n * (gb + ub) + x_b + T * cfg.k * cfg.F * 4,
-                "down": n * db + T * cfg.k * cfg.F * 4 + T * cfg.k * cfg.D * 4,
-                "route": (cfg.D * cfg.E * 4 if base_router(self) else T * cfg.E * 4) + x_b,
+                "gateup": n * (gb + ub) + sg + su + x_b + h_b,
+                "down": n * db + sd + h_b + T * cfg.D * yb,
+                "route": (cfg.D * cfg.E * 4 if self.inputs[T].w_router is not None else T * cfg.E * 4) + x_b,
             }
-            per_call[T] = {"distinct": n, "seg_bytes": seg, "flops": flops,
+            per_call[T] = {"distinct": n, "seg_bytes": seg, "flops": fl_gu + fl_dn,
+                           "seg_flops": {"gateup": fl_gu, "down": fl_dn, "ffn_decode": fl_gu + fl_dn},
                            "weight_bytes": n * (gb + ub + db) + self.shared_bytes}
         return per_call
-
-
-def base_router(wl):
-    return wl.inputs[wl.Ts[0]].w_router is not None
 
 
 # ------------------------------------------------------------- our arm
@@ -289,37 +304,35 @@ def capture_graph(torch, fn, n):
     return g
 
 
-def run_ours(args, world, rank, local):
-    import torch
-    import quantized_routed_expert_top_b200 as moe
-    from quantized_routed_expert_top_b200 import build as B
-    if rank == 0 or not os.path.exists(moe.LIB_PATH):
-        B.build()
-    barrier(world)
-    moe.lib()
-    peaks = measured_peaks()
-    wl = Workload(args.workload, torch, moe, args.replicas)
+class _Eager:
+    def __init__(self, fn, n):
+        self.fn, self.n = fn, n
+
+    def replay(self):
+        for _ in range(self.n):
+            self.fn()
+
+
+def measure_layer(wl, steps, warmup, world, local, peaks, no_graph=False, cpu=True,
+                  cpu_seconds=10.0):
+    """Timed pass, traced pass, end-to-end pass of one workload; returns the
+    JSON fields of its line (or sub-object)."""
+    torch, moe = wl.torch, wl.moe
     algo = wl.algorithmic()
     stream = torch.cuda.current_stream()
-
-    # eager calls first (first-use set-up), then the steps as CUDA graphs: the
-    # decode layer is a handful of short kernels and would otherwise wait on
-    # the host's launch path (--no-graph launches every step eagerly)
+    # eager calls first (first-use set-up), then the steps as CUDA graphs:
+    # the decode layer is a handful of short kernels and would otherwise wait
+    # on the host's launch path (--no-graph launches every step eagerly)
     wl.step()
     torch.cuda.synchronize()
-    trace = moe.KernelTrace(n_calls=args.steps * wl.calls_per_step)
-    if args.no_graph:
-        class _Eager:
-            def __init__(self, fn, n): self.fn, self.n = fn, n
-            def replay(self):
-                for _ in range(self.n): self.fn()
-        g_warm = _Eager(wl.step, args.warmup)
-        g_plain = _Eager(wl.step, args.steps)
-        g_traced = _Eager(lambda: wl.step(trace=trace), args.steps)
+    trace = moe.KernelTrace(n_calls=steps * wl.calls_per_step)
+    if no_graph:
+        g_warm, g_plain = _Eager(wl.step, warmup), _Eager(wl.step, steps)
+        g_traced = _Eager(lambda: wl.step(trace=trace), steps)
     else:
-        g_warm = capture_graph(torch, wl.step, args.warmup)
-        g_plain = capture_graph(torch, wl.step, args.steps)
-        g_traced = capture_graph(torch, lambda: wl.step(trace=trace), args.steps)
+        g_warm = capture_graph(torch, wl.step, warmup)
+        g_plain = capture_graph(torch, wl.step, steps)
+        g_traced = capture_graph(torch, lambda: wl.step(trace=trace), steps)
     g_warm.replay()
     torch.cuda.synchronize()
 
@@ -336,8 +349,7 @@ def run_ours(args, world, rank, local):
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    ms_step = t0.elapsed_time(t1) / args.steps
-    ms_step = max_over_ranks(ms_step, world)
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / steps, world)
 
     # ---- traced pass: the same K steps with the library's trace events
     # between its kernels (per-kernel durations for the roofline)
@@ -349,11 +361,11 @@ def run_ours(args, world, rank, local):
     u1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    ms_traced = max_over_ranks(u0.elapsed_time(u1) / args.steps, world)
+    ms_traced = max_over_ranks(u0.elapsed_time(u1) / steps, world)
     durs = trace.durations()
-    launches = wl.kernels_per_call * wl.calls_per_step * args.steps
 
-    # ---- end to end: pinned host x -> device, layer, device -> pinned host y
+    # ---- end to end: pinned host x (and logits) -> device, layer, device
+    # -> pinned host y, all inside the timed region
     xh = {T: wl.x[T].cpu().pin_memory() for T in wl.Ts}
     yh = {T: torch.empty(wl.y[T].shape, dtype=wl.ydt).pin_memory() for T in wl.Ts}
     xd = {T: torch.empty_like(wl.x[T]) for T in wl.Ts}
@@ -372,13 +384,13 @@ def run_ours(args, world, rank, local):
         for T in wl.Ts:
             yh[T].copy_(wl.y[T], non_blocking=True)
 
-    if args.no_graph:
-        for _ in range(args.warmup):
+    if no_graph:
+        for _ in range(warmup):
             e2e_step()
-        g_e2e = _Eager(e2e_step, args.steps)
+        g_e2e = _Eager(e2e_step, steps)
     else:
-        g_e2e = capture_graph(torch, e2e_step, args.steps)
-        capture_graph(torch, e2e_step, args.warmup).replay()
+        g_e2e = capture_graph(torch, e2e_step, steps)
+        capture_graph(torch, e2e_step, warmup).replay()
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -386,46 +398,31 @@ def run_ours(args, world, rank, local):
     g_e2e.replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
     barrier(world)
 
     tokens = wl.tokens_per_step * world
-    value = tokens / (ms_step / 1e3)
-    roof = roofline(wl, algo, durs, peaks, args)
     out = {
-        "metric": "MoE-layer tokens/s",
-        "value": round(value, 2),
+        "value": round(tokens / (ms_step / 1e3), 2),
         "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": round(ms_step, 5),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": dtype_of(wl.cfg),
-        "data": "synthetic (seeded; random-init Q4_0/Q8_0 experts, no checkpoint)",
         "config": config_of(wl),
-        "roofline": roof,
+        "roofline": roofline(wl, algo, durs, peaks, steps),
         "kernels_ms": {k: round(sum(v) / len(v), 5) for k, v in sorted(durs.items())},
         "kernels_pass": {"ms_per_step": round(ms_traced, 5),
                          "note": "kernels_ms and the roofline come from a second pass of the same "
                                  "K steps with trace events between the library's kernels; those "
                                  "events cut the launch overlap, so that pass runs slower than the "
                                  "timed one"},
-        "gpu_launches": launches,
+        "gpu_launches": wl.kernels_per_call * wl.calls_per_step * steps,
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
-        "peaks": peaks,
-        "launch": "eager" if args.no_graph else "cuda-graph replay",
+        "launch": "eager" if no_graph else "cuda-graph replay",
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, args)
-    if rank == 0 and args.workload == "decode" and not args.no_extra:
-        out["prefill"] = extra_prefill(args, torch, moe, peaks)
-    if rank == 0:
-        print(json.dumps(out), flush=True)
+    if cpu:
+        out["cpu_baseline"] = cpu_baseline(wl, cpu_seconds)
+    return out
 
 
 def dtype_of(cfg):
@@ -443,31 +440,54 @@ def config_of(wl):
     return c
 
 
-def roofline(wl, algo, durs, peaks, args):
+# the dominant kernel's bound per workload: the tensor-core GEMM at T=8192
+# (about 960 FLOP per weight byte, above the B200's ridge of about 250), HBM
+# for everything else (the wide layer at T=2048 does about 140 FLOP per byte)
+TENSOR_BOUND = {"prefill"}
+
+
+def roofline(wl, algo, durs, peaks, steps):
     """Roofline of the dominant traced segment over the timed steps."""
     tot = {k: sum(v) for k, v in durs.items()}
     dom = max(tot, key=tot.get)
     launches = len(durs[dom])
     avg_ms = tot[dom] / launches
-    if wl.name == "prefill" and dom in ("gateup", "down", "ffn_tc"):
-        frac_flops = {"gateup": 2 / 3, "down": 1 / 3}.get(dom, 1.0)
-        work_step = sum(algo[T]["flops"] for T in wl.Ts) * frac_flops
-        achieved = work_step * args.steps / (tot[dom] / 1e3) / 1e12
-        bound, peak, unit, spec = "tensor", peaks["bf16_tflops"], "TFLOP/s", TC_SPEC_TFLOPS
-        psrc = "bf16_tflops (fp16 operands run at the bf16 rate)"
+    flops_step = sum(algo[T]["seg_flops"].get(dom, 0.0) for T in wl.Ts)
+    bytes_step = sum(algo[T]["seg_bytes"].get(dom, 0) for T in wl.Ts)
+    tflops = flops_step * steps / (tot[dom] / 1e3) / 1e12
+    gbs = bytes_step * steps / (tot[dom] / 1e3) / 1e9
+    if wl.name in TENSOR_BOUND and dom in ("gateup", "down"):
+        bound, achieved, peak, unit, spec = "tensor", tflops, peaks["bf16_tflops"], "TFLOP/s", TC_SPEC_TFLOPS
+        psrc = "bf16_tflops burst (fp16 operands run at the bf16 rate)"
+        work = flops_step
     else:
-        work_step = sum(algo[T]["seg_bytes"].get(dom, 0) for T in wl.Ts)
-        achieved = work_step * args.steps / (tot[dom] / 1e3) / 1e9
-        bound, peak, unit, spec = "hbm", peaks["hbm_gbs"], "GB/s", HBM_SPEC_GBS
+        bound, achieved, peak, unit, spec = "hbm", gbs, peaks["hbm_gbs"], "GB/s", HBM_SPEC_GBS
         psrc = "hbm_gbs"
-    return {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
-            "unit": unit, "frac": round(achieved / peak, 4), "frac_of_spec": round(achieved / spec, 4),
-            "algorithmic_per_launch": round(work_step / wl.calls_per_step, 1),
-            "avg_launch_ms": round(avg_ms, 5),
-            "per_T": {str(T): {"work": algo[T]["seg_bytes"].get(dom) if bound == "hbm" else algo[T]["flops"],
-                               "distinct_experts": algo[T]["distinct"]} for T in wl.Ts},
-            "peak_source": f"{peaks['source']} {psrc}",
-            "traffic": ncu_traffic(dom, wl.name)}
+        work = bytes_step
+    r = {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+         "unit": unit, "frac": round(achieved / peak, 4), "frac_of_spec": round(achieved / spec, 4),
+         "algorithmic_per_launch": round(work / wl.calls_per_step, 1),
+         "avg_launch_ms": round(avg_ms, 5),
+         "per_T": {str(T): {"work": algo[T]["seg_flops" if bound == "tensor" else "seg_bytes"].get(dom),
+                            "distinct_experts": algo[T]["distinct"]} for T in wl.Ts},
+         "peak_source": f"{peaks['source']} {psrc}",
+         "traffic": ncu_traffic(dom, wl.name)}
+    if flops_step and bound == "hbm":
+        r["tensor_frac_of_measured"] = round(tflops / peaks["bf16_tflops"], 4)
+    if bound == "tensor":
+        r["frac_of_sustained"] = round(tflops / peaks["bf16_tflops_sustained"], 4)
+        r["hbm_gbs_at_algorithmic_bytes"] = round(gbs, 1)
+    # the other FFN kernels of the step, for context
+    others = {}
+    for k in ("gateup", "down", "ffn_decode"):
+        if k in tot and k != dom:
+            fl = sum(algo[T]["seg_flops"].get(k, 0.0) for T in wl.Ts) * steps / (tot[k] / 1e3) / 1e12
+            by = sum(algo[T]["seg_bytes"].get(k, 0) for T in wl.Ts) * steps / (tot[k] / 1e3) / 1e9
+            others[k] = {"avg_launch_ms": round(tot[k] / len(durs[k]), 5), "tflops": round(fl, 2),
+                         "gbs": round(by, 1)}
+    if others:
+        r["other_kernels"] = others
+    return r
 
 
 # the source files whose code runs in each traced segment's kernels
@@ -518,6 +538,18 @@ def h2d_probe(torch, nbytes=1 << 30):
     return gbs
 
 
+CACHE_MODES = {
+    "dependent": "each layer routes on the GPU, its ids come back to the host (a 32-byte "
+                 "copy and a wait), the host LRU requests them, then the layer runs in two "
+                 "calls: the resident experts' FFN while the misses copy, then the copied "
+                 "experts' FFN and the combine",
+    "two_phase": "the host knows each layer's ids from the trace ahead of the GPU (no wait "
+                 "per layer); each layer runs in two calls around the copy wait as above",
+    "lookahead": "ids from the trace ahead of the GPU; each layer waits for all its copies, "
+                 "then runs in one call",
+}
+
+
 class CacheStack:
     """A stack of the Q8_0 decode layer whose experts live in pinned host
     memory; each layer keeps a fraction of its experts in HBM slots (LRU) and
@@ -551,6 +583,8 @@ class CacheStack:
         self.copy_stream = torch.cuda.Stream()
         self.cache = moe.ExpertCache(*self.host, cfg.qtype, self.n_slots, self.copy_stream)
         self.layers = [moe.Layer(self.cache.pools[l], D, F, E, k, 1) for l in range(n_layers)]
+        self.ids_host = torch.empty((n_layers, k), dtype=torch.int32, pin_memory=True)
+        self.ids_ready = torch.cuda.Event()
         self.resident = None
 
     def make_resident(self):
@@ -562,19 +596,40 @@ class CacheStack:
             pools.append(moe.ExpertPool(g, u, d, cfg.qtype))
         self.resident = [moe.Layer(p, cfg.D, cfg.F, cfg.E, cfg.k, 1) for p in pools]
 
-    def token(self, t, resident=False, logits=None, trace=None):
+    def token(self, t, mode="dependent", logits=None):
+        moe = self.moe
         stream = self.torch.cuda.current_stream()
         lg = self.logits[t] if logits is None else logits
         for l in range(self.n_layers):
-            if resident:
-                lay = self.resident[l]
-            else:
-                self.cache.request(l, self.sets[l][t], stream=stream)
-                self.cache.sync(l, stream=stream)
-                lay = self.layers[l]
-            lay.forward(self.x, logits=lg[l:l + 1], out=self.y, trace=trace)
-            if not resident:
-                self.cache.release(l, stream=stream)
+            if mode == "resident":
+                self.resident[l].forward(self.x, logits=lg[l:l + 1], out=self.y)
+                self.x.add_(self.y)
+                continue
+            lay, c = self.layers[l], self.cache
+            if mode == "dependent":
+                # route on the GPU; the ids come back before the request
+                lay.forward(self.x, logits=lg[l:l + 1], out=self.y, phases=moe.PHASE_ROUTE)
+                self.ids_host[l].copy_(lay.ids[0], non_blocking=True)
+                self.ids_ready.record(stream)
+                self.ids_ready.synchronize()
+                c.request(l, self.ids_host[l].numpy(), stream=stream)
+                lay.forward(self.x, logits=lg[l:l + 1], out=self.y, mask=c.hit_mask(l),
+                            phases=moe.PHASE_FFN | moe.PHASE_SHARED)
+            elif mode == "two_phase":
+                c.request(l, self.sets[l][t], stream=stream)
+                lay.forward(self.x, logits=lg[l:l + 1], out=self.y, mask=c.hit_mask(l),
+                            phases=moe.PHASE_ROUTE | moe.PHASE_FFN | moe.PHASE_SHARED)
+            else:   # lookahead, one call after the copies
+                c.request(l, self.sets[l][t], stream=stream)
+                c.sync(l, stream=stream)
+                lay.forward(self.x, logits=lg[l:l + 1], out=self.y)
+                c.release(l, stream=stream)
+                self.x.add_(self.y)
+                continue
+            c.sync(l, stream=stream)
+            lay.forward(self.x, logits=lg[l:l + 1], out=self.y, mask=c.miss_mask(l),
+                        phases=moe.PHASE_FFN | moe.PHASE_COMBINE)
+            c.release(l, stream=stream)
             self.x.add_(self.y)
 
     def kernels_per_layer_call(self):
@@ -615,80 +670,97 @@ def cache_layers(args):
                          f"memory; this host has {ram / 1e9:.0f} GB, so {max(1, fit)} layers")
 
 
-def run_cache(args, world, rank, local):
+def measure_cache(args, steps, warmup, world, local, peaks, cpu=True):
     import torch
     import quantized_routed_expert_top_b200 as moe
-    from quantized_routed_expert_top_b200 import build as B
-    if rank == 0 or not os.path.exists(moe.LIB_PATH):
-        B.build()
-    barrier(world)
-    moe.lib()
-    peaks = measured_peaks()
     n_layers, reduced = cache_layers(args)
-    n_tok = args.warmup + args.steps
+    modes = ("dependent", "two_phase", "lookahead")
+    n_tok = warmup + steps * (len(modes) + 1) + 1
     st = CacheStack(torch, moe, n_layers, n_tok)
     st.make_resident()
     kpl = st.kernels_per_layer_call()
     pcie = h2d_probe(torch)
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)
+    cursor = [0]
 
-    def timed(resident):
+    def timed(mode, n):
         st.x.copy_(st.x0)
-        for t in range(args.warmup):
-            st.token(t, resident)
         torch.cuda.synchronize()
         h0, m0, b0 = st.cache.stats()
+        x0 = st.cache.exposed_ns()
         barrier(world)
         e0, e1 = ev(), ev()
-        e0.record(stream)
-        for t in range(args.warmup, n_tok):
-            st.token(t, resident)
-        e1.record(stream)
-        torch.cuda.synchronize()
+        with ClockSampler(local, period_s=0.002) as clk:
+            e0.record(stream)
+            for _ in range(n):
+                st.token(cursor[0], mode)
+                cursor[0] += 1
+            e1.record(stream)
+            torch.cuda.synchronize()
         h1, m1, b1 = st.cache.stats()
-        return e0.elapsed_time(e1), (h1 - h0, m1 - m0, b1 - b0)
+        x1 = st.cache.exposed_ns()
+        return e0.elapsed_time(e1), (h1 - h0, m1 - m0, b1 - b0, x1 - x0), clk
 
-    with ClockSampler(local, period_s=0.002) as clk:
-        ms_cache, (hits, misses, nbytes) = timed(False)
-    ms_res, _ = timed(True)
-    ms_cache = max_over_ranks(ms_cache, world)
+    timed("dependent", warmup)               # warm the cache and the kernels
+    res = {}
+    for mode in modes:
+        ms, (hits, misses, nbytes, exp_ns), clk = timed(mode, steps)
+        res[mode] = {"tokens_per_s": round(steps * world / (max_over_ranks(ms, world) / 1e3), 3),
+                     "ms_per_token": round(ms / steps, 4),
+                     "hit_rate": round(hits / max(1, hits + misses), 4),
+                     "misses_per_token": round(misses / steps, 3),
+                     "bytes_copied_per_token": int(nbytes // steps),
+                     "copy_gbs": round(nbytes / (ms / 1e3) / 1e9, 2),
+                     "exposed_copy_ms_per_token": round(exp_ns / 1e6 / steps, 4),
+                     "how": CACHE_MODES[mode]}
+        if mode == "dependent":
+            clk_dep, ms_dep, bytes_dep = clk, ms, nbytes
+    saved = cursor[0]
+    cursor[0] = 0
+    ms_res = 0.0
+    st.x.copy_(st.x0)
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for t in range(steps):
+        st.token(t, "resident")
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_res = e0.elapsed_time(e1)
+    cursor[0] = saved
 
-    # end to end: each token's x and its per-layer trace logits come from
-    # pinned host memory, its output goes back to pinned host memory; the
-    # cache continues from where the timed run left it
+    # end to end (dependent mode): each token's x and its per-layer trace
+    # logits come from pinned host memory, its output goes back to pinned host
     xh = st.x0.cpu().pin_memory()
     yh = torch.empty_like(xh).pin_memory()
     lh = torch.from_numpy(st.logits_host).pin_memory()
     lbuf = torch.empty_like(st.logits[0])
+    n_e2e = min(steps, n_tok - cursor[0])
     torch.cuda.synchronize()
     e0, e1 = ev(), ev()
     e0.record(stream)
-    for t in range(args.warmup, n_tok):
+    for _ in range(n_e2e):
+        t = cursor[0]
+        cursor[0] += 1
         st.x.copy_(xh, non_blocking=True)
         lbuf.copy_(lh[t], non_blocking=True)
-        st.token(t, logits=lbuf)
+        st.token(t, "dependent", logits=lbuf)
         yh.copy_(st.x, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), world)
 
-    steps = args.steps
-    tok_s = steps * world / (ms_cache / 1e3)
-    achieved = nbytes / (ms_cache / 1e3) / 1e9
+    dep = res["dependent"]
+    achieved = bytes_dep / (ms_dep / 1e3) / 1e9
     cfg = st.cfg
     out = {
-        "metric": "MoE-layer tokens/s",
-        "value": round(tok_s, 3),
-        "unit": "tokens/s",
-        "n_gpus": world, "steps": steps, "warmup": args.warmup,
-        "ms_per_step": round(ms_cache / steps, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": dtype_of(cfg),
-        "data": "synthetic (seeded; random-init Q8_0 experts, per-layer locality traces)",
+        "value": dep["tokens_per_s"], "unit": "tokens/s",
+        "ms_per_step": dep["ms_per_token"],
         "config": {"workload": f"cache: one token per step through a {n_layers}-layer stack of the "
                                f"MoE layer D={cfg.D} E={cfg.E} top-{cfg.k} F={cfg.F} Q8_0, experts "
-                               f"in pinned host memory, {st.n_slots} HBM slots per layer (LRU)",
+                               f"in pinned host memory, {st.n_slots} HBM slots per layer (LRU), "
+                               f"dependent routing (value); two_phase / lookahead modes beside it",
                    "layers": n_layers, "slots_per_layer": st.n_slots,
                    "l2": "each step streams its misses from host memory; the resident comparison "
                          "keeps one pool per layer in HBM",
@@ -698,60 +770,84 @@ def run_cache(args, world, rank, local):
                      "frac": round(achieved / pcie, 4),
                      "peak_source": "pinned 1 GiB host-to-device copy measured in this run",
                      "traffic": None},
-        "cache": {"hit_rate": round(hits / max(1, hits + misses), 4),
-                  "misses_per_token": round(misses / steps, 3),
-                  "bytes_copied_per_token": int(nbytes // steps),
-                  "exposed_copy_ms_per_token": round((ms_cache - ms_res) / steps, 4),
-                  "resident_tokens_per_s": round(steps / (ms_res / 1e3), 3)},
+        "modes": res,
+        "resident_tokens_per_s": round(steps / (ms_res / 1e3), 3),
         "gpu_launches": kpl * n_layers * steps,
-        "e2e": {"value": round(steps * world / (ms_e2e / 1e3), 3), "unit": "tokens/s",
+        "e2e": {"value": round(n_e2e * world / (ms_e2e / 1e3), 3), "unit": "tokens/s",
                 "h2d_bytes_per_step": xh.numel() * xh.element_size() + lh[0].numel() * 4,
                 "d2h_bytes_per_step": yh.numel() * yh.element_size()},
-        "clocks": clk.summary(),
-        "peaks": peaks,
+        "clocks": clk_dep.summary(),
         "launch": "eager (the host LRU runs at every layer call)",
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if cpu:
         ns = min(n_layers, 4)
         v, dt = oracle_cache_sample(st.pool_np, st.logits_host, n_layers, ns)
         out["cpu_baseline"] = {"value": round(v, 5), "unit": "tokens/s", "cores": os.cpu_count() or 1,
                                "kind": "oracle",
                                "sample": f"one token through {ns} of the {n_layers} layers (fp64), "
                                          f"{dt:.1f} s, scaled to the whole stack"}
+    st.cache.close()
+    return out
+
+
+def _line(out, args, world, cfg, peaks):
+    line = {"metric": "MoE-layer tokens/s", "value": out["value"], "unit": out["unit"],
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": out["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": dtype_of(cfg),
+            "data": "synthetic (seeded; random-init Q4_0/Q8_0 experts, no checkpoint)"}
+    for k, v in out.items():
+        if k not in line:
+            line[k] = v
+    line["peaks"] = peaks
+    return line
+
+
+# the other configurations of the default run: (key, workload)
+EXTRA = [("tiny", "tiny"), ("prefill", "prefill"), ("wide_t1", "wide_t1"),
+         ("wide_t2048", "wide_t2048")]
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import quantized_routed_expert_top_b200 as moe
+    from quantized_routed_expert_top_b200 import build as B
+    if rank == 0 or not os.path.exists(moe.LIB_PATH):
+        B.build()
+    barrier(world)
+    moe.lib()
+    peaks = measured_peaks()
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if args.workload == "cache":
+        out = measure_cache(args, args.steps, args.warmup, world, local, peaks, cpu=with_cpu)
+        if rank == 0:
+            print(json.dumps(_line(out, args, world, S.CONFIGS["cache"], peaks)), flush=True)
+        return
+    wl = Workload(args.workload, torch, moe, args.replicas)
+    out = measure_layer(wl, args.steps, args.warmup, world, local, peaks, args.no_graph, cpu=with_cpu)
+    line = _line(out, args, world, wl.cfg, peaks)
+    del wl
+    if args.workload == "decode" and not args.no_extra and world == 1:
+        # every other configuration, each with its own roofline, end-to-end
+        # number and oracle baseline (fewer steps: the decode line is the
+        # headline, these keep the whole run within a few minutes)
+        steps = max(5, min(args.steps, 20))
+        line["configs"] = {}
+        bases = {}
+        for key, name in EXTRA:
+            cfg_name = name.split("_")[0]
+            if cfg_name not in bases:      # one expert pool per configuration
+                T_big = max(max(WORKLOADS[n][0]) for _, n in EXTRA if n.split("_")[0] == cfg_name)
+                bases[cfg_name] = S.make_layer(S.CONFIGS[cfg_name], T=T_big)
+            w = Workload(name, torch, moe, base=bases[cfg_name])
+            line["configs"][key] = measure_layer(w, steps, args.warmup, world, local, peaks,
+                                                 args.no_graph, cpu=with_cpu, cpu_seconds=6.0)
+            del w
+            torch.cuda.empty_cache()
+        line["configs"]["cache"] = measure_cache(args, max(5, min(args.steps, 16)), args.warmup,
+                                                 world, local, peaks, cpu=with_cpu)
     if rank == 0:
-        print(json.dumps(out), flush=True)
-
-
-# ------------------------------------------------------------ prefill extra
-def extra_prefill(args, torch, moe, peaks):
-    wl = Workload("prefill", torch, moe)
-    algo = wl.algorithmic()
-    for _ in range(3):
-        wl.step()
-    torch.cuda.synchronize()
-    steps = max(3, min(args.steps, 10))
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(steps):
-        wl.step()
-    t1.record()
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
-    # per-kernel durations from a second, traced pass (see run_ours)
-    trace = moe.KernelTrace(n_calls=steps)
-    for _ in range(steps):
-        wl.step(trace=trace)
-    torch.cuda.synchronize()
-    durs = trace.durations()
-    flops = sum(algo[T]["flops"] for T in wl.Ts)
-    ffn_ms = sum(sum(durs.get(k, [])) for k in ("gateup", "down")) / steps
-    return {"workload": config_of(wl)["workload"], "tokens_per_s": round(8192 / (ms / 1e3), 1),
-            "ms_per_step": round(ms, 4),
-            "kernels_ms": {k: round(sum(v) / len(v), 4) for k, v in sorted(durs.items())},
-            "ffn_tflops": round(flops / (ffn_ms / 1e3) / 1e12, 2),
-            "ffn_tc_frac_of_measured": round(flops / (ffn_ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
-            "ffn_tc_frac_of_spec": round(flops / (ffn_ms / 1e3) / 1e12 / TC_SPEC_TFLOPS, 4),
-            "flops_per_step": flops}
+        print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -776,16 +872,16 @@ def oracle_step_fn(wl_inputs, cfg, Ts, frac=1.0):
     return step
 
 
-def cpu_baseline(wl, args):
+def cpu_baseline(wl, seconds=10.0):
     """The oracle as it stands, on the host cores, on a bounded sample."""
     cores = os.cpu_count() or 1
-    frac = 1.0 if wl.name == "decode" else 32.0 / max(wl.Ts)
+    frac = 1.0 if max(wl.Ts) <= 16 else 32.0 / max(wl.Ts)
     step = oracle_step_fn(wl.inputs, wl.cfg, wl.Ts, frac)
     t = time.perf_counter()
     n = step()
     dt = time.perf_counter() - t
     reps = 1
-    while time.perf_counter() - t < 10.0 and reps < 20:
+    while time.perf_counter() - t < seconds and reps < 20:
         n += step()
         reps += 1
     dt = time.perf_counter() - t
@@ -835,11 +931,11 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     name = args.workload
-    cfg = S.CONFIGS[name]
+    cfg = S.CONFIGS[name.split("_")[0]]
     if name == "cache":
         run_reference_cache(args, world)
         return
-    Ts = {"decode": (1, 4, 16), "prefill": (8192,), "wide": (1, 2048)}[name]
+    Ts = WORKLOADS[name][0]
     base = S.make_layer(cfg, T=max(Ts))
     inputs = {max(Ts): base}
     for T in Ts:
@@ -848,7 +944,8 @@ def run_reference(args, world, rank):
             inputs[T].gate, inputs[T].up, inputs[T].down = base.gate, base.up, base.down
             inputs[T].shared = base.shared
     # size the per-step sample so that warmup + steps end within ~3 minutes
-    step = oracle_step_fn(inputs, cfg, Ts, 1.0 if name == "decode" else 16.0 / max(Ts))
+    small = max(Ts) <= 16
+    step = oracle_step_fn(inputs, cfg, Ts, 1.0 if small else 16.0 / max(Ts))
     t = time.perf_counter()
     n1 = step()
     t1 = time.perf_counter() - t
@@ -856,8 +953,8 @@ def run_reference(args, world, rank):
     frac = 1.0
     if t1 > budget:
         frac = max(budget / t1, 1.0 / n1)
-    total = sum(Ts) if name == "decode" else 16 * len(Ts)
-    step = oracle_step_fn(inputs, cfg, Ts, frac * (1.0 if name == "decode" else 16.0 / max(Ts)))
+    total = sum(Ts)
+    step = oracle_step_fn(inputs, cfg, Ts, frac * (1.0 if small else 16.0 / max(Ts)))
     for _ in range(max(0, args.warmup - 1)):
         step()
     t = time.perf_counter()
@@ -888,7 +985,9 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "prefill", "wide", "cache"], default="decode")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["cache"], default="decode",
+                    help="the workload of the line (decode also reports every other one under "
+                         "'configs' unless --no-extra)")
     ap.add_argument("--cache-layers", type=int, default=0,
                     help="layers of the cache stack (default: 40, fewer if host memory is short)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -907,10 +1006,7 @@ def main():
         return
     world, rank, local = dist_setup()
     try:
-        if args.workload == "cache":
-            run_cache(args, world, rank, local)
-        else:
-            run_ours(args, world, rank, local)
+        run_ours(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

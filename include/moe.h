@@ -366,6 +366,13 @@ moe_status moe_layer_forward(const moe_layer_args *args, void *workspace,
  *   dev_slot_map        device int32 [n_layers][E]; entries of experts that
  *                       are not resident hold -1
  *   copy_stream         stream for the host-to-device copies (not NULL)
+ *   dev_masks           device uint8 [n_layers][2][E] or NULL: per layer, the
+ *                       last request's hit mask (requested and already
+ *                       resident) and miss mask (requested and copied by
+ *                       that request), written with the slot map; they are
+ *                       the expert_mask arguments of the two moe_layer_forward
+ *                       calls that overlap the copies with the FFN of the
+ *                       resident experts (see moe_layer_args)
  * The cache keeps pointers to the caller's buffers; they must outlive it. */
 typedef struct moe_cache moe_cache;
 typedef struct {
@@ -379,6 +386,7 @@ typedef struct {
     void *dev_down;
     int32_t *dev_slot_map;
     moe_stream copy_stream;
+    uint8_t *dev_masks;
 } moe_cache_desc;
 
 moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out);
@@ -406,6 +414,16 @@ moe_status moe_cache_sync(moe_cache *cache, int layer, moe_stream compute);
 moe_status moe_cache_release(moe_cache *cache, int layer, moe_stream compute);
 /* The device pool view of one layer (slot-mapped). */
 moe_status moe_cache_layer_pool(moe_cache *cache, int layer, moe_pool *out);
+/* Device addresses of one layer's hit and miss masks (dev_masks).  The
+ * flow of one cached layer step, with the copies overlapping compute:
+ *   moe_cache_request(c, l, ids, ...)
+ *   moe_layer_forward(ROUTE | FFN | SHARED, expert_mask = hit)
+ *   moe_cache_sync(c, l, compute)
+ *   moe_layer_forward(FFN | COMBINE, expert_mask = miss)
+ *   moe_cache_release(c, l, compute)
+ * MOE_ERR_INVALID_ARG without dev_masks. */
+moe_status moe_cache_layer_masks(moe_cache *cache, int layer, const uint8_t **hit,
+                                 const uint8_t **miss);
 /* Counters since moe_cache_init: hits, misses, bytes copied, and
  * exposed_ns, the time the compute stream spent waiting in moe_cache_sync
  * for miss copies (measured on the GPU between two events recorded around

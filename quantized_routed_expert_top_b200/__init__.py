@@ -73,7 +73,8 @@ class CacheDesc(C.Structure):
                 ("bytes_down", C.c_size_t), ("host_gate", C.POINTER(C.c_void_p)),
                 ("host_up", C.POINTER(C.c_void_p)), ("host_down", C.POINTER(C.c_void_p)),
                 ("dev_gate", C.c_void_p), ("dev_up", C.c_void_p), ("dev_down", C.c_void_p),
-                ("dev_slot_map", C.c_void_p), ("copy_stream", C.c_void_p)]
+                ("dev_slot_map", C.c_void_p), ("copy_stream", C.c_void_p),
+                ("dev_masks", C.c_void_p)]
 
 
 _lib = None
@@ -111,6 +112,7 @@ def lib():
         L.moe_cache_sync.argtypes = [_v, _i, _v]
         L.moe_cache_release.argtypes = [_v, _i, _v]
         L.moe_cache_layer_pool.argtypes = [_v, _i, C.POINTER(Pool)]
+        L.moe_cache_layer_masks.argtypes = [_v, _i, C.POINTER(_v), C.POINTER(_v)]
         L.moe_cache_stats.argtypes = [_v, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
                                       C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
         L.moe_route_noalloc.argtypes = [_v, C.c_int32, _v, _v, _i, _i, _i, _i, _i, _v, _v, _v,
@@ -403,6 +405,8 @@ class ExpertCache:
         self.dev_down = torch.empty((self.n_layers, n_slots) + tuple(host_down[0].shape[1:]),
                                     dtype=torch.uint8, device=dev)
         self.slot_map = torch.full((self.n_layers, self.E), -1, dtype=torch.int32, device=dev)
+        # per layer: [hit mask, miss mask] of the last request
+        self.masks = torch.zeros((self.n_layers, 2, self.E), dtype=torch.uint8, device=dev)
         self.copy_stream = copy_stream
         arr = lambda lst: (C.c_void_p * self.n_layers)(*[t.data_ptr() for t in lst])
         self._ptrs = [arr(l) for l in self.host]
@@ -416,6 +420,7 @@ class ExpertCache:
                                             self.dev_down.data_ptr())
         d.dev_slot_map = self.slot_map.data_ptr()
         d.copy_stream = copy_stream.cuda_stream
+        d.dev_masks = self.masks.data_ptr()
         self._desc = d
         h = C.c_void_p()
         _check(lib().moe_cache_init(C.byref(d), C.byref(h)))
@@ -442,6 +447,14 @@ class ExpertCache:
         _check(lib().moe_cache_request(self._h, layer, f(ids), n, f(slots), f(miss), f(ev),
                                        C.byref(nm), _stream(stream)))
         return slots, miss.astype(bool), ev
+
+    def hit_mask(self, layer: int):
+        """Device uint8 [E]: experts of the layer's last request already resident."""
+        return self.masks[layer, 0]
+
+    def miss_mask(self, layer: int):
+        """Device uint8 [E]: experts the layer's last request copied."""
+        return self.masks[layer, 1]
 
     def sync(self, layer: int, stream=None):
         _check(lib().moe_cache_sync(self._h, layer, _stream(stream)))

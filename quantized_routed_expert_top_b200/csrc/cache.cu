@@ -30,6 +30,7 @@
 #include "moe_internal.cuh"
 
 #include <chrono>
+#include <cstring>
 #include <new>
 #include <thread>
 #include <vector>
@@ -49,7 +50,12 @@ struct moe_cache {
         int map_buf = 0;
     };
     std::vector<Layer> layers;
-    int32_t *pinned_maps = nullptr;       // [n_layers][2][E]
+    // pinned staging per (layer, buffer): the slot map (int32[E]), then the
+    // request's hit and miss masks (uint8[E] each)
+    uint8_t *pinned_stage = nullptr;
+    size_t stage_stride = 0;
+    int32_t *stage_map(int l, int b) { return (int32_t *)(pinned_stage + ((size_t)l * 2 + b) * stage_stride); }
+    uint8_t *stage_masks(int l, int b) { return (uint8_t *)(stage_map(l, b) + d.E); }
     cudaEvent_t compute_ready = nullptr;
     int64_t hits = 0, misses = 0, bytes = 0;
     int fail_copy_at = -1;                // test hook: fail the n-th copy
@@ -145,7 +151,8 @@ moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out) {
     c->d = d;
     c->layers.resize(d.n_layers);
     moe_status st = MOE_OK;
-    cudaError_t e = cudaHostAlloc((void **)&c->pinned_maps, sizeof(int32_t) * d.n_layers * 2 * d.E,
+    c->stage_stride = round_up(sizeof(int32_t) * d.E + 2 * (size_t)d.E, 64);
+    cudaError_t e = cudaHostAlloc((void **)&c->pinned_stage, c->stage_stride * d.n_layers * 2,
                                   cudaHostAllocDefault);
     if (e != cudaSuccess) st = cuda_status(e, "moe_cache_init: pinned slot maps");
     if (st == MOE_OK) st = cuda_status(cudaEventCreateWithFlags(&c->compute_ready, cudaEventDisableTiming), "cudaEventCreate");
@@ -159,16 +166,22 @@ moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out) {
             st = cuda_status(cudaEventCreateWithFlags(&L.release_ev, cudaEventDisableTiming), "cudaEventCreate");
         for (int b = 0; b < 2 && st == MOE_OK; b++)
             st = cuda_status(cudaEventCreateWithFlags(&L.map_done[b], cudaEventDisableTiming), "cudaEventCreate");
-        for (int i = 0; i < 2 * d.E; i++) c->pinned_maps[(size_t)l * 2 * d.E + i] = -1;
+        if (st == MOE_OK)
+            for (int b = 0; b < 2; b++) {
+                for (int i = 0; i < d.E; i++) c->stage_map(l, b)[i] = -1;
+                memset(c->stage_masks(l, b), 0, 2 * (size_t)d.E);
+            }
     }
-    // all slot maps start empty (-1)
-    if (st == MOE_OK)
-        st = cuda_status(cudaMemcpy(d.dev_slot_map, c->pinned_maps, sizeof(int32_t) * d.E,
-                                    cudaMemcpyHostToDevice), "moe_cache_init: slot map");
-    for (int l = 1; l < d.n_layers && st == MOE_OK; l++)
-        st = cuda_status(cudaMemcpy(d.dev_slot_map + (size_t)l * d.E, c->pinned_maps,
+    // all slot maps start empty (-1), all masks zero
+    for (int l = 0; l < d.n_layers && st == MOE_OK; l++) {
+        st = cuda_status(cudaMemcpy(d.dev_slot_map + (size_t)l * d.E, c->stage_map(l, 0),
                                     sizeof(int32_t) * d.E, cudaMemcpyHostToDevice),
                          "moe_cache_init: slot map");
+        if (st == MOE_OK && d.dev_masks)
+            st = cuda_status(cudaMemcpy(d.dev_masks + (size_t)l * 2 * d.E, c->stage_masks(l, 0),
+                                        2 * (size_t)d.E, cudaMemcpyHostToDevice),
+                             "moe_cache_init: masks");
+    }
     if (st != MOE_OK) { moe_cache_destroy(c); return st; }
     *out = c;
     return MOE_OK;
@@ -187,7 +200,7 @@ void moe_cache_destroy(moe_cache *c) {
         cudaEventDestroy(pr.second);
     }
     for (auto ev : c->free_events) cudaEventDestroy(ev);
-    if (c->pinned_maps) cudaFreeHost(c->pinned_maps);
+    if (c->pinned_stage) cudaFreeHost(c->pinned_stage);
     delete c;
 }
 
@@ -304,12 +317,25 @@ moe_status moe_cache_request(moe_cache *c, int layer, const int32_t *ids, int n,
     L.pending = L.pending || (!miss_idx.empty() && cst == MOE_OK);
     L.released = false;                   // the release point covered the previous request only
 
-    // device slot map of the layer
-    int32_t *hm = c->pinned_maps + ((size_t)layer * 2 + buf) * d.E;
+    // device slot map of the layer (and the request's hit / miss masks)
+    int32_t *hm = c->stage_map(layer, buf);
     for (int e = 0; e < d.E; e++) hm[e] = L.expert_slot[e];
     moe_status mst = cuda_status(cudaMemcpyAsync(d.dev_slot_map + (size_t)layer * d.E, hm,
                                                  sizeof(int32_t) * d.E, cudaMemcpyHostToDevice, cs),
                                  "moe_cache_request: slot map copy");
+    if (mst == MOE_OK && d.dev_masks) {
+        uint8_t *hit = c->stage_masks(layer, buf), *mis = hit + d.E;
+        memset(hit, 0, 2 * (size_t)d.E);
+        std::vector<char> missed(n, 0);
+        if (cst == MOE_OK) for (int i : miss_idx) missed[i] = 1;
+        for (int i = 0; i < n; i++) {
+            if (missed[i]) mis[ids[i]] = 1;
+            else if (L.expert_slot[ids[i]] >= 0) hit[ids[i]] = 1;
+        }
+        mst = cuda_status(cudaMemcpyAsync(d.dev_masks + (size_t)layer * 2 * d.E, hit, 2 * (size_t)d.E,
+                                          cudaMemcpyHostToDevice, cs),
+                          "moe_cache_request: mask copy");
+    }
     if (mst == MOE_OK) mst = cuda_status(cudaEventRecord(L.map_done[buf], cs), "cudaEventRecord");
     L.map_buf ^= 1;
     if (cst != MOE_OK) return cst;
@@ -358,6 +384,18 @@ moe_status moe_cache_release(moe_cache *c, int layer, moe_stream compute) {
     moe_status st = cuda_status(cudaEventRecord(L.release_ev, (cudaStream_t)compute), "cudaEventRecord");
     L.released = st == MOE_OK;
     return st;
+}
+
+moe_status moe_cache_layer_masks(moe_cache *c, int layer, const uint8_t **hit,
+                                 const uint8_t **miss) {
+    if (!c || layer < 0 || layer >= c->d.n_layers || !c->d.dev_masks) {
+        set_error("moe_cache_layer_masks: bad cache or layer, or the cache has no dev_masks");
+        return MOE_ERR_INVALID_ARG;
+    }
+    const uint8_t *base = c->d.dev_masks + (size_t)layer * 2 * c->d.E;
+    if (hit) *hit = base;
+    if (miss) *miss = base + c->d.E;
+    return MOE_OK;
 }
 
 moe_status moe_cache_layer_pool(moe_cache *c, int layer, moe_pool *out) {

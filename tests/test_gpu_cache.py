@@ -169,16 +169,20 @@ def _masks(E, ids, miss):
     return torch.from_numpy(hit).cuda(), torch.from_numpy(mis).cuda()
 
 
-def _two_phase(moe, cache, lay, l, ids, x, lg, out, stream):
+def _two_phase(moe, cache, lay, l, ids, x, lg, out, stream, check_masks=False):
     """One cached layer step with the miss copies overlapping the FFN of the
     resident experts: route + resident FFN, wait for the copies, the copied
-    experts' FFN + combine."""
+    experts' FFN + combine.  The masks are the ones the cache writes with
+    the slot map (optionally checked against the host's request result)."""
     _, miss, _ = cache.request(l, ids, stream=stream)
-    m_hit, m_miss = _masks(lay.E, ids, miss)
-    lay.forward(x, logits=lg, out=out, mask=m_hit,
+    lay.forward(x, logits=lg, out=out, mask=cache.hit_mask(l),
                 phases=moe.PHASE_ROUTE | moe.PHASE_FFN | moe.PHASE_SHARED)
     cache.sync(l, stream=stream)
-    lay.forward(x, logits=lg, out=out, mask=m_miss, phases=moe.PHASE_FFN | moe.PHASE_COMBINE)
+    lay.forward(x, logits=lg, out=out, mask=cache.miss_mask(l),
+                phases=moe.PHASE_FFN | moe.PHASE_COMBINE)
+    if check_masks:
+        m_hit, m_miss = _masks(lay.E, ids, miss)
+        assert torch.equal(cache.hit_mask(l), m_hit) and torch.equal(cache.miss_mask(l), m_miss)
     return int(miss.sum())
 
 
@@ -197,7 +201,7 @@ def test_two_phase_cached_layers_are_bit_identical_to_resident(moe, stack):
             lg = torch.from_numpy(traces[l][t:t + 1]).cuda()
             y_c = torch.full((1, D), float("nan"), device="cuda")
             n_miss += _two_phase(moe, cache, cached[l], l, _ids(traces[l][t]), xd[t:t + 1], lg,
-                                 y_c, stream)
+                                 y_c, stream, check_masks=(t % 7 == 0))
             cache.release(l, stream=stream)
             y_r = resident[l].forward(xd[t:t + 1], logits=lg).clone()
             torch.cuda.synchronize()
