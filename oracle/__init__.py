@@ -75,6 +75,14 @@ def _declare(L):
     L.orc_lru_free.argtypes = [_p]
     L.orc_lru_request.restype = _i
     L.orc_lru_request.argtypes = [_p, _p, _i, _p, _p, _p]
+    L.orc_glru_new.restype = _p
+    L.orc_glru_new.argtypes = [_i, _i, _i, _i]
+    L.orc_glru_free.restype = None
+    L.orc_glru_free.argtypes = [_p]
+    L.orc_glru_request.restype = _i
+    L.orc_glru_request.argtypes = [_p, _i, _p, _i, _p, _p, _p]
+    L.orc_glru_resize.restype = _i
+    L.orc_glru_resize.argtypes = [_p, _i, _p, _p, _p, _p]
 
 
 def _ptr(a):
@@ -228,6 +236,48 @@ class LRU:
         h = getattr(self, "_h", None)
         if h:
             lib().orc_lru_free(h)
+            self._h = None
+
+
+class GlobalLRU:
+    """Expert-cache LRU simulation shared by all layers, with run-time resize
+    (rules in moe_oracle.c, orc_glru_request / orc_glru_resize).  Entries are
+    keyed layer * E + expert."""
+
+    def __init__(self, n_layers: int, E: int, max_slots: int, cap: int):
+        self._h = lib().orc_glru_new(n_layers, E, max_slots, cap)
+        if not self._h:
+            raise ValueError("bad global LRU shape")
+        self.n_layers, self.E, self.max_slots = n_layers, E, max_slots
+
+    def request(self, layer: int, ids):
+        ids = _c(ids, np.int32)
+        n = len(ids)
+        slot = np.empty(n, np.int32)
+        miss = np.empty(n, np.int32)
+        ev = np.empty(n, np.int32)
+        rc = lib().orc_glru_request(self._h, layer, _ptr(ids), n, _ptr(slot), _ptr(miss),
+                                    _ptr(ev))
+        if rc == -2:
+            raise OverflowError("more ids than the capacity")
+        if rc < 0:
+            raise ValueError("bad layer, or bad or duplicate expert id")
+        return slot, miss.astype(bool), ev
+
+    def resize(self, cap: int):
+        """-> (evicted keys, moves as an [n, 2] array of (from, to) slots)."""
+        ev = np.empty(self.max_slots, np.int32)
+        mv = np.empty(2 * self.max_slots, np.int32)
+        ne, nm = C.c_int(0), C.c_int(0)
+        rc = lib().orc_glru_resize(self._h, cap, _ptr(ev), C.byref(ne), _ptr(mv), C.byref(nm))
+        if rc < 0:
+            raise ValueError("capacity out of range")
+        return ev[: ne.value].copy(), mv[: 2 * nm.value].reshape(-1, 2).copy()
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            lib().orc_glru_free(h)
             self._h = None
 
 

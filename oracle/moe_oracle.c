@@ -400,3 +400,154 @@ int orc_lru_request(void *p, const int32_t *ids, int n, int32_t *slot,
     free(wanted);
     return misses;
 }
+
+/* ------------------------------------------------------------------------
+ * Expert-cache LRU simulation, global across layers, with run-time resize
+ * (FreeToken fork README, "About": global LRU expert caching, and
+ * "Elastic Memory Management": run-time re-allocation of the expert cache's
+ * VRAM; FreeToken wiki explainer: shared LRU expert caching, elastic cache
+ * resizing; kongchang article, "Dynamic Cache Adjustment Experiments").
+ *
+ * Rules (the pages name a global LRU and resizing only; these fill in the
+ * rest, and reduce to orc_lru_request when there is one layer):
+ *  - one pool of max_slots device slots shared by every layer; the first
+ *    `cap` of them are in use (the capacity), all empty at start;
+ *  - an entry is (layer, expert), keyed layer * E + expert;
+ *  - a request is a list of distinct expert ids of one layer for one step;
+ *    it fails (returns -2) if it holds more ids than the capacity, -1 on a
+ *    bad id or layer; one step counter serves every layer;
+ *  - every requested entry is stamped with the step number;
+ *  - ids are served in the order given; a resident entry is a hit;
+ *  - a missing entry takes the empty slot of lowest index below cap if
+ *    there is one, otherwise evicts the resident entry with the oldest stamp
+ *    among all layers that is not requested in this step (entries of the
+ *    same layer and id), the lower key on equal stamps;
+ *  - resize to a capacity c (1 <= c <= max_slots): a larger c only adds
+ *    empty slots; a smaller c first evicts, oldest stamp first (lower key on
+ *    equal stamps), until at most c entries are resident, then moves every
+ *    entry held in a slot >= c, in increasing slot order, to the empty slot
+ *    of lowest index below c.
+ * Outputs of a request per id: slot[i], miss[i], evicted[i] (key of the
+ * entry evicted to make room, or -1); returns the number of misses.
+ * Outputs of a resize: the keys evicted (in order, *n_evicted of them) and
+ * the moves as (from, to) slot pairs (in order, *n_moves of them).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int n_layers, E, max_slots, cap;
+    int64_t step;
+    int32_t *slot_key;      /* [max_slots], -1 = empty */
+    int32_t *key_slot;      /* [n_layers * E], -1 = not resident */
+    int64_t *stamp;         /* [n_layers * E] */
+} orc_glru;
+
+void *orc_glru_new(int n_layers, int E, int max_slots, int cap)
+{
+    if (n_layers <= 0 || E <= 0 || max_slots <= 0 || cap <= 0 || cap > max_slots) return NULL;
+    orc_glru *c = (orc_glru *)calloc(1, sizeof(orc_glru));
+    size_t nk = (size_t)n_layers * (size_t)E;
+    c->n_layers = n_layers; c->E = E; c->max_slots = max_slots; c->cap = cap; c->step = 0;
+    c->slot_key = (int32_t *)malloc(sizeof(int32_t) * (size_t)max_slots);
+    c->key_slot = (int32_t *)malloc(sizeof(int32_t) * nk);
+    c->stamp = (int64_t *)calloc(nk, sizeof(int64_t));
+    for (int s = 0; s < max_slots; s++) c->slot_key[s] = -1;
+    for (size_t k = 0; k < nk; k++) c->key_slot[k] = -1;
+    return c;
+}
+
+void orc_glru_free(void *p)
+{
+    orc_glru *c = (orc_glru *)p;
+    if (!c) return;
+    free(c->slot_key); free(c->key_slot); free(c->stamp); free(c);
+}
+
+/* The resident entry with the oldest stamp (lower key on equal stamps),
+ * skipping entries of `layer` whose id is marked in `wanted` (NULL: none). */
+static int glru_oldest(const orc_glru *c, int layer, const char *wanted)
+{
+    int best = -1;
+    int nk = c->n_layers * c->E;
+    for (int k = 0; k < nk; k++) {
+        if (c->key_slot[k] < 0) continue;
+        if (wanted && k / c->E == layer && wanted[k % c->E]) continue;
+        if (best < 0 || c->stamp[k] < c->stamp[best]) best = k;
+    }
+    return best;
+}
+
+int orc_glru_request(void *p, int layer, const int32_t *ids, int n, int32_t *slot,
+                     int32_t *miss, int32_t *evicted)
+{
+    orc_glru *c = (orc_glru *)p;
+    if (layer < 0 || layer >= c->n_layers) return -1;
+    if (n > c->cap) return -2;
+    for (int i = 0; i < n; i++) {
+        if (ids[i] < 0 || ids[i] >= c->E) return -1;
+        for (int j = 0; j < i; j++) if (ids[j] == ids[i]) return -1;
+    }
+    c->step++;
+    char *wanted = (char *)calloc((size_t)c->E, 1);
+    for (int i = 0; i < n; i++) wanted[ids[i]] = 1;
+    int misses = 0;
+    for (int i = 0; i < n; i++) {
+        int key = layer * c->E + ids[i];
+        evicted[i] = -1;
+        if (c->key_slot[key] >= 0) {
+            slot[i] = c->key_slot[key];
+            miss[i] = 0;
+        } else {
+            int s = -1;
+            for (int q = 0; q < c->cap; q++)
+                if (c->slot_key[q] < 0) { s = q; break; }
+            if (s < 0) {
+                int victim = glru_oldest(c, layer, wanted);
+                s = c->key_slot[victim];
+                c->key_slot[victim] = -1;
+                evicted[i] = victim;
+            }
+            c->slot_key[s] = key;
+            c->key_slot[key] = s;
+            slot[i] = s;
+            miss[i] = 1;
+            misses++;
+        }
+        c->stamp[key] = c->step;
+    }
+    free(wanted);
+    return misses;
+}
+
+int orc_glru_resize(void *p, int cap, int32_t *evicted, int *n_evicted, int32_t *moves,
+                    int *n_moves)
+{
+    orc_glru *c = (orc_glru *)p;
+    *n_evicted = 0;
+    *n_moves = 0;
+    if (cap < 1 || cap > c->max_slots) return -1;
+    if (cap < c->cap) {
+        int resident = 0;
+        for (int s = 0; s < c->cap; s++) if (c->slot_key[s] >= 0) resident++;
+        while (resident > cap) {
+            int victim = glru_oldest(c, -1, NULL);
+            c->slot_key[c->key_slot[victim]] = -1;
+            c->key_slot[victim] = -1;
+            evicted[(*n_evicted)++] = victim;
+            resident--;
+        }
+        for (int s = cap; s < c->cap; s++) {
+            int key = c->slot_key[s];
+            if (key < 0) continue;
+            int d = -1;
+            for (int q = 0; q < cap; q++)
+                if (c->slot_key[q] < 0) { d = q; break; }
+            c->slot_key[d] = key;
+            c->slot_key[s] = -1;
+            c->key_slot[key] = d;
+            moves[2 * *n_moves] = s;
+            moves[2 * *n_moves + 1] = d;
+            (*n_moves)++;
+        }
+    }
+    c->cap = cap;
+    return 0;
+}

@@ -366,3 +366,90 @@ def test_lru_invariants_random_trace(orc):
         assert len(set(resident.values())) == len(resident)
         total_miss += int(m.sum())
     assert 0 < total_miss < 200 * k
+
+
+# ----------------------------------------------------- global LRU + resize
+def test_global_lru_hand_worked_trace(orc):
+    # 2 layers x 4 experts, keys layer*4 + e; 4 slots, capacity 3 at start.
+    # One step counter for every layer.  Worked by hand from the rules:
+    #  1: L0 [0,1]   keys 0,1 -> empty slots 0,1                 0@1 1@1
+    #  2: L1 [0]     key 4 -> empty slot 2                       4@2
+    #  3: L0 [1,2]   1 hits (slot 1); key 2: full, oldest not requested
+    #                is 0@1 (4@2 newer, 1 requested) -> slot 0, evicts 0
+    #  4: L1 [1,0]   key 5: full; keys 4, 5 of layer 1 are protected;
+    #                1@3 and 2@3 tie -> lower key 1 -> slot 1; key 4 hits
+    #  resize(4):    one more empty slot (3)
+    #  6: L0 [3]     key 3 -> empty slot 3                       3@5
+    #  resize(2):    4 resident > 2: evict 2@3, then 4@4 and 5@4 tie -> 4;
+    #                slot 3 (key 3) is >= 2 -> moves to empty slot 0
+    #  8: L1 [1]     key 5 hits in slot 1
+    #  9: L0 [0,1,2] more ids than the capacity
+    # 10: L1 [2]     key 6: full; oldest not requested of 3@5, 5@6 -> 3
+    g = orc.GlobalLRU(2, 4, 4, 3)
+    chk = lambda r, s, m, e: (list(r[0]) == s and list(r[1]) == m and list(r[2]) == e) or r
+    assert chk(g.request(0, [0, 1]), [0, 1], [True, True], [-1, -1]) is True
+    assert chk(g.request(1, [0]), [2], [True], [-1]) is True
+    assert chk(g.request(0, [1, 2]), [1, 0], [False, True], [-1, 0]) is True
+    assert chk(g.request(1, [1, 0]), [1, 2], [True, False], [1, -1]) is True
+    ev, mv = g.resize(4)
+    assert len(ev) == 0 and len(mv) == 0
+    assert chk(g.request(0, [3]), [3], [True], [-1]) is True
+    ev, mv = g.resize(2)
+    assert list(ev) == [2, 4] and mv.tolist() == [[3, 0]]
+    assert chk(g.request(1, [1]), [1], [False], [-1]) is True
+    with pytest.raises(OverflowError):
+        g.request(0, [0, 1, 2])
+    assert chk(g.request(1, [2]), [0], [True], [3]) is True
+    with pytest.raises(ValueError):
+        g.resize(5)
+    with pytest.raises(ValueError):
+        g.request(2, [0])
+
+
+def test_global_lru_one_layer_is_the_per_layer_lru(orc):
+    # with one layer and a fixed capacity the global rules are the per-layer
+    # ones (pinned by its own hand-worked trace above)
+    rng = np.random.default_rng(17)
+    E, n_slots, k = 24, 9, 6
+    a, b = orc.LRU(E, n_slots), orc.GlobalLRU(1, E, n_slots, n_slots)
+    for step in range(300):
+        req = rng.choice(E, k, replace=False).astype(np.int32)
+        ra, rb = a.request(req), b.request(0, req)
+        for x, y in zip(ra, rb):
+            assert np.array_equal(x, y), step
+
+
+def test_global_lru_invariants_random_trace_with_resizes(orc):
+    rng = np.random.default_rng(19)
+    L, E, max_slots, k = 4, 16, 40, 6
+    g = orc.GlobalLRU(L, E, max_slots, 24)
+    cap = 24
+    where = {}                      # key -> slot
+    for step in range(400):
+        if step % 37 == 36:         # shrink or grow
+            new = int(rng.integers(k, max_slots + 1))
+            ev, mv = g.resize(new)
+            if new >= cap:
+                assert len(ev) == 0 and len(mv) == 0
+            for key in ev:
+                where.pop(int(key))
+            old = dict(where)
+            for src, dst in mv:
+                key = [kk for kk, s in old.items() if s == src]
+                assert len(key) == 1 and src >= new and dst < new
+                where[key[0]] = int(dst)
+            cap = new
+            assert len(where) <= cap and all(s < cap for s in where.values())
+            assert len(set(where.values())) == len(where)
+        layer = int(rng.integers(L))
+        req = rng.choice(E, k, replace=False).astype(np.int32)
+        s, m, ev = g.request(layer, req)
+        for e, slot, miss, vic in zip(req, s, m, ev):
+            key = layer * E + int(e)
+            assert miss == (key not in where)
+            if vic >= 0:
+                assert not (vic // E == layer and vic % E in req)
+                assert where.pop(int(vic)) == slot
+            where[key] = int(slot)
+        assert len(where) <= cap and all(sl < cap for sl in where.values())
+        assert len(set(where.values())) == len(where)
