@@ -80,6 +80,7 @@ struct DecArgs {
     const uint8_t *sh_gate, *sh_up, *sh_down;
     const void *x;
     int x_bf16;
+    int x_vec;                     // x is 16-byte aligned (vector loads)
     __half *Hs;                    // [T*k + T][hrow] fragment order
     int hrow;                      // halves per Hs row
     void *y;                       // [T, D] (combine mode)
@@ -426,40 +427,68 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     }
     // The activations do not depend on the routing kernel this grid may
     // overlap with: stage them (fp16, fragment order; row T is zero) and the
-    // per-block -off * sum(x) tables before waiting for it.
-    if (warp < kDW) {
-        for (int idx = tid; idx < (T + 1) * (nbD * 4); idx += kDW * 32) {
-            const int t = idx / (nbD * 4), rem = idx % (nbD * 4), b = rem >> 2, cc = rem & 3;
-            uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-            if (t < T) {
-                const size_t xb = (size_t)t * D + b * QK;
-                const int src[8] = {4 * cc, 4 * cc + 2, 4 * cc + 1, 4 * cc + 3,
-                                    16 + 4 * cc, 18 + 4 * cc, 17 + 4 * cc, 19 + 4 * cc};
-                uint32_t h[8];
+    // per-block -off * sum(x) tables before waiting for it.  One (token,
+    // block) of 32 values per thread, all of its loads in flight at once.
+    for (int idx = tid; idx < (T + 1) * nbD; idx += kGThreads) {
+        const int t = idx / nbD, b = idx % nbD;
+        float v[32];
+        if (t < T) {
+            const size_t xb = (size_t)t * D + b * QK;
+            if (a.x_vec && a.x_bf16) {
+                const uint4 *p = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)a.x + xb);
+                uint4 w[4];
+#pragma unroll
+                for (int q = 0; q < 4; q++) w[q] = __ldg(p + q);
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const uint32_t u[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
+#pragma unroll
+                    for (int r = 0; r < 4; r++) {
+                        v[8 * q + 2 * r] = __uint_as_float(u[r] << 16);
+                        v[8 * q + 2 * r + 1] = __uint_as_float(u[r] & 0xFFFF0000u);
+                    }
+                }
+            } else if (a.x_vec) {
+                const float4 *p = reinterpret_cast<const float4 *>((const float *)a.x + xb);
+                float4 w[8];
+#pragma unroll
+                for (int q = 0; q < 8; q++) w[q] = __ldg(p + q);
 #pragma unroll
                 for (int q = 0; q < 8; q++) {
-                    const float v = a.x_bf16 ? load_act((const __nv_bfloat16 *)a.x, xb + src[q])
-                                             : load_act((const float *)a.x, xb + src[q]);
-                    h[q] = (uint32_t)__half_as_ushort(__float2half_rn(v));
+                    v[4 * q] = w[q].x; v[4 * q + 1] = w[q].y; v[4 * q + 2] = w[q].z; v[4 * q + 3] = w[q].w;
                 }
-                pk.x = h[0] | (h[1] << 16);
-                pk.y = h[2] | (h[3] << 16);
-                pk.z = h[4] | (h[5] << 16);
-                pk.w = h[6] | (h[7] << 16);
-            }
-            *reinterpret_cast<uint4 *>(xs + (size_t)t * xrow + b * 64 + cc * 16) = pk;
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(kDW * 32));
-        for (int idx = tid; idx < (T + 1) * nbD; idx += kDW * 32) {
-            const int t = idx / nbD, b = idx % nbD;
-            const __half *hp = reinterpret_cast<const __half *>(xs + (size_t)t * xrow + b * 64);
-            float sum = 0.f;
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; i++) sum += __half2float(hp[i]);
-            sxt[idx] = -magic_off<false>() * sum;
-            sxt[(size_t)(T + 1) * nbD + idx] = -magic_off<true>() * sum;
+                for (int i = 0; i < 32; i++)
+                    v[i] = a.x_bf16 ? load_act((const __nv_bfloat16 *)a.x, xb + i)
+                                    : load_act((const float *)a.x, xb + i);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; i++) v[i] = 0.f;
         }
+        uint32_t h[32];
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            const __half hv = __float2half_rn(v[i]);
+            h[i] = (uint32_t)__half_as_ushort(hv);
+            sum += __half2float(hv);
+        }
+        uint8_t *dst = xs + (size_t)t * xrow + b * 64;
+#pragma unroll
+        for (int cc = 0; cc < 4; cc++) {
+            uint4 pk;
+            pk.x = h[4 * cc] | (h[4 * cc + 2] << 16);
+            pk.y = h[4 * cc + 1] | (h[4 * cc + 3] << 16);
+            pk.z = h[16 + 4 * cc] | (h[18 + 4 * cc] << 16);
+            pk.w = h[17 + 4 * cc] | (h[19 + 4 * cc] << 16);
+            *reinterpret_cast<uint4 *>(dst + cc * 16) = pk;
+        }
+        sxt[idx] = -magic_off<false>() * sum;
+        sxt[(size_t)(T + 1) * nbD + idx] = -magic_off<true>() * sum;
     }
+    __syncthreads();
     // routing results come from the previous kernel
     pdl_wait();
     pdl_launch_dependents();
@@ -1116,6 +1145,7 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
         a.sq8 = shared->qtype == MOE_Q8_0;
     }
     a.x = x; a.x_bf16 = (x_dtype == MOE_BF16);
+    a.x_vec = ((uintptr_t)x % 16) == 0;
     a.Hs = Hs; a.hrow = std::max(F, a.sF) + 32;
     a.y = y; a.y_dtype = y_dtype; a.rows_out = rows_out; a.err = err;
     a.inv = inv;
