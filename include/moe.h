@@ -357,12 +357,28 @@ moe_status moe_layer_forward(const moe_layer_args *args, void *workspace,
  * stream, after the copy stream has waited for the compute stream (so a
  * victim slot is never overwritten while a kernel may still read it).
  *
+ * Global mode (global = 1; FreeToken fork README, "About": global LRU
+ * expert caching, and "Elastic Memory Management": run-time re-allocation
+ * of the expert cache's VRAM; kongchang article, "Dynamic Cache Adjustment
+ * Experiments"): one pool of max_slots device slots shared by every layer,
+ * of which the first n_slots are in use (the capacity, changed at run time
+ * by moe_cache_resize).  One step counter serves every layer; an entry is
+ * (layer, expert), keyed layer * E + expert; a missing entry takes the
+ * empty slot of lowest index below the capacity, else evicts the entry with
+ * the oldest stamp in ANY layer that is not requested in the same call (the
+ * lower key on equal stamps).  A miss copy waits for the release point of
+ * the victim's layer.  A request may evict the experts of another layer, so
+ * enqueue a layer's FFN (and its release point) before requesting the next
+ * layer, and request a layer before each use of it (its slot map is written
+ * by its own requests only).
+ *
  * moe_cache_desc (all pools in the layout above; sizes in bytes):
  *   n_layers, E, n_slots, qtype
  *   bytes_gate, bytes_up, bytes_down   one expert's bytes of each matrix
  *   host_gate/up/down   host arrays of n_layers pointers, each to pinned
  *                       [E] experts (expert e at e * bytes_*)
- *   dev_gate/up/down    device [n_layers][n_slots] slots
+ *   dev_gate/up/down    device [n_layers][n_slots] slots; global mode:
+ *                       device [max_slots] slots
  *   dev_slot_map        device int32 [n_layers][E]; entries of experts that
  *                       are not resident hold -1
  *   copy_stream         stream for the host-to-device copies (not NULL)
@@ -373,6 +389,9 @@ moe_status moe_layer_forward(const moe_layer_args *args, void *workspace,
  *                       the expert_mask arguments of the two moe_layer_forward
  *                       calls that overlap the copies with the FFN of the
  *                       resident experts (see moe_layer_args)
+ *   global, max_slots   0: per-layer mode (max_slots unused); 1: global
+ *                       mode with max_slots >= n_slots pool slots
+ *                       (max_slots <= n_layers * E)
  * The cache keeps pointers to the caller's buffers; they must outlive it. */
 typedef struct moe_cache moe_cache;
 typedef struct {
@@ -387,6 +406,8 @@ typedef struct {
     int32_t *dev_slot_map;
     moe_stream copy_stream;
     uint8_t *dev_masks;
+    int32_t global;
+    int32_t max_slots;
 } moe_cache_desc;
 
 moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out);
@@ -395,9 +416,10 @@ void moe_cache_destroy(moe_cache *cache);
  * runs the LRU on the host, enqueues the copies of the misses on the copy
  * stream, records the layer's copy event, and enqueues on `compute` the
  * update of the layer's device slot map.  Optional host outputs per id:
- * slots[n], miss[n] (0/1), evicted[n] (expert evicted or -1).
- * MOE_ERR_CAPACITY if n > n_slots; MOE_ERR_INVALID_ARG on a bad or repeated
- * id.  The cache state is unchanged on error. */
+ * slots[n], miss[n] (0/1), evicted[n] (expert evicted, or in global mode
+ * its key layer * E + expert; -1 when none).
+ * MOE_ERR_CAPACITY if n > the capacity; MOE_ERR_INVALID_ARG on a bad or
+ * repeated id.  The cache state is unchanged on error. */
 moe_status moe_cache_request(moe_cache *cache, int layer, const int32_t *ids,
                              int n, int32_t *slots, int32_t *miss,
                              int32_t *evicted, int *n_miss, moe_stream compute);
@@ -412,8 +434,23 @@ moe_status moe_cache_sync(moe_cache *cache, int layer, moe_stream compute);
  * falls back to waiting for all of `compute`).  MOE_ERR_INVALID_ARG on a bad
  * cache or layer. */
 moe_status moe_cache_release(moe_cache *cache, int layer, moe_stream compute);
-/* The device pool view of one layer (slot-mapped). */
+/* The device pool view of one layer (slot-mapped; in global mode the whole
+ * shared pool, n_slots = max_slots). */
 moe_status moe_cache_layer_pool(moe_cache *cache, int layer, moe_pool *out);
+/* Global mode: change the capacity to n_slots (1 <= n_slots <= max_slots)
+ * at run time, without touching the host pools.  Growing adds empty slots.
+ * Shrinking evicts entries, oldest stamp first (lower key on ties), until
+ * at most n_slots are resident, then moves every entry held in a slot >=
+ * n_slots, in increasing slot order, to the empty slot of lowest index
+ * below n_slots: device-to-device copies on the copy stream after all work
+ * enqueued on `compute` so far; work enqueued on `compute` after the call
+ * runs once they are done, and from then on the slots [n_slots, max_slots)
+ * are unused (their memory may serve something else until the cache grows
+ * again).  Layers' slot maps are rewritten by their next requests.
+ * *n_evicted / *n_moved (may be NULL) receive the counts.
+ * MOE_ERR_INVALID_ARG for a per-layer cache, MOE_ERR_SHAPE out of range. */
+moe_status moe_cache_resize(moe_cache *cache, int n_slots, int *n_evicted, int *n_moved,
+                            moe_stream compute);
 /* Device addresses of one layer's hit and miss masks (dev_masks).  The
  * flow of one cached layer step, with the copies overlapping compute:
  *   moe_cache_request(c, l, ids, ...)

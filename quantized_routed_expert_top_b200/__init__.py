@@ -74,7 +74,7 @@ class CacheDesc(C.Structure):
                 ("host_up", C.POINTER(C.c_void_p)), ("host_down", C.POINTER(C.c_void_p)),
                 ("dev_gate", C.c_void_p), ("dev_up", C.c_void_p), ("dev_down", C.c_void_p),
                 ("dev_slot_map", C.c_void_p), ("copy_stream", C.c_void_p),
-                ("dev_masks", C.c_void_p)]
+                ("dev_masks", C.c_void_p), ("global_", C.c_int32), ("max_slots", C.c_int32)]
 
 
 _lib = None
@@ -113,6 +113,7 @@ def lib():
         L.moe_cache_release.argtypes = [_v, _i, _v]
         L.moe_cache_layer_pool.argtypes = [_v, _i, C.POINTER(Pool)]
         L.moe_cache_layer_masks.argtypes = [_v, _i, C.POINTER(_v), C.POINTER(_v)]
+        L.moe_cache_resize.argtypes = [_v, _i, C.POINTER(_i), C.POINTER(_i), _v]
         L.moe_cache_stats.argtypes = [_v, C.POINTER(C.c_int64), C.POINTER(C.c_int64),
                                       C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
         L.moe_route_noalloc.argtypes = [_v, C.c_int32, _v, _v, _i, _i, _i, _i, _i, _v, _v, _v,
@@ -381,10 +382,14 @@ class KernelTrace:
 
 # ----------------------------------------------------------- expert cache
 class ExpertCache:
-    """moe_cache over pinned host pools of n_layers layers (see moe.h)."""
+    """moe_cache over pinned host pools of n_layers layers (see moe.h).
+
+    ``global_slots=0``: per-layer mode, ``n_slots`` slots per layer.
+    ``global_slots=M``: global mode, one pool of M slots shared by every
+    layer with ``n_slots`` of them in use (``resize`` changes that)."""
 
     def __init__(self, host_gate, host_up, host_down, qtype, n_slots: int, copy_stream,
-                 device="cuda"):
+                 device="cuda", global_slots: int = 0):
         # host_* : lists (one per layer) of pinned uint8 tensors [E, rows, bytes]
         self.n_layers = len(host_gate)
         self.E = host_gate[0].shape[0]
@@ -398,12 +403,11 @@ class ExpertCache:
         bg, bu, bd = (lst[0][0].numel() for lst in self.host)
         self.bytes = (bg, bu, bd)
         dev = torch.device(device)
-        self.dev_gate = torch.empty((self.n_layers, n_slots) + tuple(host_gate[0].shape[1:]),
-                                    dtype=torch.uint8, device=dev)
-        self.dev_up = torch.empty((self.n_layers, n_slots) + tuple(host_up[0].shape[1:]),
-                                  dtype=torch.uint8, device=dev)
-        self.dev_down = torch.empty((self.n_layers, n_slots) + tuple(host_down[0].shape[1:]),
-                                    dtype=torch.uint8, device=dev)
+        self.global_slots = int(global_slots)
+        lead = (self.global_slots,) if self.global_slots else (self.n_layers, n_slots)
+        self.dev_gate = torch.empty(lead + tuple(host_gate[0].shape[1:]), dtype=torch.uint8, device=dev)
+        self.dev_up = torch.empty(lead + tuple(host_up[0].shape[1:]), dtype=torch.uint8, device=dev)
+        self.dev_down = torch.empty(lead + tuple(host_down[0].shape[1:]), dtype=torch.uint8, device=dev)
         self.slot_map = torch.full((self.n_layers, self.E), -1, dtype=torch.int32, device=dev)
         # per layer: [hit mask, miss mask] of the last request
         self.masks = torch.zeros((self.n_layers, 2, self.E), dtype=torch.uint8, device=dev)
@@ -421,6 +425,8 @@ class ExpertCache:
         d.dev_slot_map = self.slot_map.data_ptr()
         d.copy_stream = copy_stream.cuda_stream
         d.dev_masks = self.masks.data_ptr()
+        d.global_ = 1 if self.global_slots else 0
+        d.max_slots = self.global_slots
         self._desc = d
         h = C.c_void_p()
         _check(lib().moe_cache_init(C.byref(d), C.byref(h)))
@@ -430,7 +436,10 @@ class ExpertCache:
             p = Pool()
             _check(lib().moe_cache_layer_pool(self._h, l, C.byref(p)))
             ep = ExpertPool.__new__(ExpertPool)
-            ep.gate, ep.up, ep.down = self.dev_gate[l], self.dev_up[l], self.dev_down[l]
+            if self.global_slots:
+                ep.gate, ep.up, ep.down = self.dev_gate, self.dev_up, self.dev_down
+            else:
+                ep.gate, ep.up, ep.down = self.dev_gate[l], self.dev_up[l], self.dev_down[l]
             ep.qtype, ep.slot_of_expert, ep.c = self.qtype, self.slot_map[l], p
             self.pools.append(ep)
 
@@ -447,6 +456,12 @@ class ExpertCache:
         _check(lib().moe_cache_request(self._h, layer, f(ids), n, f(slots), f(miss), f(ev),
                                        C.byref(nm), _stream(stream)))
         return slots, miss.astype(bool), ev
+
+    def resize(self, n_slots: int, stream=None):
+        """Global mode: change the capacity at run time -> (evicted, moved)."""
+        ne, nm = C.c_int(0), C.c_int(0)
+        _check(lib().moe_cache_resize(self._h, int(n_slots), C.byref(ne), C.byref(nm), _stream(stream)))
+        return ne.value, nm.value
 
     def hit_mask(self, layer: int):
         """Device uint8 [E]: experts of the layer's last request already resident."""

@@ -50,6 +50,16 @@ struct moe_cache {
         int map_buf = 0;
     };
     std::vector<Layer> layers;
+    // global mode: one pool of max_slots slots shared by every layer, the
+    // first `cap` in use; entries keyed layer * E + expert; one step counter
+    bool global = false;
+    struct Glob {
+        int cap = 0;
+        int64_t step = 0;
+        std::vector<int32_t> slot_key;      // [max_slots] -1 empty
+        std::vector<int32_t> key_slot;      // [n_layers * E] -1 not resident
+        std::vector<int64_t> stamp;         // [n_layers * E]
+    } g;
     // pinned staging per (layer, buffer): the slot map (int32[E]), then the
     // request's hit and miss masks (uint8[E] each)
     uint8_t *pinned_stage = nullptr;
@@ -128,8 +138,14 @@ moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out) {
     if (!desc || !out) { set_error("moe_cache_init: NULL argument"); return MOE_ERR_INVALID_ARG; }
     *out = nullptr;
     const moe_cache_desc &d = *desc;
-    if (d.n_layers <= 0 || d.E <= 0 || d.E > MOE_MAX_EXPERTS || d.n_slots <= 0 || d.n_slots > d.E) {
+    if (d.global != 0 && d.global != 1) { set_error("moe_cache_init: global must be 0 or 1"); return MOE_ERR_INVALID_ARG; }
+    if (d.n_layers <= 0 || d.E <= 0 || d.E > MOE_MAX_EXPERTS || d.n_slots <= 0 ||
+        (!d.global && d.n_slots > d.E)) {
         set_error("moe_cache_init: need n_layers > 0, 0 < n_slots <= E <= %d", MOE_MAX_EXPERTS);
+        return MOE_ERR_SHAPE;
+    }
+    if (d.global && (d.max_slots < d.n_slots || (int64_t)d.max_slots > (int64_t)d.n_layers * d.E)) {
+        set_error("moe_cache_init: global cache needs n_slots <= max_slots <= n_layers * E");
         return MOE_ERR_SHAPE;
     }
     if (d.qtype != MOE_Q4_0 && d.qtype != MOE_Q8_0) {
@@ -150,6 +166,13 @@ moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out) {
     if (!c) { set_error("moe_cache_init: out of host memory"); return MOE_ERR_INVALID_ARG; }
     c->d = d;
     c->layers.resize(d.n_layers);
+    c->global = d.global != 0;
+    if (c->global) {
+        c->g.cap = d.n_slots;
+        c->g.slot_key.assign(d.max_slots, -1);
+        c->g.key_slot.assign((size_t)d.n_layers * d.E, -1);
+        c->g.stamp.assign((size_t)d.n_layers * d.E, 0);
+    }
     moe_status st = MOE_OK;
     c->stage_stride = round_up(sizeof(int32_t) * d.E + 2 * (size_t)d.E, 64);
     cudaError_t e = cudaHostAlloc((void **)&c->pinned_stage, c->stage_stride * d.n_layers * 2,
@@ -216,8 +239,9 @@ moe_status moe_cache_request(moe_cache *c, int layer, const int32_t *ids, int n,
     const moe_cache_desc &d = c->d;
     if (layer < 0 || layer >= d.n_layers) { set_error("moe_cache_request: layer %d out of range", layer); return MOE_ERR_INVALID_ARG; }
     if (n < 0) { set_error("moe_cache_request: n < 0"); return MOE_ERR_INVALID_ARG; }
-    if (n > d.n_slots) {
-        set_error("moe_cache_request: %d experts requested but the layer has %d slots", n, d.n_slots);
+    const int capacity = c->global ? c->g.cap : d.n_slots;
+    if (n > capacity) {
+        set_error("moe_cache_request: %d experts requested but the cache has %d slots", n, capacity);
         return MOE_ERR_CAPACITY;
     }
     auto &L = c->layers[layer];
@@ -235,50 +259,67 @@ moe_status moe_cache_request(moe_cache *c, int layer, const int32_t *ids, int n,
     if (st != MOE_OK) return st;
 
     // LRU decisions (committed below; on a copy failure the touched slots are
-    // invalidated so the resident set stays truthful)
-    const int64_t step = L.step + 1;
+    // invalidated so the resident set stays truthful).  Per-layer mode: the
+    // layer's own slots, keys = expert ids.  Global mode: the shared pool,
+    // keys = layer * E + expert, victims from any layer.
     std::vector<int> miss_idx;
     std::vector<int32_t> out_slot(n), out_ev(n, -1);
-    std::vector<int32_t> se = L.slot_expert, es = L.expert_slot;
-    std::vector<int64_t> stamp = L.stamp;
+    std::vector<char> victim_layer(d.n_layers, 0);     // layers whose slots the copies overwrite
+    const bool gm = c->global;
+    const int64_t step = gm ? c->g.step + 1 : L.step + 1;
+    std::vector<int32_t> se = gm ? c->g.slot_key : L.slot_expert;
+    std::vector<int32_t> es = gm ? c->g.key_slot : L.expert_slot;
+    std::vector<int64_t> stamp = gm ? c->g.stamp : L.stamp;
+    const int key0 = gm ? layer * d.E : 0;              // key of expert 0 of this layer
+    const int nkeys = gm ? d.n_layers * d.E : d.E;
     for (int i = 0; i < n; i++) {
-        const int e = ids[i];
-        if (es[e] >= 0) {
-            out_slot[i] = es[e];
+        const int key = key0 + ids[i];
+        if (es[key] >= 0) {
+            out_slot[i] = es[key];
         } else {
             int s = -1;
-            for (int q = 0; q < d.n_slots; q++) if (se[q] < 0) { s = q; break; }
+            for (int q = 0; q < capacity; q++) if (se[q] < 0) { s = q; break; }
             if (s < 0) {
                 int victim = -1;
-                for (int v = 0; v < d.E; v++) {
-                    if (es[v] < 0 || wanted[v]) continue;
+                for (int v = 0; v < nkeys; v++) {
+                    if (es[v] < 0 || (v >= key0 && v < key0 + d.E && wanted[v - key0])) continue;
                     if (victim < 0 || stamp[v] < stamp[victim]) victim = v;
                 }
                 s = es[victim];
                 es[victim] = -1;
                 out_ev[i] = victim;
+                victim_layer[gm ? victim / d.E : layer] = 1;
             }
-            se[s] = e;
-            es[e] = s;
+            se[s] = key;
+            es[key] = s;
             out_slot[i] = s;
             miss_idx.push_back(i);
         }
-        stamp[e] = step;
+        stamp[key] = step;
     }
 
-    // copies of the misses on the copy stream, after the compute stream
+    // copies of the misses on the copy stream, after the last use of the
+    // slots they overwrite: the release point of each victim's layer when it
+    // has one, else everything enqueued on the compute stream so far (empty
+    // slots were never read, or were vacated by a resize that waited)
     moe_status cst = MOE_OK;
     if (!miss_idx.empty()) {
-        if (L.released) {
-            cst = cuda_status(cudaStreamWaitEvent(xs, L.release_ev, 0), "cudaStreamWaitEvent");
-        } else {
+        bool need_all = !gm && !L.released;
+        for (int l = 0; l < d.n_layers && cst == MOE_OK; l++) {
+            if (!victim_layer[l] && !(l == layer && !gm)) continue;
+            if (c->layers[l].released)
+                cst = cuda_status(cudaStreamWaitEvent(xs, c->layers[l].release_ev, 0), "cudaStreamWaitEvent");
+            else
+                need_all = true;
+        }
+        if (cst == MOE_OK && need_all) {
             cst = cuda_status(cudaEventRecord(c->compute_ready, cs), "cudaEventRecord");
             if (cst == MOE_OK) cst = cuda_status(cudaStreamWaitEvent(xs, c->compute_ready, 0), "cudaStreamWaitEvent");
         }
         for (size_t m = 0; m < miss_idx.size() && cst == MOE_OK; m++) {
             const int i = miss_idx[m];
             const int e = ids[i];
-            const size_t slot = (size_t)layer * d.n_slots + out_slot[i];
+            const size_t slot = gm ? (size_t)out_slot[i] : (size_t)layer * d.n_slots + out_slot[i];
             struct { void *dst; const void *src; size_t n; } cp[3] = {
                 {(char *)d.dev_gate + slot * d.bytes_gate, (const char *)d.host_gate[layer] + (size_t)e * d.bytes_gate, d.bytes_gate},
                 {(char *)d.dev_up + slot * d.bytes_up, (const char *)d.host_up[layer] + (size_t)e * d.bytes_up, d.bytes_up},
@@ -305,21 +346,28 @@ moe_status moe_cache_request(moe_cache *c, int layer, const int32_t *ids, int n,
         for (int i : miss_idx) {
             const int s = out_slot[i];
             se[s] = -1;
-            es[ids[i]] = -1;
+            es[key0 + ids[i]] = -1;
         }
         // keep the old recency of experts that were not served
-        stamp = L.stamp;
+        stamp = gm ? c->g.stamp : L.stamp;
     }
-    L.slot_expert.swap(se);
-    L.expert_slot.swap(es);
-    L.stamp.swap(stamp);
-    L.step = step;
+    if (gm) {
+        c->g.slot_key.swap(se);
+        c->g.key_slot.swap(es);
+        c->g.stamp.swap(stamp);
+        c->g.step = step;
+    } else {
+        L.slot_expert.swap(se);
+        L.expert_slot.swap(es);
+        L.stamp.swap(stamp);
+        L.step = step;
+    }
     L.pending = L.pending || (!miss_idx.empty() && cst == MOE_OK);
     L.released = false;                   // the release point covered the previous request only
 
     // device slot map of the layer (and the request's hit / miss masks)
     int32_t *hm = c->stage_map(layer, buf);
-    for (int e = 0; e < d.E; e++) hm[e] = L.expert_slot[e];
+    for (int e = 0; e < d.E; e++) hm[e] = gm ? c->g.key_slot[key0 + e] : L.expert_slot[e];
     moe_status mst = cuda_status(cudaMemcpyAsync(d.dev_slot_map + (size_t)layer * d.E, hm,
                                                  sizeof(int32_t) * d.E, cudaMemcpyHostToDevice, cs),
                                  "moe_cache_request: slot map copy");
@@ -330,7 +378,7 @@ moe_status moe_cache_request(moe_cache *c, int layer, const int32_t *ids, int n,
         if (cst == MOE_OK) for (int i : miss_idx) missed[i] = 1;
         for (int i = 0; i < n; i++) {
             if (missed[i]) mis[ids[i]] = 1;
-            else if (L.expert_slot[ids[i]] >= 0) hit[ids[i]] = 1;
+            else if (hm[ids[i]] >= 0) hit[ids[i]] = 1;
         }
         mst = cuda_status(cudaMemcpyAsync(d.dev_masks + (size_t)layer * 2 * d.E, hit, 2 * (size_t)d.E,
                                           cudaMemcpyHostToDevice, cs),
@@ -401,14 +449,77 @@ moe_status moe_cache_layer_masks(moe_cache *c, int layer, const uint8_t **hit,
 moe_status moe_cache_layer_pool(moe_cache *c, int layer, moe_pool *out) {
     if (!c || !out || layer < 0 || layer >= c->d.n_layers) { set_error("moe_cache_layer_pool: bad argument"); return MOE_ERR_INVALID_ARG; }
     const moe_cache_desc &d = c->d;
-    const size_t base = (size_t)layer * d.n_slots;
+    const size_t base = c->global ? 0 : (size_t)layer * d.n_slots;
     out->qtype = d.qtype;
-    out->n_slots = d.n_slots;
+    out->n_slots = c->global ? d.max_slots : d.n_slots;
     out->gate = (const char *)d.dev_gate + base * d.bytes_gate;
     out->up = (const char *)d.dev_up + base * d.bytes_up;
     out->down = (const char *)d.dev_down + base * d.bytes_down;
     out->slot_of_expert = d.dev_slot_map + (size_t)layer * d.E;
     return MOE_OK;
+}
+
+moe_status moe_cache_resize(moe_cache *c, int n_slots, int *n_evicted, int *n_moved,
+                            moe_stream compute) {
+    if (n_evicted) *n_evicted = 0;
+    if (n_moved) *n_moved = 0;
+    if (!c || !c->global) { set_error("moe_cache_resize: needs a global cache"); return MOE_ERR_INVALID_ARG; }
+    const moe_cache_desc &d = c->d;
+    if (n_slots < 1 || n_slots > d.max_slots) {
+        set_error("moe_cache_resize: %d slots outside [1, %d]", n_slots, d.max_slots);
+        return MOE_ERR_SHAPE;
+    }
+    auto &G = c->g;
+    if (n_slots >= G.cap) {                 // growing only adds empty slots
+        G.cap = n_slots;
+        return MOE_OK;
+    }
+    cudaStream_t cs = (cudaStream_t)compute, xs = (cudaStream_t)d.copy_stream;
+    // the moves below overwrite slots that kernels enqueued so far may still
+    // read (entries just evicted): the copy stream waits for all of them
+    moe_status st = cuda_status(cudaEventRecord(c->compute_ready, cs), "cudaEventRecord");
+    if (st == MOE_OK) st = cuda_status(cudaStreamWaitEvent(xs, c->compute_ready, 0), "cudaStreamWaitEvent");
+    if (st != MOE_OK) return st;
+    int resident = 0;
+    for (int s = 0; s < G.cap; s++) if (G.slot_key[s] >= 0) resident++;
+    const int nk = d.n_layers * d.E;
+    int ne = 0, nm = 0;
+    while (resident > n_slots) {            // oldest stamp first, lower key on ties
+        int victim = -1;
+        for (int k = 0; k < nk; k++) {
+            if (G.key_slot[k] < 0) continue;
+            if (victim < 0 || G.stamp[k] < G.stamp[victim]) victim = k;
+        }
+        G.slot_key[G.key_slot[victim]] = -1;
+        G.key_slot[victim] = -1;
+        resident--;
+        ne++;
+    }
+    for (int s = n_slots; s < G.cap && st == MOE_OK; s++) {   // compact into the first n_slots
+        const int key = G.slot_key[s];
+        if (key < 0) continue;
+        int t = 0;
+        while (G.slot_key[t] >= 0) t++;
+        const void *src[3] = {(char *)d.dev_gate + (size_t)s * d.bytes_gate, (char *)d.dev_up + (size_t)s * d.bytes_up,
+                              (char *)d.dev_down + (size_t)s * d.bytes_down};
+        void *dst[3] = {(char *)d.dev_gate + (size_t)t * d.bytes_gate, (char *)d.dev_up + (size_t)t * d.bytes_up,
+                        (char *)d.dev_down + (size_t)t * d.bytes_down};
+        const size_t nb[3] = {d.bytes_gate, d.bytes_up, d.bytes_down};
+        for (int q = 0; q < 3 && st == MOE_OK; q++)
+            st = cuda_status(cudaMemcpyAsync(dst[q], src[q], nb[q], cudaMemcpyDeviceToDevice, xs),
+                             "moe_cache_resize: move");
+        G.slot_key[t] = key;
+        G.slot_key[s] = -1;
+        G.key_slot[key] = t;
+        nm++;
+    }
+    // work enqueued on the compute stream after this call sees the moves done
+    if (st == MOE_OK) st = cuda_status(cudaEventRecord(c->compute_ready, xs), "cudaEventRecord");
+    if (st == MOE_OK) st = cuda_status(cudaStreamWaitEvent(cs, c->compute_ready, 0), "cudaStreamWaitEvent");
+    G.cap = n_slots;
+    if (n_evicted) *n_evicted = ne;
+    if (n_moved) *n_moved = nm;
+    return st;
 }
 
 moe_status moe_cache_stats(moe_cache *c, int64_t *hits, int64_t *misses, int64_t *bytes_copied,

@@ -192,3 +192,20 @@ def test_device_status_codes_agree_with_header(moe):
     assert ph == {"MOE_PHASE_ROUTE": moe.PHASE_ROUTE, "MOE_PHASE_FFN": moe.PHASE_FFN,
                   "MOE_PHASE_SHARED": moe.PHASE_SHARED, "MOE_PHASE_COMBINE": moe.PHASE_COMBINE,
                   "MOE_PHASE_ALL": moe.PHASE_ALL}
+
+
+def test_global_cache_arguments(moe):
+    L = moe.lib()
+    h = C.c_void_p()
+    d = moe.CacheDesc()
+    d.n_layers, d.E, d.n_slots, d.qtype = 2, 8, 6, moe.Q8_0
+    d.global_, d.max_slots = 1, 4                     # capacity above the pool
+    assert L.moe_cache_init(C.byref(d), C.byref(h)) == 3
+    d.max_slots = 17                                  # more than n_layers * E
+    assert L.moe_cache_init(C.byref(d), C.byref(h)) == 3
+    d.global_ = 2
+    assert L.moe_cache_init(C.byref(d), C.byref(h)) == 1
+    assert not h.value
+    ne, nm = C.c_int(-1), C.c_int(-1)
+    assert L.moe_cache_resize(None, 4, C.byref(ne), C.byref(nm), None) == 1
+    assert ne.value == 0 and nm.value == 0

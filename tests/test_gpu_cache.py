@@ -263,3 +263,66 @@ def test_cache_at_the_full_layer_shape_matches_the_oracle(moe):
         assert err <= 2e-3, (t, err)
     assert moe.workspace_status(lay.ws) == (0, moe.DEV_OK)
     cache.close()
+
+
+# ------------------------------------------------- global LRU with resizing
+def _global_cache(moe, pools, stream, cap, max_slots):
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    return moe.ExpertCache([pin(p[0]) for p in pools], [pin(p[1]) for p in pools],
+                           [pin(p[2]) for p in pools], "q8_0", cap, stream,
+                           global_slots=max_slots)
+
+
+RESIZES = {9: 6, 19: 14, 27: 5}      # step -> new capacity (shrink, grow, shrink)
+
+
+def test_global_cache_sequence_matches_simulation(moe, stack):
+    # every request's (slot, miss, evicted key) and every resize's eviction
+    # and move counts equal the oracle's global LRU simulation
+    pools, traces, _ = stack
+    cache = _global_cache(moe, pools, torch.cuda.Stream(), 10, 16)
+    sim = oracle.GlobalLRU(N_LAYERS, E, 16, 10)
+    cross = 0
+    for t in range(STEPS):
+        if t in RESIZES:
+            ne, nm = cache.resize(RESIZES[t])
+            ev, mv = sim.resize(RESIZES[t])
+            assert (ne, nm) == (len(ev), len(mv)), t
+        for l in range(N_LAYERS):
+            ids = _ids(traces[l][t])
+            got = cache.request(l, ids)
+            want = sim.request(l, ids)
+            for g, w in zip(got, want):
+                assert np.array_equal(np.asarray(g), np.asarray(w)), (t, l, got, want)
+            cross += int(np.sum((want[2] >= 0) & (want[2] // E != l)))
+    torch.cuda.synchronize()
+    assert cross > 0                  # some victims came from other layers
+    cache.close()
+
+
+def test_global_cached_layers_are_bit_identical_to_resident(moe, stack):
+    # two-phase layer calls through the shared pool, with the capacity
+    # shrunk (evictions and moves inside the pool) and grown on the way
+    pools, traces, x = stack
+    stream = torch.cuda.current_stream()
+    cache = _global_cache(moe, pools, torch.cuda.Stream(), 10, 16)
+    xd = torch.from_numpy(x.x_raw.view(np.int16)).cuda().view(torch.bfloat16)
+    resident = [moe.Layer(moe.ExpertPool.from_numpy(*p, "q8_0"), D, F, E, K, 1,
+                          y_dtype=torch.float32) for p in pools]
+    cached = [moe.Layer(cache.pools[l], D, F, E, K, 1, y_dtype=torch.float32)
+              for l in range(N_LAYERS)]
+    moved = 0
+    for t in range(STEPS):
+        if t in RESIZES:
+            moved += cache.resize(RESIZES[t], stream=stream)[1]
+        for l in range(N_LAYERS):
+            lg = torch.from_numpy(traces[l][t:t + 1]).cuda()
+            y_c = torch.full((1, D), float("nan"), device="cuda")
+            _two_phase(moe, cache, cached[l], l, _ids(traces[l][t]), xd[t:t + 1], lg, y_c, stream)
+            cache.release(l, stream=stream)
+            y_r = resident[l].forward(xd[t:t + 1], logits=lg).clone()
+            torch.cuda.synchronize()
+            assert torch.equal(y_c, y_r), (t, l)
+            assert moe.workspace_status(cached[l].ws) == (0, moe.DEV_OK)
+    assert moved > 0
+    cache.close()
