@@ -23,8 +23,10 @@ One JSON line on rank 0.  Workloads (seeded synthetic inputs, see synthetic/):
   fully resident.
 
 The default run (decode) prints the decode line with every other
-configuration under "configs" (tiny, prefill, wide_t1, wide_t2048, cache),
-each with its own roofline, end-to-end number and oracle baseline.
+configuration under "configs" (tiny, prefill, wide_t1, wide_t2048,
+prefill_stream, cache), each with its own roofline, end-to-end number and
+oracle baseline.  prefill_stream: the prefill layer stacked 8 deep with its
+experts in pinned host memory, whole layers double-buffered into HBM.
 
 Timing: W untimed steps, then K steps bracketed by a barrier and a device
 synchronize, timed with CUDA events on the launching stream; max over
@@ -838,6 +840,126 @@ def measure_cache(args, steps, warmup, world, local, peaks, cpu=True):
     return out
 
 
+# --------------------------------------------------- streamed prefill arm
+STREAM_LAYERS = 8
+
+
+def measure_prefill_stream(torch, moe, base, steps, warmup, peaks, cpu=True):
+    """The prefill layer (T=8192, Q8_0) stacked STREAM_LAYERS deep with every
+    layer's experts in pinned host memory, streamed a whole layer at a time
+    into two device buffers while the previous layer computes."""
+    cfg = base.cfg
+    gb, ub, db = S.expert_bytes(cfg.D, cfg.F, cfg.qtype)
+    layer_bytes = cfg.E * (gb + ub + db)
+    ram = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES")
+    n_layers = max(2, min(STREAM_LAYERS, int(0.3 * ram // layer_bytes)))
+    pin = lambda a: torch.empty(a.shape, dtype=torch.uint8, pin_memory=True).copy_(torch.from_numpy(a))
+    # one drawn pool's bytes for every layer (the copy and kernel costs do not
+    # depend on the values)
+    host = [[pin(a) for _ in range(n_layers)] for a in (base.gate, base.up, base.down)]
+    st = moe.LayerStreamer(*host, cfg.qtype, torch.cuda.Stream())
+    dev = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    T = base.x.shape[0]
+    lay = moe.Layer(moe.ExpertPool(dev(base.gate), dev(base.up), dev(base.down), cfg.qtype),
+                    cfg.D, cfg.F, cfg.E, cfg.k, T, w_router=dev(base.w_router), bias=dev(base.bias))
+    resident_pool = lay.pool
+    x0 = _dev_x(base, torch)
+    x = x0.clone()
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+
+    def stack_pass(streamed):
+        if streamed:
+            st.prefetch(0)
+            st.prefetch(1)
+        for l in range(n_layers):
+            lay.pool = st.acquire(l, stream=stream) if streamed else resident_pool
+            lay.forward(x, out=y)
+            if streamed:
+                st.release(l, stream=stream)
+                if l + 2 < n_layers:
+                    st.prefetch(l + 2)
+            x.add_(y)
+
+    def timed(streamed, n):
+        x.copy_(x0)
+        torch.cuda.synchronize()
+        b0, e0n = st.stats()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            stack_pass(streamed)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        b1, e1n = st.stats()
+        return e0.elapsed_time(e1), b1 - b0, e1n - e0n
+
+    passes = max(1, min(steps, 3))
+    tr = moe.KernelTrace(n_calls=1)
+    lay.forward(x0, out=y, trace=tr)
+    torch.cuda.synchronize()
+    kpl = len(tr.calls[0])                # kernels per layer call
+    timed(True, 1)
+    with ClockSampler(0, period_s=0.002) as clk:
+        ms, nbytes, exp_ns = timed(True, passes)
+    timed(False, 1)
+    ms_res, _, _ = timed(False, passes)
+    pcie = h2d_probe(torch)
+    # end to end: the prompt's activations from pinned host memory, the last
+    # layer's output back to pinned host memory, inside the timed region
+    xh = x0.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(passes):
+        x.copy_(xh, non_blocking=True)
+        stack_pass(True)
+        yh.copy_(x, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    tok = T * n_layers * passes
+    out = {
+        "value": round(tok / (ms / 1e3), 1), "unit": "tokens/s",
+        "ms_per_step": round(ms / passes / n_layers, 4),
+        "config": {"workload": f"prefill_stream: the prefill layer (T={T}, D={cfg.D}, E={cfg.E}, "
+                               f"top-{cfg.k}, F={cfg.F}, {cfg.qtype.upper()}) stacked {n_layers} deep, "
+                               f"every layer's {layer_bytes / 1e6:.0f} MB of experts in pinned host "
+                               f"memory, copied a whole layer at a time into two device buffers "
+                               f"while the previous layer computes; tokens/s per layer",
+                   "layers": n_layers, "passes": passes},
+        "roofline": {"kernel": "layer copies (host to device)", "bound": "pcie",
+                     "achieved": round(nbytes / (ms / 1e3) / 1e9, 2), "peak": round(pcie, 2),
+                     "unit": "GB/s", "frac": round(nbytes / (ms / 1e3) / 1e9 / pcie, 4),
+                     "peak_source": "pinned 1 GiB host-to-device copy measured in this run",
+                     "traffic": None},
+        "exposed_copy_ms_per_layer": round(exp_ns / 1e6 / passes / n_layers, 4),
+        "resident_ms_per_layer": round(ms_res / passes / n_layers, 4),
+        "resident_tokens_per_s": round(tok / (ms_res / 1e3), 1),
+        "gpu_launches": kpl * n_layers * passes,
+        "e2e": {"value": round(tok / (ms_e2e / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+                "d2h_bytes_per_step": yh.numel() * yh.element_size()},
+        "clocks": clk.summary(),
+    }
+    if cpu:
+        import oracle
+        oracle.build()
+        t0 = time.perf_counter()
+        m = 16
+        _, ids, g = oracle.route(base.x[:m], base.w_router, base.bias, cfg.k, cfg.renorm)
+        oracle.layer(base.x[:m], ids, g, base.gate, base.up, base.down, cfg.qtype, cfg.F)
+        dt = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": round(m / dt, 4), "unit": "tokens/s",
+                               "cores": os.cpu_count() or 1, "kind": "oracle",
+                               "sample": f"{m} tokens through one layer (route + layer, fp64; the "
+                                         f"oracle reads host memory, no streaming), {dt:.1f} s"}
+    st.close()
+    del host
+    return out
+
+
 def _line(out, args, world, cfg, peaks):
     line = {"metric": "MoE-layer tokens/s", "value": out["value"], "unit": out["unit"],
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -892,6 +1014,9 @@ def run_ours(args, world, rank, local):
                                                  args.no_graph, cpu=with_cpu, cpu_seconds=6.0)
             del w
             torch.cuda.empty_cache()
+        line["configs"]["prefill_stream"] = measure_prefill_stream(
+            torch, moe, bases["prefill"], args.steps, args.warmup, peaks, cpu=with_cpu)
+        torch.cuda.empty_cache()
         line["configs"]["cache"] = measure_cache(args, max(5, min(args.steps, 16)), args.warmup,
                                                  world, local, peaks, cpu=with_cpu)
     if rank == 0:

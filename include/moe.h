@@ -470,6 +470,54 @@ moe_status moe_cache_layer_masks(moe_cache *cache, int layer, const uint8_t **hi
 moe_status moe_cache_stats(moe_cache *cache, int64_t *hits, int64_t *misses,
                            int64_t *bytes_copied, int64_t *exposed_ns);
 
+/* --------------------------------------------- prefill layer streaming
+ * Full-layer double-buffered streaming of expert weights (FreeToken fork
+ * README, "About": full-layer double-buffered prefill streaming; kongchang
+ * article, "Dual-Buffering to Solve the Prefill Bottleneck").  A long prompt
+ * reaches nearly every expert of every layer, so whole layers move: two
+ * device buffers, each one layer's [E] experts in the pool layout; layer l
+ * uses buffer l % 2 while the copy stream fills the other with the next
+ * layer.  One stack pass:
+ *   moe_streamer_prefetch(s, 0); moe_streamer_prefetch(s, 1);
+ *   for each layer l:
+ *     moe_streamer_acquire(s, l, compute, &pool)   compute waits for l's copy
+ *     moe_layer_forward(... pool ...)               on compute
+ *     moe_streamer_release(s, l, compute)           l's kernels are enqueued
+ *     moe_streamer_prefetch(s, l + 2)               waits for that release
+ * moe_streamer_desc:
+ *   n_layers, E, qtype; bytes_gate/up/down   one expert's bytes
+ *   host_gate/up/down   host arrays of n_layers pointers to pinned [E] experts
+ *   dev_gate/up/down    two device buffers of [E] experts each
+ *   copy_stream         stream for the host-to-device copies (not NULL)
+ * The streamer keeps pointers to the caller's buffers; they must outlive it. */
+typedef struct moe_streamer moe_streamer;
+typedef struct {
+    int32_t n_layers, E, qtype, reserved;
+    size_t bytes_gate, bytes_up, bytes_down;
+    const void *const *host_gate;
+    const void *const *host_up;
+    const void *const *host_down;
+    void *dev_gate[2];
+    void *dev_up[2];
+    void *dev_down[2];
+    moe_stream copy_stream;
+} moe_streamer_desc;
+
+moe_status moe_streamer_init(const moe_streamer_desc *desc, moe_streamer **out);
+void moe_streamer_destroy(moe_streamer *s);
+/* Enqueue the copy of `layer` into buffer layer % 2 on the copy stream,
+ * after the release point of the layer that used that buffer last (a no-op
+ * if the buffer already holds `layer`). */
+moe_status moe_streamer_prefetch(moe_streamer *s, int layer);
+/* Make `compute` wait for `layer`'s copy (prefetching it first if needed)
+ * and return the pool view of its buffer (n_slots = E, no slot map). */
+moe_status moe_streamer_acquire(moe_streamer *s, int layer, moe_stream compute, moe_pool *out);
+/* Every kernel that reads `layer`'s buffer is enqueued on `compute`. */
+moe_status moe_streamer_release(moe_streamer *s, int layer, moe_stream compute);
+/* Bytes copied, and the time `compute` has waited in acquire for copies
+ * (events around each wait; waits for the pending ones). */
+moe_status moe_streamer_stats(moe_streamer *s, int64_t *bytes_copied, int64_t *exposed_ns);
+
 #ifdef __cplusplus
 }
 #endif

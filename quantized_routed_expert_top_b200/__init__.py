@@ -77,6 +77,15 @@ class CacheDesc(C.Structure):
                 ("dev_masks", C.c_void_p), ("global_", C.c_int32), ("max_slots", C.c_int32)]
 
 
+class StreamerDesc(C.Structure):
+    _fields_ = [("n_layers", C.c_int32), ("E", C.c_int32), ("qtype", C.c_int32),
+                ("reserved", C.c_int32), ("bytes_gate", C.c_size_t), ("bytes_up", C.c_size_t),
+                ("bytes_down", C.c_size_t), ("host_gate", C.POINTER(C.c_void_p)),
+                ("host_up", C.POINTER(C.c_void_p)), ("host_down", C.POINTER(C.c_void_p)),
+                ("dev_gate", C.c_void_p * 2), ("dev_up", C.c_void_p * 2),
+                ("dev_down", C.c_void_p * 2), ("copy_stream", C.c_void_p)]
+
+
 _lib = None
 _v, _i, _sz = C.c_void_p, C.c_int, C.c_size_t
 
@@ -118,6 +127,13 @@ def lib():
                                       C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
         L.moe_route_noalloc.argtypes = [_v, C.c_int32, _v, _v, _i, _i, _i, _i, _i, _v, _v, _v,
                                         _v]
+        L.moe_streamer_init.argtypes = [C.POINTER(StreamerDesc), C.POINTER(_v)]
+        L.moe_streamer_destroy.argtypes = [_v]
+        L.moe_streamer_destroy.restype = None
+        L.moe_streamer_prefetch.argtypes = [_v, _i]
+        L.moe_streamer_acquire.argtypes = [_v, _i, _v, C.POINTER(Pool)]
+        L.moe_streamer_release.argtypes = [_v, _i, _v]
+        L.moe_streamer_stats.argtypes = [_v, C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
         L.moe_cache_debug_fail_copy.argtypes = [_v, _i]
         L.moe_cache_debug_fail_copy.restype = None
         _lib = L
@@ -497,6 +513,77 @@ class ExpertCache:
     def close(self):
         if getattr(self, "_h", None):
             lib().moe_cache_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# -------------------------------------------------- prefill layer streaming
+class LayerStreamer:
+    """moe_streamer: whole layers of experts double-buffered from pinned host
+    memory (see moe.h).  host_* are lists (one per layer) of pinned uint8
+    tensors [E, rows, bytes]; two device buffers of one layer each are
+    allocated here."""
+
+    def __init__(self, host_gate, host_up, host_down, qtype, copy_stream, device="cuda"):
+        self.n_layers = len(host_gate)
+        self.E = host_gate[0].shape[0]
+        self.qtype = _qt(qtype)
+        self.host = (host_gate, host_up, host_down)
+        for lst in self.host:
+            for t in lst:
+                if t.is_cuda or not t.is_pinned():
+                    raise ValueError("host pools must be pinned host tensors")
+        dev = torch.device(device)
+        self.bufs = [[torch.empty(lst[0].shape, dtype=torch.uint8, device=dev) for lst in self.host]
+                     for _ in range(2)]
+        arr = lambda lst: (C.c_void_p * self.n_layers)(*[t.data_ptr() for t in lst])
+        self._ptrs = [arr(l) for l in self.host]
+        d = StreamerDesc()
+        d.n_layers, d.E, d.qtype = self.n_layers, self.E, self.qtype
+        d.bytes_gate, d.bytes_up, d.bytes_down = (lst[0][0].numel() for lst in self.host)
+        d.host_gate = C.cast(self._ptrs[0], C.POINTER(C.c_void_p))
+        d.host_up = C.cast(self._ptrs[1], C.POINTER(C.c_void_p))
+        d.host_down = C.cast(self._ptrs[2], C.POINTER(C.c_void_p))
+        for b in range(2):
+            d.dev_gate[b], d.dev_up[b], d.dev_down[b] = (t.data_ptr() for t in self.bufs[b])
+        d.copy_stream = copy_stream.cuda_stream
+        self.copy_stream = copy_stream
+        self._desc = d
+        h = C.c_void_p()
+        _check(lib().moe_streamer_init(C.byref(d), C.byref(h)))
+        self._h = h
+        self._pools = [None, None]
+
+    def prefetch(self, layer: int):
+        _check(lib().moe_streamer_prefetch(self._h, layer))
+
+    def acquire(self, layer: int, stream=None) -> ExpertPool:
+        """The layer's pool view (valid for work enqueued on ``stream`` after this)."""
+        p = Pool()
+        _check(lib().moe_streamer_acquire(self._h, layer, _stream(stream), C.byref(p)))
+        ep = ExpertPool.__new__(ExpertPool)
+        b = self.bufs[layer & 1]
+        ep.gate, ep.up, ep.down = b
+        ep.qtype, ep.slot_of_expert, ep.c = self.qtype, None, p
+        return ep
+
+    def release(self, layer: int, stream=None):
+        _check(lib().moe_streamer_release(self._h, layer, _stream(stream)))
+
+    def stats(self):
+        """(bytes copied, exposed ns)."""
+        b, e = C.c_int64(), C.c_int64()
+        _check(lib().moe_streamer_stats(self._h, C.byref(b), C.byref(e)))
+        return b.value, e.value
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().moe_streamer_destroy(self._h)
             self._h = None
 
     def __del__(self):

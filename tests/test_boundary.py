@@ -209,3 +209,19 @@ def test_global_cache_arguments(moe):
     ne, nm = C.c_int(-1), C.c_int(-1)
     assert L.moe_cache_resize(None, 4, C.byref(ne), C.byref(nm), None) == 1
     assert ne.value == 0 and nm.value == 0
+
+
+def test_streamer_arguments(moe):
+    L = moe.lib()
+    h = C.c_void_p()
+    assert L.moe_streamer_init(None, C.byref(h)) == 1
+    d = moe.StreamerDesc()
+    d.n_layers, d.E, d.qtype = 2, 8, 3                 # unknown quant type
+    assert L.moe_streamer_init(C.byref(d), C.byref(h)) == 2
+    d.qtype = moe.Q8_0
+    assert L.moe_streamer_init(C.byref(d), C.byref(h)) == 1   # NULL pools
+    d.n_layers = 0
+    assert L.moe_streamer_init(C.byref(d), C.byref(h)) == 3
+    assert not h.value
+    assert L.moe_streamer_prefetch(None, 0) == 1
+    assert L.moe_streamer_stats(None, None, None) == 1
