@@ -21,8 +21,11 @@ _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 Q4_0 = 2
+Q4_1 = 3
+Q5_0 = 6
+Q5_1 = 7
 Q8_0 = 8
-QTYPE = {"q4_0": Q4_0, "q8_0": Q8_0}
+QTYPE = {"q4_0": Q4_0, "q4_1": Q4_1, "q5_0": Q5_0, "q5_1": Q5_1, "q8_0": Q8_0}
 
 
 def build(force: bool = False) -> str:
@@ -155,11 +158,12 @@ def permute(ids, E: int):
 
 
 def layer(x, ids, gates, gate, up, down, qtype, F: int, shared=None,
-          tokens=None, dense: bool = False, threads: int = 0) -> np.ndarray:
+          tokens=None, dense: bool = False, threads: int = 0,
+          shared_qtype="q8_0") -> np.ndarray:
     """y [n_tok, D] (float64) of the routed layer for the listed tokens.
 
     ``gate/up/down``: pools [E, rows, bytes]; ``shared``: optional
-    (gate, up, down) of one Q8_0 expert with its own F.
+    (gate, up, down) of one expert in ``shared_qtype`` with its own F.
     """
     x = _c(x, np.float32)
     T, D = x.shape
@@ -178,7 +182,7 @@ def layer(x, ids, gates, gate, up, down, qtype, F: int, shared=None,
     y = np.empty((n, D), np.float64)
     rc = lib().orc_layer(_ptr(x), T, D, F, E, k, _qt(qtype), _ptr(gate), _ptr(up),
                          _ptr(down), _ptr(ids), _ptr(gates), _ptr(sg), _ptr(su),
-                         _ptr(sd), sF, Q8_0, _ptr(tl), n, int(dense), threads, _ptr(y))
+                         _ptr(sd), sF, _qt(shared_qtype), _ptr(tl), n, int(dense), threads, _ptr(y))
     if rc != 0:
         raise ValueError("oracle layer: bad arguments")
     return y

@@ -9,11 +9,17 @@
  * What it computes (all floating point in double unless stated):
  *
  *   Block formats -- FreeToken fork README, "Quant types" table (Standard
- *   family: Q4_0, Q8_0).  32 weights per block, one fp16 scale d:
- *     Q8_0 {fp16 d; int8 q[32]}           value q[i] * d
- *     Q4_0 {fp16 d; uint8 qs[16]}         value (q[i] - 8) * d, byte j holds
- *                                         element j (low nibble) and j+16
- *                                         (high nibble)
+ *   family: Q4_0, Q4_1, Q5_0, Q5_1, Q8_0; the page names the types, the byte
+ *   layouts are ggml's published ones).  32 weights per block, fp16 scale d
+ *   (and fp16 minimum m for the _1 types), all little endian:
+ *     Q8_0 {fp16 d; int8 q[32]}                  value q[i] * d
+ *     Q4_0 {fp16 d; uint8 qs[16]}                value (q[i] - 8) * d
+ *     Q4_1 {fp16 d; fp16 m; uint8 qs[16]}        value q[i] * d + m
+ *     Q5_0 {fp16 d; uint8 qh[4]; uint8 qs[16]}   value (q[i] - 16) * d
+ *     Q5_1 {fp16 d; fp16 m; uint8 qh[4]; uint8 qs[16]}   value q[i] * d + m
+ *   qs byte j holds the low 4 bits of element j (low nibble) and of element
+ *   j+16 (high nibble); for the 5-bit types bit i of the 32-bit word qh is
+ *   bit 4 of element i.
  *   Expert pool layout -- FreeToken fork README, "Known limits": experts back
  *   to back, expert * nrows * (ncols / 32) blocks, no padding, one type.
  *   Per expert: W_gate, W_up are [F rows][D/32 blocks], W_down [D][F/32].
@@ -50,6 +56,9 @@
 
 #define ORC_QK 32
 #define ORC_Q4_0 2
+#define ORC_Q4_1 3
+#define ORC_Q5_0 6
+#define ORC_Q5_1 7
 #define ORC_Q8_0 8
 
 /* IEEE 754 binary16 -> double, decoded bit by bit (sign, 5-bit exponent with
@@ -71,9 +80,19 @@ double orc_half_to_double(uint16_t h)
 
 int orc_block_bytes(int qtype)
 {
-    if (qtype == ORC_Q8_0) return 2 + 32;
-    if (qtype == ORC_Q4_0) return 2 + 16;
-    return 0;
+    switch (qtype) {
+    case ORC_Q8_0: return 2 + 32;
+    case ORC_Q4_0: return 2 + 16;
+    case ORC_Q4_1: return 2 + 2 + 16;
+    case ORC_Q5_0: return 2 + 4 + 16;
+    case ORC_Q5_1: return 2 + 2 + 4 + 16;
+    default: return 0;
+    }
+}
+
+static double orc_half_at(const uint8_t *p)
+{
+    return orc_half_to_double((uint16_t)(p[0] | (p[1] << 8)));   /* little endian */
 }
 
 /* Dequantize one row of ncols weights (ncols % 32 == 0) into out[]. */
@@ -81,19 +100,29 @@ int orc_dequant_row(const uint8_t *row, int qtype, int ncols, double *out)
 {
     int bs = orc_block_bytes(qtype);
     if (bs == 0 || ncols % ORC_QK) return -1;
+    const int has_m = qtype == ORC_Q4_1 || qtype == ORC_Q5_1;
+    const int has_qh = qtype == ORC_Q5_0 || qtype == ORC_Q5_1;
     for (int b = 0; b < ncols / ORC_QK; b++) {
         const uint8_t *blk = row + (size_t)b * bs;
-        uint16_t dbits = (uint16_t)(blk[0] | (blk[1] << 8));   /* little endian */
-        double d = orc_half_to_double(dbits);
+        double d = orc_half_at(blk);
+        double m = has_m ? orc_half_at(blk + 2) : 0.0;
+        const uint8_t *qh = blk + 2 + 2 * has_m;          /* 5-bit types only */
+        const uint8_t *qs = qh + 4 * has_qh;
+        uint32_t hbits = has_qh ? (uint32_t)qh[0] | ((uint32_t)qh[1] << 8) |
+                                      ((uint32_t)qh[2] << 16) | ((uint32_t)qh[3] << 24)
+                                : 0u;
         for (int i = 0; i < ORC_QK; i++) {
             double v;
             if (qtype == ORC_Q8_0) {
-                int q = (int)(int8_t)blk[2 + i];
+                int q = (int)(int8_t)qs[i];
                 v = (double)q * d;
             } else {
-                int byte = blk[2 + (i % 16)];
+                int byte = qs[i % 16];
                 int q = (i < 16) ? (byte & 0x0f) : (byte >> 4);
-                v = (double)(q - 8) * d;
+                if (has_qh) q |= (int)((hbits >> i) & 1u) << 4;
+                if (qtype == ORC_Q4_0) v = (double)(q - 8) * d;
+                else if (qtype == ORC_Q5_0) v = (double)(q - 16) * d;
+                else v = (double)q * d + m;
             }
             out[b * ORC_QK + i] = v;
         }
@@ -212,7 +241,7 @@ static size_t orc_expert_stride(int nrows, int ncols, int qtype)
 /* The routed layer for a list of tokens.
  *  x [T,D] fp32 values; ids/gates [T,k] from orc_select (any k-subset works);
  *  gate/up/down: pools of E experts in `qtype` (slot = expert id);
- *  sh_*: optional shared expert (Q8_0, F = sh_F) added with weight 1;
+ *  sh_*: optional shared expert (its own type sh_qtype, F = sh_F), weight 1;
  *  tok_list[n_tok]: the tokens to evaluate (NULL = all T, n_tok = T);
  *  y [n_tok, D] doubles.  dense != 0 evaluates all E experts per token and
  *  weights each by its gate if selected and by 0 otherwise (the dense,

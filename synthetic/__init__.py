@@ -8,13 +8,20 @@ softmax, SwiGLU or combine); the decoders live separately in ``oracle/`` and in
 the CUDA library and share no code.
 
 Block formats (the quant types named in the FreeToken fork README, "Quant
-types" table: Standard family Q4_0 / Q8_0), 32 weights per block, blocks run
-along the reduction dimension of each weight row:
+types" table: the Standard family Q4_0, Q4_1, Q5_0, Q5_1, Q8_0; the byte
+layouts are ggml's published ones), 32 weights per block, blocks run along the
+reduction dimension of each weight row, all fields little endian:
 
 * Q8_0: ``{fp16 d; int8 qs[32]}``  (34 bytes), value ``qs[i] * d``.
 * Q4_0: ``{fp16 d; uint8 qs[16]}`` (18 bytes), value ``(q_i - 8) * d`` where
   byte ``j`` holds element ``j`` in its low nibble and element ``j + 16`` in its
   high nibble (the GGUF order).
+* Q4_1: ``{fp16 d; fp16 m; uint8 qs[16]}`` (20 bytes), value ``q_i * d + m``.
+* Q5_0: ``{fp16 d; uint8 qh[4]; uint8 qs[16]}`` (22 bytes), value
+  ``(q_i - 16) * d``; bit ``i`` of the 32-bit word ``qh`` is bit 4 of ``q_i``,
+  ``qs`` holds the low four bits as in Q4_0.
+* Q5_1: ``{fp16 d; fp16 m; uint8 qh[4]; uint8 qs[16]}`` (24 bytes), value
+  ``q_i * d + m``.
 
 Expert pools follow the FreeToken fork README, "Known limits": experts stored
 back to back as ``expert * nrows * (ncols / 32)`` blocks with no padding and
@@ -34,11 +41,15 @@ import numpy as np
 
 QK = 32
 Q4_0 = "q4_0"
+Q4_1 = "q4_1"
+Q5_0 = "q5_0"
+Q5_1 = "q5_1"
 Q8_0 = "q8_0"
+QTYPES = (Q4_0, Q4_1, Q5_0, Q5_1, Q8_0)
 # bytes per 32-weight block; a test checks these against include/moe.h
-BLOCK_BYTES = {Q4_0: 18, Q8_0: 34}
+BLOCK_BYTES = {Q4_0: 18, Q4_1: 20, Q5_0: 22, Q5_1: 24, Q8_0: 34}
 # ggml type ids, also exported by the C header
-GGML_TYPE_ID = {Q4_0: 2, Q8_0: 8}
+GGML_TYPE_ID = {Q4_0: 2, Q4_1: 3, Q5_0: 6, Q5_1: 7, Q8_0: 8}
 
 
 # --------------------------------------------------------------------------
@@ -175,11 +186,82 @@ def quantize_q4_0(w: np.ndarray) -> np.ndarray:
     return out.reshape(rows, -1)
 
 
+def _nibble_bytes(q: np.ndarray) -> np.ndarray:
+    """Low four bits of codes [..., 32] as 16 bytes: element j low, j+16 high."""
+    return (q[..., :16] & 0xF) | ((q[..., 16:] & 0xF) << 4)
+
+
+def _high_bit_word(q: np.ndarray) -> np.ndarray:
+    """Bit 4 of codes [..., 32] as a little-endian 32-bit word (4 bytes)."""
+    bits = ((q.astype(np.uint32) >> 4) & 1) << np.arange(QK, dtype=np.uint32)
+    w = bits.sum(axis=-1, dtype=np.uint64).astype(np.uint32)
+    return np.stack([(w >> (8 * i)) & 0xFF for i in range(4)], axis=-1).astype(np.uint8)
+
+
+def _f16_bytes(v: np.ndarray) -> np.ndarray:
+    """fp16 little-endian bytes [..., 2] of float32 values [...]."""
+    h = v.astype(np.float16).view(np.uint16)
+    return np.stack([h & 0xFF, h >> 8], axis=-1).astype(np.uint8)
+
+
+def quantize_min_scale(w: np.ndarray, bits: int) -> np.ndarray:
+    """Encode rows of float32 weights as Q4_1 (bits=4) or Q5_1 (bits=5).
+
+    Per block: m = min, d = (max - min) / (2^bits - 1) (fp32), q =
+    clamp(floor((w - m) / d + 0.5), 0, 2^bits - 1); d and m stored as fp16;
+    value q * d + m.  A constant block gets d = 0 and q = 0.
+    """
+    rows, cols = w.shape
+    assert cols % QK == 0 and bits in (4, 5)
+    top = (1 << bits) - 1
+    b = np.ascontiguousarray(w, dtype=np.float32).reshape(rows, cols // QK, QK)
+    lo = b.min(axis=2)
+    d = ((b.max(axis=2) - lo) / np.float32(top)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.floor((b - lo[..., None]) / d[..., None] + np.float32(0.5))
+    q = np.where(d[..., None] > 0, q, 0)
+    q = np.clip(q, 0, top).astype(np.uint8)
+    parts = [_f16_bytes(d), _f16_bytes(lo)]
+    if bits == 5:
+        parts.append(_high_bit_word(q))
+    parts.append(_nibble_bytes(q))
+    return np.concatenate(parts, axis=2).reshape(rows, -1)
+
+
+def quantize_q5_0(w: np.ndarray) -> np.ndarray:
+    """Encode rows of float32 weights as Q5_0 blocks.
+
+    As Q4_0 with 32 levels: m = the signed weight of largest magnitude (the
+    positive one on a tie), d = -m / 16, q = clamp(round-half-away(w / d) +
+    16, 0, 31), d stored as fp16; value (q - 16) * d.  An all-zero block gets
+    d = 0 and q = 16.  Returns uint8 [rows, cols/32*22].
+    """
+    rows, cols = w.shape
+    assert cols % QK == 0
+    b = np.ascontiguousarray(w, dtype=np.float32).reshape(rows, cols // QK, QK)
+    hi = b.max(axis=2)
+    lo = b.min(axis=2)
+    m = np.where(hi >= -lo, hi, lo)
+    d = (m / np.float32(-16.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = _round_half_away(b / d[..., None]) + 16
+    q = np.where(d[..., None] != 0, q, 16)
+    q = np.clip(q, 0, 31).astype(np.uint8)
+    return np.concatenate([_f16_bytes(d), _high_bit_word(q), _nibble_bytes(q)],
+                          axis=2).reshape(rows, -1)
+
+
 def quantize(w: np.ndarray, qtype: str) -> np.ndarray:
     if qtype == Q8_0:
         return quantize_q8_0(w)
     if qtype == Q4_0:
         return quantize_q4_0(w)
+    if qtype == Q4_1:
+        return quantize_min_scale(w, 4)
+    if qtype == Q5_0:
+        return quantize_q5_0(w)
+    if qtype == Q5_1:
+        return quantize_min_scale(w, 5)
     raise ValueError(f"unknown qtype {qtype}")
 
 

@@ -1,13 +1,21 @@
-"""Writes blocks.txt: hand-packed Q8_0 / Q4_0 blocks and the values their
+"""Writes blocks.txt: hand-packed Standard-family blocks and the values their
 closed form gives.
 
-Each block is built from a chosen fp16 scale (an exactly representable value,
-given by its bit pattern) and chosen integer codes; the expected values are
-code * d (Q8_0) or (code - 8) * d (Q4_0), computed here from the chosen
-integers, never by decoding the bytes.  The bytes follow the block layouts of
-the ggml Standard-family types (FreeToken fork README, "Quant types" table):
-Q8_0 = fp16 d (little endian) then 32 int8 codes; Q4_0 = fp16 d then 16 bytes,
-byte j holding code j in its low nibble and code j+16 in its high nibble.
+Each block is built from a chosen fp16 scale d (and, for the _1 types, a
+chosen fp16 minimum m), each an exactly representable value given both by its
+bit pattern and by its exact value, and chosen integer codes; the expected
+values are code * d (Q8_0), (code - 8) * d (Q4_0), (code - 16) * d (Q5_0) or
+code * d + m (Q4_1, Q5_1), computed here from the chosen integers, never by
+decoding the bytes.  The bytes follow the block layouts of the ggml
+Standard-family types (FreeToken fork README, "Quant types" table, which names
+the types; the layouts are ggml's published ones), little endian:
+  Q8_0 = d, then 32 int8 codes;
+  Q4_0 = d, then 16 bytes, byte j holding code j in its low nibble and code
+         j+16 in its high nibble;
+  Q4_1 = d, m, then the 16 nibble bytes as in Q4_0;
+  Q5_0 = d, a 32-bit word whose bit i is bit 4 of code i, then the low four
+         bits of the codes as Q4_0's 16 bytes;
+  Q5_1 = d, m, then the bit-4 word and the 16 nibble bytes as in Q5_0.
 Run: python tests/golden/make_blocks.py > tests/golden/blocks.txt
 """
 from fractions import Fraction
@@ -25,26 +33,72 @@ BLOCKS = [
     ("q4_big_scale", "q4_0", 0x5A00, Fraction(192), [0, 15, 8, 7, 9, 1] + [8] * 26),
 ]
 
+# name, qtype, d bits, d exact, m bits, m exact, codes (the _1 types)
+BLOCKS_MIN = [
+    ("q4_1_ramp", "q4_1", 0x3800, Fraction(1, 2), 0xC200, Fraction(-3),
+     [i % 16 for i in range(32)]),
+    ("q4_1_negative_scale", "q4_1", 0xB400, Fraction(-1, 4), 0x3E00, Fraction(3, 2),
+     [(5 * i + 3) % 16 for i in range(32)]),
+    ("q5_1_scattered_high_bits", "q5_1", 0x3A00, Fraction(3, 4), 0xCA00, Fraction(-12),
+     [(11 * i + 5) % 32 for i in range(32)]),
+    ("q5_1_subnormal", "q5_1", 0x0001, Fraction(1, 2 ** 24), 0x8001, Fraction(-1, 2 ** 24),
+     [31, 0, 1, 30] + [16] * 27 + [15]),
+]
 
-def pack(qtype, dbits, codes):
-    b = [dbits & 0xFF, dbits >> 8]
+BLOCKS_Q5_0 = [
+    ("q5_0_full_range", "q5_0", 0x3000, Fraction(1, 8), list(range(32))),
+    ("q5_0_scattered_high_bits", "q5_0", 0x4000, Fraction(2), [(7 * i) % 32 for i in range(32)]),
+    ("q5_0_only_low_half_high", "q5_0", 0xBC00, Fraction(-1),
+     [16 + (i % 16) for i in range(16)] + [i % 16 for i in range(16)]),
+]
+
+
+def _le16(v):
+    return [v & 0xFF, v >> 8]
+
+
+def _nibbles(codes):
+    return [(codes[j] & 0xF) | ((codes[j + 16] & 0xF) << 4) for j in range(16)]
+
+
+def _high_word(codes):
+    w = sum(((c >> 4) & 1) << i for i, c in enumerate(codes))
+    return [(w >> (8 * i)) & 0xFF for i in range(4)]
+
+
+def pack(qtype, dbits, codes, mbits=None):
+    b = _le16(dbits)
+    if qtype in ("q4_1", "q5_1"):
+        b += _le16(mbits)
     if qtype == "q8_0":
         b += [c & 0xFF for c in codes]
     else:
-        b += [codes[j] | (codes[j + 16] << 4) for j in range(16)]
+        if qtype in ("q5_0", "q5_1"):
+            b += _high_word(codes)
+        b += _nibbles(codes)
     return bytes(b)
 
 
 def main():
     print("# Hand-packed ggml blocks: name qtype hex-bytes then 32 exact values.")
     print("# Derivation and layout: see make_blocks.py beside this file.")
+    def emit(name, qt, raw, vals):
+        print(name, qt, raw.hex(), " ".join(repr(float(v)) for v in vals))
+
     for name, qt, dbits, d, codes in BLOCKS:
         assert len(codes) == 32
         if qt == "q8_0":
             vals = [c * d for c in codes]
         else:
             vals = [(c - 8) * d for c in codes]
-        print(name, qt, pack(qt, dbits, codes).hex(), " ".join(repr(float(v)) for v in vals))
+        emit(name, qt, pack(qt, dbits, codes), vals)
+    for name, qt, dbits, d, codes in BLOCKS_Q5_0:
+        assert len(codes) == 32 and all(0 <= c < 32 for c in codes)
+        emit(name, qt, pack(qt, dbits, codes), [(c - 16) * d for c in codes])
+    for name, qt, dbits, d, mbits, m, codes in BLOCKS_MIN:
+        top = 16 if qt == "q4_1" else 32
+        assert len(codes) == 32 and all(0 <= c < top for c in codes)
+        emit(name, qt, pack(qt, dbits, codes, mbits), [c * d + m for c in codes])
 
 
 if __name__ == "__main__":

@@ -43,7 +43,8 @@ def test_block_tables_agree_with_header(moe, orc):
     assert moe.lib().moe_block_bytes(moe.Q4_0) == 18 == orc.block_bytes("q4_0")
     assert moe.lib().moe_block_bytes(moe.Q8_0) == 34 == orc.block_bytes("q8_0")
     assert moe.lib().moe_block_bytes(3) == 0        # unknown type -> 0, never garbage
-    assert S.GGML_TYPE_ID == {"q4_0": moe.Q4_0, "q8_0": moe.Q8_0}
+    assert {q: S.GGML_TYPE_ID[q] for q in ("q4_0", "q8_0")} == {"q4_0": moe.Q4_0,
+                                                                 "q8_0": moe.Q8_0}
 
 
 def _err(L):

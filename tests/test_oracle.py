@@ -59,15 +59,17 @@ def test_dequant_hand_packed_blocks(orc, name, qtype, raw, vals):
     np.testing.assert_array_equal(got, vals)
 
 
-def test_dequant_row_of_several_blocks_keeps_block_order(orc):
-    blocks = _golden_blocks()
-    q4 = [b for b in blocks if b[1] == "q4_0"]
-    raw = b"".join(b[2] for b in q4)
-    got = orc.dequant_row(np.frombuffer(raw, np.uint8), "q4_0", 32 * len(q4))
-    np.testing.assert_array_equal(got, np.concatenate([b[3] for b in q4]))
+@pytest.mark.parametrize("qtype", ["q8_0", "q4_0", "q4_1", "q5_0", "q5_1"])
+def test_dequant_row_of_several_blocks_keeps_block_order(orc, qtype):
+    blocks = [b for b in _golden_blocks() if b[1] == qtype]
+    assert len(blocks) >= 2
+    raw = b"".join(b[2] for b in blocks)
+    got = orc.dequant_row(np.frombuffer(raw, np.uint8), qtype, 32 * len(blocks))
+    np.testing.assert_array_equal(got, np.concatenate([b[3] for b in blocks]))
 
 
-@pytest.mark.parametrize("qtype,slack,top", [("q8_0", 127, 127), ("q4_0", 8, 7)])
+@pytest.mark.parametrize("qtype,slack,top", [("q8_0", 127, 127), ("q4_0", 8, 7),
+                                             ("q5_0", 16, 15)])
 def test_quantizer_roundtrip_error_bound(orc, qtype, slack, top):
     # encoder (input generator) + decoder (oracle): |w - dequant(w)| <= |d|/2
     # up to the fp16 rounding of d (relative 2^-11, times the largest code),
@@ -87,6 +89,49 @@ def test_quantizer_roundtrip_error_bound(orc, qtype, slack, top):
     assert np.all(np.abs(deq - w) <= bound)
     assert np.all(np.abs(deq - w) <= dd * (1 + slack * 2.0 ** -11) + 1e-12)
     assert np.all(deq[3, 32:64] == 0.0)
+
+
+@pytest.mark.parametrize("qtype,top", [("q4_1", 15), ("q5_1", 31)])
+def test_min_scale_quantizer_roundtrip_error_bound(orc, qtype, top):
+    # value = q * d + m with m = the block minimum and d = range / top: the
+    # error is at most d/2, plus the fp16 rounding of d (relative 2^-11,
+    # times the code) and of m (relative 2^-11); the block minimum itself
+    # lands on code 0 and decodes to fp16(m).
+    rng = np.random.default_rng(15)
+    w = (rng.standard_normal((16, 256)) * 0.02 + 0.003).astype(np.float32)
+    w[5, 64:96] = 0.0125                    # a constant block: d = 0, q = 0
+    packed = S.quantize(w, qtype)
+    deq = orc.dequant_matrix(packed, qtype, 256)
+    blk = packed.reshape(16, 8, S.BLOCK_BYTES[qtype])
+    d16 = blk[:, :, 0:2].copy().view(np.float16)[..., 0].astype(np.float64)
+    m16 = blk[:, :, 2:4].copy().view(np.float16)[..., 0].astype(np.float64)
+    assert np.all(d16 >= 0)
+    dd = np.repeat(d16, 32, axis=1)
+    mm = np.repeat(np.abs(m16), 32, axis=1)
+    bound = 0.5 * dd * (1 + 2.0 ** -10) + top * 2.0 ** -11 * dd + 2.0 ** -11 * mm + 1e-12
+    assert np.all(np.abs(deq - w) <= bound)
+    wb = w.reshape(16, 8, 32)
+    imin = np.argmin(wb, axis=2)
+    got = deq.reshape(16, 8, 32)[np.arange(16)[:, None], np.arange(8)[None], imin]
+    np.testing.assert_array_equal(got, m16)
+    np.testing.assert_array_equal(deq[5, 64:96], np.float64(np.float16(0.0125)))
+
+
+def test_q5_0_largest_weight_lands_on_code_zero(orc):
+    rng = np.random.default_rng(16)
+    w = (rng.standard_normal((4, 64)) * 0.02).astype(np.float32)
+    packed = S.quantize(w, "q5_0").reshape(4, 2, 22)
+    wb = w.reshape(4, 2, 32)
+    deq = orc.dequant_matrix(packed.reshape(4, -1), "q5_0", 64).reshape(4, 2, 32)
+    for r in range(4):
+        for b in range(2):
+            i = int(np.argmax(np.abs(wb[r, b])))
+            word = int.from_bytes(bytes(packed[r, b, 2:6]), "little")
+            code = ((packed[r, b, 6 + i % 16] >> (0 if i < 16 else 4)) & 0xF) | \
+                (((word >> i) & 1) << 4)
+            assert code == 0
+            d16 = float(packed[r, b, :2].copy().view(np.float16)[0])
+            assert deq[r, b, i] == -16 * d16
 
 
 def test_q4_0_largest_weight_lands_on_code_zero(orc):
@@ -196,28 +241,59 @@ def _textbook_swiglu(x, Wg, Wu, Wd):
     return h @ Wd.T
 
 
+# integer value range of each type at scale 1 (and, for the _1 types, the
+# fp16 minimum m = -8 / -16 that centres it), and the code offset
+_INT_RANGE = {"q8_0": (-20, 21), "q4_0": (-8, 8), "q4_1": (-8, 8),
+              "q5_0": (-16, 16), "q5_1": (-16, 16)}
+_CODE_OFF = {"q4_0": 8, "q4_1": 8, "q5_0": 16, "q5_1": 16}
+_MIN_BITS = {"q4_1": 0xC800, "q5_1": 0xCC00}      # fp16 -8.0, -16.0
+
+
 def _pack_int_matrix(codes, qtype, dbits=0x3C00):
     """Pack an integer matrix with scale 1.0 in every block (test-side
-    packing by the format definition; values = codes)."""
+    packing by the format definition; values = codes).  The _1 types get
+    m = -offset so that code = value + offset as in their _0 twins."""
     rows, cols = codes.shape
-    blocks = codes.reshape(rows, cols // 32, 32)
-    lo = blocks.astype(np.int64)
+    nb = cols // 32
+    lo = codes.reshape(rows, nb, 32).astype(np.int64)
+    fields = [np.full((rows, nb, 2), [dbits & 0xFF, dbits >> 8], np.uint8)]
     if qtype == "q8_0":
-        body = (lo & 0xFF).astype(np.uint8)
+        fields.append((lo & 0xFF).astype(np.uint8))
     else:
-        c = (lo + 8).astype(np.uint8)
-        body = c[..., :16] | (c[..., 16:] << 4)
-    d = np.full((rows, cols // 32, 2), [dbits & 0xFF, dbits >> 8], np.uint8)
-    return np.concatenate([d, body], axis=2).reshape(rows, -1)
+        c = (lo + _CODE_OFF[qtype]).astype(np.uint32)
+        assert c.min() >= 0 and c.max() < 2 * _CODE_OFF[qtype]
+        if qtype in _MIN_BITS:
+            mb = _MIN_BITS[qtype]
+            fields.append(np.full((rows, nb, 2), [mb & 0xFF, mb >> 8], np.uint8))
+        if qtype in ("q5_0", "q5_1"):
+            word = np.zeros((rows, nb), np.uint64)
+            for i in range(32):
+                word |= ((c[..., i] >> 4) & 1).astype(np.uint64) << np.uint64(i)
+            fields.append(np.stack([(word >> np.uint64(8 * j)) & np.uint64(0xFF)
+                                    for j in range(4)], axis=-1).astype(np.uint8))
+        n = c & 0xF
+        fields.append((n[..., :16] | (n[..., 16:] << 4)).astype(np.uint8))
+    return np.concatenate(fields, axis=2).reshape(rows, -1)
 
 
-@pytest.mark.parametrize("qtype", ["q8_0", "q4_0"])
+def test_int_matrix_packer_agrees_with_the_golden_layouts(orc):
+    # the packer above against the hand-packed golden blocks' layouts: a
+    # unit-scale block of codes 0..31 (values code - offset) decodes to them
+    for qt in ("q4_0", "q4_1", "q5_0", "q5_1", "q8_0"):
+        lo, hi = _INT_RANGE[qt]
+        vals = np.arange(32) % (hi - lo) + lo
+        raw = _pack_int_matrix(vals[None], qt)
+        assert raw.shape[1] == S.BLOCK_BYTES[qt]
+        np.testing.assert_array_equal(orc.dequant_row(raw[0], qt, 32), vals)
+
+
+@pytest.mark.parametrize("qtype", ["q8_0", "q4_0", "q4_1", "q5_0", "q5_1"])
 def test_single_expert_is_textbook_swiglu(orc, qtype):
     # integer-valued weights (scale 1) so the dequantized matrices are known
     # exactly; E=1, k=1 reduces the layer to a plain SwiGLU FFN.
     rng = np.random.default_rng(11)
     D, F = 64, 96
-    lo, hi = (-8, 8) if qtype == "q4_0" else (-20, 21)
+    lo, hi = _INT_RANGE[qtype]
     Wg = rng.integers(lo, hi, (F, D))
     Wu = rng.integers(lo, hi, (F, D))
     Wd = rng.integers(lo, hi, (D, F))
