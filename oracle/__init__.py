@@ -25,7 +25,10 @@ Q4_1 = 3
 Q5_0 = 6
 Q5_1 = 7
 Q8_0 = 8
-QTYPE = {"q4_0": Q4_0, "q4_1": Q4_1, "q5_0": Q5_0, "q5_1": Q5_1, "q8_0": Q8_0}
+Q4_K = 12
+Q6_K = 14
+QTYPE = {"q4_0": Q4_0, "q4_1": Q4_1, "q5_0": Q5_0, "q5_1": Q5_1, "q8_0": Q8_0,
+         "q4_k": Q4_K, "q6_k": Q6_K}
 
 
 def build(force: bool = False) -> str:
@@ -58,6 +61,8 @@ def _declare(L):
     L.orc_half_to_double.argtypes = [C.c_uint16]
     L.orc_block_bytes.restype = _i
     L.orc_block_bytes.argtypes = [_i]
+    L.orc_block_weights.restype = _i
+    L.orc_block_weights.argtypes = [_i]
     L.orc_dequant_row.restype = _i
     L.orc_dequant_row.argtypes = [_p, _i, _i, _p]
     L.orc_router_logits.restype = None
@@ -107,6 +112,10 @@ def half_to_double(h: int) -> float:
 
 def block_bytes(qtype) -> int:
     return lib().orc_block_bytes(_qt(qtype))
+
+
+def block_weights(qtype) -> int:
+    return lib().orc_block_weights(_qt(qtype))
 
 
 def dequant_row(row_bytes: np.ndarray, qtype, ncols: int) -> np.ndarray:

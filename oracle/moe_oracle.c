@@ -20,6 +20,19 @@
  *   qs byte j holds the low 4 bits of element j (low nibble) and of element
  *   j+16 (high nibble); for the 5-bit types bit i of the 32-bit word qh is
  *   bit 4 of element i.
+ *   K-quants (same table, K-quants row; ggml's published super-block
+ *   layouts), 256 weights per block:
+ *     Q4_K {fp16 d; fp16 dmin; uint8 scales[12]; uint8 qs[128]} (144 B):
+ *       eight sub-blocks of 32, each with a 6-bit scale sc_j and a 6-bit
+ *       min m_j packed in scales[] (orc_q4k_scale_min); value
+ *       d * sc_j * q - dmin * m_j; weight 64c + l (l < 32) is the low nibble
+ *       of qs[32c + l] (sub-block 2c), weight 64c + 32 + l its high nibble
+ *       (sub-block 2c + 1).
+ *     Q6_K {uint8 ql[128]; uint8 qh[64]; int8 scales[16]; fp16 d} (210 B):
+ *       value d * scales[i / 16] * (q_i - 32) with q_i 6-bit: in half h
+ *       (weights 128h + 32r + l, r < 4, l < 32) the low 4 bits are nibble
+ *       r / 2 of ql[64h + 32(r % 2) + l] and the high 2 bits are bits
+ *       2r, 2r+1 of qh[32h + l].
  *   Expert pool layout -- FreeToken fork README, "Known limits": experts back
  *   to back, expert * nrows * (ncols / 32) blocks, no padding, one type.
  *   Per expert: W_gate, W_up are [F rows][D/32 blocks], W_down [D][F/32].
@@ -60,6 +73,8 @@
 #define ORC_Q5_0 6
 #define ORC_Q5_1 7
 #define ORC_Q8_0 8
+#define ORC_Q4_K 12
+#define ORC_Q6_K 14
 
 /* IEEE 754 binary16 -> double, decoded bit by bit (sign, 5-bit exponent with
  * bias 15, 10-bit fraction; subnormals, infinities and NaN included). */
@@ -86,6 +101,8 @@ int orc_block_bytes(int qtype)
     case ORC_Q4_1: return 2 + 2 + 16;
     case ORC_Q5_0: return 2 + 4 + 16;
     case ORC_Q5_1: return 2 + 2 + 4 + 16;
+    case ORC_Q4_K: return 2 + 2 + 12 + 128;
+    case ORC_Q6_K: return 128 + 64 + 16 + 2;
     default: return 0;
     }
 }
@@ -95,11 +112,75 @@ static double orc_half_at(const uint8_t *p)
     return orc_half_to_double((uint16_t)(p[0] | (p[1] << 8)));   /* little endian */
 }
 
-/* Dequantize one row of ncols weights (ncols % 32 == 0) into out[]. */
+/* Weights per block: 256 for the K-quants, 32 for the rest, 0 if unknown. */
+int orc_block_weights(int qtype)
+{
+    if (orc_block_bytes(qtype) == 0) return 0;
+    return (qtype == ORC_Q4_K || qtype == ORC_Q6_K) ? 256 : ORC_QK;
+}
+
+/* Bytes of a row of ncols weights (ncols a multiple of the block). */
+static size_t orc_row_bytes(int qtype, int ncols)
+{
+    return (size_t)(ncols / orc_block_weights(qtype)) * (size_t)orc_block_bytes(qtype);
+}
+
+/* Q4_K: the 6-bit scale and min of sub-block j (0..7) from scales[12].
+ * Sub-blocks 0-3 keep theirs in the low six bits of bytes j and j+4;
+ * sub-blocks 4-7 in the nibbles of byte j+4 (scale low, min high) plus the
+ * top two bits of bytes j-4 (scale) and j (min). */
+static void orc_q4k_scale_min(const uint8_t *sc, int j, int *scale, int *min)
+{
+    if (j < 4) {
+        *scale = sc[j] & 63;
+        *min = sc[j + 4] & 63;
+    } else {
+        *scale = (sc[j + 4] & 0x0f) | ((sc[j - 4] >> 6) << 4);
+        *min = (sc[j + 4] >> 4) | ((sc[j] >> 6) << 4);
+    }
+}
+
+static void orc_dequant_q4k(const uint8_t *blk, double *out)
+{
+    double d = orc_half_at(blk), dmin = orc_half_at(blk + 2);
+    const uint8_t *sc = blk + 4, *qs = blk + 16;
+    for (int i = 0; i < 256; i++) {
+        int j = i / 32, l = i % 32, scale, min;
+        orc_q4k_scale_min(sc, j, &scale, &min);
+        int byte = qs[32 * (j / 2) + l];
+        int q = (j % 2) ? (byte >> 4) : (byte & 0x0f);
+        out[i] = d * (double)scale * (double)q - dmin * (double)min;
+    }
+}
+
+static void orc_dequant_q6k(const uint8_t *blk, double *out)
+{
+    const uint8_t *ql = blk, *qh = blk + 128;
+    const int8_t *sc = (const int8_t *)(blk + 192);
+    double d = orc_half_at(blk + 208);
+    for (int i = 0; i < 256; i++) {
+        int h = i / 128, r = (i % 128) / 32, l = i % 32;
+        int lo = ql[64 * h + 32 * (r % 2) + l];
+        lo = (r / 2) ? (lo >> 4) : (lo & 0x0f);
+        int hi = (qh[32 * h + l] >> (2 * r)) & 3;
+        int q = lo | (hi << 4);
+        out[i] = d * (double)sc[i / 16] * (double)(q - 32);
+    }
+}
+
+
+/* Dequantize one row of ncols weights (a multiple of the block) into out[]. */
 int orc_dequant_row(const uint8_t *row, int qtype, int ncols, double *out)
 {
-    int bs = orc_block_bytes(qtype);
-    if (bs == 0 || ncols % ORC_QK) return -1;
+    int bs = orc_block_bytes(qtype), bw = orc_block_weights(qtype);
+    if (bs == 0 || ncols % bw) return -1;
+    if (bw == 256) {
+        for (int b = 0; b < ncols / 256; b++) {
+            if (qtype == ORC_Q4_K) orc_dequant_q4k(row + (size_t)b * bs, out + 256 * b);
+            else orc_dequant_q6k(row + (size_t)b * bs, out + 256 * b);
+        }
+        return 0;
+    }
     const int has_m = qtype == ORC_Q4_1 || qtype == ORC_Q5_1;
     const int has_qh = qtype == ORC_Q5_0 || qtype == ORC_Q5_1;
     for (int b = 0; b < ncols / ORC_QK; b++) {
@@ -215,8 +296,8 @@ static void orc_expert_ffn_row(const double *xt, const uint8_t *gate,
                                const uint8_t *up, const uint8_t *down, int qtype,
                                int D, int F, double *wrow, double *h, double *Y)
 {
-    size_t gate_row = (size_t)(D / ORC_QK) * orc_block_bytes(qtype);
-    size_t down_row = (size_t)(F / ORC_QK) * orc_block_bytes(qtype);
+    size_t gate_row = orc_row_bytes(qtype, D);
+    size_t down_row = orc_row_bytes(qtype, F);
     for (int r = 0; r < F; r++) {
         double a = 0.0, u = 0.0;
         orc_dequant_row(gate + r * gate_row, qtype, D, wrow);
@@ -235,7 +316,7 @@ static void orc_expert_ffn_row(const double *xt, const uint8_t *gate,
 
 static size_t orc_expert_stride(int nrows, int ncols, int qtype)
 {
-    return (size_t)nrows * (size_t)(ncols / ORC_QK) * orc_block_bytes(qtype);
+    return (size_t)nrows * orc_row_bytes(qtype, ncols);
 }
 
 /* The routed layer for a list of tokens.
@@ -254,9 +335,12 @@ int orc_layer(const float *x, int T, int D, int F, int E, int k, int qtype,
               const int32_t *tok_list, int n_tok, int dense, int nthreads,
               double *y)
 {
-    if (orc_block_bytes(qtype) == 0 || D % ORC_QK || F % ORC_QK || k > E)
+    int bw = orc_block_weights(qtype);
+    if (bw == 0 || D % bw || F % bw || k > E)
         return -1;
-    if (sh_gate && (orc_block_bytes(sh_qtype) == 0 || sh_F % ORC_QK)) return -1;
+    if (sh_gate && (orc_block_weights(sh_qtype) == 0 || D % orc_block_weights(sh_qtype) ||
+                    sh_F % orc_block_weights(sh_qtype)))
+        return -1;
     if (!tok_list) n_tok = T;
     size_t gstride = orc_expert_stride(F, D, qtype);
     size_t dstride = orc_expert_stride(D, F, qtype);
@@ -314,7 +398,8 @@ int orc_expert_rows(const float *x, int T, int D, int F, int E, int k,
                     const int32_t *offsets, const int32_t *pos_list, int n_pos,
                     int nthreads, double *Y)
 {
-    if (orc_block_bytes(qtype) == 0 || D % ORC_QK || F % ORC_QK) return -1;
+    int bw = orc_block_weights(qtype);
+    if (bw == 0 || D % bw || F % bw) return -1;
     if (!pos_list) n_pos = T * k;
     size_t gstride = orc_expert_stride(F, D, qtype);
     size_t dstride = orc_expert_stride(D, F, qtype);

@@ -23,6 +23,22 @@ reduction dimension of each weight row, all fields little endian:
 * Q5_1: ``{fp16 d; fp16 m; uint8 qh[4]; uint8 qs[16]}`` (24 bytes), value
   ``q_i * d + m``.
 
+K-quants (same table, K-quants row; ggml's published layouts), 256 weights
+per block:
+
+* Q4_K: ``{fp16 d; fp16 dmin; uint8 scales[12]; uint8 qs[128]}`` (144 bytes):
+  eight 32-weight sub-blocks with 6-bit scales ``sc_j`` and mins ``m_j``
+  (``j < 4``: low six bits of ``scales[j]`` / ``scales[j+4]``; ``j >= 4``:
+  low / high nibble of ``scales[j+4]`` plus the top two bits of
+  ``scales[j-4]`` / ``scales[j]``); value ``d * sc_j * q - dmin * m_j``;
+  weight ``64c + l`` is the low nibble of ``qs[32c + l]``, weight
+  ``64c + 32 + l`` its high nibble.
+* Q6_K: ``{uint8 ql[128]; uint8 qh[64]; int8 scales[16]; fp16 d}`` (210
+  bytes): value ``d * scales[i // 16] * (q_i - 32)``; weight
+  ``128h + 32r + l`` keeps its low four bits in nibble ``r // 2`` of
+  ``ql[64h + 32(r % 2) + l]`` and its high two in bits ``2r, 2r+1`` of
+  ``qh[32h + l]``.
+
 Expert pools follow the FreeToken fork README, "Known limits": experts stored
 back to back as ``expert * nrows * (ncols / 32)`` blocks with no padding and
 one quant type for the whole pool.  Per expert, ``W_gate`` and ``W_up`` are
@@ -45,11 +61,22 @@ Q4_1 = "q4_1"
 Q5_0 = "q5_0"
 Q5_1 = "q5_1"
 Q8_0 = "q8_0"
-QTYPES = (Q4_0, Q4_1, Q5_0, Q5_1, Q8_0)
-# bytes per 32-weight block; a test checks these against include/moe.h
-BLOCK_BYTES = {Q4_0: 18, Q4_1: 20, Q5_0: 22, Q5_1: 24, Q8_0: 34}
+Q4_K = "q4_k"
+Q6_K = "q6_k"
+QTYPES = (Q4_0, Q4_1, Q5_0, Q5_1, Q8_0, Q4_K, Q6_K)
+QK_K = 256
+# bytes per block and weights per block; a test checks these against
+# include/moe.h
+BLOCK_BYTES = {Q4_0: 18, Q4_1: 20, Q5_0: 22, Q5_1: 24, Q8_0: 34, Q4_K: 144, Q6_K: 210}
+BLOCK_WEIGHTS = {q: (QK_K if q in (Q4_K, Q6_K) else QK) for q in QTYPES}
 # ggml type ids, also exported by the C header
-GGML_TYPE_ID = {Q4_0: 2, Q4_1: 3, Q5_0: 6, Q5_1: 7, Q8_0: 8}
+GGML_TYPE_ID = {Q4_0: 2, Q4_1: 3, Q5_0: 6, Q5_1: 7, Q8_0: 8, Q4_K: 12, Q6_K: 14}
+
+
+def row_bytes(ncols: int, qtype: str) -> int:
+    """Bytes of one weight row of ncols weights (a multiple of the block)."""
+    assert ncols % BLOCK_WEIGHTS[qtype] == 0
+    return ncols // BLOCK_WEIGHTS[qtype] * BLOCK_BYTES[qtype]
 
 
 # --------------------------------------------------------------------------
@@ -70,7 +97,8 @@ class LayerConfig:
     expert_std: float = 0.02
     zipf_s: float | None = None          # per-expert router bias (prefill config)
     logits_from_trace: bool = False      # routing logits given directly
-    shared_F: int = 0                    # always-on shared expert, Q8_0
+    shared_F: int = 0                    # always-on shared expert
+    shared_qtype: str = Q8_0             # its block type
     seed: int = 1000
     renorm: bool = True
     T_values: tuple = field(default_factory=tuple)   # documentation only
@@ -113,8 +141,7 @@ def with_T(cfg: LayerConfig, T: int) -> LayerConfig:
 
 def expert_bytes(D: int, F: int, qtype: str) -> tuple[int, int, int]:
     """Bytes of (gate, up, down) of one expert in the pool layout."""
-    bs = BLOCK_BYTES[qtype]
-    return F * (D // QK) * bs, F * (D // QK) * bs, D * (F // QK) * bs
+    return F * row_bytes(D, qtype), F * row_bytes(D, qtype), D * row_bytes(F, qtype)
 
 
 # --------------------------------------------------------------------------
@@ -251,6 +278,81 @@ def quantize_q5_0(w: np.ndarray) -> np.ndarray:
                           axis=2).reshape(rows, -1)
 
 
+def quantize_q4_k(w: np.ndarray) -> np.ndarray:
+    """Encode rows of float32 weights as Q4_K super-blocks.
+
+    Per 32-weight sub-block j: lo_j = min(min w, 0), s_j = (max w - lo_j) / 15.
+    Per super-block: d = max_j s_j / 63, dmin = max_j (-lo_j) / 63 (stored
+    fp16); sc_j = clamp(round-half-away(s_j / d), 0, 63), m_j =
+    clamp(round-half-away(-lo_j / dmin), 0, 63); q = clamp(floor((w + dmin
+    m_j) / (d sc_j) + 1/2), 0, 15) with the stored d, dmin (q = 0 where d sc_j
+    is 0).  Returns uint8 [rows, cols/256*144].
+    """
+    rows, cols = w.shape
+    assert cols % QK_K == 0
+    nsb = cols // QK_K
+    b = np.ascontiguousarray(w, dtype=np.float32).reshape(rows, nsb, 8, 32)
+    lo = np.minimum(b.min(axis=3), 0)
+    s = ((b.max(axis=3) - lo) / np.float32(15)).astype(np.float32)
+    d16 = (s.max(axis=2) / np.float32(63)).astype(np.float16)
+    m16 = ((-lo).max(axis=2) / np.float32(63)).astype(np.float16)
+    d32, m32 = d16.astype(np.float32), m16.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        sc = np.where(d32[..., None] > 0, _round_half_away(s / d32[..., None]), 0)
+        mn = np.where(m32[..., None] > 0, _round_half_away(-lo / m32[..., None]), 0)
+    sc = np.clip(sc, 0, 63).astype(np.uint8)
+    mn = np.clip(mn, 0, 63).astype(np.uint8)
+    eff = d32[..., None] * sc.astype(np.float32)
+    off = m32[..., None] * mn.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.floor((b + off[..., None]) / eff[..., None] + np.float32(0.5))
+    q = np.where(eff[..., None] > 0, q, 0)
+    q = np.clip(q, 0, 15).astype(np.uint8)                         # [rows, nsb, 8, 32]
+    s12 = np.zeros((rows, nsb, 12), np.uint8)
+    s12[..., 0:4] = (sc[..., 0:4] & 63) | ((sc[..., 4:8] >> 4) << 6)
+    s12[..., 4:8] = (mn[..., 0:4] & 63) | ((mn[..., 4:8] >> 4) << 6)
+    s12[..., 8:12] = (sc[..., 4:8] & 15) | ((mn[..., 4:8] & 15) << 4)
+    qs = (q[..., 0::2, :] | (q[..., 1::2, :] << 4)).reshape(rows, nsb, 128)
+    return np.concatenate([_f16_bytes(d32), _f16_bytes(m32), s12, qs], axis=2).reshape(rows, -1)
+
+
+def quantize_q6_k(w: np.ndarray) -> np.ndarray:
+    """Encode rows of float32 weights as Q6_K super-blocks.
+
+    Per 16-weight sub-block j: m_j = the signed weight of largest magnitude
+    (the positive one on a tie), s_j = -m_j / 32.  Per super-block: d =
+    max_j |s_j| / 127 (stored fp16), sc_j = clamp(round-half-away(s_j / d),
+    -128, 127); q = clamp(round-half-away(w / (d sc_j)) + 32, 0, 63) (32 where
+    d sc_j is 0).  Returns uint8 [rows, cols/256*210].
+    """
+    rows, cols = w.shape
+    assert cols % QK_K == 0
+    nsb = cols // QK_K
+    b = np.ascontiguousarray(w, dtype=np.float32).reshape(rows, nsb, 16, 16)
+    hi, lo = b.max(axis=3), b.min(axis=3)
+    m = np.where(hi >= -lo, hi, lo)
+    s = (m / np.float32(-32)).astype(np.float32)
+    d16 = (np.abs(s).max(axis=2) / np.float32(127)).astype(np.float16)
+    d32 = d16.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        sc = np.where(d32[..., None] > 0, _round_half_away(s / d32[..., None]), 0)
+    sc = np.clip(sc, -128, 127).astype(np.int8)
+    eff = d32[..., None] * sc.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = _round_half_away(b / eff[..., None]) + 32
+    q = np.where(eff[..., None] != 0, q, 32)
+    q = np.clip(q, 0, 63).astype(np.uint8).reshape(rows, nsb, 2, 4, 32)   # [h, r, l]
+    ql = np.zeros((rows, nsb, 2, 2, 32), np.uint8)                       # [h, r % 2, l]
+    ql |= q[:, :, :, 0:2, :] & 15
+    ql |= (q[:, :, :, 2:4, :] & 15) << 4
+    qh = np.zeros((rows, nsb, 2, 32), np.uint8)
+    for r in range(4):
+        qh |= (q[:, :, :, r, :] >> 4) << (2 * r)
+    return np.concatenate([ql.reshape(rows, nsb, 128), qh.reshape(rows, nsb, 64),
+                           sc.view(np.uint8).reshape(rows, nsb, 16), _f16_bytes(d32)],
+                          axis=2).reshape(rows, -1)
+
+
 def quantize(w: np.ndarray, qtype: str) -> np.ndarray:
     if qtype == Q8_0:
         return quantize_q8_0(w)
@@ -262,6 +364,10 @@ def quantize(w: np.ndarray, qtype: str) -> np.ndarray:
         return quantize_q5_0(w)
     if qtype == Q5_1:
         return quantize_min_scale(w, 5)
+    if qtype == Q4_K:
+        return quantize_q4_k(w)
+    if qtype == Q6_K:
+        return quantize_q6_k(w)
     raise ValueError(f"unknown qtype {qtype}")
 
 
@@ -277,10 +383,9 @@ def gen_expert_pool(seed: int, n_experts: int, D: int, F: int, qtype: str,
     Returns (gate, up, down) uint8 arrays of shapes
     [n, F, D/32*bs], [n, F, D/32*bs], [n, D, F/32*bs] (the pool layout).
     """
-    bs = BLOCK_BYTES[qtype]
-    gate = np.empty((n_experts, F, D // QK * bs), np.uint8)
+    gate = np.empty((n_experts, F, row_bytes(D, qtype)), np.uint8)
     up = np.empty_like(gate)
-    down = np.empty((n_experts, D, F // QK * bs), np.uint8)
+    down = np.empty((n_experts, D, row_bytes(F, qtype)), np.uint8)
     s32 = np.float32(std)
 
     def one(e):
@@ -359,7 +464,7 @@ class LayerInputs:
     gate: np.ndarray              # pool bytes (see gen_expert_pool)
     up: np.ndarray
     down: np.ndarray
-    shared: tuple | None          # (gate, up, down) with one expert, Q8_0
+    shared: tuple | None          # (gate, up, down) with one expert, cfg.shared_qtype
 
 
 def gen_activations(rng: np.random.Generator, T: int, D: int, dtype: str):
@@ -382,7 +487,8 @@ def make_layer(cfg: LayerConfig, T: int | None = None, seed: int | None = None,
         gate = up = down = None
     shared = None
     if cfg.shared_F:
-        shared = gen_expert_pool(seed + 7777, 1, cfg.D, cfg.shared_F, Q8_0, cfg.expert_std)
+        shared = gen_expert_pool(seed + 7777, 1, cfg.D, cfg.shared_F, cfg.shared_qtype,
+                                 cfg.expert_std)
     w_router = bias = logits = None
     if cfg.logits_from_trace:
         logits, _ = locality_trace(rng, T, cfg.E, cfg.k)

@@ -16,6 +16,17 @@ the types; the layouts are ggml's published ones), little endian:
   Q5_0 = d, a 32-bit word whose bit i is bit 4 of code i, then the low four
          bits of the codes as Q4_0's 16 bytes;
   Q5_1 = d, m, then the bit-4 word and the 16 nibble bytes as in Q5_0.
+K-quants (same table, K-quants row; ggml's published layouts), 256 weights:
+  Q4_K = d, dmin, 12 bytes of 6-bit scales sc_j and mins m_j of the eight
+         32-weight sub-blocks (j < 4: low six bits of bytes j and j+4;
+         j >= 4: the low / high nibble of byte j+4 plus the top two bits of
+         bytes j-4 / j), then 128 bytes: weight 64c + l is the low nibble of
+         byte 32c + l, weight 64c + 32 + l its high nibble; value
+         d * sc_j * q - dmin * m_j;
+  Q6_K = 128 bytes ql, 64 bytes qh, 16 int8 scales, d: weight 128h + 32r + l
+         has the low four bits in nibble r // 2 of ql[64h + 32(r % 2) + l]
+         and the high two in bits 2r, 2r+1 of qh[32h + l]; value
+         d * scale[i // 16] * (q - 32).
 Run: python tests/golden/make_blocks.py > tests/golden/blocks.txt
 """
 from fractions import Fraction
@@ -53,6 +64,48 @@ BLOCKS_Q5_0 = [
 ]
 
 
+# name, d bits, d exact, dmin bits, dmin exact, scales[8], mins[8], codes[256]
+BLOCKS_Q4K = [
+    ("q4_k_mixed_scales", 0x3800, Fraction(1, 2), 0x3400, Fraction(1, 4),
+     [1, 2, 3, 63, 17, 40, 5, 33], [0, 1, 62, 7, 48, 3, 21, 63],
+     [(7 * i + 3) % 16 for i in range(256)]),
+    ("q4_k_negative_scale", 0xBC00, Fraction(-1), 0x4000, Fraction(2),
+     [33, 0, 16, 47, 1, 62, 31, 32], [5, 60, 0, 17, 33, 1, 48, 2],
+     [(i // 3) % 16 for i in range(256)]),
+]
+
+# name, d bits, d exact, scales[16] (int8), codes[256] (0..63)
+BLOCKS_Q6K = [
+    ("q6_k_signed_scales", 0x3000, Fraction(1, 8),
+     [1, -1, 2, -2, 127, -128, 3, 5, -7, 9, 11, -13, 64, -64, 0, 100],
+     [(5 * i + 1) % 64 for i in range(256)]),
+    ("q6_k_subnormal", 0x0001, Fraction(1, 2 ** 24), [-1] * 16, [i % 64 for i in range(256)]),
+]
+
+
+def pack_q4k(dbits, mbits, sc, mn, codes):
+    b = _le16(dbits) + _le16(mbits)
+    s12 = [0] * 12
+    for j in range(4):
+        s12[j] = (sc[j] & 63) | ((sc[j + 4] >> 4) << 6)
+        s12[j + 4] = (mn[j] & 63) | ((mn[j + 4] >> 4) << 6)
+        s12[j + 8] = (sc[j + 4] & 15) | ((mn[j + 4] & 15) << 4)
+    qs = [0] * 128
+    for c in range(4):
+        for l in range(32):
+            qs[32 * c + l] = codes[64 * c + l] | (codes[64 * c + 32 + l] << 4)
+    return bytes(b + s12 + qs)
+
+
+def pack_q6k(dbits, scales, codes):
+    ql, qh = [0] * 128, [0] * 64
+    for i, q in enumerate(codes):
+        h, r, l = i // 128, (i % 128) // 32, i % 32
+        ql[64 * h + 32 * (r % 2) + l] |= (q & 15) << (4 * (r // 2))
+        qh[32 * h + l] |= (q >> 4) << (2 * r)
+    return bytes(ql + qh + [v & 0xFF for v in scales] + _le16(dbits))
+
+
 def _le16(v):
     return [v & 0xFF, v >> 8]
 
@@ -80,7 +133,7 @@ def pack(qtype, dbits, codes, mbits=None):
 
 
 def main():
-    print("# Hand-packed ggml blocks: name qtype hex-bytes then 32 exact values.")
+    print("# Hand-packed ggml blocks: name qtype hex-bytes then the exact values (32 or 256).")
     print("# Derivation and layout: see make_blocks.py beside this file.")
     def emit(name, qt, raw, vals):
         print(name, qt, raw.hex(), " ".join(repr(float(v)) for v in vals))
@@ -99,6 +152,16 @@ def main():
         top = 16 if qt == "q4_1" else 32
         assert len(codes) == 32 and all(0 <= c < top for c in codes)
         emit(name, qt, pack(qt, dbits, codes, mbits), [c * d + m for c in codes])
+    for name, dbits, d, mbits, dmin, sc, mn, codes in BLOCKS_Q4K:
+        assert len(codes) == 256 and all(0 <= c < 16 for c in codes)
+        assert all(0 <= v < 64 for v in sc + mn)
+        vals = [d * sc[i // 32] * codes[i] - dmin * mn[i // 32] for i in range(256)]
+        emit(name, "q4_k", pack_q4k(dbits, mbits, sc, mn, codes), vals)
+    for name, dbits, d, scales, codes in BLOCKS_Q6K:
+        assert len(codes) == 256 and all(0 <= c < 64 for c in codes)
+        assert all(-128 <= v < 128 for v in scales)
+        vals = [d * scales[i // 16] * (codes[i] - 32) for i in range(256)]
+        emit(name, "q6_k", pack_q6k(dbits, scales, codes), vals)
 
 
 if __name__ == "__main__":

@@ -55,16 +55,19 @@ def _golden_blocks():
                          ids=[b[0] for b in _golden_blocks()])
 def test_dequant_hand_packed_blocks(orc, name, qtype, raw, vals):
     assert len(raw) == S.BLOCK_BYTES[qtype] == orc.block_bytes(qtype)
-    got = orc.dequant_row(np.frombuffer(raw, np.uint8), qtype, 32)
+    n = S.BLOCK_WEIGHTS[qtype]
+    assert len(vals) == n == orc.block_weights(qtype)
+    got = orc.dequant_row(np.frombuffer(raw, np.uint8), qtype, n)
     np.testing.assert_array_equal(got, vals)
 
 
-@pytest.mark.parametrize("qtype", ["q8_0", "q4_0", "q4_1", "q5_0", "q5_1"])
+@pytest.mark.parametrize("qtype", ["q8_0", "q4_0", "q4_1", "q5_0", "q5_1", "q4_k", "q6_k"])
 def test_dequant_row_of_several_blocks_keeps_block_order(orc, qtype):
     blocks = [b for b in _golden_blocks() if b[1] == qtype]
     assert len(blocks) >= 2
     raw = b"".join(b[2] for b in blocks)
-    got = orc.dequant_row(np.frombuffer(raw, np.uint8), qtype, 32 * len(blocks))
+    got = orc.dequant_row(np.frombuffer(raw, np.uint8), qtype,
+                          S.BLOCK_WEIGHTS[qtype] * len(blocks))
     np.testing.assert_array_equal(got, np.concatenate([b[3] for b in blocks]))
 
 
@@ -132,6 +135,36 @@ def test_q5_0_largest_weight_lands_on_code_zero(orc):
             assert code == 0
             d16 = float(packed[r, b, :2].copy().view(np.float16)[0])
             assert deq[r, b, i] == -16 * d16
+
+
+@pytest.mark.parametrize("qtype", ["q4_k", "q6_k"])
+def test_k_quant_encoder_roundtrip_bound(orc, qtype):
+    # encoder (input generator) + decoder (oracle).  Q6_K: |w - v| <= |d sc|/2
+    # where the code does not clip; Q4_K: <= d sc/2 inside the sub-block's
+    # range, and in any case <= d sc/2 + 7.5 d + dmin/2 (rounding the scale
+    # and the min to integers moves the range's ends by at most that); fp16
+    # slack on top
+    rng = np.random.default_rng(17)
+    w = (rng.standard_normal((8, 512)) * 0.02).astype(np.float32)
+    w[2, 256:512] = 0.0                                     # an all-zero super-block
+    packed = S.quantize(w, qtype)
+    deq = orc.dequant_matrix(packed, qtype, 512)
+    blk = packed.reshape(8, 2, S.BLOCK_BYTES[qtype])
+    if qtype == "q4_k":
+        d = blk[..., 0:2].copy().view(np.float16)[..., 0].astype(np.float64)
+        dmin = blk[..., 2:4].copy().view(np.float16)[..., 0].astype(np.float64)
+        # d sc/2 <= 31.5 d for sc <= 63
+        bound = np.repeat(39.5 * d + 0.5 * dmin, 256, axis=1) + 2.0 ** -9 * np.abs(w) + 1e-9
+        assert np.all(np.abs(deq - w) <= bound)
+    else:
+        d = blk[..., 208:210].copy().view(np.float16)[..., 0].astype(np.float64)
+        sc = blk[..., 192:208].copy().view(np.int8).astype(np.float64)     # [8, 2, 16]
+        eff = np.abs(d[..., None] * sc).reshape(8, 32)
+        step = np.repeat(eff, 16, axis=1)
+        assert np.all(np.abs(deq - w) <= np.maximum(0.5 * step, np.abs(w) - 31 * step)
+                      + 2.0 ** -9 * np.abs(w) + 1e-9)
+    assert np.all(deq[2, 256:512] == 0.0)
+    assert np.abs(deq - w).max() < 0.25 * np.abs(w).max()
 
 
 def test_q4_0_largest_weight_lands_on_code_zero(orc):
@@ -244,15 +277,47 @@ def _textbook_swiglu(x, Wg, Wu, Wd):
 # integer value range of each type at scale 1 (and, for the _1 types, the
 # fp16 minimum m = -8 / -16 that centres it), and the code offset
 _INT_RANGE = {"q8_0": (-20, 21), "q4_0": (-8, 8), "q4_1": (-8, 8),
-              "q5_0": (-16, 16), "q5_1": (-16, 16)}
+              "q5_0": (-16, 16), "q5_1": (-16, 16), "q4_k": (-8, 8), "q6_k": (-32, 32)}
 _CODE_OFF = {"q4_0": 8, "q4_1": 8, "q5_0": 16, "q5_1": 16}
 _MIN_BITS = {"q4_1": 0xC800, "q5_1": 0xCC00}      # fp16 -8.0, -16.0
+
+
+def _pack_int_matrix_k(codes, qtype):
+    """K-quant packing of an integer matrix, by the format definition: Q4_K
+    with d = dmin = 1, every sub-block scale 1 and min 8 (value = code - 8);
+    Q6_K with d = 1 and every scale 1 (value = code - 32)."""
+    rows, cols = codes.shape
+    nsb = cols // 256
+    c = codes.reshape(rows, nsb, 256).astype(np.int64)
+    out = np.zeros((rows, nsb, S.BLOCK_BYTES[qtype]), np.uint8)
+    if qtype == "q4_k":
+        q = c + 8
+        assert q.min() >= 0 and q.max() < 16
+        out[..., 0:4] = [0x00, 0x3C, 0x00, 0x3C]              # d = dmin = 1.0
+        out[..., 4:8] = 1                                      # sc_0..3 = 1
+        out[..., 8:12] = 8                                     # m_0..3 = 8
+        out[..., 12:16] = 1 | (8 << 4)                         # sc_4..7 = 1, m_4..7 = 8
+        for ch in range(4):
+            out[..., 16 + 32 * ch:16 + 32 * ch + 32] = (
+                q[..., 64 * ch:64 * ch + 32] | (q[..., 64 * ch + 32:64 * ch + 64] << 4))
+    else:
+        q = c + 32
+        assert q.min() >= 0 and q.max() < 64
+        for i in range(256):
+            h, r, l = i // 128, (i % 128) // 32, i % 32
+            out[..., 64 * h + 32 * (r % 2) + l] |= ((q[..., i] & 15) << (4 * (r // 2))).astype(np.uint8)
+            out[..., 128 + 32 * h + l] |= ((q[..., i] >> 4) << (2 * r)).astype(np.uint8)
+        out[..., 192:208] = 1                                  # scales = 1
+        out[..., 208:210] = [0x00, 0x3C]                       # d = 1.0
+    return out.reshape(rows, -1)
 
 
 def _pack_int_matrix(codes, qtype, dbits=0x3C00):
     """Pack an integer matrix with scale 1.0 in every block (test-side
     packing by the format definition; values = codes).  The _1 types get
     m = -offset so that code = value + offset as in their _0 twins."""
+    if qtype in ("q4_k", "q6_k"):
+        return _pack_int_matrix_k(codes, qtype)
     rows, cols = codes.shape
     nb = cols // 32
     lo = codes.reshape(rows, nb, 32).astype(np.int64)
@@ -279,20 +344,21 @@ def _pack_int_matrix(codes, qtype, dbits=0x3C00):
 def test_int_matrix_packer_agrees_with_the_golden_layouts(orc):
     # the packer above against the hand-packed golden blocks' layouts: a
     # unit-scale block of codes 0..31 (values code - offset) decodes to them
-    for qt in ("q4_0", "q4_1", "q5_0", "q5_1", "q8_0"):
+    for qt in ("q4_0", "q4_1", "q5_0", "q5_1", "q8_0", "q4_k", "q6_k"):
         lo, hi = _INT_RANGE[qt]
-        vals = np.arange(32) % (hi - lo) + lo
+        n = S.BLOCK_WEIGHTS[qt]
+        vals = (np.arange(n) * 7) % (hi - lo) + lo
         raw = _pack_int_matrix(vals[None], qt)
         assert raw.shape[1] == S.BLOCK_BYTES[qt]
-        np.testing.assert_array_equal(orc.dequant_row(raw[0], qt, 32), vals)
+        np.testing.assert_array_equal(orc.dequant_row(raw[0], qt, n), vals)
 
 
-@pytest.mark.parametrize("qtype", ["q8_0", "q4_0", "q4_1", "q5_0", "q5_1"])
+@pytest.mark.parametrize("qtype", ["q8_0", "q4_0", "q4_1", "q5_0", "q5_1", "q4_k", "q6_k"])
 def test_single_expert_is_textbook_swiglu(orc, qtype):
     # integer-valued weights (scale 1) so the dequantized matrices are known
     # exactly; E=1, k=1 reduces the layer to a plain SwiGLU FFN.
     rng = np.random.default_rng(11)
-    D, F = 64, 96
+    D, F = (256, 512) if qtype in ("q4_k", "q6_k") else (64, 96)
     lo, hi = _INT_RANGE[qtype]
     Wg = rng.integers(lo, hi, (F, D))
     Wu = rng.integers(lo, hi, (F, D))
