@@ -43,6 +43,7 @@ the oracle besides the cpu_baseline leg.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -187,16 +188,33 @@ WORKLOADS = {
 }
 
 
+# the other block types (the rest of the Standard family, the K-quants), each
+# on the decode and prefill layer shapes: workload "<decode|prefill>_<type>",
+# the configuration with its experts encoded in that type
+STD_TYPES = ("q4_1", "q5_0", "q5_1", "q4_k", "q6_k")
+STD_WORKLOADS = [f"{c}_{q}" for q in STD_TYPES for c in ("decode", "prefill")]
+
+
+def workload_spec(name):
+    """(layer configuration, T per call, pool replicas) of a workload name."""
+    if name in WORKLOADS:
+        Ts, replicas = WORKLOADS[name]
+        return S.CONFIGS[name.split("_")[0]], Ts, replicas
+    base, qt = name.split("_", 1)
+    if base not in ("decode", "prefill") or qt not in STD_TYPES:
+        raise ValueError(f"unknown workload {name}")
+    Ts, replicas = WORKLOADS[base]
+    return dataclasses.replace(S.CONFIGS[base], qtype=qt, name=name), Ts, replicas
+
+
 class Workload:
     """A list of layer calls making one step; replicas rotate per call."""
 
     def __init__(self, name: str, torch, moe, n_replicas=0, base=None):
         self.name = name
         self.torch, self.moe = torch, moe
-        cfg_name = name.split("_")[0]
-        cfg = S.CONFIGS[cfg_name]
+        cfg, Ts, replicas = workload_spec(name)
         self.cfg = cfg
-        Ts, replicas = WORKLOADS[name]
         if n_replicas:     # fewer replicas: a small case for profilers (weights may hit L2)
             replicas = int(n_replicas)
         self.Ts = Ts
@@ -221,8 +239,8 @@ class Workload:
         shared = None
         if base.shared is not None:
             sg, su, sd = (dev(a) for a in base.shared)
-            shared = moe.ExpertPool(sg, su, sd, "q8_0")
-            self.shared_bytes = sum(S.expert_bytes(cfg.D, cfg.shared_F, "q8_0"))
+            shared = moe.ExpertPool(sg, su, sd, cfg.shared_qtype)
+            self.shared_bytes = sum(S.expert_bytes(cfg.D, cfg.shared_F, cfg.shared_qtype))
         else:
             self.shared_bytes = 0
         xdt = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
@@ -273,7 +291,8 @@ class Workload:
         cfg = self.cfg
         distinct = self.distinct_experts()
         gb, ub, db = S.expert_bytes(cfg.D, cfg.F, cfg.qtype)
-        sg, su, sd = (S.expert_bytes(cfg.D, cfg.shared_F, "q8_0") if cfg.shared_F else (0, 0, 0))
+        sg, su, sd = (S.expert_bytes(cfg.D, cfg.shared_F, cfg.shared_qtype) if cfg.shared_F
+                      else (0, 0, 0))
         act = 2 if cfg.x_dtype == "bf16" else 4
         yb = 2 if cfg.y_dtype == "bf16" else 4
         per_call = {}
@@ -434,7 +453,8 @@ def dtype_of(cfg):
 def config_of(wl):
     cfg = wl.cfg
     c = {"workload": f"{wl.name}: MoE layer D={cfg.D} E={cfg.E} top-{cfg.k} F={cfg.F} "
-                     f"{cfg.qtype.upper()}" + (f" + shared F={cfg.shared_F} Q8_0" if cfg.shared_F else "")
+                     f"{cfg.qtype.upper()}"
+                     + (f" + shared F={cfg.shared_F} {cfg.shared_qtype.upper()}" if cfg.shared_F else "")
                      + f", T per call {list(wl.Ts)}",
          "tokens_per_step": wl.tokens_per_step,
          "l2": f"{len(wl.layers)} rotating replicas of the expert pool "
@@ -458,7 +478,7 @@ def roofline(wl, algo, durs, peaks, steps):
     bytes_step = sum(algo[T]["seg_bytes"].get(dom, 0) for T in wl.Ts)
     tflops = flops_step * steps / (tot[dom] / 1e3) / 1e12
     gbs = bytes_step * steps / (tot[dom] / 1e3) / 1e9
-    if wl.name in TENSOR_BOUND and dom in ("gateup", "down"):
+    if wl.name.split("_")[0] in TENSOR_BOUND and dom in ("gateup", "down"):
         bound, achieved, peak, unit, spec = "tensor", tflops, peaks["bf16_tflops"], "TFLOP/s", TC_SPEC_TFLOPS
         psrc = "bf16_tflops burst (fp16 operands run at the bf16 rate)"
         work = flops_step
@@ -493,7 +513,7 @@ def roofline(wl, algo, durs, peaks, steps):
 
 
 # the source files whose code runs in each traced segment's kernels
-SEGMENT_SOURCES = {"ffn_decode": ("ffn_decode.cu", "sm100.cuh"),
+SEGMENT_SOURCES = {"ffn_decode": ("ffn_decode.cu", "sm100.cuh", "moe_internal.cuh"),
                    "gateup": ("ffn_prefill.cu", "sm100.cuh", "moe_internal.cuh"),
                    "down": ("ffn_prefill.cu", "sm100.cuh", "moe_internal.cuh")}
 
@@ -965,7 +985,7 @@ def _line(out, args, world, cfg, peaks):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": out["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": dtype_of(cfg),
-            "data": "synthetic (seeded; random-init Q4_0/Q8_0 experts, no checkpoint)"}
+            "data": "synthetic (seeded; random-init experts in ggml Standard blocks, no checkpoint)"}
     for k, v in out.items():
         if k not in line:
             line[k] = v
@@ -976,6 +996,35 @@ def _line(out, args, world, cfg, peaks):
 # the other configurations of the default run: (key, workload)
 EXTRA = [("tiny", "tiny"), ("prefill", "prefill"), ("wide_t1", "wide_t1"),
          ("wide_t2048", "wide_t2048")]
+
+
+def std_base(cfg_name, qtype, pool):
+    """Inputs of the decode or prefill configuration (T = its largest call)
+    over a given expert pool."""
+    cfg, Ts, _ = workload_spec(f"{cfg_name}_{qtype}")
+    L = S.make_layer(cfg, T=max(Ts), experts=False)
+    L.gate, L.up, L.down = pool
+    return L
+
+
+def measure_std_types(torch, moe, steps, warmup, world, local, peaks, no_graph, cpu):
+    """The decode and prefill layers with experts in Q4_1, Q5_0, Q5_1, Q4_K
+    and Q6_K: one expert pool per type (the decode shape's weights, encoded
+    in that type), each workload with its own roofline and end-to-end
+    number (Q6_K runs the portable kernels)."""
+    out = {}
+    for qt in STD_TYPES:
+        cfg = S.CONFIGS["decode"]
+        pool = S.gen_expert_pool(cfg.seed, cfg.E, cfg.D, cfg.F, qt, cfg.expert_std)
+        for c in ("decode", "prefill"):
+            name = f"{c}_{qt}"
+            w = Workload(name, torch, moe, base=std_base(c, qt, pool))
+            out[name] = measure_layer(w, steps, warmup, world, local, peaks, no_graph, cpu=cpu,
+                                      cpu_seconds=3.0)
+            del w
+            torch.cuda.empty_cache()
+        del pool
+    return out
 
 
 def run_ours(args, world, rank, local):
@@ -1014,6 +1063,10 @@ def run_ours(args, world, rank, local):
                                                  args.no_graph, cpu=with_cpu, cpu_seconds=6.0)
             del w
             torch.cuda.empty_cache()
+        line["configs"]["standard_types"] = measure_std_types(torch, moe, steps, args.warmup,
+                                                              world, local, peaks, args.no_graph,
+                                                              with_cpu)
+        torch.cuda.empty_cache()
         line["configs"]["prefill_stream"] = measure_prefill_stream(
             torch, moe, bases["prefill"], args.steps, args.warmup, peaks, cpu=with_cpu)
         torch.cuda.empty_cache()
@@ -1039,7 +1092,7 @@ def oracle_step_fn(wl_inputs, cfg, Ts, frac=1.0):
             m = max(1, int(round(T * frac)))
             toks = np.arange(m, dtype=np.int32)
             oracle.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F, shared=L.shared,
-                         tokens=toks)
+                         tokens=toks, shared_qtype=cfg.shared_qtype)
             n += m
         return n
     return step
@@ -1104,11 +1157,10 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     name = args.workload
-    cfg = S.CONFIGS[name.split("_")[0]]
     if name == "cache":
         run_reference_cache(args, world)
         return
-    Ts = WORKLOADS[name][0]
+    cfg, Ts, _ = workload_spec(name)
     base = S.make_layer(cfg, T=max(Ts))
     inputs = {max(Ts): base}
     for T in Ts:
@@ -1158,7 +1210,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["cache"], default="decode",
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + STD_WORKLOADS + ["cache"],
+                    default="decode",
                     help="the workload of the line (decode also reports every other one under "
                          "'configs' unless --no-extra)")
     ap.add_argument("--cache-layers", type=int, default=0,

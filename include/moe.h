@@ -11,11 +11,30 @@
  *   Y[t,j]  = W_down,e ( silu(W_gate,e x_t) * (W_up,e x_t) ),  e = S_tj
  *   y_t     = sum_j g[t,j] Y[t,j]  (+ shared expert, weight 1)
  *
- * Weight formats: the ggml Standard-family types Q4_0 and Q8_0 named in the
- * FreeToken fork README, "Quant types" table.  32 weights per block with
- * one fp16 scale d: Q8_0 = {fp16 d; int8 q[32]} (34 B), value q*d;
- * Q4_0 = {fp16 d; uint8 qs[16]} (18 B), value (q-8)*d, byte j holding
- * element j in its low nibble and element j+16 in its high nibble.
+ * Weight formats: the ggml Standard-family types Q4_0, Q4_1, Q5_0, Q5_1 and
+ * Q8_0 named in the FreeToken fork README, "Quant types" table (the page
+ * names the types; the byte layouts are ggml's published ones).  32 weights
+ * per block, an fp16 scale d and, for the _1 types, an fp16 minimum m; all
+ * fields little endian:
+ *   Q8_0 = {fp16 d; int8 q[32]}                       (34 B) value q*d
+ *   Q4_0 = {fp16 d; uint8 qs[16]}                     (18 B) value (q-8)*d
+ *   Q4_1 = {fp16 d; fp16 m; uint8 qs[16]}             (20 B) value q*d + m
+ *   Q5_0 = {fp16 d; uint8 qh[4]; uint8 qs[16]}        (22 B) value (q-16)*d
+ *   Q5_1 = {fp16 d; fp16 m; uint8 qh[4]; uint8 qs[16]} (24 B) value q*d + m
+ * qs byte j holds the low four bits of element j (low nibble) and of element
+ * j+16 (high nibble); bit i of the 32-bit word qh is bit 4 of element i.
+ * K-quants (the same table, K-quants row; ggml's published layouts), 256
+ * weights per block:
+ *   Q4_K = {fp16 d; fp16 dmin; uint8 scales[12]; uint8 qs[128]}  (144 B):
+ *          eight 32-weight sub-blocks j with 6-bit scale sc_j and min m_j
+ *          (j < 4: low six bits of scales[j], scales[j+4]; j >= 4: low and
+ *          high nibble of scales[j+4] plus the top two bits of scales[j-4]
+ *          and scales[j]); value d*sc_j*q - dmin*m_j; weight 64c+l is the
+ *          low nibble of qs[32c+l], weight 64c+32+l its high nibble.
+ *   Q6_K = {uint8 ql[128]; uint8 qh[64]; int8 scales[16]; fp16 d} (210 B):
+ *          value d*scales[i/16]*(q_i - 32); weight 128h+32r+l has its low
+ *          four bits in nibble r/2 of ql[64h+32(r%2)+l] and its high two in
+ *          bits 2r, 2r+1 of qh[32h+l].
  * Expert pool (FreeToken fork README, "Known limits"): one allocation per
  * matrix kind, experts back to back as slot * nrows * (ncols / 32) blocks,
  * no padding, ONE quant type for the whole pool.  Per slot:
@@ -36,8 +55,9 @@
  *    be zero-filled once before its first use; every call leaves it in a
  *    state the next call accepts.  Calls that share a workspace must be
  *    ordered (same stream, or synchronised).
- *  - Shapes: D % 32 == 0, F % 32 == 0 (blocks run along the reduction
- *    dimension), 1 <= k <= E <= MOE_MAX_EXPERTS, k <= MOE_MAX_TOPK, T >= 0.
+ *  - Shapes: D and F multiples of the block (32 weights; 256 for the
+ *    K-quants: blocks run along the reduction dimension), 1 <= k <= E <=
+ *    MOE_MAX_EXPERTS, k <= MOE_MAX_TOPK, T >= 0.
  *    T == 0 is a no-op that succeeds.
  *  - Errors found on the GPU (a bounded wait inside a kernel that ran out,
  *    an expert whose slot is outside [0, n_slots)) cannot be returned by the
@@ -47,8 +67,10 @@
  *    MOE_DEV_OK.  A kernel that records an error skips the work it concerns
  *    and returns; the outputs that work would have written are unspecified,
  *    every other output is exact.
- *  - Numerics: activations (x) and the hidden rows h are rounded to fp16
- *    inside the FFN kernels (bf16 has 8 significant bits, fp16 11, so a bf16
+ *  - Numerics: the decode kernels apply block scales (and minimums) to fp32
+ *    partial sums of exact codes; the tensor-core kernels round each weight
+ *    to fp16 (Q4_K: its sub-block scale and minimum first).  Activations (x)
+ *    and the hidden rows h are rounded to fp16 inside the FFN kernels (bf16 has 8 significant bits, fp16 11, so a bf16
  *    x in fp16's normal range [2^-14, 65504] converts exactly).  Inputs
  *    with |x| > 65504 overflow to inf and values under 2^-14 lose bits;
  *    keep activations inside that range (post-normalisation hidden states
@@ -68,14 +90,20 @@ extern "C" {
 
 #define MOE_QK 32
 #define MOE_Q4_0_BLOCK_BYTES 18
+#define MOE_Q4_1_BLOCK_BYTES 20
+#define MOE_Q5_0_BLOCK_BYTES 22
+#define MOE_Q5_1_BLOCK_BYTES 24
 #define MOE_Q8_0_BLOCK_BYTES 34
+#define MOE_QK_K 256
+#define MOE_Q4_K_BLOCK_BYTES 144
+#define MOE_Q6_K_BLOCK_BYTES 210
 #define MOE_MAX_EXPERTS 1024
 #define MOE_MAX_TOPK 32
 
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1,        /* null pointer, bad enum, bad flag */
-    MOE_ERR_UNSUPPORTED_QTYPE = 2,  /* quant type not Q4_0 / Q8_0, or mixed */
+    MOE_ERR_UNSUPPORTED_QTYPE = 2,  /* quant type not one of moe_qtype */
     MOE_ERR_SHAPE = 3,              /* a size rule above is broken */
     MOE_ERR_CUDA = 4,               /* a CUDA runtime call failed */
     MOE_ERR_CAPACITY = 5,           /* more experts requested than cache slots */
@@ -94,7 +122,10 @@ typedef enum {
 } moe_device_status;
 
 /* ggml type ids */
-typedef enum { MOE_Q4_0 = 2, MOE_Q8_0 = 8 } moe_qtype;
+typedef enum {
+    MOE_Q4_0 = 2, MOE_Q4_1 = 3, MOE_Q5_0 = 6, MOE_Q5_1 = 7, MOE_Q8_0 = 8,
+    MOE_Q4_K = 12, MOE_Q6_K = 14
+} moe_qtype;
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_F16 = 2 } moe_dtype;
 
@@ -119,8 +150,11 @@ typedef struct {
 /* ---------------------------------------------------------------- misc */
 const char *moe_last_error(void);
 const char *moe_version(void);
-/* Bytes of one 32-weight block of a quant type; 0 for an unknown type. */
+/* Bytes of one block of a quant type; 0 for an unknown type. */
 int moe_block_bytes(int32_t qtype);
+/* Weights of one block of a quant type (32, or 256 for the K-quants); 0 for
+ * an unknown type. */
+int moe_block_weights(int32_t qtype);
 
 /* moe_workspace_status: the device status word of a workspace (its first
  * int32, written by the kernels of the calls that used it; see the
@@ -208,7 +242,9 @@ moe_status moe_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
  *     the dequant-fused grouped GEMV (mma.sync, TMA-streamed weights);
  *   T > 16, D % 256 == 0, F % 256 == 0, E <= 720: the grouped GEMM on the
  *     tcgen05 tensor cores (weights dequantised to fp16 in shared memory);
- *   any other shape: a portable CUDA-core kernel (correct, not tuned).
+ *   any other shape, and Q6_K on every shape: a portable CUDA-core kernel
+ *     (correct, not tuned; Q6_K rows of 768 weights are 630 bytes, which
+ *     tensor copies cannot address).
  *   x           device [T, D], x_dtype F32 or BF16.
  *   perm,offsets from moe_permute.
  *   pool        expert weights (see moe_pool); pool->qtype fixes the format.
@@ -249,7 +285,7 @@ moe_status moe_combine(const float *rows, const int32_t *inv, const float *gates
  *   w_router, bias       as moe_route; w_router NULL -> logits_in is used
  *   logits_in            device fp32 [T, E] or NULL
  *   pool                 routed experts
- *   shared               NULL or a pool with one slot (Q8_0 or Q4_0) of a
+ *   shared               NULL or a pool with one slot (any moe_qtype) of a
  *                        SwiGLU expert with F = shared_F, added with weight 1
  *   y, y_dtype           device [T, D] output (F32 or BF16)
  *   ids_out, gates_out   device [T, k] or NULL: routing decisions

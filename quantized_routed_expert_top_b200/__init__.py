@@ -17,10 +17,12 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 # enums of include/moe.h
 MOE_OK = 0
-Q4_0, Q8_0 = 2, 8
+Q4_0, Q4_1, Q5_0, Q5_1, Q8_0, Q4_K, Q6_K = 2, 3, 6, 7, 8, 12, 14
 F32, BF16, F16 = 0, 1, 2
-QTYPES = {"q4_0": Q4_0, "q8_0": Q8_0}
-BLOCK_BYTES = {Q4_0: 18, Q8_0: 34}
+QTYPES = {"q4_0": Q4_0, "q4_1": Q4_1, "q5_0": Q5_0, "q5_1": Q5_1, "q8_0": Q8_0,
+          "q4_k": Q4_K, "q6_k": Q6_K}
+BLOCK_BYTES = {Q4_0: 18, Q4_1: 20, Q5_0: 22, Q5_1: 24, Q8_0: 34, Q4_K: 144, Q6_K: 210}
+BLOCK_WEIGHTS = {q: (256 if q in (Q4_K, Q6_K) else 32) for q in BLOCK_BYTES}
 _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_QTYPE",
           3: "MOE_ERR_SHAPE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_CAPACITY",

@@ -42,7 +42,7 @@ int num_sms() {
     return cached[dev];
 }
 
-static bool qtype_ok(int q) { return q == MOE_Q4_0 || q == MOE_Q8_0; }
+static bool qtype_ok(int q) { return qt_known(q); }
 static bool act_dtype_ok(int d) { return d == MOE_F32 || d == MOE_BF16; }
 
 static moe_status check_shapes(const char *fn, int T, int D, int F, int E, int k) {
@@ -66,7 +66,8 @@ static moe_status check_shapes(const char *fn, int T, int D, int F, int E, int k
 static moe_status check_pool(const char *fn, const moe_pool *p, int E) {
     if (!p) { set_error("%s: pool is NULL", fn); return MOE_ERR_INVALID_ARG; }
     if (!qtype_ok(p->qtype)) {
-        set_error("%s: unsupported quant type %d (Q4_0=2, Q8_0=8)", fn, (int)p->qtype);
+        set_error("%s: unsupported quant type %d (Q4_0=2, Q4_1=3, Q5_0=6, Q5_1=7, Q8_0=8)", fn,
+                  (int)p->qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }
     if (!p->gate || !p->up || !p->down || p->n_slots <= 0) {
@@ -75,6 +76,18 @@ static moe_status check_pool(const char *fn, const moe_pool *p, int E) {
     }
     if (!p->slot_of_expert && p->n_slots < E) {
         set_error("%s: pool without a slot map holds %d slots for %d experts", fn, (int)p->n_slots, E);
+        return MOE_ERR_SHAPE;
+    }
+    return MOE_OK;
+}
+
+// D and F must hold whole blocks of the pool's type (256 weights for the
+// K-quants)
+static moe_status check_block_shape(const char *fn, const moe_pool *p, int D, int F) {
+    const int bw = qt_weights(p->qtype);
+    if (D % bw || F % bw) {
+        set_error("%s: D=%d and F=%d must be multiples of %d for quant type %d", fn, D, F, bw,
+                  (int)p->qtype);
         return MOE_ERR_SHAPE;
     }
     return MOE_OK;
@@ -91,12 +104,10 @@ const char *moe_last_error(void) { return g_err.c_str(); }
 const char *moe_version(void) { return "libmoe 0.1 (sm_100a)"; }
 
 int moe_block_bytes(int32_t qtype) {
-    switch (qtype) {
-    case MOE_Q4_0: return MOE_Q4_0_BLOCK_BYTES;
-    case MOE_Q8_0: return MOE_Q8_0_BLOCK_BYTES;
-    default: return 0;
-    }
+    return qt_bytes(qtype);
 }
+
+int moe_block_weights(int32_t qtype) { return qt_weights(qtype); }
 
 // ------------------------------------------------------ device status word
 moe_status moe_workspace_status(void *workspace, int32_t *code, int clear, moe_stream stream) {
@@ -176,25 +187,28 @@ moe_status moe_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
 // ------------------------------------------------------------ expert FFN
 // Workspace pieces of moe_expert_ffn: the status word, then the decode
 // path's fp16 hidden rows, or the tensor-core path's fp16 activations and
-// hidden rows, or the portable path's fp32 hidden rows.  E is not an
-// argument of the size query, so for T > 16 it covers both of the latter.
+// hidden rows, or the portable path's fp32 hidden rows.  Neither E nor the
+// quant type is an argument of the size query, so it covers every path the
+// shape admits (the portable one always).
 size_t moe_expert_ffn_workspace_size(int T, int k, int D, int F) {
     T = T < 0 ? 0 : T;
     Carver c(nullptr, 0);
     c.take<int>(16);
-    if (decode_path_ok(T, D, F, 0)) {
-        c.take<__half>(decode_hs_halves(T, k, F, 0));
-        return c.off;
-    }
     Carver g = c;
     g.take<float>((size_t)T * k * F);
+    size_t need = g.off;
+    if (decode_path_ok(T, D, F, 0, MOE_Q4_0, 0)) {
+        Carver d = c;
+        d.take<__half>(decode_hs_halves(T, k, F, 0));
+        need = d.off > need ? d.off : need;
+    }
     if (T > 16 && D % 256 == 0 && F % 256 == 0) {
         Carver p = c;
         p.take<__half>(prefill_x16_halves(T, D));
         p.take<__half>(prefill_h_halves(T, k, F, 0));
-        return p.off > g.off ? p.off : g.off;
+        need = p.off > need ? p.off : need;
     }
-    return g.off;
+    return need;
 }
 
 moe_status moe_expert_ffn(const void *x, int32_t x_dtype, int T, int D, int F, int E, int k,
@@ -205,6 +219,7 @@ moe_status moe_expert_ffn(const void *x, int32_t x_dtype, int T, int D, int F, i
     moe_status st = check_shapes("moe_expert_ffn", T, D, F, E, k);
     if (st != MOE_OK) return st;
     if ((st = check_pool("moe_expert_ffn", pool, E)) != MOE_OK) return st;
+    if ((st = check_block_shape("moe_expert_ffn", pool, D, F)) != MOE_OK) return st;
     if (!act_dtype_ok(x_dtype)) { set_error("moe_expert_ffn: x dtype %d not F32/BF16", x_dtype); return MOE_ERR_INVALID_ARG; }
     if (T == 0) return MOE_OK;
     if (!x || !perm || !offsets || !out_rows) { set_error("moe_expert_ffn: NULL x, perm, offsets or out_rows"); return MOE_ERR_INVALID_ARG; }
@@ -215,13 +230,13 @@ moe_status moe_expert_ffn(const void *x, int32_t x_dtype, int T, int D, int F, i
     }
     Carver c(workspace, ws_bytes);
     int *status = c.take<int>(16);
-    if (decode_path_ok(T, D, F, 0)) {
+    if (decode_path_ok(T, D, F, 0, pool->qtype, 0)) {
         __half *Hs = c.take<__half>(decode_hs_halves(T, k, F, 0));
         return launch_ffn_decode(x, x_dtype, T, D, F, E, k, perm, nullptr, offsets, nullptr, *pool,
                                  expert_mask, true, nullptr, 0, false, Hs, nullptr, MOE_F32,
                                  out_rows, status, (cudaStream_t)stream, nullptr);
     }
-    if (prefill_path_ok(T, D, F, 0, E)) {
+    if (prefill_path_ok(T, D, F, 0, E, pool->qtype, 0)) {
         __half *x16 = c.take<__half>(prefill_x16_halves(T, D));
         __half *H16 = c.take<__half>(prefill_h_halves(T, k, F, 0));
         return launch_ffn_prefill(x, x_dtype, T, D, F, E, k, perm, offsets, *pool, expert_mask,
@@ -261,12 +276,15 @@ moe_status moe_layer_forward(const moe_layer_args *a, void *workspace, size_t ws
     moe_status st = check_shapes("moe_layer_forward", a->T, D_eff, a->F, a->E, a->k);
     if (st != MOE_OK) return st;
     if ((st = check_pool("moe_layer_forward", a->pool, a->E)) != MOE_OK) return st;
+    if ((st = check_block_shape("moe_layer_forward", a->pool, a->D, a->F)) != MOE_OK) return st;
     if (a->shared) {
         if ((st = check_pool("moe_layer_forward (shared)", a->shared, 1)) != MOE_OK) return st;
         if (a->shared_F <= 0 || a->shared_F % QK) {
             set_error("moe_layer_forward: shared_F=%d must be a positive multiple of 32", a->shared_F);
             return MOE_ERR_SHAPE;
         }
+        if ((st = check_block_shape("moe_layer_forward (shared)", a->shared, a->D, a->shared_F)) != MOE_OK)
+            return st;
     }
     if (!act_dtype_ok(a->x_dtype)) { set_error("moe_layer_forward: x dtype %d not F32/BF16", a->x_dtype); return MOE_ERR_INVALID_ARG; }
     if (a->y_dtype != MOE_F32 && a->y_dtype != MOE_BF16) {

@@ -148,7 +148,7 @@ moe_status moe_cache_init(const moe_cache_desc *desc, moe_cache **out) {
         set_error("moe_cache_init: global cache needs n_slots <= max_slots <= n_layers * E");
         return MOE_ERR_SHAPE;
     }
-    if (d.qtype != MOE_Q4_0 && d.qtype != MOE_Q8_0) {
+    if (!qt_known(d.qtype)) {
         set_error("moe_cache_init: unsupported quant type %d", (int)d.qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }

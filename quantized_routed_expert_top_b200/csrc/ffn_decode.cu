@@ -17,7 +17,11 @@
 //    constant is removed through the MMA's accumulator input: it starts at
 //    -c * sum_k x_k (per block and token, precomputed once), so the block's
 //    result is sum (q - off) x exactly up to fp32 rounding, and the block
-//    scale d multiplies that fp32 result; no weight is rounded.  A fixed-
+//    scale d multiplies that fp32 result; no weight is rounded.  The _1
+//    types (value q*d + m) add m * sum_k x_k, read from the same table.
+//    The other Standard types work the same way: 4-bit codes become
+//    1024 + q (Q4_1: off 1024; Q5_0/Q5_1 OR in the fifth bit from the
+//    block's qh word: off 1040 / 1024).  A fixed-
 //    order cross-warp sum, SwiGLU and the token's gate weight give Hs = g * h
 //    in fp16, stored in the fragment order the next kernel reads.
 //  * dec_down: work unit = (expert, 64 rows of D): one 2-D box of the
@@ -26,7 +30,9 @@
 //    Consumer warps form 4 groups of 4; a group owns every 4th unit of the
 //    CTA and a warp one 16-row M-tile of it over the whole reduction, so no
 //    partial sums cross warps.  Codes become exact (q - off) fp16 values and
-//    the block scale multiplies the fp32 MMA result.  Each warp stores its
+//    the block scale multiplies the fp32 MMA result; for the _1 types a
+//    second MMA with an all-ones A gives each column's block sum of Hs,
+//    which m multiplies.  Each warp stores its
 //    fp32 Y rows (permuted order) to global memory.
 //  * dec_combine (fused layer only): y[t] = sum over j of the Y row of
 //    (t, j), then the shared expert's row, in that fixed order; the gate
@@ -68,7 +74,7 @@ constexpr int kMaxTk = 16 * MOE_MAX_TOPK;       // T*k entries the token tables 
 
 struct DecArgs {
     int T, D, F, E, k, sF;         // sF: shared expert's F when this call runs it, else 0
-    int q8, sq8;                   // routed / shared experts are Q8_0 (else Q4_0)
+    int qt, sqt;                   // block types (ggml ids) of the routed / shared experts
     int routed;                    // this call runs the routed experts (those mask admits)
     int n_slots;                   // slots of the routed pool
     int comb_shared;               // the combine adds the shared rows (layer has one)
@@ -233,7 +239,7 @@ struct Virt {
     int seg0, cnt, Fv;
     size_t slot;
     bool shared;
-    bool q8;
+    int qt;
 };
 
 __device__ __forceinline__ Virt virt(const DecArgs &a, const int *act, int n_routed, int v) {
@@ -245,14 +251,14 @@ __device__ __forceinline__ Virt virt(const DecArgs &a, const int *act, int n_rou
         r.Fv = a.F;
         r.slot = (size_t)aslot[v];
         r.shared = false;
-        r.q8 = a.q8 != 0;
+        r.qt = a.qt;
     } else {
         r.seg0 = a.T * a.k;
         r.cnt = a.T;
         r.Fv = a.sF;
         r.slot = 0;
         r.shared = true;
-        r.q8 = a.sq8 != 0;
+        r.qt = a.sqt;
     }
     return r;
 }
@@ -294,18 +300,29 @@ __host__ __device__ __forceinline__ int frag_slot(int i) {
 // ---------------------------------------------------- code extraction
 // Exact fp16 pairs of (const + code) for the 8 weights of one row that
 // thread c owns in a block: r[0] = (v4c, v4c+2), r[1] = (v4c+1, v4c+3),
-// r[2] = (v16+4c, v18+4c), r[3] = (v17+4c, v19+4c), where
-// v = 1024 + q (Q4_0, 0 <= q < 16) or v = 1152 + q (Q8_0, int8 q).
-// qa: shared address of the block's first code byte + 4c.
-template <bool Q8, int MIS>
-__device__ __forceinline__ void magic_codes(uint32_t qa, uint32_t *r) {
-    if constexpr (!Q8) {
+// r[2] = (v16+4c, v18+4c), r[3] = (v17+4c, v19+4c), where v = 1024 + q for
+// the 4- and 5-bit types (0 <= q < 32) or v = 1152 + q (Q8_0, int8 q).
+// blk: shared address of the block; MIS = alignment mod 4 of its codes
+// (the 5-bit types' qh word sits 4 bytes before them: the same alignment).
+template <int QT, int MIS>
+__device__ __forceinline__ void magic_codes(uint32_t blk, int c, uint32_t *r) {
+    const uint32_t qa = blk + qt_qs_off(QT) + 4 * c;
+    if constexpr (QT != MOE_Q8_0) {
         const uint32_t w = lds_word<MIS>(qa);
         const uint32_t M = 0x000F000Fu, MAG = 0x64006400u;
         r[0] = lop3_and_or(w, M, MAG);
         r[2] = lop3_and_or(w >> 4, M, MAG);
         r[1] = lop3_and_or(w >> 8, M, MAG);
         r[3] = lop3_and_or(w >> 12, M, MAG);
+        if constexpr (qt_has_high(QT)) {
+            // bit i of qh is bit 4 of element i: for this thread, elements
+            // 4c..4c+3 and 16+4c..19+4c, into bit 4 of each half
+            const uint32_t h = lds_word<MIS>(blk + qt_qh_off(QT)) >> (4 * c);
+            r[0] |= ((h & 1u) << 4) | ((h & 4u) << 18);
+            r[1] |= ((h & 2u) << 3) | ((h & 8u) << 17);
+            r[2] |= ((h >> 12) & 0x10u) | ((h << 2) & 0x100000u);
+            r[3] |= ((h >> 13) & 0x10u) | ((h << 1) & 0x100000u);
+        }
     } else {
         const uint32_t w0 = lds_word<MIS>(qa) ^ 0x80808080u;
         const uint32_t w1 = lds_word<MIS>(qa + 16) ^ 0x80808080u;
@@ -317,12 +334,21 @@ __device__ __forceinline__ void magic_codes(uint32_t qa, uint32_t *r) {
     }
 }
 
-// offset of the magic constant in half2 form: 1032 (Q4_0) or 1152 (Q8_0)
-template <bool Q8> __device__ __forceinline__ uint32_t magic_off2() {
-    return Q8 ? 0x64806480u : 0x64086408u;
+// the magic constant minus the code of value zero: (v - off) * d is the
+// weight of a _0 type, (v - off) * d + m of a _1 type
+__host__ __device__ constexpr float magic_off(int qt) {
+    return qt == MOE_Q8_0 ? 1152.f : 1024.f + (float)qt_zero(qt);
 }
-template <bool Q8> __host__ __device__ constexpr float magic_off() { return Q8 ? 1152.f : 1032.f; }
-template <bool Q8> __host__ __device__ constexpr int qbytes() { return Q8 ? kQ8Bytes : kQ4Bytes; }
+// the same in half2 form (1024 + z is exact in fp16: z < 32)
+template <int QT> __device__ __forceinline__ uint32_t magic_off2() {
+    constexpr uint32_t h = QT == MOE_Q8_0 ? 0x6480u : 0x6400u + (uint32_t)qt_zero(QT);
+    return h | (h << 16);
+}
+// alignment mod 4 of the codes of block bl when the block group starts at
+// alignment MIS0
+template <int QT, int MIS0> __device__ __forceinline__ constexpr int codes_mis(int bl) {
+    return (MIS0 + bl * qt_bytes(QT) + qt_qs_off(QT)) & 3;
+}
 
 // ---------------------------------------------------------------- gate/up
 // One K-slice of one 16-row tile for one warp: WB blocks starting at the
@@ -330,22 +356,29 @@ template <bool Q8> __host__ __device__ constexpr int qbytes() { return Q8 ? kQ8B
 // row of column g (and g+8) at that block; sa: the -off*sum(x) entries of
 // columns 2c, 2c+1 (and +8) at that block.  MIS0 = alignment mod 4 of the
 // first block's start (the code bytes start 2 bytes later; BS is 2 mod 4).
-template <bool Q8, int NTILE, int WB, int MIS0>
+// For the _1 types the table entries are -1024 * sum(x), so m * sum(x) =
+// (-m / 1024) * entry, the scaling by a power of two being exact.
+template <int QT, int NTILE, int WB, int MIS0>
 __device__ __forceinline__ void gateup_slice(uint32_t row, uint32_t r8, const uint32_t *xa,
                                              const uint32_t (*sa)[2], int c, float (*acc)[4]) {
-    constexpr int BS = qbytes<Q8>();
+    constexpr int BS = qt_bytes(QT);
 #pragma unroll
     for (int bl = 0; bl < WB; bl++) {
         const uint32_t blk = row + bl * BS;
         uint32_t lo[4], hi[4];
-        if (((MIS0 + 2 * bl + 2) & 3) == 0) {
-            magic_codes<Q8, 0>(blk + 2 + 4 * c, lo);
-            magic_codes<Q8, 0>(blk + r8 + 2 + 4 * c, hi);
+        if (codes_mis<QT, MIS0>(bl) == 0) {
+            magic_codes<QT, 0>(blk, c, lo);
+            magic_codes<QT, 0>(blk + r8, c, hi);
         } else {
-            magic_codes<Q8, 2>(blk + 2 + 4 * c, lo);
-            magic_codes<Q8, 2>(blk + r8 + 2 + 4 * c, hi);
+            magic_codes<QT, 2>(blk, c, lo);
+            magic_codes<QT, 2>(blk + r8, c, hi);
         }
         const float dlo = h2f(lds16(blk)), dhi = h2f(lds16(blk + r8));
+        float mlo = 0.f, mhi = 0.f;
+        if constexpr (qt_has_min(QT)) {
+            mlo = h2f(lds16(blk + 2)) * (-1.f / 1024.f);
+            mhi = h2f(lds16(blk + r8 + 2)) * (-1.f / 1024.f);
+        }
         const uint32_t a0[4] = {lo[0], hi[0], lo[1], hi[1]};
         const uint32_t a1[4] = {lo[2], hi[2], lo[3], hi[3]};
 #pragma unroll
@@ -359,6 +392,81 @@ __device__ __forceinline__ void gateup_slice(uint32_t row, uint32_t r8, const ui
             acc[nt][1] = fmaf(dlo, p[1], acc[nt][1]);
             acc[nt][2] = fmaf(dhi, p[2], acc[nt][2]);
             acc[nt][3] = fmaf(dhi, p[3], acc[nt][3]);
+            if constexpr (qt_has_min(QT)) {
+                acc[nt][0] = fmaf(mlo, s0, acc[nt][0]);
+                acc[nt][1] = fmaf(mlo, s1, acc[nt][1]);
+                acc[nt][2] = fmaf(mhi, s0, acc[nt][2]);
+                acc[nt][3] = fmaf(mhi, s1, acc[nt][3]);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- Q4_K
+// Q4_K rows are runs of 144-byte blocks (16-byte aligned in a staged row):
+// unit b of a row (32 weights) is sub-block b % 8 of block b / 8.  Its codes
+// for thread c, in the fragment order above, are nibble (j & 1) of the two
+// words at bytes 4c and 16 + 4c of the block's 32-byte chunk j / 2.
+__device__ __forceinline__ void q4k_codes(uint32_t blk, int j, int c, uint32_t *r) {
+    const uint32_t qa = blk + 16 + 32 * (j >> 1) + 4 * c;
+    const int sh = 4 * (j & 1);
+    const uint32_t w0 = (lds32(qa) >> sh) & 0x0F0F0F0Fu, w1 = (lds32(qa + 16) >> sh) & 0x0F0F0F0Fu;
+    const uint32_t HI = 0x64646464u;
+    r[0] = prmt(w0, HI, 0x4240);
+    r[1] = prmt(w0, HI, 0x4341);
+    r[2] = prmt(w1, HI, 0x4240);
+    r[3] = prmt(w1, HI, 0x4341);
+}
+// Scale D = d * sc_j and min M = dmin * m_j of sub-block j (weight D q - M)
+__device__ __forceinline__ void q4k_params(uint32_t blk, int j, float *D, float *M) {
+    const uint32_t s0 = lds32(blk + 4), s1 = lds32(blk + 8), s2 = lds32(blk + 12);
+    const int jj = j & 3, sh = 8 * jj;
+    int sc, m;
+    if (j < 4) {
+        sc = (s0 >> sh) & 63;
+        m = (s1 >> sh) & 63;
+    } else {
+        sc = ((s2 >> sh) & 15) | (((s0 >> (sh + 6)) & 3) << 4);
+        m = ((s2 >> (sh + 4)) & 15) | (((s1 >> (sh + 6)) & 3) << 4);
+    }
+    *D = h2f(lds16(blk)) * (float)sc;
+    *M = h2f(lds16(blk + 2)) * (float)m;
+}
+
+// As gateup_slice for Q4_K: units kb0 .. kb0 + WB - 1 of the slice whose
+// staged row starts at rowbase.  The Sx table entries are -1024 * sum(x),
+// so the min's share -M * sum(x) is (M / 1024) * entry.
+template <int NTILE, int WB>
+__device__ __forceinline__ void gateup_slice_q4k(uint32_t rowbase, uint32_t r8, int kb0,
+                                                 const uint32_t *xa, const uint32_t (*sa)[2], int c,
+                                                 float (*acc)[4]) {
+#pragma unroll
+    for (int bl = 0; bl < WB; bl++) {
+        // WB == 8: the warp's units are one whole block (kb0 a multiple of 8)
+        const int b = kb0 + bl;
+        const int j = WB == 8 ? bl : (b & 7);
+        const uint32_t blk = rowbase + (uint32_t)((WB == 8 ? kb0 : b) >> 3) * 144u;
+        uint32_t lo[4], hi[4];
+        q4k_codes(blk, j, c, lo);
+        q4k_codes(blk + r8, j, c, hi);
+        float dlo, mlo, dhi, mhi;
+        q4k_params(blk, j, &dlo, &mlo);
+        q4k_params(blk + r8, j, &dhi, &mhi);
+        mlo *= 1.f / 1024.f;
+        mhi *= 1.f / 1024.f;
+        const uint32_t a0[4] = {lo[0], hi[0], lo[1], hi[1]};
+        const uint32_t a1[4] = {lo[2], hi[2], lo[3], hi[3]};
+#pragma unroll
+        for (int nt = 0; nt < NTILE; nt++) {
+            const uint4 b4 = lds128(xa[nt] + bl * 64);
+            const float s0 = ldsf(sa[nt][0] + bl * 4), s1 = ldsf(sa[nt][1] + bl * 4);
+            float p[4] = {s0, s1, s0, s1};
+            mma_16816(p, a0, b4.x, b4.y, p);
+            mma_16816(p, a1, b4.z, b4.w, p);
+            acc[nt][0] = fmaf(mlo, s0, fmaf(dlo, p[0], acc[nt][0]));
+            acc[nt][1] = fmaf(mlo, s1, fmaf(dlo, p[1], acc[nt][1]));
+            acc[nt][2] = fmaf(mhi, s0, fmaf(dhi, p[2], acc[nt][2]));
+            acc[nt][3] = fmaf(mhi, s1, fmaf(dhi, p[3], acc[nt][3]));
         }
     }
 }
@@ -368,8 +476,8 @@ struct GuGeo {
     int sb, nsl, pitch;                 // blocks per slice, slices, staged row pitch
 };
 // max_sb: the largest slice (in blocks) a stage may hold
-__host__ __device__ inline GuGeo gu_geo(int D, bool q8, int max_sb) {
-    const int bs = q8 ? kQ8Bytes : kQ4Bytes, nb = D / QK;
+__host__ __device__ inline GuGeo gu_geo(int D, int qt, int max_sb) {
+    const int bs = qt_unit_bytes(qt), nb = D / QK;
     GuGeo g;
     g.sb = slice_blocks_q(nb, bs, max_sb);
     g.nsl = nb / g.sb;
@@ -377,7 +485,9 @@ __host__ __device__ inline GuGeo gu_geo(int D, bool q8, int max_sb) {
     return g;
 }
 
-template <int MAXSB, int WB4, int WB8>
+// ALL: the call has a type other than Q4_0 and Q8_0 (a separate
+// instantiation keeps the other types' code out of the two types' kernel)
+template <int MAXSB, int WB4, int WB8, bool ALL>
 __global__ void __launch_bounds__(kGThreads, 1)
 dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     constexpr int NT = 1;
@@ -387,9 +497,8 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     const int T = a.T, D = a.D;
     const int nbD = D / QK;
     constexpr int kMaxSb = MAXSB;
-    const GuGeo geo4 = gu_geo(D, false, kMaxSb), geo8 = gu_geo(D, true, kMaxSb);
-    const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
-    const int pitch_max = max(any4 ? geo4.pitch : 0, any8 ? geo8.pitch : 0);
+    const GuGeo geoR = gu_geo(D, a.qt, kMaxSb), geoS = gu_geo(D, a.sqt, kMaxSb);
+    const int pitch_max = max(geoR.pitch, a.sF > 0 ? geoS.pitch : 0);
     const int stage_bytes = (int)round_up((size_t)2 * kTile * pitch_max, 128);
     const int xrow = staged_act_bytes(D);
     const int mat = warp >> 3, kg = warp & 7;
@@ -485,8 +594,8 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
             pk.w = h[17 + 4 * cc] | (h[19 + 4 * cc] << 16);
             *reinterpret_cast<uint4 *>(dst + cc * 16) = pk;
         }
-        sxt[idx] = -magic_off<false>() * sum;
-        sxt[(size_t)(T + 1) * nbD + idx] = -magic_off<true>() * sum;
+        sxt[idx] = -magic_off(a.qt) * sum;
+        sxt[(size_t)(T + 1) * nbD + idx] = -magic_off(a.sqt) * sum;
     }
     __syncthreads();
     // routing results come from the previous kernel
@@ -550,8 +659,8 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
             for (int i = 0; i < n_local && ok; i++) {
                 const int v = utab[i].x, tile = utab[i].y;
                 const Virt vi = virt(a, act, A.n_routed, v);
-                const int bs = vi.q8 ? kQ8Bytes : kQ4Bytes;
-                const GuGeo gg = vi.q8 ? geo8 : geo4;
+                const int bs = qt_unit_bytes(vi.qt);
+                const GuGeo gg = vi.shared ? geoS : geoR;
                 const CUtensorMap *mg = vi.shared ? &maps.sgate : &maps.gate;
                 const CUtensorMap *mu = vi.shared ? &maps.sup : &maps.up;
                 const int y = (vi.shared ? 0 : (int)vi.slot * a.F) + tile * kTile;
@@ -615,12 +724,13 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     for (int j = 0; j < n_local && ok; j++) {
         const int4 ud = utab[j];
         const int tile = ud.y, seg0 = ud.z, cnt = ud.w;
-        const bool q8 = ud.x < A.n_routed ? a.q8 != 0 : a.sq8 != 0;
-        const GuGeo gg = q8 ? geo8 : geo4;
-        const int kb0 = kg * (q8 ? WB8 : WB4);          // warp's first block in a slice
+        const bool shu = ud.x >= A.n_routed;
+        const int qt = shu ? a.sqt : a.qt;
+        const GuGeo gg = shu ? geoS : geoR;
+        const int kb0 = kg * (qt == MOE_Q8_0 ? WB8 : WB4);   // warp's first block in a slice
         // B rows (column g, g+8) and C columns (2c, 2c+1, +8) of this unit
         uint32_t xa[NT], sa[NT][2];
-        const uint32_t sxq = sx_a + (q8 ? (uint32_t)((T + 1) * nbD * 4) : 0u);
+        const uint32_t sxq = sx_a + (shu ? (uint32_t)((T + 1) * nbD * 4) : 0u);
 #pragma unroll
         for (int nt = 0; nt < NT; nt++) {
             const int n = g + 8 * nt;
@@ -638,7 +748,7 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
         for (int nt = 0; nt < NT; nt++)
 #pragma unroll
             for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
-        const int bsz = q8 ? kQ8Bytes : kQ4Bytes;
+        const int bsz = qt_unit_bytes(qt);
         const int mis0 = (kb0 * bsz) & 3;               // 0 or 2
         const uint32_t r8 = 8u * gg.pitch;
 
@@ -652,9 +762,20 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
                 sa_s[nt][0] = sa[nt][0] + sl * gg.sb * 4;
                 sa_s[nt][1] = sa[nt][1] + sl * gg.sb * 4;
             }
-#define MOE_GU(Q8, NTL, MIS) gateup_slice<Q8, NTL, (Q8 ? WB8 : WB4), MIS>(row, r8, xs_s, sa_s, c, acc)
-            if (!q8) { if (mis0 == 0) MOE_GU(false, 1, 0); else MOE_GU(false, 1, 2); }
-            else { if (mis0 == 0) MOE_GU(true, 1, 0); else MOE_GU(true, 1, 2); }
+#define MOE_GU(QT, MIS) gateup_slice<QT, 1, (QT == MOE_Q8_0 ? WB8 : WB4), MIS>(row, r8, xs_s, sa_s, c, acc)
+            if (!ALL || qt == MOE_Q4_0 || qt == MOE_Q8_0) {
+                if (qt == MOE_Q4_0) { if (mis0 == 0) MOE_GU(MOE_Q4_0, 0); else MOE_GU(MOE_Q4_0, 2); }
+                else { if (mis0 == 0) MOE_GU(MOE_Q8_0, 0); else MOE_GU(MOE_Q8_0, 2); }
+            } else if constexpr (ALL) {
+                switch (qt) {
+                case MOE_Q5_0: if (mis0 == 0) MOE_GU(MOE_Q5_0, 0); else MOE_GU(MOE_Q5_0, 2); break;
+                case MOE_Q4_1: MOE_GU(MOE_Q4_1, 0); break;      // 20-byte blocks: always aligned
+                case MOE_Q5_1: MOE_GU(MOE_Q5_1, 0); break;      // 24-byte blocks: always aligned
+                default:                                         // Q4_K
+                    gateup_slice_q4k<1, WB4>(row - kb0 * bsz, r8, kb0, xs_s, sa_s, c, acc);
+                    break;
+                }
+            }
 #undef MOE_GU
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
@@ -690,25 +811,33 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
 constexpr int kDnRows = 64;
 
 // 8 consecutive blocks of one 16-row tile for one warp; the block group
-// starts 4-byte aligned (8 blocks of 18 or 34 bytes).
-template <bool Q8, int NTILE>
+// starts 4-byte aligned (8 blocks of an even size).  For the _1 types the
+// all-ones A of a second MMA pair sums each Hs column over the block, and m
+// multiplies that sum.
+template <int QT, int NTILE>
 __device__ __forceinline__ void down_blocks8(uint32_t row, uint32_t r8, const uint32_t *ha, int c,
                                              float (*acc)[4]) {
-    constexpr int BS = qbytes<Q8>();
-    const uint32_t off2 = magic_off2<Q8>();
+    constexpr int BS = qt_bytes(QT);
+    const uint32_t off2 = magic_off2<QT>();
     const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t ones[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};
 #pragma unroll
     for (int bl = 0; bl < 8; bl++) {
         const uint32_t blk = row + bl * BS;
         uint32_t lo[4], hi[4];
-        if (((2 * bl + 2) & 3) == 0) {
-            magic_codes<Q8, 0>(blk + 2 + 4 * c, lo);
-            magic_codes<Q8, 0>(blk + r8 + 2 + 4 * c, hi);
+        if (codes_mis<QT, 0>(bl) == 0) {
+            magic_codes<QT, 0>(blk, c, lo);
+            magic_codes<QT, 0>(blk + r8, c, hi);
         } else {
-            magic_codes<Q8, 2>(blk + 2 + 4 * c, lo);
-            magic_codes<Q8, 2>(blk + r8 + 2 + 4 * c, hi);
+            magic_codes<QT, 2>(blk, c, lo);
+            magic_codes<QT, 2>(blk + r8, c, hi);
         }
         const float dlo = h2f(lds16(blk)), dhi = h2f(lds16(blk + r8));
+        float mlo = 0.f, mhi = 0.f;
+        if constexpr (qt_has_min(QT)) {
+            mlo = h2f(lds16(blk + 2));
+            mhi = h2f(lds16(blk + r8 + 2));
+        }
         const uint32_t a0[4] = {hsub2_u(lo[0], off2), hsub2_u(hi[0], off2), hsub2_u(lo[1], off2),
                                 hsub2_u(hi[1], off2)};
         const uint32_t a1[4] = {hsub2_u(lo[2], off2), hsub2_u(hi[2], off2), hsub2_u(lo[3], off2),
@@ -723,6 +852,50 @@ __device__ __forceinline__ void down_blocks8(uint32_t row, uint32_t r8, const ui
             acc[nt][1] = fmaf(dlo, p[1], acc[nt][1]);
             acc[nt][2] = fmaf(dhi, p[2], acc[nt][2]);
             acc[nt][3] = fmaf(dhi, p[3], acc[nt][3]);
+            if constexpr (qt_has_min(QT)) {
+                float hs[4];
+                mma_16816(hs, ones, b.x, b.y, zero);
+                mma_16816(hs, ones, b.z, b.w, hs);
+                acc[nt][0] = fmaf(mlo, hs[0], acc[nt][0]);
+                acc[nt][1] = fmaf(mlo, hs[1], acc[nt][1]);
+                acc[nt][2] = fmaf(mhi, hs[0], acc[nt][2]);
+                acc[nt][3] = fmaf(mhi, hs[1], acc[nt][3]);
+            }
+        }
+    }
+}
+
+// As down_blocks8 for Q4_K: the 8 units are one 144-byte block (blk).
+template <int NTILE>
+__device__ __forceinline__ void down_block_q4k(uint32_t blk, uint32_t r8, const uint32_t *ha, int c,
+                                               float (*acc)[4]) {
+    const uint32_t off2 = 0x64006400u;
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t ones[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        uint32_t lo[4], hi[4];
+        q4k_codes(blk, j, c, lo);
+        q4k_codes(blk + r8, j, c, hi);
+        float dlo, mlo, dhi, mhi;
+        q4k_params(blk, j, &dlo, &mlo);
+        q4k_params(blk + r8, j, &dhi, &mhi);
+        const uint32_t a0[4] = {hsub2_u(lo[0], off2), hsub2_u(hi[0], off2), hsub2_u(lo[1], off2),
+                                hsub2_u(hi[1], off2)};
+        const uint32_t a1[4] = {hsub2_u(lo[2], off2), hsub2_u(hi[2], off2), hsub2_u(lo[3], off2),
+                                hsub2_u(hi[3], off2)};
+#pragma unroll
+        for (int nt = 0; nt < NTILE; nt++) {
+            const uint4 b = lds128(ha[nt] + j * 64);
+            float p[4], hs[4];
+            mma_16816(p, a0, b.x, b.y, zero);
+            mma_16816(p, a1, b.z, b.w, p);
+            mma_16816(hs, ones, b.x, b.y, zero);
+            mma_16816(hs, ones, b.z, b.w, hs);
+            acc[nt][0] = fmaf(-mlo, hs[0], fmaf(dlo, p[0], acc[nt][0]));
+            acc[nt][1] = fmaf(-mlo, hs[1], fmaf(dlo, p[1], acc[nt][1]));
+            acc[nt][2] = fmaf(-mhi, hs[0], fmaf(dhi, p[2], acc[nt][2]));
+            acc[nt][3] = fmaf(-mhi, hs[1], fmaf(dhi, p[3], acc[nt][3]));
         }
     }
 }
@@ -740,7 +913,10 @@ __device__ __forceinline__ DnSlot dn_slot(int i, int G, int Sg) {
     return {i % G + G * (m % Sg), (uint32_t)((m / Sg) & 1)};
 }
 
-template <int NT>
+// ALL: the call has a type other than Q4_0 and Q8_0 (a separate
+// instantiation keeps the other types' code and registers out of the two
+// types' kernel)
+template <int NT, bool ALL>
 __global__ void __launch_bounds__(kDThreads, 1)
 dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ DecMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -749,8 +925,8 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
     const int D = a.D;
     const int S = G * Sg;
     const int hbytes = a.hrow * 2;                      // staged Hs row = its global stride
-    const int pr = tma_row_bytes((a.F / QK) * (a.q8 ? kQ8Bytes : kQ4Bytes));
-    const int ps = a.sF > 0 ? tma_row_bytes((a.sF / QK) * (a.sq8 ? kQ8Bytes : kQ4Bytes)) : 0;
+    const int pr = tma_row_bytes((int)qt_row_bytes(a.qt, a.F));
+    const int ps = a.sF > 0 ? tma_row_bytes((int)qt_row_bytes(a.sqt, a.sF)) : 0;
     const int wbytes = kDnRows * (pr > ps ? pr : ps);
     const int stage_bytes = (int)round_up((size_t)wbytes + (size_t)hrows * hbytes, 128);
     const int grp = warp >> 2, mt = warp & 3;
@@ -830,7 +1006,7 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
         const int v = u / tiles, dt = u % tiles;
         const DnSlot sl = dn_slot(i, G, Sg);
         const Virt vi = virt(a, act, A.n_routed, v);
-        const int bsz = vi.q8 ? kQ8Bytes : kQ4Bytes;
+        const int bsz = qt_unit_bytes(vi.qt);
         const int pitch = vi.shared ? ps : pr;
         const int nb = vi.Fv / QK;
         const int ntile = vi.cnt > 8 ? 2 : 1;
@@ -853,9 +1029,28 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
             ha[nt] = sbase + wbytes + (n < hrows ? n : 0) * hbytes + c * 16;
         }
         for (int kb = 0; kb < nb; kb += 8) {
-#define MOE_DN(Q8, NTL) down_blocks8<Q8, NTL>(row, r8, ha, c, acc)
-            if (!vi.q8) { if (ntile == 1) MOE_DN(false, 1); else if (NT > 1) MOE_DN(false, NT); }
-            else { if (ntile == 1) MOE_DN(true, 1); else if (NT > 1) MOE_DN(true, NT); }
+#define MOE_DN(QT)                                                     \
+    case QT:                                                           \
+        if (ntile == 1) down_blocks8<QT, 1>(row, r8, ha, c, acc);      \
+        else if (NT > 1) down_blocks8<QT, NT>(row, r8, ha, c, acc);    \
+        break;
+            if (!ALL || vi.qt == MOE_Q4_0 || vi.qt == MOE_Q8_0) {
+                switch (vi.qt) {
+                    MOE_DN(MOE_Q4_0)
+                    default:
+                        if (ntile == 1) down_blocks8<MOE_Q8_0, 1>(row, r8, ha, c, acc);
+                        else if (NT > 1) down_blocks8<MOE_Q8_0, NT>(row, r8, ha, c, acc);
+                }
+            } else if constexpr (ALL) {
+                switch (vi.qt) {
+                    MOE_DN(MOE_Q4_1)
+                    MOE_DN(MOE_Q5_0)
+                    MOE_DN(MOE_Q5_1)
+                    default:                                 // Q4_K
+                        if (ntile == 1) down_block_q4k<1>(row, r8, ha, c, acc);
+                        else if (NT > 1) down_block_q4k<NT>(row, r8, ha, c, acc);
+                }
+            }
 #undef MOE_DN
             row += 8 * bsz;
 #pragma unroll
@@ -909,9 +1104,14 @@ dec_combine_kernel(const float *__restrict__ rows, const int32_t *__restrict__ i
 // multiples of 256 up to 1024 (one box per expert tile in the down kernel).
 static bool gu_shape_ok(int D) { return D == 256 || D == 512 || D == 768 || D == 1024 || D == 2048; }
 
-bool decode_path_ok(int T, int D, int F, int sF) {
+// Block types the kernels decode: the 32-weight Standard family and Q4_K
+// (Q6_K's 210-byte blocks leave rows of F=768 weights unaligned for tensor
+// copies; it takes the portable kernels)
+static bool dec_type_ok(int qt) { return qt_known(qt) && qt != MOE_Q6_K; }
+
+bool decode_path_ok(int T, int D, int F, int sF, int qt, int sqt) {
     return T >= 1 && T <= 16 && gu_shape_ok(D) && F % 256 == 0 && F <= 1024 &&
-           (sF == 0 || (sF % 256 == 0 && sF <= 1024));
+           dec_type_ok(qt) && (sF == 0 || (sF % 256 == 0 && sF <= 1024 && dec_type_ok(sqt)));
 }
 
 // Hs rows are padded by 32 halves (64 bytes): row stride = 64 mod 128 bytes,
@@ -961,23 +1161,22 @@ static moe_status encode_rows(CUtensorMap *m, const void *base, size_t row_bytes
 
 static moe_status encode_maps(const DecArgs &a, int n_slots, int max_sb, DecMaps *m) {
     memset(m, 0, sizeof(*m));
-    const int nbD = a.D / QK;
-    const int br = a.q8 ? kQ8Bytes : kQ4Bytes;
-    const GuGeo gr = gu_geo(a.D, a.q8, max_sb);
+    const size_t rg = qt_row_bytes(a.qt, a.D);
+    const GuGeo gr = gu_geo(a.D, a.qt, max_sb);
     moe_status st;
-    if ((st = encode_rows(&m->gate, a.gate, (size_t)nbD * br, (size_t)n_slots * a.F, gr.pitch, kTile)))
+    if ((st = encode_rows(&m->gate, a.gate, rg, (size_t)n_slots * a.F, gr.pitch, kTile)))
         return st;
-    if ((st = encode_rows(&m->up, a.up, (size_t)nbD * br, (size_t)n_slots * a.F, gr.pitch, kTile)))
+    if ((st = encode_rows(&m->up, a.up, rg, (size_t)n_slots * a.F, gr.pitch, kTile)))
         return st;
-    const size_t rbd = (size_t)(a.F / QK) * br;
+    const size_t rbd = qt_row_bytes(a.qt, a.F);
     if ((st = encode_rows(&m->down, a.down, rbd, (size_t)n_slots * a.D, tma_row_bytes((int)rbd), kDnRows)))
         return st;
     if (a.sF > 0) {
-        const int bsh = a.sq8 ? kQ8Bytes : kQ4Bytes;
-        const GuGeo gs = gu_geo(a.D, a.sq8, max_sb);
-        if ((st = encode_rows(&m->sgate, a.sh_gate, (size_t)nbD * bsh, a.sF, gs.pitch, kTile))) return st;
-        if ((st = encode_rows(&m->sup, a.sh_up, (size_t)nbD * bsh, a.sF, gs.pitch, kTile))) return st;
-        const size_t rbs = (size_t)(a.sF / QK) * bsh;
+        const size_t rgs = qt_row_bytes(a.sqt, a.D);
+        const GuGeo gs = gu_geo(a.D, a.sqt, max_sb);
+        if ((st = encode_rows(&m->sgate, a.sh_gate, rgs, a.sF, gs.pitch, kTile))) return st;
+        if ((st = encode_rows(&m->sup, a.sh_up, rgs, a.sF, gs.pitch, kTile))) return st;
+        const size_t rbs = qt_row_bytes(a.sqt, a.sF);
         if ((st = encode_rows(&m->sdown, a.sh_down, rbs, a.D, tma_row_bytes((int)rbs), kDnRows))) return st;
     }
     return MOE_OK;
@@ -1022,18 +1221,31 @@ static size_t tables_bytes(int E) {
 // at D=2048, Q4_0)
 static int gu_max_sb(int T) { (void)T; return 64; }
 
-static cudaError_t launch_gateup(const DecArgs &a, const DecMaps &m, int grid, size_t smem,
-                                 cudaStream_t s, int S) {
+// the call has a type other than Q4_0 and Q8_0
+static bool dec_all_types(const DecArgs &a) {
+    auto basic = [](int q) { return q == MOE_Q4_0 || q == MOE_Q8_0; };
+    return !basic(a.qt) || (a.sF > 0 && !basic(a.sqt));
+}
+
+template <bool ALL>
+static cudaError_t launch_gateup1(const DecArgs &a, const DecMaps &m, int grid, size_t smem,
+                                  cudaStream_t s, int S) {
     const bool wide = gu_max_sb(a.T) == 64;
     switch (a.D) {
-    case 256: return launch_pdl(dec_gateup_kernel<32, 1, 1>, grid, kGThreads, smem, s, a, S, m);
-    case 512: return launch_pdl(dec_gateup_kernel<32, 2, 2>, grid, kGThreads, smem, s, a, S, m);
-    case 768: return launch_pdl(dec_gateup_kernel<32, 3, 3>, grid, kGThreads, smem, s, a, S, m);
-    case 1024: return launch_pdl(dec_gateup_kernel<32, 4, 4>, grid, kGThreads, smem, s, a, S, m);
+    case 256: return launch_pdl(dec_gateup_kernel<32, 1, 1, ALL>, grid, kGThreads, smem, s, a, S, m);
+    case 512: return launch_pdl(dec_gateup_kernel<32, 2, 2, ALL>, grid, kGThreads, smem, s, a, S, m);
+    case 768: return launch_pdl(dec_gateup_kernel<32, 3, 3, ALL>, grid, kGThreads, smem, s, a, S, m);
+    case 1024: return launch_pdl(dec_gateup_kernel<32, 4, 4, ALL>, grid, kGThreads, smem, s, a, S, m);
     default:
-        return wide ? launch_pdl(dec_gateup_kernel<64, 8, 4>, grid, kGThreads, smem, s, a, S, m)
-                    : launch_pdl(dec_gateup_kernel<32, 4, 4>, grid, kGThreads, smem, s, a, S, m);
+        return wide ? launch_pdl(dec_gateup_kernel<64, 8, 4, ALL>, grid, kGThreads, smem, s, a, S, m)
+                    : launch_pdl(dec_gateup_kernel<32, 4, 4, ALL>, grid, kGThreads, smem, s, a, S, m);
     }
+}
+
+static cudaError_t launch_gateup(const DecArgs &a, const DecMaps &m, int grid, size_t smem,
+                                 cudaStream_t s, int S) {
+    return dec_all_types(a) ? launch_gateup1<true>(a, m, grid, smem, s, S)
+                            : launch_gateup1<false>(a, m, grid, smem, s, S);
 }
 
 template <int NT>
@@ -1043,14 +1255,13 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
     const int max_sb = a.D <= 1024 ? 32 : gu_max_sb(a.T);
     moe_status st = encode_maps(a, n_slots, max_sb, &maps);
     if (st != MOE_OK) return st;
-    const bool any8 = a.q8 || (a.sF > 0 && a.sq8), any4 = !a.q8 || (a.sF > 0 && !a.sq8);
     // gate/up and down run when this call has routed experts or the shared one
     if (a.routed || a.sF > 0) {
     // ---- gate/up
     {
         const int nbD = a.D / QK;
-        const int pitch = std::max(any4 ? gu_geo(a.D, false, max_sb).pitch : 0,
-                                   any8 ? gu_geo(a.D, true, max_sb).pitch : 0);
+        const int pitch = std::max(gu_geo(a.D, a.qt, max_sb).pitch,
+                                   a.sF > 0 ? gu_geo(a.D, a.sqt, max_sb).pitch : 0);
         const int stage_bytes = (int)round_up((size_t)2 * kTile * pitch, 128);
         // mirrors the kernel's carve; + 1024 for aligning the base
         const size_t fixed = round_up(round_up((size_t)(a.T + 1) * staged_act_bytes(a.D), 16) +
@@ -1071,8 +1282,8 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
     // ---- down: Y rows
     {
         const int hrows = std::min(a.T, 16);
-        const int pr = tma_row_bytes((a.F / QK) * (a.q8 ? kQ8Bytes : kQ4Bytes));
-        const int ps = a.sF > 0 ? tma_row_bytes((a.sF / QK) * (a.sq8 ? kQ8Bytes : kQ4Bytes)) : 0;
+        const int pr = tma_row_bytes((int)qt_row_bytes(a.qt, a.F));
+        const int ps = a.sF > 0 ? tma_row_bytes((int)qt_row_bytes(a.sqt, a.sF)) : 0;
         const size_t wbytes = (size_t)kDnRows * std::max(pr, ps);
         const size_t stage_bytes = round_up(wbytes + (size_t)hrows * a.hrow * 2, 128);
         const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
@@ -1090,7 +1301,10 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         const int grid = std::max(1, std::min(sms, U_max));
         // no trace mark here: an event between the two kernels would cancel
         // their programmatic overlap
-        cudaError_t e = launch_pdl(dec_down_kernel<NT>, grid, kDThreads, smem, s, a, G, Sg, hrows, maps);
+        cudaError_t e = dec_all_types(a) ? launch_pdl(dec_down_kernel<NT, true>, grid, kDThreads, smem,
+                                                      s, a, G, Sg, hrows, maps)
+                                         : launch_pdl(dec_down_kernel<NT, false>, grid, kDThreads, smem,
+                                                      s, a, G, Sg, hrows, maps);
         if (e != cudaSuccess) return cuda_status(e, "dec_down_kernel");
     }
     }
@@ -1126,7 +1340,7 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
     a.perm = perm; a.offsets = offsets; a.gates = gates; a.mask = mask;
     a.gate = (const uint8_t *)pool.gate; a.up = (const uint8_t *)pool.up;
     a.down = (const uint8_t *)pool.down; a.slot_map = pool.slot_of_expert;
-    if (pool.qtype != MOE_Q4_0 && pool.qtype != MOE_Q8_0) {
+    if (!dec_type_ok(pool.qtype)) {
         set_error("decode path: unsupported quant type %d", (int)pool.qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }
@@ -1134,15 +1348,16 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
         set_error("decode path: T*k=%d exceeds %d", T * k, kMaxTk);
         return MOE_ERR_SHAPE;
     }
-    a.q8 = pool.qtype == MOE_Q8_0;
+    a.qt = pool.qtype;
+    a.sqt = pool.qtype;
     if (shared) {
         a.sh_gate = (const uint8_t *)shared->gate; a.sh_up = (const uint8_t *)shared->up;
         a.sh_down = (const uint8_t *)shared->down;
-        if (shared->qtype != MOE_Q4_0 && shared->qtype != MOE_Q8_0) {
+        if (!dec_type_ok(shared->qtype)) {
             set_error("decode path: unsupported shared-expert quant type %d", (int)shared->qtype);
             return MOE_ERR_UNSUPPORTED_QTYPE;
         }
-        a.sq8 = shared->qtype == MOE_Q8_0;
+        a.sqt = shared->qtype;
     }
     a.x = x; a.x_bf16 = (x_dtype == MOE_BF16);
     a.x_vec = ((uintptr_t)x % 16) == 0;

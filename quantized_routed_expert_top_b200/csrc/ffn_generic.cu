@@ -1,9 +1,10 @@
-// ffn_generic.cu -- portable SIMT expert FFN for every shape and both types.
+// ffn_generic.cu -- portable SIMT expert FFN for every shape and block type.
 //
 // Per permuted row pos (token t = perm[pos] / k, expert e = its segment):
 //   H[pos, r]  = silu(x_t . W_gate,e[r]) * (x_t . W_up,e[r])      (fp32)
 //   out[pos, d] = H[pos, :] . W_down,e[d]                           (fp32)
-// One warp per weight row, lanes over blocks; each weight row is read once
+// One warp per weight row, lanes over 32-weight units (a block of the
+// 32-weight types, a sub-block of the K-quants); each weight row is read once
 // per group of kTokGroup tokens of the segment.  This path favours
 // simplicity over speed: the tuned decode (GEMV) and prefill (tensor-core)
 // paths live in their own files and are checked against the same oracle.
@@ -68,7 +69,7 @@ ffn_gateup_generic_kernel(const XT *__restrict__ x, int T, int D, int F, int E, 
     const int n_act = build_active(offsets, mask, slot_map, n_slots, E, err, act);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nb = D / QK;
-    const size_t row_bytes = (size_t)nb * block_bytes<QT>();
+    const size_t row_bytes = qt_row_bytes(QT, D);
     const int tiles = (F + kGenWarps - 1) / kGenWarps;
     for (int w = blockIdx.x; w < n_act * tiles; w += gridDim.x) {
         const int e = act[w / tiles];
@@ -89,8 +90,8 @@ ffn_gateup_generic_kernel(const XT *__restrict__ x, int T, int D, int F, int E, 
             float ag[kTokGroup] = {}, au[kTokGroup] = {};
             for (int b = lane; b < nb; b += 32) {
                 float wg[QK], wu[QK];
-                decode_block_global<QT>(grow + (size_t)b * block_bytes<QT>(), wg);
-                decode_block_global<QT>(urow + (size_t)b * block_bytes<QT>(), wu);
+                decode_unit_global<QT>(grow, b, wg);
+                decode_unit_global<QT>(urow, b, wu);
 #pragma unroll
                 for (int q = 0; q < kTokGroup; q++) {
                     if (tok[q] < 0) continue;
@@ -124,7 +125,7 @@ ffn_down_generic_kernel(const float *__restrict__ H, int T, int D, int F, int E,
     const int n_act = build_active(offsets, mask, slot_map, n_slots, E, err, act);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nb = F / QK;
-    const size_t row_bytes = (size_t)nb * block_bytes<QT>();
+    const size_t row_bytes = qt_row_bytes(QT, F);
     const int tiles = (D + kGenWarps - 1) / kGenWarps;
     for (int w = blockIdx.x; w < n_act * tiles; w += gridDim.x) {
         const int e = act[w / tiles];
@@ -138,7 +139,7 @@ ffn_down_generic_kernel(const float *__restrict__ H, int T, int D, int F, int E,
             float acc[kTokGroup] = {};
             for (int b = lane; b < nb; b += 32) {
                 float wd[QK];
-                decode_block_global<QT>(drow + (size_t)b * block_bytes<QT>(), wd);
+                decode_unit_global<QT>(drow, b, wd);
 #pragma unroll
                 for (int q = 0; q < kTokGroup; q++) {
                     if (p0 + q >= seg1) continue;
@@ -185,13 +186,19 @@ moe_status launch_ffn_generic(const void *x, int x_dtype, int T, int D, int F, i
                               const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
                               const uint8_t *mask, float *H, float *out_rows, int *err,
                               cudaStream_t s, Tracer *tr, bool shared) {
+#define MOE_RUN(QT)                                                                           \
+    case QT:                                                                                  \
+        return run_generic<QT>(x, x_dtype, T, D, F, E, k, perm, offsets, pool, mask, H,       \
+                               out_rows, err, s, tr, shared);
     switch (pool.qtype) {
-    case MOE_Q4_0:
-        return run_generic<MOE_Q4_0>(x, x_dtype, T, D, F, E, k, perm, offsets, pool, mask, H,
-                                     out_rows, err, s, tr, shared);
-    case MOE_Q8_0:
-        return run_generic<MOE_Q8_0>(x, x_dtype, T, D, F, E, k, perm, offsets, pool, mask, H,
-                                     out_rows, err, s, tr, shared);
+        MOE_RUN(MOE_Q4_0)
+        MOE_RUN(MOE_Q4_1)
+        MOE_RUN(MOE_Q5_0)
+        MOE_RUN(MOE_Q5_1)
+        MOE_RUN(MOE_Q8_0)
+        MOE_RUN(MOE_Q4_K)
+        MOE_RUN(MOE_Q6_K)
+#undef MOE_RUN
     default:
         set_error("expert FFN: unsupported quant type %d", (int)pool.qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;

@@ -27,7 +27,8 @@
 // accumulators (2 x 256 columns) let the epilogue warps drain one tile while
 // the next accumulates.
 //
-// Numerics: weights d*q rounded to fp16 (relative error <= 2^-11 per weight),
+// Numerics: weights (q - z)*d, or q*d + m for the _1 types, rounded once to
+// fp16 (relative error <= 2^-11 per weight),
 // activations fp16 (a bf16 x in fp16's normal range converts exactly; an fp32
 // x is rounded to fp16's 11 significant bits), fp32 accumulation; H is
 // stored fp16.
@@ -62,8 +63,9 @@ constexpr int kPThreads = (kPAW + kPBW + 1 + kPEW) * 32;     // 480
 constexpr int kPARows = kPM / (kPAW * 32 / 8);               // rows per A thread (16)
 constexpr int kPTmemCols = 512;                              // 2 accumulators x 256
 // A raw window holds four blocks (K = 128, two MMA stages) of each of the
-// 256 weight rows: the 16-byte-aligned 144 bytes (Q8_0) or 80 bytes (Q4_0)
-// around them; four blocks start 0 or 8 bytes past a 16-byte boundary.
+// 256 weight rows: the 16-byte-aligned bytes around them (pf_window_bytes).
+// Four blocks of 18, 22 or 34 bytes start 0 or 8 bytes past a 16-byte
+// boundary (every other window), four of 20 or 24 bytes always on one.
 constexpr int kPRawRow = 144;
 constexpr int kPRaw = 256 * kPRawRow;    // one raw window buffer (36 KB)
 constexpr int kPfMaxExperts = 720;       // segs + tcum of E + 2 entries each fit with the rings
@@ -75,6 +77,18 @@ __host__ __device__ inline size_t pf_smem_bytes(int E) {
 
 enum : int { kPGateUp = 0, kPDown = 1 };
 
+// K stages (of 64 weights) per raw window: two (four 32-weight blocks), or
+// four for Q4_K (one 144-byte block: its scales sit at the block's head)
+__host__ __device__ constexpr int pf_stages_per_window(int qt) { return qt == MOE_Q4_K ? 4 : 2; }
+// row bytes a window covers
+__host__ __device__ constexpr int pf_window_span(int qt) {
+    return pf_stages_per_window(qt) * 2 * qt_unit_bytes(qt);
+}
+// bytes of a raw window row: 144 (Q8_0, Q4_K), 80 (Q4_0, Q4_1), 96 (Q5_0, Q5_1)
+__host__ __device__ constexpr int pf_window_bytes(int qt) {
+    return pf_window_span(qt) % 16 == 0 ? pf_window_span(qt) : (pf_window_span(qt) + 8 + 15) / 16 * 16;
+}
+
 // Tensor maps over the weight pools (8-byte elements, one row of blocks per
 // tensor row), boxes of one raw window (the 16-byte-aligned 144 or 80 bytes
 // holding four blocks) x 128 rows (gate, up) or 256 rows (down).
@@ -85,8 +99,8 @@ struct PfMaps {
 
 struct PfArgs {
     int T, D, F, E, k;
-    int q8;                       // routed pool is Q8_0 (else Q4_0)
-    int shared, sq8;              // this call runs the shared expert (F columns, Q8_0 / Q4_0)
+    int qt;                       // block type (ggml id) of the routed pool
+    int shared, sqt;              // this call runs the shared expert (F columns, its type)
     int routed;                   // this call runs the routed experts the mask admits
     int n_slots;                  // slots of the routed pool
     const uint8_t *mask;          // [E] or NULL
@@ -220,6 +234,134 @@ __device__ __forceinline__ void dq_pair_q4(const uint32_t *w, uint4 *out) {
     }
 }
 
+// 32-bit word / 16-bit field at an even byte offset of a run of words
+__device__ __forceinline__ uint32_t word_at(const uint32_t *w, int byte) {
+    return (byte & 3) ? __funnelshift_r(w[byte >> 2], w[(byte >> 2) + 1], 16) : w[byte >> 2];
+}
+__device__ __forceinline__ uint32_t half_at(const uint32_t *w, int byte) {
+    return (w[byte >> 2] >> (8 * (byte & 3))) & 0xFFFFu;
+}
+
+// Q4_1, Q5_0, Q5_1 pair starting at byte P of w (natural order, 8 chunks as
+// above): the low four bits from qs (element j low nibble, j+16 high), the
+// fifth from bit i of qh, v = 1024 + q exact in fp16, then (v - 1040) * d
+// (Q5_0) or (v - 1024) * d + m (the _1 types) with one rounding.
+template <int QT, int P>
+__device__ __forceinline__ void dq_pair_std(const uint32_t *w, uint4 *out) {
+    constexpr int BS = qt_bytes(QT), QS = qt_qs_off(QT), QH = qt_qh_off(QT);
+    const uint32_t M = 0x000F000Fu, MAG = 0x64006400u;
+    const uint32_t OFF = 0x64006400u + 0x00010001u * (uint32_t)qt_zero(QT);
+    uint32_t lo[16], hi[16];
+#pragma unroll
+    for (int b = 0; b < 2; b++) {
+        const int B = P + b * BS;
+        const uint32_t d = half_at(w, B), dd = d | (d << 16);
+        uint32_t mm = 0, qh = 0;
+        if constexpr (qt_has_min(QT)) {
+            const uint32_t m = half_at(w, B + 2);
+            mm = m | (m << 16);
+        }
+        if constexpr (qt_has_high(QT)) qh = word_at(w, B + QH);
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const uint32_t c = word_at(w, B + QS + 4 * i);        // bytes 4i .. 4i+3
+            const uint32_t t0 = prmt(c, 0u, 0x4140), t1 = prmt(c, 0u, 0x4342);
+            uint32_t v[4] = {lop3_and_or(t0, M, MAG), lop3_and_or(t1, M, MAG),
+                             lop3_and_or(t0 >> 4, M, MAG), lop3_and_or(t1 >> 4, M, MAG)};
+            if constexpr (qt_has_high(QT)) {
+                // v: elements (4i, 4i+1), (4i+2, 4i+3), (16+4i, 17+4i), (18+4i, 19+4i)
+                const uint32_t h = qh >> (4 * i);
+                v[0] |= ((h & 1u) << 4) | ((h & 2u) << 19);
+                v[1] |= ((h & 4u) << 2) | ((h & 8u) << 17);
+                v[2] |= ((h >> 12) & 0x10u) | ((h << 3) & 0x100000u);
+                v[3] |= ((h >> 14) & 0x10u) | ((h << 1) & 0x100000u);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+                v[q] = qt_has_min(QT) ? hfma2_u(hsub2_u(v[q], OFF), dd, mm)
+                                      : hmul2_u(hsub2_u(v[q], OFF), dd);
+            lo[8 * b + 2 * i] = v[0];
+            lo[8 * b + 2 * i + 1] = v[1];
+            hi[8 * b + 2 * i] = v[2];
+            hi[8 * b + 2 * i + 1] = v[3];
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < 2; b++) {
+        out[4 * b + 0] = make_uint4(lo[8 * b + 0], lo[8 * b + 1], lo[8 * b + 2], lo[8 * b + 3]);
+        out[4 * b + 1] = make_uint4(lo[8 * b + 4], lo[8 * b + 5], lo[8 * b + 6], lo[8 * b + 7]);
+        out[4 * b + 2] = make_uint4(hi[8 * b + 0], hi[8 * b + 1], hi[8 * b + 2], hi[8 * b + 3]);
+        out[4 * b + 3] = make_uint4(hi[8 * b + 4], hi[8 * b + 5], hi[8 * b + 6], hi[8 * b + 7]);
+    }
+}
+
+// The pair of a K stage of a Q4_1 / Q5_0 / Q5_1 row: it starts P bytes into
+// the row's window (rp, 16-byte aligned; rows pf_window_bytes apart).  Loads
+// the 16-byte vectors from P rounded down to 16 through 2 bytes past the
+// pair (a misaligned last word reads them): at most 16 bytes past the
+// window, which is the next row's landed window or, for the last row, the
+// unused tail of the raw buffer (sized for 144-byte rows).
+template <int QT, int P>
+__device__ __forceinline__ void dq_stage_std(const uint8_t *rp, uint4 *out) {
+    constexpr int B0 = P & ~15, NV = (P - B0 + 2 * qt_bytes(QT) + 2 + 15) / 16;
+    static_assert(255 * pf_window_bytes(QT) + B0 + 16 * NV <= kPRaw,
+                  "the last row's reads stay inside its raw buffer");
+    uint32_t w[4 * NV];
+#pragma unroll
+    for (int q = 0; q < NV; q++) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(rp + B0 + 16 * q);
+        w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+    }
+    dq_pair_std<QT, P - B0>(w, out);
+}
+
+// Q4_K: K stage P (0..3) of a 144-byte block (rp, 16-byte aligned) is its
+// 32-byte chunk P: the low nibbles are sub-block 2P (weights 0..31 of the
+// stage), the high nibbles sub-block 2P+1 (weights 32..63).  Each weight is
+// D * q - M with D = d * sc_j and M = dmin * m_j rounded to fp16, then one
+// fp16 multiply-add (three roundings in all).
+template <int P>
+__device__ __forceinline__ void dq_stage_q4k(const uint8_t *rp, uint4 *out) {
+    const uint4 h = *reinterpret_cast<const uint4 *>(rp);          // d, dmin, scales[12]
+    const uint4 q0 = *reinterpret_cast<const uint4 *>(rp + 16 + 32 * P);
+    const uint4 q1 = *reinterpret_cast<const uint4 *>(rp + 32 + 32 * P);
+    const float d = __half2float(__ushort_as_half((unsigned short)(h.x & 0xFFFFu)));
+    const float dmin = __half2float(__ushort_as_half((unsigned short)(h.x >> 16)));
+    uint8_t sb[12];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        sb[i] = (uint8_t)(h.y >> (8 * i));
+        sb[4 + i] = (uint8_t)(h.z >> (8 * i));
+        sb[8 + i] = (uint8_t)(h.w >> (8 * i));
+    }
+    uint32_t Dh[2], Mh[2];
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+        int sc, m;
+        q4k_scale_min(sb, 2 * P + u, &sc, &m);
+        const __half2 dd = __float2half2_rn(d * (float)sc), mm = __float2half2_rn(-dmin * (float)m);
+        Dh[u] = *reinterpret_cast<const uint32_t *>(&dd);
+        Mh[u] = *reinterpret_cast<const uint32_t *>(&mm);
+    }
+    const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const uint32_t HI = 0x64646464u, MAG = 0x64006400u, M4 = 0x0F0F0F0Fu;
+    uint32_t v[2][16];                       // [sub-block][pair of elements]
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            const uint32_t n = (qw[i] >> (4 * u)) & M4;             // elements 4i .. 4i+3
+            v[u][2 * i] = hfma2_u(hsub2_u(prmt(n, HI, 0x5140), MAG), Dh[u], Mh[u]);
+            v[u][2 * i + 1] = hfma2_u(hsub2_u(prmt(n, HI, 0x7362), MAG), Dh[u], Mh[u]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; u++)
+#pragma unroll
+        for (int k = 0; k < 4; k++)
+            out[4 * u + k] = make_uint4(v[u][4 * k], v[u][4 * k + 1], v[u][4 * k + 2], v[u][4 * k + 3]);
+}
+
 // ------------------------------------------------------------------ tiles
 // Virtual experts 0..E-1 (segments of the permutation) and, with a shared
 // expert, E (rows T*k .. T*k+T-1, token = row - T*k).  Tiles are listed
@@ -246,7 +388,10 @@ __device__ __forceinline__ PfTile pf_tile(const int *tcum, const int *segs, int 
     return t;
 }
 
-template <int MODE>
+// ALL: the call has a type other than Q4_0 and Q8_0 (a separate
+// instantiation keeps the other types' dequantisers and window logic out of
+// the two types' kernel)
+template <int MODE, bool ALL>
 __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const __grid_constant__ PfMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_pf[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -383,32 +528,32 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
     } else if (warp < kPAW + kPBW) {
         // ------------------------------------------------- B producers
         // Raw windows (the 16-byte-aligned bytes holding four blocks = two
-        // K stages, for all 256 weight rows of the tile) arrive by tensor
-        // copies kPR - 1 windows ahead.  Each warp dequantises its 32 rows of the
-        // window into the swizzled fp16 stage on its own; lane 0 of the
-        // first warp refills a raw buffer once all warps have read it.
+        // K stages, or one Q4_K block = four, for all 256 weight rows of the
+        // tile) arrive by tensor copies kPR - 1 windows ahead.  Each warp
+        // dequantises its 32 rows of the window into the swizzled fp16 stage
+        // on its own; lane 0 of the first warp refills a raw buffer once all
+        // warps have read it.
         const int bw = warp - kPAW, bt = tid - kPAW * 32;
         const bool issuer = bw == 0 && lane == 0;
-        const int nw = nk / 2;                           // windows per tile
-        const int n_win = n_loc * nw;
-        int gi = 0, ti = -1, wi = nw;                    // window issue cursor
+        int gi = 0, ti = -1, wi = 0, nwI = 0;            // window issue cursor; windows of tile ti
         PfTile tI{};
         auto issue = [&]() -> bool {
-            if (gi >= n_win) return true;
+            if (wi == nwI) {                             // next tile of this CTA, if any
+                if (ti + 1 >= n_loc) return true;
+                ti++;
+                wi = 0;
+                tI = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
+                nwI = ALL ? nk / pf_stages_per_window(tI.v == a.E ? a.sqt : a.qt) : nk / 2;
+            }
             if (gi >= kPR) {                             // the buffer's previous window is read
                 const int q = gi - kPR;
                 if (!mbar_wait(&rempty[q % kPR], (uint32_t)((q / kPR) & 1), a.err, kErrTimeoutEmpty)) return false;
             }
-            if (wi == nw) {
-                ti++;
-                wi = 0;
-                tI = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
-            }
             const bool sh = tI.v == a.E;
-            const bool q8 = sh ? a.sq8 != 0 : a.q8 != 0;
-            const int bs = q8 ? kQ8Bytes : kQ4Bytes;
-            const int wb = q8 ? 144 : 80;                        // window bytes
-            const int x = (int)(((size_t)wi * 4 * bs & ~(size_t)15) / 8);
+            const int qt = sh ? a.sqt : a.qt;
+            const int wb = pf_window_bytes(qt);
+            const int span = ALL ? pf_window_span(qt) : 4 * qt_bytes(qt);
+            const int x = (int)(((size_t)wi * span & ~(size_t)15) / 8);
             const int slot = sh ? 0 : (a.slot_map ? __ldg(a.slot_map + tI.v) : tI.v);
             const int r = gi % kPR;
             uint8_t *dst = raw + (size_t)r * kPRaw;
@@ -431,24 +576,46 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
         int g = 0, gw = 0;                               // stage, window counters
         for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
             const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
-            const bool q8 = (t.v == a.E) ? a.sq8 != 0 : a.q8 != 0;
-            const int wb = q8 ? 144 : 80;
+            const int qt = (t.v == a.E) ? a.sqt : a.qt;
+            const int wb = pf_window_bytes(qt);
+            const int spw = ALL ? pf_stages_per_window(qt) : 2;
             for (int ks = 0; ks < nk && ok; ks++, g++) {
+                const int pos = ks & (spw - 1);                  // stage within the window
                 const int half = ks & 1;                         // which block pair of the window
-                if (half == 0) {
+                if (pos == 0) {
                     bool iok = true;
                     if (issuer) iok = issue();                   // window gw + kPR - 1
                     ok = __shfl_sync(0xffffffffu, iok ? 1 : 0, 0) != 0;
                     if (!ok) break;
                 }
                 const int r = gw % kPR;
-                if (half == 0 &&
+                if (pos == 0 &&
                     !mbar_wait_warp(&rfull[r], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutFull)) { ok = false; break; }
                 uint4 c[8];
-                // the pair starts 8 * (group % 2) + (2 * bs) * half bytes into the window
+                // the pair starts skew(window) + (2 * bs) * half bytes into the
+                // window; the skew is 8 for odd windows of 18-, 22- and 34-byte
+                // blocks, else 0
                 const int odd = (ks >> 1) & 1;
                 const uint8_t *rp = raw + (size_t)r * kPRaw + bt * wb;
-                if (q8) {
+                if (ALL && qt == MOE_Q4_K) {
+                    switch (pos) {
+                    case 0: dq_stage_q4k<0>(rp, c); break;
+                    case 1: dq_stage_q4k<1>(rp, c); break;
+                    case 2: dq_stage_q4k<2>(rp, c); break;
+                    default: dq_stage_q4k<3>(rp, c); break;
+                    }
+                } else if (ALL && qt == MOE_Q4_1) {
+                    if (half == 0) dq_stage_std<MOE_Q4_1, 0>(rp, c); else dq_stage_std<MOE_Q4_1, 40>(rp, c);
+                } else if (ALL && qt == MOE_Q5_1) {
+                    if (half == 0) dq_stage_std<MOE_Q5_1, 0>(rp, c); else dq_stage_std<MOE_Q5_1, 48>(rp, c);
+                } else if (ALL && qt == MOE_Q5_0) {
+                    switch (2 * odd + half) {
+                    case 0: dq_stage_std<MOE_Q5_0, 0>(rp, c); break;
+                    case 1: dq_stage_std<MOE_Q5_0, 44>(rp, c); break;
+                    case 2: dq_stage_std<MOE_Q5_0, 8>(rp, c); break;
+                    default: dq_stage_std<MOE_Q5_0, 52>(rp, c); break;
+                    }
+                } else if (qt == MOE_Q8_0) {
                     // words 16 * half .. +19 hold the pair at word 2*odd + half
                     uint32_t w[20];
 #pragma unroll
@@ -477,7 +644,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
                     default: dq_pair_q4<3>(w, c); break;
                     }
                 }
-                if (half == 1) {
+                if (pos == spw - 1) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&rempty[r]);      // this warp is done with the window
                     gw++;
@@ -611,13 +778,19 @@ __global__ void __launch_bounds__(256) pf_convert_kernel(const XT *__restrict__ 
 }
 
 // ------------------------------------------------------------------- host
-// K (D for gate/up, F for down) a multiple of 256: a row is then a multiple of
-// 272 (Q8_0) or 144 (Q4_0) bytes, its last four blocks start 8 bytes past a
-// 16-byte boundary and their window ends exactly at the row's end, so no
-// window reads past a row
-bool prefill_path_ok(int T, int D, int F, int sF, int E) {
+// K (D for gate/up, F for down) a multiple of 256: a row is then 8m blocks,
+// a multiple of 16 bytes; with 18-, 22- or 34-byte blocks its last four
+// blocks start 8 bytes past a 16-byte boundary, so every window, the last
+// included, ends at or before the row's end and no window reads past a row
+// Block types the B producers dequantise: the 32-weight Standard family and
+// Q4_K (Q6_K's 210-byte blocks leave rows of F=768 weights unaligned for
+// tensor copies; it takes the portable kernels)
+static bool pf_type_ok(int qt) { return qt_known(qt) && qt != MOE_Q6_K; }
+
+bool prefill_path_ok(int T, int D, int F, int sF, int E, int qt, int sqt) {
     return T > 16 && D % kPNd == 0 && F % kPNg == 0 && D % 256 == 0 && F % 256 == 0 &&
-           (sF == 0 || sF == F) && E <= kPfMaxExperts && pf_smem_bytes(E) <= 227 * 1024;
+           (sF == 0 || (sF == F && pf_type_ok(sqt))) && pf_type_ok(qt) &&
+           E <= kPfMaxExperts && pf_smem_bytes(E) <= 227 * 1024;
 }
 
 size_t prefill_x16_halves(int T, int D) { return (size_t)T * D; }
@@ -655,8 +828,8 @@ static moe_status pf_encode(CUtensorMap *m, const void *base, size_t row_bytes, 
     return MOE_OK;
 }
 
-template <int MODE>
-static cudaError_t launch_pf(const PfArgs &a, const PfMaps &m, int grid, cudaStream_t s) {
+template <int MODE, bool ALL>
+static cudaError_t launch_pf1(const PfArgs &a, const PfMaps &m, int grid, cudaStream_t s) {
     const size_t smem = pf_smem_bytes(a.E);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -668,10 +841,17 @@ static cudaError_t launch_pf(const PfArgs &a, const PfMaps &m, int grid, cudaStr
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaFuncSetAttribute(pf_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(pf_gemm_kernel<MODE, ALL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, pf_gemm_kernel<MODE>, a, m);
+    return cudaLaunchKernelEx(&cfg, pf_gemm_kernel<MODE, ALL>, a, m);
+}
+
+template <int MODE>
+static cudaError_t launch_pf(const PfArgs &a, const PfMaps &m, int grid, cudaStream_t s) {
+    auto basic = [](int q) { return q == MOE_Q4_0 || q == MOE_Q8_0; };
+    const bool all = !basic(a.qt) || (a.shared && !basic(a.sqt));
+    return all ? launch_pf1<MODE, true>(a, m, grid, s) : launch_pf1<MODE, false>(a, m, grid, s);
 }
 
 moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, int E, int k,
@@ -679,23 +859,23 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
                               const uint8_t *mask, bool routed, const moe_pool *shared, int sF,
                               __half *x16, __half *H, float *Y, int *err, cudaStream_t s,
                               Tracer *tr) {
-    if (pool.qtype != MOE_Q4_0 && pool.qtype != MOE_Q8_0) {
+    if (!pf_type_ok(pool.qtype)) {
         set_error("prefill path: unsupported quant type %d", (int)pool.qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }
-    if (shared && shared->qtype != MOE_Q4_0 && shared->qtype != MOE_Q8_0) {
+    if (shared && !pf_type_ok(shared->qtype)) {
         set_error("prefill path: unsupported shared-expert quant type %d", (int)shared->qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }
-    if (!prefill_path_ok(T, D, F, shared ? sF : 0, E)) {
+    if (!prefill_path_ok(T, D, F, shared ? sF : 0, E, pool.qtype, shared ? shared->qtype : 0)) {
         set_error("prefill path: shape T=%d D=%d F=%d not supported", T, D, F);
         return MOE_ERR_SHAPE;
     }
     PfArgs a{};
     a.T = T; a.D = D; a.F = F; a.E = E; a.k = k;
-    a.q8 = pool.qtype == MOE_Q8_0;
+    a.qt = pool.qtype;
     a.shared = shared ? 1 : 0;
-    a.sq8 = shared ? shared->qtype == MOE_Q8_0 : 0;
+    a.sqt = shared ? shared->qtype : pool.qtype;
     a.routed = routed ? 1 : 0;
     a.n_slots = pool.n_slots;
     a.mask = mask;
@@ -718,24 +898,24 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
         pf_convert_kernel<float><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const float *)x, x16, n8);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "pf_convert_kernel");
-    // weight tensor maps: raw windows of 144 (Q8_0) or 80 (Q4_0) bytes
-    const int br = pool.qtype == MOE_Q8_0 ? kQ8Bytes : kQ4Bytes;
-    const int wr = pool.qtype == MOE_Q8_0 ? 144 : 80;
+    // weight tensor maps: boxes of one raw window row
+    const size_t rg = qt_row_bytes(pool.qtype, D), rd = qt_row_bytes(pool.qtype, F);
+    const int wr = pf_window_bytes(pool.qtype);
     PfMaps mg, md;
     memset(&mg, 0, sizeof(mg));
     memset(&md, 0, sizeof(md));
     moe_status st;
     const size_t rows_f = (size_t)pool.n_slots * F, rows_d = (size_t)pool.n_slots * D;
-    if ((st = pf_encode(&mg.w0, pool.gate, (size_t)(D / QK) * br, rows_f, wr, kPNg)) ||
-        (st = pf_encode(&mg.w1, pool.up, (size_t)(D / QK) * br, rows_f, wr, kPNg)) ||
-        (st = pf_encode(&md.w0, pool.down, (size_t)(F / QK) * br, rows_d, wr, kPNd)))
+    if ((st = pf_encode(&mg.w0, pool.gate, rg, rows_f, wr, kPNg)) ||
+        (st = pf_encode(&mg.w1, pool.up, rg, rows_f, wr, kPNg)) ||
+        (st = pf_encode(&md.w0, pool.down, rd, rows_d, wr, kPNd)))
         return st;
     if (shared) {
-        const int bsh = shared->qtype == MOE_Q8_0 ? kQ8Bytes : kQ4Bytes;
-        const int wsh = shared->qtype == MOE_Q8_0 ? 144 : 80;
-        if ((st = pf_encode(&mg.s0, shared->gate, (size_t)(D / QK) * bsh, F, wsh, kPNg)) ||
-            (st = pf_encode(&mg.s1, shared->up, (size_t)(D / QK) * bsh, F, wsh, kPNg)) ||
-            (st = pf_encode(&md.s0, shared->down, (size_t)(F / QK) * bsh, D, wsh, kPNd)))
+        const size_t rgs = qt_row_bytes(shared->qtype, D), rds = qt_row_bytes(shared->qtype, F);
+        const int wsh = pf_window_bytes(shared->qtype);
+        if ((st = pf_encode(&mg.s0, shared->gate, rgs, F, wsh, kPNg)) ||
+            (st = pf_encode(&mg.s1, shared->up, rgs, F, wsh, kPNg)) ||
+            (st = pf_encode(&md.s0, shared->down, rds, D, wsh, kPNd)))
             return st;
     }
     const int grid = num_sms();

@@ -35,12 +35,13 @@ static LayerWs carve(const moe_layer_args &a, Carver &c) {
     w.offsets = c.take<int32_t>(a.E + 1);
     w.perm = c.take<int32_t>(Tk);
     w.inv = c.take<int32_t>(Tk);
-    if (decode_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0)) {
+    const int qt = a.pool ? a.pool->qtype : 0, sqt = a.shared ? a.shared->qtype : 0;
+    if (decode_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0, qt, sqt)) {
         w.Hs = c.take<__half>(decode_hs_halves(a.T, a.k, a.F, a.shared ? a.shared_F : 0));
         w.rows = c.take<float>(decode_rows_floats(a.T, a.k, a.D));
         return w;
     }
-    if (prefill_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0, a.E)) {
+    if (prefill_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0, a.E, qt, sqt)) {
         const int sF = a.shared ? a.shared_F : 0;
         w.x16 = c.take<__half>(prefill_x16_halves(a.T, a.D));
         w.H16 = c.take<__half>(prefill_h_halves(a.T, a.k, a.F, sF));

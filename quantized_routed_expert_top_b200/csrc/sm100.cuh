@@ -175,4 +175,11 @@ __device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
     return r;
 }
 
+// a * b + c in fp16x2, one rounding
+__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
 }  // namespace moe

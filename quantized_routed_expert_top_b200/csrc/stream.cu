@@ -71,7 +71,7 @@ moe_status moe_streamer_init(const moe_streamer_desc *desc, moe_streamer **out) 
         set_error("moe_streamer_init: need n_layers > 0 and 0 < E <= %d", MOE_MAX_EXPERTS);
         return MOE_ERR_SHAPE;
     }
-    if (d.qtype != MOE_Q4_0 && d.qtype != MOE_Q8_0) {
+    if (!qt_known(d.qtype)) {
         set_error("moe_streamer_init: unsupported quant type %d", (int)d.qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }

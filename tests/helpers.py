@@ -42,7 +42,7 @@ def dev_shared(moe, L: S.LayerInputs, device="cuda"):
     if L.shared is None:
         return None
     g, u, d = L.shared
-    return moe.ExpertPool(dev(g, device), dev(u, device), dev(d, device), "q8_0")
+    return moe.ExpertPool(dev(g, device), dev(u, device), dev(d, device), L.cfg.shared_qtype)
 
 
 def oracle_route(L: S.LayerInputs):

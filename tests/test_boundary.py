@@ -38,13 +38,18 @@ def test_every_declared_symbol_is_exported(moe):
 def test_block_tables_agree_with_header(moe, orc):
     h = _header_defines()
     assert h["MOE_QK"] == S.QK == 32
-    assert h["MOE_Q4_0_BLOCK_BYTES"] == S.BLOCK_BYTES["q4_0"] == moe.BLOCK_BYTES[moe.Q4_0]
-    assert h["MOE_Q8_0_BLOCK_BYTES"] == S.BLOCK_BYTES["q8_0"] == moe.BLOCK_BYTES[moe.Q8_0]
-    assert moe.lib().moe_block_bytes(moe.Q4_0) == 18 == orc.block_bytes("q4_0")
-    assert moe.lib().moe_block_bytes(moe.Q8_0) == 34 == orc.block_bytes("q8_0")
-    assert moe.lib().moe_block_bytes(3) == 0        # unknown type -> 0, never garbage
-    assert {q: S.GGML_TYPE_ID[q] for q in ("q4_0", "q8_0")} == {"q4_0": moe.Q4_0,
-                                                                 "q8_0": moe.Q8_0}
+    assert h["MOE_QK_K"] == S.QK_K == 256
+    for q in S.QTYPES:
+        qid = moe.QTYPES[q]
+        assert qid == S.GGML_TYPE_ID[q]
+        assert h[f"MOE_{q.upper()}_BLOCK_BYTES"] == S.BLOCK_BYTES[q] == moe.BLOCK_BYTES[qid]
+        assert moe.lib().moe_block_bytes(qid) == S.BLOCK_BYTES[q] == orc.block_bytes(q)
+        assert moe.lib().moe_block_weights(qid) == S.BLOCK_WEIGHTS[q] == orc.block_weights(q) \
+            == moe.BLOCK_WEIGHTS[qid]
+    for unknown in (0, 1, 4, 5, 9, 10, 11, 13, 15, -1):    # unknown type -> 0, never garbage
+        assert moe.lib().moe_block_bytes(unknown) == 0
+        assert moe.lib().moe_block_weights(unknown) == 0
+    assert set(moe.QTYPES) == set(S.QTYPES)
 
 
 def _err(L):
@@ -80,13 +85,20 @@ def test_route_argument_errors(moe):
 
 def test_expert_ffn_rejects_unknown_and_missing_pools(moe):
     L = moe.lib()
-    bad = moe.Pool(3, 8, 0x1000, 0x1000, 0x1000, None)       # qtype 3 is not supported
+    bad = moe.Pool(9, 8, 0x1000, 0x1000, 0x1000, None)       # type 9 (Q8_1) is not supported
     assert L.moe_expert_ffn(FAKE, moe.BF16, 4, 256, 512, 8, 2, FAKE, FAKE, C.byref(bad), None,
                             FAKE, FAKE, 1 << 30, None) == 2
     assert "quant type" in _err(L)
     nul = moe.Pool(moe.Q8_0, 8, 0x1000, 0, 0x1000, None)
     assert L.moe_expert_ffn(FAKE, moe.BF16, 4, 256, 512, 8, 2, FAKE, FAKE, C.byref(nul), None,
                             FAKE, FAKE, 1 << 30, None) == 1
+    # K-quant blocks hold 256 weights: D or F not a multiple of 256 is a shape error
+    for qk in (moe.Q4_K, moe.Q6_K):
+        kp = moe.Pool(qk, 8, 0x1000, 0x1000, 0x1000, None)
+        for D, F in ((256, 384), (384, 256), (96, 512)):
+            assert L.moe_expert_ffn(FAKE, moe.BF16, 4, D, F, 8, 2, FAKE, FAKE, C.byref(kp), None,
+                                    FAKE, FAKE, 1 << 30, None) == 3
+            assert "multiples of 256" in _err(L)
     ok = moe.Pool(moe.Q8_0, 8, 0x1000, 0x1000, 0x1000, None)
     # F not a multiple of 32
     assert L.moe_expert_ffn(FAKE, moe.BF16, 4, 256, 500, 8, 2, FAKE, FAKE, C.byref(ok), None,
@@ -140,7 +152,7 @@ def test_cache_init_argument_errors(moe):
     d = moe.CacheDesc()
     d.n_layers, d.E, d.n_slots, d.qtype = 2, 8, 9, moe.Q8_0      # more slots than experts
     assert L.moe_cache_init(C.byref(d), C.byref(h)) == 3
-    d.n_slots, d.qtype = 4, 3
+    d.n_slots, d.qtype = 4, 9
     assert L.moe_cache_init(C.byref(d), C.byref(h)) == 2
     d.qtype = moe.Q8_0
     assert L.moe_cache_init(C.byref(d), C.byref(h)) == 1          # NULL pools
@@ -217,7 +229,7 @@ def test_streamer_arguments(moe):
     h = C.c_void_p()
     assert L.moe_streamer_init(None, C.byref(h)) == 1
     d = moe.StreamerDesc()
-    d.n_layers, d.E, d.qtype = 2, 8, 3                 # unknown quant type
+    d.n_layers, d.E, d.qtype = 2, 8, 9                 # unknown quant type
     assert L.moe_streamer_init(C.byref(d), C.byref(h)) == 2
     d.qtype = moe.Q8_0
     assert L.moe_streamer_init(C.byref(d), C.byref(h)) == 1   # NULL pools

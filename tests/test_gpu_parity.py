@@ -179,7 +179,7 @@ def _check_layer(moe, L, y_gpu, ids_gpu, n_tok, log=print, extra=None):
         use_ids[tied] = ids_gpu[tied]
         use_g[tied] = gates_at(ref_logits[tied], ids_gpu[tied], cfg.renorm)
     ref = oracle.layer(L.x, use_ids, use_g, L.gate, L.up, L.down, cfg.qtype, cfg.F,
-                       shared=L.shared, tokens=toks)
+                       shared=L.shared, tokens=toks, shared_qtype=cfg.shared_qtype)
     got = y_gpu.float().cpu().numpy()[toks]
     err = rel_err(got, ref)
     assert err <= REL_TOL, err
