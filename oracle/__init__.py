@@ -77,6 +77,11 @@ def _declare(L):
     L.orc_expert_rows.restype = _i
     L.orc_expert_rows.argtypes = [_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p,
                                   _p, _i, _i, _p]
+    L.orc_quantize_act8.restype = None
+    L.orc_quantize_act8.argtypes = [_p, _i, _p, _p]
+    L.orc_layer_a8.restype = _i
+    L.orc_layer_a8.argtypes = [_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p,
+                               _p, _p, _p, _i, _i, _p, _i, _i, C.c_double, _p, _p]
     L.orc_lru_new.restype = _p
     L.orc_lru_new.argtypes = [_i, _i]
     L.orc_lru_free.restype = None
@@ -195,6 +200,50 @@ def layer(x, ids, gates, gate, up, down, qtype, F: int, shared=None,
     if rc != 0:
         raise ValueError("oracle layer: bad arguments")
     return y
+
+
+def quantize_act8(v):
+    """8-bit activation blocks of the rows of v [.., n] (n % 32 == 0):
+    (q int8 [.., n], d float32 [.., n/32])."""
+    v = _c(v, np.float32)
+    n = v.shape[-1]
+    flat = v.reshape(-1, n)
+    q = np.empty(flat.shape, np.int8)
+    d = np.empty((flat.shape[0], n // 32), np.float32)
+    for r in range(flat.shape[0]):
+        qr, dr = q[r], d[r]
+        lib().orc_quantize_act8(_ptr(np.ascontiguousarray(flat[r])), n, _ptr(qr), _ptr(dr))
+    return q.reshape(v.shape), d.reshape(v.shape[:-1] + (n // 32,))
+
+
+def layer_a8(x, ids, gates, gate, up, down, qtype, F: int, shared=None, tokens=None,
+             threads: int = 0, shared_qtype="q8_0", eps: float = 0.0, want_bound=False):
+    """y [n_tok, D] (float64) of the layer with 8-bit activations into every
+    expert matmul; with want_bound, also the per-output room that h codes
+    within eps of a rounding boundary leave (see the C function)."""
+    x = _c(x, np.float32)
+    T, D = x.shape
+    ids = _c(ids, np.int32)
+    k = ids.shape[1]
+    gates = _c(gates, np.float64)
+    gate, up, down = (_c(a, np.uint8) for a in (gate, up, down))
+    E = gate.shape[0]
+    sg = su = sd = None
+    sF = 0
+    if shared is not None:
+        sg, su, sd = (_c(a, np.uint8) for a in shared)
+        sF = sg.shape[1]
+    tl = _c(tokens, np.int32)
+    n = T if tl is None else len(tl)
+    y = np.empty((n, D), np.float64)
+    b = np.empty((n, D), np.float64) if want_bound else None
+    rc = lib().orc_layer_a8(_ptr(x), T, D, F, E, k, _qt(qtype), _ptr(gate), _ptr(up),
+                            _ptr(down), _ptr(ids), _ptr(gates), _ptr(sg), _ptr(su), _ptr(sd),
+                            sF, _qt(shared_qtype), _ptr(tl), n, threads, float(eps), _ptr(y),
+                            _ptr(b))
+    if rc != 0:
+        raise ValueError("oracle layer_a8: bad arguments")
+    return (y, b) if want_bound else y
 
 
 def expert_rows(x, perm, offsets, k: int, gate, up, down, qtype, F: int,

@@ -428,6 +428,151 @@ int orc_expert_rows(const float *x, int T, int D, int F, int E, int k,
     return bad ? -1 : 0;
 }
 
+/* ------------------------------------------------------------------
+ * 8-bit activations (the pages' W4A8 / W8A8 mode: the FreeToken fork README's
+ * note on CUDA W4A8 MMVQ against CPU AVX; the blocks follow ggml's 8-bit
+ * activation format).  Per 32-value block, all in fp32:
+ *   amax = max |v_i|, d = amax / 127, id = (d != 0) ? 1 / d : 0,
+ *   q_i  = round-half-away-from-zero(v_i * id)       (|q_i| <= 127),
+ * and q_i stands for the value q_i * d.  Both sides of a parity test take
+ * these integer decisions with the same fp32 operations. */
+void orc_quantize_act8(const float *v, int n, int8_t *q, float *d)
+{
+    for (int b = 0; b < n / ORC_QK; b++) {
+        const float *vb = v + (size_t)b * ORC_QK;
+        float amax = 0.0f;
+        for (int i = 0; i < ORC_QK; i++) {
+            float a = fabsf(vb[i]);
+            if (a > amax) amax = a;
+        }
+        float db = amax / 127.0f;
+        float id = (db != 0.0f) ? 1.0f / db : 0.0f;
+        d[b] = db;
+        for (int i = 0; i < ORC_QK; i++) {
+            float s = vb[i] * id;
+            q[(size_t)b * ORC_QK + i] = (int8_t)roundf(s);
+        }
+    }
+}
+
+/* Sum over the blocks of one row of d_b * sum_i w_i q_i (w exact, double). */
+static double orc_dot_a8(const double *w, const int8_t *q, const float *d, int n)
+{
+    double acc = 0.0;
+    for (int b = 0; b < n / ORC_QK; b++) {
+        double s = 0.0;
+        for (int i = 0; i < ORC_QK; i++) s += w[b * ORC_QK + i] * (double)q[b * ORC_QK + i];
+        acc += (double)d[b] * s;
+    }
+    return acc;
+}
+
+/* One expert with 8-bit activations: a, u from the quantized x; h = silu(a)
+ * u in double, rounded to fp32 and quantized per block; Y = W_down h^.
+ * If Bd != NULL, Bd[d] = sum over h elements f whose scaled value h_f * id
+ * lies within eps (in code units) of a rounding boundary (k + 1/2) of
+ * dh * |W_down[d, f]|: what one code step of such an element, which an fp32
+ * computation of h may round the other way, can move Y[d]. */
+static void orc_expert_ffn_row_a8(const int8_t *qx, const float *dx, const uint8_t *gate,
+                                  const uint8_t *up, const uint8_t *down, int qtype, int D,
+                                  int F, double *wrow, float *hf, int8_t *qh, float *dh,
+                                  double *Y, double eps, double *Bd)
+{
+    size_t gate_row = orc_row_bytes(qtype, D);
+    size_t down_row = orc_row_bytes(qtype, F);
+    for (int r = 0; r < F; r++) {
+        orc_dequant_row(gate + r * gate_row, qtype, D, wrow);
+        double a = orc_dot_a8(wrow, qx, dx, D);
+        orc_dequant_row(up + r * gate_row, qtype, D, wrow);
+        double u = orc_dot_a8(wrow, qx, dx, D);
+        hf[r] = (float)(orc_silu(a) * u);
+    }
+    orc_quantize_act8(hf, F, qh, dh);
+    for (int d = 0; d < D; d++) {
+        orc_dequant_row(down + d * down_row, qtype, F, wrow);
+        Y[d] = orc_dot_a8(wrow, qh, dh, F);
+        if (Bd) {
+            double bsum = 0.0;
+            for (int f = 0; f < F; f++) {
+                float db = dh[f / ORC_QK];
+                float id = (db != 0.0f) ? 1.0f / db : 0.0f;
+                double sc = (double)(hf[f] * id);
+                double dist = fabs(sc - (floor(sc) + 0.5));
+                if (dist < eps) bsum += (double)db * fabs(wrow[f]);
+            }
+            Bd[d] = bsum;
+        }
+    }
+}
+
+/* The routed layer with 8-bit activations into every expert matmul: x_t
+ * quantized per block (orc_quantize_act8), each expert as above, y_t =
+ * sum_j g_tj Y_tj (+ the shared expert's Y, weight 1).  Arguments as
+ * orc_layer (no dense form; D, F, sh_F multiples of 32 and of the types'
+ * blocks).  bound[n_tok, D] (NULL: not wanted) = sum_j g_tj Bd_tj (+ the
+ * shared Bd) for the given eps. */
+int orc_layer_a8(const float *x, int T, int D, int F, int E, int k, int qtype,
+                 const uint8_t *gate, const uint8_t *up, const uint8_t *down,
+                 const int32_t *ids, const double *gates,
+                 const uint8_t *sh_gate, const uint8_t *sh_up,
+                 const uint8_t *sh_down, int sh_F, int sh_qtype,
+                 const int32_t *tok_list, int n_tok, int nthreads, double eps,
+                 double *y, double *bound)
+{
+    int bw = orc_block_weights(qtype);
+    if (bw == 0 || D % bw || F % bw || k > E || D % ORC_QK || F % ORC_QK) return -1;
+    if (sh_gate && (orc_block_weights(sh_qtype) == 0 || D % orc_block_weights(sh_qtype) ||
+                    sh_F % orc_block_weights(sh_qtype) || sh_F % ORC_QK))
+        return -1;
+    if (!tok_list) n_tok = T;
+    size_t gstride = orc_expert_stride(F, D, qtype);
+    size_t dstride = orc_expert_stride(D, F, qtype);
+    int maxF = F > sh_F ? F : sh_F;
+    int maxW = D > maxF ? D : maxF;
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+#endif
+    for (int n = 0; n < n_tok; n++) {
+        int t = tok_list ? tok_list[n] : n;
+        if (t < 0 || t >= T) { bad |= 1; continue; }
+        int8_t *qx = (int8_t *)malloc((size_t)D);
+        float *dx = (float *)malloc(sizeof(float) * (size_t)(D / ORC_QK));
+        double *wrow = (double *)malloc(sizeof(double) * (size_t)maxW);
+        float *hf = (float *)malloc(sizeof(float) * (size_t)maxF);
+        int8_t *qh = (int8_t *)malloc((size_t)maxF);
+        float *dh = (float *)malloc(sizeof(float) * (size_t)(maxF / ORC_QK));
+        double *Y = (double *)malloc(sizeof(double) * (size_t)D);
+        double *Bd = bound ? (double *)malloc(sizeof(double) * (size_t)D) : NULL;
+        double *yt = y + (size_t)n * D;
+        double *bt = bound ? bound + (size_t)n * D : NULL;
+        orc_quantize_act8(x + (size_t)t * D, D, qx, dx);
+        for (int i = 0; i < D; i++) { yt[i] = 0.0; if (bt) bt[i] = 0.0; }
+        for (int j = 0; j < k; j++) {
+            int e = ids[(size_t)t * k + j];
+            if (e < 0 || e >= E) { bad |= 1; break; }
+            orc_expert_ffn_row_a8(qx, dx, gate + e * gstride, up + e * gstride,
+                                  down + e * dstride, qtype, D, F, wrow, hf, qh, dh, Y, eps, Bd);
+            double g = gates[(size_t)t * k + j];
+            for (int i = 0; i < D; i++) {
+                yt[i] += g * Y[i];
+                if (bt) bt[i] += fabs(g) * Bd[i];
+            }
+        }
+        if (sh_gate) {
+            orc_expert_ffn_row_a8(qx, dx, sh_gate, sh_up, sh_down, sh_qtype, D, sh_F, wrow, hf,
+                                  qh, dh, Y, eps, Bd);
+            for (int i = 0; i < D; i++) {
+                yt[i] += Y[i];
+                if (bt) bt[i] += Bd[i];
+            }
+        }
+        free(qx); free(dx); free(wrow); free(hf); free(qh); free(dh); free(Y); free(Bd);
+    }
+    return bad ? -1 : 0;
+}
+
 /* ------------------------------------------------------------------------
  * Expert-cache LRU simulation (one layer).
  *

@@ -595,3 +595,129 @@ def test_global_lru_invariants_random_trace_with_resizes(orc):
             where[key] = int(slot)
         assert len(where) <= cap and all(sl < cap for sl in where.values())
         assert len(set(where.values())) == len(where)
+
+
+# ------------------------------------------------------- 8-bit activations
+# Hand-worked blocks: with amax = 127 the scale is 1 and the codes are the
+# values rounded half away from zero; with amax = 254 (scale 2, 1/scale = 0.5)
+# and amax = 63.5 (scale 0.5, 1/scale = 2) every product is exact in fp32,
+# so the codes below follow from the rounding rule alone.
+ACT8_CASES = [
+    # values (rest of the 32 zero), scale, codes
+    ([63.5, -63.5, 0.5, -0.5, 1.49, -1.5, 2.5, 126.5, -127.0, 127.0], 1.0,
+     [64, -64, 1, -1, 1, -2, 3, 127, -127, 127]),
+    ([254.0, 3.0, -3.0, 5.0, 1.0, -1.0, 100.9, -0.9], 2.0,
+     [127, 2, -2, 3, 1, -1, 50, 0]),
+    ([63.5, 0.25, -0.25, 0.2, 31.75, -63.5], 0.5,
+     [127, 1, -1, 0, 64, -127]),
+    ([], 0.0, []),                                   # all zero: scale 0, codes 0
+]
+
+
+@pytest.mark.parametrize("vals,scale,codes", ACT8_CASES)
+def test_act8_hand_worked_blocks(orc, vals, scale, codes):
+    v = np.zeros(32, np.float32)
+    v[:len(vals)] = vals
+    q, d = orc.quantize_act8(v[None])
+    assert d[0, 0] == np.float32(scale)
+    want = np.zeros(32, np.int8)
+    want[:len(codes)] = codes
+    np.testing.assert_array_equal(q[0], want)
+
+
+def test_act8_invariants(orc):
+    rng = np.random.default_rng(23)
+    v = (rng.standard_normal((64, 128)) * rng.uniform(0.01, 10, (64, 1))).astype(np.float32)
+    q, d = orc.quantize_act8(v)
+    vb, qb = v.reshape(64, 4, 32), q.reshape(64, 4, 32).astype(np.int64)
+    assert np.abs(qb).max() <= 127
+    # the largest magnitude of each block takes code +-127 with its sign
+    i = np.abs(vb).argmax(axis=2)
+    top = np.take_along_axis(qb, i[..., None], 2)[..., 0]
+    np.testing.assert_array_equal(np.abs(top), 127)
+    assert np.all(np.sign(top) == np.sign(np.take_along_axis(vb, i[..., None], 2)[..., 0]))
+    # round trip within half a step (plus the fp32 rounding of 1/d and v/d)
+    err = np.abs(qb * d[..., None].astype(np.float64) - vb)
+    assert np.all(err <= 0.5 * d[..., None] * (1 + 2.0 ** -20) + 1e-30)
+    # odd symmetry and power-of-two scale invariance
+    qn, dn = orc.quantize_act8(-v)
+    np.testing.assert_array_equal(qn, -q)
+    np.testing.assert_array_equal(dn, d)
+    q4, d4 = orc.quantize_act8(v * np.float32(4))
+    np.testing.assert_array_equal(q4, q)
+    np.testing.assert_array_equal(d4, d * np.float32(4))
+
+
+def test_a8_layer_is_the_a16_layer_when_quantization_is_exact(orc):
+    # x: block 0 holds 127 (scale 1), block 1 holds 254 and 2 (scale 2, codes
+    # 127 and 1): both exact.  Gate rows read x_0 only (a = 127 * 127 =
+    # 16129, where silu(a) = a in double), up rows read x_32 with weight c_r
+    # in {-1, 0, 1} (u = 254 c_r), so h_r = 4096766 c_r = 127 * 32258 c_r:
+    # every h block has scale 32258 (or 0) and codes 127 c_r exactly.  Then
+    # the 8-bit-activation layer equals the 16-bit one in double.
+    D, F = 64, 64
+    x = np.zeros((1, D), np.float32)
+    x[0, 0], x[0, 32], x[0, 33] = 127, 254, 2
+    rng = np.random.default_rng(29)
+    Wg = np.zeros((F, D), np.int64)
+    Wg[:, 0] = 127
+    Wu = np.zeros((F, D), np.int64)
+    c = rng.integers(-1, 2, F)
+    c[:32] = np.where(c[:32] == 0, 1, c[:32])       # block 0 of h is not all zero
+    Wu[:, 32] = c
+    Wd = rng.integers(-3, 4, (D, F))
+    gate, up, down = (_pack_int_matrix(W, "q8_0")[None] for W in (Wg, Wu, Wd))
+    ids, g = np.zeros((1, 1), np.int32), np.ones((1, 1))
+    y16 = orc.layer(x, ids, g, gate, up, down, "q8_0", F)
+    y8, b8 = orc.layer_a8(x, ids, g, gate, up, down, "q8_0", F, eps=1e-3, want_bound=True)
+    np.testing.assert_array_equal(y8, y16)
+    np.testing.assert_array_equal(b8, 0.0)
+    assert np.abs(y16).max() > 1e8                   # not a trivial zero
+
+
+def test_a8_layer_stays_within_the_quantization_error_of_the_a16_layer(orc):
+    # With x on its own 8-bit grid the gate/up part is exact, and the down
+    # projection is linear: y8 - y16 = sum_j g_j W_down (h^ - h) with
+    # |h^_f - h_f| <= dh_b / 2 (+ the fp32 rounding of h), dh_b = max|h_b|/127
+    # (h recomputed here with numpy from the dequantized weights).
+    cfg = S.LayerConfig("a8", T=3, D=256, E=4, k=2, F=256, qtype="q8_0", x_dtype="f32",
+                        y_dtype="f32", seed=31)
+    L = S.make_layer(cfg)
+    # put x on its own 8-bit grid: q * d is exactly representable
+    q, d = orc.quantize_act8(L.x)
+    xg = (q.reshape(3, 8, 32).astype(np.float32) * d[..., None]).reshape(3, 256)
+    _, ids, g = orc.route(xg, L.w_router, None, cfg.k)
+    y16 = orc.layer(xg, ids, g, L.gate, L.up, L.down, "q8_0", cfg.F)
+    y8 = orc.layer_a8(xg, ids, g, L.gate, L.up, L.down, "q8_0", cfg.F)
+    Wd = [orc.dequant_matrix(L.down[e], "q8_0", cfg.F) for e in range(cfg.E)]
+    for t in range(3):
+        bound = np.zeros(cfg.D)
+        for j in range(cfg.k):
+            e = ids[t, j]
+            Wg = orc.dequant_matrix(L.gate[e], "q8_0", cfg.D)
+            Wu = orc.dequant_matrix(L.up[e], "q8_0", cfg.D)
+            a, u = Wg @ xg[t].astype(np.float64), Wu @ xg[t].astype(np.float64)
+            h = a / (1 + np.exp(-a)) * u
+            step = np.abs(h).reshape(-1, 32).max(axis=1) / 127
+            bound += g[t, j] * (np.abs(Wd[e]) @ (np.repeat(step, 32) * (0.5 + 2.0 ** -20)
+                                                 + np.abs(h) * 2.0 ** -23))
+        diff = np.abs(y8[t] - y16[t])
+        assert np.all(diff <= bound + 1e-12), (diff - bound).max()
+        assert diff.max() > 0                          # h was quantized
+
+
+def test_a8_boundary_room_grows_with_eps(orc):
+    cfg = S.LayerConfig("a8b", T=2, D=256, E=4, k=2, F=256, qtype="q4_0", x_dtype="f32",
+                        y_dtype="f32", seed=37)
+    L = S.make_layer(cfg)
+    _, ids, g = orc.route(L.x, L.w_router, None, cfg.k)
+    out = [orc.layer_a8(L.x, ids, g, L.gate, L.up, L.down, "q4_0", cfg.F, eps=e,
+                        want_bound=True) for e in (0.0, 1e-3, 0.5 + 1e-9)]
+    ys = [o[0] for o in out]
+    bs = [o[1] for o in out]
+    for y in ys[1:]:
+        np.testing.assert_array_equal(y, ys[0])        # eps only changes the bound
+    assert np.all(bs[0] == 0.0)
+    assert np.all(bs[1] <= bs[2]) and np.all(bs[1] >= 0)
+    # eps past 1/2: every element counts
+    assert np.all(bs[2] > 0)
