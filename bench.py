@@ -193,6 +193,13 @@ WORKLOADS = {
 # the configuration with its experts encoded in that type
 STD_TYPES = ("q4_1", "q5_0", "q5_1", "q4_k", "q6_k")
 STD_WORKLOADS = [f"{c}_{q}" for q in STD_TYPES for c in ("decode", "prefill")]
+# 8-bit activations into every expert matmul (the W4A8 / W8A8 mode) on the
+# decode layer: Q4_0 experts (W4A8) and the same weights in Q8_0 (W8A8)
+A8_WORKLOADS = {"decode_a8": "q4_0", "decode_w8a8": "q8_0"}
+
+
+def act_bits_of(name):
+    return 8 if name in A8_WORKLOADS else 16
 
 
 def workload_spec(name):
@@ -200,6 +207,9 @@ def workload_spec(name):
     if name in WORKLOADS:
         Ts, replicas = WORKLOADS[name]
         return S.CONFIGS[name.split("_")[0]], Ts, replicas
+    if name in A8_WORKLOADS:
+        Ts, replicas = WORKLOADS["decode"]
+        return dataclasses.replace(S.CONFIGS["decode"], qtype=A8_WORKLOADS[name], name=name), Ts, replicas
     base, qt = name.split("_", 1)
     if base not in ("decode", "prefill") or qt not in STD_TYPES:
         raise ValueError(f"unknown workload {name}")
@@ -245,9 +255,11 @@ class Workload:
             self.shared_bytes = 0
         xdt = torch.bfloat16 if cfg.x_dtype == "bf16" else torch.float32
         ydt = torch.bfloat16 if cfg.y_dtype == "bf16" else torch.float32
+        self.act_bits = act_bits_of(name)
         self.layers = [moe.Layer(p, cfg.D, cfg.F, cfg.E, cfg.k, max(Ts), w_router=dev(base.w_router),
                                  bias=dev(base.bias), shared=shared, shared_F=cfg.shared_F,
-                                 renorm=cfg.renorm, x_dtype=xdt, y_dtype=ydt) for p in pools]
+                                 renorm=cfg.renorm, x_dtype=xdt, y_dtype=ydt,
+                                 act_bits=self.act_bits) for p in pools]
         self.x = {T: _dev_x(self.inputs[T], torch) for T in Ts}
         self.logits = {T: dev(self.inputs[T].logits) for T in Ts}
         self.y = {T: torch.empty((T, cfg.D), dtype=ydt, device="cuda") for T in Ts}
@@ -446,7 +458,9 @@ def measure_layer(wl, steps, warmup, world, local, peaks, no_graph=False, cpu=Tr
     return out
 
 
-def dtype_of(cfg):
+def dtype_of(cfg, act_bits=16):
+    if act_bits == 8:
+        return f"{cfg.qtype} weights, 8-bit activation blocks, int32 accumulate"
     return f"{cfg.qtype} weights, bf16 activations, fp32 accumulate"
 
 
@@ -984,7 +998,7 @@ def _line(out, args, world, cfg, peaks):
     line = {"metric": "MoE-layer tokens/s", "value": out["value"], "unit": out["unit"],
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": out["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": dtype_of(cfg),
+            "vs_baseline": None, "dtype": dtype_of(cfg, act_bits_of(args.workload)),
             "data": "synthetic (seeded; random-init experts in ggml Standard blocks, no checkpoint)"}
     for k, v in out.items():
         if k not in line:
@@ -1004,6 +1018,14 @@ def std_base(cfg_name, qtype, pool):
     cfg, Ts, _ = workload_spec(f"{cfg_name}_{qtype}")
     L = S.make_layer(cfg, T=max(Ts), experts=False)
     L.gate, L.up, L.down = pool
+    return L
+
+
+def std_base_a8(name):
+    """Inputs of the decode configuration over its expert pool encoded in
+    the 8-bit-activation workload's type."""
+    cfg, Ts, _ = workload_spec(name)
+    L = S.make_layer(cfg, T=max(Ts))
     return L
 
 
@@ -1063,6 +1085,13 @@ def run_ours(args, world, rank, local):
                                                  args.no_graph, cpu=with_cpu, cpu_seconds=6.0)
             del w
             torch.cuda.empty_cache()
+        for name in sorted(A8_WORKLOADS):
+            w = Workload(name, torch, moe, base=std_base_a8(name))
+            line["configs"][name] = measure_layer(w, steps, args.warmup, world, local, peaks,
+                                                  args.no_graph, cpu=with_cpu, cpu_seconds=3.0)
+            line["configs"][name]["dtype"] = dtype_of(w.cfg, 8)
+            del w
+            torch.cuda.empty_cache()
         line["configs"]["standard_types"] = measure_std_types(torch, moe, steps, args.warmup,
                                                               world, local, peaks, args.no_graph,
                                                               with_cpu)
@@ -1077,9 +1106,10 @@ def run_ours(args, world, rank, local):
 
 
 # ------------------------------------------------------------ CPU oracle
-def oracle_step_fn(wl_inputs, cfg, Ts, frac=1.0):
+def oracle_step_fn(wl_inputs, cfg, Ts, frac=1.0, act_bits=16):
     import oracle
     oracle.build()
+    run = oracle.layer_a8 if act_bits == 8 else oracle.layer
 
     def step():
         n = 0
@@ -1091,8 +1121,8 @@ def oracle_step_fn(wl_inputs, cfg, Ts, frac=1.0):
                 _, ids, g = oracle.route(L.x, L.w_router, L.bias, cfg.k, cfg.renorm)
             m = max(1, int(round(T * frac)))
             toks = np.arange(m, dtype=np.int32)
-            oracle.layer(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F, shared=L.shared,
-                         tokens=toks, shared_qtype=cfg.shared_qtype)
+            run(L.x, ids, g, L.gate, L.up, L.down, cfg.qtype, cfg.F, shared=L.shared,
+                tokens=toks, shared_qtype=cfg.shared_qtype)
             n += m
         return n
     return step
@@ -1102,7 +1132,7 @@ def cpu_baseline(wl, seconds=10.0):
     """The oracle as it stands, on the host cores, on a bounded sample."""
     cores = os.cpu_count() or 1
     frac = 1.0 if max(wl.Ts) <= 16 else 32.0 / max(wl.Ts)
-    step = oracle_step_fn(wl.inputs, wl.cfg, wl.Ts, frac)
+    step = oracle_step_fn(wl.inputs, wl.cfg, wl.Ts, frac, wl.act_bits)
     t = time.perf_counter()
     n = step()
     dt = time.perf_counter() - t
@@ -1170,7 +1200,7 @@ def run_reference(args, world, rank):
             inputs[T].shared = base.shared
     # size the per-step sample so that warmup + steps end within ~3 minutes
     small = max(Ts) <= 16
-    step = oracle_step_fn(inputs, cfg, Ts, 1.0 if small else 16.0 / max(Ts))
+    step = oracle_step_fn(inputs, cfg, Ts, 1.0 if small else 16.0 / max(Ts), act_bits_of(name))
     t = time.perf_counter()
     n1 = step()
     t1 = time.perf_counter() - t
@@ -1179,7 +1209,7 @@ def run_reference(args, world, rank):
     if t1 > budget:
         frac = max(budget / t1, 1.0 / n1)
     total = sum(Ts)
-    step = oracle_step_fn(inputs, cfg, Ts, frac * (1.0 if small else 16.0 / max(Ts)))
+    step = oracle_step_fn(inputs, cfg, Ts, frac * (1.0 if small else 16.0 / max(Ts)), act_bits_of(name))
     for _ in range(max(0, args.warmup - 1)):
         step()
     t = time.perf_counter()
@@ -1210,7 +1240,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + STD_WORKLOADS + ["cache"],
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + STD_WORKLOADS + sorted(A8_WORKLOADS) + ["cache"],
                     default="decode",
                     help="the workload of the line (decode also reports every other one under "
                          "'configs' unless --no-extra)")

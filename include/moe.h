@@ -300,6 +300,18 @@ moe_status moe_combine(const float *rows, const int32_t *inv, const float *gates
  *                        permutation as moe_permute defines it; when given,
  *                        the call keeps its permutation there instead of in
  *                        the workspace.
+ *   act_bits             0 or 16: 16-bit activations into the expert FFNs (as
+ *                        above); 8: the inputs of every expert matmul (x, and
+ *                        h before the down projection) quantized to 8-bit
+ *                        blocks of 32 -- the fork README's W4A8 / W8A8 MMVQ
+ *                        mode: per block, in fp32, d = max|v| / 127,
+ *                        q = round-half-away-from-zero(v * (1 / d)) (0 when
+ *                        d = 0), and int8 tensor-core products scaled by the
+ *                        weight and activation block scales; the gate weight
+ *                        multiplies each expert's output.  Decode shapes
+ *                        (1 <= T <= 16, the decode GEMV's D and F) with Q4_0
+ *                        or Q8_0 experts only: MOE_ERR_SHAPE or
+ *                        MOE_ERR_UNSUPPORTED_QTYPE otherwise.
  * Phases let an expert cache overlap its miss copies with the FFN of the
  * experts already resident (kongchang article, "From Static Allocation to
  * Dynamic Scheduling"; FreeToken wiki explainer on hiding transfer time):
@@ -372,6 +384,7 @@ typedef struct {
     int32_t *offsets_out;
     int32_t *perm_out;
     int32_t *inv_out;
+    int32_t act_bits;
 } moe_layer_args;
 
 size_t moe_layer_workspace_size(const moe_layer_args *args);

@@ -66,7 +66,7 @@ class LayerArgs(C.Structure):
                 ("gates_out", C.c_void_p), ("logits_out", C.c_void_p),
                 ("trace", C.POINTER(Trace)), ("expert_mask", C.c_void_p),
                 ("counts_out", C.c_void_p), ("offsets_out", C.c_void_p),
-                ("perm_out", C.c_void_p), ("inv_out", C.c_void_p)]
+                ("perm_out", C.c_void_p), ("inv_out", C.c_void_p), ("act_bits", C.c_int32)]
 
 
 class CacheDesc(C.Structure):
@@ -283,8 +283,11 @@ class Layer:
     def __init__(self, pool: ExpertPool, D: int, F: int, E: int, k: int, T_max: int,
                  w_router=None, bias=None, shared: ExpertPool | None = None, shared_F: int = 0,
                  renorm: bool = True, x_dtype=torch.bfloat16, y_dtype=torch.bfloat16,
-                 device="cuda"):
+                 device="cuda", act_bits: int = 16):
+        """act_bits=8: 8-bit activation blocks into every expert matmul (the
+        W4A8 / W8A8 mode; decode shapes with Q4_0 / Q8_0 experts)."""
         _dev(w_router, bias)
+        self.act_bits = int(act_bits)
         self.pool, self.shared = pool, shared
         self.D, self.F, self.E, self.k, self.shared_F = D, F, E, k, shared_F
         self.w_router, self.bias = w_router, bias
@@ -315,6 +318,7 @@ class Layer:
         a.logits_out = None if logits_out is None else logits_out.data_ptr()
         a.trace = C.pointer(trace) if trace is not None else None
         a.phases = int(phases)
+        a.act_bits = self.act_bits
         a.expert_mask = None if mask is None else mask.data_ptr()
         if routing_out is not None:
             a.counts_out, a.offsets_out, a.perm_out, a.inv_out = (t.data_ptr() for t in routing_out)

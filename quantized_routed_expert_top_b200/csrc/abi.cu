@@ -296,6 +296,28 @@ moe_status moe_layer_forward(const moe_layer_args *a, void *workspace, size_t ws
         set_error("moe_layer_forward: phases %d has bits outside MOE_PHASE_ALL", (int)a->phases);
         return MOE_ERR_INVALID_ARG;
     }
+    if (a->act_bits != 0 && a->act_bits != 8 && a->act_bits != 16) {
+        set_error("moe_layer_forward: act_bits %d is not 0, 8 or 16", (int)a->act_bits);
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (a->act_bits == 8) {
+        const int sqt = a->shared ? a->shared->qtype : MOE_Q8_0;
+        if (a->pool->qtype != MOE_Q4_0 && a->pool->qtype != MOE_Q8_0) {
+            set_error("moe_layer_forward: 8-bit activations need Q4_0 or Q8_0 experts (got %d)",
+                      (int)a->pool->qtype);
+            return MOE_ERR_UNSUPPORTED_QTYPE;
+        }
+        if (sqt != MOE_Q4_0 && sqt != MOE_Q8_0) {
+            set_error("moe_layer_forward: 8-bit activations need a Q4_0 or Q8_0 shared expert (got %d)", sqt);
+            return MOE_ERR_UNSUPPORTED_QTYPE;
+        }
+        if (a->T > 0 && !decode_a8_ok(a->T, a->D, a->F, a->shared ? a->shared_F : 0, a->pool->qtype, sqt)) {
+            set_error("moe_layer_forward: 8-bit activations run on decode shapes only (1 <= T <= 16, "
+                      "D in {256, 512, 768, 1024, 2048}, F and shared_F multiples of 256 up to 1024; "
+                      "T=%d D=%d F=%d)", a->T, a->D, a->F);
+            return MOE_ERR_SHAPE;
+        }
+    }
     if (a->T == 0) return MOE_OK;
     const unsigned ph = a->phases ? (unsigned)a->phases : MOE_PHASE_ALL;
     const bool need_x = (ph & (MOE_PHASE_FFN | MOE_PHASE_SHARED)) || ((ph & MOE_PHASE_ROUTE) && a->w_router);

@@ -1071,6 +1071,559 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
     }
 }
 
+// ------------------------------------------------------ 8-bit activations
+// The W4A8 / W8A8 mode (FreeToken fork README, the note on CUDA W4A8 MMVQ):
+// the inputs of every expert matmul are 8-bit blocks of 32 (per block, in
+// fp32: d = max|v| / 127, q = round-half-away(v * (1 / d))), and int8 tensor-
+// core products (mma.sync m16n8k32, int32 accumulate) are scaled by the
+// weight block's d and the activation block's d.  Q8_0 codes are the A
+// fragment as they lie in shared memory; Q4_0 nibbles become unsigned bytes
+// with two masks, the -8 offset entering through the accumulator input as
+// -8 * (sum of the activation codes).  Gate/up units hold 32 rows of F (one
+// h block), so the epilogue quantizes h in place; the down kernel scales its
+// rows by the gate weight (h is quantized without it).
+struct A8Args {
+    DecArgs d;
+    int8_t *hq;          // [T*k + T][hq_row] h codes, permuted order (+ shared rows)
+    float2 *hs;          // [T*k + T][hq_row / 32] (scale, sum of the codes) per h block
+    int hq_row;          // bytes per hq row = max(F, shared F)
+};
+struct A8Maps {
+    DecMaps m;           // gate/up: boxes of 32 rows; down: boxes of 64 rows
+    CUtensorMap hq;      // h codes: boxes of hrows rows x a padded row
+};
+constexpr int kA8Rows = 32;
+constexpr int kA8MaxSb = 32;                     // blocks per K-slice
+__host__ __device__ inline int a8_xrow(int D) { return D + 16; }   // staged x-code row
+
+// 32 activations of token t, block b (bf16 or fp32, as the 16-bit path reads them)
+__device__ __forceinline__ void a8_load_block(const DecArgs &a, int t, int b, float *v) {
+    const size_t xb = (size_t)t * a.D + (size_t)b * QK;
+    if (a.x_vec && a.x_bf16) {
+        const uint4 *p = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)a.x + xb);
+        uint4 w[4];
+#pragma unroll
+        for (int q = 0; q < 4; q++) w[q] = __ldg(p + q);
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const uint32_t u[4] = {w[q].x, w[q].y, w[q].z, w[q].w};
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                v[8 * q + 2 * r] = __uint_as_float(u[r] << 16);
+                v[8 * q + 2 * r + 1] = __uint_as_float(u[r] & 0xFFFF0000u);
+            }
+        }
+    } else if (a.x_vec) {
+        const float4 *p = reinterpret_cast<const float4 *>((const float *)a.x + xb);
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+            const float4 w = __ldg(p + q);
+            v[4 * q] = w.x; v[4 * q + 1] = w.y; v[4 * q + 2] = w.z; v[4 * q + 3] = w.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++)
+            v[i] = a.x_bf16 ? load_act((const __nv_bfloat16 *)a.x, xb + i)
+                            : load_act((const float *)a.x, xb + i);
+    }
+}
+
+// 8-bit code of v with block scale reciprocal id (round half away from zero)
+__device__ __forceinline__ int a8_code(float v, float id) { return (int)roundf(v * id); }
+
+// A fragment of a Q8_0 / Q4_0 block for rows g (blk_lo) and g+8 (blk_hi);
+// MIS: alignment mod 4 of the block's codes
+template <bool Q8, int MIS>
+__device__ __forceinline__ void a8_weight_frag(uint32_t blk_lo, uint32_t blk_hi, int c, uint32_t *a) {
+    const uint32_t o = 2 + 4 * c;
+    if constexpr (Q8) {
+        a[0] = lds_word<MIS>(blk_lo + o);
+        a[1] = lds_word<MIS>(blk_hi + o);
+        a[2] = lds_word<MIS>(blk_lo + o + 16);
+        a[3] = lds_word<MIS>(blk_hi + o + 16);
+    } else {
+        const uint32_t wl = lds_word<MIS>(blk_lo + o), wh = lds_word<MIS>(blk_hi + o);
+        a[0] = wl & 0x0F0F0F0Fu;
+        a[2] = (wl >> 4) & 0x0F0F0F0Fu;
+        a[1] = wh & 0x0F0F0F0Fu;
+        a[3] = (wh >> 4) & 0x0F0F0F0Fu;
+    }
+}
+
+// One K-slice of the 32-row unit for one warp: WB blocks from the warp's
+// first block; row: staged row g at that block (tile 0); xb: column g's x
+// codes at that block + 4c; dx0/dx1, s0/s1: column 2c / 2c+1's block scales
+// and code sums at that block.
+template <bool Q8, int WB, int MIS0>
+__device__ __forceinline__ void gateup_slice_a8(uint32_t row, uint32_t r8, uint32_t r16, uint32_t xb,
+                                                uint32_t dx0a, uint32_t dx1a, uint32_t s0a, uint32_t s1a,
+                                                int c, float (*acc)[4]) {
+    constexpr int BS = Q8 ? kQ8Bytes : kQ4Bytes;
+#pragma unroll
+    for (int bl = 0; bl < WB; bl++) {
+        const uint32_t blk = row + bl * BS;
+        const uint32_t b0 = lds32(xb + bl * 32), b1 = lds32(xb + bl * 32 + 16);
+        const float dx0 = ldsf(dx0a + bl * 4), dx1 = ldsf(dx1a + bl * 4);
+        int ci[4] = {0, 0, 0, 0};
+        if constexpr (!Q8) {
+            const int c0 = -8 * (int)lds32(s0a + bl * 4), c1 = -8 * (int)lds32(s1a + bl * 4);
+            ci[0] = c0; ci[1] = c1; ci[2] = c0; ci[3] = c1;
+        }
+#pragma unroll
+        for (int tt = 0; tt < 2; tt++) {
+            const uint32_t bt = blk + tt * r16;
+            uint32_t af[4];
+            if (((MIS0 + bl * BS + 2) & 3) == 0) a8_weight_frag<Q8, 0>(bt, bt + r8, c, af);
+            else a8_weight_frag<Q8, 2>(bt, bt + r8, c, af);
+            const float dlo = h2f(lds16(bt)), dhi = h2f(lds16(bt + r8));
+            int p[4];
+            if constexpr (Q8) imma_s8s8(p, af, b0, b1, ci);
+            else imma_u8s8(p, af, b0, b1, ci);
+            acc[tt][0] = fmaf(dlo * dx0, (float)p[0], acc[tt][0]);
+            acc[tt][1] = fmaf(dlo * dx1, (float)p[1], acc[tt][1]);
+            acc[tt][2] = fmaf(dhi * dx0, (float)p[2], acc[tt][2]);
+            acc[tt][3] = fmaf(dhi * dx1, (float)p[3], acc[tt][3]);
+        }
+    }
+}
+
+template <int WB>
+__global__ void __launch_bounds__(kGThreads, 1)
+dec_gateup_a8_kernel(A8Args A, int S, const __grid_constant__ A8Maps maps) {
+    const DecArgs &a = A.d;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int T = a.T, D = a.D;
+    const int nbD = D / QK;
+    const GuGeo geoR = gu_geo(D, a.qt, kA8MaxSb), geoS = gu_geo(D, a.sqt, kA8MaxSb);
+    const int pitch_max = max(geoR.pitch, a.sF > 0 ? geoS.pitch : 0);
+    const int stage_bytes = (int)round_up((size_t)2 * kA8Rows * pitch_max, 128);
+    const int xrow = a8_xrow(D);
+    const int mat = warp >> 3, kg = warp & 7;
+
+    // carve (1024-aligned base): x codes [T+1 rows, the last zero] | scales
+    // [T+1][nbD] | code sums [T+1][nbD] | stages | red [NB][kDW][2][32][4] |
+    // barriers | act | tok | units
+    uint8_t *base = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
+    const size_t xs_bytes = round_up((size_t)(T + 1) * xrow, 16);
+    uint8_t *xs = base;
+    float *dxt = (float *)(base + xs_bytes);
+    int *sqt = (int *)(dxt + (size_t)(T + 1) * nbD);
+    uint8_t *stages = base + round_up(xs_bytes + (size_t)2 * (T + 1) * nbD * 4, 1024);
+    constexpr int NB = kGuRedBufs;
+    float *red = (float *)(stages + (size_t)S * stage_bytes);
+    uint64_t *full = (uint64_t *)(red + NB * kDW * 2 * 32 * 4);
+    uint64_t *empty = full + kMaxStages;
+    uint64_t *rfull = empty + kMaxStages;
+    uint64_t *rempty = rfull + 4;
+    int *act = (int *)(rempty + 4);
+    int *tok = act + 6 * (a.E + 1);
+    int4 *utab = reinterpret_cast<int4 *>(
+        (reinterpret_cast<uintptr_t>(tok + kMaxTk + 16 + kMaxTk + 16) + 15) & ~(uintptr_t)15);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kDW);
+        }
+        for (int b = 0; b < NB; b++) {
+            mbar_init(&rfull[b], kDW);
+            mbar_init(&rempty[b], kEW);
+        }
+        fence_mbar_init();
+    }
+    // x -> 8-bit codes, one (token, block) per thread (row T: zero codes),
+    // before waiting for the routing kernel this grid may overlap with
+    for (int idx = tid; idx < (T + 1) * nbD; idx += kGThreads) {
+        const int t = idx / nbD, b = idx % nbD;
+        float v[32];
+        if (t < T) {
+            a8_load_block(a, t, b, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; i++) v[i] = 0.f;
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
+        const float dx = amax / 127.f;
+        const float id = dx != 0.f ? 1.f / dx : 0.f;
+        uint32_t w[8];
+        int sum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                const int code = a8_code(v[4 * q + r], id);
+                sum += code;
+                word |= ((uint32_t)code & 0xFFu) << (8 * r);
+            }
+            w[q] = word;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)t * xrow + b * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        dxt[idx] = dx;
+        sqt[idx] = sum;
+    }
+    __syncthreads();
+    pdl_wait();
+    pdl_launch_dependents();
+    load_token_tables(a, tok, nullptr);
+    const Active Av = build_active_list(a, act);   // includes __syncthreads
+    const int tiles_r = a.F / kA8Rows, tiles_s = a.sF / kA8Rows;
+    int *ucum = act + 4 * (a.E + 1);
+    if (warp == 0) {
+        int base_u = 0;
+        for (int v0 = 0; v0 < Av.n_virt; v0 += 32) {
+            const int v = v0 + lane;
+            int nu = 0;
+            if (v < Av.n_virt) {
+                const Virt vi = virt(a, act, Av.n_routed, v);
+                nu = (vi.cnt + kGuCols - 1) / kGuCols * (vi.shared ? tiles_s : tiles_r);
+            }
+            int incl = nu;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t2;
+            }
+            if (v < Av.n_virt) ucum[v] = base_u + incl - nu;
+            base_u += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) ucum[Av.n_virt] = base_u;
+    }
+    __syncthreads();
+    const int U = ucum[Av.n_virt];
+    const int n_local = U > (int)blockIdx.x ? (U - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    for (int i = tid; i < n_local; i += blockDim.x) {
+        const int u = blockIdx.x + i * gridDim.x;
+        int lo = 0, hi = Av.n_virt - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (ucum[mid] <= u) lo = mid; else hi = mid - 1;
+        }
+        const Virt vi = virt(a, act, Av.n_routed, lo);
+        const int tv = vi.shared ? tiles_s : tiles_r;
+        const int rem = u - ucum[lo], grp = rem / tv, tile = rem % tv;
+        utab[i] = make_int4(lo, tile, vi.seg0 + grp * kGuCols, min(kGuCols, vi.cnt - grp * kGuCols));
+    }
+    __syncthreads();
+
+    if (warp == kDW) {
+        // ---------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol = l2_evict_first_policy();
+            int stage = 0;
+            uint32_t phase = 0, used = 0u, last_ph = 0u;
+            bool ok = true;
+            for (int i = 0; i < n_local && ok; i++) {
+                const int v = utab[i].x, tile = utab[i].y;
+                const Virt vi = virt(a, act, Av.n_routed, v);
+                const int bs = qt_bytes(vi.qt);
+                const GuGeo gg = vi.shared ? geoS : geoR;
+                const CUtensorMap *mg = vi.shared ? &maps.m.sgate : &maps.m.gate;
+                const CUtensorMap *mu = vi.shared ? &maps.m.sup : &maps.m.up;
+                const int y = (vi.shared ? 0 : (int)vi.slot * a.F) + tile * kA8Rows;
+                for (int sl = 0; sl < gg.nsl; sl++) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                    uint8_t *dst = stages + (size_t)stage * stage_bytes;
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(2 * kA8Rows * gg.pitch));
+                    const int x = sl * gg.sb * bs / 8;
+                    tma_load_2d_hint(dst, mg, x, y, &full[stage], pol);
+                    tma_load_2d_hint(dst + kA8Rows * gg.pitch, mu, x, y, &full[stage], pol);
+                    used |= 1u << stage;
+                    last_ph = (last_ph & ~(1u << stage)) | (phase << stage);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+            drain_fills(full, S, used, last_ph, a.err);
+        }
+        return;
+    }
+
+    if (warp > kDW) {
+        // ----------------------------------------------------- epilogue
+        // unit j: thread (column n = et / 8, row group rg = et % 8) sums the
+        // K-group partials of rows 4rg..4rg+3, forms h, and quantizes the
+        // column's 32 h values with the 8 threads of its column
+        const int et = tid - kDThreads;
+        const int n = et >> 3, rg = et & 7;
+        for (int j = 0; j < n_local; j++) {
+            const int b = j % NB;
+            if (!mbar_wait_warp(&rfull[b], (uint32_t)((j / NB) & 1), a.err, kErrTimeoutFull)) return;
+            const int4 ud = utab[j];
+            const int tile = ud.y, seg0 = ud.z, cnt = ud.w;
+            const float *redb = red + (size_t)b * kDW * 2 * 128;
+            float h[4];
+            float m = 0.f;
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                const int row = 4 * rg + r, tt = row >> 4, rr = row & 15;
+                const int L = (rr & 7) * 4 + (n >> 1);
+                const int q = ((rr >> 3) << 1) | (n & 1);
+                float sg = 0.f, su = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; w++) {
+                    sg += redb[((size_t)w * 2 + tt) * 128 + L * 4 + q];
+                    su += redb[((size_t)(8 + w) * 2 + tt) * 128 + L * 4 + q];
+                }
+                h[r] = silu(sg) * su;
+                m = fmaxf(m, fabsf(h[r]));
+            }
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            const float dh = m / 127.f;
+            const float id = dh != 0.f ? 1.f / dh : 0.f;
+            uint32_t word = 0;
+            int sum = 0;
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                const int code = a8_code(h[r], id);
+                sum += code;
+                word |= ((uint32_t)code & 0xFFu) << (8 * r);
+            }
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (n < cnt) {
+                const int pos = seg0 + n;
+                *reinterpret_cast<uint32_t *>(A.hq + (size_t)pos * A.hq_row + tile * kA8Rows + 4 * rg) = word;
+                if (rg == 0) A.hs[(size_t)pos * (A.hq_row / QK) + tile] = make_float2(dh, (float)sum);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[b]);
+        }
+        return;
+    }
+
+    // ------------------------------------------------------ MMA warps
+    const uint32_t xs_a = smem_u32(xs), dx_a = smem_u32(dxt), sq_a = smem_u32(sqt);
+    const uint32_t st_a = smem_u32(stages);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int j = 0; j < n_local && ok; j++) {
+        const int4 ud = utab[j];
+        const int seg0 = ud.z, cnt = ud.w;
+        const bool shu = ud.x >= Av.n_routed;
+        const bool q8 = (shu ? a.sqt : a.qt) == MOE_Q8_0;
+        const GuGeo gg = shu ? geoS : geoR;
+        const int kb0 = kg * WB;
+        const int tb = g < cnt ? tok[seg0 + g] : T;
+        const int t0 = 2 * c < cnt ? tok[seg0 + 2 * c] : T;
+        const int t1 = 2 * c + 1 < cnt ? tok[seg0 + 2 * c + 1] : T;
+        const uint32_t xb = xs_a + tb * xrow + kb0 * 32 + c * 4;
+        float acc[2][4];
+#pragma unroll
+        for (int tt = 0; tt < 2; tt++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) acc[tt][q] = 0.f;
+        const int bsz = q8 ? kQ8Bytes : kQ4Bytes;
+        const int mis0 = (kb0 * bsz) & 3;
+        const uint32_t r8 = 8u * gg.pitch, r16 = 16u * gg.pitch;
+        for (int sl = 0; sl < gg.nsl; sl++) {
+            if (!mbar_wait_warp(&full[stage], phase, a.err, kErrTimeoutFull)) { ok = false; break; }
+            const uint32_t row = st_a + stage * stage_bytes + (mat * kA8Rows + g) * gg.pitch + kb0 * bsz;
+            const int kb = sl * gg.sb + kb0;              // first block of this warp in the row
+            const uint32_t xbs = xb + sl * gg.sb * 32;
+            const uint32_t d0 = dx_a + (uint32_t)((t0 * nbD + kb) * 4), d1 = dx_a + (uint32_t)((t1 * nbD + kb) * 4);
+            const uint32_t s0 = sq_a + (uint32_t)((t0 * nbD + kb) * 4), s1 = sq_a + (uint32_t)((t1 * nbD + kb) * 4);
+            if (q8) {
+                if (mis0 == 0) gateup_slice_a8<true, WB, 0>(row, r8, r16, xbs, d0, d1, s0, s1, c, acc);
+                else gateup_slice_a8<true, WB, 2>(row, r8, r16, xbs, d0, d1, s0, s1, c, acc);
+            } else {
+                if (mis0 == 0) gateup_slice_a8<false, WB, 0>(row, r8, r16, xbs, d0, d1, s0, s1, c, acc);
+                else gateup_slice_a8<false, WB, 2>(row, r8, r16, xbs, d0, d1, s0, s1, c, acc);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        const int b = j % NB;
+        if (j >= NB && !mbar_wait_warp(&rempty[b], (uint32_t)((j / NB - 1) & 1), a.err, kErrTimeoutEmpty)) {
+            ok = false;
+            break;
+        }
+        float *rw = red + ((size_t)b * kDW + warp) * 2 * 128;
+#pragma unroll
+        for (int tt = 0; tt < 2; tt++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) rw[tt * 128 + lane * 4 + q] = acc[tt][q];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfull[b]);
+    }
+}
+
+// Down with 8-bit h: unit = (expert, 64 rows of D) as the 16-bit kernel; the
+// stage holds the 64-row weight box, the expert's h-code rows (one box of
+// hrows rows, padded so that the B loads of 8 columns hit distinct banks)
+// and their (scale, code sum) pairs.
+template <int NT>
+__global__ void __launch_bounds__(kDThreads, 1)
+dec_down_a8_kernel(A8Args A, int G, int Sg, int hrows, int hpitch, const __grid_constant__ A8Maps maps) {
+    const DecArgs &a = A.d;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int D = a.D;
+    const int S = G * Sg;
+    const int hsrow = A.hq_row / QK * 8;                 // bytes of one row of (scale, sum) pairs
+    const int pr = tma_row_bytes((int)qt_row_bytes(a.qt, a.F));
+    const int ps = a.sF > 0 ? tma_row_bytes((int)qt_row_bytes(a.sqt, a.sF)) : 0;
+    const int wbytes = kDnRows * (pr > ps ? pr : ps);
+    const int hbytes = (int)round_up((size_t)hrows * hpitch, 128);
+    const int stage_bytes = (int)round_up((size_t)wbytes + hbytes + (size_t)hrows * hsrow, 128);
+    const int grp = warp >> 2, mt = warp & 3;
+
+    uint8_t *stages = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
+    uint64_t *full = (uint64_t *)(stages + (size_t)S * stage_bytes);
+    uint64_t *empty = full + kMaxStages;
+    int *act = (int *)(empty + kMaxStages);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 4);
+        }
+        fence_mbar_init();
+    }
+    const Active Av = build_active_list(a, act);
+    const int tiles = D / kDnRows;
+    const int U = Av.n_virt * tiles;
+
+    if (warp == kDW) {
+        if (lane == 0) {
+            const uint64_t pol = l2_evict_first_policy();
+            bool ok = true, waited = false;
+            uint32_t used = 0u, last_ph = 0u;
+            int pend_s[kMaxStages], pend_v[kMaxStages];
+            int npend = 0;
+            auto issue_h = [&](int st, int v) {
+                const Virt vi = virt(a, act, Av.n_routed, v);
+                uint8_t *dst = stages + (size_t)st * stage_bytes + wbytes;
+                tma_load_2d(dst, &maps.hq, 0, vi.seg0, &full[st]);
+                bulk_g2s(dst + hbytes, A.hs + (size_t)vi.seg0 * (A.hq_row / QK),
+                         (uint32_t)(vi.cnt * hsrow), &full[st]);
+            };
+            int i = 0;
+            for (int u = blockIdx.x; u < U && ok; u += gridDim.x, i++) {
+                const int v = u / tiles, dt = u % tiles;
+                const DnSlot sl = dn_slot(i, G, Sg);
+                const Virt vi = virt(a, act, Av.n_routed, v);
+                const int pitch = vi.shared ? ps : pr;
+                if (!mbar_wait(&empty[sl.stage], sl.phase ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                uint8_t *dst = stages + (size_t)sl.stage * stage_bytes;
+                mbar_arrive_expect_tx(&full[sl.stage],
+                                      (uint32_t)(kDnRows * pitch + hrows * hpitch + vi.cnt * hsrow));
+                tma_load_2d_hint(dst, vi.shared ? &maps.m.sdown : &maps.m.down, 0,
+                                 (vi.shared ? 0 : (int)vi.slot * D) + dt * kDnRows, &full[sl.stage], pol);
+                used |= 1u << sl.stage;
+                last_ph = (last_ph & ~(1u << sl.stage)) | (sl.phase << sl.stage);
+                if (waited) {
+                    issue_h(sl.stage, v);
+                } else {
+                    pend_s[npend] = sl.stage; pend_v[npend] = v; npend++;
+                    if (npend == S) {
+                        pdl_wait();
+                        waited = true;
+                        for (int q = 0; q < npend; q++) issue_h(pend_s[q], pend_v[q]);
+                        npend = 0;
+                    }
+                }
+            }
+            if (!waited) {
+                pdl_wait();
+                for (int q = 0; q < npend; q++) issue_h(pend_s[q], pend_v[q]);
+            }
+            drain_fills(full, S, used, last_ph, a.err);
+        }
+        return;
+    }
+    if (grp >= G) return;
+
+    const uint32_t st_a = smem_u32(stages);
+    int i = grp;
+    for (int u = blockIdx.x + grp * gridDim.x; u < U; u += G * gridDim.x, i += G) {
+        const int v = u / tiles, dt = u % tiles;
+        const DnSlot sl = dn_slot(i, G, Sg);
+        const Virt vi = virt(a, act, Av.n_routed, v);
+        const bool q8 = vi.qt == MOE_Q8_0;
+        const int bsz = q8 ? kQ8Bytes : kQ4Bytes;
+        const int pitch = vi.shared ? ps : pr;
+        const int nb = vi.Fv / QK;
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
+        if (!mbar_wait_warp(&full[sl.stage], sl.phase, a.err, kErrTimeoutFull)) break;
+        const uint32_t sbase = st_a + sl.stage * stage_bytes;
+        const uint32_t row = sbase + (mt * kTile + g) * pitch;
+        const uint32_t r8 = 8u * pitch;
+        const uint32_t hq_s = sbase + wbytes;
+        const float2 *hs_s = reinterpret_cast<const float2 *>(stages + (size_t)sl.stage * stage_bytes +
+                                                              wbytes + hbytes);
+        const int hs2 = hsrow / 8;                        // pairs per row
+        uint32_t hb[NT];
+        const float2 *sc0[NT], *sc1[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+            const int n = g + 8 * nt, n0 = 8 * nt + 2 * c, n1 = n0 + 1;
+            // columns past the expert's rows read whatever the stage holds
+            // there; a column depends only on its own B column and its own
+            // scale, and those columns are never stored
+            hb[nt] = hq_s + (n < hrows ? n : 0) * hpitch + c * 4;
+            sc0[nt] = hs_s + (n0 < hrows ? n0 : 0) * hs2;
+            sc1[nt] = hs_s + (n1 < hrows ? n1 : 0) * hs2;
+        }
+        const int ntile = vi.cnt > 8 ? 2 : 1;
+        for (int b = 0; b < nb; b++) {
+            const uint32_t blk = row + b * bsz;
+            const int mis = (b * bsz + 2) & 3;
+            uint32_t af[4];
+            if (q8) { if (mis == 0) a8_weight_frag<true, 0>(blk, blk + r8, c, af); else a8_weight_frag<true, 2>(blk, blk + r8, c, af); }
+            else { if (mis == 0) a8_weight_frag<false, 0>(blk, blk + r8, c, af); else a8_weight_frag<false, 2>(blk, blk + r8, c, af); }
+            const float dlo = h2f(lds16(blk)), dhi = h2f(lds16(blk + r8));
+#pragma unroll
+            for (int nt = 0; nt < NT; nt++) {
+                if (nt >= ntile) break;
+                const uint32_t b0 = lds32(hb[nt] + b * 32), b1 = lds32(hb[nt] + b * 32 + 16);
+                const float2 h0 = sc0[nt][b], h1 = sc1[nt][b];
+                int ci[4] = {0, 0, 0, 0};
+                if (!q8) {
+                    const int c0 = -8 * (int)h0.y, c1 = -8 * (int)h1.y;
+                    ci[0] = c0; ci[1] = c1; ci[2] = c0; ci[3] = c1;
+                }
+                int p[4];
+                if (q8) imma_s8s8(p, af, b0, b1, ci);
+                else imma_u8s8(p, af, b0, b1, ci);
+                acc[nt][0] = fmaf(dlo * h0.x, (float)p[0], acc[nt][0]);
+                acc[nt][1] = fmaf(dlo * h1.x, (float)p[1], acc[nt][1]);
+                acc[nt][2] = fmaf(dhi * h0.x, (float)p[2], acc[nt][2]);
+                acc[nt][3] = fmaf(dhi * h1.x, (float)p[3], acc[nt][3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[sl.stage]);
+        // the gate weight of each column (1 for the shared expert's rows)
+        float* out = a.rows_out + (size_t)vi.seg0 * D + dt * kDnRows + mt * kTile;
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const int n = nt * 8 + 2 * c + (q & 1);
+                const int r = g + ((q >> 1) << 3);
+                if (n < vi.cnt) {
+                    const float gw = (vi.shared || !a.gates) ? 1.f : __ldg(a.gates + __ldg(a.perm + vi.seg0 + n));
+                    out[(size_t)n * D + r] = acc[nt][q] * gw;
+                }
+            }
+    }
+}
+
 // y[t, :] = sum_j rows[inv[t*k + j], :] (+ rows[T*k + t, :] for the shared
 // expert), in j order; rows already carry the gate weight.
 __global__ void __launch_bounds__(256)
@@ -1369,6 +1922,167 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
         return MOE_ERR_INVALID_ARG;
     }
     return T > 8 ? run_decode<2>(a, pool.n_slots, s, tr) : run_decode<1>(a, pool.n_slots, s, tr);
+}
+
+// ------------------------------------------------ 8-bit activations: host
+static bool a8_type_ok(int q) { return q == MOE_Q4_0 || q == MOE_Q8_0; }
+
+bool decode_a8_ok(int T, int D, int F, int sF, int qt, int sqt) {
+    return decode_path_ok(T, D, F, sF, qt, sqt) && a8_type_ok(qt) && (sF == 0 || a8_type_ok(sqt));
+}
+size_t decode_a8_hq_bytes(int T, int k, int F, int sF) {
+    return (size_t)(T * k + T) * (size_t)std::max(F, sF);
+}
+size_t decode_a8_hs_bytes(int T, int k, int F, int sF) {
+    return (size_t)(T * k + T) * (size_t)(std::max(F, sF) / QK) * sizeof(float2);
+}
+
+static moe_status encode_maps_a8(const A8Args &A, int n_slots, int hrows, int hpitch, A8Maps *m) {
+    memset(m, 0, sizeof(*m));
+    const DecArgs &a = A.d;
+    const size_t rg = qt_row_bytes(a.qt, a.D);
+    const GuGeo gr = gu_geo(a.D, a.qt, kA8MaxSb);
+    moe_status st;
+    if ((st = encode_rows(&m->m.gate, a.gate, rg, (size_t)n_slots * a.F, gr.pitch, kA8Rows))) return st;
+    if ((st = encode_rows(&m->m.up, a.up, rg, (size_t)n_slots * a.F, gr.pitch, kA8Rows))) return st;
+    const size_t rbd = qt_row_bytes(a.qt, a.F);
+    if ((st = encode_rows(&m->m.down, a.down, rbd, (size_t)n_slots * a.D, tma_row_bytes((int)rbd), kDnRows)))
+        return st;
+    if (a.sF > 0) {
+        const size_t rgs = qt_row_bytes(a.sqt, a.D);
+        const GuGeo gs = gu_geo(a.D, a.sqt, kA8MaxSb);
+        if ((st = encode_rows(&m->m.sgate, a.sh_gate, rgs, a.sF, gs.pitch, kA8Rows))) return st;
+        if ((st = encode_rows(&m->m.sup, a.sh_up, rgs, a.sF, gs.pitch, kA8Rows))) return st;
+        const size_t rbs = qt_row_bytes(a.sqt, a.sF);
+        if ((st = encode_rows(&m->m.sdown, a.sh_down, rbs, a.D, tma_row_bytes((int)rbs), kDnRows))) return st;
+    }
+    // h codes: rows of hq_row bytes; a box of hrows rows and hpitch bytes
+    // (the bytes past a row read as zeros)
+    return encode_rows(&m->hq, A.hq, (size_t)A.hq_row, (size_t)(a.T * a.k + a.T), hpitch, hrows);
+}
+
+template <int WB>
+static cudaError_t launch_gateup_a8(const A8Args &A, const A8Maps &m, int grid, size_t smem,
+                                    cudaStream_t s, int S) {
+    return launch_pdl(dec_gateup_a8_kernel<WB>, grid, kGThreads, smem, s, A, S, m);
+}
+
+template <int NT>
+static moe_status run_decode_a8(const A8Args &A, int n_slots, cudaStream_t s, Tracer *tr) {
+    const DecArgs &a = A.d;
+    const int sms = num_sms();
+    const int hrows = std::min(a.T, 16);
+    const int hpitch = tma_row_bytes(A.hq_row);
+    A8Maps maps;
+    moe_status st = encode_maps_a8(A, n_slots, hrows, hpitch, &maps);
+    if (st != MOE_OK) return st;
+    if (a.routed || a.sF > 0) {
+        // ---- gate/up with h quantized in the epilogue
+        const int nbD = a.D / QK;
+        const int pitch = std::max(gu_geo(a.D, a.qt, kA8MaxSb).pitch,
+                                   a.sF > 0 ? gu_geo(a.D, a.sqt, kA8MaxSb).pitch : 0);
+        const int stage_bytes = (int)round_up((size_t)2 * kA8Rows * pitch, 128);
+        const int groups = a.E + (a.T * a.k) / kGuCols;
+        const int U_max = groups * (a.F / kA8Rows) + (a.T + kGuCols - 1) / kGuCols * (a.sF / kA8Rows);
+        const int grid = std::max(1, std::min(sms, U_max));
+        const size_t units = (size_t)((U_max + grid - 1) / grid) * 16 + 16;
+        const size_t fixed = round_up(round_up((size_t)(a.T + 1) * a8_xrow(a.D), 16) +
+                                      (size_t)2 * (a.T + 1) * nbD * 4, 1024) +
+                             (size_t)kGuRedBufs * kDW * 2 * 32 * 4 * sizeof(float) +
+                             (2 * kMaxStages + 8) * sizeof(uint64_t) + tables_bytes(a.E) + units + 1024;
+        if (fixed >= kDecSmemMax) { set_error("decode path (8-bit activations): shared memory too small"); return MOE_ERR_SHAPE; }
+        const int S = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - fixed) / stage_bytes);
+        if (S < 2) { set_error("decode path (8-bit activations): shared memory too small"); return MOE_ERR_SHAPE; }
+        const size_t smem = fixed + (size_t)S * stage_bytes;
+        const int WB = std::min(nbD, kA8MaxSb) / 8;
+        mark(tr, MOE_KERNEL_FFN_DECODE);
+        cudaError_t e;
+        switch (WB) {
+        case 1: e = launch_gateup_a8<1>(A, maps, grid, smem, s, S); break;
+        case 2: e = launch_gateup_a8<2>(A, maps, grid, smem, s, S); break;
+        case 3: e = launch_gateup_a8<3>(A, maps, grid, smem, s, S); break;
+        default: e = launch_gateup_a8<4>(A, maps, grid, smem, s, S); break;
+        }
+        if (e != cudaSuccess) return cuda_status(e, "dec_gateup_a8_kernel");
+        // ---- down on the h codes
+        const int pr = tma_row_bytes((int)qt_row_bytes(a.qt, a.F));
+        const int ps = a.sF > 0 ? tma_row_bytes((int)qt_row_bytes(a.sqt, a.sF)) : 0;
+        const size_t wbytes = (size_t)kDnRows * std::max(pr, ps);
+        const size_t hsrow = (size_t)(A.hq_row / QK) * 8;
+        const size_t dstage = round_up(wbytes + round_up((size_t)hrows * hpitch, 128) + hrows * hsrow, 128);
+        const size_t dfixed = 2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
+        if (dfixed + dstage > kDecSmemMax) {
+            set_error("decode path (8-bit activations): a %zu-byte stage does not fit shared memory", dstage);
+            return MOE_ERR_SHAPE;
+        }
+        const int fit = (int)std::min<size_t>(kMaxStages, (kDecSmemMax - dfixed) / dstage);
+        const int G = fit >= 4 ? 4 : fit >= 2 ? 2 : 1;
+        const int Sg = std::min(2, fit / G);
+        const size_t dsmem = dfixed + (size_t)G * Sg * dstage;
+        const int dgrid = std::max(1, std::min(sms, (a.E + 1) * (a.D / kDnRows)));
+        e = launch_pdl(dec_down_a8_kernel<NT>, dgrid, kDThreads, dsmem, s, A, G, Sg, hrows, hpitch, maps);
+        if (e != cudaSuccess) return cuda_status(e, "dec_down_a8_kernel");
+    }
+    if (a.y) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(a.T, (a.D / 4 + 255) / 256);
+        cfg.blockDim = dim3(256);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, dec_combine_kernel, (const float *)a.rows_out,
+                                           a.inv, a.T, a.k, a.D, a.comb_shared, a.y, a.y_dtype);
+        if (e != cudaSuccess) return cuda_status(e, "dec_combine_kernel");
+    }
+    return MOE_OK;
+}
+
+moe_status launch_ffn_decode_a8(const void *x, int x_dtype, int T, int D, int F, int E, int k,
+                                const int32_t *perm, const int32_t *inv, const int32_t *offsets,
+                                const float *gates, const moe_pool &pool, const uint8_t *mask,
+                                bool routed, const moe_pool *shared, int sF, bool comb_shared,
+                                int8_t *hq, float2 *hs, void *y, int y_dtype, float *rows_out,
+                                int *err, cudaStream_t s, Tracer *tr) {
+    if (!a8_type_ok(pool.qtype) || (shared && !a8_type_ok(shared->qtype))) {
+        set_error("8-bit activations: Q4_0 and Q8_0 experts only (got %d%s%d)", (int)pool.qtype,
+                  shared ? ", shared " : "", shared ? (int)shared->qtype : 0);
+        return MOE_ERR_UNSUPPORTED_QTYPE;
+    }
+    if (T * k > kMaxTk) {
+        set_error("decode path: T*k=%d exceeds %d", T * k, kMaxTk);
+        return MOE_ERR_SHAPE;
+    }
+    if (!gates || !perm || !inv || !rows_out) {
+        set_error("8-bit activations: the fused layer's gates, permutation and rows are needed");
+        return MOE_ERR_INVALID_ARG;
+    }
+    A8Args A{};
+    DecArgs &a = A.d;
+    a.T = T; a.D = D; a.F = F; a.E = E; a.k = k; a.sF = shared ? sF : 0;
+    a.routed = routed ? 1 : 0;
+    a.n_slots = pool.n_slots;
+    a.comb_shared = comb_shared ? 1 : 0;
+    a.perm = perm; a.offsets = offsets; a.gates = gates; a.mask = mask;
+    a.gate = (const uint8_t *)pool.gate; a.up = (const uint8_t *)pool.up;
+    a.down = (const uint8_t *)pool.down; a.slot_map = pool.slot_of_expert;
+    a.qt = pool.qtype;
+    a.sqt = pool.qtype;
+    if (shared) {
+        a.sh_gate = (const uint8_t *)shared->gate; a.sh_up = (const uint8_t *)shared->up;
+        a.sh_down = (const uint8_t *)shared->down;
+        a.sqt = shared->qtype;
+    }
+    a.x = x; a.x_bf16 = (x_dtype == MOE_BF16);
+    a.x_vec = ((uintptr_t)x % 16) == 0;
+    a.y = y; a.y_dtype = y_dtype; a.rows_out = rows_out; a.err = err;
+    a.inv = inv;
+    A.hq = hq;
+    A.hs = hs;
+    A.hq_row = std::max(F, a.sF);
+    return T > 8 ? run_decode_a8<2>(A, pool.n_slots, s, tr) : run_decode_a8<1>(A, pool.n_slots, s, tr);
 }
 
 }  // namespace moe

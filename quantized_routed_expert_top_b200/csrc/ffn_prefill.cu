@@ -526,142 +526,259 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kPAW + kPBW) {
-        // ------------------------------------------------- B producers
-        // Raw windows (the 16-byte-aligned bytes holding four blocks = two
-        // K stages, or one Q4_K block = four, for all 256 weight rows of the
-        // tile) arrive by tensor copies kPR - 1 windows ahead.  Each warp
-        // dequantises its 32 rows of the window into the swizzled fp16 stage
-        // on its own; lane 0 of the first warp refills a raw buffer once all
-        // warps have read it.
-        const int bw = warp - kPAW, bt = tid - kPAW * 32;
-        const bool issuer = bw == 0 && lane == 0;
-        int gi = 0, ti = -1, wi = 0, nwI = 0;            // window issue cursor; windows of tile ti
-        PfTile tI{};
-        auto issue = [&]() -> bool {
-            if (wi == nwI) {                             // next tile of this CTA, if any
-                if (ti + 1 >= n_loc) return true;
-                ti++;
-                wi = 0;
-                tI = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
-                nwI = ALL ? nk / pf_stages_per_window(tI.v == a.E ? a.sqt : a.qt) : nk / 2;
-            }
-            if (gi >= kPR) {                             // the buffer's previous window is read
-                const int q = gi - kPR;
-                if (!mbar_wait(&rempty[q % kPR], (uint32_t)((q / kPR) & 1), a.err, kErrTimeoutEmpty)) return false;
-            }
-            const bool sh = tI.v == a.E;
-            const int qt = sh ? a.sqt : a.qt;
-            const int wb = pf_window_bytes(qt);
-            const int span = ALL ? pf_window_span(qt) : 4 * qt_bytes(qt);
-            const int x = (int)(((size_t)wi * span & ~(size_t)15) / 8);
-            const int slot = sh ? 0 : (a.slot_map ? __ldg(a.slot_map + tI.v) : tI.v);
-            const int r = gi % kPR;
-            uint8_t *dst = raw + (size_t)r * kPRaw;
-            mbar_arrive_expect_tx(&rfull[r], (uint32_t)(256 * wb));
-            if (MODE == kPGateUp) {
-                const int y = slot * a.F + tI.n * kPNg;
-                tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, y, &rfull[r]);
-                tma_load_2d(dst + 128 * wb, sh ? &maps.s1 : &maps.w1, x, y, &rfull[r]);
-            } else {
-                tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, slot * a.D + tI.n * kPNd, &rfull[r]);
-            }
-            gi++;
-            wi++;
-            return true;
-        };
-        bool ok = true;
-        if (issuer)
-            for (int q = 0; q < kPR - 1 && ok; q++) ok = issue();
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        int g = 0, gw = 0;                               // stage, window counters
-        for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
-            const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
-            const int qt = (t.v == a.E) ? a.sqt : a.qt;
-            const int wb = pf_window_bytes(qt);
-            const int spw = ALL ? pf_stages_per_window(qt) : 2;
-            for (int ks = 0; ks < nk && ok; ks++, g++) {
-                const int pos = ks & (spw - 1);                  // stage within the window
-                const int half = ks & 1;                         // which block pair of the window
-                if (pos == 0) {
-                    bool iok = true;
-                    if (issuer) iok = issue();                   // window gw + kPR - 1
-                    ok = __shfl_sync(0xffffffffu, iok ? 1 : 0, 0) != 0;
-                    if (!ok) break;
+        if constexpr (!ALL) {
+            // ------------------------------------ B producers, Q4_0 / Q8_0
+            // (the other types' code below ran these two types 5-8% slower)
+            // Raw windows (the 16-byte-aligned bytes holding four blocks = two
+            // K stages, for all 256 weight rows of the tile) arrive by tensor
+            // copies kPR - 1 windows ahead.  Each warp dequantises its 32 rows of the
+            // window into the swizzled fp16 stage on its own; lane 0 of the
+            // first warp refills a raw buffer once all warps have read it.
+            const int bw = warp - kPAW, bt = tid - kPAW * 32;
+            const bool issuer = bw == 0 && lane == 0;
+            const int nw = nk / 2;                           // windows per tile
+            const int n_win = n_loc * nw;
+            int gi = 0, ti = -1, wi = nw;                    // window issue cursor
+            PfTile tI{};
+            auto issue = [&]() -> bool {
+                if (gi >= n_win) return true;
+                if (gi >= kPR) {                             // the buffer's previous window is read
+                    const int q = gi - kPR;
+                    if (!mbar_wait(&rempty[q % kPR], (uint32_t)((q / kPR) & 1), a.err, kErrTimeoutEmpty)) return false;
                 }
-                const int r = gw % kPR;
-                if (pos == 0 &&
-                    !mbar_wait_warp(&rfull[r], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutFull)) { ok = false; break; }
-                uint4 c[8];
-                // the pair starts skew(window) + (2 * bs) * half bytes into the
-                // window; the skew is 8 for odd windows of 18-, 22- and 34-byte
-                // blocks, else 0
-                const int odd = (ks >> 1) & 1;
-                const uint8_t *rp = raw + (size_t)r * kPRaw + bt * wb;
-                if (ALL && qt == MOE_Q4_K) {
-                    switch (pos) {
-                    case 0: dq_stage_q4k<0>(rp, c); break;
-                    case 1: dq_stage_q4k<1>(rp, c); break;
-                    case 2: dq_stage_q4k<2>(rp, c); break;
-                    default: dq_stage_q4k<3>(rp, c); break;
-                    }
-                } else if (ALL && qt == MOE_Q4_1) {
-                    if (half == 0) dq_stage_std<MOE_Q4_1, 0>(rp, c); else dq_stage_std<MOE_Q4_1, 40>(rp, c);
-                } else if (ALL && qt == MOE_Q5_1) {
-                    if (half == 0) dq_stage_std<MOE_Q5_1, 0>(rp, c); else dq_stage_std<MOE_Q5_1, 48>(rp, c);
-                } else if (ALL && qt == MOE_Q5_0) {
-                    switch (2 * odd + half) {
-                    case 0: dq_stage_std<MOE_Q5_0, 0>(rp, c); break;
-                    case 1: dq_stage_std<MOE_Q5_0, 44>(rp, c); break;
-                    case 2: dq_stage_std<MOE_Q5_0, 8>(rp, c); break;
-                    default: dq_stage_std<MOE_Q5_0, 52>(rp, c); break;
-                    }
-                } else if (qt == MOE_Q8_0) {
-                    // words 16 * half .. +19 hold the pair at word 2*odd + half
-                    uint32_t w[20];
-#pragma unroll
-                    for (int q = 0; q < 5; q++) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(rp + 64 * half + 16 * q);
-                        w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-                    }
-                    switch (2 * odd + half) {
-                    case 0: dq_pair_q8<0>(w, c); break;
-                    case 1: dq_pair_q8<1>(w, c); break;
-                    case 2: dq_pair_q8<2>(w, c); break;
-                    default: dq_pair_q8<3>(w, c); break;
-                    }
+                if (wi == nw) {
+                    ti++;
+                    wi = 0;
+                    tI = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
+                }
+                const bool sh = tI.v == a.E;
+                const bool q8 = (sh ? a.sqt : a.qt) == MOE_Q8_0;
+                const int bs = q8 ? kQ8Bytes : kQ4Bytes;
+                const int wb = q8 ? 144 : 80;                        // window bytes
+                const int x = (int)(((size_t)wi * 4 * bs & ~(size_t)15) / 8);
+                const int slot = sh ? 0 : (a.slot_map ? __ldg(a.slot_map + tI.v) : tI.v);
+                const int r = gi % kPR;
+                uint8_t *dst = raw + (size_t)r * kPRaw;
+                mbar_arrive_expect_tx(&rfull[r], (uint32_t)(256 * wb));
+                if (MODE == kPGateUp) {
+                    const int y = slot * a.F + tI.n * kPNg;
+                    tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, y, &rfull[r]);
+                    tma_load_2d(dst + 128 * wb, sh ? &maps.s1 : &maps.w1, x, y, &rfull[r]);
                 } else {
-                    // words 8 * half .. +11 hold the pair at word 2*odd + half
-                    uint32_t w[12];
-#pragma unroll
-                    for (int q = 0; q < 3; q++) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(rp + 32 * half + 16 * q);
-                        w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-                    }
-                    switch (2 * odd + half) {
-                    case 0: dq_pair_q4<0>(w, c); break;
-                    case 1: dq_pair_q4<1>(w, c); break;
-                    case 2: dq_pair_q4<2>(w, c); break;
-                    default: dq_pair_q4<3>(w, c); break;
-                    }
+                    tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, slot * a.D + tI.n * kPNd, &rfull[r]);
                 }
-                if (pos == spw - 1) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&rempty[r]);      // this warp is done with the window
-                    gw++;
+                gi++;
+                wi++;
+                return true;
+            };
+            bool ok = true;
+            if (issuer)
+                for (int q = 0; q < kPR - 1 && ok; q++) ok = issue();
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            int g = 0, gw = 0;                               // stage, window counters
+            for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
+                const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
+                const bool q8 = ((t.v == a.E) ? a.sqt : a.qt) == MOE_Q8_0;
+                const int wb = q8 ? 144 : 80;
+                for (int ks = 0; ks < nk && ok; ks++, g++) {
+                    const int half = ks & 1;                         // which block pair of the window
+                    if (half == 0) {
+                        bool iok = true;
+                        if (issuer) iok = issue();                   // window gw + kPR - 1
+                        ok = __shfl_sync(0xffffffffu, iok ? 1 : 0, 0) != 0;
+                        if (!ok) break;
+                    }
+                    const int r = gw % kPR;
+                    if (half == 0 &&
+                        !mbar_wait_warp(&rfull[r], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutFull)) { ok = false; break; }
+                    uint4 c[8];
+                    // the pair starts 8 * (group % 2) + (2 * bs) * half bytes into the window
+                    const int odd = (ks >> 1) & 1;
+                    const uint8_t *rp = raw + (size_t)r * kPRaw + bt * wb;
+                    if (q8) {
+                        // words 16 * half .. +19 hold the pair at word 2*odd + half
+                        uint32_t w[20];
+    #pragma unroll
+                        for (int q = 0; q < 5; q++) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(rp + 64 * half + 16 * q);
+                            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                        }
+                        switch (2 * odd + half) {
+                        case 0: dq_pair_q8<0>(w, c); break;
+                        case 1: dq_pair_q8<1>(w, c); break;
+                        case 2: dq_pair_q8<2>(w, c); break;
+                        default: dq_pair_q8<3>(w, c); break;
+                        }
+                    } else {
+                        // words 8 * half .. +11 hold the pair at word 2*odd + half
+                        uint32_t w[12];
+    #pragma unroll
+                        for (int q = 0; q < 3; q++) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(rp + 32 * half + 16 * q);
+                            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                        }
+                        switch (2 * odd + half) {
+                        case 0: dq_pair_q4<0>(w, c); break;
+                        case 1: dq_pair_q4<1>(w, c); break;
+                        case 2: dq_pair_q4<2>(w, c); break;
+                        default: dq_pair_q4<3>(w, c); break;
+                        }
+                    }
+                    if (half == 1) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&rempty[r]);      // this warp is done with the window
+                        gw++;
+                    }
+                    const int s = g % kPSB;
+                    if (!mbar_wait_warp(&emptyB[s], ((g / kPSB) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                    uint8_t *dst = ringB + (size_t)s * kPStageB;
+    #pragma unroll
+                    for (int jj = 0; jj < 8; jj++) *reinterpret_cast<uint4 *>(dst + sw128_off(bt, jj)) = c[jj];
+                    fence_proxy_async_smem();
+                    mbar_arrive(&fullB[s]);
                 }
-                const int s = g % kPSB;
-                if (!mbar_wait_warp(&emptyB[s], ((g / kPSB) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
-                uint8_t *dst = ringB + (size_t)s * kPStageB;
-#pragma unroll
-                for (int jj = 0; jj < 8; jj++) *reinterpret_cast<uint4 *>(dst + sw128_off(bt, jj)) = c[jj];
-                fence_proxy_async_smem();
-                mbar_arrive(&fullB[s]);
             }
+            // windows still in flight must land before the CTA exits
+            if (issuer)
+                for (; gw < gi; gw++)
+                    mbar_wait(&rfull[gw % kPR], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutDrain);
+        } else {
+            // ------------------------------------------------- B producers
+            // Raw windows (the 16-byte-aligned bytes holding four blocks = two
+            // K stages, or one Q4_K block = four, for all 256 weight rows of the
+            // tile) arrive by tensor copies kPR - 1 windows ahead.  Each warp
+            // dequantises its 32 rows of the window into the swizzled fp16 stage
+            // on its own; lane 0 of the first warp refills a raw buffer once all
+            // warps have read it.
+            const int bw = warp - kPAW, bt = tid - kPAW * 32;
+            const bool issuer = bw == 0 && lane == 0;
+            int gi = 0, ti = -1, wi = 0, nwI = 0;            // window issue cursor; windows of tile ti
+            PfTile tI{};
+            auto issue = [&]() -> bool {
+                if (wi == nwI) {                             // next tile of this CTA, if any
+                    if (ti + 1 >= n_loc) return true;
+                    ti++;
+                    wi = 0;
+                    tI = pf_tile(tcum, segs, nv, nt, blockIdx.x + ti * gridDim.x);
+                    nwI = nk / pf_stages_per_window(tI.v == a.E ? a.sqt : a.qt);
+                }
+                if (gi >= kPR) {                             // the buffer's previous window is read
+                    const int q = gi - kPR;
+                    if (!mbar_wait(&rempty[q % kPR], (uint32_t)((q / kPR) & 1), a.err, kErrTimeoutEmpty)) return false;
+                }
+                const bool sh = tI.v == a.E;
+                const int qt = sh ? a.sqt : a.qt;
+                const int wb = pf_window_bytes(qt);
+                const int x = (int)(((size_t)wi * pf_window_span(qt) & ~(size_t)15) / 8);
+                const int slot = sh ? 0 : (a.slot_map ? __ldg(a.slot_map + tI.v) : tI.v);
+                const int r = gi % kPR;
+                uint8_t *dst = raw + (size_t)r * kPRaw;
+                mbar_arrive_expect_tx(&rfull[r], (uint32_t)(256 * wb));
+                if (MODE == kPGateUp) {
+                    const int y = slot * a.F + tI.n * kPNg;
+                    tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, y, &rfull[r]);
+                    tma_load_2d(dst + 128 * wb, sh ? &maps.s1 : &maps.w1, x, y, &rfull[r]);
+                } else {
+                    tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, x, slot * a.D + tI.n * kPNd, &rfull[r]);
+                }
+                gi++;
+                wi++;
+                return true;
+            };
+            bool ok = true;
+            if (issuer)
+                for (int q = 0; q < kPR - 1 && ok; q++) ok = issue();
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            int g = 0, gw = 0;                               // stage, window counters
+            for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
+                const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
+                const int qt = (t.v == a.E) ? a.sqt : a.qt;
+                const int wb = pf_window_bytes(qt);
+                const int spw = pf_stages_per_window(qt);
+                for (int ks = 0; ks < nk && ok; ks++, g++) {
+                    const int pos = ks & (spw - 1);                  // stage within the window
+                    const int half = ks & 1;                         // which block pair of the window
+                    if (pos == 0) {
+                        bool iok = true;
+                        if (issuer) iok = issue();                   // window gw + kPR - 1
+                        ok = __shfl_sync(0xffffffffu, iok ? 1 : 0, 0) != 0;
+                        if (!ok) break;
+                    }
+                    const int r = gw % kPR;
+                    if (pos == 0 &&
+                        !mbar_wait_warp(&rfull[r], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutFull)) { ok = false; break; }
+                    uint4 c[8];
+                    // the pair starts skew(window) + (2 * bs) * half bytes into the
+                    // window; the skew is 8 for odd windows of 18-, 22- and 34-byte
+                    // blocks, else 0
+                    const int odd = (ks >> 1) & 1;
+                    const uint8_t *rp = raw + (size_t)r * kPRaw + bt * wb;
+                    if (qt == MOE_Q4_K) {
+                        switch (pos) {
+                        case 0: dq_stage_q4k<0>(rp, c); break;
+                        case 1: dq_stage_q4k<1>(rp, c); break;
+                        case 2: dq_stage_q4k<2>(rp, c); break;
+                        default: dq_stage_q4k<3>(rp, c); break;
+                        }
+                    } else if (qt == MOE_Q4_1) {
+                        if (half == 0) dq_stage_std<MOE_Q4_1, 0>(rp, c); else dq_stage_std<MOE_Q4_1, 40>(rp, c);
+                    } else if (qt == MOE_Q5_1) {
+                        if (half == 0) dq_stage_std<MOE_Q5_1, 0>(rp, c); else dq_stage_std<MOE_Q5_1, 48>(rp, c);
+                    } else if (qt == MOE_Q5_0) {
+                        switch (2 * odd + half) {
+                        case 0: dq_stage_std<MOE_Q5_0, 0>(rp, c); break;
+                        case 1: dq_stage_std<MOE_Q5_0, 44>(rp, c); break;
+                        case 2: dq_stage_std<MOE_Q5_0, 8>(rp, c); break;
+                        default: dq_stage_std<MOE_Q5_0, 52>(rp, c); break;
+                        }
+                    } else if (qt == MOE_Q8_0) {
+                        // words 16 * half .. +19 hold the pair at word 2*odd + half
+                        uint32_t w[20];
+    #pragma unroll
+                        for (int q = 0; q < 5; q++) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(rp + 64 * half + 16 * q);
+                            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                        }
+                        switch (2 * odd + half) {
+                        case 0: dq_pair_q8<0>(w, c); break;
+                        case 1: dq_pair_q8<1>(w, c); break;
+                        case 2: dq_pair_q8<2>(w, c); break;
+                        default: dq_pair_q8<3>(w, c); break;
+                        }
+                    } else {
+                        // words 8 * half .. +11 hold the pair at word 2*odd + half
+                        uint32_t w[12];
+    #pragma unroll
+                        for (int q = 0; q < 3; q++) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(rp + 32 * half + 16 * q);
+                            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                        }
+                        switch (2 * odd + half) {
+                        case 0: dq_pair_q4<0>(w, c); break;
+                        case 1: dq_pair_q4<1>(w, c); break;
+                        case 2: dq_pair_q4<2>(w, c); break;
+                        default: dq_pair_q4<3>(w, c); break;
+                        }
+                    }
+                    if (pos == spw - 1) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&rempty[r]);      // this warp is done with the window
+                        gw++;
+                    }
+                    const int s = g % kPSB;
+                    if (!mbar_wait_warp(&emptyB[s], ((g / kPSB) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                    uint8_t *dst = ringB + (size_t)s * kPStageB;
+    #pragma unroll
+                    for (int jj = 0; jj < 8; jj++) *reinterpret_cast<uint4 *>(dst + sw128_off(bt, jj)) = c[jj];
+                    fence_proxy_async_smem();
+                    mbar_arrive(&fullB[s]);
+                }
+            }
+            // windows still in flight must land before the CTA exits
+            if (issuer)
+                for (; gw < gi; gw++)
+                    mbar_wait(&rfull[gw % kPR], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutDrain);
         }
-        // windows still in flight must land before the CTA exits
-        if (issuer)
-            for (; gw < gi; gw++)
-                mbar_wait(&rfull[gw % kPR], (uint32_t)((gw / kPR) & 1), a.err, kErrTimeoutDrain);
     } else if (warp == kPMmaWarp) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0) {

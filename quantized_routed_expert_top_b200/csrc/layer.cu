@@ -21,6 +21,8 @@ struct LayerWs {
     float *sh_rows;      // [T, D]
     __half *Hs;          // decode path: g*h in fp16 fragment order
     __half *x16, *H16;   // prefill path: fp16 activations and hidden rows
+    int8_t *hq;          // 8-bit activations: h codes and their (scale, code sum)
+    float2 *hs;
 };
 
 static LayerWs carve(const moe_layer_args &a, Carver &c) {
@@ -36,6 +38,13 @@ static LayerWs carve(const moe_layer_args &a, Carver &c) {
     w.perm = c.take<int32_t>(Tk);
     w.inv = c.take<int32_t>(Tk);
     const int qt = a.pool ? a.pool->qtype : 0, sqt = a.shared ? a.shared->qtype : 0;
+    if (a.act_bits == 8) {
+        const int sF = a.shared ? a.shared_F : 0;
+        w.hq = c.take<int8_t>(decode_a8_hq_bytes(a.T, a.k, a.F, sF));
+        w.hs = c.take<float2>(decode_a8_hs_bytes(a.T, a.k, a.F, sF) / sizeof(float2));
+        w.rows = c.take<float>(decode_rows_floats(a.T, a.k, a.D));
+        return w;
+    }
     if (decode_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0, qt, sqt)) {
         w.Hs = c.take<__half>(decode_hs_halves(a.T, a.k, a.F, a.shared ? a.shared_F : 0));
         w.rows = c.take<float>(decode_rows_floats(a.T, a.k, a.D));
@@ -116,6 +125,14 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
             return st;
     }
     const int sF = a.shared ? a.shared_F : 0;
+    if (w.hq) {
+        if (!do_ffn && !do_shared && !do_comb) return end_trace(tr, MOE_OK);
+        st = launch_ffn_decode_a8(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, perm, inv, offsets,
+                                  gates, *a.pool, a.expert_mask, do_ffn,
+                                  do_shared ? a.shared : nullptr, sF, a.shared != nullptr, w.hq,
+                                  w.hs, do_comb ? a.y : nullptr, a.y_dtype, w.rows, w.status, s, tr);
+        return end_trace(tr, st);
+    }
     if (w.Hs) {
         if (!do_ffn && !do_shared && !do_comb) return end_trace(tr, MOE_OK);
         st = launch_ffn_decode(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, perm, inv, offsets, gates,

@@ -322,6 +322,18 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
                              bool routed, const moe_pool *shared, int sF, bool comb_shared,
                              __half *Hs, void *y, int y_dtype, float *rows_out, int *err,
                              cudaStream_t s, Tracer *tr);
+// The same with 8-bit activation blocks into every expert matmul (the W4A8 /
+// W8A8 mode): decode shapes, Q4_0 / Q8_0 experts; hq, hs: the h codes and
+// their (scale, code sum) pairs (decode_a8_hq_bytes, decode_a8_hs_bytes).
+bool decode_a8_ok(int T, int D, int F, int sF, int qt, int sqt);
+size_t decode_a8_hq_bytes(int T, int k, int F, int sF);
+size_t decode_a8_hs_bytes(int T, int k, int F, int sF);
+moe_status launch_ffn_decode_a8(const void *x, int x_dtype, int T, int D, int F, int E, int k,
+                                const int32_t *perm, const int32_t *inv, const int32_t *offsets,
+                                const float *gates, const moe_pool &pool, const uint8_t *mask,
+                                bool routed, const moe_pool *shared, int sF, bool comb_shared,
+                                int8_t *hq, float2 *hs, void *y, int y_dtype, float *rows_out,
+                                int *err, cudaStream_t s, Tracer *tr);
 // combine.cu
 moe_status launch_combine(const float *rows, const int32_t *inv, const float *gates,
                           int T, int k, int D, const float *shared_rows, void *y,

@@ -150,6 +150,28 @@ __device__ __forceinline__ void mma_16816(float *d, const uint32_t *a, uint32_t 
           "f"(c[2]), "f"(c[3]));
 }
 
+// int8 tensor-core products, int32 accumulate: A 16x32 (row), B 32x8 (col).
+// Fragments: a[0] row g, k 4c..4c+3; a[1] row g+8, same k; a[2], a[3] the
+// same rows at k 16+4c..; b0 k 4c..4c+3 of column g, b1 k 16+4c..; c/d as
+// the f16 shape (rows g, g+8; columns 2c, 2c+1).
+__device__ __forceinline__ void imma_s8s8(int *d, const uint32_t *a, uint32_t b0, uint32_t b1,
+                                          const int *c) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%11,%12,%13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]),
+          "r"(c[2]), "r"(c[3]));
+}
+// the same with unsigned 8-bit A (Q4_0 nibble codes)
+__device__ __forceinline__ void imma_u8s8(int *d, const uint32_t *a, uint32_t b0, uint32_t b1,
+                                          const int *c) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%11,%12,%13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]),
+          "r"(c[2]), "r"(c[3]));
+}
+
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
     uint32_t r;
     // (a & mask) | magic  -> lut 0xEA for (a & b) | c

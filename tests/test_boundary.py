@@ -238,3 +238,34 @@ def test_streamer_arguments(moe):
     assert not h.value
     assert L.moe_streamer_prefetch(None, 0) == 1
     assert L.moe_streamer_stats(None, None, None) == 1
+
+
+def test_layer_forward_act_bits_errors(moe):
+    # 8-bit activations: a bad act_bits, a type other than Q4_0/Q8_0, and a
+    # shape outside the decode kernels are refused before any kernel runs
+    L = moe.lib()
+
+    def args(qtype, T=4, act_bits=8):
+        pool = moe.Pool(qtype, 8, 0x1000, 0x1000, 0x1000, None)
+        a = moe.LayerArgs()
+        a.T, a.D, a.E, a.k, a.F, a.renorm = T, 256, 8, 2, 512, 1
+        a.x_dtype, a.y_dtype = moe.BF16, moe.BF16
+        a.x, a.y, a.w_router = 0x1000, 0x1000, 0x1000
+        a.pool = C.pointer(pool)
+        a.act_bits = act_bits
+        return a, pool
+
+    a, _p = args(moe.Q4_0, act_bits=5)
+    assert L.moe_layer_forward(C.byref(a), FAKE, 1 << 40, None) == 1
+    assert "act_bits" in _err(L)
+    for q in (moe.Q5_0, moe.Q4_1, moe.Q4_K):
+        a, _p = args(q)
+        assert L.moe_layer_forward(C.byref(a), FAKE, 1 << 40, None) == 2
+        assert "8-bit activations" in _err(L)
+    a, _p = args(moe.Q8_0, T=32)
+    assert L.moe_layer_forward(C.byref(a), FAKE, 1 << 40, None) == 3
+    assert "decode shapes" in _err(L)
+    # a valid 8-bit call sizes its own workspace (h codes instead of fp16 rows)
+    a8, _p = args(moe.Q8_0)
+    a16, _p2 = args(moe.Q8_0, act_bits=0)
+    assert L.moe_layer_workspace_size(C.byref(a8)) != L.moe_layer_workspace_size(C.byref(a16))
