@@ -505,7 +505,11 @@ def roofline(wl, algo, durs, peaks, steps):
          "algorithmic_per_launch": round(work / wl.calls_per_step, 1),
          "avg_launch_ms": round(avg_ms, 5),
          "per_T": {str(T): {"work": algo[T]["seg_flops" if bound == "tensor" else "seg_bytes"].get(dom),
-                            "distinct_experts": algo[T]["distinct"]} for T in wl.Ts},
+                            "distinct_experts": algo[T]["distinct"],
+                            # launches run in T order within a step
+                            "avg_ms": round(sum(durs[dom][i::len(wl.Ts)]) /
+                                            max(1, len(durs[dom][i::len(wl.Ts)])), 5)}
+                   for i, T in enumerate(wl.Ts)},
          "peak_source": f"{peaks['source']} {psrc}",
          "traffic": ncu_traffic(dom, wl.name)}
     if flops_step and bound == "hbm":

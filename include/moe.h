@@ -156,6 +156,17 @@ int moe_block_bytes(int32_t qtype);
  * an unknown type. */
 int moe_block_weights(int32_t qtype);
 
+/* moe_selftest_wait_timeout: exercises the kernels' bounded-wait path.  One
+ * warp waits, with the same wait routine the FFN kernels use, on a shared-
+ * memory barrier that nothing arrives at, for budget_cycles SM clock cycles
+ * (1 .. 4e9); the wait runs out, records MOE_DEV_TIMEOUT_FULL in the status
+ * word of `workspace` (device, >= 64 bytes, as moe_workspace_status reads it)
+ * and the kernel returns: no fault, no hang, the context stays usable.
+ * Enqueues one kernel on `stream`; MOE_ERR_INVALID_ARG for a budget out of
+ * range, MOE_ERR_WORKSPACE for a missing or short workspace. */
+moe_status moe_selftest_wait_timeout(void *workspace, size_t ws_bytes, int64_t budget_cycles,
+                                     moe_stream stream);
+
 /* moe_workspace_status: the device status word of a workspace (its first
  * int32, written by the kernels of the calls that used it; see the
  * conventions above).  Waits for the work enqueued on `stream` so far, then

@@ -104,6 +104,8 @@ def lib():
         L.moe_version.restype = C.c_char_p
         L.moe_block_bytes.argtypes = [C.c_int32]
         L.moe_workspace_status.argtypes = [_v, C.POINTER(C.c_int32), _i, _v]
+        L.moe_selftest_wait_timeout.argtypes = [_v, _sz, C.c_int64, _v]
+        L.moe_block_weights.argtypes = [C.c_int32]
         L.moe_route_workspace_size.restype = _sz
         L.moe_route_workspace_size.argtypes = [_i, _i, _i, _i]
         L.moe_route.argtypes = [_v, C.c_int32, _v, _v, _i, _i, _i, _i, _i, _v, _v, _v, _v, _sz, _v]
@@ -179,6 +181,14 @@ def workspace_status(ws, clear: bool = True, stream=None):
     code = C.c_int32(0)
     st = lib().moe_workspace_status(_p(ws), C.byref(code), int(clear), _stream(stream))
     return st, code.value
+
+
+def selftest_wait_timeout(ws, budget_cycles: int, stream=None):
+    """moe_selftest_wait_timeout: one warp waits, with the kernels' bounded
+    wait, on a barrier nothing arrives at; the status word of ``ws`` then
+    reads DEV_TIMEOUT_FULL (see workspace_status)."""
+    _check(lib().moe_selftest_wait_timeout(_p(ws), ws.numel() * ws.element_size(),
+                                           int(budget_cycles), _stream(stream)))
 
 
 # ----------------------------------------------------------------- pools

@@ -93,6 +93,20 @@ static moe_status check_block_shape(const char *fn, const moe_pool *p, int D, in
     return MOE_OK;
 }
 
+// The bounded-wait self test: one warp waits, with the kernels' wait
+// routine and a short budget, on an mbarrier that nothing arrives at; the
+// wait runs out, records MOE_DEV_TIMEOUT_FULL in the status word and the
+// kernel returns (no fault, no hang: the context stays usable).
+__global__ void selftest_wait_kernel(int *status, long long budget) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    (void)__all_sync(0xffffffffu, mbar_wait_budget(&bar, 0, status, kErrTimeoutFull, budget));
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -108,6 +122,18 @@ int moe_block_bytes(int32_t qtype) {
 }
 
 int moe_block_weights(int32_t qtype) { return qt_weights(qtype); }
+
+moe_status moe_selftest_wait_timeout(void *workspace, size_t ws_bytes, int64_t budget_cycles,
+                                     moe_stream stream) {
+    g_err.clear();
+    if (!workspace || ws_bytes < 64) { set_error("moe_selftest_wait_timeout: workspace of at least 64 bytes needed"); return MOE_ERR_WORKSPACE; }
+    if (budget_cycles <= 0 || budget_cycles > 4000000000LL) {
+        set_error("moe_selftest_wait_timeout: budget_cycles must be in (0, 4e9]");
+        return MOE_ERR_INVALID_ARG;
+    }
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((int *)workspace, (long long)budget_cycles);
+    return cuda_status(cudaGetLastError(), "selftest_wait_kernel");
+}
 
 // ------------------------------------------------------ device status word
 moe_status moe_workspace_status(void *workspace, int32_t *code, int clear, moe_stream stream) {

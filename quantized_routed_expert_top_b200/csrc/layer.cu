@@ -15,6 +15,7 @@ struct LayerWs {
     int32_t *ids;
     float *gates;
     int32_t *counts, *offsets, *perm, *inv;
+    int32_t *perm_scratch;   // per-CTA expert counts of the many-CTA permutation
     float *H;            // [T*k, F] fp32
     float *rows;         // [T*k, D] fp32
     float *shH;          // [T, shared_F]
@@ -37,6 +38,7 @@ static LayerWs carve(const moe_layer_args &a, Carver &c) {
     w.offsets = c.take<int32_t>(a.E + 1);
     w.perm = c.take<int32_t>(Tk);
     w.inv = c.take<int32_t>(Tk);
+    w.perm_scratch = c.take<int32_t>(permute_scratch_ints(a.E));
     const int qt = a.pool ? a.pool->qtype : 0, sqt = a.shared ? a.shared->qtype : 0;
     if (a.act_bits == 8) {
         const int sF = a.shared ? a.shared_F : 0;
@@ -121,7 +123,8 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
                                       inv, w.status, w.route_ws, w.route_bytes, s, tr, &permuted);
         if (st != MOE_OK) return st;
         if (!permuted &&
-            (st = launch_permute(ids, a.T, a.k, a.E, counts, offsets, perm, inv, s, tr)) != MOE_OK)
+            (st = launch_permute(ids, a.T, a.k, a.E, counts, offsets, perm, inv, s, tr,
+                                 w.perm_scratch)) != MOE_OK)
             return st;
     }
     const int sF = a.shared ? a.shared_F : 0;

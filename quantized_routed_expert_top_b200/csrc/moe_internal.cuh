@@ -283,9 +283,12 @@ moe_status launch_route_permute(const void *x, int x_dtype, const float *w_route
                                 void *ws, size_t ws_bytes, cudaStream_t s, Tracer *tr,
                                 bool *permuted);
 // permute.cu
+// scratch: NULL (one CTA) or permute_scratch_ints(E) ints of device memory,
+// which lets large T*k run over many CTAs (the same result)
 moe_status launch_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
                           int32_t *offsets, int32_t *perm, int32_t *inv,
-                          cudaStream_t s, Tracer *tr = nullptr);
+                          cudaStream_t s, Tracer *tr = nullptr, int32_t *scratch = nullptr);
+size_t permute_scratch_ints(int E);
 // ffn_generic.cu -- portable SIMT path for every shape
 moe_status launch_ffn_generic(const void *x, int x_dtype, int T, int D, int F, int E,
                               int k, const int32_t *perm, const int32_t *offsets,

@@ -262,21 +262,34 @@ route_logits_tiled_kernel(const XT *__restrict__ x, const float *__restrict__ W,
 // Large-T router logits, register-tiled SIMT GEMM: a CTA computes 64 tokens
 // x 128 experts, a thread 4 tokens x 8 experts (two runs of 4, so its
 // 16-byte shared loads of W_r are conflict-free), with the next 32-row
-// K-tile loaded into registers while the current one is used.  Every
-// logit is one thread's fmaf chain over k in ascending order plus the bias,
-// the same arithmetic as route_logits_tiled_kernel.  E % 4 == 0.
+// K-tile loaded into registers while the current one is used.  With
+// nsplit > 1 the K range is cut into nsplit equal segments (blockIdx.z): a
+// segment's partial is one thread's fmaf chain over its k in ascending
+// order, written without the bias to part[z]; route_reduce_select_kernel
+// adds the partials in segment order, then the bias.  (More CTAs per SM:
+// at T = 8192 one segment gives 128 CTAs of 8 warps for 148 SMs.)
+// E % 4 == 0.
 constexpr int kSM = 64, kSN = 128, kSK = 32;
+constexpr int kLgSplit = 4;          // K segments when T is large
+__host__ __device__ inline int logits_nsplit(int T, int D) {
+    return (T >= 512 && D % (kLgSplit * kSK) == 0) ? kLgSplit : 1;
+}
 
 template <typename XT>
 __global__ void __launch_bounds__(256)
 route_logits_sgemm_kernel(const XT *__restrict__ x, const float *__restrict__ W,
                           const float *__restrict__ bias, int T, int D, int E,
-                          float *__restrict__ logits) {
+                          float *__restrict__ logits, int kseg) {
     extern __shared__ __align__(16) float smem_lg[];
     float *As = smem_lg;                                   // [2][kSK][kSM + 1]
     float *Bs = As + 2 * kSK * (kSM + 1);                  // [2][kSK][kSN + 4]
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const int t0 = blockIdx.x * kSM, e0 = blockIdx.y * kSN;
+    const int kbeg = blockIdx.z * kseg, kend = kbeg + kseg;
+    if (gridDim.z > 1) {                  // partial of segment z, no bias
+        logits += (size_t)blockIdx.z * T * E;
+        bias = nullptr;
+    }
     // global -> register staging: A = 8 consecutive k of one token, B = 4
     // float4 of W_r rows
     const int am = tid >> 2, ak = (tid & 3) * 8;
@@ -307,12 +320,12 @@ route_logits_sgemm_kernel(const XT *__restrict__ x, const float *__restrict__ W,
     for (int i = 0; i < 4; i++)
 #pragma unroll
         for (int j = 0; j < 8; j++) acc[i][j] = 0.f;
-    load(0);
+    load(kbeg);
     store(0);
     __syncthreads();
     int buf = 0;
-    for (int k0 = 0; k0 < D; k0 += kSK) {
-        if (k0 + kSK < D) load(k0 + kSK);
+    for (int k0 = kbeg; k0 < kend; k0 += kSK) {
+        if (k0 + kSK < kend) load(k0 + kSK);
         const float *a = As + buf * kSK * (kSM + 1);
         const float *b = Bs + buf * kSK * (kSN + 4);
 #pragma unroll
@@ -328,7 +341,7 @@ route_logits_sgemm_kernel(const XT *__restrict__ x, const float *__restrict__ W,
 #pragma unroll
                 for (int j = 0; j < 8; j++) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
-        if (k0 + kSK < D) {
+        if (k0 + kSK < kend) {
             store(buf ^ 1);
             __syncthreads();
             buf ^= 1;
@@ -363,6 +376,25 @@ route_select_kernel(const float *__restrict__ logits, const float *__restrict__ 
         L = C;
     }
     warp_select(L, E, k, renorm, ids + (size_t)warp * k, gates + (size_t)warp * k);
+}
+
+// Sum of the nsplit logit partials in segment order, plus the bias, into L
+// (one warp per token), then the selection on that row.
+__global__ void __launch_bounds__(256)
+route_reduce_select_kernel(const float *__restrict__ part, int nsplit, const float *__restrict__ bias,
+                           int T, int E, int k, int renorm, int32_t *__restrict__ ids,
+                           float *__restrict__ gates, float *__restrict__ L) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (warp >= T) return;
+    const int lane = threadIdx.x & 31;
+    float *row = L + (size_t)warp * E;
+    for (int e = lane; e < E; e += 32) {
+        float v = __ldg(part + (size_t)warp * E + e);
+        for (int z = 1; z < nsplit; z++) v += __ldg(part + ((size_t)z * T + warp) * E + e);
+        row[e] = v + (bias ? __ldg(bias + e) : 0.0f);
+    }
+    __syncwarp();
+    warp_select(row, E, k, renorm, ids + (size_t)warp * k, gates + (size_t)warp * k);
 }
 
 // ------------------------------------ small T: one cluster, DSMEM reduction
@@ -589,8 +621,12 @@ size_t route_ws_bytes(int T, int D, int E, int k) {
     (void)k;
     Carver c(nullptr, 0);
     c.take<unsigned>(64);
-    if (T <= kSplitMaxT) c.take<char>(splitk_partial_bytes(T, D, E));
-    else c.take<float>((size_t)T * E);   // logits scratch when none requested
+    if (T <= kSplitMaxT) {
+        c.take<char>(splitk_partial_bytes(T, D, E));
+    } else {
+        c.take<float>((size_t)T * E);    // logits scratch when none requested
+        if (logits_nsplit(T, D) > 1) c.take<float>((size_t)logits_nsplit(T, D) * T * E);   // partials
+    }
     return c.off;
 }
 
@@ -713,24 +749,39 @@ moe_status launch_route(const void *x, int x_dtype, const float *w_router,
         if (!c.fits()) { set_error("moe_route: workspace too small"); return MOE_ERR_WORKSPACE; }
     }
     mark(tr, MOE_KERNEL_ROUTE_LOGITS);
+    const int nsplit = E % 4 == 0 ? logits_nsplit(T, D) : 1;
+    float *part = nullptr;
+    if (nsplit > 1) {
+        part = c.take<float>((size_t)nsplit * T * E);
+        if (!c.fits()) { set_error("moe_route: workspace too small"); return MOE_ERR_WORKSPACE; }
+    }
     if (E % 4 == 0) {
-        const dim3 grid((T + kSM - 1) / kSM, (E + kSN - 1) / kSN);
+        const dim3 grid((T + kSM - 1) / kSM, (E + kSN - 1) / kSN, nsplit);
         const size_t sm = (size_t)(2 * kSK * (kSM + 1) + 2 * kSK * (kSN + 4)) * sizeof(float);
+        float *dst = nsplit > 1 ? part : L;
         cudaError_t e;
         if (x_dtype == MOE_BF16) {
             e = cudaFuncSetAttribute(route_logits_sgemm_kernel<__nv_bfloat16>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
             if (e == cudaSuccess)
                 route_logits_sgemm_kernel<__nv_bfloat16><<<grid, 256, sm, s>>>(
-                    (const __nv_bfloat16 *)x, w_router, bias, T, D, E, L);
+                    (const __nv_bfloat16 *)x, w_router, bias, T, D, E, dst, D / nsplit);
         } else {
             e = cudaFuncSetAttribute(route_logits_sgemm_kernel<float>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
             if (e == cudaSuccess)
                 route_logits_sgemm_kernel<float><<<grid, 256, sm, s>>>((const float *)x, w_router,
-                                                                       bias, T, D, E, L);
+                                                                       bias, T, D, E, dst, D / nsplit);
         }
         if (e != cudaSuccess) return cuda_status(e, "route_logits_sgemm_kernel attribute");
+        if (nsplit > 1) {
+            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "route_logits_sgemm_kernel");
+            const int blocks = (T * 32 + 255) / 256;
+            mark(tr, MOE_KERNEL_ROUTE_SELECT);
+            route_reduce_select_kernel<<<blocks, 256, 0, s>>>(part, nsplit, bias, T, E, k, renorm, ids,
+                                                             gates, L);
+            return cuda_status(cudaGetLastError(), "route_reduce_select_kernel");
+        }
     } else {
         dim3 grid((T + kTM - 1) / kTM, (E + kTN - 1) / kTN);
         if (x_dtype == MOE_BF16)

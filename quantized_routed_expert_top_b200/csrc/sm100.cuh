@@ -72,16 +72,21 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 
 // Bounded wait on a phase parity; on timeout records `code` in *err (first
 // error wins) and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err, int code) {
+// budget: clock cycles before giving up (the kernels pass kWaitBudgetCycles)
+__device__ __forceinline__ bool mbar_wait_budget(uint64_t *bar, uint32_t parity, int *err, int code,
+                                                 long long budget) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait_sleep(bar, parity, 100000u)) {
-        if (clock64() - t0 > kWaitBudgetCycles) {
+        if (clock64() - t0 > budget) {
             if (err) atomicCAS(err, 0, code);
             return false;
         }
     }
     return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err, int code) {
+    return mbar_wait_budget(bar, parity, err, code, kWaitBudgetCycles);
 }
 
 // mbar_wait by every lane of a warp with one outcome for the whole warp (a

@@ -269,3 +269,13 @@ def test_layer_forward_act_bits_errors(moe):
     a8, _p = args(moe.Q8_0)
     a16, _p2 = args(moe.Q8_0, act_bits=0)
     assert L.moe_layer_workspace_size(C.byref(a8)) != L.moe_layer_workspace_size(C.byref(a16))
+
+
+def test_selftest_wait_timeout_argument_errors(moe):
+    L = moe.lib()
+    # 7 = MOE_ERR_WORKSPACE, 1 = MOE_ERR_INVALID_ARG; nothing is launched
+    assert L.moe_selftest_wait_timeout(None, 64, 1000, None) == 7
+    assert L.moe_selftest_wait_timeout(FAKE, 16, 1000, None) == 7
+    assert L.moe_selftest_wait_timeout(FAKE, 64, 0, None) == 1
+    assert L.moe_selftest_wait_timeout(FAKE, 64, 5_000_000_000, None) == 1
+    assert "budget" in _err(L)
