@@ -248,7 +248,9 @@ moe_status moe_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
  * the segment of offsets that holds pos):
  *   out_rows[pos, :] = W_down,e ( silu(W_gate,e x_t) * (W_up,e x_t) )
  * (no gate weight; moe_combine applies it).
- * Kernels, by shape (the same as moe_layer_forward's):
+ * Kernels, by shape (the same as moe_layer_forward's, except that the layer
+ * runs Q6_K at T > 16 on the tensor cores from fp16 copies of the pools it
+ * makes in its workspace, which is larger by the pools' size in fp16):
  *   1 <= T <= 16, D in {256, 512, 768, 1024, 2048}, F % 256 == 0, F <= 1024:
  *     the dequant-fused grouped GEMV (mma.sync, TMA-streamed weights);
  *   T > 16, D % 256 == 0, F % 256 == 0, E <= 720: the grouped GEMM on the

@@ -936,6 +936,7 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
     uint64_t *full = (uint64_t *)(stages + (size_t)S * stage_bytes);
     uint64_t *empty = full + kMaxStages;
     int *act = (int *)(empty + kMaxStages);
+    int2 *ent = reinterpret_cast<int2 *>(act + 6 * (a.E + 1));     // (virtual expert, column group)
 
     if (tid == 0) {
         for (int s = 0; s < S; s++) {
@@ -947,8 +948,39 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
     // routing (perm/offsets) is complete: the gate/up kernel waited for it
     // before letting this grid launch
     const Active A = build_active_list(a, act);
+    // entries: every virtual expert's tokens in column groups of <= 8
+    // (one MMA N tile; at most 8 staged Hs rows a unit)
+    int *ecum = act + 4 * (a.E + 1);                  // raw-table space, free now
+    if (warp == 0) {
+        int base = 0;
+        for (int v0 = 0; v0 < A.n_virt; v0 += 32) {
+            const int v = v0 + lane;
+            const int ng = v < A.n_virt ? (virt(a, act, A.n_routed, v).cnt + kGuCols - 1) / kGuCols : 0;
+            int incl = ng;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t2 = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t2;
+            }
+            if (v < A.n_virt) ecum[v] = base + incl - ng;
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) ecum[A.n_virt] = base;
+    }
+    __syncthreads();
+    for (int v = tid; v < A.n_virt; v += blockDim.x)
+        for (int q = ecum[v]; q < ecum[v + 1]; q++) ent[q] = make_int2(v, q - ecum[v]);
+    __syncthreads();
+    const int n_ent = ecum[A.n_virt];
     const int tiles = D / kDnRows;
-    const int U = A.n_virt * tiles;
+    const int U = n_ent * tiles;
+    // the rows of entry q: (first permuted row, count <= 8, shared, slot, type)
+    auto entry = [&](int q, Virt *vi) {
+        const int2 e2 = ent[q];
+        *vi = virt(a, act, A.n_routed, e2.x);
+        vi->seg0 += e2.y * kGuCols;
+        vi->cnt = min(kGuCols, vi->cnt - e2.y * kGuCols);
+    };
 
     if (warp == kDW) {
         if (lane == 0) {
@@ -957,16 +989,18 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
             uint32_t used = 0u, last_ph = 0u;
             int pend_s[kMaxStages], pend_v[kMaxStages];
             int npend = 0;
-            auto issue_h = [&](int st, int v) {
-                const Virt vi = virt(a, act, A.n_routed, v);
+            auto issue_h = [&](int st, int q) {
+                Virt vi;
+                entry(q, &vi);
                 bulk_g2s(stages + (size_t)st * stage_bytes + wbytes, a.Hs + (size_t)vi.seg0 * a.hrow,
                          (uint32_t)(vi.cnt * hbytes), &full[st]);
             };
             int i = 0;                          // local unit index
             for (int u = blockIdx.x; u < U && ok; u += gridDim.x, i++) {
-                const int v = u / tiles, dt = u % tiles;
+                const int v = u / tiles, dt = u % tiles;    // v: entry
                 const DnSlot sl = dn_slot(i, G, Sg);
-                const Virt vi = virt(a, act, A.n_routed, v);
+                Virt vi;
+                entry(v, &vi);
                 const int pitch = vi.shared ? ps : pr;
                 if (!mbar_wait(&empty[sl.stage], sl.phase ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
                 uint8_t *dst = stages + (size_t)sl.stage * stage_bytes;
@@ -1003,9 +1037,10 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
     const uint32_t st_a = smem_u32(stages);
     int i = grp;
     for (int u = blockIdx.x + grp * gridDim.x; u < U; u += G * gridDim.x, i += G) {
-        const int v = u / tiles, dt = u % tiles;
+        const int v = u / tiles, dt = u % tiles;            // v: entry
         const DnSlot sl = dn_slot(i, G, Sg);
-        const Virt vi = virt(a, act, A.n_routed, v);
+        Virt vi;
+        entry(v, &vi);
         const int bsz = qt_unit_bytes(vi.qt);
         const int pitch = vi.shared ? ps : pr;
         const int nb = vi.Fv / QK;
@@ -1834,12 +1869,13 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
     }
     // ---- down: Y rows
     {
-        const int hrows = std::min(a.T, 16);
+        const int hrows = std::min(a.T, kGuCols);
         const int pr = tma_row_bytes((int)qt_row_bytes(a.qt, a.F));
         const int ps = a.sF > 0 ? tma_row_bytes((int)qt_row_bytes(a.sqt, a.sF)) : 0;
         const size_t wbytes = (size_t)kDnRows * std::max(pr, ps);
         const size_t stage_bytes = round_up(wbytes + (size_t)hrows * a.hrow * 2, 128);
-        const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) + 1024;
+        const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) +
+                             (size_t)(a.E + 2 + kMaxTk / kGuCols + 2) * sizeof(int2) + 1024;
         if (fixed + stage_bytes > kDecSmemMax) {
             set_error("decode path: a %zu-byte stage does not fit shared memory", stage_bytes);
             return MOE_ERR_SHAPE;
@@ -1850,7 +1886,7 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         const int G = fit >= 4 ? 4 : fit >= 2 ? 2 : 1;
         const int Sg = std::min(2, fit / G);
         const size_t smem = fixed + (size_t)G * Sg * stage_bytes;
-        const int U_max = (a.E + 1) * (a.D / kDnRows);
+        const int U_max = (a.E + 1 + a.T * a.k / kGuCols) * (a.D / kDnRows);
         const int grid = std::max(1, std::min(sms, U_max));
         // no trace mark here: an event between the two kernels would cancel
         // their programmatic overlap
@@ -1921,7 +1957,8 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
         set_error("decode path: the fused combine needs a rows buffer");
         return MOE_ERR_INVALID_ARG;
     }
-    return T > 8 ? run_decode<2>(a, pool.n_slots, s, tr) : run_decode<1>(a, pool.n_slots, s, tr);
+    // the down kernel takes at most 8 tokens a unit: one column tile
+    return run_decode<1>(a, pool.n_slots, s, tr);
 }
 
 // ------------------------------------------------ 8-bit activations: host

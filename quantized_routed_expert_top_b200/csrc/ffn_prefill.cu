@@ -388,11 +388,17 @@ __device__ __forceinline__ PfTile pf_tile(const int *tcum, const int *segs, int 
     return t;
 }
 
-// ALL: the call has a type other than Q4_0 and Q8_0 (a separate
-// instantiation keeps the other types' dequantisers and window logic out of
-// the two types' kernel)
-template <int MODE, bool ALL>
+// BK, how the weights reach the B stages: kBkBasic, Q4_0 / Q8_0 dequantised
+// from raw windows; kBkAll, any 32-weight type or Q4_K dequantised the same
+// way (a separate instantiation keeps their code out of the two types'
+// kernel); kBkF16, fp16 weights (a pool converted by pf_dequant_f16_kernel)
+// copied straight into the swizzled stages by tensor copies, no
+// dequantising warps.
+enum : int { kBkBasic = 0, kBkAll = 1, kBkF16 = 2 };
+
+template <int MODE, int BK>
 __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const __grid_constant__ PfMaps maps) {
+    constexpr bool ALL = BK == kBkAll;
     extern __shared__ __align__(1024) uint8_t smem_pf[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t *ringA = smem_pf + ((1024u - (smem_u32(smem_pf) & 1023u)) & 1023u);
@@ -424,7 +430,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
             mbar_init(&emptyA[s], 1);
         }
         for (int s = 0; s < kPSB; s++) {
-            mbar_init(&fullB[s], kPBW * 32);
+            mbar_init(&fullB[s], BK == kBkF16 ? 1 : kPBW * 32);
             mbar_init(&emptyB[s], 1);
         }
         for (int r = 0; r < kPR; r++) {
@@ -526,7 +532,38 @@ __global__ void __launch_bounds__(kPThreads, 1) pf_gemm_kernel(PfArgs a, const _
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp < kPAW + kPBW) {
-        if constexpr (!ALL) {
+        if constexpr (BK == kBkF16) {
+            // ------------------------------------ B producer, fp16 weights
+            // one thread copies each K stage of the tile's 256 weight rows
+            // (64 fp16 = 128 bytes a row) into the stage with the 128-byte
+            // swizzle the MMA descriptors name
+            if (warp == kPAW && lane == 0) {
+                int g = 0;
+                bool ok = true;
+                for (int tau = blockIdx.x; tau < n_tiles && ok; tau += gridDim.x) {
+                    const PfTile t = pf_tile(tcum, segs, nv, nt, tau);
+                    const bool sh = t.v == a.E;
+                    const int slot = sh ? 0 : (a.slot_map ? __ldg(a.slot_map + t.v) : t.v);
+                    for (int ks = 0; ks < nk; ks++, g++) {
+                        const int s = g % kPSB;
+                        if (!mbar_wait(&emptyB[s], ((g / kPSB) & 1) ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
+                        uint8_t *dst = ringB + (size_t)s * kPStageB;
+                        mbar_arrive_expect_tx(&fullB[s], (uint32_t)kPStageB);
+                        if (MODE == kPGateUp) {
+                            const int y = slot * a.F + t.n * kPNg;
+                            tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, ks * kPK, y, &fullB[s]);
+                            tma_load_2d(dst + kPStageB / 2, sh ? &maps.s1 : &maps.w1, ks * kPK, y, &fullB[s]);
+                        } else {
+                            tma_load_2d(dst, sh ? &maps.s0 : &maps.w0, ks * kPK, slot * a.D + t.n * kPNd,
+                                        &fullB[s]);
+                        }
+                    }
+                }
+                // copies still in flight must land before the CTA exits
+                for (int q = g > kPSB ? g - kPSB : 0; q < g; q++)
+                    mbar_wait(&fullB[q % kPSB], (uint32_t)((q / kPSB) & 1), a.err, kErrTimeoutDrain);
+            }
+        } else if constexpr (!ALL) {
             // ------------------------------------ B producers, Q4_0 / Q8_0
             // (the other types' code below ran these two types 5-8% slower)
             // Raw windows (the 16-byte-aligned bytes holding four blocks = two
@@ -904,9 +941,10 @@ __global__ void __launch_bounds__(256) pf_convert_kernel(const XT *__restrict__ 
 // tensor copies; it takes the portable kernels)
 static bool pf_type_ok(int qt) { return qt_known(qt) && qt != MOE_Q6_K; }
 
-bool prefill_path_ok(int T, int D, int F, int sF, int E, int qt, int sqt) {
+bool prefill_path_ok(int T, int D, int F, int sF, int E, int qt, int sqt, bool allow_f16) {
+    auto ok = [&](int q) { return pf_type_ok(q) || (allow_f16 && qt_known(q)); };
     return T > 16 && D % kPNd == 0 && F % kPNg == 0 && D % 256 == 0 && F % 256 == 0 &&
-           (sF == 0 || (sF == F && pf_type_ok(sqt))) && pf_type_ok(qt) &&
+           (sF == 0 || (sF == F && ok(sqt))) && ok(qt) &&
            E <= kPfMaxExperts && pf_smem_bytes(E) <= 227 * 1024;
 }
 
@@ -945,7 +983,7 @@ static moe_status pf_encode(CUtensorMap *m, const void *base, size_t row_bytes, 
     return MOE_OK;
 }
 
-template <int MODE, bool ALL>
+template <int MODE, int BK>
 static cudaError_t launch_pf1(const PfArgs &a, const PfMaps &m, int grid, cudaStream_t s) {
     const size_t smem = pf_smem_bytes(a.E);
     cudaLaunchConfig_t cfg = {};
@@ -958,33 +996,116 @@ static cudaError_t launch_pf1(const PfArgs &a, const PfMaps &m, int grid, cudaSt
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaFuncSetAttribute(pf_gemm_kernel<MODE, ALL>,
+    cudaError_t e = cudaFuncSetAttribute(pf_gemm_kernel<MODE, BK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, pf_gemm_kernel<MODE, ALL>, a, m);
+    return cudaLaunchKernelEx(&cfg, pf_gemm_kernel<MODE, BK>, a, m);
 }
 
 template <int MODE>
-static cudaError_t launch_pf(const PfArgs &a, const PfMaps &m, int grid, cudaStream_t s) {
+static cudaError_t launch_pf(const PfArgs &a, const PfMaps &m, int grid, cudaStream_t s, bool f16) {
+    if (f16) return launch_pf1<MODE, kBkF16>(a, m, grid, s);
     auto basic = [](int q) { return q == MOE_Q4_0 || q == MOE_Q8_0; };
     const bool all = !basic(a.qt) || (a.shared && !basic(a.sqt));
-    return all ? launch_pf1<MODE, true>(a, m, grid, s) : launch_pf1<MODE, false>(a, m, grid, s);
+    return all ? launch_pf1<MODE, kBkAll>(a, m, grid, s) : launch_pf1<MODE, kBkBasic>(a, m, grid, s);
 }
+
+// fp16 tensor maps over a converted pool: [rows][K] halves, boxes of 64
+// halves (128 bytes, the 128-byte swizzle's span) x box_rows rows
+static moe_status pf_encode_f16(CUtensorMap *m, const __half *base, int K, size_t nrows, int box_rows) {
+    static PfEncodeFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PfEncodeFn)p;
+    }
+    if (!fn) { set_error("prefill path: cuTensorMapEncodeTiled unavailable"); return MOE_ERR_CUDA; }
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)nrows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half *>(base), dims, strides, box,
+                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("prefill path: fp16 tensor map encoding failed (%d)", (int)r);
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+// A pool's rows of any block type -> fp16 rows (one warp a row, lanes over
+// 32-weight units; each weight the portable decoder's fp32 value rounded
+// once to fp16)
+template <int QT>
+__global__ void __launch_bounds__(256)
+pf_dequant_f16_kernel(const uint8_t *__restrict__ src, size_t nrows, int ncols, __half *__restrict__ dst) {
+    const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= nrows) return;
+    const int lane = threadIdx.x & 31;
+    const uint8_t *r = src + row * qt_row_bytes(QT, ncols);
+    for (int b = lane; b < ncols / QK; b += 32) {
+        float w[32];
+        decode_unit_global<QT>(r, b, w);
+        uint4 *o = reinterpret_cast<uint4 *>(dst + row * ncols + (size_t)b * QK);
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            __half2 h[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) h[i] = __floats2half2_rn(w[8 * q + 2 * i], w[8 * q + 2 * i + 1]);
+            o[q] = *reinterpret_cast<uint4 *>(h);
+        }
+    }
+}
+
+static moe_status dequant_f16(const uint8_t *src, int qt, size_t nrows, int ncols, __half *dst,
+                              cudaStream_t s) {
+    const unsigned grid = (unsigned)((nrows + 7) / 8);
+    switch (qt) {
+#define MOE_DQ(QT) case QT: pf_dequant_f16_kernel<QT><<<grid, 256, 0, s>>>(src, nrows, ncols, dst); break;
+        MOE_DQ(MOE_Q4_0)
+        MOE_DQ(MOE_Q4_1)
+        MOE_DQ(MOE_Q5_0)
+        MOE_DQ(MOE_Q5_1)
+        MOE_DQ(MOE_Q8_0)
+        MOE_DQ(MOE_Q4_K)
+        MOE_DQ(MOE_Q6_K)
+#undef MOE_DQ
+    default:
+        set_error("prefill path: unsupported quant type %d", qt);
+        return MOE_ERR_UNSUPPORTED_QTYPE;
+    }
+    return cuda_status(cudaGetLastError(), "pf_dequant_f16_kernel");
+}
+
+// halves of the fp16 copies the fp16-weight mode needs (routed pool, then the
+// shared expert)
+size_t prefill_f16_halves(int n_slots, int D, int F, int sF) {
+    return (size_t)n_slots * 3 * D * F + (size_t)3 * D * sF;
+}
+bool prefill_needs_f16(int qt, int sqt, int sF) { return qt == MOE_Q6_K || (sF > 0 && sqt == MOE_Q6_K); }
 
 moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, int E, int k,
                               const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
                               const uint8_t *mask, bool routed, const moe_pool *shared, int sF,
                               __half *x16, __half *H, float *Y, int *err, cudaStream_t s,
-                              Tracer *tr) {
-    if (!pf_type_ok(pool.qtype)) {
+                              Tracer *tr, __half *w16) {
+    const bool f16 = prefill_needs_f16(pool.qtype, shared ? shared->qtype : 0, shared ? sF : 0);
+    if (f16 && !w16) {
+        set_error("prefill path: Q6_K needs the fp16 pool copies (the layer's workspace)");
+        return MOE_ERR_UNSUPPORTED_QTYPE;
+    }
+    if (!f16 && !pf_type_ok(pool.qtype)) {
         set_error("prefill path: unsupported quant type %d", (int)pool.qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }
-    if (shared && !pf_type_ok(shared->qtype)) {
+    if (!f16 && shared && !pf_type_ok(shared->qtype)) {
         set_error("prefill path: unsupported shared-expert quant type %d", (int)shared->qtype);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }
-    if (!prefill_path_ok(T, D, F, shared ? sF : 0, E, pool.qtype, shared ? shared->qtype : 0)) {
+    if (!prefill_path_ok(T, D, F, shared ? sF : 0, E, pool.qtype, shared ? shared->qtype : 0, f16)) {
         set_error("prefill path: shape T=%d D=%d F=%d not supported", T, D, F);
         return MOE_ERR_SHAPE;
     }
@@ -1015,14 +1136,45 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
         pf_convert_kernel<float><<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>((const float *)x, x16, n8);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "pf_convert_kernel");
-    // weight tensor maps: boxes of one raw window row
-    const size_t rg = qt_row_bytes(pool.qtype, D), rd = qt_row_bytes(pool.qtype, F);
-    const int wr = pf_window_bytes(pool.qtype);
     PfMaps mg, md;
     memset(&mg, 0, sizeof(mg));
     memset(&md, 0, sizeof(md));
     moe_status st;
     const size_t rows_f = (size_t)pool.n_slots * F, rows_d = (size_t)pool.n_slots * D;
+    if (f16) {
+        // every slot's weights (and the shared expert's) to fp16 rows, then
+        // tensor maps over those
+        __half *g16 = w16, *u16 = g16 + rows_f * D, *d16 = u16 + rows_f * D;
+        mark(tr, MOE_KERNEL_CONVERT);
+        if ((st = dequant_f16((const uint8_t *)pool.gate, pool.qtype, rows_f, D, g16, s)) ||
+            (st = dequant_f16((const uint8_t *)pool.up, pool.qtype, rows_f, D, u16, s)) ||
+            (st = dequant_f16((const uint8_t *)pool.down, pool.qtype, rows_d, F, d16, s)))
+            return st;
+        if ((st = pf_encode_f16(&mg.w0, g16, D, rows_f, kPNg)) ||
+            (st = pf_encode_f16(&mg.w1, u16, D, rows_f, kPNg)) ||
+            (st = pf_encode_f16(&md.w0, d16, F, rows_d, kPNd)))
+            return st;
+        if (shared) {
+            __half *sg16 = d16 + rows_d * F, *su16 = sg16 + (size_t)sF * D, *sd16 = su16 + (size_t)sF * D;
+            if ((st = dequant_f16((const uint8_t *)shared->gate, shared->qtype, sF, D, sg16, s)) ||
+                (st = dequant_f16((const uint8_t *)shared->up, shared->qtype, sF, D, su16, s)) ||
+                (st = dequant_f16((const uint8_t *)shared->down, shared->qtype, D, sF, sd16, s)))
+                return st;
+            if ((st = pf_encode_f16(&mg.s0, sg16, D, sF, kPNg)) ||
+                (st = pf_encode_f16(&mg.s1, su16, D, sF, kPNg)) ||
+                (st = pf_encode_f16(&md.s0, sd16, sF, D, kPNd)))
+                return st;
+        }
+        const int grid = num_sms();
+        mark(tr, MOE_KERNEL_GATEUP);
+        if ((e = launch_pf<kPGateUp>(a, mg, grid, s, true)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<gate/up, fp16>");
+        mark(tr, MOE_KERNEL_DOWN);
+        if ((e = launch_pf<kPDown>(a, md, grid, s, true)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<down, fp16>");
+        return MOE_OK;
+    }
+    // weight tensor maps: boxes of one raw window row
+    const size_t rg = qt_row_bytes(pool.qtype, D), rd = qt_row_bytes(pool.qtype, F);
+    const int wr = pf_window_bytes(pool.qtype);
     if ((st = pf_encode(&mg.w0, pool.gate, rg, rows_f, wr, kPNg)) ||
         (st = pf_encode(&mg.w1, pool.up, rg, rows_f, wr, kPNg)) ||
         (st = pf_encode(&md.w0, pool.down, rd, rows_d, wr, kPNd)))
@@ -1037,9 +1189,9 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
     }
     const int grid = num_sms();
     mark(tr, MOE_KERNEL_GATEUP);
-    if ((e = launch_pf<kPGateUp>(a, mg, grid, s)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<gate/up>");
+    if ((e = launch_pf<kPGateUp>(a, mg, grid, s, false)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<gate/up>");
     mark(tr, MOE_KERNEL_DOWN);
-    if ((e = launch_pf<kPDown>(a, md, grid, s)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<down>");
+    if ((e = launch_pf<kPDown>(a, md, grid, s, false)) != cudaSuccess) return cuda_status(e, "pf_gemm_kernel<down>");
     return MOE_OK;
 }
 

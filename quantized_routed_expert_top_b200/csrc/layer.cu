@@ -22,6 +22,7 @@ struct LayerWs {
     float *sh_rows;      // [T, D]
     __half *Hs;          // decode path: g*h in fp16 fragment order
     __half *x16, *H16;   // prefill path: fp16 activations and hidden rows
+    __half *w16;         // prefill path: fp16 copies of the pools (Q6_K)
     int8_t *hq;          // 8-bit activations: h codes and their (scale, code sum)
     float2 *hs;
 };
@@ -52,8 +53,10 @@ static LayerWs carve(const moe_layer_args &a, Carver &c) {
         w.rows = c.take<float>(decode_rows_floats(a.T, a.k, a.D));
         return w;
     }
-    if (prefill_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0, a.E, qt, sqt)) {
+    if (prefill_path_ok(a.T, a.D, a.F, a.shared ? a.shared_F : 0, a.E, qt, sqt, true)) {
         const int sF = a.shared ? a.shared_F : 0;
+        if (prefill_needs_f16(qt, sqt, sF))
+            w.w16 = c.take<__half>(prefill_f16_halves(a.pool ? a.pool->n_slots : a.E, a.D, a.F, sF));
         w.x16 = c.take<__half>(prefill_x16_halves(a.T, a.D));
         w.H16 = c.take<__half>(prefill_h_halves(a.T, a.k, a.F, sF));
         w.rows = c.take<float>(prefill_y_floats(a.T, a.k, a.D, sF));
@@ -149,7 +152,7 @@ moe_status layer_forward(const moe_layer_args &a, void *ws, size_t ws_bytes, cud
             (st = launch_ffn_prefill(a.x, a.x_dtype, a.T, a.D, a.F, a.E, a.k, perm, offsets,
                                      *a.pool, a.expert_mask, do_ffn,
                                      do_shared ? a.shared : nullptr, sF, w.x16, w.H16, w.rows,
-                                     w.status, s, tr)) != MOE_OK)
+                                     w.status, s, tr, w.w16)) != MOE_OK)
             return st;
         st = MOE_OK;
         if (do_comb)

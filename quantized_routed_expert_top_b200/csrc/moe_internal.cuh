@@ -303,7 +303,11 @@ size_t decode_hs_halves(int T, int k, int F, int sF);
 size_t decode_rows_floats(int T, int k, int D);
 // ffn_prefill.cu -- large T on the tensor cores: x -> fp16, gate/up grouped
 // GEMM (H fp16), down grouped GEMM (Y fp32 rows, then the combine kernel)
-bool prefill_path_ok(int T, int D, int F, int sF, int E, int qt, int sqt);
+// allow_f16: the caller can give fp16 copies of the pools (prefill_f16_halves),
+// which lets any block type (Q6_K needs it) take the tensor-core path
+bool prefill_path_ok(int T, int D, int F, int sF, int E, int qt, int sqt, bool allow_f16 = false);
+bool prefill_needs_f16(int qt, int sqt, int sF);
+size_t prefill_f16_halves(int n_slots, int D, int F, int sF);
 size_t prefill_x16_halves(int T, int D);
 size_t prefill_h_halves(int T, int k, int F, int sF);
 size_t prefill_y_floats(int T, int k, int D, int sF);
@@ -313,7 +317,7 @@ moe_status launch_ffn_prefill(const void *x, int x_dtype, int T, int D, int F, i
                               const int32_t *perm, const int32_t *offsets, const moe_pool &pool,
                               const uint8_t *mask, bool routed, const moe_pool *shared, int sF,
                               __half *x16, __half *H, float *Y, int *err, cudaStream_t s,
-                              Tracer *tr);
+                              Tracer *tr, __half *w16 = nullptr);
 // gates != NULL: fused layer (gates folded into the rows; rows_out holds
 // [T*k + T, D] gated rows); gates == NULL: rows mode (un-gated Y rows [T*k, D]
 // in permuted order).  routed: run the routed experts the mask admits;

@@ -6,8 +6,10 @@ Each type runs the decode GEMV (T <= 16, every compiled D geometry), the
 tcgen05 grouped GEMM (T > 16, ragged row tiles, experts with a handful of
 rows) and the portable kernel (D, F not multiples of 256, or F > 1024), as
 a routed pool and as the shared expert beside a routed pool of another type.
-Q6_K runs the portable kernel on every shape (its 210-byte blocks leave
-rows of 768 weights without the 16-byte alignment tensor copies need).  The
+Q6_K runs the portable kernel at decode shapes and through moe_expert_ffn
+(its 210-byte blocks leave rows of 768 weights without the 16-byte alignment
+tensor copies need), and the tensor-core GEMM on fp16 copies of its pool in
+the fused layer at T > 16.  The
 bar is the one of the Q4_0 / Q8_0 parity tests: max|gpu - oracle| /
 max|oracle| <= 2e-3 on fp32 outputs, and bit-identical rows for a masked
 two-call split.
@@ -168,3 +170,21 @@ def test_masked_two_phase_rows_are_bit_identical(moe, qtype, T):
     moe.expert_ffn(x, perm, offsets, pool, cfg.k, cfg.F, mask=1 - m, out=two)
     torch.cuda.synchronize()
     assert torch.equal(full, two)
+
+
+def test_q6k_prefill_layer_phases_are_bit_identical(moe):
+    # Q6_K at T > 16 runs the tensor-core GEMM on fp16 copies of the pool made
+    # in the layer's workspace; a masked two-call split gives the same bits
+    L = _inputs(_cfg("q6_k", 300, D=1024, F=512, E=16, k=4, shared_F=512, shared_qtype="q6_k",
+                     seed=580))
+    lay = _layer(moe, L)
+    x = dev_x(L)
+    y1 = lay.forward(x).clone()
+    m = torch.from_numpy(np.random.default_rng(9).integers(0, 2, L.cfg.E).astype(np.uint8)).cuda()
+    y2 = torch.full_like(y1, float("nan"))
+    lay.forward(x, out=y2, mask=m, phases=moe.PHASE_ROUTE | moe.PHASE_FFN | moe.PHASE_SHARED)
+    lay.forward(x, out=y2, mask=1 - m, phases=moe.PHASE_FFN | moe.PHASE_COMBINE)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    _check_layer(moe, L, y1, lay.ids, 40)
+    assert moe.workspace_status(lay.ws) == (0, moe.DEV_OK)
