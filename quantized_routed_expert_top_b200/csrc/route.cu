@@ -279,7 +279,7 @@ template <typename XT>
 __global__ void __launch_bounds__(256)
 route_logits_sgemm_kernel(const XT *__restrict__ x, const float *__restrict__ W,
                           const float *__restrict__ bias, int T, int D, int E,
-                          float *__restrict__ logits, int kseg) {
+                          float *__restrict__ logits, int kseg, int xvec) {
     extern __shared__ __align__(16) float smem_lg[];
     float *As = smem_lg;                                   // [2][kSK][kSM + 1]
     float *Bs = As + 2 * kSK * (kSM + 1);                  // [2][kSK][kSN + 4]
@@ -298,8 +298,29 @@ route_logits_sgemm_kernel(const XT *__restrict__ x, const float *__restrict__ W,
     float4 rb[4];
     auto load = [&](int k0) {
         const int t = t0 + am;
+        const size_t xo = (size_t)t * D + k0 + ak;
+        if (t >= T) {
 #pragma unroll
-        for (int i = 0; i < 8; i++) ra[i] = (t < T) ? load_act(x, (size_t)t * D + k0 + ak + i) : 0.f;
+            for (int i = 0; i < 8; i++) ra[i] = 0.f;
+        } else if (xvec) {                 // 8 activations in 16 (bf16) or 32 (fp32) bytes
+            if constexpr (sizeof(XT) == 2) {
+                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(x + xo));
+                const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    ra[2 * i] = __uint_as_float(u[i] << 16);
+                    ra[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+                }
+            } else {
+                const float4 w0 = __ldg(reinterpret_cast<const float4 *>(x + xo));
+                const float4 w1 = __ldg(reinterpret_cast<const float4 *>(x + xo) + 1);
+                ra[0] = w0.x; ra[1] = w0.y; ra[2] = w0.z; ra[3] = w0.w;
+                ra[4] = w1.x; ra[5] = w1.y; ra[6] = w1.z; ra[7] = w1.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; i++) ra[i] = load_act(x, xo + i);
+        }
 #pragma unroll
         for (int i = 0; i < 4; i++) {
             const int e = e0 + bc;
@@ -759,19 +780,21 @@ moe_status launch_route(const void *x, int x_dtype, const float *w_router,
         const dim3 grid((T + kSM - 1) / kSM, (E + kSN - 1) / kSN, nsplit);
         const size_t sm = (size_t)(2 * kSK * (kSM + 1) + 2 * kSK * (kSN + 4)) * sizeof(float);
         float *dst = nsplit > 1 ? part : L;
+        // 16-byte loads of 8 activations: x 16-byte aligned (rows then are too: D % 32 == 0)
+        const int xvec = ((uintptr_t)x % 16) == 0;
         cudaError_t e;
         if (x_dtype == MOE_BF16) {
             e = cudaFuncSetAttribute(route_logits_sgemm_kernel<__nv_bfloat16>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
             if (e == cudaSuccess)
                 route_logits_sgemm_kernel<__nv_bfloat16><<<grid, 256, sm, s>>>(
-                    (const __nv_bfloat16 *)x, w_router, bias, T, D, E, dst, D / nsplit);
+                    (const __nv_bfloat16 *)x, w_router, bias, T, D, E, dst, D / nsplit, xvec);
         } else {
             e = cudaFuncSetAttribute(route_logits_sgemm_kernel<float>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
             if (e == cudaSuccess)
                 route_logits_sgemm_kernel<float><<<grid, 256, sm, s>>>((const float *)x, w_router,
-                                                                       bias, T, D, E, dst, D / nsplit);
+                                                                       bias, T, D, E, dst, D / nsplit, xvec);
         }
         if (e != cudaSuccess) return cuda_status(e, "route_logits_sgemm_kernel attribute");
         if (nsplit > 1) {
