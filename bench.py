@@ -1037,7 +1037,8 @@ def measure_std_types(torch, moe, steps, warmup, world, local, peaks, no_graph, 
     """The decode and prefill layers with experts in Q4_1, Q5_0, Q5_1, Q4_K
     and Q6_K: one expert pool per type (the decode shape's weights, encoded
     in that type), each workload with its own roofline and end-to-end
-    number (Q6_K runs the portable kernels)."""
+    number (Q6_K prefill converts its pool to fp16 rows for the tensor-core
+    GEMM)."""
     out = {}
     for qt in STD_TYPES:
         cfg = S.CONFIGS["decode"]

@@ -255,9 +255,12 @@ moe_status moe_permute(const int32_t *ids, int T, int k, int E, int32_t *counts,
  *     the dequant-fused grouped GEMV (mma.sync, TMA-streamed weights);
  *   T > 16, D % 256 == 0, F % 256 == 0, E <= 720: the grouped GEMM on the
  *     tcgen05 tensor cores (weights dequantised to fp16 in shared memory);
- *   any other shape, and Q6_K on every shape: a portable CUDA-core kernel
- *     (correct, not tuned; Q6_K rows of 768 weights are 630 bytes, which
- *     tensor copies cannot address).
+ *   any other shape: a portable CUDA-core kernel (correct, not tuned).
+ * Q6_K (210-byte blocks) takes the GEMV only at D = 2048, where its gate/up
+ * rows are whole 16-byte units for the tensor copies (its down rows are
+ * copied in 8-row groups, which always are), and the portable kernel at
+ * every other shape here, T > 16 included (630-byte rows of 768 weights are
+ * not tensor-copyable; the fused layer converts instead, as above).
  *   x           device [T, D], x_dtype F32 or BF16.
  *   perm,offsets from moe_permute.
  *   pool        expert weights (see moe_pool); pool->qtype fixes the format.

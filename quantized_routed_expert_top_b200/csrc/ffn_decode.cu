@@ -118,6 +118,18 @@ __host__ __device__ inline int tma_row_bytes(int rb) {
     if (((r / 16) & 1) == 0) r += 16;
     return r;
 }
+// Shared-memory pitch of a down-projection row (F weights): as
+// tma_row_bytes, except Q6_K, whose rows (210 * F / 256 bytes, 2-byte
+// aligned when F / 256 is odd) arrive as whole 8-row groups (16-byte
+// multiples) and stay packed.
+__host__ __device__ inline int dn_pitch(int qt, int F) {
+    const int rb = (int)qt_row_bytes(qt, F);
+    return qt == MOE_Q6_K ? rb : tma_row_bytes(rb);
+}
+// Q6_K down rows as a 3-D tensor: 560-byte chunks (70 elements of 8 bytes),
+// 3 F / 256 chunks an 8-row group, one group per 8 rows of D
+constexpr int kQ6Chunk = 560;
+
 // Blocks per K-slice for a block size: the largest multiple of 8 dividing
 // the row's nb blocks whose staged row still fits one box (<= 256 elements
 // of 8 bytes = 2048 bytes).
@@ -417,20 +429,28 @@ __device__ __forceinline__ void q4k_codes(uint32_t blk, int j, int c, uint32_t *
     r[2] = prmt(w1, HI, 0x4240);
     r[3] = prmt(w1, HI, 0x4341);
 }
+// A Q4_K block's head: d, dmin and the packed 6-bit scales and mins
+struct Q4kHead {
+    uint32_t s0, s1, s2;
+    float d, dmin;
+};
+__device__ __forceinline__ Q4kHead q4k_head(uint32_t blk) {
+    const uint32_t w = lds32(blk);
+    return {lds32(blk + 4), lds32(blk + 8), lds32(blk + 12), h2f(w & 0xFFFFu), h2f(w >> 16)};
+}
 // Scale D = d * sc_j and min M = dmin * m_j of sub-block j (weight D q - M)
-__device__ __forceinline__ void q4k_params(uint32_t blk, int j, float *D, float *M) {
-    const uint32_t s0 = lds32(blk + 4), s1 = lds32(blk + 8), s2 = lds32(blk + 12);
+__device__ __forceinline__ void q4k_params(const Q4kHead &h, int j, float *D, float *M) {
     const int jj = j & 3, sh = 8 * jj;
     int sc, m;
     if (j < 4) {
-        sc = (s0 >> sh) & 63;
-        m = (s1 >> sh) & 63;
+        sc = (h.s0 >> sh) & 63;
+        m = (h.s1 >> sh) & 63;
     } else {
-        sc = ((s2 >> sh) & 15) | (((s0 >> (sh + 6)) & 3) << 4);
-        m = ((s2 >> (sh + 4)) & 15) | (((s1 >> (sh + 6)) & 3) << 4);
+        sc = ((h.s2 >> sh) & 15) | (((h.s0 >> (sh + 6)) & 3) << 4);
+        m = ((h.s2 >> (sh + 4)) & 15) | (((h.s1 >> (sh + 6)) & 3) << 4);
     }
-    *D = h2f(lds16(blk)) * (float)sc;
-    *M = h2f(lds16(blk + 2)) * (float)m;
+    *D = h.d * (float)sc;
+    *M = h.dmin * (float)m;
 }
 
 // As gateup_slice for Q4_K: units kb0 .. kb0 + WB - 1 of the slice whose
@@ -440,18 +460,30 @@ template <int NTILE, int WB>
 __device__ __forceinline__ void gateup_slice_q4k(uint32_t rowbase, uint32_t r8, int kb0,
                                                  const uint32_t *xa, const uint32_t (*sa)[2], int c,
                                                  float (*acc)[4]) {
+    // WB dividing 8: the warp's units lie in one block (kb0 a multiple of
+    // WB), whose head is read once
+    constexpr bool ONE = 8 % WB == 0;
+    Q4kHead hlo{}, hhi{};
+    if constexpr (ONE) {
+        const uint32_t blk0 = rowbase + (uint32_t)(kb0 >> 3) * 144u;
+        hlo = q4k_head(blk0);
+        hhi = q4k_head(blk0 + r8);
+    }
 #pragma unroll
     for (int bl = 0; bl < WB; bl++) {
-        // WB == 8: the warp's units are one whole block (kb0 a multiple of 8)
         const int b = kb0 + bl;
         const int j = WB == 8 ? bl : (b & 7);
         const uint32_t blk = rowbase + (uint32_t)((WB == 8 ? kb0 : b) >> 3) * 144u;
         uint32_t lo[4], hi[4];
         q4k_codes(blk, j, c, lo);
         q4k_codes(blk + r8, j, c, hi);
+        if constexpr (!ONE) {
+            hlo = q4k_head(blk);
+            hhi = q4k_head(blk + r8);
+        }
         float dlo, mlo, dhi, mhi;
-        q4k_params(blk, j, &dlo, &mlo);
-        q4k_params(blk + r8, j, &dhi, &mhi);
+        q4k_params(hlo, j, &dlo, &mlo);
+        q4k_params(hhi, j, &dhi, &mhi);
         mlo *= 1.f / 1024.f;
         mhi *= 1.f / 1024.f;
         const uint32_t a0[4] = {lo[0], hi[0], lo[1], hi[1]};
@@ -471,6 +503,68 @@ __device__ __forceinline__ void gateup_slice_q4k(uint32_t rowbase, uint32_t r8, 
     }
 }
 
+// ---------------------------------------------------------------- Q6_K
+// Q6_K blocks are 210 bytes (ql[128], qh[64], int8 scales[16], fp16 d), so
+// consecutive blocks alternate between 4-byte and 2-byte alignment: MIS is
+// the block's alignment mod 4.  Sub-block j (32 weights, unit j of the block)
+// lies in half h = j / 4, quarter r = j % 4: weight l of it has its low four
+// bits in nibble r / 2 of ql[64h + 32(r % 2) + l] and its high two in bits
+// 2r, 2r+1 of qh[32h + l], scale scales[8h + 2r + l / 16].  Codes for thread
+// c in the fragment order of magic_codes, as exact fp16 (q - 32).
+template <int MIS>
+__device__ __forceinline__ void q6k_codes(uint32_t blk, int j, int c, uint32_t *r) {
+    const int h = j >> 2, q = j & 3;
+    const uint32_t la = blk + 64 * h + 32 * (q & 1) + 4 * c, ha = blk + 128 + 32 * h + 4 * c;
+    const int s4 = 4 * (q >> 1), s2 = 2 * q;
+    const uint32_t w0 = ((lds_word<MIS>(la) >> s4) & 0x0F0F0F0Fu) |
+                        (((lds_word<MIS>(ha) >> s2) & 0x03030303u) << 4);
+    const uint32_t w1 = ((lds_word<MIS>(la + 16) >> s4) & 0x0F0F0F0Fu) |
+                        (((lds_word<MIS>(ha + 16) >> s2) & 0x03030303u) << 4);
+    const uint32_t HI = 0x64646464u, OFF = 0x64206420u;          // 1024 + code, minus 1056
+    r[0] = hsub2_u(prmt(w0, HI, 0x4240), OFF);
+    r[1] = hsub2_u(prmt(w0, HI, 0x4341), OFF);
+    r[2] = hsub2_u(prmt(w1, HI, 0x4240), OFF);
+    r[3] = hsub2_u(prmt(w1, HI, 0x4341), OFF);
+}
+// d * scale of the two 16-weight halves of sub-block j (d: the block's)
+__device__ __forceinline__ void q6k_scales(uint32_t blk, int j, float d, float *D0, float *D1) {
+    const uint32_t s = lds16(blk + 192 + 2 * j);
+    *D0 = d * (float)(int)(int8_t)(s & 0xFFu);
+    *D1 = d * (float)(int)(int8_t)(s >> 8);
+}
+// One Q6_K block (8 units) of a 16-row tile against the B fragments at ba
+// (64 bytes a unit): each unit's two 16-weight halves take their own MMA and
+// scale.  Used by the gate/up warps (B = activations) and the down warps
+// (B = Hs).
+template <int MIS, int NTILE>
+__device__ __forceinline__ void block_q6k(uint32_t blk, uint32_t r8, const uint32_t *ba, int c,
+                                          float (*acc)[4]) {
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    const float dl = h2f(lds16(blk + 208)), dh = h2f(lds16(blk + r8 + 208));
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        uint32_t lo[4], hi[4];
+        q6k_codes<MIS>(blk, j, c, lo);
+        q6k_codes<MIS>(blk + r8, j, c, hi);
+        float d0lo, d1lo, d0hi, d1hi;
+        q6k_scales(blk, j, dl, &d0lo, &d1lo);
+        q6k_scales(blk + r8, j, dh, &d0hi, &d1hi);
+        const uint32_t a0[4] = {lo[0], hi[0], lo[1], hi[1]};
+        const uint32_t a1[4] = {lo[2], hi[2], lo[3], hi[3]};
+#pragma unroll
+        for (int nt = 0; nt < NTILE; nt++) {
+            const uint4 b4 = lds128(ba[nt] + j * 64);
+            float p0[4], p1[4];
+            mma_16816(p0, a0, b4.x, b4.y, zero);
+            mma_16816(p1, a1, b4.z, b4.w, zero);
+            acc[nt][0] = fmaf(d1lo, p1[0], fmaf(d0lo, p0[0], acc[nt][0]));
+            acc[nt][1] = fmaf(d1lo, p1[1], fmaf(d0lo, p0[1], acc[nt][1]));
+            acc[nt][2] = fmaf(d1hi, p1[2], fmaf(d0hi, p0[2], acc[nt][2]));
+            acc[nt][3] = fmaf(d1hi, p1[3], fmaf(d0hi, p0[3], acc[nt][3]));
+        }
+    }
+}
+
 // K1 geometry of one quant type at a given D
 struct GuGeo {
     int sb, nsl, pitch;                 // blocks per slice, slices, staged row pitch
@@ -479,6 +573,12 @@ struct GuGeo {
 __host__ __device__ inline GuGeo gu_geo(int D, int qt, int max_sb) {
     const int bs = qt_unit_bytes(qt), nb = D / QK;
     GuGeo g;
+    if (qt == MOE_Q6_K) {             // whole rows of 8 blocks (D = 2048: 1680 bytes)
+        g.sb = nb;
+        g.nsl = 1;
+        g.pitch = tma_row_bytes((int)qt_row_bytes(qt, D));
+        return g;
+    }
     g.sb = slice_blocks_q(nb, bs, max_sb);
     g.nsl = nb / g.sb;
     g.pitch = tma_row_bytes(g.sb * bs);
@@ -749,12 +849,14 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
 #pragma unroll
             for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
         const int bsz = qt_unit_bytes(qt);
-        const int mis0 = (kb0 * bsz) & 3;               // 0 or 2
+        // byte offset of the warp's first unit in a staged row (Q6_K: block kb0 / 8)
+        const int uoff = qt == MOE_Q6_K ? (kb0 >> 3) * MOE_Q6_K_BLOCK_BYTES : kb0 * bsz;
+        const int mis0 = uoff & 3;                      // 0 or 2
         const uint32_t r8 = 8u * gg.pitch;
 
         for (int sl = 0; sl < gg.nsl; sl++) {
             if (!mbar_wait_warp(&full[stage], phase, a.err, kErrTimeoutFull)) { ok = false; break; }
-            const uint32_t row = st_a + stage * stage_bytes + (mat * kTile + g) * gg.pitch + kb0 * bsz;
+            const uint32_t row = st_a + stage * stage_bytes + (mat * kTile + g) * gg.pitch + uoff;
             uint32_t xs_s[NT], sa_s[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; nt++) {
@@ -771,6 +873,12 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
                 case MOE_Q5_0: if (mis0 == 0) MOE_GU(MOE_Q5_0, 0); else MOE_GU(MOE_Q5_0, 2); break;
                 case MOE_Q4_1: MOE_GU(MOE_Q4_1, 0); break;      // 20-byte blocks: always aligned
                 case MOE_Q5_1: MOE_GU(MOE_Q5_1, 0); break;      // 24-byte blocks: always aligned
+                case MOE_Q6_K:                                   // one block a warp (WB4 == 8)
+                    if constexpr (WB4 == 8) {
+                        if (mis0 == 0) block_q6k<0, 1>(row, r8, xs_s, c, acc);
+                        else block_q6k<2, 1>(row, r8, xs_s, c, acc);
+                    }
+                    break;
                 default:                                         // Q4_K
                     gateup_slice_q4k<1, WB4>(row - kb0 * bsz, r8, kb0, xs_s, sa_s, c, acc);
                     break;
@@ -872,14 +980,15 @@ __device__ __forceinline__ void down_block_q4k(uint32_t blk, uint32_t r8, const 
     const uint32_t off2 = 0x64006400u;
     const float zero[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t ones[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};
+    const Q4kHead hlo = q4k_head(blk), hhi = q4k_head(blk + r8);
 #pragma unroll
     for (int j = 0; j < 8; j++) {
         uint32_t lo[4], hi[4];
         q4k_codes(blk, j, c, lo);
         q4k_codes(blk + r8, j, c, hi);
         float dlo, mlo, dhi, mhi;
-        q4k_params(blk, j, &dlo, &mlo);
-        q4k_params(blk + r8, j, &dhi, &mhi);
+        q4k_params(hlo, j, &dlo, &mlo);
+        q4k_params(hhi, j, &dhi, &mhi);
         const uint32_t a0[4] = {hsub2_u(lo[0], off2), hsub2_u(hi[0], off2), hsub2_u(lo[1], off2),
                                 hsub2_u(hi[1], off2)};
         const uint32_t a1[4] = {hsub2_u(lo[2], off2), hsub2_u(hi[2], off2), hsub2_u(lo[3], off2),
@@ -925,8 +1034,8 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
     const int D = a.D;
     const int S = G * Sg;
     const int hbytes = a.hrow * 2;                      // staged Hs row = its global stride
-    const int pr = tma_row_bytes((int)qt_row_bytes(a.qt, a.F));
-    const int ps = a.sF > 0 ? tma_row_bytes((int)qt_row_bytes(a.sqt, a.sF)) : 0;
+    const int pr = dn_pitch(a.qt, a.F);
+    const int ps = a.sF > 0 ? dn_pitch(a.sqt, a.sF) : 0;
     const int wbytes = kDnRows * (pr > ps ? pr : ps);
     const int stage_bytes = (int)round_up((size_t)wbytes + (size_t)hrows * hbytes, 128);
     const int grp = warp >> 2, mt = warp & 3;
@@ -1005,8 +1114,12 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
                 if (!mbar_wait(&empty[sl.stage], sl.phase ^ 1, a.err, kErrTimeoutEmpty)) { ok = false; break; }
                 uint8_t *dst = stages + (size_t)sl.stage * stage_bytes;
                 mbar_arrive_expect_tx(&full[sl.stage], (uint32_t)(kDnRows * pitch + vi.cnt * hbytes));
-                tma_load_2d_hint(dst, vi.shared ? &maps.sdown : &maps.down, 0,
-                                 (vi.shared ? 0 : (int)vi.slot * D) + dt * kDnRows, &full[sl.stage], pol);
+                const int y0 = (vi.shared ? 0 : (int)vi.slot * D) + dt * kDnRows;
+                if (vi.qt == MOE_Q6_K)          // 8 whole 8-row groups, rows packed
+                    tma_load_3d_hint(dst, vi.shared ? &maps.sdown : &maps.down, 0, 0, y0 / 8,
+                                     &full[sl.stage], pol);
+                else
+                    tma_load_2d_hint(dst, vi.shared ? &maps.sdown : &maps.down, 0, y0, &full[sl.stage], pol);
                 used |= 1u << sl.stage;
                 last_ph = (last_ph & ~(1u << sl.stage)) | (sl.phase << sl.stage);
                 if (waited) {
@@ -1045,6 +1158,12 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
         const int pitch = vi.shared ? ps : pr;
         const int nb = vi.Fv / QK;
         const int ntile = vi.cnt > 8 ? 2 : 1;
+        // Q6_K rows are packed at an even pitch that may be 2 mod 4: warp mt
+        // takes the rows of one parity, 2i + (mt & 1) + 32 (mt >> 1) for tile
+        // row i, so that a block's alignment is the same in all its rows
+        const bool q6 = ALL && vi.qt == MOE_Q6_K;
+        const int mrow = q6 ? 32 * (mt >> 1) + (mt & 1) : mt * kTile;   // tile row 0
+        const int mstep = q6 ? 2 : 1;                                      // rows per tile row
         float acc[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; nt++)
@@ -1052,8 +1171,8 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
             for (int q = 0; q < 4; q++) acc[nt][q] = 0.f;
         if (!mbar_wait_warp(&full[sl.stage], sl.phase, a.err, kErrTimeoutFull)) break;
         const uint32_t sbase = st_a + sl.stage * stage_bytes;
-        uint32_t row = sbase + (mt * kTile + g) * pitch;
-        const uint32_t r8 = 8u * pitch;
+        uint32_t row = sbase + (mrow + mstep * g) * pitch;
+        const uint32_t r8 = 8u * mstep * pitch;
         uint32_t ha[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; nt++) {
@@ -1063,6 +1182,24 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
             // and those columns are never stored
             ha[nt] = sbase + wbytes + (n < hrows ? n : 0) * hbytes + c * 16;
         }
+        if (q6) {
+            if constexpr (ALL) {
+                // block b starts (row parity * pitch + 210 b) mod 4 bytes off
+                const int nblk = nb / 8;
+                const bool mis0 = ((mt & 1) * pitch) & 3;
+                for (int b = 0; b < nblk; b += 2) {
+                    const uint32_t blk = row + b * MOE_Q6_K_BLOCK_BYTES;
+                    if (!mis0) block_q6k<0, 1>(blk, r8, ha, c, acc);
+                    else block_q6k<2, 1>(blk, r8, ha, c, acc);
+                    if (b + 1 < nblk) {
+                        uint32_t hb[1] = {ha[0] + 8 * 64};
+                        if (!mis0) block_q6k<2, 1>(blk + MOE_Q6_K_BLOCK_BYTES, r8, hb, c, acc);
+                        else block_q6k<0, 1>(blk + MOE_Q6_K_BLOCK_BYTES, r8, hb, c, acc);
+                    }
+                    ha[0] += 16 * 64;
+                }
+            }
+        } else
         for (int kb = 0; kb < nb; kb += 8) {
 #define MOE_DN(QT)                                                     \
     case QT:                                                           \
@@ -1093,14 +1230,14 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[sl.stage]);
-        // C fragment: rows g / g+8 of the M-tile, columns 2c, 2c+1 (+8 nt)
-        float *out = a.rows_out + (size_t)vi.seg0 * D + dt * kDnRows + mt * kTile;
+        // C fragment: tile rows g / g+8, columns 2c, 2c+1 (+8 nt)
+        float *out = a.rows_out + (size_t)vi.seg0 * D + dt * kDnRows + mrow;
 #pragma unroll
         for (int nt = 0; nt < NT; nt++)
 #pragma unroll
             for (int q = 0; q < 4; q++) {
                 const int n = nt * 8 + 2 * c + (q & 1);
-                const int r = g + ((q >> 1) << 3);
+                const int r = mstep * (g + ((q >> 1) << 3));
                 if (n < vi.cnt) out[(size_t)n * D + r] = acc[nt][q];
             }
     }
@@ -1692,14 +1829,17 @@ dec_combine_kernel(const float *__restrict__ rows, const int32_t *__restrict__ i
 // multiples of 256 up to 1024 (one box per expert tile in the down kernel).
 static bool gu_shape_ok(int D) { return D == 256 || D == 512 || D == 768 || D == 1024 || D == 2048; }
 
-// Block types the kernels decode: the 32-weight Standard family and Q4_K
-// (Q6_K's 210-byte blocks leave rows of F=768 weights unaligned for tensor
-// copies; it takes the portable kernels)
-static bool dec_type_ok(int qt) { return qt_known(qt) && qt != MOE_Q6_K; }
+// Block types the kernels decode at a given D: all of them, Q6_K when its
+// gate/up rows (210 * D / 256 bytes) are whole 16-byte units for the tensor
+// copies, i.e. D = 2048 (its down rows arrive in 8-row groups, which always
+// are)
+static bool dec_type_ok(int qt, int D) {
+    return qt_known(qt) && (qt != MOE_Q6_K || qt_row_bytes(qt, D) % 16 == 0);
+}
 
 bool decode_path_ok(int T, int D, int F, int sF, int qt, int sqt) {
     return T >= 1 && T <= 16 && gu_shape_ok(D) && F % 256 == 0 && F <= 1024 &&
-           dec_type_ok(qt) && (sF == 0 || (sF % 256 == 0 && sF <= 1024 && dec_type_ok(sqt)));
+           dec_type_ok(qt, D) && (sF == 0 || (sF % 256 == 0 && sF <= 1024 && dec_type_ok(sqt, D)));
 }
 
 // Hs rows are padded by 32 halves (64 bytes): row stride = 64 mod 128 bytes,
@@ -1747,6 +1887,35 @@ static moe_status encode_rows(CUtensorMap *m, const void *base, size_t row_bytes
     return MOE_OK;
 }
 
+// Q6_K down rows (F weights, nrows rows, nrows a multiple of 8): a 3-D tensor
+// of 560-byte chunks, 3 F / 256 of them an 8-row group; boxes of kDnRows rows
+// land packed (kDnRows * the row bytes)
+static moe_status encode_q6k_down(CUtensorMap *m, const void *base, int F, size_t nrows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) { set_error("decode path: cuTensorMapEncodeTiled unavailable"); return MOE_ERR_CUDA; }
+    const size_t group = 8 * qt_row_bytes(MOE_Q6_K, F);          // 1680 * F / 256
+    const cuuint32_t nch = (cuuint32_t)(group / kQ6Chunk);
+    const cuuint64_t dims[3] = {(cuuint64_t)(kQ6Chunk / 8), nch, (cuuint64_t)(nrows / 8)};
+    const cuuint64_t strides[2] = {(cuuint64_t)kQ6Chunk, (cuuint64_t)group};
+    const cuuint32_t box[3] = {(cuuint32_t)(kQ6Chunk / 8), nch, (cuuint32_t)(kDnRows / 8)};
+    const cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void *>(base), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("decode path: Q6_K tensor map encoding failed (%d) for %zu rows of F = %d", (int)r,
+                  nrows, F);
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+static moe_status encode_down(CUtensorMap *m, const void *base, int qt, int F, size_t nrows) {
+    if (qt == MOE_Q6_K) return encode_q6k_down(m, base, F, nrows);
+    const size_t rb = qt_row_bytes(qt, F);
+    return encode_rows(m, base, rb, nrows, tma_row_bytes((int)rb), kDnRows);
+}
+
 static moe_status encode_maps(const DecArgs &a, int n_slots, int max_sb, DecMaps *m) {
     memset(m, 0, sizeof(*m));
     const size_t rg = qt_row_bytes(a.qt, a.D);
@@ -1756,16 +1925,13 @@ static moe_status encode_maps(const DecArgs &a, int n_slots, int max_sb, DecMaps
         return st;
     if ((st = encode_rows(&m->up, a.up, rg, (size_t)n_slots * a.F, gr.pitch, kTile)))
         return st;
-    const size_t rbd = qt_row_bytes(a.qt, a.F);
-    if ((st = encode_rows(&m->down, a.down, rbd, (size_t)n_slots * a.D, tma_row_bytes((int)rbd), kDnRows)))
-        return st;
+    if ((st = encode_down(&m->down, a.down, a.qt, a.F, (size_t)n_slots * a.D))) return st;
     if (a.sF > 0) {
         const size_t rgs = qt_row_bytes(a.sqt, a.D);
         const GuGeo gs = gu_geo(a.D, a.sqt, max_sb);
         if ((st = encode_rows(&m->sgate, a.sh_gate, rgs, a.sF, gs.pitch, kTile))) return st;
         if ((st = encode_rows(&m->sup, a.sh_up, rgs, a.sF, gs.pitch, kTile))) return st;
-        const size_t rbs = qt_row_bytes(a.sqt, a.sF);
-        if ((st = encode_rows(&m->sdown, a.sh_down, rbs, a.D, tma_row_bytes((int)rbs), kDnRows))) return st;
+        if ((st = encode_down(&m->sdown, a.sh_down, a.sqt, a.sF, a.D))) return st;
     }
     return MOE_OK;
 }
@@ -1870,8 +2036,8 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
     // ---- down: Y rows
     {
         const int hrows = std::min(a.T, kGuCols);
-        const int pr = tma_row_bytes((int)qt_row_bytes(a.qt, a.F));
-        const int ps = a.sF > 0 ? tma_row_bytes((int)qt_row_bytes(a.sqt, a.sF)) : 0;
+        const int pr = dn_pitch(a.qt, a.F);
+        const int ps = a.sF > 0 ? dn_pitch(a.sqt, a.sF) : 0;
         const size_t wbytes = (size_t)kDnRows * std::max(pr, ps);
         const size_t stage_bytes = round_up(wbytes + (size_t)hrows * a.hrow * 2, 128);
         const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + tables_bytes(a.E) +
@@ -1929,8 +2095,8 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
     a.perm = perm; a.offsets = offsets; a.gates = gates; a.mask = mask;
     a.gate = (const uint8_t *)pool.gate; a.up = (const uint8_t *)pool.up;
     a.down = (const uint8_t *)pool.down; a.slot_map = pool.slot_of_expert;
-    if (!dec_type_ok(pool.qtype)) {
-        set_error("decode path: unsupported quant type %d", (int)pool.qtype);
+    if (!dec_type_ok(pool.qtype, D)) {
+        set_error("decode path: unsupported quant type %d at D = %d", (int)pool.qtype, D);
         return MOE_ERR_UNSUPPORTED_QTYPE;
     }
     if (T * k > kMaxTk) {
@@ -1942,8 +2108,9 @@ moe_status launch_ffn_decode(const void *x, int x_dtype, int T, int D, int F, in
     if (shared) {
         a.sh_gate = (const uint8_t *)shared->gate; a.sh_up = (const uint8_t *)shared->up;
         a.sh_down = (const uint8_t *)shared->down;
-        if (!dec_type_ok(shared->qtype)) {
-            set_error("decode path: unsupported shared-expert quant type %d", (int)shared->qtype);
+        if (!dec_type_ok(shared->qtype, D)) {
+            set_error("decode path: unsupported shared-expert quant type %d at D = %d",
+                      (int)shared->qtype, D);
             return MOE_ERR_UNSUPPORTED_QTYPE;
         }
         a.sqt = shared->qtype;

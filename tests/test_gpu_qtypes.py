@@ -6,13 +6,14 @@ Each type runs the decode GEMV (T <= 16, every compiled D geometry), the
 tcgen05 grouped GEMM (T > 16, ragged row tiles, experts with a handful of
 rows) and the portable kernel (D, F not multiples of 256, or F > 1024), as
 a routed pool and as the shared expert beside a routed pool of another type.
-Q6_K runs the portable kernel at decode shapes and through moe_expert_ffn
-(its 210-byte blocks leave rows of 768 weights without the 16-byte alignment
-tensor copies need), and the tensor-core GEMM on fp16 copies of its pool in
-the fused layer at T > 16.  The
-bar is the one of the Q4_0 / Q8_0 parity tests: max|gpu - oracle| /
-max|oracle| <= 2e-3 on fp32 outputs, and bit-identical rows for a masked
-two-call split.
+Q6_K's 210-byte blocks give rows that are whole 16-byte units only at
+D = 2048 (gate/up) or in 8-row groups (down): it runs the decode GEMV at
+D = 2048 (down rows packed at a pitch that is 2 mod 4 when F / 256 is odd,
+each warp taking rows of one parity), the portable kernel at other decode
+shapes and through moe_expert_ffn at T > 16, and the tensor-core GEMM on
+fp16 copies of its pool in the fused layer at T > 16.  The bar is the one of
+the Q4_0 / Q8_0 parity tests: max|gpu - oracle| / max|oracle| <= 2e-3 on fp32
+outputs, and bit-identical rows for a masked two-call split.
 """
 import numpy as np
 import pytest
@@ -188,3 +189,44 @@ def test_q6k_prefill_layer_phases_are_bit_identical(moe):
     assert torch.equal(y1, y2)
     _check_layer(moe, L, y1, lay.ids, 40)
     assert moe.workspace_status(lay.ws) == (0, moe.DEV_OK)
+
+
+# ------------------------------------------------------------- Q6_K decode
+def _kinds(moe, L):
+    lay = _layer(moe, L)
+    tr = moe.KernelTrace(n_calls=1)
+    y = lay.forward(dev_x(L), trace=tr)
+    torch.cuda.synchronize()
+    return lay, y, {k for call in tr.calls for k, _, _ in call}
+
+
+@pytest.mark.parametrize("F", [256, 512, 768, 1024])
+@pytest.mark.parametrize("T", [1, 16])
+def test_q6k_decode_kernels(moe, T, F):
+    # D = 2048: the decode GEMV, not the portable kernel; F / 256 odd packs
+    # the down rows at a pitch of 2 mod 4
+    L = _inputs(_cfg("q6_k", T, D=2048, F=F, E=16, k=4, seed=590))
+    lay, y, kinds = _kinds(moe, L)
+    assert "ffn_decode" in kinds and "gateup" not in kinds, kinds
+    err = _check_layer(moe, L, y, lay.ids, 99)
+    assert moe.workspace_status(lay.ws) == (0, moe.DEV_OK)
+    print(f"q6_k T={T} F={F}: rel err {err:.3e}")
+
+
+@pytest.mark.parametrize("routed,shared", [("q6_k", "q4_0"), ("q4_0", "q6_k"), ("q6_k", "q6_k"),
+                                           ("q5_1", "q6_k")])
+@pytest.mark.parametrize("T", [2, 16])
+def test_q6k_decode_with_shared_expert(moe, routed, shared, T):
+    L = _inputs(_cfg(routed, T, D=2048, F=768, E=16, k=4, shared_F=512, shared_qtype=shared,
+                     seed=591))
+    lay, y, kinds = _kinds(moe, L)
+    assert "ffn_decode" in kinds, kinds
+    _check_layer(moe, L, y, lay.ids, 99)
+    assert moe.workspace_status(lay.ws) == (0, moe.DEV_OK)
+
+
+def test_q6k_decode_at_other_d_takes_the_portable_kernel(moe):
+    L = _inputs(_cfg("q6_k", 4, D=1024, F=768, E=16, k=4, seed=592))
+    lay, y, kinds = _kinds(moe, L)
+    assert "ffn_decode" not in kinds and "gateup" in kinds, kinds
+    _check_layer(moe, L, y, lay.ids, 99)
