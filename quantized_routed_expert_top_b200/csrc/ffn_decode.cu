@@ -586,8 +586,10 @@ __host__ __device__ inline GuGeo gu_geo(int D, int qt, int max_sb) {
 }
 
 // ALL: the call has a type other than Q4_0 and Q8_0 (a separate
-// instantiation keeps the other types' code out of the two types' kernel)
-template <int MAXSB, int WB4, int WB8, bool ALL>
+// instantiation keeps the other types' code out of the two types' kernel);
+// ONE >= 0: every expert of the call has block type ONE (an instantiation
+// with only that type's code: smaller, fewer instruction-cache misses)
+template <int MAXSB, int WB4, int WB8, bool ALL, int ONE = -1>
 __global__ void __launch_bounds__(kGThreads, 1)
 dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
     constexpr int NT = 1;
@@ -825,7 +827,7 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
         const int4 ud = utab[j];
         const int tile = ud.y, seg0 = ud.z, cnt = ud.w;
         const bool shu = ud.x >= A.n_routed;
-        const int qt = shu ? a.sqt : a.qt;
+        const int qt = ONE >= 0 ? ONE : shu ? a.sqt : a.qt;
         const GuGeo gg = shu ? geoS : geoR;
         const int kb0 = kg * (qt == MOE_Q8_0 ? WB8 : WB4);   // warp's first block in a slice
         // B rows (column g, g+8) and C columns (2c, 2c+1, +8) of this unit
@@ -1024,8 +1026,8 @@ __device__ __forceinline__ DnSlot dn_slot(int i, int G, int Sg) {
 
 // ALL: the call has a type other than Q4_0 and Q8_0 (a separate
 // instantiation keeps the other types' code and registers out of the two
-// types' kernel)
-template <int NT, bool ALL>
+// types' kernel); ONE >= 0: every expert has block type ONE
+template <int NT, bool ALL, int ONE = -1>
 __global__ void __launch_bounds__(kDThreads, 1)
 dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ DecMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -1087,6 +1089,7 @@ dec_down_kernel(DecArgs a, int G, int Sg, int hrows, const __grid_constant__ Dec
     auto entry = [&](int q, Virt *vi) {
         const int2 e2 = ent[q];
         *vi = virt(a, act, A.n_routed, e2.x);
+        if (ONE >= 0) vi->qt = ONE;
         vi->seg0 += e2.y * kGuCols;
         vi->cnt = min(kGuCols, vi->cnt - e2.y * kGuCols);
     };
@@ -1980,6 +1983,12 @@ static bool dec_all_types(const DecArgs &a) {
     auto basic = [](int q) { return q == MOE_Q4_0 || q == MOE_Q8_0; };
     return !basic(a.qt) || (a.sF > 0 && !basic(a.sqt));
 }
+// the block type of every expert of a call whose types are not Q4_0 / Q8_0
+// only, when there is one (-1 otherwise)
+static int dec_one_type(const DecArgs &a) {
+    if (!dec_all_types(a) || (a.sF > 0 && a.sqt != a.qt)) return -1;
+    return a.qt;
+}
 
 template <bool ALL>
 static cudaError_t launch_gateup1(const DecArgs &a, const DecMaps &m, int grid, size_t smem,
@@ -1991,6 +2000,15 @@ static cudaError_t launch_gateup1(const DecArgs &a, const DecMaps &m, int grid, 
     case 768: return launch_pdl(dec_gateup_kernel<32, 3, 3, ALL>, grid, kGThreads, smem, s, a, S, m);
     case 1024: return launch_pdl(dec_gateup_kernel<32, 4, 4, ALL>, grid, kGThreads, smem, s, a, S, m);
     default:
+        if (ALL && wide && dec_one_type(a) >= 0) {
+            switch (dec_one_type(a)) {
+            case MOE_Q4_1: return launch_pdl(dec_gateup_kernel<64, 8, 4, true, MOE_Q4_1>, grid, kGThreads, smem, s, a, S, m);
+            case MOE_Q5_0: return launch_pdl(dec_gateup_kernel<64, 8, 4, true, MOE_Q5_0>, grid, kGThreads, smem, s, a, S, m);
+            case MOE_Q5_1: return launch_pdl(dec_gateup_kernel<64, 8, 4, true, MOE_Q5_1>, grid, kGThreads, smem, s, a, S, m);
+            case MOE_Q4_K: return launch_pdl(dec_gateup_kernel<64, 8, 4, true, MOE_Q4_K>, grid, kGThreads, smem, s, a, S, m);
+            default: return launch_pdl(dec_gateup_kernel<64, 8, 4, true, MOE_Q6_K>, grid, kGThreads, smem, s, a, S, m);
+            }
+        }
         return wide ? launch_pdl(dec_gateup_kernel<64, 8, 4, ALL>, grid, kGThreads, smem, s, a, S, m)
                     : launch_pdl(dec_gateup_kernel<32, 4, 4, ALL>, grid, kGThreads, smem, s, a, S, m);
     }
@@ -2056,10 +2074,24 @@ static moe_status run_decode(const DecArgs &a, int n_slots, cudaStream_t s, Trac
         const int grid = std::max(1, std::min(sms, U_max));
         // no trace mark here: an event between the two kernels would cancel
         // their programmatic overlap
-        cudaError_t e = dec_all_types(a) ? launch_pdl(dec_down_kernel<NT, true>, grid, kDThreads, smem,
-                                                      s, a, G, Sg, hrows, maps)
-                                         : launch_pdl(dec_down_kernel<NT, false>, grid, kDThreads, smem,
-                                                      s, a, G, Sg, hrows, maps);
+        cudaError_t e;
+        switch (dec_one_type(a)) {
+#define MOE_DN1(QT)                                                                          \
+    case QT:                                                                                 \
+        e = launch_pdl(dec_down_kernel<NT, true, QT>, grid, kDThreads, smem, s, a, G, Sg, hrows, maps); \
+        break;
+            MOE_DN1(MOE_Q4_1)
+            MOE_DN1(MOE_Q5_0)
+            MOE_DN1(MOE_Q5_1)
+            MOE_DN1(MOE_Q4_K)
+            MOE_DN1(MOE_Q6_K)
+#undef MOE_DN1
+        default:
+            e = dec_all_types(a) ? launch_pdl(dec_down_kernel<NT, true>, grid, kDThreads, smem, s, a,
+                                              G, Sg, hrows, maps)
+                                 : launch_pdl(dec_down_kernel<NT, false>, grid, kDThreads, smem, s, a,
+                                              G, Sg, hrows, maps);
+        }
         if (e != cudaSuccess) return cuda_status(e, "dec_down_kernel");
     }
     }
