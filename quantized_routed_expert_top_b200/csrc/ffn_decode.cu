@@ -869,11 +869,14 @@ dec_gateup_kernel(DecArgs a, int S, const __grid_constant__ DecMaps maps) {
             }
 #define MOE_GU(QT, MIS) gateup_slice<QT, 1, (QT == MOE_Q8_0 ? WB8 : WB4), MIS>(row, r8, xs_s, sa_s, c, acc)
             if (!ALL || qt == MOE_Q4_0 || qt == MOE_Q8_0) {
-                if (qt == MOE_Q4_0) { if (mis0 == 0) MOE_GU(MOE_Q4_0, 0); else MOE_GU(MOE_Q4_0, 2); }
-                else { if (mis0 == 0) MOE_GU(MOE_Q8_0, 0); else MOE_GU(MOE_Q8_0, 2); }
+                // with an even number of blocks a warp, an 18-, 22- or 34-byte
+                // block group always starts 4-byte aligned (mis0 == 0): the
+                // other variant is compiled only where it can run
+                if (qt == MOE_Q4_0) { if (WB4 % 2 == 0 || mis0 == 0) MOE_GU(MOE_Q4_0, 0); else MOE_GU(MOE_Q4_0, 2); }
+                else { if (WB8 % 2 == 0 || mis0 == 0) MOE_GU(MOE_Q8_0, 0); else MOE_GU(MOE_Q8_0, 2); }
             } else if constexpr (ALL) {
                 switch (qt) {
-                case MOE_Q5_0: if (mis0 == 0) MOE_GU(MOE_Q5_0, 0); else MOE_GU(MOE_Q5_0, 2); break;
+                case MOE_Q5_0: if (WB4 % 2 == 0 || mis0 == 0) MOE_GU(MOE_Q5_0, 0); else MOE_GU(MOE_Q5_0, 2); break;
                 case MOE_Q4_1: MOE_GU(MOE_Q4_1, 0); break;      // 20-byte blocks: always aligned
                 case MOE_Q5_1: MOE_GU(MOE_Q5_1, 0); break;      // 24-byte blocks: always aligned
                 case MOE_Q6_K:                                   // one block a warp (WB4 == 8)
