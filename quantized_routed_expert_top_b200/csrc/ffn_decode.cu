@@ -319,22 +319,26 @@ __host__ __device__ __forceinline__ int frag_slot(int i) {
 template <int QT, int MIS>
 __device__ __forceinline__ void magic_codes(uint32_t blk, int c, uint32_t *r) {
     const uint32_t qa = blk + qt_qs_off(QT) + 4 * c;
-    if constexpr (QT != MOE_Q8_0) {
+    if constexpr (qt_has_high(QT)) {
+        // 5-bit codes as bytes (low four bits from qs, bit i of qh is bit 4
+        // of element i): elements 4c..4c+3 and 16+4c..19+4c, then bytes
+        // into the halves of the fragment order
+        const uint32_t w = lds_word<MIS>(qa);
+        const uint32_t h = lds_word<MIS>(blk + qt_qh_off(QT)) >> (4 * c);
+        const uint32_t lo = lop3_and_or(w, 0x0F0F0F0Fu, spread4_bit4(h & 0xFu));
+        const uint32_t hi = lop3_and_or(w >> 4, 0x0F0F0F0Fu, spread4_bit4((h >> 16) & 0xFu));
+        const uint32_t HI = 0x64646464u;
+        r[0] = prmt(lo, HI, 0x4240);
+        r[1] = prmt(lo, HI, 0x4341);
+        r[2] = prmt(hi, HI, 0x4240);
+        r[3] = prmt(hi, HI, 0x4341);
+    } else if constexpr (QT != MOE_Q8_0) {
         const uint32_t w = lds_word<MIS>(qa);
         const uint32_t M = 0x000F000Fu, MAG = 0x64006400u;
         r[0] = lop3_and_or(w, M, MAG);
         r[2] = lop3_and_or(w >> 4, M, MAG);
         r[1] = lop3_and_or(w >> 8, M, MAG);
         r[3] = lop3_and_or(w >> 12, M, MAG);
-        if constexpr (qt_has_high(QT)) {
-            // bit i of qh is bit 4 of element i: for this thread, elements
-            // 4c..4c+3 and 16+4c..19+4c, into bit 4 of each half
-            const uint32_t h = lds_word<MIS>(blk + qt_qh_off(QT)) >> (4 * c);
-            r[0] |= ((h & 1u) << 4) | ((h & 4u) << 18);
-            r[1] |= ((h & 2u) << 3) | ((h & 8u) << 17);
-            r[2] |= ((h >> 12) & 0x10u) | ((h << 2) & 0x100000u);
-            r[3] |= ((h >> 13) & 0x10u) | ((h << 1) & 0x100000u);
-        }
     } else {
         const uint32_t w0 = lds_word<MIS>(qa) ^ 0x80808080u;
         const uint32_t w1 = lds_word<MIS>(qa + 16) ^ 0x80808080u;

@@ -265,16 +265,25 @@ __device__ __forceinline__ void dq_pair_std(const uint32_t *w, uint4 *out) {
 #pragma unroll
         for (int i = 0; i < 4; i++) {
             const uint32_t c = word_at(w, B + QS + 4 * i);        // bytes 4i .. 4i+3
-            const uint32_t t0 = prmt(c, 0u, 0x4140), t1 = prmt(c, 0u, 0x4342);
-            uint32_t v[4] = {lop3_and_or(t0, M, MAG), lop3_and_or(t1, M, MAG),
-                             lop3_and_or(t0 >> 4, M, MAG), lop3_and_or(t1 >> 4, M, MAG)};
+            // v: elements (4i, 4i+1), (4i+2, 4i+3), (16+4i, 17+4i), (18+4i, 19+4i)
+            uint32_t v[4];
             if constexpr (qt_has_high(QT)) {
-                // v: elements (4i, 4i+1), (4i+2, 4i+3), (16+4i, 17+4i), (18+4i, 19+4i)
+                // 5-bit codes as bytes (bit 4 of element j from bit j of qh),
+                // then bytes into halves
                 const uint32_t h = qh >> (4 * i);
-                v[0] |= ((h & 1u) << 4) | ((h & 2u) << 19);
-                v[1] |= ((h & 4u) << 2) | ((h & 8u) << 17);
-                v[2] |= ((h >> 12) & 0x10u) | ((h << 3) & 0x100000u);
-                v[3] |= ((h >> 14) & 0x10u) | ((h << 1) & 0x100000u);
+                const uint32_t lo = lop3_and_or(c, 0x0F0F0F0Fu, spread4_bit4(h & 0xFu));
+                const uint32_t hi = lop3_and_or(c >> 4, 0x0F0F0F0Fu, spread4_bit4((h >> 16) & 0xFu));
+                const uint32_t HI = 0x64646464u;
+                v[0] = prmt(lo, HI, 0x5140);
+                v[1] = prmt(lo, HI, 0x7362);
+                v[2] = prmt(hi, HI, 0x5140);
+                v[3] = prmt(hi, HI, 0x7362);
+            } else {
+                const uint32_t t0 = prmt(c, 0u, 0x4140), t1 = prmt(c, 0u, 0x4342);
+                v[0] = lop3_and_or(t0, M, MAG);
+                v[1] = lop3_and_or(t1, M, MAG);
+                v[2] = lop3_and_or(t0 >> 4, M, MAG);
+                v[3] = lop3_and_or(t1 >> 4, M, MAG);
             }
 #pragma unroll
             for (int q = 0; q < 4; q++)

@@ -196,6 +196,14 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
     return r;
 }
 
+// Bit k of x (x < 16) to bit 4 of byte k: the four copies of x in
+// x * (2^4 + 2^11 + 2^18 + 2^25) sit 7 bits apart (no overlap, no carries)
+// and copy k puts bit k on bit 8k + 4.  The fifth bit of four 5-bit codes
+// held as bytes.
+__device__ __forceinline__ uint32_t spread4_bit4(uint32_t x) {
+    return (x * 0x02040810u) & 0x10101010u;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
