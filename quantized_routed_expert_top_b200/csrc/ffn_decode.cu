@@ -433,28 +433,32 @@ __device__ __forceinline__ void q4k_codes(uint32_t blk, int j, int c, uint32_t *
     r[2] = prmt(w1, HI, 0x4240);
     r[3] = prmt(w1, HI, 0x4341);
 }
-// A Q4_K block's head: d, dmin and the packed 6-bit scales and mins
+// A Q4_K block's head: d, dmin and its eight 6-bit scales and mins, unpacked
+// four to a word (byte j & 3 of word j / 4) with a few word-wide masks and
+// shifts: sub-block j < 4 keeps the low six bits of byte j of scales[0..3]
+// (scale) and scales[4..7] (min); j >= 4 takes the low (scale) or high (min)
+// nibble of scales[8 + j - 4] and, as bits 4 and 5, the top two bits of
+// byte j - 4 of scales[0..3] (scale) or scales[4..7] (min)
 struct Q4kHead {
-    uint32_t s0, s1, s2;
+    uint32_t sc[2], mn[2];
     float d, dmin;
 };
 __device__ __forceinline__ Q4kHead q4k_head(uint32_t blk) {
-    const uint32_t w = lds32(blk);
-    return {lds32(blk + 4), lds32(blk + 8), lds32(blk + 12), h2f(w & 0xFFFFu), h2f(w >> 16)};
+    const uint32_t w = lds32(blk), s0 = lds32(blk + 4), s1 = lds32(blk + 8), s2 = lds32(blk + 12);
+    Q4kHead h;
+    h.sc[0] = s0 & 0x3F3F3F3Fu;
+    h.mn[0] = s1 & 0x3F3F3F3Fu;
+    h.sc[1] = (s2 & 0x0F0F0F0Fu) | ((s0 >> 2) & 0x30303030u);
+    h.mn[1] = ((s2 >> 4) & 0x0F0F0F0Fu) | ((s1 >> 2) & 0x30303030u);
+    h.d = h2f(w & 0xFFFFu);
+    h.dmin = h2f(w >> 16);
+    return h;
 }
 // Scale D = d * sc_j and min M = dmin * m_j of sub-block j (weight D q - M)
 __device__ __forceinline__ void q4k_params(const Q4kHead &h, int j, float *D, float *M) {
-    const int jj = j & 3, sh = 8 * jj;
-    int sc, m;
-    if (j < 4) {
-        sc = (h.s0 >> sh) & 63;
-        m = (h.s1 >> sh) & 63;
-    } else {
-        sc = ((h.s2 >> sh) & 15) | (((h.s0 >> (sh + 6)) & 3) << 4);
-        m = ((h.s2 >> (sh + 4)) & 15) | (((h.s1 >> (sh + 6)) & 3) << 4);
-    }
-    *D = h.d * (float)sc;
-    *M = h.dmin * (float)m;
+    const uint32_t sel = 0x4440u | (uint32_t)(j & 3);          // byte j & 3, zero above
+    *D = h.d * (float)prmt(j < 4 ? h.sc[0] : h.sc[1], 0u, sel);
+    *M = h.dmin * (float)prmt(j < 4 ? h.mn[0] : h.mn[1], 0u, sel);
 }
 
 // As gateup_slice for Q4_K: units kb0 .. kb0 + WB - 1 of the slice whose
