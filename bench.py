@@ -524,6 +524,12 @@ def measure_layer(wl, steps, warmup, world, local, peaks, no_graph=False, cpu=Tr
 
     serial_ms = timed(g_e2e)
     e2e_ms = timed(g_pipe)
+    # the pipelined steps compute what the plain ones do (same inputs, same
+    # deterministic kernels, replicas of the same weights): the last result
+    # that reached host memory equals the device output of the plain steps
+    for T in wl.Ts:
+        if not torch.equal(pipe.yh[T], wl.y[T].cpu()):
+            raise RuntimeError(f"{wl.name}: pipelined end-to-end result differs at T={T}")
 
     tokens = wl.tokens_per_step * world
     out = {
